@@ -1,0 +1,287 @@
+/*
+ * moe_oracle.c -- plain fp64 CPU oracle for the sparse top-k MoE layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header or table with the CUDA library; it reads the same input bytes
+ * (bf16 or fp32, widened to double on every access) and computes every step
+ * in double precision with plain loops, in the order the pages describe.
+ *
+ * Page references (title, section):
+ *   [Mixtral explained]  "Mixtral 8x7B and MoE explained: sparse mixture of
+ *                         experts, only 2 experts active per token"
+ *   [MoE wiki]           "Mixture of experts" (wiki entry), "How it works"
+ *   [Routing explained]  "MoE routing fully explained: the expert-mixture
+ *                         structure Mixtral and DeepSeek use, load balancing,
+ *                         capacity factor"
+ *
+ * Where the pages leave a step open, the reading taken is stated at the step.
+ * Build: gcc -O2 -fopenmp -shared -fPIC (see oracle/build.py).  OpenMP only
+ * splits independent outputs (tokens) across threads; each output's sum runs
+ * in one fixed order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+typedef struct {
+    int64_t T;           /* tokens */
+    int32_t d, h, E, k;  /* model width, expert hidden width, experts, kept per token */
+    int32_t n_shared;    /* shared experts (0 if none) */
+    int32_t h_shared;    /* hidden width of each shared expert */
+    int64_t cf_num, cf_den; /* capacity factor as a fraction; cf_den == 0 means no limit */
+    int32_t dtype;       /* ORACLE_F32 or ORACLE_BF16 for x and expert weights */
+    int32_t has_bias;    /* router bias present */
+} oracle_cfg;
+
+/* Widen element i of a bf16 or fp32 array to double.  bf16 is the top half of
+ * an IEEE binary32, so the widening is exact. */
+static double elem(const void* p, int dtype, int64_t i) {
+    float f;
+    if (dtype == ORACLE_F32) {
+        f = ((const float*)p)[i];
+    } else {
+        uint32_t bits = ((uint32_t)((const uint16_t*)p)[i]) << 16;
+        memcpy(&f, &bits, sizeof f);
+    }
+    return (double)f;
+}
+
+/* Expert capacity [Routing explained, "Easy explanation" ¶5]: the buffer per
+ * expert is about batch x top-k x capacity factor / number of experts.  The
+ * "about" is read as the ceiling, taken in exact integer arithmetic on
+ * cf = cf_num / cf_den.  No limit (cf_den == 0) gives T: a token never picks
+ * the same expert twice, so no expert can receive more than T tokens. */
+int64_t oracle_capacity(const oracle_cfg* c) {
+    if (c->cf_den == 0) return c->T;
+    int64_t num = c->T * (int64_t)c->k * c->cf_num;
+    int64_t den = (int64_t)c->E * c->cf_den;
+    return (num + den - 1) / den;
+}
+
+/* Router logits [Mixtral explained, "Easy explanation" ¶3; MoE wiki, "How it
+ * works"]: a score for every expert, as in a classifier.  Linear router:
+ * z[t][e] = sum_c x[t][c] * Wr[c][e] + b[e], c ascending. */
+void oracle_logits(const oracle_cfg* c, const void* x, const float* Wr, const float* bias,
+                   double* z) {
+    const int64_t T = c->T;
+    const int d = c->d, E = c->E;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int j = 0; j < d; ++j)
+                s += elem(x, c->dtype, t * d + j) * (double)Wr[(int64_t)j * E + e];
+            if (c->has_bias) s += (double)bias[e];
+            z[t * E + e] = s;
+        }
+    }
+}
+
+/* Top-k and gates [Mixtral explained, "Easy explanation" ¶3]: keep the k
+ * highest-scoring experts and softmax over those k alone.  Ties (equal
+ * logits) go to the lower expert index, a reading the pages leave open.
+ * idx[t][j] lists the kept experts in descending-logit order; gate[t][j] is
+ * exp(z_j - z_max) / sum over the kept k of exp(z - z_max). */
+void oracle_topk(const oracle_cfg* c, const double* z, int32_t* idx, double* gate) {
+    const int64_t T = c->T;
+    const int E = c->E, k = c->k;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double* zt = z + t * E;
+        int32_t* it = idx + t * k;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int q = 0; q < j; ++q) taken |= (it[q] == e);
+                if (taken) continue;
+                if (best < 0 || zt[e] > zt[best]) best = e; /* strict: lower index keeps a tie */
+            }
+            it[j] = best;
+        }
+        double zmax = zt[it[0]];
+        double den = 0.0;
+        for (int j = 0; j < k; ++j) den += exp(zt[it[j]] - zmax);
+        for (int j = 0; j < k; ++j) gate[t * k + j] = exp(zt[it[j]] - zmax) / den;
+    }
+}
+
+/* Full softmax over all E experts [Routing explained, "Easy explanation" ¶2:
+ * the router forms a probability distribution over every expert].  Used for
+ * the load-balancing loss and the router entropy only. */
+void oracle_probs(const oracle_cfg* c, const double* z, double* p) {
+    const int64_t T = c->T;
+    const int E = c->E;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double* zt = z + t * E;
+        double zmax = zt[0];
+        for (int e = 1; e < E; ++e) if (zt[e] > zmax) zmax = zt[e];
+        double den = 0.0;
+        for (int e = 0; e < E; ++e) den += exp(zt[e] - zmax);
+        for (int e = 0; e < E; ++e) p[t * E + e] = exp(zt[e] - zmax) / den;
+    }
+}
+
+/* Dispatch under capacity [Routing explained, "Easy explanation" ¶3 and ¶5]:
+ * each expert takes at most C tokens per batch; the overflow is dropped.
+ * Which assignments overflow is left open by the pages; the reading taken is
+ * arrival order by token index: an expert's queue fills with its tokens in
+ * increasing t and the rest are dropped.
+ *   rank[t][j]  position of token t in expert idx[t][j]'s queue
+ *   keep[t][j]  1 if rank < C
+ *   routed[e]   assignments to e before the limit; kept[e] = min(routed[e], C) */
+void oracle_dispatch(const oracle_cfg* c, const int32_t* idx, int64_t C,
+                     int32_t* routed, int32_t* kept, int32_t* rank, int8_t* keep) {
+    const int64_t T = c->T;
+    const int E = c->E, k = c->k;
+    for (int e = 0; e < E; ++e) routed[e] = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int e = idx[t * k + j];
+            int32_t r = routed[e]++;
+            rank[t * k + j] = r;
+            keep[t * k + j] = (r < C) ? 1 : 0;
+        }
+    }
+    for (int e = 0; e < E; ++e) kept[e] = routed[e] < C ? routed[e] : (int32_t)C;
+}
+
+/* Statistics.
+ * Load-balancing loss [Routing explained, "Easy explanation" ¶4]: for each
+ * expert multiply the share of tokens it actually received by the total
+ * probability the router gave it, and sum.  Reading: share f_e = routed[e] /
+ * (T k) (hard assignments before the capacity limit, so sum f = 1); mass
+ * P_e = mean over tokens of the full softmax (sum P = 1); the sum is scaled by
+ * E, so that perfectly even routing gives exactly 1.
+ * Overflow rate and router entropy [Routing explained, "Main insights" ¶3]:
+ * dropped / (T k), and the mean over tokens of -sum_e p ln p (nats).
+ * out[0] = aux, out[1] = overflow rate, out[2] = mean entropy,
+ * out[3 .. 3+E) = P_e.  T == 0 gives zeros. */
+void oracle_stats(const oracle_cfg* c, const double* p, const int32_t* routed,
+                  const int32_t* kept, double* out) {
+    const int64_t T = c->T;
+    const int E = c->E, k = c->k;
+    for (int i = 0; i < 3 + E; ++i) out[i] = 0.0;
+    if (T == 0) return;
+    double ent = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        double ht = 0.0;
+        for (int e = 0; e < E; ++e) {
+            double q = p[t * E + e];
+            if (q > 0.0) ht -= q * log(q);
+        }
+        ent += ht;
+    }
+    double aux = 0.0, dropped = 0.0;
+    for (int e = 0; e < E; ++e) {
+        double Pe = 0.0;
+        for (int64_t t = 0; t < T; ++t) Pe += p[t * E + e];
+        Pe /= (double)T;
+        double fe = (double)routed[e] / ((double)T * k);
+        aux += fe * Pe;
+        dropped += (double)(routed[e] - kept[e]);
+        out[3 + e] = Pe;
+    }
+    out[0] = (double)E * aux;
+    out[1] = dropped / ((double)T * k);
+    out[2] = ent / (double)T;
+}
+
+/* One expert's FFN for one token [Mixtral explained, "Easy explanation" ¶2:
+ * widen d to h, then narrow back], in the SiLU-gated form
+ * y = (silu(x w1) * (x w3)) w2 with silu(a) = a / (1 + e^-a).
+ * w1, w3 are [d][h] and w2 is [h][d], row-major, as in y = x W; w_off13 and
+ * w_off2 select the expert inside stacked arrays.  x is row x_off of x.
+ * a, b are scratch of length h; the result goes to y[d]. */
+static void ffn(int d, int h, int dtype, const void* x, int64_t x_off, const void* w1,
+                const void* w3, const void* w2, int64_t w_off13, int64_t w_off2, double* y,
+                double* a, double* b) {
+    for (int i = 0; i < h; ++i) { a[i] = 0.0; b[i] = 0.0; }
+    for (int j = 0; j < d; ++j) {
+        const double xj = elem(x, dtype, x_off + j);
+        const int64_t row = w_off13 + (int64_t)j * h;
+        for (int i = 0; i < h; ++i) {
+            a[i] += xj * elem(w1, dtype, row + i);
+            b[i] += xj * elem(w3, dtype, row + i);
+        }
+    }
+    for (int i = 0; i < h; ++i) a[i] = a[i] / (1.0 + exp(-a[i])) * b[i];
+    for (int o = 0; o < d; ++o) y[o] = 0.0;
+    for (int i = 0; i < h; ++i) {
+        const int64_t row = w_off2 + (int64_t)i * d;
+        for (int o = 0; o < d; ++o) y[o] += a[i] * elem(w2, dtype, row + o);
+    }
+}
+
+/* Single expert FFN on one row, exported for the oracle's own checks. */
+void oracle_ffn(int d, int h, int dtype, const void* x_row, const void* w1, const void* w3,
+                const void* w2, double* y) {
+    double* a = (double*)malloc(sizeof(double) * (size_t)h);
+    double* b = (double*)malloc(sizeof(double) * (size_t)h);
+    ffn(d, h, dtype, x_row, 0, w1, w3, w2, 0, 0, y, a, b);
+    free(a);
+    free(b);
+}
+
+/* Layer output for selected tokens [Mixtral explained, "Easy explanation" ¶3;
+ * MoE wiki, "How it works"; Routing explained, "Easy explanation" ¶4]:
+ *   out[t] = sum over kept j of gate[t][j] * FFN_{idx[t][j]}(x_t)
+ *          + sum over shared experts s of FFN^shared_s(x_t).
+ * A dropped assignment simply contributes nothing; the remaining gates are
+ * not renormalised (the pages are silent; this is the reading taken).
+ * Unselected experts are not evaluated at all.
+ * rows[n_rows] lists the tokens to evaluate (NULL = all T); out is
+ * [n_rows][d].  w1/w3 are [E][d][h], w2 [E][h][d]; the shared ones are
+ * [S][d][hs] and [S][hs][d] (may be NULL when n_shared == 0). */
+void oracle_layer_rows(const oracle_cfg* c, const void* x, const int32_t* idx,
+                       const double* gate, const int8_t* keep, const void* w1,
+                       const void* w3, const void* w2, const void* w1s, const void* w3s,
+                       const void* w2s, const int64_t* rows, int64_t n_rows, double* out) {
+    const int d = c->d, h = c->h, k = c->k, hs = c->h_shared, S = c->n_shared;
+    const int hmax = h > hs ? h : hs;
+    if (rows == NULL) n_rows = c->T;
+#pragma omp parallel
+    {
+        double* a = (double*)malloc(sizeof(double) * (size_t)hmax);
+        double* b = (double*)malloc(sizeof(double) * (size_t)hmax);
+        double* y = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            const int64_t t = rows ? rows[r] : r;
+            double* acc = out + r * d;
+            for (int o = 0; o < d; ++o) acc[o] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                if (!keep[t * k + j]) continue;
+                const int64_t e = idx[t * k + j];
+                ffn(d, h, c->dtype, x, t * d, w1, w3, w2, e * d * h, e * h * d, y, a, b);
+                for (int o = 0; o < d; ++o) acc[o] += gate[t * k + j] * y[o];
+            }
+            for (int s = 0; s < S; ++s) {
+                ffn(d, hs, c->dtype, x, t * d, w1s, w3s, w2s, (int64_t)s * d * hs,
+                    (int64_t)s * hs * d, y, a, b);
+                for (int o = 0; o < d; ++o) acc[o] += y[o];
+            }
+        }
+        free(a);
+        free(b);
+        free(y);
+    }
+}
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+/* Threads the oracle's parallel loops use (reported beside CPU timings). */
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
