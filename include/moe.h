@@ -1,0 +1,236 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse top-k mixture-of-experts layer.
+ *
+ * The layer (pages: "Mixtral 8x7B and MoE explained: sparse mixture of
+ * experts, only 2 experts active per token", section "Easy explanation";
+ * "Mixture of experts" wiki entry, section "How it works"; "MoE routing fully
+ * explained: the expert-mixture structure Mixtral and DeepSeek use, load
+ * balancing, capacity factor", sections "Easy explanation" and "Main
+ * insights") computes, for a batch x[T][d]:
+ *
+ *   z      = x W_r + b                      linear router, fp32 logits
+ *   S_t    = the k largest z[t][.]          ties go to the lower expert index
+ *   g[t,j] = softmax of z over S_t          gates over the kept k only
+ *   C      = ceil(T k cf / E)               expert capacity (cf = inf: C = T)
+ *   each expert keeps its first C assignments in token order; the rest drop
+ *   out[t] = sum_{kept j} g[t,j] FFN_{S_t[j]}(x_t) + sum_s FFNshared_s(x_t)
+ *   FFN(x) = (silu(x w1) * (x w3)) w2
+ *   aux    = E sum_e f_e P_e,  f_e = routed_e / (T k),  P_e = mean_t softmax(z_t)_e
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated; the caller owns every
+ *     buffer.  The library never allocates device memory and never
+ *     synchronises the stream (except moe_read_device_status, which says so).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *   - Calls are asynchronous.  The return value reports host-side argument
+ *     checks and launch errors only; nothing is launched when a check fails.
+ *     A device-side error (a bounded wait that ran out) is recorded in the
+ *     status word inside the workspace; read it with moe_read_device_status.
+ *   - 16-byte alignment is required for every tensor pointer.
+ *   - `ws`/`ws_bytes` is the caller's workspace of at least
+ *     moe_workspace_size(cfg) bytes (else MOE_ERR_WORKSPACE).
+ *   - Row-major layouts throughout.  "act" is the activation/weight dtype
+ *     of the config (bf16 or fp32).
+ *   - moe_last_error() returns a thread-local text for the last failing call.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = 1,         /* null pointer or invalid scalar argument */
+    MOE_ERR_SHAPE = 2,       /* unsupported sizes (see moe_config) */
+    MOE_ERR_DTYPE = 3,       /* unsupported dtype */
+    MOE_ERR_ALIGN = 4,       /* pointer not 16-byte aligned */
+    MOE_ERR_WORKSPACE = 5,   /* workspace smaller than moe_workspace_size */
+    MOE_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    MOE_ERR_TIMEOUT = 7,     /* a device-side bounded wait ran out (device status) */
+    MOE_ERR_UNSUPPORTED = 8  /* no sm_100 device, or a feature not built */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer configuration.
+ *   T         tokens in the batch (0 allowed: every call is a no-op that
+ *             writes zero statistics)
+ *   d         model width, multiple of 128
+ *   h         routed-expert hidden width, multiple of 128
+ *   E         routed experts, 1..1024
+ *   k         experts kept per token, 1..min(E, 8)
+ *   n_shared  shared experts applied to every token (0 = none); they are
+ *             fused into one expert of width n_shared * h_shared
+ *   h_shared  hidden width of each shared expert, multiple of 128
+ *   cf_num / cf_den  capacity factor; cf_den == 0 means no capacity limit
+ *   act_dtype MOE_BF16 (tensor-core path) or MOE_F32 (fp32 SIMT path; no TF32)
+ *   has_bias  1 if the router has a bias vector b[E]                       */
+typedef struct {
+    int64_t T;
+    int32_t d, h, E, k, n_shared, h_shared;
+    int64_t cf_num, cf_den;
+    int32_t act_dtype;
+    int32_t has_bias;
+} moe_config;
+
+/* Routing statistics [MoE routing fully explained, "Easy explanation" ¶4 and
+ * "Main insights" ¶3], written to DEVICE memory by moe_aux_stats.
+ *   aux_loss       E * sum_e f_e P_e  (f from assignments before the capacity
+ *                  limit; exactly 1 for perfectly even routing)
+ *   overflow_rate  dropped assignments / (T k)
+ *   mean_entropy   mean over tokens of -sum_e p ln p of the full softmax (nats)
+ *   tokens, dropped  T and the dropped assignment count (as doubles)      */
+typedef struct {
+    double aux_loss;
+    double overflow_rate;
+    double mean_entropy;
+    double tokens;
+    double dropped;
+} moe_stats;
+
+/* ---- host-only helpers (no device work) -------------------------------- */
+
+/* Expert capacity C = ceil(T k cf_num / (E cf_den)) in exact integer
+ * arithmetic [MoE routing fully explained, "Easy explanation" ¶5: batch x
+ * top-k x capacity factor / experts, e.g. 2048, 8, top-2, 1.25 -> 640].
+ * cf_den == 0 gives C = T.  Writes *C; returns MOE_OK or MOE_ERR_ARG. */
+MOE_API int moe_capacity(const moe_config* cfg, int64_t* C);
+
+/* Bytes of device workspace every call below needs for this config (the same
+ * buffer may be reused across calls with the same config).  Layout inside is
+ * private; its first 256 bytes hold the device status word. */
+MOE_API int moe_workspace_size(const moe_config* cfg, size_t* bytes);
+
+/* Upper bound on the rows of the permuted (expert-sorted, padded) buffers
+ * x_perm / y_perm that moe_dispatch and moe_expert_ffn use. */
+MOE_API int moe_perm_rows(const moe_config* cfg, int64_t* rows);
+
+/* Number of split-K partial buffers moe_expert_ffn writes into y_perm
+ * (y_perm is [splits][moe_perm_rows][d] fp32). */
+MOE_API int moe_ffn_splits(const moe_config* cfg, int32_t* splits);
+
+/* Text of the last failing call on this thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* ---- layout transform -------------------------------------------------- */
+
+/* Packs expert weights from the y = x W layout into the tensor-core layout.
+ * which = 0 (routed): w1, w3 [E][d][h], w2 [E][h][d] ->
+ *   W13 [E][2h][d]: for hidden block b (128 wide) rows 256b..256b+127 are
+ *   columns 128b.. of w1 (gate) transposed, rows 256b+128.. the same columns
+ *   of w3 (up); W2p [E][d][h] = w2 transposed (reduction dim contiguous).
+ * which = 1 (shared): w1, w3 [S][d][hs], w2 [S][hs][d] are fused into one
+ *   expert of width S*hs (hidden index s*hs + j) and packed the same way:
+ *   W13 [2*S*hs][d], W2p [d][S*hs].
+ * All in act dtype.  One-time transform; inputs are not modified. */
+MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const void* w3,
+                     const void* w2, void* W13, void* W2p, void* stream);
+
+/* ---- the layer's steps ------------------------------------------------- */
+
+/* Router [Mixtral explained, "Easy explanation" ¶3]: z = x W_r + b in fp32,
+ * top-k per token (descending logit, ties to the lower index) and gates
+ * softmax over the kept k.  Also writes the full-softmax partial sums used
+ * by moe_aux_stats into ws.
+ *   x [T][d] act; Wr [d][E] fp32; bias [E] fp32 (ignored unless has_bias)
+ *   topk_idx [T][k] int32; topk_gate [T][k] fp32                          */
+MOE_API int moe_route(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
+              int32_t* topk_idx, float* topk_gate, void* ws, size_t ws_bytes,
+              void* stream);
+
+/* Dispatch under capacity [MoE routing fully explained, "Easy explanation"
+ * ¶3 and ¶5]: per-expert counts, stable rank of every assignment within its
+ * expert by token index, truncation at C (overflow dropped), and the gather
+ * of kept rows into expert-sorted order.  Needs ws from moe_route (block
+ * histograms).
+ *   routed [E], kept [E] int32      assignments before / after the limit
+ *   offsets [E+1] int32             first row of each expert in x_perm
+ *                                   (segments padded for the tensor-core tiles)
+ *   perm_token [moe_perm_rows] int32  token of each row (-1 in padding)
+ *   slot_of [T][k] int32            row of x_perm holding (t, j), -1 if dropped
+ *   x_perm [moe_perm_rows][d] act   gathered rows (padding rows undefined)   */
+MOE_API int moe_dispatch(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                 int32_t* routed, int32_t* kept, int32_t* offsets, int32_t* perm_token,
+                 int32_t* slot_of, void* x_perm, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/* Expert FFNs [Mixtral explained, "Easy explanation" ¶2 and ¶4]: for every
+ * expert with kept tokens, H = silu(x_perm W1) * (x_perm W3) then y = H W2,
+ * as grouped GEMMs on the tensor cores (bf16 in, fp32 accumulate, H stored
+ * bf16); experts with no tokens are not read.  The shared experts (if any)
+ * run on x directly.
+ *   x_perm, offsets, kept  from moe_dispatch
+ *   W13, W2p               packed routed weights; W13s, W2s packed shared
+ *   y_perm [splits][moe_perm_rows][d] fp32  split-K partial outputs (ungated)
+ *   y_shared [T][d] fp32   sum of the shared experts (may be NULL if none)  */
+MOE_API int moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                   const int32_t* kept, const void* W13, const void* W2p, const void* x,
+                   const void* W13s, const void* W2s, float* y_perm, float* y_shared,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* Combine [Mixtral explained, "Easy explanation" ¶3; wiki, "How it works"]:
+ * out[t] = sum_j gate[t][j] * (sum over splits of y_perm[.][slot_of[t][j]])
+ * + y_shared[t], summed in fixed j order in fp32, stored in act dtype.
+ *   out [T][d] act; must not alias x                                        */
+MOE_API int moe_combine(const moe_config* cfg, const float* y_perm, const int32_t* slot_of,
+                const float* topk_gate, const float* y_shared, void* out, void* stream);
+
+/* Statistics [MoE routing fully explained, "Easy explanation" ¶4, "Main
+ * insights" ¶3]: reduces the router partials in ws (fixed order, fp64) with
+ * the counts into *stats (device).  Needs ws from moe_route. */
+MOE_API int moe_aux_stats(const moe_config* cfg, const int32_t* routed, const int32_t* kept,
+                  const void* ws, size_t ws_bytes, moe_stats* stats, void* stream);
+
+/* Split form of moe_aux_stats for data-parallel use: moe_stats_sums writes
+ * the additive sums [2 + 3E] doubles (T, entropy sum, P sums [E], routed [E],
+ * kept [E]) to `sums` (device); after the caller has summed them across
+ * ranks, moe_stats_finalize turns them into *stats. */
+MOE_API int moe_stats_sums(const moe_config* cfg, const int32_t* routed, const int32_t* kept,
+                   const void* ws, size_t ws_bytes, double* sums, void* stream);
+MOE_API int moe_stats_finalize(const moe_config* cfg, const double* sums, moe_stats* stats,
+                       void* stream);
+
+/* The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine and
+ * moe_aux_stats in sequence on one stream, with the intermediates in ws.
+ * W13s/W2s may be NULL when n_shared == 0; bias may be NULL when !has_bias;
+ * stats may be NULL to skip the statistics. */
+MOE_API int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
+                const void* W13, const void* W2p, const void* W13s, const void* W2s,
+                void* out, int32_t* topk_idx, float* topk_gate, int32_t* routed,
+                int32_t* kept, int32_t* slot_of, moe_stats* stats, void* ws, size_t ws_bytes,
+                void* stream);
+
+/* ---- status, tracing, limits ------------------------------------------- */
+
+/* Copies the device status word from ws to *status (MOE_OK or
+ * MOE_ERR_TIMEOUT) and clears it.  This call synchronises `stream`. */
+MOE_API int moe_read_device_status(const void* ws, int32_t* status, void* stream);
+
+/* Upper bound, in nanoseconds, on every device-side wait of the tensor-core
+ * kernels (default 2e9).  A wait that runs out records MOE_ERR_TIMEOUT in
+ * the device status word and its kernel returns early.  Process-wide. */
+MOE_API int moe_set_wait_limit_ns(uint64_t ns);
+
+/* Per-kernel timing of moe_forward.  moe_trace_begin(n) records CUDA events
+ * around every kernel moe_forward launches, for up to n calls;
+ * moe_trace_end synchronises and writes, per kernel, its name, launch count
+ * and summed milliseconds (up to cap entries; *n_out = entries written).
+ * Process-wide; not thread-safe. */
+MOE_API int moe_trace_begin(int max_calls);
+MOE_API int moe_trace_end(char (*names)[32], int* launches, double* ms, int cap, int* n_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,772 @@
+// capi.cu -- the C ABI (include/moe.h): argument checks, the per-config plan,
+// TMA descriptors and the launch sequence of the layer.
+//
+// Every entry point validates on the host before launching anything and
+// returns a moe_status; it never throws, allocates device memory or
+// synchronises (moe_read_device_status and moe_trace_end excepted, as the
+// header says).
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- errors
+
+static thread_local std::string g_err;
+
+static int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+static int ok() {
+    g_err.clear();
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                   \
+    do {                                \
+        int _s = (expr);                \
+        if (_s != MOE_OK) return _s;    \
+    } while (0)
+
+static int launched(int rc, const char* what) {
+    if (rc == 0) return MOE_OK;
+    cudaError_t e = cudaGetLastError();
+    return fail(MOE_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- plan
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+int make_plan(const moe_config* cfg, Plan* p, const char** why) {
+    if (!cfg) { *why = "cfg is NULL"; return MOE_ERR_ARG; }
+    const moe_config& c = *cfg;
+    if (c.T < 0 || c.T > (1LL << 30)) { *why = "T must be in [0, 2^30]"; return MOE_ERR_SHAPE; }
+    if (c.d < 128 || c.d % 128 || c.d > 65536) { *why = "d must be a multiple of 128 in [128, 65536]"; return MOE_ERR_SHAPE; }
+    if (c.h < 128 || c.h % 128 || c.h > 262144) { *why = "h must be a multiple of 128 in [128, 262144]"; return MOE_ERR_SHAPE; }
+    if (c.E < 1 || c.E > MAX_E) { *why = "E must be in [1, 1024]"; return MOE_ERR_SHAPE; }
+    if (c.k < 1 || c.k > MAX_K || c.k > c.E) { *why = "k must be in [1, min(E, 8)]"; return MOE_ERR_SHAPE; }
+    if (c.n_shared < 0 || c.n_shared > 64) { *why = "n_shared must be in [0, 64]"; return MOE_ERR_SHAPE; }
+    if (c.n_shared > 0 && (c.h_shared < 128 || c.h_shared % 128)) { *why = "h_shared must be a multiple of 128"; return MOE_ERR_SHAPE; }
+    if (c.cf_den < 0 || (c.cf_den > 0 && (c.cf_num <= 0 || c.cf_num > (1 << 20) || c.cf_den > (1 << 20)))) {
+        *why = "capacity factor must be cf_num/cf_den with 0 < cf_num, cf_den <= 2^20 (cf_den = 0: no limit)";
+        return MOE_ERR_ARG;
+    }
+    if (c.act_dtype != MOE_F32 && c.act_dtype != MOE_BF16) { *why = "act_dtype must be MOE_F32 or MOE_BF16"; return MOE_ERR_DTYPE; }
+    if (c.has_bias != 0 && c.has_bias != 1) { *why = "has_bias must be 0 or 1"; return MOE_ERR_ARG; }
+
+    Plan& P = *p;
+    P.T = c.T; P.d = c.d; P.h = c.h; P.E = c.E; P.k = c.k; P.S = c.n_shared;
+    P.hs = c.n_shared ? c.h_shared : 0;
+    P.hsum = P.S * P.hs;
+    P.capped = c.cf_den > 0;
+    if (P.capped) {
+        const int64_t num = c.T * (int64_t)c.k * c.cf_num;
+        const int64_t den = (int64_t)c.E * c.cf_den;
+        P.C = (num + den - 1) / den;
+    } else {
+        P.C = c.T;
+    }
+    const int64_t nmax = P.C < P.T ? P.C : P.T;  // most rows one expert can keep
+    P.bf16 = c.act_dtype == MOE_BF16;
+    P.act_bytes = P.bf16 ? 2 : 4;
+    if (!P.bf16) {
+        P.path = PATH_F32;
+        P.shared_path = PATH_F32;
+        P.pad = 16;
+    } else {
+        P.path = nmax <= SWAP_MAX_TOKENS ? PATH_SWAP : PATH_TOKEN_MAJOR;
+        P.shared_path = P.T <= SWAP_MAX_TOKENS ? PATH_SWAP : PATH_TOKEN_MAJOR;
+        P.pad = P.path == PATH_TOKEN_MAJOR ? 128 : 16;
+    }
+    P.nt_max = (int)(((nmax > 0 ? nmax : 1) + 15) / 16 * 16);
+    // split-K of the swapped down projection: enough units for ~6.5 waves of 148 SMs
+    P.splits = 1;
+    if (P.path == PATH_SWAP) {
+        const int64_t units = (int64_t)P.E * (P.d / 128);
+        const int kblocks = P.h / 64;
+        while (P.splits < 8 && units * P.splits < 960 && kblocks % (P.splits * 2) == 0)
+            P.splits *= 2;
+    }
+    const int64_t assign = c.T * (int64_t)c.k;
+    const int64_t cap_all = (int64_t)c.E * nmax;
+    const int64_t kept_max = assign < cap_all ? assign : cap_all;
+    P.perm_rows = c.T > 0 ? kept_max + (int64_t)c.E * (P.pad - 1) : 0;
+    P.nblk = (int)((c.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+    P.off_status = take(256);
+    P.off_logits = take((size_t)c.T * c.E * 4);
+    P.off_ppart = take((size_t)P.nblk * c.E * 4);
+    P.off_hpart = take((size_t)P.nblk * 4);
+    P.off_cnt = take((size_t)P.nblk * c.E * 4);
+    P.off_offsets = take((size_t)(c.E + 1) * 4);
+    P.off_perm = take((size_t)P.perm_rows * 4);
+    P.off_xperm = take((size_t)P.perm_rows * c.d * P.act_bytes);
+    P.off_H = take((size_t)P.perm_rows * c.h * P.act_bytes);
+    P.off_y = take((size_t)P.splits * P.perm_rows * c.d * 4);
+    P.off_Hs = take(P.S ? (size_t)c.T * P.hsum * P.act_bytes : 0);
+    P.off_ys = take(P.S ? (size_t)c.T * c.d * 4 : 0);
+    P.off_sums = take((size_t)(2 + 3 * c.E) * 8);
+    P.total = o;
+    return MOE_OK;
+}
+
+static int plan_or_fail(const moe_config* cfg, Plan* p) {
+    const char* why = "";
+    int s = make_plan(cfg, p, &why);
+    if (s != MOE_OK) return fail(s, "invalid config: %s", why);
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------- device facts
+
+struct Device {
+    int sms = 0;
+    int smem_optin = 0;
+    bool sm100 = false;
+};
+
+static int device_facts(Device* dv) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaGetDevice failed");
+    static std::mutex mu;
+    static std::vector<Device> cache;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1);
+    Device& c = cache[dev];
+    if (c.sms == 0) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&c.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        c.sm100 = (major == 10 && minor == 0);
+        if (c.sms == 0) return fail(MOE_ERR_CUDA, "could not query the device");
+    }
+    *dv = c;
+    if (!c.sm100) return fail(MOE_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) only");
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 row-major [rows][cols], box of 64 columns (128 B, 128-byte swizzle) x box_rows.
+static int tmap_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a %lldx%lld tensor", (int)r,
+                    (long long)rows, (long long)cols);
+    return MOE_OK;
+}
+
+// ---------------------------------------------------------------- limits and tracing
+
+static uint64_t g_wait_limit_ns = 2000000000ull;
+
+struct TraceMark {
+    cudaEvent_t ev;
+    const char* name;
+    int call;
+};
+
+struct Tracer {
+    bool on = false;
+    int max_calls = 0;
+    int calls = 0;
+    std::vector<cudaEvent_t> pool;
+    std::vector<TraceMark> marks;
+};
+
+static Tracer g_trace;
+
+static void trace_mark(cudaStream_t st, const char* name) {
+    if (!g_trace.on || g_trace.calls > g_trace.max_calls) return;
+    if (g_trace.marks.size() >= g_trace.pool.size()) return;
+    cudaEvent_t ev = g_trace.pool[g_trace.marks.size()];
+    cudaEventRecord(ev, st);
+    g_trace.marks.push_back({ev, name, g_trace.calls});
+}
+
+static void trace_call_begin(cudaStream_t st) {
+    if (!g_trace.on) return;
+    ++g_trace.calls;
+    trace_mark(st, "begin");
+}
+
+// ---------------------------------------------------------------- checks
+
+static int need_ws(const void* ws, size_t ws_bytes, const Plan& P) {
+    if (!ws) return fail(MOE_ERR_ARG, "ws is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255)
+        return fail(MOE_ERR_ALIGN, "ws is not 256-byte aligned");
+    if (ws_bytes < P.total)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes; this config needs %zu", ws_bytes,
+                    P.total);
+    return MOE_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static int need(const void* p, const char* name) {
+    if (!p) return fail(MOE_ERR_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(MOE_ERR_ALIGN, "%s is not 16-byte aligned", name);
+    return MOE_OK;
+}
+
+static int maybe(const void* p, const char* name) {
+    if (p && !aligned16(p)) return fail(MOE_ERR_ALIGN, "%s is not 16-byte aligned", name);
+    return MOE_OK;
+}
+
+template <typename T>
+static T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
+template <typename T>
+static const T* at(const void* ws, size_t off) {
+    return reinterpret_cast<const T*>(reinterpret_cast<const uint8_t*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- steps
+
+static int step_route(const Plan& P, const Device& dv, const void* x, const float* Wr,
+                      const float* bias, int32_t* topk_idx, float* topk_gate, void* ws,
+                      cudaStream_t st) {
+    if (P.T == 0) {
+        if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "status reset failed");
+        return MOE_OK;
+    }
+    float* z = at<float>(ws, P.off_logits);
+    MOE_TRY(launched(launch_router_logits(x, P.bf16, Wr, bias, z, P.T, P.d, P.E, dv.sms, st),
+                     "router_logits"));
+    trace_mark(st, "router_logits");
+    MOE_TRY(launched(launch_topk(z, P.T, P.E, P.k, topk_idx, topk_gate, at<float>(ws, P.off_ppart),
+                                 at<float>(ws, P.off_hpart), at<int32_t>(ws, P.off_cnt),
+                                 at<int32_t>(ws, P.off_status), st),
+                     "topk"));
+    trace_mark(st, "topk");
+    return MOE_OK;
+}
+
+static int step_dispatch(const Plan& P, const Device& dv, const int32_t* topk_idx, const void* x,
+                         int32_t* routed, int32_t* kept, int32_t* offsets, int32_t* perm_token,
+                         int32_t* slot_of, void* x_perm, void* ws, cudaStream_t st) {
+    if (P.T == 0) {
+        // empty batch: zero counts and offsets so later steps see no work
+        if (cudaMemsetAsync(routed, 0, P.E * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(kept, 0, P.E * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, (P.E + 1) * 4, st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "memset failed");
+        return MOE_OK;
+    }
+    MOE_TRY(launched(launch_dispatch(topk_idx, at<int32_t>(ws, P.off_cnt), P.T, P.E, P.k, P.C,
+                                     P.pad, P.perm_rows, x, P.d * P.act_bytes, routed, kept,
+                                     offsets, perm_token, slot_of, x_perm, dv.sms, st),
+                     "dispatch"));
+    trace_mark(st, "dispatch");
+    return MOE_OK;
+}
+
+// One grouped GEMM pair (gate/up then down) on the tensor cores.
+static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
+                      const int32_t* rows, const int32_t* offs, int dense_rows, const void* act,
+                      int64_t act_rows, const void* W13, const void* W2p, int hid, void* H,
+                      float* y, int splits, int nt_max, int32_t* status, cudaStream_t st,
+                      const char* tag1, const char* tag2) {
+    const bool tok = path == PATH_TOKEN_MAJOR;
+    CUtensorMap m_act, m_w;
+    TcArgs a;
+    memset(&a, 0, sizeof a);
+    a.num_groups = groups;
+    a.group_rows = rows;
+    a.group_off = offs;
+    a.dense_rows = dense_rows;
+    a.status = status;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.nt_max = nt_max;
+    const int smem_limit = dv.smem_optin;
+
+    // gate/up: act [act_rows][d] x W13 [groups * 2hid][d] -> H [act_rows][hid]
+    const int mode1 = tok ? TC_GATEUP_TOK : TC_GATEUP_SWAP;
+    MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, tok ? 128 : 16));
+    MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, tok ? 256 : 128));
+    a.K = P.d;
+    a.n_feat = hid;
+    a.w_rows_per_group = 2 * hid;
+    a.splits = 1;
+    a.out = H;
+    a.out_ld = hid;
+    a.split_stride = 0;
+    a.stages = tc_max_stages(mode1, 256, nt_max, groups, smem_limit);
+    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
+    trace_mark(st, tag1);
+
+    // down: H [act_rows][hid] x W2p [groups * d][hid] -> y [splits][act_rows][d]
+    const int mode2 = tok ? TC_DOWN_TOK : TC_DOWN_SWAP;
+    const int bn = (P.d % 256 == 0) ? 256 : 128;
+    MOE_TRY(tmap_bf16(&m_act, H, act_rows, hid, tok ? 128 : 16));
+    MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, tok ? bn : 128));
+    a.K = hid;
+    a.n_feat = P.d;
+    a.w_rows_per_group = P.d;
+    a.splits = tok ? 1 : splits;
+    a.out = y;
+    a.out_ld = P.d;
+    a.split_stride = act_rows * (int64_t)P.d;
+    a.stages = tc_max_stages(mode2, bn, nt_max, groups, smem_limit);
+    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    MOE_TRY(launched(launch_tc_gemm(mode2, bn, m_act, m_w, a, dv.sms, st), tag2));
+    trace_mark(st, tag2);
+    return MOE_OK;
+}
+
+static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const int32_t* offsets,
+                    const int32_t* kept, const void* W13, const void* W2p, const void* x,
+                    const void* W13s, const void* W2s, float* y_perm, float* y_shared, void* ws,
+                    cudaStream_t st) {
+    if (P.T == 0) return MOE_OK;
+    void* H = at<void>(ws, P.off_H);
+    int32_t* status = at<int32_t>(ws, P.off_status);
+    if (P.path == PATH_F32) {
+        MOE_TRY(launched(launch_f32_gateup(reinterpret_cast<const float*>(x_perm),
+                                           reinterpret_cast<const float*>(W13),
+                                           reinterpret_cast<float*>(H), P.E, kept, offsets, 0,
+                                           P.perm_rows, P.d, P.h, st),
+                         "f32_gateup"));
+        trace_mark(st, "f32_gateup");
+        MOE_TRY(launched(launch_f32_down(reinterpret_cast<const float*>(H),
+                                         reinterpret_cast<const float*>(W2p), y_perm, P.E, kept,
+                                         offsets, 0, P.perm_rows, P.d, P.h, st),
+                         "f32_down"));
+        trace_mark(st, "f32_down");
+    } else {
+        MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, 0, x_perm, P.perm_rows, W13, W2p,
+                           P.h, H, y_perm, P.splits, P.nt_max, status, st, "gemm_gateup",
+                           "gemm_down"));
+    }
+    if (P.S > 0) {
+        void* Hs = at<void>(ws, P.off_Hs);
+        if (P.shared_path == PATH_F32) {
+            MOE_TRY(launched(launch_f32_gateup(reinterpret_cast<const float*>(x),
+                                               reinterpret_cast<const float*>(W13s),
+                                               reinterpret_cast<float*>(Hs), 1, nullptr, nullptr,
+                                               (int)P.T, P.T, P.d, P.hsum, st),
+                             "f32_shared_gateup"));
+            trace_mark(st, "f32_shared_gateup");
+            MOE_TRY(launched(launch_f32_down(reinterpret_cast<const float*>(Hs),
+                                             reinterpret_cast<const float*>(W2s), y_shared, 1,
+                                             nullptr, nullptr, (int)P.T, P.T, P.d, P.hsum, st),
+                             "f32_shared_down"));
+            trace_mark(st, "f32_shared_down");
+        } else {
+            const int nt = (int)((P.T + 15) / 16 * 16);
+            MOE_TRY(run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, (int)P.T, x, P.T, W13s,
+                               W2s, P.hsum, Hs, y_shared, 1, nt, status, st, "gemm_shared_gateup",
+                               "gemm_shared_down"));
+        }
+    }
+    return MOE_OK;
+}
+
+static int step_combine(const Plan& P, const float* y_perm, const int32_t* slot_of,
+                        const float* gate, const float* y_shared, void* out, cudaStream_t st) {
+    const int splits = P.path == PATH_F32 ? 1 : (P.path == PATH_SWAP ? P.splits : 1);
+    MOE_TRY(launched(launch_combine(y_perm, splits, P.perm_rows * (int64_t)P.d, slot_of, gate,
+                                    P.S > 0 ? y_shared : nullptr, out, P.bf16, P.T, P.d, P.k, st),
+                     "combine"));
+    trace_mark(st, "combine");
+    return MOE_OK;
+}
+
+static int step_stats(const Plan& P, const int32_t* routed, const int32_t* kept, const void* ws,
+                      double* sums, moe_stats* stats, cudaStream_t st) {
+    MOE_TRY(launched(launch_stats_sums(at<float>(ws, P.off_ppart), at<float>(ws, P.off_hpart),
+                                       P.nblk, routed, kept, P.T, P.E, sums, st),
+                     "stats_sums"));
+    trace_mark(st, "stats_sums");
+    if (stats) {
+        MOE_TRY(launched(launch_stats_finalize(sums, P.E, P.k, stats, st), "stats_finalize"));
+        trace_mark(st, "stats_finalize");
+    }
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+// ================================================================ C ABI
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+int moe_capacity(const moe_config* cfg, int64_t* C) {
+    if (!C) return fail(MOE_ERR_ARG, "C is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (cfg->cf_den == 0) {
+        *C = cfg->T;
+    } else {
+        const int64_t num = cfg->T * (int64_t)cfg->k * cfg->cf_num;
+        const int64_t den = (int64_t)cfg->E * cfg->cf_den;
+        *C = (num + den - 1) / den;
+    }
+    return ok();
+}
+
+int moe_workspace_size(const moe_config* cfg, size_t* bytes) {
+    if (!bytes) return fail(MOE_ERR_ARG, "bytes is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    *bytes = P.total;
+    return ok();
+}
+
+int moe_perm_rows(const moe_config* cfg, int64_t* rows) {
+    if (!rows) return fail(MOE_ERR_ARG, "rows is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    *rows = P.perm_rows;
+    return ok();
+}
+
+int moe_ffn_splits(const moe_config* cfg, int32_t* splits) {
+    if (!splits) return fail(MOE_ERR_ARG, "splits is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    *splits = P.path == PATH_SWAP ? P.splits : 1;
+    return ok();
+}
+
+int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const void* w3,
+                     const void* w2, void* W13, void* W2p, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (which != 0 && which != 1) return fail(MOE_ERR_ARG, "which must be 0 (routed) or 1 (shared)");
+    if (which == 1 && P.S == 0) return fail(MOE_ERR_ARG, "config has no shared experts");
+    MOE_TRY(need(w1, "w1"));
+    MOE_TRY(need(w3, "w3"));
+    MOE_TRY(need(w2, "w2"));
+    MOE_TRY(need(W13, "W13"));
+    MOE_TRY(need(W2p, "W2p"));
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int eb = P.act_bytes;
+    const int n = which == 0 ? P.E : P.S;
+    const int hid = which == 0 ? P.h : P.hs;
+    const int64_t d = P.d;
+    for (int e = 0; e < n; ++e) {
+        const uint8_t* s1 = reinterpret_cast<const uint8_t*>(w1) + (size_t)e * d * hid * eb;
+        const uint8_t* s3 = reinterpret_cast<const uint8_t*>(w3) + (size_t)e * d * hid * eb;
+        const uint8_t* s2 = reinterpret_cast<const uint8_t*>(w2) + (size_t)e * hid * d * eb;
+        if (which == 0) {
+            uint8_t* d13 = reinterpret_cast<uint8_t*>(W13) + (size_t)e * 2 * hid * d * eb;
+            uint8_t* d2 = reinterpret_cast<uint8_t*>(W2p) + (size_t)e * d * hid * eb;
+            MOE_TRY(launched(launch_pack(s1, d13, eb, (int)d, hid, d, 0, 0, st), "pack"));
+            MOE_TRY(launched(launch_pack(s3, d13, eb, (int)d, hid, d, 0, 1, st), "pack"));
+            MOE_TRY(launched(launch_pack(s2, d2, eb, hid, (int)d, hid, 0, -1, st), "pack"));
+        } else {
+            // shared experts fused into one of width S*hs: hidden index e*hs + j
+            MOE_TRY(launched(launch_pack(s1, W13, eb, (int)d, hid, d, e * hid, 0, st), "pack"));
+            MOE_TRY(launched(launch_pack(s3, W13, eb, (int)d, hid, d, e * hid, 1, st), "pack"));
+            uint8_t* d2 = reinterpret_cast<uint8_t*>(W2p) + (size_t)e * hid * eb;
+            MOE_TRY(launched(launch_pack(s2, d2, eb, hid, (int)d, P.hsum, 0, -1, st), "pack"));
+        }
+    }
+    return ok();
+}
+
+int moe_route(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
+              int32_t* topk_idx, float* topk_gate, void* ws, size_t ws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    if (P.T > 0) {
+        MOE_TRY(need(x, "x"));
+        MOE_TRY(need(Wr, "Wr"));
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(topk_gate, "topk_gate"));
+        if (cfg->has_bias) MOE_TRY(need(bias, "bias"));
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    MOE_TRY(step_route(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate, ws,
+                       reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_dispatch(const moe_config* cfg, const int32_t* topk_idx, const void* x, int32_t* routed,
+                 int32_t* kept, int32_t* offsets, int32_t* perm_token, int32_t* slot_of,
+                 void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(routed, "routed"));
+    MOE_TRY(need(kept, "kept"));
+    MOE_TRY(need(offsets, "offsets"));
+    if (P.T > 0) {
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(x, "x"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(need(x_perm, "x_perm"));
+        MOE_TRY(maybe(perm_token, "perm_token"));
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    MOE_TRY(step_dispatch(P, dv, topk_idx, x, routed, kept, offsets, perm_token, slot_of, x_perm,
+                          ws, reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                   const int32_t* kept, const void* W13, const void* W2p, const void* x,
+                   const void* W13s, const void* W2s, float* y_perm, float* y_shared, void* ws,
+                   size_t ws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    if (P.T > 0) {
+        MOE_TRY(need(x_perm, "x_perm"));
+        MOE_TRY(need(offsets, "offsets"));
+        MOE_TRY(need(kept, "kept"));
+        MOE_TRY(need(W13, "W13"));
+        MOE_TRY(need(W2p, "W2p"));
+        MOE_TRY(need(y_perm, "y_perm"));
+        if (P.S > 0) {
+            MOE_TRY(need(x, "x"));
+            MOE_TRY(need(W13s, "W13s"));
+            MOE_TRY(need(W2s, "W2s"));
+            MOE_TRY(need(y_shared, "y_shared"));
+        }
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    MOE_TRY(step_ffn(P, dv, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y_perm, y_shared, ws,
+                     reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_combine(const moe_config* cfg, const float* y_perm, const int32_t* slot_of,
+                const float* topk_gate, const float* y_shared, void* out, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (P.T > 0) {
+        MOE_TRY(need(y_perm, "y_perm"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(need(topk_gate, "topk_gate"));
+        MOE_TRY(need(out, "out"));
+        if (P.S > 0) MOE_TRY(need(y_shared, "y_shared"));
+    }
+    MOE_TRY(step_combine(P, y_perm, slot_of, topk_gate, y_shared, out,
+                         reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_stats_sums(const moe_config* cfg, const int32_t* routed, const int32_t* kept,
+                   const void* ws, size_t ws_bytes, double* sums, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(sums, "sums"));
+    MOE_TRY(need(routed, "routed"));
+    MOE_TRY(need(kept, "kept"));
+    MOE_TRY(step_stats(P, routed, kept, ws, sums, nullptr, reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_stats_finalize(const moe_config* cfg, const double* sums, moe_stats* stats,
+                       void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need(sums, "sums"));
+    MOE_TRY(need(stats, "stats"));
+    MOE_TRY(launched(launch_stats_finalize(sums, P.E, P.k, stats,
+                                           reinterpret_cast<cudaStream_t>(stream)),
+                     "stats_finalize"));
+    return ok();
+}
+
+int moe_aux_stats(const moe_config* cfg, const int32_t* routed, const int32_t* kept,
+                  const void* ws, size_t ws_bytes, moe_stats* stats, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(stats, "stats"));
+    MOE_TRY(need(routed, "routed"));
+    MOE_TRY(need(kept, "kept"));
+    double* sums = const_cast<double*>(at<double>(ws, P.off_sums));
+    MOE_TRY(step_stats(P, routed, kept, ws, sums, stats, reinterpret_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
+                const void* W13, const void* W2p, const void* W13s, const void* W2s, void* out,
+                int32_t* topk_idx, float* topk_gate, int32_t* routed, int32_t* kept,
+                int32_t* slot_of, moe_stats* stats, void* ws, size_t ws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(routed, "routed"));
+    MOE_TRY(need(kept, "kept"));
+    MOE_TRY(maybe(stats, "stats"));
+    if (P.T > 0) {
+        MOE_TRY(need(x, "x"));
+        MOE_TRY(need(Wr, "Wr"));
+        MOE_TRY(need(W13, "W13"));
+        MOE_TRY(need(W2p, "W2p"));
+        MOE_TRY(need(out, "out"));
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(topk_gate, "topk_gate"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        if (cfg->has_bias) MOE_TRY(need(bias, "bias"));
+        if (P.S > 0) {
+            MOE_TRY(need(W13s, "W13s"));
+            MOE_TRY(need(W2s, "W2s"));
+        }
+        if (out == x) return fail(MOE_ERR_ARG, "out must not alias x");
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    trace_call_begin(st);
+    int32_t* offsets = at<int32_t>(ws, P.off_offsets);
+    int32_t* perm = at<int32_t>(ws, P.off_perm);
+    void* x_perm = at<void>(ws, P.off_xperm);
+    float* y = at<float>(ws, P.off_y);
+    float* ys = P.S ? at<float>(ws, P.off_ys) : nullptr;
+    MOE_TRY(step_route(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate, ws, st));
+    MOE_TRY(step_dispatch(P, dv, topk_idx, x, routed, kept, offsets, perm, slot_of, x_perm, ws,
+                          st));
+    MOE_TRY(step_ffn(P, dv, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st));
+    if (P.T > 0) MOE_TRY(step_combine(P, y, slot_of, topk_gate, ys, out, st));
+    if (stats)
+        MOE_TRY(step_stats(P, routed, kept, ws, at<double>(ws, P.off_sums), stats, st));
+    return ok();
+}
+
+int moe_read_device_status(const void* ws, int32_t* status, void* stream) {
+    MOE_TRY(need(ws, "ws"));
+    if (!status) return fail(MOE_ERR_ARG, "status is NULL");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "reading the device status failed: %s",
+                    cudaGetErrorString(cudaGetLastError()));
+    if (cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof v, st) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "clearing the device status failed");
+    *status = v;
+    return ok();
+}
+
+int moe_set_wait_limit_ns(uint64_t ns) {
+    g_wait_limit_ns = ns;
+    return ok();
+}
+
+int moe_trace_begin(int max_calls) {
+    if (max_calls < 1 || max_calls > 100000) return fail(MOE_ERR_ARG, "max_calls out of range");
+    const size_t need_ev = (size_t)max_calls * 16;
+    while (g_trace.pool.size() < need_ev) {
+        cudaEvent_t ev;
+        if (cudaEventCreate(&ev) != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaEventCreate failed");
+        g_trace.pool.push_back(ev);
+    }
+    g_trace.marks.clear();
+    g_trace.calls = 0;
+    g_trace.max_calls = max_calls;
+    g_trace.on = true;
+    return ok();
+}
+
+int moe_trace_end(char (*names)[32], int* launches, double* ms, int cap, int* n_out) {
+    g_trace.on = false;
+    if (!n_out) return fail(MOE_ERR_ARG, "n_out is NULL");
+    std::vector<std::string> nm;
+    std::vector<int> cnt;
+    std::vector<double> tot;
+    for (size_t i = 1; i < g_trace.marks.size(); ++i) {
+        const TraceMark& a = g_trace.marks[i - 1];
+        const TraceMark& b = g_trace.marks[i];
+        if (a.call != b.call) continue;
+        if (cudaEventSynchronize(b.ev) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "cudaEventSynchronize failed");
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, a.ev, b.ev) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "cudaEventElapsedTime failed");
+        size_t j = 0;
+        while (j < nm.size() && nm[j] != b.name) ++j;
+        if (j == nm.size()) {
+            nm.push_back(b.name);
+            cnt.push_back(0);
+            tot.push_back(0.0);
+        }
+        cnt[j] += 1;
+        tot[j] += t;
+    }
+    int n = 0;
+    for (size_t j = 0; j < nm.size() && n < cap; ++j, ++n) {
+        if (names) {
+            strncpy(names[n], nm[j].c_str(), 31);
+            names[n][31] = 0;
+        }
+        if (launches) launches[n] = cnt[j];
+        if (ms) ms[n] = tot[j];
+    }
+    *n_out = n;
+    g_trace.marks.clear();
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,185 @@
+// combine.cu -- gate-weighted combine, routing statistics and weight packing.
+//
+// Combine [Mixtral 8x7B and MoE explained, "Easy explanation" ¶3: the chosen
+// experts' outputs are summed with the gate weights; "Mixture of experts"
+// wiki, "How it works": weighted by the router's confidence; MoE routing
+// fully explained, "Easy explanation" ¶4: shared experts see every token]:
+//   out[t] = sum_j g[t,j] * (sum_s y[s][slot(t,j)]) + y_shared[t]
+// with j and s in fixed order, fp32, one thread per 8 output columns (two
+// 16-byte loads per row read, one 16-byte bf16x8 store).  A dropped
+// assignment contributes nothing and the other gates are not renormalised.
+//
+// Statistics [MoE routing fully explained, "Easy explanation" ¶4, "Main
+// insights" ¶3]: the load-balancing loss E * sum_e f_e P_e, the overflow
+// rate and the mean router entropy, reduced from the per-block partials in a
+// fixed order in fp64.
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+
+namespace moe {
+
+namespace {
+
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float* __restrict__ y, int splits, int64_t split_stride,
+                   const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
+                   const float* __restrict__ ys, void* __restrict__ out, int64_t T, int d, int k) {
+    const int vecs = d / 8;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * vecs) return;
+    const int64_t t = i / vecs;
+    const int c = (int)(i % vecs) * 8;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j = 0; j < k; ++j) {
+        const int32_t slot = slot_of[t * k + j];
+        if (slot < 0) continue;
+        const float g = gate[t * k + j];
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float* p = y + s * split_stride + (int64_t)slot * d + c;
+            const float4 a = *reinterpret_cast<const float4*>(p);
+            const float4 b = *reinterpret_cast<const float4*>(p + 4);
+            v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+            v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(g, v[q], acc[q]);
+    }
+    if (ys) {
+        const float* p = ys + t * d + c;
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    if (OUT_BF16) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + t * d + c) = o;
+    } else {
+        float* p = reinterpret_cast<float*>(out) + t * d + c;
+        *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
+// sums = [T, entropy sum, P sums (E), routed (E), kept (E)]
+__global__ void stats_sums_kernel(const float* __restrict__ ppart, const float* __restrict__ hpart,
+                                  int nblk, const int32_t* __restrict__ routed,
+                                  const int32_t* __restrict__ kept, int64_t T, int E,
+                                  double* __restrict__ sums) {
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        double h = 0.0;
+        for (int b = 0; b < nblk; ++b) h += (double)hpart[b];
+        sums[0] = (double)T;
+        sums[1] = h;
+    }
+    for (int e = tid; e < E; e += blockDim.x) {
+        double p = 0.0;
+        for (int b = 0; b < nblk; ++b) p += (double)ppart[(int64_t)b * E + e];
+        sums[2 + e] = p;
+        sums[2 + E + e] = T > 0 ? (double)routed[e] : 0.0;
+        sums[2 + 2 * E + e] = T > 0 ? (double)kept[e] : 0.0;
+    }
+}
+
+__global__ void stats_finalize_kernel(const double* __restrict__ sums, int E, int k,
+                                      moe_stats* __restrict__ st) {
+    if (threadIdx.x != 0) return;
+    const double T = sums[0];
+    moe_stats r{0.0, 0.0, 0.0, T, 0.0};
+    if (T > 0.0) {
+        const double tk = T * k;
+        double aux = 0.0, dropped = 0.0;
+        for (int e = 0; e < E; ++e) {
+            const double f = sums[2 + E + e] / tk;  // share of assignments (before the limit)
+            const double P = sums[2 + e] / T;       // mean router probability
+            aux += f * P;
+            dropped += sums[2 + E + e] - sums[2 + 2 * E + e];
+        }
+        r.aux_loss = (double)E * aux;
+        r.overflow_rate = dropped / tk;
+        r.mean_entropy = sums[1] / T;
+        r.dropped = dropped;
+    }
+    *st = r;
+}
+
+// Tiled transpose with a row remap for the packed weight layouts.
+// src [R][Cc]; dst[row(c)][r + 0] with row(c) = c + col_off, or, when
+// interleave >= 0, the gate/up interleave of 128-wide hidden blocks:
+// hidden index j = c + col_off -> row 256 * (j / 128) + 128 * interleave + j % 128.
+template <typename Tv>
+__global__ void pack_kernel(const Tv* __restrict__ src, Tv* __restrict__ dst, int R, int Cc,
+                            int64_t ld_dst, int col_off, int interleave) {
+    __shared__ Tv tile[32][33];
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < R && c < Cc) tile[i][threadIdx.x] = src[(int64_t)r * Cc + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < R && c < Cc) {
+            const int j = c + col_off;
+            const int64_t row =
+                interleave < 0 ? j : (int64_t)256 * (j / 128) + 128 * interleave + (j % 128);
+            dst[row * ld_dst + r] = tile[threadIdx.x][i];
+        }
+    }
+}
+
+}  // namespace
+
+int launch_combine(const float* y, int splits, int64_t split_stride, const int32_t* slot_of,
+                   const float* gate, const float* y_shared, void* out, bool out_bf16, int64_t T,
+                   int d, int k, cudaStream_t st) {
+    if (T == 0) return 0;
+    const int64_t n = T * (d / 8);
+    const unsigned blocks = (unsigned)((n + 255) / 256);
+    if (out_bf16)
+        combine_kernel<true><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
+                                                     y_shared, out, T, d, k);
+    else
+        combine_kernel<false><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
+                                                      y_shared, out, T, d, k);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_stats_sums(const float* ppart, const float* hpart, int nblk, const int32_t* routed,
+                      const int32_t* kept, int64_t T, int E, double* sums, cudaStream_t st) {
+    stats_sums_kernel<<<1, 256, 0, st>>>(ppart, hpart, nblk, routed, kept, T, E, sums);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStream_t st) {
+    stats_finalize_kernel<<<1, 32, 0, st>>>(sums, E, k, reinterpret_cast<moe_stats*>(stats));
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64_t ld_dst,
+                int col_off, int interleave, cudaStream_t st) {
+    dim3 grid((Cc + 31) / 32, (R + 31) / 32), block(32, 8);
+    if (elem_bytes == 2)
+        pack_kernel<uint16_t><<<grid, block, 0, st>>>(reinterpret_cast<const uint16_t*>(src),
+                                                      reinterpret_cast<uint16_t*>(dst), R, Cc,
+                                                      ld_dst, col_off, interleave);
+    else
+        pack_kernel<float><<<grid, block, 0, st>>>(reinterpret_cast<const float*>(src),
+                                                   reinterpret_cast<float*>(dst), R, Cc, ld_dst,
+                                                   col_off, interleave);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace moe

@@ -1,0 +1,486 @@
+// gemm_tc.cu -- grouped expert GEMMs on the sm_100a tensor cores.
+//
+// The expert FFN [Mixtral 8x7B and MoE explained, "Easy explanation" ¶2: each
+// expert widens the ~4k embedding to a ~14k hidden size and narrows it back;
+// ¶4: unselected experts are not computed at all] runs as two grouped GEMMs
+// over the expert-sorted token rows that dispatch produced:
+//
+//   gate/up : H[r, f] = silu(x_r . w1[:, f]) * (x_r . w3[:, f])   (bf16 out)
+//   down    : y[r, o] = H_r . w2[:, o]                              (fp32 out)
+//
+// One group per expert (or one dense group for the fused shared expert).
+// Group sizes live on the device (kept counts from dispatch); the host never
+// reads them, so the whole layer runs without a host synchronisation.
+//
+// Two tile layouts, chosen on the host from the largest possible group:
+//   token-major  (groups may exceed 256 rows: prefill)
+//     D[128 tokens x BN] = A(tokens, K-major) * B(weights, K-major)^T
+//     gate/up tiles hold 128 gate + 128 up features of the same hidden block
+//     (the packed W13 layout interleaves them), so the SiLU*mul epilogue
+//     finds both operands in one thread's TMEM lane.
+//   swapped      (every group has <= 256 rows: decode, many small experts)
+//     D[128 weight rows x N tokens] = A(weights) * B(tokens)^T, N = the
+//     group's token count rounded up to 16; each expert's weights are read
+//     exactly once.  gate and up rows go to two accumulators; the down
+//     projection may be split along K into partial outputs.
+//
+// Structure (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: fills a ring of shared-memory stages
+//   warp 1      MMA issuer (one thread) and TMEM owner
+//   warps 2..5  epilogue: TMEM -> registers -> global
+// Barriers: full/empty per stage (TMA <-> MMA), acc_full/acc_empty per TMEM
+// accumulator buffer (MMA <-> epilogue).  Every wait is bounded; a wait that
+// runs out records a timeout in the status word and the CTA winds down,
+// letting its in-flight copies and MMAs finish before TMEM is released.
+#include <stdio.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;      // MMA M (TMEM lanes)
+constexpr int BK = 64;       // K elements per stage: one 128-byte swizzle row of bf16
+constexpr int UK = 16;       // K per tcgen05.mma (bf16)
+constexpr int THREADS = 192;
+constexpr uint64_t TEARDOWN_NS = 200000000ull;  // 0.2 s bound on draining in-flight work
+
+struct SharedLayout {
+    uint32_t a_bytes, b_bytes, stage_bytes;
+    uint32_t bar_off, grp_off, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Bytes of operand per stage for each mode.
+__host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, uint32_t* a, uint32_t* b) {
+    switch (mode) {
+        case TC_GATEUP_TOK:
+        case TC_DOWN_TOK:
+            *a = BM * BK * 2;
+            *b = bn * BK * 2;
+            break;
+        case TC_GATEUP_SWAP:
+            *a = 2 * BM * BK * 2;
+            *b = nt_max * BK * 2;
+            break;
+        default:
+            *a = BM * BK * 2;
+            *b = nt_max * BK * 2;
+            break;
+    }
+}
+
+__host__ __device__ inline SharedLayout shared_layout(int mode, int bn, int nt_max, int stages,
+                                                      int groups) {
+    SharedLayout L;
+    stage_bytes(mode, bn, nt_max, &L.a_bytes, &L.b_bytes);
+    L.a_bytes = align_up(L.a_bytes, 1024);
+    L.b_bytes = align_up(L.b_bytes, 1024);
+    L.stage_bytes = L.a_bytes + L.b_bytes;
+    L.bar_off = L.stage_bytes * stages;
+    // full[S], empty[S], acc_full[2], acc_empty[2], drain, tmem slot
+    L.grp_off = L.bar_off + align_up((2 * stages + 5) * 8 + 8, 16);
+    L.total = L.grp_off + (3 * groups + 1) * 4 + 1024;  // + 1 KB for base alignment
+    return L;
+}
+
+// Where one unit of work sits.
+struct Unit {
+    int g;        // group
+    int rows;     // valid rows of the group
+    int row0;     // first row of the group in the activation/output tensors
+    int mt, nb;   // token-major: m tile, n tile;  swapped: feature block
+    int ks;       // split-K index (swapped down)
+    int kb0, kb1; // k-block range
+    int ntok;     // swapped: token columns (multiple of 16)
+};
+
+struct GroupTable {
+    const int* start;  // [groups + 1] unit prefix
+    const int* rows;   // [groups]
+    const int* off;    // [groups]
+    int groups;
+};
+
+__device__ __forceinline__ int find_group(const GroupTable& t, int u) {
+    int lo = 0, hi = t.groups - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (t.start[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+template <int MODE, int BN>
+__device__ __forceinline__ Unit decode_unit(const GroupTable& t, int u, const TcArgs& a) {
+    Unit x;
+    x.g = find_group(t, u);
+    x.rows = t.rows[x.g];
+    x.row0 = t.off[x.g];
+    const int local = u - t.start[x.g];
+    const int kblocks = a.K / BK;
+    x.ks = 0;
+    x.kb0 = 0;
+    x.kb1 = kblocks;
+    x.ntok = 0;
+    if (MODE == TC_GATEUP_TOK || MODE == TC_DOWN_TOK) {
+        const int mtiles = (x.rows + BM - 1) / BM;
+        x.mt = local % mtiles;
+        x.nb = local / mtiles;
+    } else if (MODE == TC_GATEUP_SWAP) {
+        x.mt = 0;
+        x.nb = local;
+        x.ntok = (x.rows + 15) & ~15;
+    } else {
+        x.mt = 0;
+        x.nb = local / a.splits;
+        x.ks = local % a.splits;
+        const int per = kblocks / a.splits;
+        x.kb0 = x.ks * per;
+        x.kb1 = x.kb0 + per;
+        x.ntok = (x.rows + 15) & ~15;
+    }
+    return x;
+}
+
+template <int MODE, int BN>
+__device__ __forceinline__ int units_of_group(int rows, const TcArgs& a) {
+    if (rows <= 0) return 0;
+    if (MODE == TC_GATEUP_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / 128);
+    if (MODE == TC_DOWN_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / BN);
+    if (MODE == TC_GATEUP_SWAP) return a.n_feat / 128;
+    return (a.n_feat / 128) * a.splits;
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
+                   const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
+    constexpr bool TOK = (MODE == TC_GATEUP_TOK || MODE == TC_DOWN_TOK);
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (align_up(raw, 1024) - raw);
+
+    const int groups = args.num_groups;
+    const SharedLayout L = shared_layout(MODE, BN, args.nt_max, args.stages, groups);
+    const int S = args.stages;
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+    uint64_t* empty = full + S;
+    uint64_t* acc_full = empty + S;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    int* g_start = reinterpret_cast<int*>(smem + L.grp_off);
+    int* g_rows = g_start + groups + 1;
+    int* g_off = g_rows + groups;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // accumulator geometry (TMEM columns)
+    int acc_stride, n_acc;
+    if (TOK) {
+        acc_stride = BN;
+        n_acc = 2;
+    } else if (MODE == TC_GATEUP_SWAP) {
+        acc_stride = 2 * args.nt_max;
+        n_acc = (2 * acc_stride <= 512) ? 2 : 1;
+    } else {
+        acc_stride = args.nt_max;
+        n_acc = 2;
+    }
+    uint32_t tmem_cols = 32;
+    while (tmem_cols < (uint32_t)(acc_stride * n_acc)) tmem_cols <<= 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 128);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_act);
+        prefetch_tmap(&tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    if (warp == 2 && lane == 0) {
+        int acc = 0;
+        for (int g = 0; g < groups; ++g) {
+            int r = args.group_rows ? args.group_rows[g] : args.dense_rows;
+            int o = args.group_off ? args.group_off[g] : 0;
+            g_rows[g] = r;
+            g_off[g] = o;
+            g_start[g] = acc;
+            acc += units_of_group<MODE, BN>(r, args);
+        }
+        g_start[groups] = acc;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    GroupTable tab{g_start, g_rows, g_off, groups};
+    const int total = g_start[groups];
+    const uint64_t limit = args.wait_limit_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint64_t pol_w = 0, pol_a = 0;
+            if (!TOK) {
+                pol_w = l2_policy_evict_first();
+                pol_a = l2_policy_evict_last();
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_par = 0;  // per-stage bits: loads issued / their parity
+            bool ok = true;
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                const Unit x = decode_unit<MODE, BN>(tab, u, args);
+                for (int kb = x.kb0; kb < x.kb1; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, limit)) {
+                        report_timeout(args.status);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * L.stage_bytes;
+                    uint8_t* sb = sa + L.a_bytes;
+                    const int kc = kb * BK;
+                    if (TOK) {
+                        mbar_arrive_expect_tx(&full[stage], (BM + BN) * BK * 2);
+                        tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
+                        tma_load_2d(sb, &tm_w, &full[stage], kc,
+                                    x.g * args.w_rows_per_group +
+                                        x.nb * (MODE == TC_GATEUP_TOK ? 256 : BN));
+                    } else {
+                        const int wa = (MODE == TC_GATEUP_SWAP) ? 2 * BM : BM;
+                        mbar_arrive_expect_tx(&full[stage], (wa + x.ntok) * BK * 2);
+                        const int wrow = x.g * args.w_rows_per_group +
+                                         x.nb * (MODE == TC_GATEUP_SWAP ? 256 : BM);
+                        tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
+                        if (MODE == TC_GATEUP_SWAP)
+                            tma_load_2d_hint(sa + BM * BK * 2, &tm_w, &full[stage], kc, wrow + BM,
+                                             pol_w);
+                        for (int r = 0; r < x.ntok; r += 16)
+                            tma_load_2d_hint(sb + r * BK * 2, &tm_act, &full[stage], kc,
+                                             x.row0 + r, pol_a);
+                    }
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // let every issued copy land before the CTA can release its memory
+            for (int s = 0; s < S; ++s)
+                if (issued & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1, TEARDOWN_NS);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            const uint32_t idesc_tok = idesc_bf16_f32(BM, BN);
+            for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+                const Unit x = decode_unit<MODE, BN>(tab, u, args);
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, limit)) {
+                    report_timeout(args.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * acc_stride;
+                const uint32_t idesc = TOK ? idesc_tok : idesc_bf16_f32(BM, x.ntok);
+                for (int kb = x.kb0; kb < x.kb1; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, limit)) {
+                        report_timeout(args.status);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + stage * L.stage_bytes);
+                    const uint32_t sb = sa + L.a_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk) {
+                        const uint32_t acc_flag = (kb > x.kb0 || kk > 0) ? 1u : 0u;
+                        const uint64_t bdesc = sdesc_kmajor_sw128(sb + kk * UK * 2);
+                        umma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * UK * 2), bdesc, idesc,
+                                  acc_flag);
+                        if (MODE == TC_GATEUP_SWAP)
+                            umma_bf16(d_tmem + args.nt_max,
+                                      sdesc_kmajor_sw128(sa + BM * BK * 2 + kk * UK * 2), bdesc,
+                                      idesc, acc_flag);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[acc]);
+                if (++acc == n_acc) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // every MMA issued by this thread completes before TMEM is released
+            umma_commit(drain);
+            mbar_wait(drain, 0, TEARDOWN_NS);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;          // accumulator row (TMEM lane)
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < total; u += gridDim.x) {
+            const Unit x = decode_unit<MODE, BN>(tab, u, args);
+            if (!mbar_wait(&acc_full[acc], acc_phase, limit)) {
+                report_timeout(args.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = lane_addr + acc * acc_stride;
+            if (MODE == TC_GATEUP_TOK) {
+                const int r = x.mt * BM + row;
+                const bool valid = r < x.rows;
+                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
+                                     (int64_t)(x.row0 + r) * args.out_ld + x.nb * 128;
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 16) {
+                    float g[16], v[16];
+                    tmem_ld16(t0 + c, g);
+                    tmem_ld16(t0 + 128 + c, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint4 o0, o1;
+                        o0.x = pack_bf16x2(silu_f(g[0]) * v[0], silu_f(g[1]) * v[1]);
+                        o0.y = pack_bf16x2(silu_f(g[2]) * v[2], silu_f(g[3]) * v[3]);
+                        o0.z = pack_bf16x2(silu_f(g[4]) * v[4], silu_f(g[5]) * v[5]);
+                        o0.w = pack_bf16x2(silu_f(g[6]) * v[6], silu_f(g[7]) * v[7]);
+                        o1.x = pack_bf16x2(silu_f(g[8]) * v[8], silu_f(g[9]) * v[9]);
+                        o1.y = pack_bf16x2(silu_f(g[10]) * v[10], silu_f(g[11]) * v[11]);
+                        o1.z = pack_bf16x2(silu_f(g[12]) * v[12], silu_f(g[13]) * v[13]);
+                        o1.w = pack_bf16x2(silu_f(g[14]) * v[14], silu_f(g[15]) * v[15]);
+                        *reinterpret_cast<uint4*>(dst + c) = o0;
+                        *reinterpret_cast<uint4*>(dst + c + 8) = o1;
+                    }
+                }
+            } else if (MODE == TC_DOWN_TOK) {
+                const int r = x.mt * BM + row;
+                const bool valid = r < x.rows;
+                float* dst = reinterpret_cast<float*>(args.out) +
+                             (int64_t)(x.row0 + r) * args.out_ld + x.nb * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(t0 + c, v);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<float4*>(dst + c + i) =
+                                make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    }
+                }
+            } else if (MODE == TC_GATEUP_SWAP) {
+                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
+                                     (int64_t)x.row0 * args.out_ld + x.nb * 128 + row;
+#pragma unroll 1
+                for (int c = 0; c < x.ntok; c += 16) {
+                    float g[16], v[16];
+                    tmem_ld16(t0 + c, g);
+                    tmem_ld16(t0 + args.nt_max + c, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c + i < x.rows)
+                            dst[(int64_t)(c + i) * args.out_ld] =
+                                __float2bfloat16_rn(silu_f(g[i]) * v[i]);
+                }
+            } else {
+                float* dst = reinterpret_cast<float*>(args.out) + x.ks * args.split_stride +
+                             (int64_t)x.row0 * args.out_ld + x.nb * BM + row;
+#pragma unroll 1
+                for (int c = 0; c < x.ntok; c += 16) {
+                    float v[16];
+                    tmem_ld16(t0 + c, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c + i < x.rows) dst[(int64_t)(c + i) * args.out_ld] = v[i];
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+            if (++acc == n_acc) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+template <int MODE, int BN>
+int launch_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, int grid,
+                cudaStream_t st) {
+    const SharedLayout L = shared_layout(MODE, BN, a.nt_max, a.stages, a.num_groups);
+    auto kern = tc_gemm_kernel<MODE, BN>;
+    static int configured_bytes = 0;
+    if ((int)L.total > configured_bytes) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) !=
+            cudaSuccess)
+            return -1;
+        configured_bytes = L.total;
+    }
+    kern<<<grid, THREADS, L.total, st>>>(act, w, a);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace
+
+int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit) {
+    for (int s = 8; s >= 2; --s)
+        if ((int)shared_layout(mode, bn, nt_max, s, groups).total <= smem_limit) return s;
+    return 0;
+}
+
+int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& w,
+                   const TcArgs& a, int grid, cudaStream_t st) {
+    switch (mode) {
+        case TC_GATEUP_TOK:
+            return launch_mode<TC_GATEUP_TOK, 256>(act, w, a, grid, st);
+        case TC_DOWN_TOK:
+            return bn == 256 ? launch_mode<TC_DOWN_TOK, 256>(act, w, a, grid, st)
+                             : launch_mode<TC_DOWN_TOK, 128>(act, w, a, grid, st);
+        case TC_GATEUP_SWAP:
+            return launch_mode<TC_GATEUP_SWAP, 128>(act, w, a, grid, st);
+        case TC_DOWN_SWAP:
+            return launch_mode<TC_DOWN_SWAP, 128>(act, w, a, grid, st);
+    }
+    return -1;
+}
+
+}  // namespace moe

@@ -1,0 +1,72 @@
+// kernels.h -- internal launchers of the MoE library's CUDA kernels.
+// Each returns 0 on a successful launch, -1 otherwise.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---------------------------------------------------------------- router
+// logits z[T][E] = x[T][d] Wr[d][E] + bias (fp32 accumulate)
+int launch_router_logits(const void* x, bool x_bf16, const float* Wr, const float* bias,
+                         float* z, int64_t T, int d, int E, int num_sms, cudaStream_t st);
+// per-token top-k, gates over the kept k, full-softmax partials and block histograms
+int launch_topk(const float* z, int64_t T, int E, int k, int32_t* topk_idx, float* topk_gate,
+                float* ppart, float* hpart, int32_t* cnt, int32_t* status, cudaStream_t st);
+
+// ---------------------------------------------------------------- dispatch
+int launch_dispatch(const int32_t* topk_idx, const int32_t* cnt, int64_t T, int E, int k,
+                    int64_t C, int pad, int64_t perm_rows, const void* x, int row_bytes,
+                    int32_t* routed, int32_t* kept, int32_t* offsets, int32_t* perm_token,
+                    int32_t* slot_of, void* x_perm, int num_sms, cudaStream_t st);
+
+// ---------------------------------------------------------------- tensor-core GEMMs
+enum TcMode : int { TC_GATEUP_TOK = 0, TC_DOWN_TOK = 1, TC_GATEUP_SWAP = 2, TC_DOWN_SWAP = 3 };
+
+struct TcArgs {
+    int num_groups;
+    const int32_t* group_rows;  // device [num_groups] valid rows, or nullptr -> dense_rows
+    const int32_t* group_off;   // device [num_groups] first row, or nullptr -> 0
+    int dense_rows;
+    int K;                      // reduction length
+    int n_feat;                 // gate/up: hidden width; down: model width
+    int w_rows_per_group;       // weight rows per group (gate/up: 2h; down: d)
+    int splits;                 // split-K of the swapped down projection
+    int nt_max;                 // swapped: max tokens per group, multiple of 16
+    int stages;                 // shared-memory pipeline depth
+    void* out;                  // H (bf16) or y (fp32)
+    int64_t out_ld;             // elements per output row
+    int64_t split_stride;       // elements between split-K partial outputs
+    int32_t* status;            // device status word
+    uint64_t wait_limit_ns;
+};
+
+int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);
+int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& w,
+                   const TcArgs& a, int grid, cudaStream_t st);
+
+// ---------------------------------------------------------------- fp32 SIMT FFN
+// gate/up: H[r][f] = silu(A_r . W13[g][gate f]) * (A_r . W13[g][up f]);
+// down: Y[r][o] = H_r . W2p[g][o].  Groups as in TcArgs.
+int launch_f32_gateup(const float* A, const float* W13, float* H, int num_groups,
+                      const int32_t* group_rows, const int32_t* group_off, int dense_rows,
+                      int64_t rows_bound, int d, int h, cudaStream_t st);
+int launch_f32_down(const float* H, const float* W2p, float* Y, int num_groups,
+                    const int32_t* group_rows, const int32_t* group_off, int dense_rows,
+                    int64_t rows_bound, int d, int h, cudaStream_t st);
+
+// ---------------------------------------------------------------- combine / stats / pack
+int launch_combine(const float* y, int splits, int64_t split_stride, const int32_t* slot_of,
+                   const float* gate, const float* y_shared, void* out, bool out_bf16,
+                   int64_t T, int d, int k, cudaStream_t st);
+int launch_stats_sums(const float* ppart, const float* hpart, int nblk, const int32_t* routed,
+                      const int32_t* kept, int64_t T, int E, double* sums, cudaStream_t st);
+int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStream_t st);
+// dst[remap(c)][r + row_off] = src[r][c] for a [R][Cc] source; remap interleaves
+// 128-wide hidden blocks (gate/up) when `interleave` >= 0 (0 = gate, 1 = up).
+int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64_t ld_dst,
+                int col_off, int interleave, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,49 @@
+// plan.h -- host-side plan of one layer configuration: which kernels run,
+// how expert segments are padded, and where each intermediate lives inside
+// the caller's workspace.  A pure function of moe_config.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// How the expert FFN GEMMs are laid out.
+enum FfnPath : int {
+    PATH_TOKEN_MAJOR = 0,  // tensor cores, 128 tokens x 256 features per tile
+    PATH_SWAP = 1,         // tensor cores, 128 weight rows x (tokens of one expert) per tile
+    PATH_F32 = 2,          // fp32 SIMT (fp32 configs; no TF32)
+};
+
+constexpr int ROUTE_BLOCK = 128;  // tokens per router / dispatch block
+constexpr int MAX_E = 1024;
+constexpr int MAX_K = 8;
+constexpr int SWAP_MAX_TOKENS = 256;  // largest per-expert token count the swap path covers
+
+struct Plan {
+    int64_t T;
+    int d, h, E, k, S, hs;
+    int64_t C;          // capacity (T when unlimited)
+    bool capped;
+    bool bf16;
+    int act_bytes;
+    int path;           // FfnPath for the routed experts
+    int shared_path;    // FfnPath for the fused shared expert
+    int pad;            // row padding of each expert segment in x_perm
+    int nt_max;         // swap path: max tokens per expert, rounded up to 16
+    int splits;         // split-K partials of the down projection
+    int64_t perm_rows;  // rows of x_perm / each y_perm split
+    int nblk;           // router blocks of ROUTE_BLOCK tokens
+    int hsum;           // S * hs (fused shared width)
+
+    // workspace byte offsets
+    size_t off_status, off_logits, off_ppart, off_hpart, off_cnt, off_offsets, off_perm,
+        off_xperm, off_H, off_y, off_Hs, off_ys, off_sums, total;
+};
+
+// Fills *p; returns MOE_OK or an error code with the message in *why.
+int make_plan(const moe_config* cfg, Plan* p, const char** why);
+
+}  // namespace moe

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/moe.h declares, and its host-only calls (capacity, workspace size,
+argument checks) behave, without touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_22_b200 as M
+from sparse_mixture_experts_22_b200 import binding as B
+from sparse_mixture_experts_22_b200 import build as build_mod
+from sparse_mixture_experts_22_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build_mod.build()
+
+
+def declared():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", txt)
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared()
+    assert len(names) >= 18
+    lib = ctypes.CDLL(B.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(B.EXPORTS) <= set(names)
+
+
+def test_capacity_matches_the_worked_example():
+    # batch 2048, 8 experts, top-2, capacity factor 1.25 -> 640 per expert
+    assert M.moe_capacity(M.make_config(2048, 4096, 14336, 8, 2, cf=(5, 4))) == 640
+    assert M.moe_capacity(M.config_of(WORKLOADS["deepseek"])) == 231
+    assert M.moe_capacity(M.config_of(WORKLOADS["large"])) == 6144
+    assert M.moe_capacity(M.config_of(WORKLOADS["decode"])) == 32  # no limit: T
+
+
+def test_workspace_and_perm_rows():
+    for name, wl in WORKLOADS.items():
+        cfg = M.config_of(wl)
+        ws = M.moe_workspace_size(cfg)
+        rows = M.moe_perm_rows(cfg)
+        splits = M.moe_ffn_splits(cfg)
+        assert rows >= min(wl.T * wl.k, wl.E * M.moe_capacity(cfg))
+        assert ws >= rows * wl.d * (2 if wl.dtype == "bf16" else 4) * 2
+        assert 1 <= splits <= 8
+    # decode streams the weights with a split-K down projection
+    assert M.moe_ffn_splits(M.config_of(WORKLOADS["decode"])) > 1
+    assert M.moe_workspace_size(M.make_config(0, 128, 128, 4, 2)) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=8, d=100, h=128, E=4, k=2), 2),          # d not a multiple of 128
+    (dict(T=8, d=128, h=200, E=4, k=2), 2),          # h not a multiple of 128
+    (dict(T=8, d=128, h=128, E=4, k=5), 2),          # k > E
+    (dict(T=8, d=128, h=128, E=16, k=9), 2),         # k > 8
+    (dict(T=8, d=128, h=128, E=0, k=1), 2),          # no experts
+    (dict(T=-1, d=128, h=128, E=4, k=2), 2),         # negative T
+    (dict(T=8, d=128, h=128, E=4, k=2, cf=(0, 4)), 1),  # zero capacity factor
+    (dict(T=8, d=128, h=128, E=4, k=2, n_shared=2, h_shared=100), 2),
+])
+def test_invalid_configs_are_rejected(kw, code):
+    with pytest.raises(B.MoEError) as e:
+        M.moe_workspace_size(M.make_config(**kw))
+    assert e.value.code == code
+    assert "invalid config" in str(e.value)
+
+
+def test_bad_dtype_is_rejected():
+    cfg = M.make_config(8, 128, 128, 4, 2)
+    cfg.act_dtype = 7
+    with pytest.raises(B.MoEError) as e:
+        M.moe_capacity(cfg)
+    assert e.value.code == 3
+
+
+def test_null_config_is_rejected():
+    lib = B.load()
+    v = ctypes.c_int64()
+    assert lib.moe_capacity(None, ctypes.byref(v)) == 1
+    assert b"NULL" in lib.moe_last_error()
