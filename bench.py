@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Throughput of the sparse top-k MoE layer on B200.
+
+One step = one pass of the whole layer (router, top-k, capacity dispatch,
+expert FFNs, combine, statistics) over one batch of synthetic tokens, through
+the library's public call (moe_forward).  Default workload: the Mixtral-shaped
+decode layer (T=32 tokens, d=4096, h=14336, 8 experts, top-2, bf16), which
+streams all 2.82 GB of expert weights per step.  Under torchrun every rank
+runs its own batch (weak scaling; weights replicated) and the per-rank
+routing statistics are summed across ranks with one NCCL all-reduce.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+instead, on a bounded sample of the same workload.
+"""
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_22_b200 import binding as B  # noqa: E402
+from sparse_mixture_experts_22_b200 import inputs as I  # noqa: E402
+from sparse_mixture_experts_22_b200.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (1xB200) and % of roofline (BF16 TC / HBM)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILES = os.path.join(ROOT, "profiles")
+GEMM_SRC = os.path.join(ROOT, "sparse_mixture_experts_22_b200", "csrc", "gemm_tc.cu")
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="decode", choices=list(WORKLOADS))
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="budget of the CPU-baseline sample")
+    p.add_argument("--no-trace", action="store_true",
+                   help="skip the per-kernel CUDA events in the timed region")
+    p.add_argument("--trace-all", action="store_true",
+                   help="time every kernel (one event after each launch) instead of only "
+                        "the gate/up GEMM")
+    p.add_argument("--hidden", type=int, default=0,
+                   help="override the expert hidden width (small profiling cases only)")
+    p.add_argument("--graph", action="store_true",
+                   help="capture one step in a CUDA graph and replay it (1 GPU)")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_label(wl):
+    return f"{wl.name}: {wl.describe()}"
+
+
+def algorithmic(wl, kept):
+    """Algorithmic FLOPs and bytes of one layer pass (kept assignments only;
+    experts with no token are not read)."""
+    d, h, E = wl.d, wl.h, wl.E
+    ab = 2 if wl.dtype == "bf16" else 4
+    N = int(sum(kept))
+    active = sum(1 for n in kept if n > 0)
+    T = wl.T
+    flops = 2 * T * d * E + 6 * d * h * N + wl.n_shared * 6 * d * wl.h_shared * T
+    wbytes = active * 3 * d * h * ab + wl.n_shared * 3 * d * wl.h_shared * ab
+    byt = T * d * ab + 4 * d * E + wbytes + T * d * ab
+    return flops, byt, N, active
+
+
+def kernel_work(name, wl, kept, splits):
+    """Algorithmic work of one launch of a GEMM kernel: (bound, amount, unit)."""
+    d, h = wl.d, wl.h
+    ab = 2 if wl.dtype == "bf16" else 4
+    N = int(sum(kept))
+    active = sum(1 for n in kept if n > 0)
+    C = min(B.moe_capacity(B.config_of(wl)), wl.T)
+    swapped = C <= 256
+    if name == "gemm_gateup":
+        if swapped:
+            return "hbm", active * 2 * h * d * ab + N * d * ab + N * h * ab, "bytes"
+        return "tensor", 4.0 * N * d * h, "flops"
+    if name == "gemm_down":
+        if swapped:
+            return "hbm", active * d * h * ab + N * h * ab + splits * N * d * 4, "bytes"
+        return "tensor", 2.0 * N * d * h, "flops"
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"samples": 0, "note": "nvidia-smi unavailable"}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                power.append(float(r[3]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_from_profile(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current GEMM source; None otherwise."""
+    path = os.path.join(PROFILES, f"{kernel}_{workload}.ncu.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                k, v = line.split("=", 1)
+                vals[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
+    if vals.get("gemm_source_sha256") != sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ---------------------------------------------------------------- inputs
+
+def build_inputs(wl, rank, world, dev, keep_host):
+    """Per-rank tokens; expert weights drawn on rank 0 and broadcast."""
+    Wr = I.router_weights(wl)
+    bias = I.router_bias(wl)
+    x, _ = I.tokens(wl, Wr=Wr, b=bias, stream="x" if rank == 0 else f"x.rank{rank}")
+    cfg = B.config_of(wl)
+    host = {"x": x, "Wr": Wr, "bias": bias}
+    dt = I.torch_dtype(wl.dtype)
+    if rank == 0:
+        w = I.expert_weights(wl)
+        w1, w3, w2 = (w[k].to(dev) for k in ("w1", "w3", "w2"))
+        W13, W2p = B.pack_weights(cfg, w1, w3, w2)
+        del w1, w3, w2
+        if keep_host:
+            host.update(w)
+        W13s = W2s = None
+        if wl.n_shared:
+            s = I.expert_weights(wl, shared=True)
+            s1, s3, s2 = (s[k].to(dev) for k in ("w1", "w3", "w2"))
+            W13s, W2s = B.pack_weights(cfg, s1, s3, s2, shared=True)
+            del s1, s3, s2
+            if keep_host:
+                host.update({"w1s": s["w1"], "w3s": s["w3"], "w2s": s["w2"]})
+    else:
+        W13 = torch.empty((wl.E, 2 * wl.h, wl.d), dtype=dt, device=dev)
+        W2p = torch.empty((wl.E, wl.d, wl.h), dtype=dt, device=dev)
+        W13s = W2s = None
+        if wl.n_shared:
+            hs = wl.n_shared * wl.h_shared
+            W13s = torch.empty((2 * hs, wl.d), dtype=dt, device=dev)
+            W2s = torch.empty((wl.d, hs), dtype=dt, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        for t in (W13, W2p, W13s, W2s):
+            if t is not None:
+                dist.broadcast(t, src=0)
+    torch.cuda.synchronize()
+    dev_in = {"x": x.to(dev), "Wr": Wr.to(dev), "bias": bias.to(dev) if bias is not None else None}
+    return cfg, host, dev_in, (W13, W2p, W13s, W2s)
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def time_oracle(wl, host, budget_s):
+    """Oracle on the host cores: routing of the whole batch plus the expert
+    FFN rows of as many tokens as fit in about budget_s seconds."""
+    import numpy as np
+    import oracle as O
+    cfg = O.cfg_of(wl)
+    t0 = time.perf_counter()
+    r = O.route(cfg, host["x"], host["Wr"], host["bias"])
+    t_route = time.perf_counter() - t0
+    # probe one row, then size the sample
+    t0 = time.perf_counter()
+    O.layer_rows(cfg, host["x"], r["idx"], r["gate"], r["keep"], host["w1"], host["w3"],
+                 host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"), [0])
+    t_row = max(time.perf_counter() - t0, 1e-4)
+    rows_per_pass = max(1, min(wl.T, int(budget_s / (t_row + t_route / max(wl.T, 1)))))
+    done, elapsed, passes = 0, 0.0, 0
+    while elapsed < budget_s * 0.5 or passes == 0:
+        t0 = time.perf_counter()
+        r = O.route(cfg, host["x"], host["Wr"], host["bias"])
+        O.layer_rows(cfg, host["x"], r["idx"], r["gate"], r["keep"], host["w1"], host["w3"],
+                     host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"),
+                     np.arange(rows_per_pass))
+        elapsed += time.perf_counter() - t0
+        done += rows_per_pass
+        passes += 1
+        if rows_per_pass < wl.T:
+            break
+    sample = (f"{passes} pass(es): fp64 routing, capacity dispatch and statistics of the whole "
+              f"T={wl.T} batch plus the layer output of {rows_per_pass} token row(s) per pass")
+    return {"value": done / elapsed, "unit": UNIT, "cores": O.threads(), "kind": "oracle",
+            "sample": sample, "seconds": elapsed}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    Wr = I.router_weights(wl)
+    bias = I.router_bias(wl)
+    x, _ = I.tokens(wl, Wr=Wr, b=bias)
+    host = {"x": x, "Wr": Wr, "bias": bias}
+    host.update(I.expert_weights(wl))
+    if wl.n_shared:
+        s = I.expert_weights(wl, shared=True)
+        host.update({"w1s": s["w1"], "w3s": s["w3"], "w2s": s["w2"]})
+    import numpy as np
+    import oracle as O
+    cfg = O.cfg_of(wl)
+    # each step: the whole batch routed, and the outputs of a bounded row sample
+    t0 = time.perf_counter()
+    O.layer_rows(cfg, x, *(lambda r: (r["idx"], r["gate"], r["keep"]))(
+        O.route(cfg, x, Wr, bias)), host["w1"], host["w3"], host["w2"], host.get("w1s"),
+        host.get("w3s"), host.get("w2s"), [0])
+    t_row = time.perf_counter() - t0
+    rows = max(1, min(wl.T, int(0.5 / max(t_row, 1e-4))))
+    sample_rows = np.arange(rows)
+
+    def step():
+        r = O.route(cfg, x, Wr, bias)
+        O.layer_rows(cfg, x, r["idx"], r["gate"], r["keep"], host["w1"], host["w3"], host["w2"],
+                     host.get("w1s"), host.get("w3s"), host.get("w2s"), sample_rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = rows * args.steps / el
+    sample = (f"each step: fp64 routing, dispatch and statistics of the whole T={wl.T} batch "
+              f"plus the layer output of {rows} token row(s)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_label(wl), "global_batch": wl.T, "tokens_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": O.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    wl = WORKLOADS[args.workload]
+    if args.hidden:
+        wl = wl.scaled(h=args.hidden, name=f"{wl.name}_h{args.hidden}")
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    cfg, host, g, W = build_inputs(wl, rank, world, dev, keep_host=want_cpu)
+    W13, W2p, W13s, W2s = W
+    bufs = B.alloc_layer(cfg, dev)
+    sums = torch.zeros(2 + 3 * wl.E, dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if world == 1:
+            B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
+                          bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
+                          bufs["slot_of"], bufs["stats"], bufs["ws"])
+        else:
+            B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
+                          bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
+                          bufs["slot_of"], None, bufs["ws"])
+            B.moe_stats_sums(cfg, bufs["routed"], bufs["kept"], bufs["ws"], sums)
+            dist.all_reduce(sums)
+            B.moe_stats_finalize(cfg, sums, bufs["stats"])
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    status = B.moe_read_device_status(bufs["ws"])
+    if status != 0:
+        raise SystemExit(f"device status {status} after warm-up")
+
+    graph = None
+    if args.graph and world == 1:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(graph, stream=side):
+                step()
+        torch.cuda.synchronize()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step
+    trace_on = not args.no_trace and graph is None
+
+    # ------------------------------------------------ timed region (device resident)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if trace_on:
+        # bracket only the dominant kernel (the one the roofline is quoted on)
+        B.moe_trace_begin(args.steps, None if args.trace_all else "gemm_gateup")
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    trace = B.moe_trace_end() if trace_on else []
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    status = B.moe_read_device_status(bufs["ws"])
+
+    # ------------------------------------------------ end to end (host buffers, copies timed)
+    e2e = None
+    if not args.no_e2e:
+        x_h = g["x"].cpu().pin_memory()
+        out_h = torch.empty(bufs["out"].shape, dtype=bufs["out"].dtype).pin_memory()
+        st_h = torch.empty(bufs["stats"].shape, dtype=bufs["stats"].dtype).pin_memory()
+
+        def e2e_step():
+            g["x"].copy_(x_h, non_blocking=True)
+            step()
+            out_h.copy_(bufs["out"], non_blocking=True)
+            st_h.copy_(bufs["stats"], non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if dist:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * wl.T * args.steps / (float(e_ms.item()) / 1000.0), "unit": UNIT,
+               "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
+               "d2h_bytes_per_step": out_h.numel() * out_h.element_size()
+               + st_h.numel() * st_h.element_size()}
+
+    # ------------------------------------------------ report
+    kept = bufs["kept"].cpu().tolist()
+    stats = B.stats_dict(bufs["stats"])
+    pk, pk_kind = peaks()
+    flops, byts, N, active = algorithmic(wl, kept)
+    t_step = ms_max / 1000.0 / args.steps
+    roof_t = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    kernels = {n: {"launches": c, "ms_per_launch": t / c} for n, c, t in trace}
+    top = max(trace, key=lambda r: r[2]) if trace else None
+    roofline = None
+    splits = B.moe_ffn_splits(cfg)
+    if top is not None:
+        name, launches, tot_ms = top
+        per = tot_ms / launches / 1000.0
+        work = kernel_work(name, wl, kept, splits)
+        if work:
+            bound, amount, _ = work
+            if bound == "hbm":
+                ach, peak, unit = amount / per / 1e9, pk["hbm_gbs"], "GB/s"
+            else:
+                ach, peak, unit = amount / per / 1e12, pk.get("bf16_tflops_sustained",
+                                                            pk["bf16_tflops"]), "TFLOP/s"
+            roofline = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak,
+                        "unit": unit, "frac": ach / peak, "peak_source": pk_kind,
+                        "algorithmic_per_launch": amount,
+                        "traffic": traffic_from_profile(name, wl.name)}
+    launches_total = sum(c for _, c, _ in trace)
+    line = {
+        "metric": METRIC,
+        "value": world * wl.T * args.steps / (ms_max / 1000.0),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic",
+        "config": {"workload": workload_label(wl), "global_batch": world * wl.T,
+                   "tokens_per_rank": wl.T,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": ("inputs larger than L2: the active expert weights "
+                          f"({active * 3 * wl.d * wl.h * 2 / 1e9:.2f} GB) stream from HBM "
+                          "every step")},
+        "roofline": roofline,
+        "layer_roofline": {"flops": flops, "bytes": byts, "time_us": roof_t * 1e6,
+                           "frac": roof_t / t_step, "kept_assignments": N,
+                           "active_experts": active},
+        "kernels": kernels,
+        "gpu_launches": launches_total,
+        "clocks": clk,
+        "e2e": e2e,
+        "stats": stats,
+        "device_status": status,
+    }
+    if want_cpu:
+        line["cpu_baseline"] = time_oracle(wl, host, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

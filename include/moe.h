@@ -144,9 +144,13 @@ MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w1, c
  * softmax over the kept k.  Also writes the full-softmax partial sums used
  * by moe_aux_stats into ws.
  *   x [T][d] act; Wr [d][E] fp32; bias [E] fp32 (ignored unless has_bias)
- *   topk_idx [T][k] int32; topk_gate [T][k] fp32                          */
+ *   topk_idx [T][k] int32; topk_gate [T][k] fp32
+ *   logits [T][E] fp32, optional (NULL = not written): the router logits z.
+ * Precision: for bf16 batches of more than 256 tokens the logits run on the
+ * tensor cores against W_r split into three bf16 parts (carrying W_r to 24
+ * bits) with fp32 accumulation; otherwise as fp32 dot products.            */
 MOE_API int moe_route(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
-              int32_t* topk_idx, float* topk_gate, void* ws, size_t ws_bytes,
+              int32_t* topk_idx, float* topk_gate, float* logits, void* ws, size_t ws_bytes,
               void* stream);
 
 /* Dispatch under capacity [MoE routing fully explained, "Easy explanation"
@@ -222,12 +226,14 @@ MOE_API int moe_read_device_status(const void* ws, int32_t* status, void* stream
  * the device status word and its kernel returns early.  Process-wide. */
 MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 
-/* Per-kernel timing of moe_forward.  moe_trace_begin(n) records CUDA events
- * around every kernel moe_forward launches, for up to n calls;
- * moe_trace_end synchronises and writes, per kernel, its name, launch count
- * and summed milliseconds (up to cap entries; *n_out = entries written).
- * Process-wide; not thread-safe. */
-MOE_API int moe_trace_begin(int max_calls);
+/* Per-kernel timing of moe_forward.  moe_trace_begin(n, only) records CUDA
+ * events for up to n moe_forward calls: with only == NULL, one event after
+ * every kernel launch (each kernel is timed from the end of the previous
+ * one); with only naming a kernel (e.g. "gemm_gateup"), one event before and
+ * one after that kernel alone.  moe_trace_end synchronises and writes, per
+ * kernel, its name, launch count and summed milliseconds (up to cap entries;
+ * *n_out = entries written).  Process-wide; not thread-safe. */
+MOE_API int moe_trace_begin(int max_calls, const char* only);
 MOE_API int moe_trace_end(char (*names)[32], int* launches, double* ms, int cap, int* n_out);
 
 #ifdef __cplusplus

@@ -72,7 +72,7 @@ def load() -> ctypes.CDLL:
             "moe_perm_rows": [C, P],
             "moe_ffn_splits": [C, P],
             "moe_pack_weights": [C, I, P, P, P, P, P, P],
-            "moe_route": [C, P, P, P, P, P, P, S, P],
+            "moe_route": [C, P, P, P, P, P, P, P, S, P],
             "moe_dispatch": [C, P, P, P, P, P, P, P, P, P, S, P],
             "moe_expert_ffn": [C, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_combine": [C, P, P, P, P, P, P],
@@ -82,7 +82,7 @@ def load() -> ctypes.CDLL:
             "moe_forward": [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_read_device_status": [P, P, P],
             "moe_set_wait_limit_ns": [ctypes.c_uint64],
-            "moe_trace_begin": [I],
+            "moe_trace_begin": [I, ctypes.c_char_p],
             "moe_trace_end": [P, P, P, I, P],
         }
         for name, args in sig.items():
@@ -169,9 +169,9 @@ def moe_pack_weights(cfg, which, w1, w3, w2, W13, W2p, stream=None):
                                    _p(W2p), _stream(stream)))
 
 
-def moe_route(cfg, x, Wr, bias, topk_idx, topk_gate, ws, stream=None):
+def moe_route(cfg, x, Wr, bias, topk_idx, topk_gate, ws, logits=None, stream=None):
     _check(load().moe_route(ctypes.byref(cfg), _p(x), _p(Wr), _p(bias), _p(topk_idx),
-                            _p(topk_gate), _p(ws), ws.numel() * ws.element_size(),
+                            _p(topk_gate), _p(logits), _p(ws), ws.numel() * ws.element_size(),
                             _stream(stream)))
 
 
@@ -226,8 +226,8 @@ def moe_set_wait_limit_ns(ns: int):
     _check(load().moe_set_wait_limit_ns(int(ns)))
 
 
-def moe_trace_begin(max_calls: int):
-    _check(load().moe_trace_begin(max_calls))
+def moe_trace_begin(max_calls: int, only: Optional[str] = None):
+    _check(load().moe_trace_begin(max_calls, only.encode() if only else None))
 
 
 def moe_trace_end(cap: int = 64) -> List[Tuple[str, int, float]]:

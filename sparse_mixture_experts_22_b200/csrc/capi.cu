@@ -105,6 +105,31 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
         while (P.splits < 8 && units * P.splits < 960 && kblocks % (P.splits * 2) == 0)
             P.splits *= 2;
     }
+    // router: split-d partials for small batches; tensor cores (three bf16 parts
+    // of W_r) for larger bf16 batches; fp32 dot products for larger fp32 batches
+    P.router_npad = P.E;
+    P.router_ld = P.E;
+    P.router_bn = 0;
+    P.router_splits = 1;
+    if (P.T <= SWAP_MAX_TOKENS) {
+        P.router_kind = ROUTER_PARTIAL;
+        P.router_splits = (P.d + 255) / 256;
+    } else if (P.bf16) {
+        P.router_kind = ROUTER_TC;
+        P.router_bn = 3 * P.E <= 128 ? 128 : 256;
+        P.router_npad = (3 * P.E + P.router_bn - 1) / P.router_bn * P.router_bn;
+        // split K four ways at least (each fp32 accumulation chain in TMEM
+        // covers at most a quarter of d; the partial sums are added in fp32
+        // afterwards) and further until the tiles cover most SMs
+        const int64_t units = ((P.T + 127) / 128) * (P.router_npad / P.router_bn);
+        const int kblocks = P.d / 64;
+        while (P.router_splits < 8 && kblocks % (P.router_splits * 2) == 0 &&
+               (P.router_splits < 4 || units * P.router_splits < 120))
+            P.router_splits *= 2;
+        P.router_ld = (3 * P.E + 3) / 4 * 4;
+    } else {
+        P.router_kind = ROUTER_SIMT;
+    }
     const int64_t assign = c.T * (int64_t)c.k;
     const int64_t cap_all = (int64_t)c.E * nmax;
     const int64_t kept_max = assign < cap_all ? assign : cap_all;
@@ -115,6 +140,11 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
     P.off_status = take(256);
     P.off_logits = take((size_t)c.T * c.E * 4);
+    P.off_wsplit = take(P.router_kind == ROUTER_TC ? (size_t)3 * c.E * c.d * 2 : 0);
+    P.off_z3 = take(P.router_kind == ROUTER_SIMT
+                        ? 0
+                        : (size_t)P.router_splits * c.T *
+                              (P.router_kind == ROUTER_TC ? P.router_ld : P.router_npad) * 4);
     P.off_ppart = take((size_t)P.nblk * c.E * 4);
     P.off_hpart = take((size_t)P.nblk * 4);
     P.off_cnt = take((size_t)P.nblk * c.E * 4);
@@ -213,30 +243,45 @@ struct TraceMark {
     cudaEvent_t ev;
     const char* name;
     int call;
+    bool pre;
 };
 
+// Per-kernel timing.  Without a filter every kernel of a moe_forward call is
+// timed from the end of the previous one (one event after each launch).  With
+// a filter only the named kernel is bracketed (one event before and one after
+// its launch), which perturbs the rest of the step least.
 struct Tracer {
     bool on = false;
     int max_calls = 0;
     int calls = 0;
+    std::string only;
     std::vector<cudaEvent_t> pool;
     std::vector<TraceMark> marks;
 };
 
 static Tracer g_trace;
 
-static void trace_mark(cudaStream_t st, const char* name) {
-    if (!g_trace.on || g_trace.calls > g_trace.max_calls) return;
+static void trace_record(cudaStream_t st, const char* name, bool pre) {
+    if (!g_trace.on || g_trace.calls > g_trace.max_calls || g_trace.calls == 0) return;
     if (g_trace.marks.size() >= g_trace.pool.size()) return;
     cudaEvent_t ev = g_trace.pool[g_trace.marks.size()];
     cudaEventRecord(ev, st);
-    g_trace.marks.push_back({ev, name, g_trace.calls});
+    g_trace.marks.push_back({ev, name, g_trace.calls, pre});
+}
+
+static void trace_pre(cudaStream_t st, const char* name) {
+    if (g_trace.on && !g_trace.only.empty() && g_trace.only == name) trace_record(st, name, true);
+}
+
+static void trace_mark(cudaStream_t st, const char* name) {
+    if (!g_trace.on) return;
+    if (g_trace.only.empty() || g_trace.only == name) trace_record(st, name, false);
 }
 
 static void trace_call_begin(cudaStream_t st) {
     if (!g_trace.on) return;
     ++g_trace.calls;
-    trace_mark(st, "begin");
+    if (g_trace.only.empty()) trace_record(st, "begin", true);
 }
 
 // ---------------------------------------------------------------- checks
@@ -276,22 +321,133 @@ static const T* at(const void* ws, size_t off) {
 
 // ---------------------------------------------------------------- steps
 
-static int step_route(const Plan& P, const Device& dv, const void* x, const float* Wr,
-                      const float* bias, int32_t* topk_idx, float* topk_gate, void* ws,
-                      cudaStream_t st) {
-    if (P.T == 0) {
-        if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess)
-            return fail(MOE_ERR_CUDA, "status reset failed");
-        return MOE_OK;
-    }
+static int run_tc_router(const Plan& P, const Device& dv, const void* x, const void* Ws,
+                         float* z3, int32_t* status, cudaStream_t st) {
+    CUtensorMap m_act, m_w;
+    TcArgs a;
+    memset(&a, 0, sizeof a);
+    a.num_groups = 1;
+    a.dense_rows = (int)P.T;
+    a.K = P.d;
+    a.n_feat = P.router_npad;
+    a.w_rows_per_group = P.router_npad;
+    a.status = status;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.out = z3;
+    a.out_ld = P.router_ld;       // compact rows: only the 3E logit parts are stored
+    a.out_cols = P.router_ld;
+    a.splits = P.router_splits;
+    a.split_stride = P.T * (int64_t)P.router_ld;
+    // rows past 3E of the split weights lie outside the tensor map: TMA reads zeros there
+    MOE_TRY(tmap_bf16(&m_act, x, P.T, P.d, 128));
+    MOE_TRY(tmap_bf16(&m_w, Ws, 3LL * P.E, P.d, P.router_bn));
+    a.stages = tc_max_stages(TC_DOWN_TOK, P.router_bn, 16, 1, dv.smem_optin);
+    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    trace_pre(st, "router_gemm");
+    MOE_TRY(launched(launch_tc_gemm(TC_DOWN_TOK, P.router_bn, m_act, m_w, a, dv.sms, st),
+                     "router_gemm"));
+    trace_mark(st, "router_gemm");
+    return MOE_OK;
+}
+
+// Router logits (partials), ready for top-k: fills r.src / nsplit / nparts / strides / bias.
+static int step_logits(const Plan& P, const Device& dv, const void* x, const float* Wr,
+                       const float* bias, void* ws, RouteParams& r, cudaStream_t st) {
     float* z = at<float>(ws, P.off_logits);
-    MOE_TRY(launched(launch_router_logits(x, P.bf16, Wr, bias, z, P.T, P.d, P.E, dv.sms, st),
-                     "router_logits"));
-    trace_mark(st, "router_logits");
-    MOE_TRY(launched(launch_topk(z, P.T, P.E, P.k, topk_idx, topk_gate, at<float>(ws, P.off_ppart),
-                                 at<float>(ws, P.off_hpart), at<int32_t>(ws, P.off_cnt),
-                                 at<int32_t>(ws, P.off_status), st),
-                     "topk"));
+    float* z3 = at<float>(ws, P.off_z3);
+    r.src = z;
+    r.nsplit = 1;
+    r.nparts = 1;
+    r.row_stride = P.E;
+    r.split_stride = 0;
+    r.bias = bias;
+    if (P.router_kind == ROUTER_PARTIAL) {
+        trace_pre(st, "router_partial");
+        MOE_TRY(launched(launch_router_partial(x, P.bf16, Wr, z3, (int)P.T, P.d, P.E, st),
+                         "router_partial"));
+        trace_mark(st, "router_partial");
+        r.src = z3;
+        r.nsplit = P.router_splits;
+        r.split_stride = P.T * (int64_t)P.E;
+    } else if (P.router_kind == ROUTER_TC) {
+        void* Ws = at<void>(ws, P.off_wsplit);
+        trace_pre(st, "router_split");
+        MOE_TRY(launched(launch_router_split(Wr, Ws, P.d, P.E, st), "router_split"));
+        trace_mark(st, "router_split");
+        MOE_TRY(run_tc_router(P, dv, x, Ws, z3, r.status, st));
+        trace_pre(st, "router_reduce");
+        MOE_TRY(launched(launch_router_reduce(z3, P.router_splits, P.T * (int64_t)P.router_ld,
+                                              P.router_ld, 3, bias, z, P.T, P.E, st),
+                         "router_reduce"));
+        trace_mark(st, "router_reduce");
+        r.bias = nullptr;  // already added
+    } else {
+        trace_pre(st, "router_logits");
+        MOE_TRY(launched(launch_router_logits(x, P.bf16, Wr, z, P.T, P.d, P.E, dv.sms, st),
+                         "router_logits"));
+        trace_mark(st, "router_logits");
+    }
+    return MOE_OK;
+}
+
+static RouteParams route_params(const Plan& P, void* ws, int32_t* topk_idx, float* topk_gate,
+                                float* logits) {
+    RouteParams r;
+    memset(&r, 0, sizeof r);
+    r.zbuf = at<float>(ws, P.off_logits);
+    r.logits = logits;
+    r.T = P.T;
+    r.E = P.E;
+    r.k = P.k;
+    r.topk_idx = topk_idx;
+    r.topk_gate = topk_gate;
+    r.ppart = at<float>(ws, P.off_ppart);
+    r.hpart = at<float>(ws, P.off_hpart);
+    r.cnt = at<int32_t>(ws, P.off_cnt);
+    r.status = at<int32_t>(ws, P.off_status);
+    return r;
+}
+
+static DispatchParams dispatch_params(const Plan& P, const void* x, int32_t* routed,
+                                      int32_t* kept, int32_t* offsets, int32_t* perm_token,
+                                      int32_t* slot_of, void* x_perm) {
+    DispatchParams d;
+    d.T = P.T;
+    d.E = P.E;
+    d.k = P.k;
+    d.C = P.C;
+    d.pad = P.pad;
+    d.perm_rows = P.perm_rows;
+    d.x = x;
+    d.row_bytes = P.d * P.act_bytes;
+    d.routed = routed;
+    d.kept = kept;
+    d.offsets = offsets;
+    d.perm_token = perm_token;
+    d.slot_of = slot_of;
+    d.x_perm = x_perm;
+    return d;
+}
+
+static int empty_batch(const Plan& P, void* ws, int32_t* routed, int32_t* kept,
+                       int32_t* offsets, cudaStream_t st) {
+    // status reset; zero counts and offsets so later steps see no work
+    if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess ||
+        (routed && cudaMemsetAsync(routed, 0, P.E * 4, st) != cudaSuccess) ||
+        (kept && cudaMemsetAsync(kept, 0, P.E * 4, st) != cudaSuccess) ||
+        (offsets && cudaMemsetAsync(offsets, 0, (P.E + 1) * 4, st) != cudaSuccess))
+        return fail(MOE_ERR_CUDA, "memset failed");
+    return MOE_OK;
+}
+
+static int step_route(const Plan& P, const Device& dv, const void* x, const float* Wr,
+                      const float* bias, int32_t* topk_idx, float* topk_gate, float* logits,
+                      void* ws, cudaStream_t st) {
+    if (P.T == 0) return empty_batch(P, ws, nullptr, nullptr, nullptr, st);
+    RouteParams r = route_params(P, ws, topk_idx, topk_gate, logits);
+    MOE_TRY(step_logits(P, dv, x, Wr, bias, ws, r, st));
+    trace_pre(st, "topk");
+    MOE_TRY(launched(launch_topk(r, st), "topk"));
     trace_mark(st, "topk");
     return MOE_OK;
 }
@@ -299,19 +455,34 @@ static int step_route(const Plan& P, const Device& dv, const void* x, const floa
 static int step_dispatch(const Plan& P, const Device& dv, const int32_t* topk_idx, const void* x,
                          int32_t* routed, int32_t* kept, int32_t* offsets, int32_t* perm_token,
                          int32_t* slot_of, void* x_perm, void* ws, cudaStream_t st) {
-    if (P.T == 0) {
-        // empty batch: zero counts and offsets so later steps see no work
-        if (cudaMemsetAsync(routed, 0, P.E * 4, st) != cudaSuccess ||
-            cudaMemsetAsync(kept, 0, P.E * 4, st) != cudaSuccess ||
-            cudaMemsetAsync(offsets, 0, (P.E + 1) * 4, st) != cudaSuccess)
-            return fail(MOE_ERR_CUDA, "memset failed");
-        return MOE_OK;
-    }
-    MOE_TRY(launched(launch_dispatch(topk_idx, at<int32_t>(ws, P.off_cnt), P.T, P.E, P.k, P.C,
-                                     P.pad, P.perm_rows, x, P.d * P.act_bytes, routed, kept,
-                                     offsets, perm_token, slot_of, x_perm, dv.sms, st),
+    if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st);
+    DispatchParams d = dispatch_params(P, x, routed, kept, offsets, perm_token, slot_of, x_perm);
+    trace_pre(st, "dispatch");
+    MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt), dv.sms, st),
                      "dispatch"));
     trace_mark(st, "dispatch");
+    return MOE_OK;
+}
+
+// Router, top-k and dispatch of moe_forward: one fused launch for top-k and
+// dispatch when the batch fits one routing block.
+static int step_route_dispatch(const Plan& P, const Device& dv, const void* x, const float* Wr,
+                               const float* bias, int32_t* topk_idx, float* topk_gate,
+                               int32_t* routed, int32_t* kept, int32_t* offsets,
+                               int32_t* perm_token, int32_t* slot_of, void* x_perm, void* ws,
+                               cudaStream_t st) {
+    if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st);
+    if (P.T > ROUTE_BLOCK) {
+        MOE_TRY(step_route(P, dv, x, Wr, bias, topk_idx, topk_gate, nullptr, ws, st));
+        return step_dispatch(P, dv, topk_idx, x, routed, kept, offsets, perm_token, slot_of,
+                             x_perm, ws, st);
+    }
+    RouteParams r = route_params(P, ws, topk_idx, topk_gate, nullptr);
+    MOE_TRY(step_logits(P, dv, x, Wr, bias, ws, r, st));
+    DispatchParams d = dispatch_params(P, x, routed, kept, offsets, perm_token, slot_of, x_perm);
+    trace_pre(st, "route_dispatch");
+    MOE_TRY(launched(launch_route_dispatch(r, d, dv.sms, st), "route_dispatch"));
+    trace_mark(st, "route_dispatch");
     return MOE_OK;
 }
 
@@ -347,6 +518,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.split_stride = 0;
     a.stages = tc_max_stages(mode1, 256, nt_max, groups, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    trace_pre(st, tag1);
     MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
     trace_mark(st, tag1);
 
@@ -364,6 +536,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.split_stride = act_rows * (int64_t)P.d;
     a.stages = tc_max_stages(mode2, bn, nt_max, groups, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    trace_pre(st, tag2);
     MOE_TRY(launched(launch_tc_gemm(mode2, bn, m_act, m_w, a, dv.sms, st), tag2));
     trace_mark(st, tag2);
     return MOE_OK;
@@ -417,11 +590,30 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
     return MOE_OK;
 }
 
+static StatsParams stats_params(const Plan& P, const int32_t* routed, const int32_t* kept,
+                                const void* ws, double* sums, moe_stats* stats) {
+    StatsParams a;
+    a.ppart = at<float>(ws, P.off_ppart);
+    a.hpart = at<float>(ws, P.off_hpart);
+    a.nblk = P.nblk;
+    a.routed = routed;
+    a.kept = kept;
+    a.T = P.T;
+    a.E = P.E;
+    a.k = P.k;
+    a.sums = sums;
+    a.stats = stats;
+    return a;
+}
+
 static int step_combine(const Plan& P, const float* y_perm, const int32_t* slot_of,
-                        const float* gate, const float* y_shared, void* out, cudaStream_t st) {
-    const int splits = P.path == PATH_F32 ? 1 : (P.path == PATH_SWAP ? P.splits : 1);
+                        const float* gate, const float* y_shared, void* out,
+                        const StatsParams* sp, cudaStream_t st) {
+    const int splits = P.path == PATH_SWAP ? P.splits : 1;
+    trace_pre(st, "combine");
     MOE_TRY(launched(launch_combine(y_perm, splits, P.perm_rows * (int64_t)P.d, slot_of, gate,
-                                    P.S > 0 ? y_shared : nullptr, out, P.bf16, P.T, P.d, P.k, st),
+                                    P.S > 0 ? y_shared : nullptr, out, P.bf16, P.T, P.d, P.k, sp,
+                                    st),
                      "combine"));
     trace_mark(st, "combine");
     return MOE_OK;
@@ -429,14 +621,9 @@ static int step_combine(const Plan& P, const float* y_perm, const int32_t* slot_
 
 static int step_stats(const Plan& P, const int32_t* routed, const int32_t* kept, const void* ws,
                       double* sums, moe_stats* stats, cudaStream_t st) {
-    MOE_TRY(launched(launch_stats_sums(at<float>(ws, P.off_ppart), at<float>(ws, P.off_hpart),
-                                       P.nblk, routed, kept, P.T, P.E, sums, st),
-                     "stats_sums"));
-    trace_mark(st, "stats_sums");
-    if (stats) {
-        MOE_TRY(launched(launch_stats_finalize(sums, P.E, P.k, stats, st), "stats_finalize"));
-        trace_mark(st, "stats_finalize");
-    }
+    trace_pre(st, "stats");
+    MOE_TRY(launched(launch_stats(stats_params(P, routed, kept, ws, sums, stats), st), "stats"));
+    trace_mark(st, "stats");
     return MOE_OK;
 }
 
@@ -528,7 +715,8 @@ int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const voi
 }
 
 int moe_route(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
-              int32_t* topk_idx, float* topk_gate, void* ws, size_t ws_bytes, void* stream) {
+              int32_t* topk_idx, float* topk_gate, float* logits, void* ws, size_t ws_bytes,
+              void* stream) {
     Plan P;
     MOE_TRY(plan_or_fail(cfg, &P));
     MOE_TRY(need_ws(ws, ws_bytes, P));
@@ -538,11 +726,12 @@ int moe_route(const moe_config* cfg, const void* x, const float* Wr, const float
         MOE_TRY(need(topk_idx, "topk_idx"));
         MOE_TRY(need(topk_gate, "topk_gate"));
         if (cfg->has_bias) MOE_TRY(need(bias, "bias"));
+        MOE_TRY(maybe(logits, "logits"));
     }
     Device dv;
     MOE_TRY(device_facts(&dv));
-    MOE_TRY(step_route(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate, ws,
-                       reinterpret_cast<cudaStream_t>(stream)));
+    MOE_TRY(step_route(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate, logits,
+                       ws, reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
 
@@ -608,7 +797,7 @@ int moe_combine(const moe_config* cfg, const float* y_perm, const int32_t* slot_
         MOE_TRY(need(out, "out"));
         if (P.S > 0) MOE_TRY(need(y_shared, "y_shared"));
     }
-    MOE_TRY(step_combine(P, y_perm, slot_of, topk_gate, y_shared, out,
+    MOE_TRY(step_combine(P, y_perm, slot_of, topk_gate, y_shared, out, nullptr,
                          reinterpret_cast<cudaStream_t>(stream)));
     return ok();
 }
@@ -685,12 +874,14 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
     void* x_perm = at<void>(ws, P.off_xperm);
     float* y = at<float>(ws, P.off_y);
     float* ys = P.S ? at<float>(ws, P.off_ys) : nullptr;
-    MOE_TRY(step_route(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate, ws, st));
-    MOE_TRY(step_dispatch(P, dv, topk_idx, x, routed, kept, offsets, perm, slot_of, x_perm, ws,
-                          st));
+    MOE_TRY(step_route_dispatch(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate,
+                                routed, kept, offsets, perm, slot_of, x_perm, ws, st));
     MOE_TRY(step_ffn(P, dv, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st));
-    if (P.T > 0) MOE_TRY(step_combine(P, y, slot_of, topk_gate, ys, out, st));
-    if (stats)
+    // combine, with the statistics computed by one extra block of the same launch
+    StatsParams sp = stats_params(P, routed, kept, ws, at<double>(ws, P.off_sums), stats);
+    if (P.T > 0)
+        MOE_TRY(step_combine(P, y, slot_of, topk_gate, ys, out, stats ? &sp : nullptr, st));
+    else if (stats)
         MOE_TRY(step_stats(P, routed, kept, ws, at<double>(ws, P.off_sums), stats, st));
     return ok();
 }
@@ -715,9 +906,9 @@ int moe_set_wait_limit_ns(uint64_t ns) {
     return ok();
 }
 
-int moe_trace_begin(int max_calls) {
+int moe_trace_begin(int max_calls, const char* only) {
     if (max_calls < 1 || max_calls > 100000) return fail(MOE_ERR_ARG, "max_calls out of range");
-    const size_t need_ev = (size_t)max_calls * 16;
+    const size_t need_ev = (size_t)max_calls * 24;
     while (g_trace.pool.size() < need_ev) {
         cudaEvent_t ev;
         if (cudaEventCreate(&ev) != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaEventCreate failed");
@@ -726,6 +917,7 @@ int moe_trace_begin(int max_calls) {
     g_trace.marks.clear();
     g_trace.calls = 0;
     g_trace.max_calls = max_calls;
+    g_trace.only = only ? only : "";
     g_trace.on = true;
     return ok();
 }
@@ -739,7 +931,7 @@ int moe_trace_end(char (*names)[32], int* launches, double* ms, int cap, int* n_
     for (size_t i = 1; i < g_trace.marks.size(); ++i) {
         const TraceMark& a = g_trace.marks[i - 1];
         const TraceMark& b = g_trace.marks[i];
-        if (a.call != b.call) continue;
+        if (a.call != b.call || b.pre) continue;
         if (cudaEventSynchronize(b.ev) != cudaSuccess)
             return fail(MOE_ERR_CUDA, "cudaEventSynchronize failed");
         float t = 0.f;

@@ -13,6 +13,8 @@
 // insights" ¶3]: the load-balancing loss E * sum_e f_e P_e, the overflow
 // rate and the mean router entropy, reduced from the per-block partials in a
 // fixed order in fp64.
+#include <string.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -21,11 +23,71 @@ namespace moe {
 
 namespace {
 
+__device__ void finalize_stats(const double* sums, int E, int k, moe_stats* st) {
+    const double T = sums[0];
+    moe_stats r{0.0, 0.0, 0.0, T, 0.0};
+    if (T > 0.0) {
+        const double tk = T * k;
+        double aux = 0.0, dropped = 0.0;
+        for (int e = 0; e < E; ++e) {
+            const double f = sums[2 + E + e] / tk;  // share of assignments (before the limit)
+            const double P = sums[2 + e] / T;       // mean router probability
+            aux += f * P;
+            dropped += sums[2 + E + e] - sums[2 + 2 * E + e];
+        }
+        r.aux_loss = (double)E * aux;
+        r.overflow_rate = dropped / tk;
+        r.mean_entropy = sums[1] / T;
+        r.dropped = dropped;
+    }
+    *st = r;
+}
+
+// sums = [T, entropy sum, P sums (E), routed (E), kept (E)], each a fixed-order
+// fp64 reduction of the router's per-block partials; then the statistics.
+// Run by one block of any size.
+__device__ void stats_block(const StatsParams& a) {
+    const float* ppart = a.ppart;
+    const float* hpart = a.hpart;
+    const int nblk = a.nblk, E = a.E, k = a.k;
+    const int32_t* routed = a.routed;
+    const int32_t* kept = a.kept;
+    const int64_t T = a.T;
+    double* sums = a.sums;
+    moe_stats* st = reinterpret_cast<moe_stats*>(a.stats);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        double h = 0.0;
+        for (int b = 0; b < nblk; ++b) h += (double)hpart[b];
+        sums[0] = (double)T;
+        sums[1] = h;
+    }
+    for (int e = tid; e < E; e += blockDim.x) {
+        double p = 0.0;
+        for (int b = 0; b < nblk; ++b) p += (double)ppart[(int64_t)b * E + e];
+        sums[2 + e] = p;
+        sums[2 + E + e] = T > 0 ? (double)routed[e] : 0.0;
+        sums[2 + 2 * E + e] = T > 0 ? (double)kept[e] : 0.0;
+    }
+    if (!st) return;
+    __syncthreads();
+    if (tid == 0) finalize_stats(sums, E, k, st);
+}
+
+__global__ void stats_kernel(StatsParams a) { stats_block(a); }
+
+// The last block of the grid computes the statistics instead when
+// sp.sums is set (they need only the router partials and the counts).
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ y, int splits, int64_t split_stride,
                    const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
-                   const float* __restrict__ ys, void* __restrict__ out, int64_t T, int d, int k) {
+                   const float* __restrict__ ys, void* __restrict__ out, int64_t T, int d, int k,
+                   StatsParams sp) {
+    if (sp.sums && blockIdx.x == gridDim.x - 1) {
+        stats_block(sp);
+        return;
+    }
     const int vecs = d / 8;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= T * vecs) return;
@@ -72,47 +134,9 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// sums = [T, entropy sum, P sums (E), routed (E), kept (E)]
-__global__ void stats_sums_kernel(const float* __restrict__ ppart, const float* __restrict__ hpart,
-                                  int nblk, const int32_t* __restrict__ routed,
-                                  const int32_t* __restrict__ kept, int64_t T, int E,
-                                  double* __restrict__ sums) {
-    const int tid = threadIdx.x;
-    if (tid == 0) {
-        double h = 0.0;
-        for (int b = 0; b < nblk; ++b) h += (double)hpart[b];
-        sums[0] = (double)T;
-        sums[1] = h;
-    }
-    for (int e = tid; e < E; e += blockDim.x) {
-        double p = 0.0;
-        for (int b = 0; b < nblk; ++b) p += (double)ppart[(int64_t)b * E + e];
-        sums[2 + e] = p;
-        sums[2 + E + e] = T > 0 ? (double)routed[e] : 0.0;
-        sums[2 + 2 * E + e] = T > 0 ? (double)kept[e] : 0.0;
-    }
-}
-
 __global__ void stats_finalize_kernel(const double* __restrict__ sums, int E, int k,
                                       moe_stats* __restrict__ st) {
-    if (threadIdx.x != 0) return;
-    const double T = sums[0];
-    moe_stats r{0.0, 0.0, 0.0, T, 0.0};
-    if (T > 0.0) {
-        const double tk = T * k;
-        double aux = 0.0, dropped = 0.0;
-        for (int e = 0; e < E; ++e) {
-            const double f = sums[2 + E + e] / tk;  // share of assignments (before the limit)
-            const double P = sums[2 + e] / T;       // mean router probability
-            aux += f * P;
-            dropped += sums[2 + E + e] - sums[2 + 2 * E + e];
-        }
-        r.aux_loss = (double)E * aux;
-        r.overflow_rate = dropped / tk;
-        r.mean_entropy = sums[1] / T;
-        r.dropped = dropped;
-    }
-    *st = r;
+    if (threadIdx.x == 0) finalize_stats(sums, E, k, st);
 }
 
 // Tiled transpose with a row remap for the packed weight layouts.
@@ -144,22 +168,24 @@ __global__ void pack_kernel(const Tv* __restrict__ src, Tv* __restrict__ dst, in
 
 int launch_combine(const float* y, int splits, int64_t split_stride, const int32_t* slot_of,
                    const float* gate, const float* y_shared, void* out, bool out_bf16, int64_t T,
-                   int d, int k, cudaStream_t st) {
-    if (T == 0) return 0;
+                   int d, int k, const StatsParams* sp, cudaStream_t st) {
+    if (T == 0) return sp ? launch_stats(*sp, st) : 0;
     const int64_t n = T * (d / 8);
-    const unsigned blocks = (unsigned)((n + 255) / 256);
+    StatsParams none;
+    memset(&none, 0, sizeof none);
+    const StatsParams& s = sp ? *sp : none;
+    const unsigned blocks = (unsigned)((n + 255) / 256) + (sp ? 1 : 0);
     if (out_bf16)
         combine_kernel<true><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
-                                                     y_shared, out, T, d, k);
+                                                     y_shared, out, T, d, k, s);
     else
         combine_kernel<false><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
-                                                      y_shared, out, T, d, k);
+                                                      y_shared, out, T, d, k, s);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
-int launch_stats_sums(const float* ppart, const float* hpart, int nblk, const int32_t* routed,
-                      const int32_t* kept, int64_t T, int E, double* sums, cudaStream_t st) {
-    stats_sums_kernel<<<1, 256, 0, st>>>(ppart, hpart, nblk, routed, kept, T, E, sums);
+int launch_stats(const StatsParams& a, cudaStream_t st) {
+    stats_kernel<<<1, 256, 0, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -126,10 +126,21 @@ __device__ __forceinline__ Unit decode_unit(const GroupTable& t, int u, const Tc
     x.kb0 = 0;
     x.kb1 = kblocks;
     x.ntok = 0;
-    if (MODE == TC_GATEUP_TOK || MODE == TC_DOWN_TOK) {
+    if (MODE == TC_GATEUP_TOK) {
         const int mtiles = (x.rows + BM - 1) / BM;
         x.mt = local % mtiles;
         x.nb = local / mtiles;
+    } else if (MODE == TC_DOWN_TOK) {
+        // m tile fastest, then n tile, then K split
+        const int mtiles = (x.rows + BM - 1) / BM;
+        const int ntiles = a.n_feat / BN;
+        x.mt = local % mtiles;
+        const int rest = local / mtiles;
+        x.nb = rest % ntiles;
+        x.ks = rest / ntiles;
+        const int per = kblocks / a.splits;
+        x.kb0 = x.ks * per;
+        x.kb1 = x.kb0 + per;
     } else if (MODE == TC_GATEUP_SWAP) {
         x.mt = 0;
         x.nb = local;
@@ -150,7 +161,7 @@ template <int MODE, int BN>
 __device__ __forceinline__ int units_of_group(int rows, const TcArgs& a) {
     if (rows <= 0) return 0;
     if (MODE == TC_GATEUP_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / 128);
-    if (MODE == TC_DOWN_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / BN);
+    if (MODE == TC_DOWN_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / BN) * a.splits;
     if (MODE == TC_GATEUP_SWAP) return a.n_feat / 128;
     return (a.n_feat / 128) * a.splits;
 }
@@ -386,18 +397,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             } else if (MODE == TC_DOWN_TOK) {
                 const int r = x.mt * BM + row;
                 const bool valid = r < x.rows;
-                float* dst = reinterpret_cast<float*>(args.out) +
+                float* dst = reinterpret_cast<float*>(args.out) + x.ks * args.split_stride +
                              (int64_t)(x.row0 + r) * args.out_ld + x.nb * BN;
+                // columns past out_cols (padding of the router GEMM) are not stored
+                const int ncol = args.out_cols > 0 ? min(BN, args.out_cols - x.nb * BN) : BN;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
+                for (int c = 0; c < ncol; c += 16) {
                     float v[16];
                     tmem_ld16(t0 + c, v);
                     tmem_ld_wait();
                     if (valid) {
 #pragma unroll
                         for (int i = 0; i < 16; i += 4)
-                            *reinterpret_cast<float4*>(dst + c + i) =
-                                make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                            if (c + i < ncol)
+                                *reinterpret_cast<float4*>(dst + c + i) =
+                                    make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
                     }
                 }
             } else if (MODE == TC_GATEUP_SWAP) {

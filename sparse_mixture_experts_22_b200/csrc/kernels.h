@@ -9,18 +9,61 @@
 namespace moe {
 
 // ---------------------------------------------------------------- router
-// logits z[T][E] = x[T][d] Wr[d][E] + bias (fp32 accumulate)
-int launch_router_logits(const void* x, bool x_bf16, const float* Wr, const float* bias,
-                         float* z, int64_t T, int d, int E, int num_sms, cudaStream_t st);
-// per-token top-k, gates over the kept k, full-softmax partials and block histograms
-int launch_topk(const float* z, int64_t T, int E, int k, int32_t* topk_idx, float* topk_gate,
-                float* ppart, float* hpart, int32_t* cnt, int32_t* status, cudaStream_t st);
+// logits z[T][E] = x[T][d] Wr[d][E] on the CUDA cores (fp32 accumulate, no bias)
+int launch_router_logits(const void* x, bool x_bf16, const float* Wr, float* z, int64_t T, int d,
+                         int E, int num_sms, cudaStream_t st);
+// T <= 256: partial logits zp[ceil(d/256)][T][E] (256-wide chunks of d, fp32)
+int launch_router_partial(const void* x, bool x_bf16, const float* Wr, float* zp, int T, int d,
+                          int E, cudaStream_t st);
+// W_r [d][E] fp32 -> three bf16 parts, K-major: Ws[p*E + e][d]
+int launch_router_split(const float* Wr, void* Ws, int d, int E, cudaStream_t st);
+// z[t][e] = bias[e] + sum_s sum_p src[s*split_stride + t*row_stride + p*E + e]
+int launch_router_reduce(const float* src, int nsplit, int64_t split_stride, int row_stride,
+                         int nparts, const float* bias, float* z, int64_t T, int E,
+                         cudaStream_t st);
 
-// ---------------------------------------------------------------- dispatch
-int launch_dispatch(const int32_t* topk_idx, const int32_t* cnt, int64_t T, int E, int k,
-                    int64_t C, int pad, int64_t perm_rows, const void* x, int row_bytes,
-                    int32_t* routed, int32_t* kept, int32_t* offsets, int32_t* perm_token,
-                    int32_t* slot_of, void* x_perm, int num_sms, cudaStream_t st);
+// ---------------------------------------------------------------- top-k and dispatch
+struct RouteParams {
+    const float* src;       // logit partials (summed as in launch_router_reduce)
+    int nsplit;
+    int64_t split_stride;
+    int row_stride;
+    int nparts;
+    const float* bias;      // may be null
+    float* zbuf;            // [T][E] scratch
+    float* logits;          // optional copy of the logits for the caller
+    int64_t T;
+    int E, k;
+    int32_t* topk_idx;      // [T][k]
+    float* topk_gate;       // [T][k]
+    float* ppart;           // [blocks][E] full-softmax partial sums
+    float* hpart;           // [blocks] entropy partial sums
+    int32_t* cnt;           // [blocks][E] histogram of kept-expert choices
+    int32_t* status;        // device status word (+ combine ticket)
+};
+
+struct DispatchParams {
+    int64_t T;
+    int E, k;
+    int64_t C;
+    int pad;
+    int64_t perm_rows;
+    const void* x;
+    int row_bytes;
+    int32_t* routed;
+    int32_t* kept;
+    int32_t* offsets;
+    int32_t* perm_token;    // may be null
+    int32_t* slot_of;
+    void* x_perm;
+};
+
+int launch_topk(const RouteParams& r, cudaStream_t st);
+int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, const int32_t* cnt,
+                    int num_sms, cudaStream_t st);
+// T <= 128: top-k and dispatch in one launch
+int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num_sms,
+                          cudaStream_t st);
 
 // ---------------------------------------------------------------- tensor-core GEMMs
 enum TcMode : int { TC_GATEUP_TOK = 0, TC_DOWN_TOK = 1, TC_GATEUP_SWAP = 2, TC_DOWN_SWAP = 3 };
@@ -33,11 +76,12 @@ struct TcArgs {
     int K;                      // reduction length
     int n_feat;                 // gate/up: hidden width; down: model width
     int w_rows_per_group;       // weight rows per group (gate/up: 2h; down: d)
-    int splits;                 // split-K of the swapped down projection
+    int splits;                 // split-K (down projection / router; 1 for gate/up)
     int nt_max;                 // swapped: max tokens per group, multiple of 16
     int stages;                 // shared-memory pipeline depth
     void* out;                  // H (bf16) or y (fp32)
     int64_t out_ld;             // elements per output row
+    int out_cols;               // token-major down: columns written (0 = all)
     int64_t split_stride;       // elements between split-K partial outputs
     int32_t* status;            // device status word
     uint64_t wait_limit_ns;
@@ -58,11 +102,24 @@ int launch_f32_down(const float* H, const float* W2p, float* Y, int num_groups,
                     int64_t rows_bound, int d, int h, cudaStream_t st);
 
 // ---------------------------------------------------------------- combine / stats / pack
+struct StatsParams {
+    const float* ppart;     // [nblk][E]
+    const float* hpart;     // [nblk]
+    int nblk;
+    const int32_t* routed;  // [E]
+    const int32_t* kept;    // [E]
+    int64_t T;
+    int E, k;
+    double* sums;           // [2 + 3E]: T, entropy sum, P sums, routed, kept
+    void* stats;            // moe_stats, or null for the sums alone
+};
+
+// out[t] = sum_j gate * sum_s y[s][slot] + y_shared[t]; with sp, one more block
+// computes the statistics in the same launch
 int launch_combine(const float* y, int splits, int64_t split_stride, const int32_t* slot_of,
                    const float* gate, const float* y_shared, void* out, bool out_bf16,
-                   int64_t T, int d, int k, cudaStream_t st);
-int launch_stats_sums(const float* ppart, const float* hpart, int nblk, const int32_t* routed,
-                      const int32_t* kept, int64_t T, int E, double* sums, cudaStream_t st);
+                   int64_t T, int d, int k, const StatsParams* sp, cudaStream_t st);
+int launch_stats(const StatsParams& a, cudaStream_t st);
 int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStream_t st);
 // dst[remap(c)][r + row_off] = src[r][c] for a [R][Cc] source; remap interleaves
 // 128-wide hidden blocks (gate/up) when `interleave` >= 0 (0 = gate, 1 = up).

@@ -17,6 +17,13 @@ enum FfnPath : int {
     PATH_F32 = 2,          // fp32 SIMT (fp32 configs; no TF32)
 };
 
+// How the router logits are computed.
+enum RouterKind : int {
+    ROUTER_PARTIAL = 0,  // T <= 256: split-d partial dot products on the CUDA cores
+    ROUTER_TC = 1,       // bf16, T > 256: tensor-core GEMM against 3 bf16 parts of W_r
+    ROUTER_SIMT = 2,     // fp32, T > 256: fp32 dot products on the CUDA cores
+};
+
 constexpr int ROUTE_BLOCK = 128;  // tokens per router / dispatch block
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 8;
@@ -37,9 +44,14 @@ struct Plan {
     int64_t perm_rows;  // rows of x_perm / each y_perm split
     int nblk;           // router blocks of ROUTE_BLOCK tokens
     int hsum;           // S * hs (fused shared width)
+    int router_kind;    // RouterKind
+    int router_npad;    // tensor cores: padded GEMM width of the 3 bf16 parts of W_r
+    int router_bn;      // tensor cores: tile width of the router GEMM
+    int router_ld;      // tensor cores: row length of the partial logits (3E rounded to 4)
+    int router_splits;  // tensor cores: split-K; partial: number of d chunks
 
     // workspace byte offsets
-    size_t off_status, off_logits, off_ppart, off_hpart, off_cnt, off_offsets, off_perm,
+    size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_offsets, off_perm,
         off_xperm, off_H, off_y, off_Hs, off_ys, off_sums, total;
 };
 

@@ -12,11 +12,10 @@
 // every 256 elements with 16-byte (fp32) or 8-byte (bf16) loads.  The work is
 // HBM-bound for E = 8 (x is read once) and FP32-pipe bound for E = 160.
 //
-// Kernel 2 (topk): one thread per token.  Keeps the k largest logits in
-// registers (strictly greater wins, so the lower index keeps a tie), gates
-// = softmax over the kept k, then the full softmax for the block partial sums
-// of P_e, the per-token entropy and the per-block expert histogram that
-// dispatch scans.  All block sums run in a fixed order (deterministic).
+// Small batches (<= 256 tokens) use split-d partial dot products instead, and
+// bf16 batches above that a tensor-core GEMM against W_r split into three
+// bf16 parts; the partial sums are added in a fixed order (router_reduce, or
+// inside the top-k kernel).  Top-k and gates live in routing.cu.
 #include <math.h>
 
 #include "common.cuh"
@@ -52,8 +51,7 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
 template <typename XT, int TPW>
 __global__ void __launch_bounds__(RT_WARPS * 32)
     router_logits_kernel(const XT* __restrict__ x, const float* __restrict__ Wr,
-                         const float* __restrict__ bias, float* __restrict__ z, int64_t T, int d,
-                         int E, int dch) {
+                         float* __restrict__ z, int64_t T, int d, int E, int dch) {
     // W_r columns e0..e0+7, transposed: [RT_EXP][dch + 4] (the +4 staggers banks)
     extern __shared__ float ws[];
     const int pitch = dch + 4;
@@ -122,7 +120,6 @@ __global__ void __launch_bounds__(RT_WARPS * 32)
             acc[i][e] = v;
         }
     if (lane < RT_EXP && lane < ne) {
-        const float b = bias ? bias[e0 + lane] : 0.f;
 #pragma unroll
         for (int i = 0; i < TPW; ++i) {
             const int64_t t = t0 + i;
@@ -130,14 +127,14 @@ __global__ void __launch_bounds__(RT_WARPS * 32)
 #pragma unroll
             for (int e = 0; e < RT_EXP; ++e)
                 if (e == lane) v = acc[i][e];
-            if (t < T) z[t * E + e0 + lane] = v + b;
+            if (t < T) z[t * E + e0 + lane] = v;
         }
     }
 }
 
 template <typename XT, int TPW>
-int launch_logits_t(const XT* x, const float* Wr, const float* bias, float* z, int64_t T, int d,
-                    int E, cudaStream_t st) {
+int launch_logits_t(const XT* x, const float* Wr, float* z, int64_t T, int d, int E,
+                    cudaStream_t st) {
     const int tok_per_cta = RT_WARPS * TPW;
     dim3 grid((unsigned)((T + tok_per_cta - 1) / tok_per_cta), (E + RT_EXP - 1) / RT_EXP);
     const int dch = d < RT_DCH ? d : RT_DCH;
@@ -150,149 +147,174 @@ int launch_logits_t(const XT* x, const float* Wr, const float* bias, float* z, i
             return -1;
         configured = smem;
     }
-    kern<<<grid, RT_WARPS * 32, smem, st>>>(x, Wr, bias, z, T, d, E, dch);
+    kern<<<grid, RT_WARPS * 32, smem, st>>>(x, Wr, z, T, d, E, dch);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 template <typename XT>
-int launch_logits_dispatch(const XT* x, const float* Wr, const float* bias, float* z, int64_t T,
-                           int d, int E, int num_sms, cudaStream_t st) {
+int launch_logits_dispatch(const XT* x, const float* Wr, float* z, int64_t T, int d, int E,
+                           int num_sms, cudaStream_t st) {
     // tokens per warp: as many as keep at least ~2 CTAs per SM busy
     const int64_t ctas_e = (E + RT_EXP - 1) / RT_EXP;
     const int64_t want = 2LL * num_sms;
-    if ((T + 63) / 64 * ctas_e >= want) return launch_logits_t<XT, 8>(x, Wr, bias, z, T, d, E, st);
-    if ((T + 31) / 32 * ctas_e >= want) return launch_logits_t<XT, 4>(x, Wr, bias, z, T, d, E, st);
-    if ((T + 15) / 16 * ctas_e >= want) return launch_logits_t<XT, 2>(x, Wr, bias, z, T, d, E, st);
-    return launch_logits_t<XT, 1>(x, Wr, bias, z, T, d, E, st);
+    if ((T + 63) / 64 * ctas_e >= want) return launch_logits_t<XT, 8>(x, Wr, z, T, d, E, st);
+    if ((T + 31) / 32 * ctas_e >= want) return launch_logits_t<XT, 4>(x, Wr, z, T, d, E, st);
+    if ((T + 15) / 16 * ctas_e >= want) return launch_logits_t<XT, 2>(x, Wr, z, T, d, E, st);
+    return launch_logits_t<XT, 1>(x, Wr, z, T, d, E, st);
 }
 
-// ---------------------------------------------------------------- top-k
+// ---------------------------------------------------------------- small batches
+//
+// With at most 256 tokens the router is a latency problem, not a bandwidth
+// one: the d dimension is cut into 256-wide chunks and every (chunk, 8-expert
+// group) pair is its own CTA, so W_r and x are read by ~d/256 CTAs at once.  Thread t owns token t; the chunk of W_r sits in shared memory and
+// is read as a broadcast.  Each CTA writes its partial logits
+// zp[chunk][t][e]; topk adds the chunks in fixed order.
+constexpr int RP_DC = 256;
 
-constexpr int TK_CHUNK = 32;  // experts per shared-memory pass of the P partial sums
+template <typename XT>
+__device__ __forceinline__ void load8(const XT* p, float* v);
 
-__global__ void __launch_bounds__(ROUTE_BLOCK)
-    topk_kernel(const float* __restrict__ z, int64_t T, int E, int k, int32_t* __restrict__ idx,
-                float* __restrict__ gate, float* __restrict__ ppart, float* __restrict__ hpart,
-                int32_t* __restrict__ cnt, int32_t* __restrict__ status) {
-    __shared__ float ps[ROUTE_BLOCK][TK_CHUNK + 1];
-    __shared__ float hs[ROUTE_BLOCK];
-    extern __shared__ int32_t hist[];  // [E]
-    const int tid = threadIdx.x;
-    const int64_t t = (int64_t)blockIdx.x * ROUTE_BLOCK + tid;
-    const bool valid = t < T;
-    const float* zt = z + (valid ? t : 0) * E;
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float* v) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 
-    for (int e = tid; e < E; e += ROUTE_BLOCK) hist[e] = 0;
-    // a new layer call starts here: clear the device status word
-    if (blockIdx.x == 0 && tid == 0 && status) *status = DEV_OK;
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
 
-    float val[MAX_K];
-    int id[MAX_K];
-#pragma unroll
-    for (int j = 0; j < MAX_K; ++j) {
-        val[j] = -INFINITY;
-        id[j] = -1;
+template <typename XT>
+__global__ void __launch_bounds__(256)
+    router_partial_kernel(const XT* __restrict__ x, const float* __restrict__ Wr,
+                          float* __restrict__ zp, int T, int d, int E) {
+    __shared__ float ws[RP_DC][RT_EXP];
+    const int c0 = blockIdx.x * RP_DC;
+    const int e0 = blockIdx.y * RT_EXP;
+    const int ne = min(RT_EXP, E - e0);
+    const int len = min(RP_DC, d - c0);
+    for (int i = threadIdx.x; i < RP_DC * RT_EXP; i += blockDim.x) {
+        const int c = i / RT_EXP, e = i % RT_EXP;
+        ws[c][e] = (c < len && e < ne) ? Wr[(int64_t)(c0 + c) * E + e0 + e] : 0.f;
     }
-    if (valid) {
-        for (int e = 0; e < E; ++e) {
-            float v = zt[e];
-            if (v != v) v = -INFINITY;  // a NaN logit ranks last
-            // insert if larger than the current k-th (or a slot is still empty):
-            // walk the sorted list; from the insertion point on, every entry
-            // shifts down one place and the old k-th falls off
-            if (id[k - 1] < 0 || v > val[k - 1]) {
-                float cv = v;
-                int ci = e;
-                bool ins = false;
-#pragma unroll
-                for (int q = 0; q < MAX_K; ++q) {
-                    if (q < k && (ins || id[q] < 0 || cv > val[q])) {
-                        const float tv = val[q];
-                        const int ti = id[q];
-                        val[q] = cv;
-                        id[q] = ci;
-                        cv = tv;
-                        ci = ti;
-                        ins = true;
-                    }
-                }
-            }
-        }
-    }
-    __syncthreads();  // hist cleared
-    float m = val[0];
-    if (valid) {
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < MAX_K; ++j)
-            if (j < k) s += __expf(val[j] - m);
-        const float inv = 1.f / s;
-#pragma unroll
-        for (int j = 0; j < MAX_K; ++j)
-            if (j < k) {
-                idx[t * k + j] = id[j];
-                gate[t * k + j] = __expf(val[j] - m) * inv;
-                atomicAdd(&hist[id[j]], 1);
-            }
-    }
-    // full softmax over E: S = sum exp(z - m); p = exp(z - m) / S;
-    // entropy = ln S - sum p (z - m)
-    float S = 0.f;
-    if (valid)
-        for (int e = 0; e < E; ++e) {
-            float v = zt[e];
-            S += __expf((v != v ? -INFINITY : v) - m);
-        }
-    const float invS = valid ? 1.f / S : 0.f;
-    float pz = 0.f;
-    for (int c0 = 0; c0 < E; c0 += TK_CHUNK) {
-        const int n = min(TK_CHUNK, E - c0);
-        for (int i = 0; i < n; ++i) {
-            float p = 0.f;
-            if (valid) {
-                float v = zt[c0 + i];
-                v = (v != v) ? -INFINITY : v;
-                p = __expf(v - m) * invS;
-                if (p > 0.f) pz += p * (v - m);
-            }
-            ps[tid][i] = p;
-        }
-        __syncthreads();
-        if (tid < n) {
-            float acc = 0.f;
-            for (int r = 0; r < ROUTE_BLOCK; ++r) acc += ps[r][tid];
-            ppart[(int64_t)blockIdx.x * E + c0 + tid] = acc;
-        }
-        __syncthreads();
-    }
-    hs[tid] = valid ? (__logf(S) - pz) : 0.f;
     __syncthreads();
-    if (tid == 0) {
-        float acc = 0.f;
-        for (int r = 0; r < ROUTE_BLOCK; ++r) acc += hs[r];
-        hpart[blockIdx.x] = acc;
+    const int t = threadIdx.x;
+    if (t >= T) return;
+    float acc[RT_EXP];
+#pragma unroll
+    for (int e = 0; e < RT_EXP; ++e) acc[e] = 0.f;
+    const XT* xr = x + (int64_t)t * d + c0;
+#pragma unroll 2
+    for (int c = 0; c < len; c += 8) {
+        float xv[8];
+        load8<XT>(xr + c, xv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < RT_EXP; ++e) acc[e] = fmaf(xv[j], ws[c + j][e], acc[e]);
     }
-    for (int e = tid; e < E; e += ROUTE_BLOCK) cnt[(int64_t)blockIdx.x * E + e] = hist[e];
+    float* out = zp + ((int64_t)blockIdx.x * T + t) * E + e0;
+#pragma unroll
+    for (int e = 0; e < RT_EXP; ++e)
+        if (e < ne) out[e] = acc[e];
+}
+
+// ---------------------------------------------------------------- router on the tensor cores
+//
+// For bf16 tokens the logits run as a tensor-core GEMM (gemm_tc.cu) against
+// W_r split into three bf16 parts, W = W_hi + W_mid + W_lo (each part the
+// bf16 rounding of what the earlier parts leave), stored transposed
+// (K-major): Ws[p*E + e][c].  Every product of a bf16 token element with a
+// bf16 part is exact in fp32 and the three partial sums together carry W to
+// 24 bits, so the logits keep fp32 accuracy.  topk sums the parts.
+__global__ void router_split_kernel(const float* __restrict__ Wr, __nv_bfloat16* __restrict__ Ws,
+                                    int d, int E) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)d * E) return;
+    const int e = (int)(i % E);
+    const int64_t c = i / E;
+    const float w = Wr[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+    Ws[(int64_t)e * d + c] = hi;
+    Ws[(int64_t)(E + e) * d + c] = mid;
+    Ws[(int64_t)(2 * E + e) * d + c] = lo;
+}
+
+// ---------------------------------------------------------------- partial-sum reduction
+//
+// z[t][e] = bias[e] + sum over splits s and parts p of src[s][t][p*E + e], in
+// that fixed order; one thread per logit, coalesced along e.
+__global__ void __launch_bounds__(256)
+    router_reduce_kernel(const float* __restrict__ src, int nsplit, int64_t split_stride,
+                         int row_stride, int nparts, const float* __restrict__ bias,
+                         float* __restrict__ z, int64_t T, int E) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * E) return;
+    const int64_t t = i / E;
+    const int e = (int)(i % E);
+    float v = bias ? bias[e] : 0.f;
+    const float* base = src + t * row_stride + e;
+    for (int q = 0; q < nsplit; ++q) {
+        const float* r = base + q * split_stride;
+#pragma unroll 4
+        for (int p = 0; p < nparts; ++p) v += r[p * E];
+    }
+    z[i] = v;
 }
 
 }  // namespace
 
-int launch_router_logits(const void* x, bool x_bf16, const float* Wr, const float* bias,
-                         float* z, int64_t T, int d, int E, int num_sms, cudaStream_t st) {
+int launch_router_logits(const void* x, bool x_bf16, const float* Wr, float* z, int64_t T, int d,
+                         int E, int num_sms, cudaStream_t st) {
     if (T == 0) return 0;
     if (x_bf16)
-        return launch_logits_dispatch(reinterpret_cast<const __nv_bfloat16*>(x), Wr, bias, z, T, d,
-                                      E, num_sms, st);
-    return launch_logits_dispatch(reinterpret_cast<const float*>(x), Wr, bias, z, T, d, E,
-                                  num_sms, st);
+        return launch_logits_dispatch(reinterpret_cast<const __nv_bfloat16*>(x), Wr, z, T, d, E,
+                                      num_sms, st);
+    return launch_logits_dispatch(reinterpret_cast<const float*>(x), Wr, z, T, d, E, num_sms, st);
 }
 
-int launch_topk(const float* z, int64_t T, int E, int k, int32_t* topk_idx, float* topk_gate,
-                float* ppart, float* hpart, int32_t* cnt, int32_t* status, cudaStream_t st) {
+int launch_router_partial(const void* x, bool x_bf16, const float* Wr, float* zp, int T, int d,
+                          int E, cudaStream_t st) {
     if (T == 0) return 0;
-    const unsigned blocks = (unsigned)((T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
-    topk_kernel<<<blocks, ROUTE_BLOCK, E * sizeof(int32_t), st>>>(z, T, E, k, topk_idx, topk_gate,
-                                                                  ppart, hpart, cnt, status);
+    if (T > 256) return -1;
+    dim3 grid((d + RP_DC - 1) / RP_DC, (E + RT_EXP - 1) / RT_EXP);
+    if (x_bf16)
+        router_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(x), Wr, zp, T, d, E);
+    else
+        router_partial_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(x), Wr,
+                                                           zp, T, d, E);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_router_reduce(const float* src, int nsplit, int64_t split_stride, int row_stride,
+                         int nparts, const float* bias, float* z, int64_t T, int E,
+                         cudaStream_t st) {
+    if (T == 0) return 0;
+    const int64_t n = T * E;
+    router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        src, nsplit, split_stride, row_stride, nparts, bias, z, T, E);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_router_split(const float* Wr, void* Ws, int d, int E, cudaStream_t st) {
+    const int64_t n = (int64_t)d * E;
+    router_split_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        Wr, reinterpret_cast<__nv_bfloat16*>(Ws), d, E);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

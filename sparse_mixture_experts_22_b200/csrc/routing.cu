@@ -1,0 +1,474 @@
+// routing.cu -- top-k selection, gates, router statistics partials, and the
+// capacity-limited dispatch of token rows to experts.
+//
+// Top-k and gates [Mixtral 8x7B and MoE explained, "Easy explanation" ¶3]:
+// keep the k highest-scoring experts and softmax over those k to weight their
+// outputs.  One thread per token keeps the k largest logits in registers
+// (strictly greater wins, so the lower expert index keeps a tie).  The full
+// softmax over all E experts [MoE routing fully explained, "Easy explanation"
+// ¶2] feeds the per-block partial sums of P_e and of the token entropy.
+//
+// Dispatch [MoE routing fully explained, "Easy explanation" ¶3 and ¶5]: every
+// expert takes at most C = ceil(T k cf / E) tokens per batch and the overflow
+// is dropped, in arrival order by token index: the rank of assignment (t, j)
+// in expert e is the number of earlier tokens that chose e, kept if rank < C.
+// The rank needs no atomics on the order: per-128-token block histograms, a
+// scan over earlier blocks, then inside the block one warp ballot per expert
+// and per-warp counts.  Results are identical on every run.
+//
+// Batches of at most 128 tokens run top-k and dispatch in one kernel
+// (route_dispatch_kernel); several CTAs repeat the cheap routing and share the
+// row copies into x_perm, so a decode batch spreads its gather over many SMs.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int TK_CHUNK = 32;     // experts per shared-memory pass of the P partial sums
+constexpr int TK_SMEM_E = 256;   // up to this many experts a block's logits sit in shared memory
+constexpr int DWARPS = ROUTE_BLOCK / 32;
+
+struct TopkArgs {
+    const float* src;      // logit partials: z = bias + sum_s sum_p src[s][t][p*E + e]
+    int nsplit;
+    int64_t split_stride;
+    int row_stride;
+    int nparts;
+    const float* bias;     // may be null
+    float* zbuf;           // [T][E] scratch for E > TK_SMEM_E
+    float* logits;         // optional user copy of z [T][E]
+    int64_t T;
+    int E, k;
+    int32_t* idx;          // [T][k]
+    float* gate;           // [T][k]
+    float* ppart;          // [blocks][E]
+    float* hpart;          // [blocks]
+    int32_t* status;       // device status word (cleared here: a layer call starts)
+};
+
+// Shared memory of topk_block: hist [E] int32, then (E <= TK_SMEM_E) the
+// block's logits [ROUTE_BLOCK][E + 1] fp32.
+__host__ __device__ inline size_t topk_smem_bytes(int E) {
+    size_t b = (size_t)E * sizeof(int32_t);
+    if (E <= TK_SMEM_E) b += (size_t)ROUTE_BLOCK * (E + 1) * sizeof(float);
+    return b;
+}
+
+// Routes the ROUTE_BLOCK tokens of block `blk`.  Leaves the per-expert
+// histogram of the block in hist[] (shared) and the thread's kept experts in
+// my[] (-1 past k or for padding threads).  Global outputs are written only
+// when `write` is set.
+__device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist, float* zs,
+                           int32_t* my) {
+    __shared__ float ps[ROUTE_BLOCK][TK_CHUNK + 1];
+    __shared__ float hs[ROUTE_BLOCK];
+    const int E = a.E, k = a.k;
+    const bool in_smem = E <= TK_SMEM_E;
+    const int tid = threadIdx.x;
+    const int64_t tb = (int64_t)blk * ROUTE_BLOCK;
+    const int nvalid = (int)(a.T - tb < ROUTE_BLOCK ? a.T - tb : ROUTE_BLOCK);
+    const int64_t t = tb + tid;
+    const bool valid = tid < nvalid;
+
+    for (int e = tid; e < E; e += ROUTE_BLOCK) hist[e] = 0;
+
+    // logits of the block, all threads, coalesced; partials added in fixed order
+    for (int i = tid; i < nvalid * E; i += ROUTE_BLOCK) {
+        const int tl = i / E, e = i % E;
+        const int64_t tt = tb + tl;
+        float v = a.bias ? a.bias[e] : 0.f;
+        const float* base = a.src + tt * a.row_stride + e;
+        if (a.nparts == 1) {
+#pragma unroll 8
+            for (int q = 0; q < a.nsplit; ++q) v += base[q * a.split_stride];
+        } else {
+            for (int q = 0; q < a.nsplit; ++q) {
+                const float* r = base + q * a.split_stride;
+                for (int p = 0; p < a.nparts; ++p) v += r[p * E];
+            }
+        }
+        if (in_smem) zs[tl * (E + 1) + e] = v;
+        else a.zbuf[tt * E + e] = v;
+        if (write && a.logits) a.logits[tt * E + e] = v;
+    }
+    __syncthreads();
+    const float* zt = in_smem ? zs + tid * (E + 1) : a.zbuf + (valid ? t : 0) * E;
+
+    float val[MAX_K];
+    int id[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        val[j] = -INFINITY;
+        id[j] = -1;
+    }
+    if (valid) {
+        for (int e = 0; e < E; ++e) {
+            float v = zt[e];
+            if (v != v) v = -INFINITY;  // a NaN logit ranks last
+            // insert if larger than the current k-th (or a slot is still empty):
+            // from the insertion point on every entry shifts down one place and
+            // the old k-th falls off
+            if (id[k - 1] < 0 || v > val[k - 1]) {
+                float cv = v;
+                int ci = e;
+                bool ins = false;
+#pragma unroll
+                for (int q = 0; q < MAX_K; ++q) {
+                    if (q < k && (ins || id[q] < 0 || cv > val[q])) {
+                        const float tv = val[q];
+                        const int ti = id[q];
+                        val[q] = cv;
+                        id[q] = ci;
+                        cv = tv;
+                        ci = ti;
+                        ins = true;
+                    }
+                }
+            }
+        }
+    }
+    const float m = val[0];
+    if (valid) {
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j)
+            if (j < k) s += __expf(val[j] - m);
+        const float inv = 1.f / s;
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j)
+            if (j < k) {
+                if (write) {
+                    a.idx[t * k + j] = id[j];
+                    a.gate[t * k + j] = __expf(val[j] - m) * inv;
+                }
+                atomicAdd(&hist[id[j]], 1);
+            }
+    }
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) my[j] = (valid && j < k) ? id[j] : -1;
+
+    // full softmax over E: S = sum exp(z - m); p = exp(z - m) / S;
+    // entropy = ln S - sum p (z - m)
+    float S = 0.f;
+    if (valid)
+        for (int e = 0; e < E; ++e) {
+            const float v = zt[e];
+            S += __expf((v != v ? -INFINITY : v) - m);
+        }
+    const float invS = valid ? 1.f / S : 0.f;
+    float pz = 0.f;
+    for (int c0 = 0; c0 < E; c0 += TK_CHUNK) {
+        const int n = min(TK_CHUNK, E - c0);
+        for (int i = 0; i < n; ++i) {
+            float p = 0.f;
+            if (valid) {
+                float v = zt[c0 + i];
+                v = (v != v) ? -INFINITY : v;
+                p = __expf(v - m) * invS;
+                if (p > 0.f) pz += p * (v - m);
+            }
+            ps[tid][i] = p;
+        }
+        __syncthreads();
+        if (write && tid < n) {
+            float acc = 0.f;
+            for (int r = 0; r < ROUTE_BLOCK; ++r) acc += ps[r][tid];
+            a.ppart[(int64_t)blk * E + c0 + tid] = acc;
+        }
+        __syncthreads();
+    }
+    hs[tid] = valid ? (__logf(S) - pz) : 0.f;
+    __syncthreads();
+    if (write && tid == 0) {
+        float acc = 0.f;
+        for (int r = 0; r < ROUTE_BLOCK; ++r) acc += hs[r];
+        a.hpart[blk] = acc;
+    }
+}
+
+struct DispatchArgs {
+    int64_t T;
+    int E, k;
+    int64_t C;
+    int pad;
+    int64_t perm_rows;
+    const uint4* x;
+    int row_vecs;          // 16-byte vectors per row of x
+    int32_t* routed;       // [E]
+    int32_t* kept;         // [E]
+    int32_t* offsets;      // [E+1]
+    int32_t* perm_token;   // [perm_rows] (may be null)
+    int32_t* slot_of;      // [T][k]
+    uint4* x_perm;         // [perm_rows][d]
+};
+
+// Shared memory of dispatch_block: base [E], tot [E], off [E+1], wcnt [DWARPS][E],
+// slots [ROUTE_BLOCK * k].
+__host__ __device__ inline size_t dispatch_smem_bytes(int E, int k) {
+    return sizeof(int32_t) * ((size_t)3 * E + 1 + (size_t)DWARPS * E + (size_t)ROUTE_BLOCK * k);
+}
+
+// Ranks, slots and row copies of block `blk`.  base[e] (assignments to e in
+// earlier blocks) and tot[e] (in all blocks) must be in shared memory; my[]
+// holds the thread's token choices.  `split`/`nsplit`: this CTA copies every
+// nsplit-th row.  Outputs other than the copies are written when `writer`.
+__device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool writer, int split,
+                               int nsplit, int32_t* base, int32_t* tot, int32_t* off,
+                               int32_t* wcnt, int32_t* slots, const int32_t* my) {
+    const int E = a.E, k = a.k;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        int32_t o = 0;
+        for (int e = 0; e < E; ++e) {
+            off[e] = o;
+            const int32_t kept = (int64_t)tot[e] < a.C ? tot[e] : (int32_t)a.C;
+            o += (kept + a.pad - 1) / a.pad * a.pad;
+        }
+        off[E] = o;
+    }
+    __syncthreads();
+    if (writer) {
+        if (blk == 0) {
+            for (int e = tid; e < E; e += ROUTE_BLOCK) {
+                a.routed[e] = tot[e];
+                a.kept[e] = (int64_t)tot[e] < a.C ? tot[e] : (int32_t)a.C;
+            }
+            for (int e = tid; e <= E; e += ROUTE_BLOCK) a.offsets[e] = off[e];
+        }
+        if (a.perm_token) {
+            // padding rows of each expert segment, and the unused tail, hold -1
+            for (int e = blk; e < E; e += nblk) {
+                const int32_t kept = (int64_t)tot[e] < a.C ? tot[e] : (int32_t)a.C;
+                for (int r = off[e] + kept + tid; r < off[e + 1]; r += ROUTE_BLOCK)
+                    a.perm_token[r] = -1;
+            }
+            for (int64_t r = off[E] + (int64_t)blk * ROUTE_BLOCK + tid; r < a.perm_rows;
+                 r += (int64_t)nblk * ROUTE_BLOCK)
+                a.perm_token[r] = -1;
+        }
+    }
+
+    const int64_t t = (int64_t)blk * ROUTE_BLOCK + tid;
+    const bool valid = t < a.T;
+    int32_t rank_w[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) rank_w[j] = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int e = 0; e < E; ++e) {
+        bool chose = false;
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) chose |= (my[j] == e);
+        const unsigned msk = __ballot_sync(0xffffffffu, chose);
+        if (lane == 0) wcnt[warp * E + e] = __popc(msk);
+        if (chose) {
+            const int r = __popc(msk & lt);
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j)
+                if (my[j] == e) rank_w[j] = r;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        if (j >= k) break;
+        int32_t slot = -1;
+        if (valid) {
+            const int e = my[j];
+            int32_t r = base[e] + rank_w[j];
+            for (int w = 0; w < warp; ++w) r += wcnt[w * E + e];
+            if ((int64_t)r < a.C) slot = off[e] + r;
+            if (writer) {
+                a.slot_of[t * k + j] = slot;
+                if (slot >= 0 && a.perm_token) a.perm_token[slot] = (int32_t)t;
+            }
+        }
+        slots[tid * k + j] = slot;
+    }
+    __syncthreads();
+
+    // gather: this CTA copies every nsplit-th (t, j) row of its block
+    const int nrow = ROUTE_BLOCK * k;
+    for (int r = split; r < nrow; r += nsplit) {
+        const int32_t slot = slots[r];
+        if (slot < 0) continue;
+        const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
+        const uint4* __restrict__ src = a.x + tok * a.row_vecs;
+        uint4* __restrict__ dst = a.x_perm + (int64_t)slot * a.row_vecs;
+        const int nv = a.row_vecs;
+#pragma unroll 4
+        for (int c = tid; c < nv; c += ROUTE_BLOCK) dst[c] = __ldg(src + c);
+    }
+}
+
+__global__ void __launch_bounds__(ROUTE_BLOCK)
+    topk_kernel(TopkArgs a, int32_t* __restrict__ cnt) {
+    extern __shared__ int32_t dyn[];
+    int32_t* hist = dyn;
+    float* zs = reinterpret_cast<float*>(dyn + a.E);
+    int32_t my[MAX_K];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && a.status) {
+        a.status[0] = DEV_OK;  // a new layer call starts here
+        a.status[1] = 0;       // combine's completion ticket
+    }
+    topk_block(a, blockIdx.x, true, hist, zs, my);
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK)
+        cnt[(int64_t)blockIdx.x * a.E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(ROUTE_BLOCK)
+    dispatch_kernel(DispatchArgs a, const int32_t* __restrict__ topk_idx,
+                    const int32_t* __restrict__ cnt) {
+    extern __shared__ int32_t sm[];
+    int32_t* base = sm;
+    int32_t* tot = base + a.E;
+    int32_t* off = tot + a.E;
+    int32_t* wcnt = off + a.E + 1;
+    int32_t* slots = wcnt + DWARPS * a.E;
+    const int blk = blockIdx.x, nblk = gridDim.x;
+    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) {
+        int32_t b = 0, s = 0;
+        for (int q = 0; q < nblk; ++q) {
+            const int32_t c = cnt[(int64_t)q * a.E + e];
+            if (q < blk) b += c;
+            s += c;
+        }
+        base[e] = b;
+        tot[e] = s;
+    }
+    const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
+    int32_t my[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) my[j] = (t < a.T && j < a.k) ? topk_idx[t * a.k + j] : -1;
+    __syncthreads();
+    dispatch_block(a, blk, nblk, blockIdx.y == 0, blockIdx.y, gridDim.y, base, tot, off, wcnt,
+                   slots, my);
+}
+
+// T <= ROUTE_BLOCK: top-k and dispatch in one launch.  Every CTA routes the
+// whole batch (cheap) and copies its share of the rows; CTA 0 writes the
+// routing outputs.
+__global__ void __launch_bounds__(ROUTE_BLOCK)
+    route_dispatch_kernel(TopkArgs ta, DispatchArgs da, int32_t* __restrict__ cnt) {
+    extern __shared__ int32_t dyn[];
+    const int E = ta.E;
+    int32_t* hist = dyn;
+    float* zs = reinterpret_cast<float*>(dyn + E);
+    int32_t* dsm = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dyn) + topk_smem_bytes(E));
+    int32_t* base = dsm;
+    int32_t* tot = base + E;
+    int32_t* off = tot + E;
+    int32_t* wcnt = off + E + 1;
+    int32_t* slots = wcnt + DWARPS * E;
+    const bool leader = blockIdx.x == 0;
+    if (leader && threadIdx.x == 0 && ta.status) {
+        ta.status[0] = DEV_OK;
+        ta.status[1] = 0;
+    }
+    int32_t my[MAX_K];
+    topk_block(ta, 0, leader, hist, zs, my);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += ROUTE_BLOCK) {
+        base[e] = 0;
+        tot[e] = hist[e];
+        if (leader) cnt[e] = hist[e];
+    }
+    __syncthreads();
+    dispatch_block(da, 0, 1, leader, blockIdx.x, gridDim.x, base, tot, off, wcnt, slots, my);
+}
+
+template <typename K>
+int set_smem(K kern, size_t bytes) {
+    if (bytes <= 48 * 1024) return 0;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
+                   cudaSuccess
+               ? 0
+               : -1;
+}
+
+TopkArgs topk_args(const RouteParams& r) {
+    TopkArgs a;
+    a.src = r.src;
+    a.nsplit = r.nsplit;
+    a.split_stride = r.split_stride;
+    a.row_stride = r.row_stride;
+    a.nparts = r.nparts;
+    a.bias = r.bias;
+    a.zbuf = r.zbuf;
+    a.logits = r.logits;
+    a.T = r.T;
+    a.E = r.E;
+    a.k = r.k;
+    a.idx = r.topk_idx;
+    a.gate = r.topk_gate;
+    a.ppart = r.ppart;
+    a.hpart = r.hpart;
+    a.status = r.status;
+    return a;
+}
+
+DispatchArgs dispatch_args(const DispatchParams& p) {
+    DispatchArgs a;
+    a.T = p.T;
+    a.E = p.E;
+    a.k = p.k;
+    a.C = p.C;
+    a.pad = p.pad;
+    a.perm_rows = p.perm_rows;
+    a.x = reinterpret_cast<const uint4*>(p.x);
+    a.row_vecs = p.row_bytes / 16;
+    a.routed = p.routed;
+    a.kept = p.kept;
+    a.offsets = p.offsets;
+    a.perm_token = p.perm_token;
+    a.slot_of = p.slot_of;
+    a.x_perm = reinterpret_cast<uint4*>(p.x_perm);
+    return a;
+}
+
+// CTAs per token block for the row copies: about two per SM in total
+int copy_splits(int nblk, int k, int num_sms) {
+    int ny = (2 * num_sms + nblk - 1) / nblk;
+    if (ny > ROUTE_BLOCK * k) ny = ROUTE_BLOCK * k;
+    return ny < 1 ? 1 : ny;
+}
+
+}  // namespace
+
+int launch_topk(const RouteParams& r, cudaStream_t st) {
+    if (r.T == 0) return 0;
+    const unsigned blocks = (unsigned)((r.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    const size_t smem = topk_smem_bytes(r.E);
+    if (set_smem(topk_kernel, smem)) return -1;
+    topk_kernel<<<blocks, ROUTE_BLOCK, smem, st>>>(topk_args(r), r.cnt);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, const int32_t* cnt,
+                    int num_sms, cudaStream_t st) {
+    if (p.T == 0) return 0;
+    const int nblk = (int)((p.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    const size_t smem = dispatch_smem_bytes(p.E, p.k);
+    if (set_smem(dispatch_kernel, smem)) return -1;
+    dim3 grid(nblk, copy_splits(nblk, p.k, num_sms));
+    dispatch_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(dispatch_args(p), topk_idx, cnt);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num_sms,
+                          cudaStream_t st) {
+    if (r.T == 0) return 0;
+    if (r.T > ROUTE_BLOCK) return -1;
+    const size_t smem = topk_smem_bytes(r.E) + dispatch_smem_bytes(p.E, p.k);
+    if (set_smem(route_dispatch_kernel, smem)) return -1;
+    route_dispatch_kernel<<<copy_splits(1, p.k, num_sms), ROUTE_BLOCK, smem, st>>>(
+        topk_args(r), dispatch_args(p), r.cnt);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace moe

@@ -13,9 +13,9 @@ import numpy as np
 import pytest
 import torch
 
-from layer_check import (check_offsets, check_output, check_routing, check_slots, check_stats,
-                         device_layer, host_inputs, oracle_route, oracle_rows, run_forward,
-                         run_steps, sample_rows)
+from layer_check import (check_logits, check_offsets, check_output, check_routing, check_slots,
+                         check_stats, device_layer, host_inputs, oracle_route, oracle_rows,
+                         route_logits, run_forward, run_steps, sample_rows)
 from sparse_mixture_experts_22_b200 import binding as B
 from sparse_mixture_experts_22_b200.workloads import WORKLOADS, Workload
 
@@ -73,12 +73,13 @@ def test_small_layer_matches_oracle(name):
     check_routing(wl, r, b)
     s = run_steps(cfg, g, W)
     assert s["status"] == 0
+    zerr = check_logits(r, s["logits"])
     offsets = s["offsets"].cpu().numpy()
     check_offsets(wl, r, offsets, _pad(cfg))
     check_slots(wl, r, s, offsets, s["perm_token"].cpu().numpy())
     check_slots(wl, r, b, offsets)
     e = check_output(b["out"], ref)
-    print(f"{name}: {e}")
+    print(f"{name}: {e} logit_err={zerr:.2e}")
     check_stats(r, b["stats"], wl.T)
     check_stats(r, s["stats"], wl.T)
     check_stats(r, s["stats2"], wl.T)
@@ -146,6 +147,7 @@ def test_full_size_workload(name):
     b = run_forward(cfg, g, W)
     check_routing(wl, r, b)
     check_stats(r, b["stats"], wl.T)
+    zerr = check_logits(r, route_logits(cfg, g))
     # dropped set and ranks for every assignment (offsets rebuilt from the oracle's kept counts)
     pad = _pad(cfg)
     offsets = np.zeros(wl.E + 1, dtype=np.int64)
@@ -154,4 +156,5 @@ def test_full_size_workload(name):
     check_slots(wl, r, b, offsets)
     rows = sample_rows(wl.T, FULL_SAMPLE[name], seed=1)
     ref = oracle_rows(wl, inp, r, rows)
-    check_output(b["out"][torch.as_tensor(rows, device="cuda")], ref, f"{name} sampled rows")
+    e = check_output(b["out"][torch.as_tensor(rows, device="cuda")], ref, f"{name} sampled rows")
+    print(f"{name}: {e} logit_err={zerr:.2e}")
