@@ -105,15 +105,14 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
         while (P.splits < 8 && units * P.splits < 960 && kblocks % (P.splits * 2) == 0)
             P.splits *= 2;
     }
-    // router: split-d partials for small batches; tensor cores (three bf16 parts
+    // router: one CTA per token for small batches; tensor cores (three bf16 parts
     // of W_r) for larger bf16 batches; fp32 dot products for larger fp32 batches
     P.router_npad = P.E;
     P.router_ld = P.E;
     P.router_bn = 0;
     P.router_splits = 1;
     if (P.T <= SWAP_MAX_TOKENS) {
-        P.router_kind = ROUTER_PARTIAL;
-        P.router_splits = (P.d + 255) / 256;
+        P.router_kind = ROUTER_ROWS;
     } else if (P.bf16) {
         P.router_kind = ROUTER_TC;
         P.router_bn = 3 * P.E <= 128 ? 128 : 256;
@@ -141,10 +140,8 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.off_status = take(256);
     P.off_logits = take((size_t)c.T * c.E * 4);
     P.off_wsplit = take(P.router_kind == ROUTER_TC ? (size_t)3 * c.E * c.d * 2 : 0);
-    P.off_z3 = take(P.router_kind == ROUTER_SIMT
-                        ? 0
-                        : (size_t)P.router_splits * c.T *
-                              (P.router_kind == ROUTER_TC ? P.router_ld : P.router_npad) * 4);
+    P.off_z3 = take(P.router_kind == ROUTER_TC ? (size_t)P.router_splits * c.T * P.router_ld * 4
+                                               : 0);
     P.off_ppart = take((size_t)P.nblk * c.E * 4);
     P.off_hpart = take((size_t)P.nblk * 4);
     P.off_cnt = take((size_t)P.nblk * c.E * 4);
@@ -361,14 +358,11 @@ static int step_logits(const Plan& P, const Device& dv, const void* x, const flo
     r.row_stride = P.E;
     r.split_stride = 0;
     r.bias = bias;
-    if (P.router_kind == ROUTER_PARTIAL) {
-        trace_pre(st, "router_partial");
-        MOE_TRY(launched(launch_router_partial(x, P.bf16, Wr, z3, (int)P.T, P.d, P.E, st),
-                         "router_partial"));
-        trace_mark(st, "router_partial");
-        r.src = z3;
-        r.nsplit = P.router_splits;
-        r.split_stride = P.T * (int64_t)P.E;
+    if (P.router_kind == ROUTER_ROWS) {
+        trace_pre(st, "router_rows");
+        MOE_TRY(launched(launch_router_rows(x, P.bf16, Wr, z, (int)P.T, P.d, P.E, st),
+                         "router_rows"));
+        trace_mark(st, "router_rows");
     } else if (P.router_kind == ROUTER_TC) {
         void* Ws = at<void>(ws, P.off_wsplit);
         trace_pre(st, "router_split");
@@ -693,23 +687,23 @@ int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const voi
     const int n = which == 0 ? P.E : P.S;
     const int hid = which == 0 ? P.h : P.hs;
     const int64_t d = P.d;
-    for (int e = 0; e < n; ++e) {
-        const uint8_t* s1 = reinterpret_cast<const uint8_t*>(w1) + (size_t)e * d * hid * eb;
-        const uint8_t* s3 = reinterpret_cast<const uint8_t*>(w3) + (size_t)e * d * hid * eb;
-        const uint8_t* s2 = reinterpret_cast<const uint8_t*>(w2) + (size_t)e * hid * d * eb;
-        if (which == 0) {
-            uint8_t* d13 = reinterpret_cast<uint8_t*>(W13) + (size_t)e * 2 * hid * d * eb;
-            uint8_t* d2 = reinterpret_cast<uint8_t*>(W2p) + (size_t)e * d * hid * eb;
-            MOE_TRY(launched(launch_pack(s1, d13, eb, (int)d, hid, d, 0, 0, st), "pack"));
-            MOE_TRY(launched(launch_pack(s3, d13, eb, (int)d, hid, d, 0, 1, st), "pack"));
-            MOE_TRY(launched(launch_pack(s2, d2, eb, hid, (int)d, hid, 0, -1, st), "pack"));
-        } else {
-            // shared experts fused into one of width S*hs: hidden index e*hs + j
-            MOE_TRY(launched(launch_pack(s1, W13, eb, (int)d, hid, d, e * hid, 0, st), "pack"));
-            MOE_TRY(launched(launch_pack(s3, W13, eb, (int)d, hid, d, e * hid, 1, st), "pack"));
-            uint8_t* d2 = reinterpret_cast<uint8_t*>(W2p) + (size_t)e * hid * eb;
-            MOE_TRY(launched(launch_pack(s2, d2, eb, hid, (int)d, P.hsum, 0, -1, st), "pack"));
-        }
+    const int64_t m13 = d * hid;  // elements of one w1 / w3 / w2 matrix
+    if (which == 0) {
+        // expert e: W13[e] [2h][d] and W2p[e] [d][h]
+        MOE_TRY(launched(launch_pack(w1, W13, eb, (int)d, hid, d, 0, 0, n, m13, 2 * m13, 0, st),
+                         "pack"));
+        MOE_TRY(launched(launch_pack(w3, W13, eb, (int)d, hid, d, 0, 1, n, m13, 2 * m13, 0, st),
+                         "pack"));
+        MOE_TRY(launched(launch_pack(w2, W2p, eb, hid, (int)d, hid, 0, -1, n, m13, m13, 0, st),
+                         "pack"));
+    } else {
+        // shared experts fused into one of width S*hs: hidden index e*hs + j
+        MOE_TRY(launched(launch_pack(w1, W13, eb, (int)d, hid, d, 0, 0, n, m13, 0, hid, st),
+                         "pack"));
+        MOE_TRY(launched(launch_pack(w3, W13, eb, (int)d, hid, d, 0, 1, n, m13, 0, hid, st),
+                         "pack"));
+        MOE_TRY(launched(launch_pack(w2, W2p, eb, hid, (int)d, P.hsum, 0, -1, n, m13, hid, 0, st),
+                         "pack"));
     }
     return ok();
 }

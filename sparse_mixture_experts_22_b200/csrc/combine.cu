@@ -145,8 +145,12 @@ __global__ void stats_finalize_kernel(const double* __restrict__ sums, int E, in
 // hidden index j = c + col_off -> row 256 * (j / 128) + 128 * interleave + j % 128.
 template <typename Tv>
 __global__ void pack_kernel(const Tv* __restrict__ src, Tv* __restrict__ dst, int R, int Cc,
-                            int64_t ld_dst, int col_off, int interleave) {
+                            int64_t ld_dst, int col_off, int interleave, int64_t src_stride,
+                            int64_t dst_stride, int col_step) {
     __shared__ Tv tile[32][33];
+    src += blockIdx.z * src_stride;
+    dst += blockIdx.z * dst_stride;
+    col_off += blockIdx.z * col_step;
     const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int r = r0 + i, c = c0 + threadIdx.x;
@@ -195,16 +199,17 @@ int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStr
 }
 
 int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64_t ld_dst,
-                int col_off, int interleave, cudaStream_t st) {
-    dim3 grid((Cc + 31) / 32, (R + 31) / 32), block(32, 8);
+                int col_off, int interleave, int n, int64_t src_stride, int64_t dst_stride,
+                int col_step, cudaStream_t st) {
+    dim3 grid((Cc + 31) / 32, (R + 31) / 32, n), block(32, 8);
     if (elem_bytes == 2)
-        pack_kernel<uint16_t><<<grid, block, 0, st>>>(reinterpret_cast<const uint16_t*>(src),
-                                                      reinterpret_cast<uint16_t*>(dst), R, Cc,
-                                                      ld_dst, col_off, interleave);
+        pack_kernel<uint16_t><<<grid, block, 0, st>>>(
+            reinterpret_cast<const uint16_t*>(src), reinterpret_cast<uint16_t*>(dst), R, Cc,
+            ld_dst, col_off, interleave, src_stride, dst_stride, col_step);
     else
-        pack_kernel<float><<<grid, block, 0, st>>>(reinterpret_cast<const float*>(src),
-                                                   reinterpret_cast<float*>(dst), R, Cc, ld_dst,
-                                                   col_off, interleave);
+        pack_kernel<float><<<grid, block, 0, st>>>(
+            reinterpret_cast<const float*>(src), reinterpret_cast<float*>(dst), R, Cc, ld_dst,
+            col_off, interleave, src_stride, dst_stride, col_step);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

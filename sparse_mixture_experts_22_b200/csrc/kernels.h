@@ -12,9 +12,9 @@ namespace moe {
 // logits z[T][E] = x[T][d] Wr[d][E] on the CUDA cores (fp32 accumulate, no bias)
 int launch_router_logits(const void* x, bool x_bf16, const float* Wr, float* z, int64_t T, int d,
                          int E, int num_sms, cudaStream_t st);
-// T <= 256: partial logits zp[ceil(d/256)][T][E] (256-wide chunks of d, fp32)
-int launch_router_partial(const void* x, bool x_bf16, const float* Wr, float* zp, int T, int d,
-                          int E, cudaStream_t st);
+// small batches: z[T][E] = x W_r (no bias), one CTA per (token, 8 experts)
+int launch_router_rows(const void* x, bool x_bf16, const float* Wr, float* z, int T, int d,
+                       int E, cudaStream_t st);
 // W_r [d][E] fp32 -> three bf16 parts, K-major: Ws[p*E + e][d]
 int launch_router_split(const float* Wr, void* Ws, int d, int E, cudaStream_t st);
 // z[t][e] = bias[e] + sum_s sum_p src[s*split_stride + t*row_stride + p*E + e]
@@ -123,7 +123,10 @@ int launch_stats(const StatsParams& a, cudaStream_t st);
 int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStream_t st);
 // dst[remap(c)][r + row_off] = src[r][c] for a [R][Cc] source; remap interleaves
 // 128-wide hidden blocks (gate/up) when `interleave` >= 0 (0 = gate, 1 = up).
+// n independent matrices: src + i * src_stride -> dst + i * dst_stride, and the
+// hidden column offset grows by col_step per matrix (fused shared experts)
 int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64_t ld_dst,
-                int col_off, int interleave, cudaStream_t st);
+                int col_off, int interleave, int n, int64_t src_stride, int64_t dst_stride,
+                int col_step, cudaStream_t st);
 
 }  // namespace moe

@@ -19,7 +19,7 @@ enum FfnPath : int {
 
 // How the router logits are computed.
 enum RouterKind : int {
-    ROUTER_PARTIAL = 0,  // T <= 256: split-d partial dot products on the CUDA cores
+    ROUTER_ROWS = 0,     // T <= 256: one CTA per token on the CUDA cores (fp32)
     ROUTER_TC = 1,       // bf16, T > 256: tensor-core GEMM against 3 bf16 parts of W_r
     ROUTER_SIMT = 2,     // fp32, T > 256: fp32 dot products on the CUDA cores
 };
@@ -48,7 +48,7 @@ struct Plan {
     int router_npad;    // tensor cores: padded GEMM width of the 3 bf16 parts of W_r
     int router_bn;      // tensor cores: tile width of the router GEMM
     int router_ld;      // tensor cores: row length of the partial logits (3E rounded to 4)
-    int router_splits;  // tensor cores: split-K; partial: number of d chunks
+    int router_splits;  // tensor cores: split-K
 
     // workspace byte offsets
     size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_offsets, off_perm,

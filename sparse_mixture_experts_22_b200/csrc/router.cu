@@ -12,7 +12,7 @@
 // every 256 elements with 16-byte (fp32) or 8-byte (bf16) loads.  The work is
 // HBM-bound for E = 8 (x is read once) and FP32-pipe bound for E = 160.
 //
-// Small batches (<= 256 tokens) use split-d partial dot products instead, and
+// Small batches (<= 256 tokens) use one CTA per token instead, and
 // bf16 batches above that a tensor-core GEMM against W_r split into three
 // bf16 parts; the partial sums are added in a fixed order (router_reduce, or
 // inside the top-k kernel).  Top-k and gates live in routing.cu.
@@ -166,11 +166,14 @@ int launch_logits_dispatch(const XT* x, const float* Wr, float* z, int64_t T, in
 // ---------------------------------------------------------------- small batches
 //
 // With at most 256 tokens the router is a latency problem, not a bandwidth
-// one: the d dimension is cut into 256-wide chunks and every (chunk, 8-expert
-// group) pair is its own CTA, so W_r and x are read by ~d/256 CTAs at once.  Thread t owns token t; the chunk of W_r sits in shared memory and
-// is read as a broadcast.  Each CTA writes its partial logits
-// zp[chunk][t][e]; topk adds the chunks in fixed order.
-constexpr int RP_DC = 256;
+// one.  One CTA per (token, group of 8 experts): its 256 threads split the d
+// dimension (8 contiguous elements per thread per 2048-wide slab), multiply
+// by the matching rows of W_r, and a fixed-order block reduction (warp
+// shuffles, then the 8 warp sums in order) gives the token's 8 logits.  Every
+// CTA issues all of its loads at once, so the whole router takes about two
+// memory latencies.
+constexpr int RR_THREADS = 256;
+constexpr int RR_SLAB = RR_THREADS * 8;
 
 template <typename XT>
 __device__ __forceinline__ void load8(const XT* p, float* v);
@@ -195,38 +198,52 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
 }
 
 template <typename XT>
-__global__ void __launch_bounds__(256)
-    router_partial_kernel(const XT* __restrict__ x, const float* __restrict__ Wr,
-                          float* __restrict__ zp, int T, int d, int E) {
-    __shared__ float ws[RP_DC][RT_EXP];
-    const int c0 = blockIdx.x * RP_DC;
+__global__ void __launch_bounds__(RR_THREADS)
+    router_rows_kernel(const XT* __restrict__ x, const float* __restrict__ Wr,
+                       float* __restrict__ z, int d, int E) {
+    __shared__ float red[RR_THREADS / 32][RT_EXP];
+    const int t = blockIdx.x;
     const int e0 = blockIdx.y * RT_EXP;
     const int ne = min(RT_EXP, E - e0);
-    const int len = min(RP_DC, d - c0);
-    for (int i = threadIdx.x; i < RP_DC * RT_EXP; i += blockDim.x) {
-        const int c = i / RT_EXP, e = i % RT_EXP;
-        ws[c][e] = (c < len && e < ne) ? Wr[(int64_t)(c0 + c) * E + e0 + e] : 0.f;
-    }
-    __syncthreads();
-    const int t = threadIdx.x;
-    if (t >= T) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float acc[RT_EXP];
 #pragma unroll
     for (int e = 0; e < RT_EXP; ++e) acc[e] = 0.f;
-    const XT* xr = x + (int64_t)t * d + c0;
-#pragma unroll 2
-    for (int c = 0; c < len; c += 8) {
+    const bool full8 = ne == RT_EXP && (E % 4) == 0;
+    for (int c0 = 8 * tid; c0 < d; c0 += RR_SLAB) {
         float xv[8];
-        load8<XT>(xr + c, xv);
+        load8<XT>(x + (int64_t)t * d + c0, xv);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 8; ++j) {
+            const float* wrow = Wr + (int64_t)(c0 + j) * E + e0;
+            float w[RT_EXP];
+            if (full8) {
+                const float4 a = *reinterpret_cast<const float4*>(wrow);
+                const float4 b = *reinterpret_cast<const float4*>(wrow + 4);
+                w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+                w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+            } else {
 #pragma unroll
-            for (int e = 0; e < RT_EXP; ++e) acc[e] = fmaf(xv[j], ws[c + j][e], acc[e]);
+                for (int e = 0; e < RT_EXP; ++e) w[e] = e < ne ? wrow[e] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < RT_EXP; ++e) acc[e] = fmaf(xv[j], w[e], acc[e]);
+        }
     }
-    float* out = zp + ((int64_t)blockIdx.x * T + t) * E + e0;
 #pragma unroll
-    for (int e = 0; e < RT_EXP; ++e)
-        if (e < ne) out[e] = acc[e];
+    for (int e = 0; e < RT_EXP; ++e) {
+        float v = acc[e];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp][e] = v;
+    }
+    __syncthreads();
+    if (tid < ne) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < RR_THREADS / 32; ++w) v += red[w][tid];
+        z[(int64_t)t * E + e0 + tid] = v;
+    }
 }
 
 // ---------------------------------------------------------------- router on the tensor cores
@@ -287,17 +304,16 @@ int launch_router_logits(const void* x, bool x_bf16, const float* Wr, float* z, 
     return launch_logits_dispatch(reinterpret_cast<const float*>(x), Wr, z, T, d, E, num_sms, st);
 }
 
-int launch_router_partial(const void* x, bool x_bf16, const float* Wr, float* zp, int T, int d,
-                          int E, cudaStream_t st) {
+int launch_router_rows(const void* x, bool x_bf16, const float* Wr, float* z, int T, int d,
+                       int E, cudaStream_t st) {
     if (T == 0) return 0;
-    if (T > 256) return -1;
-    dim3 grid((d + RP_DC - 1) / RP_DC, (E + RT_EXP - 1) / RT_EXP);
+    dim3 grid(T, (E + RT_EXP - 1) / RT_EXP);
     if (x_bf16)
-        router_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(x), Wr, zp, T, d, E);
+        router_rows_kernel<__nv_bfloat16><<<grid, RR_THREADS, 0, st>>>(
+            reinterpret_cast<const __nv_bfloat16*>(x), Wr, z, d, E);
     else
-        router_partial_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(x), Wr,
-                                                           zp, T, d, E);
+        router_rows_kernel<float><<<grid, RR_THREADS, 0, st>>>(reinterpret_cast<const float*>(x),
+                                                               Wr, z, d, E);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

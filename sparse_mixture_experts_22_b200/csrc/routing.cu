@@ -431,10 +431,12 @@ DispatchArgs dispatch_args(const DispatchParams& p) {
     return a;
 }
 
-// CTAs per token block for the row copies: about two per SM in total
-int copy_splits(int nblk, int k, int num_sms) {
+// CTAs per token block for the row copies: about two per SM in total, and no
+// more than the block has rows
+int copy_splits(int nblk, int64_t T, int k, int num_sms) {
     int ny = (2 * num_sms + nblk - 1) / nblk;
-    if (ny > ROUTE_BLOCK * k) ny = ROUTE_BLOCK * k;
+    const int64_t rows = (T < ROUTE_BLOCK ? T : ROUTE_BLOCK) * (int64_t)k;
+    if (ny > rows) ny = (int)rows;
     return ny < 1 ? 1 : ny;
 }
 
@@ -455,7 +457,7 @@ int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, const int3
     const int nblk = (int)((p.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
     const size_t smem = dispatch_smem_bytes(p.E, p.k);
     if (set_smem(dispatch_kernel, smem)) return -1;
-    dim3 grid(nblk, copy_splits(nblk, p.k, num_sms));
+    dim3 grid(nblk, copy_splits(nblk, p.T, p.k, num_sms));
     dispatch_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(dispatch_args(p), topk_idx, cnt);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -466,7 +468,7 @@ int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num
     if (r.T > ROUTE_BLOCK) return -1;
     const size_t smem = topk_smem_bytes(r.E) + dispatch_smem_bytes(p.E, p.k);
     if (set_smem(route_dispatch_kernel, smem)) return -1;
-    route_dispatch_kernel<<<copy_splits(1, p.k, num_sms), ROUTE_BLOCK, smem, st>>>(
+    route_dispatch_kernel<<<copy_splits(1, p.T, p.k, num_sms), ROUTE_BLOCK, smem, st>>>(
         topk_args(r), dispatch_args(p), r.cnt);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
