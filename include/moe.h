@@ -215,6 +215,30 @@ MOE_API int moe_forward(const moe_config* cfg, const void* x, const float* Wr, c
                 int32_t* kept, int32_t* slot_of, moe_stats* stats, void* ws, size_t ws_bytes,
                 void* stream);
 
+/* ---- routing without a workspace ----------------------------------------- */
+
+/* The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: code running inside a framework whose
+ * allocator they do not control, a plugin handed only its input and output
+ * buffers, or a process that must not grow its device footprint after it
+ * starts.  moe_route_static computes exactly what moe_route computes (same
+ * kernels, same results: topk_idx [T][k] int32 and topk_gate [T][k] fp32) but
+ * takes no workspace and allocates nothing.  Its scratch (the logits and the
+ * statistics partials) is a file-scope device array of
+ * MOE_ROUTE_STATIC_SCRATCH bytes inside the library, held by every GPU that
+ * loads the library until the process exits.  Limits: T <= MOE_ROUTE_STATIC_MAX_T
+ * and T * E <= MOE_ROUTE_STATIC_MAX_TE, else MOE_ERR_SHAPE.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and should
+ * come before any stream capture.  All calls share the array and each call
+ * overwrites what the last one left; calls that overlap on the GPU race, so
+ * the caller must serialise them (one stream, or events between streams). */
+#define MOE_ROUTE_STATIC_SCRATCH (512u * 1024u)
+#define MOE_ROUTE_STATIC_MAX_T 256
+#define MOE_ROUTE_STATIC_MAX_TE 65536
+MOE_API int moe_route_static(const moe_config* cfg, const void* x, const float* Wr,
+                             const float* bias, int32_t* topk_idx, float* topk_gate,
+                             void* stream);
+
 /* ---- status, tracing, limits ------------------------------------------- */
 
 /* Copies the device status word from ws to *status (MOE_OK or

@@ -39,6 +39,13 @@ static int ok() {
     return MOE_OK;
 }
 
+// Records `text` as this thread's last error (cleared for MOE_OK); returns code.
+int report_error(int code, const char* text) {
+    if (code == MOE_OK) g_err.clear();
+    else g_err = text;
+    return code;
+}
+
 #define MOE_TRY(expr)                   \
     do {                                \
         int _s = (expr);                \
