@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sparse_mixture_experts_22_b200 import binding as B  # noqa: E402
+from sparse_mixture_experts_22_b200 import dp  # noqa: E402
 from sparse_mixture_experts_22_b200 import inputs as I  # noqa: E402
 from sparse_mixture_experts_22_b200.workloads import WORKLOADS  # noqa: E402
 
@@ -194,7 +195,7 @@ def build_inputs(wl, rank, world, dev, keep_host):
     """Per-rank tokens; expert weights drawn on rank 0 and broadcast."""
     Wr = I.router_weights(wl)
     bias = I.router_bias(wl)
-    x, _ = I.tokens(wl, Wr=Wr, b=bias, stream="x" if rank == 0 else f"x.rank{rank}")
+    x, _ = I.tokens(wl, Wr=Wr, b=bias, stream=dp.token_stream(rank))
     cfg = B.config_of(wl)
     host = {"x": x, "Wr": Wr, "bias": bias}
     dt = I.torch_dtype(wl.dtype)
@@ -222,10 +223,7 @@ def build_inputs(wl, rank, world, dev, keep_host):
             W13s = torch.empty((2 * hs, wl.d), dtype=dt, device=dev)
             W2s = torch.empty((wl.d, hs), dtype=dt, device=dev)
     if world > 1:
-        import torch.distributed as dist
-        for t in (W13, W2p, W13s, W2s):
-            if t is not None:
-                dist.broadcast(t, src=0)
+        dp.broadcast_weights([W13, W2p, W13s, W2s], src=0)
     torch.cuda.synchronize()
     dev_in = {"x": x.to(dev), "Wr": Wr.to(dev), "bias": bias.to(dev) if bias is not None else None}
     return cfg, host, dev_in, (W13, W2p, W13s, W2s)
@@ -249,7 +247,7 @@ def time_oracle(wl, host, budget_s):
     t_row = max(time.perf_counter() - t0, 1e-4)
     rows_per_pass = max(1, min(wl.T, int(budget_s / (t_row + t_route / max(wl.T, 1)))))
     done, elapsed, passes = 0, 0.0, 0
-    while elapsed < budget_s * 0.5 or passes == 0:
+    while elapsed < budget_s or passes == 0:
         t0 = time.perf_counter()
         r = O.route(cfg, host["x"], host["Wr"], host["bias"])
         O.layer_rows(cfg, host["x"], r["idx"], r["gate"], r["keep"], host["w1"], host["w3"],
@@ -345,7 +343,7 @@ def main():
     cfg, host, g, W = build_inputs(wl, rank, world, dev, keep_host=want_cpu)
     W13, W2p, W13s, W2s = W
     bufs = B.alloc_layer(cfg, dev)
-    sums = torch.zeros(2 + 3 * wl.E, dtype=torch.float64, device=dev)
+    sums = torch.zeros(dp.sums_len(wl.E), dtype=torch.float64, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -357,9 +355,7 @@ def main():
             B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
                           bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
                           bufs["slot_of"], None, bufs["ws"])
-            B.moe_stats_sums(cfg, bufs["routed"], bufs["kept"], bufs["ws"], sums)
-            dist.all_reduce(sums)
-            B.moe_stats_finalize(cfg, sums, bufs["stats"])
+            dp.global_stats(cfg, bufs["routed"], bufs["kept"], bufs["ws"], sums, bufs["stats"])
 
     for _ in range(max(args.warmup, 3)):
         step()
