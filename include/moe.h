@@ -250,6 +250,15 @@ MOE_API int moe_read_device_status(const void* ws, int32_t* status, void* stream
  * the device status word and its kernel returns early.  Process-wide. */
 MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 
+/* Test hook for the time-out path (off by default).  When on, in every expert
+ * FFN GEMM launch the first work unit of CTA 0 withholds its
+ * "accumulator ready" signal, so that CTA's epilogue wait can only run out:
+ * after the wait limit (set a short one with moe_set_wait_limit_ns) the
+ * kernel records MOE_ERR_TIMEOUT, drains its in-flight copies and MMAs,
+ * releases tensor memory and returns.  Results of such a call are garbage;
+ * the device stays usable.  Process-wide. */
+MOE_API int moe_set_test_stall(int on);
+
 /* Per-kernel timing of moe_forward.  moe_trace_begin(n, only) records CUDA
  * events for up to n moe_forward calls: with only == NULL, one event after
  * every kernel launch (each kernel is timed from the end of the previous

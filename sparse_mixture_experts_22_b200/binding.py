@@ -26,7 +26,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_SHAPE", 3: "MOE_ERR_DTYPE",
 EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_splits",
            "moe_last_error", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_aux_stats", "moe_stats_sums", "moe_stats_finalize", "moe_forward",
-           "moe_read_device_status", "moe_set_wait_limit_ns", "moe_trace_begin", "moe_trace_end"]
+           "moe_read_device_status", "moe_set_wait_limit_ns", "moe_set_test_stall",
+           "moe_trace_begin", "moe_trace_end"]
 
 
 class MoEError(RuntimeError):
@@ -82,6 +83,7 @@ def load() -> ctypes.CDLL:
             "moe_forward": [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_read_device_status": [P, P, P],
             "moe_set_wait_limit_ns": [ctypes.c_uint64],
+            "moe_set_test_stall": [I],
             "moe_trace_begin": [I, ctypes.c_char_p],
             "moe_trace_end": [P, P, P, I, P],
         }
@@ -224,6 +226,10 @@ def moe_read_device_status(ws, stream=None) -> int:
 
 def moe_set_wait_limit_ns(ns: int):
     _check(load().moe_set_wait_limit_ns(int(ns)))
+
+
+def moe_set_test_stall(on: bool):
+    _check(load().moe_set_test_stall(1 if on else 0))
 
 
 def moe_trace_begin(max_calls: int, only: Optional[str] = None):

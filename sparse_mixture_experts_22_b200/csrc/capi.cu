@@ -242,6 +242,7 @@ static int tmap_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
 // ---------------------------------------------------------------- limits and tracing
 
 static uint64_t g_wait_limit_ns = 2000000000ull;
+static int g_test_stall = 0;
 
 struct TraceMark {
     cudaEvent_t ev;
@@ -503,6 +504,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.dense_rows = dense_rows;
     a.status = status;
     a.wait_limit_ns = g_wait_limit_ns;
+    a.test_stall = g_test_stall;
     a.nt_max = nt_max;
     const int smem_limit = dv.smem_optin;
 
@@ -904,6 +906,11 @@ int moe_read_device_status(const void* ws, int32_t* status, void* stream) {
 
 int moe_set_wait_limit_ns(uint64_t ns) {
     g_wait_limit_ns = ns;
+    return ok();
+}
+
+int moe_set_test_stall(int on) {
+    g_test_stall = on ? 1 : 0;
     return ok();
 }
 

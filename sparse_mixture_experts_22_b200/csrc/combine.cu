@@ -93,25 +93,32 @@ __global__ void __launch_bounds__(256)
     if (i >= T * vecs) return;
     const int64_t t = i / vecs;
     const int c = (int)(i % vecs) * 8;
+    // all slots and gates first, so that every row load below is independent
+    int32_t slot[MAX_K];
+    float g[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        slot[j] = j < k ? slot_of[t * k + j] : -1;
+        g[j] = j < k ? gate[t * k + j] : 0.f;
+    }
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-        const int32_t slot = slot_of[t * k + j];
-        if (slot < 0) continue;
-        const float g = gate[t * k + j];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        if (slot[j] < 0) continue;
         float v[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) v[q] = 0.f;
         for (int s = 0; s < splits; ++s) {
-            const float* p = y + s * split_stride + (int64_t)slot * d + c;
-            const float4 a = *reinterpret_cast<const float4*>(p);
-            const float4 b = *reinterpret_cast<const float4*>(p + 4);
+            const float* p = y + s * split_stride + (int64_t)slot[j] * d + c;
+            const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+            const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
             v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
             v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = fmaf(g, v[q], acc[q]);
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(g[j], v[q], acc[q]);
     }
     if (ys) {
         const float* p = ys + t * d + c;

@@ -85,6 +85,7 @@ struct TcArgs {
     int64_t split_stride;       // elements between split-K partial outputs
     int32_t* status;            // device status word
     uint64_t wait_limit_ns;
+    int test_stall;             // test hook: CTA 0 withholds its first accumulator-ready signal
 };
 
 int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);

@@ -256,19 +256,27 @@ __global__ void __launch_bounds__(RR_THREADS)
 // 24 bits, so the logits keep fp32 accuracy.  topk sums the parts.
 __global__ void router_split_kernel(const float* __restrict__ Wr, __nv_bfloat16* __restrict__ Ws,
                                     int d, int E) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)d * E) return;
-    const int e = (int)(i % E);
-    const int64_t c = i / E;
-    const float w = Wr[i];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-    Ws[(int64_t)e * d + c] = hi;
-    Ws[(int64_t)(E + e) * d + c] = mid;
-    Ws[(int64_t)(2 * E + e) * d + c] = lo;
+    // 32 x 32 tile of W_r (rows c, columns e) transposed through shared memory
+    __shared__ float tile[32][33];
+    const int c0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, e = e0 + threadIdx.x;
+        tile[i][threadIdx.x] = (c < d && e < E) ? Wr[(int64_t)c * E + e] : 0.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int e = e0 + i, c = c0 + threadIdx.x;
+        if (e >= E || c >= d) continue;
+        const float w = tile[threadIdx.x][i];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+        Ws[(int64_t)e * d + c] = hi;
+        Ws[(int64_t)(E + e) * d + c] = mid;
+        Ws[(int64_t)(2 * E + e) * d + c] = lo;
+    }
 }
 
 // ---------------------------------------------------------------- partial-sum reduction
@@ -285,10 +293,26 @@ __global__ void __launch_bounds__(256)
     const int e = (int)(i % E);
     float v = bias ? bias[e] : 0.f;
     const float* base = src + t * row_stride + e;
-    for (int q = 0; q < nsplit; ++q) {
-        const float* r = base + q * split_stride;
-#pragma unroll 4
-        for (int p = 0; p < nparts; ++p) v += r[p * E];
+    if (nparts == 3) {
+        // all loads first (independent), then the adds in fixed order
+        float part[8][3];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (q < nsplit)
+#pragma unroll
+                for (int p = 0; p < 3; ++p) part[q][p] = base[q * split_stride + p * E];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (q < nsplit)
+#pragma unroll
+                for (int p = 0; p < 3; ++p) v += part[q][p];
+        for (int q = 8; q < nsplit; ++q)
+            for (int p = 0; p < 3; ++p) v += base[q * split_stride + p * E];
+    } else {
+        for (int q = 0; q < nsplit; ++q) {
+            const float* r = base + q * split_stride;
+            for (int p = 0; p < nparts; ++p) v += r[p * E];
+        }
     }
     z[i] = v;
 }
@@ -328,9 +352,8 @@ int launch_router_reduce(const float* src, int nsplit, int64_t split_stride, int
 }
 
 int launch_router_split(const float* Wr, void* Ws, int d, int E, cudaStream_t st) {
-    const int64_t n = (int64_t)d * E;
-    router_split_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        Wr, reinterpret_cast<__nv_bfloat16*>(Ws), d, E);
+    dim3 grid((d + 31) / 32, (E + 31) / 32), block(32, 8);
+    router_split_kernel<<<grid, block, 0, st>>>(Wr, reinterpret_cast<__nv_bfloat16*>(Ws), d, E);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

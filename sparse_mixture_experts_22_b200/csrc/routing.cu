@@ -51,22 +51,31 @@ struct TopkArgs {
     int32_t* status;       // device status word (cleared here: a layer call starts)
 };
 
+constexpr int TK_WARP_E = 32;    // above this many experts one warp routes one token
+constexpr int TK_WARPS = ROUTE_BLOCK / 32;
+
 // Shared memory of topk_block: hist [E] int32, then (E <= TK_SMEM_E) the
-// block's logits [ROUTE_BLOCK][E + 1] fp32.
+// block's logits [ROUTE_BLOCK][E + 1] fp32, then (E > TK_WARP_E) per-warp
+// sums of the full softmax [TK_WARPS][E] fp32.
 __host__ __device__ inline size_t topk_smem_bytes(int E) {
     size_t b = (size_t)E * sizeof(int32_t);
     if (E <= TK_SMEM_E) b += (size_t)ROUTE_BLOCK * (E + 1) * sizeof(float);
+    if (E > TK_WARP_E) b += (size_t)TK_WARPS * E * sizeof(float);
     return b;
 }
+
+__device__ __forceinline__ float finite_or_minus_inf(float v) { return v != v ? -INFINITY : v; }
 
 // Routes the ROUTE_BLOCK tokens of block `blk`.  Leaves the per-expert
 // histogram of the block in hist[] (shared) and the thread's kept experts in
 // my[] (-1 past k or for padding threads).  Global outputs are written only
-// when `write` is set.
+// when `write` is set.  Up to TK_WARP_E experts one thread routes one token;
+// above that one warp routes one token, its lanes splitting the experts.
 __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist, float* zs,
                            int32_t* my) {
     __shared__ float ps[ROUTE_BLOCK][TK_CHUNK + 1];
     __shared__ float hs[ROUTE_BLOCK];
+    __shared__ int32_t sel[ROUTE_BLOCK][MAX_K];
     const int E = a.E, k = a.k;
     const bool in_smem = E <= TK_SMEM_E;
     const int tid = threadIdx.x;
@@ -74,8 +83,10 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
     const int nvalid = (int)(a.T - tb < ROUTE_BLOCK ? a.T - tb : ROUTE_BLOCK);
     const int64_t t = tb + tid;
     const bool valid = tid < nvalid;
+    float* pw = reinterpret_cast<float*>(zs) + (in_smem ? ROUTE_BLOCK * (E + 1) : 0);
 
     for (int e = tid; e < E; e += ROUTE_BLOCK) hist[e] = 0;
+    hs[tid] = 0.f;
 
     // logits of the block, all threads, coalesced; partials added in fixed order
     for (int i = tid; i < nvalid * E; i += ROUTE_BLOCK) {
@@ -97,92 +108,175 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
         if (write && a.logits) a.logits[tt * E + e] = v;
     }
     __syncthreads();
-    const float* zt = in_smem ? zs + tid * (E + 1) : a.zbuf + (valid ? t : 0) * E;
 
-    float val[MAX_K];
-    int id[MAX_K];
+    if (E <= TK_WARP_E) {
+        // ---------------------------------------------- one thread per token
+        const float* zt = in_smem ? zs + tid * (E + 1) : a.zbuf + (valid ? t : 0) * E;
+        float val[MAX_K];
+        int id[MAX_K];
 #pragma unroll
-    for (int j = 0; j < MAX_K; ++j) {
-        val[j] = -INFINITY;
-        id[j] = -1;
-    }
-    if (valid) {
-        for (int e = 0; e < E; ++e) {
-            float v = zt[e];
-            if (v != v) v = -INFINITY;  // a NaN logit ranks last
-            // insert if larger than the current k-th (or a slot is still empty):
-            // from the insertion point on every entry shifts down one place and
-            // the old k-th falls off
-            if (id[k - 1] < 0 || v > val[k - 1]) {
-                float cv = v;
-                int ci = e;
-                bool ins = false;
+        for (int j = 0; j < MAX_K; ++j) {
+            val[j] = -INFINITY;
+            id[j] = -1;
+        }
+        if (valid) {
+            for (int e = 0; e < E; ++e) {
+                const float v = finite_or_minus_inf(zt[e]);  // a NaN logit ranks last
+                // insert if larger than the current k-th (or a slot is still
+                // empty): from the insertion point on every entry shifts down
+                // one place and the old k-th falls off
+                if (id[k - 1] < 0 || v > val[k - 1]) {
+                    float cv = v;
+                    int ci = e;
+                    bool ins = false;
 #pragma unroll
-                for (int q = 0; q < MAX_K; ++q) {
-                    if (q < k && (ins || id[q] < 0 || cv > val[q])) {
-                        const float tv = val[q];
-                        const int ti = id[q];
-                        val[q] = cv;
-                        id[q] = ci;
-                        cv = tv;
-                        ci = ti;
-                        ins = true;
+                    for (int q = 0; q < MAX_K; ++q) {
+                        if (q < k && (ins || id[q] < 0 || cv > val[q])) {
+                            const float tv = val[q];
+                            const int ti = id[q];
+                            val[q] = cv;
+                            id[q] = ci;
+                            cv = tv;
+                            ci = ti;
+                            ins = true;
+                        }
                     }
                 }
             }
         }
-    }
-    const float m = val[0];
-    if (valid) {
-        float s = 0.f;
+        const float m = val[0];
+        if (valid) {
+            float s = 0.f;
 #pragma unroll
-        for (int j = 0; j < MAX_K; ++j)
-            if (j < k) s += __expf(val[j] - m);
-        const float inv = 1.f / s;
+            for (int j = 0; j < MAX_K; ++j)
+                if (j < k) s += __expf(val[j] - m);
+            const float inv = 1.f / s;
 #pragma unroll
-        for (int j = 0; j < MAX_K; ++j)
-            if (j < k) {
-                if (write) {
-                    a.idx[t * k + j] = id[j];
-                    a.gate[t * k + j] = __expf(val[j] - m) * inv;
+            for (int j = 0; j < MAX_K; ++j)
+                if (j < k) {
+                    if (write) {
+                        a.idx[t * k + j] = id[j];
+                        a.gate[t * k + j] = __expf(val[j] - m) * inv;
+                    }
+                    atomicAdd(&hist[id[j]], 1);
                 }
-                atomicAdd(&hist[id[j]], 1);
-            }
-    }
-#pragma unroll
-    for (int j = 0; j < MAX_K; ++j) my[j] = (valid && j < k) ? id[j] : -1;
-
-    // full softmax over E: S = sum exp(z - m); p = exp(z - m) / S;
-    // entropy = ln S - sum p (z - m)
-    float S = 0.f;
-    if (valid)
-        for (int e = 0; e < E; ++e) {
-            const float v = zt[e];
-            S += __expf((v != v ? -INFINITY : v) - m);
         }
-    const float invS = valid ? 1.f / S : 0.f;
-    float pz = 0.f;
-    for (int c0 = 0; c0 < E; c0 += TK_CHUNK) {
-        const int n = min(TK_CHUNK, E - c0);
-        for (int i = 0; i < n; ++i) {
-            float p = 0.f;
-            if (valid) {
-                float v = zt[c0 + i];
-                v = (v != v) ? -INFINITY : v;
-                p = __expf(v - m) * invS;
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) my[j] = (valid && j < k) ? id[j] : -1;
+
+        // full softmax over E: S = sum exp(z - m); p = exp(z - m) / S;
+        // entropy = ln S - sum p (z - m)
+        float S = 0.f;
+        if (valid)
+            for (int e = 0; e < E; ++e) S += __expf(finite_or_minus_inf(zt[e]) - m);
+        const float invS = valid ? 1.f / S : 0.f;
+        float pz = 0.f;
+        for (int c0 = 0; c0 < E; c0 += TK_CHUNK) {
+            const int n = min(TK_CHUNK, E - c0);
+            for (int i = 0; i < n; ++i) {
+                float p = 0.f;
+                if (valid) {
+                    const float v = finite_or_minus_inf(zt[c0 + i]);
+                    p = __expf(v - m) * invS;
+                    if (p > 0.f) pz += p * (v - m);
+                }
+                ps[tid][i] = p;
+            }
+            __syncthreads();
+            if (write && tid < n) {
+                float acc = 0.f;
+                for (int r = 0; r < ROUTE_BLOCK; ++r) acc += ps[r][tid];
+                a.ppart[(int64_t)blk * E + c0 + tid] = acc;
+            }
+            __syncthreads();
+        }
+        hs[tid] = valid ? (__logf(S) - pz) : 0.f;
+    } else {
+        // ---------------------------------------------- one warp per token
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int e = lane; e < E; e += 32) pw[warp * E + e] = 0.f;
+        for (int tl = warp; tl < nvalid; tl += TK_WARPS) {
+            const int64_t tt = tb + tl;
+            const float* zr = in_smem ? zs + tl * (E + 1) : a.zbuf + tt * E;
+            // k rounds of a warp-wide arg-max over the experts not yet taken;
+            // larger value wins, equal values go to the lower index
+            uint32_t taken = 0;  // bit q: expert lane + 32 q is chosen
+            float vsel[MAX_K];
+            int isel[MAX_K];
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j) {
+                vsel[j] = -INFINITY;
+                isel[j] = -1;
+                if (j >= k) continue;
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+                for (int q = 0, e = lane; e < E; ++q, e += 32) {
+                    if ((taken >> q) & 1u) continue;
+                    const float v = finite_or_minus_inf(zr[e]);
+                    if (bi == 0x7fffffff || v > bv) {
+                        bv = v;
+                        bi = e;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                    if (ov > bv || (ov == bv && oi < bi)) {
+                        bv = ov;
+                        bi = oi;
+                    }
+                }
+                vsel[j] = bv;
+                isel[j] = bi;
+                if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            }
+            const float m = vsel[0];
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j)
+                if (j < k) s += __expf(vsel[j] - m);
+            const float inv = 1.f / s;
+            if (lane == 0) {
+#pragma unroll
+                for (int j = 0; j < MAX_K; ++j)
+                    if (j < k) {
+                        if (write) {
+                            a.idx[tt * k + j] = isel[j];
+                            a.gate[tt * k + j] = __expf(vsel[j] - m) * inv;
+                        }
+                        atomicAdd(&hist[isel[j]], 1);
+                        sel[tl][j] = isel[j];
+                    }
+            }
+            // full softmax, each lane over its experts, then a fixed shuffle tree
+            float Sl = 0.f;
+            for (int e = lane; e < E; e += 32) Sl += __expf(finite_or_minus_inf(zr[e]) - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) Sl += __shfl_xor_sync(0xffffffffu, Sl, o);
+            const float invS = 1.f / Sl;
+            float pz = 0.f;
+            for (int e = lane; e < E; e += 32) {
+                const float v = finite_or_minus_inf(zr[e]);
+                const float p = __expf(v - m) * invS;
+                pw[warp * E + e] += p;
                 if (p > 0.f) pz += p * (v - m);
             }
-            ps[tid][i] = p;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) pz += __shfl_xor_sync(0xffffffffu, pz, o);
+            if (lane == 0) hs[tl] = __logf(Sl) - pz;
         }
         __syncthreads();
-        if (write && tid < n) {
-            float acc = 0.f;
-            for (int r = 0; r < ROUTE_BLOCK; ++r) acc += ps[r][tid];
-            a.ppart[(int64_t)blk * E + c0 + tid] = acc;
-        }
-        __syncthreads();
+        if (write)
+            for (int e = tid; e < E; e += ROUTE_BLOCK) {
+                float acc = 0.f;
+#pragma unroll
+                for (int w = 0; w < TK_WARPS; ++w) acc += pw[w * E + e];
+                a.ppart[(int64_t)blk * E + e] = acc;
+            }
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) my[j] = (valid && j < k) ? sel[tid][j] : -1;
     }
-    hs[tid] = valid ? (__logf(S) - pz) : 0.f;
     __syncthreads();
     if (write && tid == 0) {
         float acc = 0.f;
@@ -291,17 +385,31 @@ __device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool wr
     }
     __syncthreads();
 
-    // gather: this CTA copies every nsplit-th (t, j) row of its block
+    // gather: this CTA copies every nsplit-th (t, j) row of its block, eight
+    // rows at a time so that each thread keeps eight loads in flight
     const int nrow = ROUTE_BLOCK * k;
-    for (int r = split; r < nrow; r += nsplit) {
-        const int32_t slot = slots[r];
-        if (slot < 0) continue;
-        const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
-        const uint4* __restrict__ src = a.x + tok * a.row_vecs;
-        uint4* __restrict__ dst = a.x_perm + (int64_t)slot * a.row_vecs;
-        const int nv = a.row_vecs;
-#pragma unroll 4
-        for (int c = tid; c < nv; c += ROUTE_BLOCK) dst[c] = __ldg(src + c);
+    const int nv = a.row_vecs;
+    constexpr int G = 8;
+    for (int r0 = split; r0 < nrow; r0 += G * nsplit) {
+        const uint4* src[G];
+        uint4* dst[G];
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            const int r = r0 + q * nsplit;
+            const int32_t slot = r < nrow ? slots[r] : -1;
+            const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
+            src[q] = slot >= 0 ? a.x + tok * nv : nullptr;
+            dst[q] = slot >= 0 ? a.x_perm + (int64_t)slot * nv : nullptr;
+        }
+        for (int c = tid; c < nv; c += ROUTE_BLOCK) {
+            uint4 v[G];
+#pragma unroll
+            for (int q = 0; q < G; ++q)
+                if (src[q]) v[q] = __ldg(src[q] + c);
+#pragma unroll
+            for (int q = 0; q < G; ++q)
+                if (dst[q]) dst[q][c] = v[q];
+        }
     }
 }
 

@@ -1,8 +1,9 @@
 """Failure detection without a GPU fault: every wait of the tensor-core kernels
-is bounded.  With the bound set to zero the waits run out at once; the kernels
-must record MOE_ERR_TIMEOUT in the device status word, let their in-flight
-copies and MMAs finish, release tensor memory and return, leaving the context
-usable -- the next call with the normal bound gives the normal result."""
+is bounded.  The test hook makes one CTA's epilogue wait on a signal that is
+never sent; with a 5 ms bound the wait runs out, and the kernels must record
+MOE_ERR_TIMEOUT in the device status word, let their in-flight copies and MMAs
+finish, release tensor memory and return, leaving the context usable -- the
+next call with the hook off gives the normal result bit for bit."""
 
 import pytest
 import torch
@@ -14,6 +15,7 @@ from sparse_mixture_experts_22_b200.workloads import Workload
 pytestmark = pytest.mark.gpu
 
 DEFAULT_LIMIT_NS = 2_000_000_000
+SHORT_LIMIT_NS = 5_000_000
 
 
 @pytest.mark.parametrize("wl", [
@@ -27,11 +29,13 @@ def test_wait_bound_reports_timeout_and_context_survives(wl):
     assert B.moe_read_device_status(ref["ws"]) == 0
     out_ref = ref["out"].clone()
 
-    B.moe_set_wait_limit_ns(0)
+    B.moe_set_wait_limit_ns(SHORT_LIMIT_NS)
+    B.moe_set_test_stall(True)
     try:
         bad = run_forward(cfg, g, W)
         status = B.moe_read_device_status(bad["ws"])
     finally:
+        B.moe_set_test_stall(False)
         B.moe_set_wait_limit_ns(DEFAULT_LIMIT_NS)
     assert status == 7  # MOE_ERR_TIMEOUT
 
