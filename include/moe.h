@@ -157,7 +157,7 @@ MOE_API int moe_route(const moe_config* cfg, const void* x, const float* Wr, con
  * ¶3 and ¶5]: per-expert counts, stable rank of every assignment within its
  * expert by token index, truncation at C (overflow dropped), and the gather
  * of kept rows into expert-sorted order.  Needs ws from moe_route (block
- * histograms).
+ * histograms, which this call consumes: run moe_route before each dispatch).
  *   routed [E], kept [E] int32      assignments before / after the limit
  *   offsets [E+1] int32             first row of each expert in x_perm
  *                                   (segments padded for the tensor-core tiles)

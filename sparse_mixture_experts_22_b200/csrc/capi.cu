@@ -152,6 +152,7 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.off_ppart = take((size_t)P.nblk * c.E * 4);
     P.off_hpart = take((size_t)P.nblk * 4);
     P.off_cnt = take((size_t)P.nblk * c.E * 4);
+    P.off_tot = take((size_t)c.E * 4);
     P.off_offsets = take((size_t)(c.E + 1) * 4);
     P.off_perm = take((size_t)P.perm_rows * 4);
     P.off_xperm = take((size_t)P.perm_rows * c.d * P.act_bytes);
@@ -361,10 +362,6 @@ static int step_logits(const Plan& P, const Device& dv, const void* x, const flo
     float* z = at<float>(ws, P.off_logits);
     float* z3 = at<float>(ws, P.off_z3);
     r.src = z;
-    r.nsplit = 1;
-    r.nparts = 1;
-    r.row_stride = P.E;
-    r.split_stride = 0;
     r.bias = bias;
     if (P.router_kind == ROUTER_ROWS) {
         trace_pre(st, "router_rows");
@@ -460,7 +457,8 @@ static int step_dispatch(const Plan& P, const Device& dv, const int32_t* topk_id
     if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st);
     DispatchParams d = dispatch_params(P, x, routed, kept, offsets, perm_token, slot_of, x_perm);
     trace_pre(st, "dispatch");
-    MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt), dv.sms, st),
+    MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
+                                     at<int32_t>(ws, P.off_tot), dv.sms, st),
                      "dispatch"));
     trace_mark(st, "dispatch");
     return MOE_OK;

@@ -24,13 +24,9 @@ int launch_router_reduce(const float* src, int nsplit, int64_t split_stride, int
 
 // ---------------------------------------------------------------- top-k and dispatch
 struct RouteParams {
-    const float* src;       // logit partials (summed as in launch_router_reduce)
-    int nsplit;
-    int64_t split_stride;
-    int row_stride;
-    int nparts;
+    const float* src;       // router logits without bias [T][E]
     const float* bias;      // may be null
-    float* zbuf;            // [T][E] scratch
+    float* zbuf;            // [T][E] scratch (may equal src)
     float* logits;          // optional copy of the logits for the caller
     int64_t T;
     int E, k;
@@ -59,7 +55,9 @@ struct DispatchParams {
 };
 
 int launch_topk(const RouteParams& r, cudaStream_t st);
-int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, const int32_t* cnt,
+// cnt [blocks][E] is turned in place into exclusive prefixes over blocks;
+// tot [E] receives the totals
+int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt, int32_t* tot,
                     int num_sms, cudaStream_t st);
 // T <= 128: top-k and dispatch in one launch
 int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num_sms,

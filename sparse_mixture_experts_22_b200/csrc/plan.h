@@ -51,7 +51,7 @@ struct Plan {
     int router_splits;  // tensor cores: split-K
 
     // workspace byte offsets
-    size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_offsets, off_perm,
+    size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_tot, off_offsets, off_perm,
         off_xperm, off_H, off_y, off_Hs, off_ys, off_sums, total;
 };
 

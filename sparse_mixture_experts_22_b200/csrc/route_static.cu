@@ -104,10 +104,6 @@ extern "C" MOE_API int moe_route_static(const moe_config* cfg, const void* x, co
         return report_error(MOE_ERR_CUDA, "moe_route_static: router launch failed");
     RouteParams r;
     r.src = z;
-    r.nsplit = 1;
-    r.split_stride = 0;
-    r.row_stride = P.E;
-    r.nparts = 1;
     r.bias = cfg->has_bias ? bias : nullptr;
     r.zbuf = z;
     r.logits = nullptr;

@@ -34,13 +34,9 @@ constexpr int TK_SMEM_E = 256;   // up to this many experts a block's logits sit
 constexpr int DWARPS = ROUTE_BLOCK / 32;
 
 struct TopkArgs {
-    const float* src;      // logit partials: z = bias + sum_s sum_p src[s][t][p*E + e]
-    int nsplit;
-    int64_t split_stride;
-    int row_stride;
-    int nparts;
+    const float* src;      // router logits without bias [T][E]
     const float* bias;     // may be null
-    float* zbuf;           // [T][E] scratch for E > TK_SMEM_E
+    float* zbuf;           // [T][E] logits + bias, for E > TK_SMEM_E (may equal src)
     float* logits;         // optional user copy of z [T][E]
     int64_t T;
     int E, k;
@@ -51,26 +47,52 @@ struct TopkArgs {
     int32_t* status;       // device status word (cleared here: a layer call starts)
 };
 
-constexpr int TK_WARP_E = 32;    // above this many experts one warp routes one token
-constexpr int TK_WARPS = ROUTE_BLOCK / 32;
+constexpr int TK_WARP_E = 32;      // above this many experts one warp routes one token
+constexpr int TK_WIDE_THREADS = 512;  // threads of the standalone top-k kernel in that case
 
-// Shared memory of topk_block: hist [E] int32, then (E <= TK_SMEM_E) the
-// block's logits [ROUTE_BLOCK][E + 1] fp32, then (E > TK_WARP_E) per-warp
-// sums of the full softmax [TK_WARPS][E] fp32.
-__host__ __device__ inline size_t topk_smem_bytes(int E) {
+// Shared memory of topk_block for `nthreads` threads: hist [E] int32, then
+// (E <= TK_SMEM_E) the block's logits [ROUTE_BLOCK][E + 1] fp32, then
+// (E > TK_WARP_E) per-warp sums of the full softmax [nthreads/32][E] fp32.
+__host__ __device__ inline size_t topk_smem_bytes(int E, int nthreads) {
     size_t b = (size_t)E * sizeof(int32_t);
     if (E <= TK_SMEM_E) b += (size_t)ROUTE_BLOCK * (E + 1) * sizeof(float);
-    if (E > TK_WARP_E) b += (size_t)TK_WARPS * E * sizeof(float);
+    if (E > TK_WARP_E) b += (size_t)(nthreads / 32) * E * sizeof(float);
     return b;
 }
 
 __device__ __forceinline__ float finite_or_minus_inf(float v) { return v != v ? -INFINITY : v; }
 
-// Routes the ROUTE_BLOCK tokens of block `blk`.  Leaves the per-expert
-// histogram of the block in hist[] (shared) and the thread's kept experts in
-// my[] (-1 past k or for padding threads).  Global outputs are written only
-// when `write` is set.  Up to TK_WARP_E experts one thread routes one token;
-// above that one warp routes one token, its lanes splitting the experts.
+// Inserts (v, e) into a descending list of at most k entries held in
+// registers; a larger value goes first, an equal one after the entries
+// already there (experts arrive in increasing index, so the lower index keeps
+// a tie).  From the insertion point on every entry shifts down one place and
+// the old k-th falls off.
+__device__ __forceinline__ void topk_insert(float* val, int* id, int k, float v, int e) {
+    if (!(id[k - 1] < 0 || v > val[k - 1])) return;
+    float cv = v;
+    int ci = e;
+    bool ins = false;
+#pragma unroll
+    for (int q = 0; q < MAX_K; ++q) {
+        if (q < k && (ins || id[q] < 0 || cv > val[q])) {
+            const float tv = val[q];
+            const int ti = id[q];
+            val[q] = cv;
+            id[q] = ci;
+            cv = tv;
+            ci = ti;
+            ins = true;
+        }
+    }
+}
+
+// Routes the ROUTE_BLOCK tokens of block `blk` with blockDim.x >= ROUTE_BLOCK
+// threads.  Leaves the per-expert histogram of the block in hist[] (shared)
+// and, for threads below ROUTE_BLOCK, the kept experts of token `tid` in my[]
+// (-1 past k or for padding).  Global outputs are written only when `write`
+// is set.  Up to TK_WARP_E experts one thread routes one token; above that one
+// warp routes one token: each lane keeps the top k of its experts, and k
+// rounds of a warp-wide arg-max over the lanes' heads merge them.
 __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist, float* zs,
                            int32_t* my) {
     __shared__ float ps[ROUTE_BLOCK][TK_CHUNK + 1];
@@ -78,40 +100,46 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
     __shared__ int32_t sel[ROUTE_BLOCK][MAX_K];
     const int E = a.E, k = a.k;
     const bool in_smem = E <= TK_SMEM_E;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, NT = blockDim.x;
     const int64_t tb = (int64_t)blk * ROUTE_BLOCK;
     const int nvalid = (int)(a.T - tb < ROUTE_BLOCK ? a.T - tb : ROUTE_BLOCK);
     const int64_t t = tb + tid;
     const bool valid = tid < nvalid;
     float* pw = reinterpret_cast<float*>(zs) + (in_smem ? ROUTE_BLOCK * (E + 1) : 0);
 
-    for (int e = tid; e < E; e += ROUTE_BLOCK) hist[e] = 0;
-    hs[tid] = 0.f;
+    for (int e = tid; e < E; e += NT) hist[e] = 0;
+    if (tid < ROUTE_BLOCK) hs[tid] = 0.f;
 
-    // logits of the block, all threads, coalesced; partials added in fixed order
-    for (int i = tid; i < nvalid * E; i += ROUTE_BLOCK) {
-        const int tl = i / E, e = i % E;
-        const int64_t tt = tb + tl;
-        float v = a.bias ? a.bias[e] : 0.f;
-        const float* base = a.src + tt * a.row_stride + e;
-        if (a.nparts == 1) {
-#pragma unroll 8
-            for (int q = 0; q < a.nsplit; ++q) v += base[q * a.split_stride];
-        } else {
-            for (int q = 0; q < a.nsplit; ++q) {
-                const float* r = base + q * a.split_stride;
-                for (int p = 0; p < a.nparts; ++p) v += r[p * E];
+    // logits of the block (+ bias), all threads, coalesced, eight loads in
+    // flight per thread
+    {
+        const int n = nvalid * E;
+        const float* zsrc = a.src + tb * E;
+        for (int i0 = tid; i0 < n; i0 += 8 * NT) {
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int i = i0 + q * NT;
+                v[q] = i < n ? zsrc[i] : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int i = i0 + q * NT;
+                if (i >= n) break;
+                const int tl = i / E, e = i - tl * E;
+                const float z = a.bias ? v[q] + a.bias[e] : v[q];
+                if (in_smem) zs[tl * (E + 1) + e] = z;
+                else a.zbuf[(tb + tl) * E + e] = z;
+                if (write && a.logits) a.logits[(tb + tl) * E + e] = z;
             }
         }
-        if (in_smem) zs[tl * (E + 1) + e] = v;
-        else a.zbuf[tt * E + e] = v;
-        if (write && a.logits) a.logits[tt * E + e] = v;
     }
     __syncthreads();
 
     if (E <= TK_WARP_E) {
         // ---------------------------------------------- one thread per token
-        const float* zt = in_smem ? zs + tid * (E + 1) : a.zbuf + (valid ? t : 0) * E;
+        const bool mine = tid < ROUTE_BLOCK;
+        const float* zt = in_smem ? zs + (mine ? tid : 0) * (E + 1) : a.zbuf + (valid ? t : 0) * E;
         float val[MAX_K];
         int id[MAX_K];
 #pragma unroll
@@ -119,31 +147,8 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
             val[j] = -INFINITY;
             id[j] = -1;
         }
-        if (valid) {
-            for (int e = 0; e < E; ++e) {
-                const float v = finite_or_minus_inf(zt[e]);  // a NaN logit ranks last
-                // insert if larger than the current k-th (or a slot is still
-                // empty): from the insertion point on every entry shifts down
-                // one place and the old k-th falls off
-                if (id[k - 1] < 0 || v > val[k - 1]) {
-                    float cv = v;
-                    int ci = e;
-                    bool ins = false;
-#pragma unroll
-                    for (int q = 0; q < MAX_K; ++q) {
-                        if (q < k && (ins || id[q] < 0 || cv > val[q])) {
-                            const float tv = val[q];
-                            const int ti = id[q];
-                            val[q] = cv;
-                            id[q] = ci;
-                            cv = tv;
-                            ci = ti;
-                            ins = true;
-                        }
-                    }
-                }
-            }
-        }
+        if (valid)
+            for (int e = 0; e < E; ++e) topk_insert(val, id, k, finite_or_minus_inf(zt[e]), e);
         const float m = val[0];
         if (valid) {
             float s = 0.f;
@@ -173,15 +178,16 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
         float pz = 0.f;
         for (int c0 = 0; c0 < E; c0 += TK_CHUNK) {
             const int n = min(TK_CHUNK, E - c0);
-            for (int i = 0; i < n; ++i) {
-                float p = 0.f;
-                if (valid) {
-                    const float v = finite_or_minus_inf(zt[c0 + i]);
-                    p = __expf(v - m) * invS;
-                    if (p > 0.f) pz += p * (v - m);
+            if (mine)
+                for (int i = 0; i < n; ++i) {
+                    float p = 0.f;
+                    if (valid) {
+                        const float v = finite_or_minus_inf(zt[c0 + i]);
+                        p = __expf(v - m) * invS;
+                        if (p > 0.f) pz += p * (v - m);
+                    }
+                    ps[tid][i] = p;
                 }
-                ps[tid][i] = p;
-            }
             __syncthreads();
             if (write && tid < n) {
                 float acc = 0.f;
@@ -190,17 +196,22 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
             }
             __syncthreads();
         }
-        hs[tid] = valid ? (__logf(S) - pz) : 0.f;
+        if (mine) hs[tid] = valid ? (__logf(S) - pz) : 0.f;
     } else {
         // ---------------------------------------------- one warp per token
-        const int lane = tid & 31, warp = tid >> 5;
+        const int lane = tid & 31, warp = tid >> 5, nw = NT >> 5;
         for (int e = lane; e < E; e += 32) pw[warp * E + e] = 0.f;
-        for (int tl = warp; tl < nvalid; tl += TK_WARPS) {
+        for (int tl = warp; tl < nvalid; tl += nw) {
             const int64_t tt = tb + tl;
             const float* zr = in_smem ? zs + tl * (E + 1) : a.zbuf + tt * E;
-            // k rounds of a warp-wide arg-max over the experts not yet taken;
-            // larger value wins, equal values go to the lower index
-            uint32_t taken = 0;  // bit q: expert lane + 32 q is chosen
+            float lv[MAX_K];
+            int li[MAX_K];
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j) {
+                lv[j] = -INFINITY;
+                li[j] = -1;
+            }
+            for (int e = lane; e < E; e += 32) topk_insert(lv, li, k, finite_or_minus_inf(zr[e]), e);
             float vsel[MAX_K];
             int isel[MAX_K];
 #pragma unroll
@@ -208,16 +219,9 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
                 vsel[j] = -INFINITY;
                 isel[j] = -1;
                 if (j >= k) continue;
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-                for (int q = 0, e = lane; e < E; ++q, e += 32) {
-                    if ((taken >> q) & 1u) continue;
-                    const float v = finite_or_minus_inf(zr[e]);
-                    if (bi == 0x7fffffff || v > bv) {
-                        bv = v;
-                        bi = e;
-                    }
-                }
+                // arg-max of the lanes' heads: larger value, then lower index
+                float bv = lv[0];
+                int bi = li[0] < 0 ? 0x7fffffff : li[0];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -229,7 +233,15 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
                 }
                 vsel[j] = bv;
                 isel[j] = bi;
-                if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+                if (li[0] == bi) {  // the winning lane pops its head
+#pragma unroll
+                    for (int q = 0; q < MAX_K - 1; ++q) {
+                        lv[q] = lv[q + 1];
+                        li[q] = li[q + 1];
+                    }
+                    lv[MAX_K - 1] = -INFINITY;
+                    li[MAX_K - 1] = -1;
+                }
             }
             const float m = vsel[0];
             float s = 0.f;
@@ -268,14 +280,15 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
         }
         __syncthreads();
         if (write)
-            for (int e = tid; e < E; e += ROUTE_BLOCK) {
+            for (int e = tid; e < E; e += NT) {
                 float acc = 0.f;
-#pragma unroll
-                for (int w = 0; w < TK_WARPS; ++w) acc += pw[w * E + e];
+                for (int w = 0; w < nw; ++w) acc += pw[w * E + e];
                 a.ppart[(int64_t)blk * E + e] = acc;
             }
+        if (tid < ROUTE_BLOCK) {
 #pragma unroll
-        for (int j = 0; j < MAX_K; ++j) my[j] = (valid && j < k) ? sel[tid][j] : -1;
+            for (int j = 0; j < MAX_K; ++j) my[j] = (valid && j < k) ? sel[tid][j] : -1;
+        }
     }
     __syncthreads();
     if (write && tid == 0) {
@@ -413,7 +426,7 @@ __device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool wr
     }
 }
 
-__global__ void __launch_bounds__(ROUTE_BLOCK)
+__global__ void __launch_bounds__(TK_WIDE_THREADS)
     topk_kernel(TopkArgs a, int32_t* __restrict__ cnt) {
     extern __shared__ int32_t dyn[];
     int32_t* hist = dyn;
@@ -425,13 +438,37 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     }
     topk_block(a, blockIdx.x, true, hist, zs, my);
     __syncthreads();
-    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK)
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
         cnt[(int64_t)blockIdx.x * a.E + e] = hist[e];
+}
+
+// Per expert e, the exclusive prefix over blocks of the histograms (in place:
+// cnt[b][e] becomes the number of assignments to e in blocks before b) and
+// the total tot[e].  One warp per expert; integer sums, any order is exact.
+__global__ void dispatch_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ tot,
+                                     int nblk, int E) {
+    const int e = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (e >= E) return;
+    int32_t carry = 0;
+    for (int q0 = 0; q0 < nblk; q0 += 32) {
+        const int q = q0 + lane;
+        const int32_t c = q < nblk ? cnt[(int64_t)q * E + e] : 0;
+        int32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (q < nblk) cnt[(int64_t)q * E + e] = carry + incl - c;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) tot[e] = carry;
 }
 
 __global__ void __launch_bounds__(ROUTE_BLOCK)
     dispatch_kernel(DispatchArgs a, const int32_t* __restrict__ topk_idx,
-                    const int32_t* __restrict__ cnt) {
+                    const int32_t* __restrict__ base_in, const int32_t* __restrict__ tot_in) {
     extern __shared__ int32_t sm[];
     int32_t* base = sm;
     int32_t* tot = base + a.E;
@@ -440,14 +477,8 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     int32_t* slots = wcnt + DWARPS * a.E;
     const int blk = blockIdx.x, nblk = gridDim.x;
     for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) {
-        int32_t b = 0, s = 0;
-        for (int q = 0; q < nblk; ++q) {
-            const int32_t c = cnt[(int64_t)q * a.E + e];
-            if (q < blk) b += c;
-            s += c;
-        }
-        base[e] = b;
-        tot[e] = s;
+        base[e] = base_in[(int64_t)blk * a.E + e];
+        tot[e] = tot_in[e];
     }
     const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
     int32_t my[MAX_K];
@@ -467,7 +498,8 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     const int E = ta.E;
     int32_t* hist = dyn;
     float* zs = reinterpret_cast<float*>(dyn + E);
-    int32_t* dsm = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dyn) + topk_smem_bytes(E));
+    int32_t* dsm =
+        reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dyn) + topk_smem_bytes(E, ROUTE_BLOCK));
     int32_t* base = dsm;
     int32_t* tot = base + E;
     int32_t* off = tot + E;
@@ -502,10 +534,6 @@ int set_smem(K kern, size_t bytes) {
 TopkArgs topk_args(const RouteParams& r) {
     TopkArgs a;
     a.src = r.src;
-    a.nsplit = r.nsplit;
-    a.split_stride = r.split_stride;
-    a.row_stride = r.row_stride;
-    a.nparts = r.nparts;
     a.bias = r.bias;
     a.zbuf = r.zbuf;
     a.logits = r.logits;
@@ -553,20 +581,25 @@ int copy_splits(int nblk, int64_t T, int k, int num_sms) {
 int launch_topk(const RouteParams& r, cudaStream_t st) {
     if (r.T == 0) return 0;
     const unsigned blocks = (unsigned)((r.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
-    const size_t smem = topk_smem_bytes(r.E);
+    const int nthreads = r.E > TK_WARP_E ? TK_WIDE_THREADS : ROUTE_BLOCK;
+    const size_t smem = topk_smem_bytes(r.E, nthreads);
     if (set_smem(topk_kernel, smem)) return -1;
-    topk_kernel<<<blocks, ROUTE_BLOCK, smem, st>>>(topk_args(r), r.cnt);
+    topk_kernel<<<blocks, nthreads, smem, st>>>(topk_args(r), r.cnt);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
-int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, const int32_t* cnt,
+int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt, int32_t* tot,
                     int num_sms, cudaStream_t st) {
     if (p.T == 0) return 0;
     const int nblk = (int)((p.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    const int64_t scan_threads = (int64_t)p.E * 32;
+    dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nblk,
+                                                                                p.E);
+    if (cudaGetLastError() != cudaSuccess) return -1;
     const size_t smem = dispatch_smem_bytes(p.E, p.k);
     if (set_smem(dispatch_kernel, smem)) return -1;
     dim3 grid(nblk, copy_splits(nblk, p.T, p.k, num_sms));
-    dispatch_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(dispatch_args(p), topk_idx, cnt);
+    dispatch_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(dispatch_args(p), topk_idx, cnt, tot);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -574,7 +607,7 @@ int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num
                           cudaStream_t st) {
     if (r.T == 0) return 0;
     if (r.T > ROUTE_BLOCK) return -1;
-    const size_t smem = topk_smem_bytes(r.E) + dispatch_smem_bytes(p.E, p.k);
+    const size_t smem = topk_smem_bytes(r.E, ROUTE_BLOCK) + dispatch_smem_bytes(p.E, p.k);
     if (set_smem(route_dispatch_kernel, smem)) return -1;
     route_dispatch_kernel<<<copy_splits(1, p.T, p.k, num_sms), ROUTE_BLOCK, smem, st>>>(
         topk_args(r), dispatch_args(p), r.cnt);
