@@ -242,7 +242,7 @@ def time_oracle(wl, host, budget_s):
     t_route = time.perf_counter() - t0
     # probe one row, then size the sample
     t0 = time.perf_counter()
-    O.layer_rows(cfg, host["x"], r["idx"], r["gate"], r["keep"], host["w1"], host["w3"],
+    O.layer_rows(cfg, host["x"], r["expert"], r["gate"], r["keep"], host["w1"], host["w3"],
                  host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"), [0])
     t_row = max(time.perf_counter() - t0, 1e-4)
     rows_per_pass = max(1, min(wl.T, int(budget_s / (t_row + t_route / max(wl.T, 1)))))
@@ -250,7 +250,7 @@ def time_oracle(wl, host, budget_s):
     while elapsed < budget_s or passes == 0:
         t0 = time.perf_counter()
         r = O.route(cfg, host["x"], host["Wr"], host["bias"])
-        O.layer_rows(cfg, host["x"], r["idx"], r["gate"], r["keep"], host["w1"], host["w3"],
+        O.layer_rows(cfg, host["x"], r["expert"], r["gate"], r["keep"], host["w1"], host["w3"],
                      host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"),
                      np.arange(rows_per_pass))
         elapsed += time.perf_counter() - t0
@@ -282,7 +282,7 @@ def run_reference(args):
     cfg = O.cfg_of(wl)
     # each step: the whole batch routed, and the outputs of a bounded row sample
     t0 = time.perf_counter()
-    O.layer_rows(cfg, x, *(lambda r: (r["idx"], r["gate"], r["keep"]))(
+    O.layer_rows(cfg, x, *(lambda r: (r["expert"], r["gate"], r["keep"]))(
         O.route(cfg, x, Wr, bias)), host["w1"], host["w3"], host["w2"], host.get("w1s"),
         host.get("w3s"), host.get("w2s"), [0])
     t_row = time.perf_counter() - t0
@@ -291,7 +291,7 @@ def run_reference(args):
 
     def step():
         r = O.route(cfg, x, Wr, bias)
-        O.layer_rows(cfg, x, r["idx"], r["gate"], r["keep"], host["w1"], host["w3"], host["w2"],
+        O.layer_rows(cfg, x, r["expert"], r["gate"], r["keep"], host["w1"], host["w3"], host["w2"],
                      host.get("w1s"), host.get("w3s"), host.get("w2s"), sample_rows)
 
     for _ in range(args.warmup):

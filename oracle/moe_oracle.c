@@ -36,7 +36,11 @@ typedef struct {
     int64_t cf_num, cf_den; /* capacity factor as a fraction; cf_den == 0 means no limit */
     int32_t dtype;       /* ORACLE_F32 or ORACLE_BF16 for x and expert weights */
     int32_t has_bias;    /* router bias present */
+    int32_t overflow;    /* ORACLE_DROP or ORACLE_REROUTE */
 } oracle_cfg;
+
+#define ORACLE_DROP 0
+#define ORACLE_REROUTE 1
 
 /* Widen element i of a bf16 or fp32 array to double.  bf16 is the top half of
  * an IEEE binary32, so the widening is exact. */
@@ -152,6 +156,42 @@ void oracle_dispatch(const oracle_cfg* c, const int32_t* idx, int64_t C,
     for (int e = 0; e < E; ++e) kept[e] = routed[e] < C ? routed[e] : (int32_t)C;
 }
 
+/* Overflow rerouted to a spare expert [Routing explained, "Easy explanation"
+ * ¶3: the second of the three ways to treat tokens beyond an expert's
+ * capacity].  Reading: after the arrival-order pass of oracle_dispatch, the
+ * dropped assignments are visited in token order (t, then j); each moves to
+ * the token's highest-scoring expert (ties: lower index) that the token does
+ * not already use and that still has room, keeping its gate, and joins the end
+ * of that expert's queue.  With no room anywhere it stays dropped.
+ *   z[t][e]      router logits (bias included)
+ *   kept[e]      in: min(routed, C); out: rows each expert serves
+ *   rank, keep   in/out: updated for rerouted assignments
+ *   expert[t][j] out: the expert serving assignment (t, j) */
+void oracle_reroute(const oracle_cfg* c, const double* z, const int32_t* idx, int64_t C,
+                    int32_t* kept, int32_t* rank, int8_t* keep, int32_t* expert) {
+    const int64_t T = c->T;
+    const int E = c->E, k = c->k;
+    for (int64_t i = 0; i < T * k; ++i) expert[i] = idx[i];
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            if (keep[t * k + j]) continue;
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (kept[e] >= C) continue;
+                int used = 0;
+                for (int q = 0; q < k; ++q)
+                    used |= (idx[t * k + q] == e) || (expert[t * k + q] == e);
+                if (used) continue;
+                if (best < 0 || z[t * E + e] > z[t * E + best]) best = e;
+            }
+            if (best < 0) continue;
+            expert[t * k + j] = best;
+            rank[t * k + j] = kept[best]++;
+            keep[t * k + j] = 1;
+        }
+    }
+}
+
 /* Statistics.
  * Load-balancing loss [Routing explained, "Easy explanation" ¶4]: for each
  * expert multiply the share of tokens it actually received by the total
@@ -231,15 +271,17 @@ void oracle_ffn(int d, int h, int dtype, const void* x_row, const void* w1, cons
 
 /* Layer output for selected tokens [Mixtral explained, "Easy explanation" ¶3;
  * MoE wiki, "How it works"; Routing explained, "Easy explanation" ¶4]:
- *   out[t] = sum over kept j of gate[t][j] * FFN_{idx[t][j]}(x_t)
- *          + sum over shared experts s of FFN^shared_s(x_t).
+ *   out[t] = sum over kept j of gate[t][j] * FFN_{expert[t][j]}(x_t)
+ *          + sum over shared experts s of FFN^shared_s(x_t),
+ * expert[t][j] being the router's choice idx[t][j], or the spare expert that
+ * serves the assignment under the reroute policy.
  * A dropped assignment simply contributes nothing; the remaining gates are
  * not renormalised (the pages are silent; this is the reading taken).
  * Unselected experts are not evaluated at all.
  * rows[n_rows] lists the tokens to evaluate (NULL = all T); out is
  * [n_rows][d].  w1/w3 are [E][d][h], w2 [E][h][d]; the shared ones are
  * [S][d][hs] and [S][hs][d] (may be NULL when n_shared == 0). */
-void oracle_layer_rows(const oracle_cfg* c, const void* x, const int32_t* idx,
+void oracle_layer_rows(const oracle_cfg* c, const void* x, const int32_t* expert,
                        const double* gate, const int8_t* keep, const void* w1,
                        const void* w3, const void* w2, const void* w1s, const void* w3s,
                        const void* w2s, const int64_t* rows, int64_t n_rows, double* out) {
@@ -258,7 +300,7 @@ void oracle_layer_rows(const oracle_cfg* c, const void* x, const int32_t* idx,
             for (int o = 0; o < d; ++o) acc[o] = 0.0;
             for (int j = 0; j < k; ++j) {
                 if (!keep[t * k + j]) continue;
-                const int64_t e = idx[t * k + j];
+                const int64_t e = expert[t * k + j];
                 ffn(d, h, c->dtype, x, t * d, w1, w3, w2, e * d * h, e * h * d, y, a, b);
                 for (int o = 0; o < d; ++o) acc[o] += gate[t * k + j] * y[o];
             }

@@ -32,6 +32,7 @@ class OracleCfg(ctypes.Structure):
         ("cf_den", ctypes.c_int64),
         ("dtype", ctypes.c_int32),
         ("has_bias", ctypes.c_int32),
+        ("overflow", ctypes.c_int32),
     ]
 
 
@@ -49,6 +50,7 @@ def _bind(path: str):
     L.oracle_probs.argtypes = [C, P, P]
     L.oracle_dispatch.argtypes = [C, P, ctypes.c_int64, P, P, P, P]
     L.oracle_stats.argtypes = [C, P, P, P, P]
+    L.oracle_reroute.argtypes = [C, P, P, ctypes.c_int64, P, P, P, P]
     L.oracle_ffn.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
     L.oracle_layer_rows.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int64, P]
     L.oracle_threads.restype = ctypes.c_int
@@ -85,16 +87,20 @@ def threads() -> int:
     return lib().oracle_threads()
 
 
+OVERFLOW = {"drop": 0, "reroute": 1}
+
+
 def make_cfg(T, d, h, E, k, n_shared=0, h_shared=0, cf=None, dtype="bf16",
-             has_bias=False) -> OracleCfg:
+             has_bias=False, overflow="drop") -> OracleCfg:
     num, den = (0, 0) if cf is None else cf
     return OracleCfg(T, d, h, E, k, n_shared, h_shared, num, den,
-                     _BF16 if dtype == "bf16" else _F32, 1 if has_bias else 0)
+                     _BF16 if dtype == "bf16" else _F32, 1 if has_bias else 0,
+                     OVERFLOW[overflow])
 
 
 def cfg_of(wl, T: Optional[int] = None) -> OracleCfg:
     return make_cfg(wl.T if T is None else T, wl.d, wl.h, wl.E, wl.k, wl.n_shared,
-                    wl.h_shared, wl.cf, wl.dtype, wl.has_bias)
+                    wl.h_shared, wl.cf, wl.dtype, wl.has_bias, wl.overflow)
 
 
 def _ptr(a):
@@ -141,6 +147,16 @@ def dispatch(cfg: OracleCfg, idx: np.ndarray, C: int):
     return routed, kept, rank, keep
 
 
+def reroute(cfg: OracleCfg, z: np.ndarray, idx: np.ndarray, C: int, kept, rank, keep):
+    """Second pass of the reroute policy (updates kept, rank, keep in place);
+    returns the expert serving each assignment."""
+    expert = np.empty((cfg.T, cfg.k), dtype=np.int32)
+    lib().oracle_reroute(ctypes.byref(cfg), _ptr(np.ascontiguousarray(z)),
+                         _ptr(np.ascontiguousarray(idx, dtype=np.int32)), C, _ptr(kept),
+                         _ptr(rank), _ptr(keep), _ptr(expert))
+    return expert
+
+
 def stats(cfg: OracleCfg, p: np.ndarray, routed: np.ndarray, kept: np.ndarray) -> Dict:
     out = np.empty(3 + cfg.E, dtype=np.float64)
     lib().oracle_stats(ctypes.byref(cfg), _ptr(np.ascontiguousarray(p)), _ptr(routed),
@@ -156,8 +172,10 @@ def ffn(d: int, h: int, dtype: str, x_row, w1, w3, w2) -> np.ndarray:
     return y
 
 
-def layer_rows(cfg: OracleCfg, x, idx, gate, keep, w1, w3, w2, w1s=None, w3s=None,
+def layer_rows(cfg: OracleCfg, x, expert, gate, keep, w1, w3, w2, w1s=None, w3s=None,
                w2s=None, rows=None) -> np.ndarray:
+    """Layer output rows; `expert` is the expert serving each assignment (the
+    router's choice, or the spare expert under the reroute policy)."""
     if rows is None:
         n = cfg.T
         rows_arr = None
@@ -165,7 +183,7 @@ def layer_rows(cfg: OracleCfg, x, idx, gate, keep, w1, w3, w2, w1s=None, w3s=Non
         rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         n = rows_arr.shape[0]
     out = np.empty((n, cfg.d), dtype=np.float64)
-    lib().oracle_layer_rows(ctypes.byref(cfg), _ptr(x), _ptr(idx), _ptr(gate), _ptr(keep),
+    lib().oracle_layer_rows(ctypes.byref(cfg), _ptr(x), _ptr(expert), _ptr(gate), _ptr(keep),
                             _ptr(w1), _ptr(w3), _ptr(w2), _ptr(w1s), _ptr(w3s), _ptr(w2s),
                             _ptr(rows_arr), n, _ptr(out))
     return out
@@ -178,15 +196,19 @@ def route(cfg: OracleCfg, x, Wr, bias=None) -> Dict:
     p = probs(cfg, z)
     C = capacity(cfg)
     routed, kept, rank, keep = dispatch(cfg, idx, C)
+    if cfg.overflow == OVERFLOW["reroute"]:
+        expert = reroute(cfg, z, idx, C, kept, rank, keep)
+    else:
+        expert = idx.copy()
     st = stats(cfg, p, routed, kept)
     return {"z": z, "idx": idx, "gate": gate, "p": p, "C": C, "routed": routed,
-            "kept": kept, "rank": rank, "keep": keep, "stats": st}
+            "kept": kept, "rank": rank, "keep": keep, "expert": expert, "stats": st}
 
 
 def forward(cfg: OracleCfg, inp: Dict, rows=None) -> Dict:
     """The whole layer; out holds the rows listed in `rows` (all tokens if None)."""
     r = route(cfg, inp["x"], inp["Wr"], inp.get("bias"))
-    r["out"] = layer_rows(cfg, inp["x"], r["idx"], r["gate"], r["keep"], inp["w1"],
+    r["out"] = layer_rows(cfg, inp["x"], r["expert"], r["gate"], r["keep"], inp["w1"],
                           inp["w3"], inp["w2"], inp.get("w1s"), inp.get("w3s"),
                           inp.get("w2s"), rows)
     return r

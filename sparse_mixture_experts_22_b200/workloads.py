@@ -27,6 +27,7 @@ class Workload:
     cf: Optional[Tuple[int, int]] = None   # capacity factor num/den; None = no limit
     dtype: str = "bf16"         # "bf16" or "f32" for activations and expert weights
     zipf_s: Optional[float] = None         # router bias b_e = -s*ln(e+1) when set
+    overflow: str = "drop"                 # "drop" or "reroute" (to a spare expert)
     seed: int = 0
 
     @property
@@ -41,6 +42,8 @@ class Workload:
             s += f" shared={self.n_shared}x{self.h_shared}"
         if self.zipf_s is not None:
             s += f" zipf={self.zipf_s}"
+        if self.overflow != "drop":
+            s += f" overflow={self.overflow}"
         return s
 
     def scaled(self, **kw) -> "Workload":

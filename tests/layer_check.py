@@ -115,7 +115,7 @@ def oracle_route(wl: Workload, inp: Dict) -> Dict:
 
 def oracle_rows(wl: Workload, inp: Dict, r: Dict, rows=None) -> np.ndarray:
     cfg = O.cfg_of(wl)
-    return O.layer_rows(cfg, inp["x"], r["idx"], r["gate"], r["keep"], inp["w1"], inp["w3"],
+    return O.layer_rows(cfg, inp["x"], r["expert"], r["gate"], r["keep"], inp["w1"], inp["w3"],
                         inp["w2"], inp.get("w1s"), inp.get("w3s"), inp.get("w2s"), rows)
 
 

@@ -50,6 +50,13 @@ MUTATIONS = [
      [pins.test_aux_is_one_when_assignment_is_uniform]),
     ("overflow counts kept", "dropped += (double)(routed[e] - kept[e]);",
      "dropped += (double)kept[e];", [pins.test_overflow_rate_closed_form]),
+    ("reroute to the worst expert", "if (best < 0 || z[t * E + e] > z[t * E + best]) best = e;",
+     "if (best < 0 || z[t * E + e] < z[t * E + best]) best = e;",
+     [pins.test_reroute_hand_example]),
+    ("reroute ignores capacity", "if (kept[e] >= C) continue;", "",
+     [pins.test_reroute_matches_simulation_and_invariants]),
+    ("reroute may reuse an expert", "if (used) continue;", "",
+     [pins.test_reroute_matches_simulation_and_invariants]),
 ]
 
 
@@ -67,13 +74,17 @@ def _build(tmp_path, name, old, new):
 
 def _run(pin):
     params = getattr(pin, "pytestmark", [])
-    args = []
+    names, args = None, []
     for m in params:
         if m.name == "parametrize":
-            args = list(m.args[1])
+            names, args = m.args[0], list(m.args[1])
     if args:
+        multi = "," in names
         for a in args:
-            pin(a)
+            if multi:
+                pin(*a)
+            else:
+                pin(a)
     else:
         pin()
 

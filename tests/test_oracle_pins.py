@@ -433,3 +433,89 @@ def test_aux_uses_assignments_before_the_capacity_limit():
     b = O.route(cfg_cap, inp["x"], inp["Wr"], inp["bias"])
     assert b["stats"]["overflow_rate"] > 0.2 and a["stats"]["overflow_rate"] == 0.0
     assert a["stats"]["aux_loss"] == b["stats"]["aux_loss"]
+
+
+# ---------------------------------------------------------------- overflow rerouted to a spare expert
+
+def test_reroute_hand_example():
+    # 4 tokens all preferring expert 0 (logits 3, 2, 1), k=1, C=1: token 0 keeps
+    # expert 0, token 1 moves to expert 1, token 2 to expert 2, token 3 finds no room
+    cfg = O.make_cfg(4, 3, 4, 3, 1, cf=(3, 4), has_bias=True, overflow="reroute")
+    r = O.route(cfg, np.zeros((4, 3), np.float32), np.zeros((3, 3), np.float32),
+                f32([3.0, 2.0, 1.0]))
+    assert r["C"] == 1
+    assert r["expert"][:, 0].tolist() == [0, 1, 2, 0]
+    assert r["keep"][:, 0].tolist() == [1, 1, 1, 0]
+    assert r["kept"].tolist() == [1, 1, 1] and r["routed"].tolist() == [4, 0, 0]
+    assert r["stats"]["overflow_rate"] == 0.25
+
+
+def reroute_sim(z, idx, E, C):
+    """Brute-force arrival-order queues, then reroutes in token order."""
+    T, k = idx.shape
+    fill = [0] * E
+    keep = np.zeros(idx.shape, bool)
+    expert = idx.copy()
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            keep[t, j] = fill[e] < C
+            fill[e] += 1
+    fill = [min(f, C) for f in fill]
+    for t in range(T):
+        for j in range(k):
+            if keep[t, j]:
+                continue
+            cands = [e for e in range(E) if fill[e] < C and e not in idx[t] and e not in expert[t]]
+            if not cands:
+                continue
+            best = sorted(cands, key=lambda e: (-z[t, e], e))[0]
+            expert[t, j] = best
+            keep[t, j] = True
+            fill[best] += 1
+    return expert, keep, fill
+
+
+@pytest.mark.parametrize("cf,k", [((1, 2), 2), ((3, 4), 2), ((1, 1), 1), ((5, 4), 3)])
+def test_reroute_matches_simulation_and_invariants(cf, k):
+    T, E = 48, 6
+    cfg, inp = tiny_layer(T=T, E=E, k=k, cf=cf, bias=[2.0, 1.5, 1.0, 0.5, 0.0, -0.5])
+    cfg.overflow = O.OVERFLOW["reroute"]
+    r = O.forward(cfg, inp)
+    expert, keep, fill = reroute_sim(r["z"], r["idx"], E, r["C"])
+    assert np.array_equal(r["expert"], expert)
+    assert np.array_equal(r["keep"].astype(bool), keep)
+    assert r["kept"].tolist() == fill
+    # no expert over capacity; no token uses an expert twice
+    assert max(r["kept"]) <= r["C"]
+    for t in range(T):
+        served = [r["expert"][t, j] for j in range(k) if r["keep"][t, j]]
+        assert len(served) == len(set(served))
+    # an assignment left dropped had no free expert it could use
+    for t in range(T):
+        for j in range(k):
+            if not r["keep"][t, j]:
+                for e in range(E):
+                    if e not in r["idx"][t] and e not in r["expert"][t]:
+                        assert r["kept"][e] == r["C"]
+    # the output sums the serving experts with the original gates
+    Y = [np_ffn(inp["x"], inp["w1"][e], inp["w3"][e], inp["w2"][e]) for e in range(E)]
+    ref = np.zeros((T, cfg.d))
+    for t in range(T):
+        for j in range(k):
+            if r["keep"][t, j]:
+                ref[t] += r["gate"][t, j] * Y[r["expert"][t, j]][t]
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-11, atol=1e-13)
+
+
+def test_reroute_with_enough_room_drops_nothing():
+    # k = 1 and E*C >= T: every overflowing token finds a spare expert
+    cfg_d, inp = tiny_layer(T=40, E=4, k=1, cf=(1, 1), bias=[3.0, 0.0, 0.0, 0.0])
+    cfg_r, _ = tiny_layer(T=40, E=4, k=1, cf=(1, 1), bias=[3.0, 0.0, 0.0, 0.0])
+    cfg_r.overflow = O.OVERFLOW["reroute"]
+    a = O.route(cfg_d, inp["x"], inp["Wr"], inp["bias"])
+    b = O.route(cfg_r, inp["x"], inp["Wr"], inp["bias"])
+    assert a["stats"]["overflow_rate"] > 0.3
+    assert b["stats"]["overflow_rate"] == 0.0 and b["keep"].all()
+    # aux counts the router's own choices, so rerouting leaves it unchanged
+    assert a["stats"]["aux_loss"] == b["stats"]["aux_loss"]
