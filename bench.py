@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--trace-all", action="store_true",
                    help="time every kernel (one event after each launch) instead of only "
                         "the gate/up GEMM")
+    p.add_argument("--overflow", default=None, choices=["drop", "reroute"],
+                   help="capacity overflow policy (default: the workload's, drop)")
     p.add_argument("--hidden", type=int, default=0,
                    help="override the expert hidden width (small profiling cases only)")
     p.add_argument("--graph", action="store_true",
@@ -339,6 +341,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if args.hidden:
         wl = wl.scaled(h=args.hidden, name=f"{wl.name}_h{args.hidden}")
+    if args.overflow:
+        wl = wl.scaled(overflow=args.overflow)
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
     cfg, host, g, W = build_inputs(wl, rank, world, dev, keep_host=want_cpu)
     W13, W2p, W13s, W2s = W

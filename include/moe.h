@@ -63,6 +63,15 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
+/* What happens to assignments beyond an expert's capacity [MoE routing fully
+ * explained, "Easy explanation" ¶3 names three choices]:
+ *   MOE_OVERFLOW_DROP     drop them (fast, loses their contribution)
+ *   MOE_OVERFLOW_REROUTE  move each, in token order, to the token's
+ *                         highest-scoring expert it does not already use that
+ *                         still has room; it keeps its gate (else it drops)
+ * The third choice, processing everything, is cf_den = 0 (no limit). */
+typedef enum { MOE_OVERFLOW_DROP = 0, MOE_OVERFLOW_REROUTE = 1 } moe_overflow;
+
 /* Layer configuration.
  *   T         tokens in the batch (0 allowed: every call is a no-op that
  *             writes zero statistics)
@@ -75,13 +84,15 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  *   h_shared  hidden width of each shared expert, multiple of 128
  *   cf_num / cf_den  capacity factor; cf_den == 0 means no capacity limit
  *   act_dtype MOE_BF16 (tensor-core path) or MOE_F32 (fp32 SIMT path; no TF32)
- *   has_bias  1 if the router has a bias vector b[E]                       */
+ *   has_bias  1 if the router has a bias vector b[E]
+ *   overflow  moe_overflow (0 = drop)                                       */
 typedef struct {
     int64_t T;
     int32_t d, h, E, k, n_shared, h_shared;
     int64_t cf_num, cf_den;
     int32_t act_dtype;
     int32_t has_bias;
+    int32_t overflow;
 } moe_config;
 
 /* Routing statistics [MoE routing fully explained, "Easy explanation" ¶4 and
@@ -158,7 +169,8 @@ MOE_API int moe_route(const moe_config* cfg, const void* x, const float* Wr, con
  * expert by token index, truncation at C (overflow dropped), and the gather
  * of kept rows into expert-sorted order.  Needs ws from moe_route (block
  * histograms, which this call consumes: run moe_route before each dispatch).
- *   routed [E], kept [E] int32      assignments before / after the limit
+ *   routed [E], kept [E] int32      assignments the router made / rows each
+ *                                   expert serves (rerouted rows included)
  *   offsets [E+1] int32             first row of each expert in x_perm
  *                                   (segments padded for the tensor-core tiles)
  *   perm_token [moe_perm_rows] int32  token of each row (-1 in padding)

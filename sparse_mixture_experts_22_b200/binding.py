@@ -49,6 +49,7 @@ class MoEConfig(ctypes.Structure):
         ("cf_den", ctypes.c_int64),
         ("act_dtype", ctypes.c_int32),
         ("has_bias", ctypes.c_int32),
+        ("overflow", ctypes.c_int32),
     ]
 
 
@@ -122,16 +123,20 @@ def _stream(stream) -> ctypes.c_void_p:
 
 # ---------------------------------------------------------------- config
 
+OVERFLOW = {"drop": 0, "reroute": 1}
+
+
 def make_config(T, d, h, E, k, n_shared=0, h_shared=0, cf=None, dtype="bf16",
-                has_bias=False) -> MoEConfig:
+                has_bias=False, overflow="drop") -> MoEConfig:
     num, den = (0, 0) if cf is None else cf
     return MoEConfig(T, d, h, E, k, n_shared, h_shared, num, den,
-                     MOE_BF16 if dtype == "bf16" else MOE_F32, 1 if has_bias else 0)
+                     MOE_BF16 if dtype == "bf16" else MOE_F32, 1 if has_bias else 0,
+                     OVERFLOW[overflow])
 
 
 def config_of(wl: Workload, T: Optional[int] = None) -> MoEConfig:
     return make_config(wl.T if T is None else T, wl.d, wl.h, wl.E, wl.k, wl.n_shared,
-                       wl.h_shared, wl.cf, wl.dtype, wl.has_bias)
+                       wl.h_shared, wl.cf, wl.dtype, wl.has_bias, wl.overflow)
 
 
 def act_dtype(cfg: MoEConfig) -> torch.dtype:

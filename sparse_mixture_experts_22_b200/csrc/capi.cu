@@ -78,12 +78,17 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     }
     if (c.act_dtype != MOE_F32 && c.act_dtype != MOE_BF16) { *why = "act_dtype must be MOE_F32 or MOE_BF16"; return MOE_ERR_DTYPE; }
     if (c.has_bias != 0 && c.has_bias != 1) { *why = "has_bias must be 0 or 1"; return MOE_ERR_ARG; }
+    if (c.overflow != MOE_OVERFLOW_DROP && c.overflow != MOE_OVERFLOW_REROUTE) {
+        *why = "overflow must be MOE_OVERFLOW_DROP or MOE_OVERFLOW_REROUTE";
+        return MOE_ERR_ARG;
+    }
 
     Plan& P = *p;
     P.T = c.T; P.d = c.d; P.h = c.h; P.E = c.E; P.k = c.k; P.S = c.n_shared;
     P.hs = c.n_shared ? c.h_shared : 0;
     P.hsum = P.S * P.hs;
     P.capped = c.cf_den > 0;
+    P.reroute = P.capped && c.overflow == MOE_OVERFLOW_REROUTE;
     if (P.capped) {
         const int64_t num = c.T * (int64_t)c.k * c.cf_num;
         const int64_t den = (int64_t)c.E * c.cf_den;
@@ -153,6 +158,8 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.off_hpart = take((size_t)P.nblk * 4);
     P.off_cnt = take((size_t)P.nblk * c.E * 4);
     P.off_tot = take((size_t)c.E * 4);
+    P.off_expert = take(P.reroute ? (size_t)c.T * c.k * 4 : 0);
+    P.off_rank = take(P.reroute ? (size_t)c.T * c.k * 4 : 0);
     P.off_offsets = take((size_t)(c.E + 1) * 4);
     P.off_perm = take((size_t)P.perm_rows * 4);
     P.off_xperm = take((size_t)P.perm_rows * c.d * P.act_bytes);
@@ -445,9 +452,15 @@ static int step_route(const Plan& P, const Device& dv, const void* x, const floa
     if (P.T == 0) return empty_batch(P, ws, nullptr, nullptr, nullptr, st);
     RouteParams r = route_params(P, ws, topk_idx, topk_gate, logits);
     MOE_TRY(step_logits(P, dv, x, Wr, bias, ws, r, st));
+    // the reroute policy ranks spare experts by logit: keep logits + bias in ws
+    if (P.reroute) r.logits = at<float>(ws, P.off_logits);
     trace_pre(st, "topk");
     MOE_TRY(launched(launch_topk(r, st), "topk"));
     trace_mark(st, "topk");
+    if (P.reroute && logits &&
+        cudaMemcpyAsync(logits, r.logits, (size_t)P.T * P.E * 4, cudaMemcpyDeviceToDevice, st) !=
+            cudaSuccess)
+        return fail(MOE_ERR_CUDA, "logits copy failed");
     return MOE_OK;
 }
 
@@ -457,9 +470,17 @@ static int step_dispatch(const Plan& P, const Device& dv, const int32_t* topk_id
     if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st);
     DispatchParams d = dispatch_params(P, x, routed, kept, offsets, perm_token, slot_of, x_perm);
     trace_pre(st, "dispatch");
-    MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
-                                     at<int32_t>(ws, P.off_tot), dv.sms, st),
-                     "dispatch"));
+    if (P.reroute)
+        MOE_TRY(launched(launch_reroute_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
+                                                 at<int32_t>(ws, P.off_tot),
+                                                 at<float>(ws, P.off_logits),
+                                                 at<int32_t>(ws, P.off_expert),
+                                                 at<int32_t>(ws, P.off_rank), dv.sms, st),
+                         "dispatch"));
+    else
+        MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
+                                         at<int32_t>(ws, P.off_tot), dv.sms, st),
+                         "dispatch"));
     trace_mark(st, "dispatch");
     return MOE_OK;
 }
@@ -472,7 +493,7 @@ static int step_route_dispatch(const Plan& P, const Device& dv, const void* x, c
                                int32_t* perm_token, int32_t* slot_of, void* x_perm, void* ws,
                                cudaStream_t st) {
     if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st);
-    if (P.T > ROUTE_BLOCK) {
+    if (P.T > ROUTE_BLOCK || P.reroute) {
         MOE_TRY(step_route(P, dv, x, Wr, bias, topk_idx, topk_gate, nullptr, ws, st));
         return step_dispatch(P, dv, topk_idx, x, routed, kept, offsets, perm_token, slot_of,
                              x_perm, ws, st);

@@ -59,6 +59,12 @@ int launch_topk(const RouteParams& r, cudaStream_t st);
 // tot [E] receives the totals
 int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt, int32_t* tot,
                     int num_sms, cudaStream_t st);
+// Reroute policy: ranks, then dropped assignments moved in token order to the
+// token's best unused expert with room (z = logits with bias), then slots and
+// row copies.  expert_of / rank_of [T][k] receive the serving expert and rank.
+int launch_reroute_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt,
+                            int32_t* tot, const float* z, int32_t* expert_of, int32_t* rank_of,
+                            int num_sms, cudaStream_t st);
 // T <= 128: top-k and dispatch in one launch
 int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num_sms,
                           cudaStream_t st);

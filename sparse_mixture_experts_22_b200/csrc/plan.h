@@ -34,6 +34,7 @@ struct Plan {
     int d, h, E, k, S, hs;
     int64_t C;          // capacity (T when unlimited)
     bool capped;
+    bool reroute;       // overflow rerouted to a spare expert (else dropped)
     bool bf16;
     int act_bytes;
     int path;           // FfnPath for the routed experts
@@ -51,7 +52,7 @@ struct Plan {
     int router_splits;  // tensor cores: split-K
 
     // workspace byte offsets
-    size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_tot, off_offsets, off_perm,
+    size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_tot, off_expert, off_rank, off_offsets, off_perm,
         off_xperm, off_H, off_y, off_Hs, off_ys, off_sums, total;
 };
 

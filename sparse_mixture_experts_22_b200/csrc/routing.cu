@@ -314,54 +314,53 @@ struct DispatchArgs {
     uint4* x_perm;         // [perm_rows][d]
 };
 
-// Shared memory of dispatch_block: base [E], tot [E], off [E+1], wcnt [DWARPS][E],
-// slots [ROUTE_BLOCK * k].
+// Shared memory of the dispatch kernels: base [E], tot [E], rows [E],
+// off [E+1], wcnt [DWARPS][E], slots [ROUTE_BLOCK * k].
 __host__ __device__ inline size_t dispatch_smem_bytes(int E, int k) {
-    return sizeof(int32_t) * ((size_t)3 * E + 1 + (size_t)DWARPS * E + (size_t)ROUTE_BLOCK * k);
+    return sizeof(int32_t) * ((size_t)4 * E + 1 + (size_t)DWARPS * E + (size_t)ROUTE_BLOCK * k);
 }
 
-// Ranks, slots and row copies of block `blk`.  base[e] (assignments to e in
-// earlier blocks) and tot[e] (in all blocks) must be in shared memory; my[]
-// holds the thread's token choices.  `split`/`nsplit`: this CTA copies every
-// nsplit-th row.  Outputs other than the copies are written when `writer`.
-__device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool writer, int split,
-                               int nsplit, int32_t* base, int32_t* tot, int32_t* off,
-                               int32_t* wcnt, int32_t* slots, const int32_t* my) {
-    const int E = a.E, k = a.k;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) {
-        int32_t o = 0;
-        for (int e = 0; e < E; ++e) {
-            off[e] = o;
-            const int32_t kept = (int64_t)tot[e] < a.C ? tot[e] : (int32_t)a.C;
-            o += (kept + a.pad - 1) / a.pad * a.pad;
-        }
-        off[E] = o;
-    }
-    __syncthreads();
-    if (writer) {
-        if (blk == 0) {
-            for (int e = tid; e < E; e += ROUTE_BLOCK) {
-                a.routed[e] = tot[e];
-                a.kept[e] = (int64_t)tot[e] < a.C ? tot[e] : (int32_t)a.C;
-            }
-            for (int e = tid; e <= E; e += ROUTE_BLOCK) a.offsets[e] = off[e];
-        }
-        if (a.perm_token) {
-            // padding rows of each expert segment, and the unused tail, hold -1
-            for (int e = blk; e < E; e += nblk) {
-                const int32_t kept = (int64_t)tot[e] < a.C ? tot[e] : (int32_t)a.C;
-                for (int r = off[e] + kept + tid; r < off[e + 1]; r += ROUTE_BLOCK)
-                    a.perm_token[r] = -1;
-            }
-            for (int64_t r = off[E] + (int64_t)blk * ROUTE_BLOCK + tid; r < a.perm_rows;
-                 r += (int64_t)nblk * ROUTE_BLOCK)
-                a.perm_token[r] = -1;
-        }
-    }
+struct DispatchSmem {
+    int32_t* base;   // assignments to e in earlier blocks
+    int32_t* tot;    // assignments to e in the batch (routed)
+    int32_t* rows;   // rows e serves (kept)
+    int32_t* off;    // padded segment starts [E+1]
+    int32_t* wcnt;   // per-warp counts [DWARPS][E]
+    int32_t* slots;  // [ROUTE_BLOCK * k]
+};
 
-    const int64_t t = (int64_t)blk * ROUTE_BLOCK + tid;
-    const bool valid = t < a.T;
+__device__ __forceinline__ DispatchSmem dispatch_smem(int32_t* sm, int E) {
+    DispatchSmem d;
+    d.base = sm;
+    d.tot = d.base + E;
+    d.rows = d.tot + E;
+    d.off = d.rows + E;
+    d.wcnt = d.off + E + 1;
+    d.slots = d.wcnt + DWARPS * E;
+    return d;
+}
+
+__device__ __forceinline__ int32_t capped(int32_t n, int64_t C) {
+    return (int64_t)n < C ? n : (int32_t)C;
+}
+
+// Thread 0: padded segment starts from the rows each expert serves.
+__device__ void segment_offsets(const int32_t* rows, int E, int pad, int32_t* off) {
+    if (threadIdx.x != 0) return;
+    int32_t o = 0;
+    for (int e = 0; e < E; ++e) {
+        off[e] = o;
+        o += (rows[e] + pad - 1) / pad * pad;
+    }
+    off[E] = o;
+}
+
+// Global rank of each of the thread's assignments in its expert's queue
+// (token order): earlier blocks (base), earlier warps (per-warp ballot
+// counts), earlier lanes (ballot).  Called by all ROUTE_BLOCK threads.
+__device__ void block_ranks(int E, const int32_t* base, int32_t* wcnt, const int32_t* my,
+                            int32_t* rank) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int32_t rank_w[MAX_K];
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) rank_w[j] = 0;
@@ -382,19 +381,47 @@ __device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool wr
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
+        rank[j] = -1;
+        if (my[j] < 0) continue;
+        const int e = my[j];
+        int32_t r = base[e] + rank_w[j];
+        for (int w = 0; w < warp; ++w) r += wcnt[w * E + e];
+        rank[j] = r;
+    }
+}
+
+// Slots and row copies of block `blk`: assignment j of this thread's token is
+// served by expert[j] at position rank[j] of its queue, kept if rank < C.
+// d.off and d.rows must be filled.  When `writer`, writes slot_of and
+// perm_token (with -1 in padding rows and the unused tail).  `split`/`nsplit`:
+// this CTA copies every nsplit-th row.
+__device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer, int split,
+                           int nsplit, const DispatchSmem& d, const int32_t* expert,
+                           const int32_t* rank) {
+    const int E = a.E, k = a.k;
+    const int tid = threadIdx.x;
+    if (writer && a.perm_token) {
+        for (int e = blk; e < E; e += nblk)
+            for (int r = d.off[e] + d.rows[e] + tid; r < d.off[e + 1]; r += ROUTE_BLOCK)
+                a.perm_token[r] = -1;
+        for (int64_t r = d.off[E] + (int64_t)blk * ROUTE_BLOCK + tid; r < a.perm_rows;
+             r += (int64_t)nblk * ROUTE_BLOCK)
+            a.perm_token[r] = -1;
+    }
+    const int64_t t = (int64_t)blk * ROUTE_BLOCK + tid;
+    const bool valid = t < a.T;
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
         if (j >= k) break;
         int32_t slot = -1;
         if (valid) {
-            const int e = my[j];
-            int32_t r = base[e] + rank_w[j];
-            for (int w = 0; w < warp; ++w) r += wcnt[w * E + e];
-            if ((int64_t)r < a.C) slot = off[e] + r;
+            if (rank[j] >= 0 && (int64_t)rank[j] < a.C) slot = d.off[expert[j]] + rank[j];
             if (writer) {
                 a.slot_of[t * k + j] = slot;
                 if (slot >= 0 && a.perm_token) a.perm_token[slot] = (int32_t)t;
             }
         }
-        slots[tid * k + j] = slot;
+        d.slots[tid * k + j] = slot;
     }
     __syncthreads();
 
@@ -409,7 +436,7 @@ __device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool wr
 #pragma unroll
         for (int q = 0; q < G; ++q) {
             const int r = r0 + q * nsplit;
-            const int32_t slot = r < nrow ? slots[r] : -1;
+            const int32_t slot = r < nrow ? d.slots[r] : -1;
             const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
             src[q] = slot >= 0 ? a.x + tok * nv : nullptr;
             dst[q] = slot >= 0 ? a.x_perm + (int64_t)slot * nv : nullptr;
@@ -424,6 +451,28 @@ __device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool wr
                 if (dst[q]) dst[q][c] = v[q];
         }
     }
+}
+
+// The drop policy: ranks, capacity, slots and row copies of block `blk`.
+// d.base and d.tot must be filled; my[] holds the thread's token choices.
+__device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool writer, int split,
+                               int nsplit, const DispatchSmem& d, const int32_t* my) {
+    const int E = a.E;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += ROUTE_BLOCK) d.rows[e] = capped(d.tot[e], a.C);
+    __syncthreads();
+    segment_offsets(d.rows, E, a.pad, d.off);
+    __syncthreads();
+    if (writer && blk == 0) {
+        for (int e = tid; e < E; e += ROUTE_BLOCK) {
+            a.routed[e] = d.tot[e];
+            a.kept[e] = d.rows[e];
+        }
+        for (int e = tid; e <= E; e += ROUTE_BLOCK) a.offsets[e] = d.off[e];
+    }
+    int32_t rank[MAX_K];
+    block_ranks(E, d.base, d.wcnt, my, rank);
+    place_rows(a, blk, nblk, writer, split, nsplit, d, my, rank);
 }
 
 __global__ void __launch_bounds__(TK_WIDE_THREADS)
@@ -470,23 +519,182 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     dispatch_kernel(DispatchArgs a, const int32_t* __restrict__ topk_idx,
                     const int32_t* __restrict__ base_in, const int32_t* __restrict__ tot_in) {
     extern __shared__ int32_t sm[];
-    int32_t* base = sm;
-    int32_t* tot = base + a.E;
-    int32_t* off = tot + a.E;
-    int32_t* wcnt = off + a.E + 1;
-    int32_t* slots = wcnt + DWARPS * a.E;
+    const DispatchSmem d = dispatch_smem(sm, a.E);
     const int blk = blockIdx.x, nblk = gridDim.x;
     for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) {
-        base[e] = base_in[(int64_t)blk * a.E + e];
-        tot[e] = tot_in[e];
+        d.base[e] = base_in[(int64_t)blk * a.E + e];
+        d.tot[e] = tot_in[e];
     }
     const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
     int32_t my[MAX_K];
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) my[j] = (t < a.T && j < a.k) ? topk_idx[t * a.k + j] : -1;
     __syncthreads();
-    dispatch_block(a, blk, nblk, blockIdx.y == 0, blockIdx.y, gridDim.y, base, tot, off, wcnt,
-                   slots, my);
+    dispatch_block(a, blk, nblk, blockIdx.y == 0, blockIdx.y, gridDim.y, d, my);
+}
+
+// ---------------------------------------------------------------- reroute policy
+//
+// [MoE routing fully explained, "Easy explanation" ¶3: the second way to treat
+// tokens beyond capacity, rerouting them to a spare expert].  Three steps:
+// rank_kernel records every assignment's rank in its expert's queue;
+// reroute_kernel visits the dropped ones in token order and moves each to the
+// token's best-scoring unused expert that still has room (it keeps its gate),
+// which is inherently sequential -- one warp walks the batch while the whole
+// CTA stages each chunk's logits in shared memory; place_kernel then writes
+// slots and copies rows as for the drop policy.
+
+__global__ void __launch_bounds__(ROUTE_BLOCK)
+    rank_kernel(DispatchArgs a, const int32_t* __restrict__ topk_idx,
+                const int32_t* __restrict__ base_in, int32_t* __restrict__ expert_of,
+                int32_t* __restrict__ rank_of) {
+    extern __shared__ int32_t sm[];
+    const DispatchSmem d = dispatch_smem(sm, a.E);
+    const int blk = blockIdx.x;
+    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) d.base[e] = base_in[(int64_t)blk * a.E + e];
+    const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
+    int32_t my[MAX_K], rank[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) my[j] = (t < a.T && j < a.k) ? topk_idx[t * a.k + j] : -1;
+    __syncthreads();
+    block_ranks(a.E, d.base, d.wcnt, my, rank);
+    if (t < a.T)
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j)
+            if (j < a.k) {
+                expert_of[t * a.k + j] = my[j];
+                rank_of[t * a.k + j] = rank[j];
+            }
+}
+
+constexpr int RR_THREADS = 1024;
+constexpr int RR_MAX_ASSIGN = 2048;  // assignments staged per chunk
+
+__host__ __device__ inline int reroute_chunk_tokens(int E, int k) {
+    // logits (E floats) and choices (2k ints) per token within ~160 KB
+    int n = RR_MAX_ASSIGN / k;
+    const int by_smem = (160 * 1024) / (E * 4 + 2 * k * 4);
+    if (n > by_smem) n = by_smem;
+    return n < 1 ? 1 : n;
+}
+
+__host__ __device__ inline size_t reroute_smem_bytes(int E, int k) {
+    const int nt = reroute_chunk_tokens(E, k);
+    return sizeof(int32_t) * ((size_t)E + (size_t)nt * 2 * k) + sizeof(float) * (size_t)nt * E;
+}
+
+__global__ void __launch_bounds__(RR_THREADS)
+    reroute_kernel(const int32_t* __restrict__ topk_idx, int32_t* __restrict__ expert_of,
+                   int32_t* __restrict__ rank_of, const int32_t* __restrict__ tot,
+                   const float* __restrict__ z, const float* __restrict__ bias, int64_t T, int E,
+                   int k, int64_t C, int pad, int32_t* __restrict__ routed,
+                   int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
+    extern __shared__ int32_t sm[];
+    const int nt = reroute_chunk_tokens(E, k);
+    int32_t* fill = sm;                     // [E]
+    int32_t* cidx = fill + E;               // [nt][k] router choices
+    int32_t* cexp = cidx + nt * k;          // [nt][k] serving experts
+    float* cz = reinterpret_cast<float*>(cexp + nt * k);  // [nt][E] logits + bias
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += RR_THREADS) {
+        fill[e] = capped(tot[e], C);
+        routed[e] = tot[e];
+    }
+    __syncthreads();
+    for (int64_t t0 = 0; t0 < T; t0 += nt) {
+        const int n = (int)(T - t0 < nt ? T - t0 : nt);
+        const int64_t a0 = t0 * k;
+        // anything dropped in this chunk?
+        int any = 0;
+        for (int i = tid; i < n * k; i += RR_THREADS) any |= (int64_t)rank_of[a0 + i] >= C;
+        if (!__syncthreads_or(any)) continue;
+        for (int i = tid; i < n * k; i += RR_THREADS) {
+            cidx[i] = topk_idx[a0 + i];
+            cexp[i] = cidx[i];
+        }
+        for (int i = tid; i < n * E; i += RR_THREADS) {
+            const int e = i % E;
+            const float v = z[t0 * E + i];
+            cz[i] = bias ? v + bias[e] : v;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            for (int i0 = 0; i0 < n * k; i0 += 32) {
+                const int i = i0 + lane;
+                const bool dropped = i < n * k && (int64_t)rank_of[a0 + i] >= C;
+                unsigned m = __ballot_sync(0xffffffffu, dropped);
+                while (m) {
+                    const int b = __ffs(m) - 1;
+                    m &= m - 1;
+                    const int ii = i0 + b;
+                    const int tl = ii / k;
+                    // best-scoring expert with room that the token does not use
+                    float bv = -INFINITY;
+                    int be = 0x7fffffff;
+                    for (int e = lane; e < E; e += 32) {
+                        if ((int64_t)fill[e] >= C) continue;
+                        bool used = false;
+                        for (int q = 0; q < k; ++q)
+                            used |= (cidx[tl * k + q] == e) || (cexp[tl * k + q] == e);
+                        if (used) continue;
+                        const float v = cz[tl * E + e];
+                        const float vv = v != v ? -INFINITY : v;
+                        if (be == 0x7fffffff || vv > bv) {
+                            bv = vv;
+                            be = e;
+                        }
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                        if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
+                            bv = ov;
+                            be = oe;
+                        }
+                    }
+                    if (be != 0x7fffffff && lane == 0) {
+                        cexp[ii] = be;
+                        expert_of[a0 + ii] = be;
+                        rank_of[a0 + ii] = fill[be];
+                        fill[be] += 1;
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < E; e += RR_THREADS) kept[e] = fill[e];
+    __syncthreads();
+    if (tid == 0) {
+        int32_t o = 0;
+        for (int e = 0; e < E; ++e) {
+            offsets[e] = o;
+            o += (fill[e] + pad - 1) / pad * pad;
+        }
+        offsets[E] = o;
+    }
+}
+
+__global__ void __launch_bounds__(ROUTE_BLOCK)
+    place_kernel(DispatchArgs a, const int32_t* __restrict__ expert_of,
+                 const int32_t* __restrict__ rank_of) {
+    extern __shared__ int32_t sm[];
+    const DispatchSmem d = dispatch_smem(sm, a.E);
+    const int blk = blockIdx.x, nblk = gridDim.x;
+    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) d.rows[e] = a.kept[e];
+    for (int e = threadIdx.x; e <= a.E; e += ROUTE_BLOCK) d.off[e] = a.offsets[e];
+    const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
+    int32_t ex[MAX_K], rank[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        const bool v = t < a.T && j < a.k;
+        ex[j] = v ? expert_of[t * a.k + j] : -1;
+        rank[j] = v ? rank_of[t * a.k + j] : -1;
+    }
+    __syncthreads();
+    place_rows(a, blk, nblk, blockIdx.y == 0, blockIdx.y, gridDim.y, d, ex, rank);
 }
 
 // T <= ROUTE_BLOCK: top-k and dispatch in one launch.  Every CTA routes the
@@ -500,11 +708,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     float* zs = reinterpret_cast<float*>(dyn + E);
     int32_t* dsm =
         reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dyn) + topk_smem_bytes(E, ROUTE_BLOCK));
-    int32_t* base = dsm;
-    int32_t* tot = base + E;
-    int32_t* off = tot + E;
-    int32_t* wcnt = off + E + 1;
-    int32_t* slots = wcnt + DWARPS * E;
+    const DispatchSmem d = dispatch_smem(dsm, E);
     const bool leader = blockIdx.x == 0;
     if (leader && threadIdx.x == 0 && ta.status) {
         ta.status[0] = DEV_OK;
@@ -514,12 +718,12 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     topk_block(ta, 0, leader, hist, zs, my);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += ROUTE_BLOCK) {
-        base[e] = 0;
-        tot[e] = hist[e];
+        d.base[e] = 0;
+        d.tot[e] = hist[e];
         if (leader) cnt[e] = hist[e];
     }
     __syncthreads();
-    dispatch_block(da, 0, 1, leader, blockIdx.x, gridDim.x, base, tot, off, wcnt, slots, my);
+    dispatch_block(da, 0, 1, leader, blockIdx.x, gridDim.x, d, my);
 }
 
 template <typename K>
@@ -600,6 +804,31 @@ int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* c
     if (set_smem(dispatch_kernel, smem)) return -1;
     dim3 grid(nblk, copy_splits(nblk, p.T, p.k, num_sms));
     dispatch_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(dispatch_args(p), topk_idx, cnt, tot);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_reroute_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt,
+                            int32_t* tot, const float* z, int32_t* expert_of, int32_t* rank_of,
+                            int num_sms, cudaStream_t st) {
+    if (p.T == 0) return 0;
+    const int nblk = (int)((p.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    const DispatchArgs a = dispatch_args(p);
+    const int64_t scan_threads = (int64_t)p.E * 32;
+    dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nblk,
+                                                                                p.E);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    const size_t smem = dispatch_smem_bytes(p.E, p.k);
+    if (set_smem(rank_kernel, smem) || set_smem(place_kernel, smem)) return -1;
+    rank_kernel<<<nblk, ROUTE_BLOCK, smem, st>>>(a, topk_idx, cnt, expert_of, rank_of);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    const size_t rsmem = reroute_smem_bytes(p.E, p.k);
+    if (set_smem(reroute_kernel, rsmem)) return -1;
+    reroute_kernel<<<1, RR_THREADS, rsmem, st>>>(topk_idx, expert_of, rank_of, tot, z, nullptr,
+                                                 p.T, p.E, p.k, p.C, p.pad, p.routed, p.kept,
+                                                 p.offsets);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    dim3 grid(nblk, copy_splits(nblk, p.T, p.k, num_sms));
+    place_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(a, expert_of, rank_of);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -68,16 +68,21 @@ def router_bias(wl: Workload) -> Optional[torch.Tensor]:
 
 
 def _near_tie_rows(x: torch.Tensor, Wr: torch.Tensor, b: Optional[torch.Tensor],
-                   k: int) -> torch.Tensor:
-    """Indices of rows whose k-th and (k+1)-th largest fp64 logits are < TIE_GAP apart."""
+                   k: int, all_gaps: bool = False) -> torch.Tensor:
+    """Indices of rows whose k-th and (k+1)-th largest fp64 logits are < TIE_GAP
+    apart (with all_gaps: any two neighbouring logits in sorted order)."""
     E = Wr.shape[1]
-    if k >= E or x.shape[0] == 0:
+    if (k >= E and not all_gaps) or x.shape[0] == 0 or E < 2:
         return torch.zeros(0, dtype=torch.long)
     z = x.double() @ Wr.double()
     if b is not None:
         z = z + b.double()
-    top = torch.topk(z, k + 1, dim=1).values
-    gap = top[:, k - 1] - top[:, k]
+    if all_gaps:
+        srt = torch.sort(z, dim=1, descending=True).values
+        gap = (srt[:, :-1] - srt[:, 1:]).min(dim=1).values
+    else:
+        top = torch.topk(z, k + 1, dim=1).values
+        gap = top[:, k - 1] - top[:, k]
     return torch.nonzero(gap < TIE_GAP).flatten()
 
 
@@ -85,6 +90,8 @@ def tokens(wl: Workload, T: Optional[int] = None, Wr: Optional[torch.Tensor] = N
            b: Optional[torch.Tensor] = None, stream: str = "x") -> (torch.Tensor, int):
     """x [T, d] in the workload dtype, with near-tie rows redrawn.
 
+    Under the reroute policy a spare expert is chosen among all experts, so
+    there every pair of neighbouring sorted logits is kept TIE_GAP apart.
     Returns (x, number of rows redrawn).  Redrawn rows come from the same
     generator stream, continuing, so the result is a pure function of the seed.
     """
@@ -98,7 +105,7 @@ def tokens(wl: Workload, T: Optional[int] = None, Wr: Optional[torch.Tensor] = N
         b = router_bias(wl)
     redrawn = 0
     for _ in range(1000):
-        bad = _near_tie_rows(x, Wr, b, wl.k)
+        bad = _near_tie_rows(x, Wr, b, wl.k, all_gaps=wl.overflow == "reroute")
         if bad.numel() == 0:
             return x, redrawn
         redrawn += bad.numel()

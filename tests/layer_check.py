@@ -159,23 +159,24 @@ def check_logits(r: Dict, logits: torch.Tensor):
 
 def check_slots(wl: Workload, r: Dict, b: Dict, offsets: np.ndarray,
                 perm_token: Optional[np.ndarray] = None):
-    """Dropped set and ranks, bit-exact, matched per (token, expert)."""
+    """Dropped set, serving expert and rank of every assignment, bit-exact,
+    matched per (token, expert the router chose)."""
     T, k = wl.T, wl.k
     idx = b["topk_idx"].cpu().numpy()
     slot = b["slot_of"].cpu().numpy()
     ref = {}
     for t in range(T):
         for j in range(k):
-            ref[(t, int(r["idx"][t, j]))] = (int(r["keep"][t, j]), int(r["rank"][t, j]))
+            ref[(t, int(r["idx"][t, j]))] = (int(r["keep"][t, j]), int(r["expert"][t, j]),
+                                             int(r["rank"][t, j]))
     for t in range(T):
         for j in range(k):
-            e = int(idx[t, j])
-            keep, rank = ref[(t, e)]
+            keep, ex, rank = ref[(t, int(idx[t, j]))]
             s = int(slot[t, j])
             if not keep:
-                assert s == -1, (t, e, s)
+                assert s == -1, (t, j, s)
             else:
-                assert s == offsets[e] + rank, (t, e, s, offsets[e], rank)
+                assert s == offsets[ex] + rank, (t, j, s, ex, offsets[ex], rank)
                 if perm_token is not None:
                     assert perm_token[s] == t
 

@@ -47,6 +47,17 @@ SMALL = {
     "k_equals_E": Workload("k_equals_E", T=64, d=128, h=128, E=4, k=4),
     "top1": Workload("top1", T=257, d=256, h=128, E=8, k=1, cf=(2, 1)),
     "collapse": Workload("collapse", T=512, d=128, h=128, E=8, k=2, cf=(5, 4), zipf_s=12.0),
+    # overflow rerouted to a spare expert: swapped and token-major tiles, top-1, many experts
+    "reroute_swap": Workload("reroute_swap", T=1000, d=256, h=256, E=8, k=2, cf=(1, 1),
+                             zipf_s=1.2, overflow="reroute"),
+    "reroute_tok": Workload("reroute_tok", T=600, d=256, h=384, E=4, k=2, cf=(5, 4), zipf_s=0.7,
+                            overflow="reroute"),
+    "reroute_top1": Workload("reroute_top1", T=300, d=128, h=128, E=8, k=1, cf=(1, 1),
+                             zipf_s=2.0, overflow="reroute"),
+    "reroute_wide": Workload("reroute_wide", T=300, d=256, h=128, E=40, k=4, cf=(1, 2),
+                             zipf_s=0.5, overflow="reroute"),
+    "reroute_f32": Workload("reroute_f32", T=90, d=128, h=128, E=4, k=2, cf=(1, 2), dtype="f32",
+                            zipf_s=1.0, overflow="reroute"),
 }
 
 
@@ -135,12 +146,14 @@ def test_bad_workspace_is_rejected():
 
 # ---------------------------------------------------------------- full-size workloads
 
-FULL_SAMPLE = {"decode": 32, "prefill": 24, "deepseek": 16, "large": 16}
+FULL = dict(WORKLOADS)
+FULL["prefill_reroute"] = WORKLOADS["prefill"].scaled(name="prefill_reroute", overflow="reroute")
+FULL_SAMPLE = {"decode": 32, "prefill": 24, "deepseek": 16, "large": 16, "prefill_reroute": 24}
 
 
-@pytest.mark.parametrize("name", ["decode", "prefill", "deepseek", "large"])
+@pytest.mark.parametrize("name", ["decode", "prefill", "deepseek", "large", "prefill_reroute"])
 def test_full_size_workload(name):
-    wl = WORKLOADS[name]
+    wl = FULL[name]
     inp = host_inputs(wl)
     r = oracle_route(wl, inp)
     cfg, g, W = device_layer(wl, inp)
@@ -150,7 +163,7 @@ def test_full_size_workload(name):
     zerr = check_logits(r, route_logits(cfg, g))
     # dropped set and ranks for every assignment (offsets rebuilt from the oracle's kept counts)
     pad = _pad(cfg)
-    offsets = np.zeros(wl.E + 1, dtype=np.int64)
+    offsets = np.zeros(wl.E + 1, dtype=np.int64)  # from the oracle's final kept counts
     for e in range(wl.E):
         offsets[e + 1] = offsets[e] + (int(r["kept"][e]) + pad - 1) // pad * pad
     check_slots(wl, r, b, offsets)
