@@ -327,3 +327,286 @@ int oracle_threads(void) {
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------ backward
+ *
+ * Gradients of the layer [the pages motivate them: the softmax weighting of
+ * the router and the load-balancing loss are what training acts on, Routing
+ * explained, "Easy explanation" ¶2 and ¶4].  The loss taken is
+ *   L = sum_t <G_t, out_t> + aux_coef * aux,
+ * G = dL/dout being given.  Readings (the pages are silent on all of them):
+ *   - the capacity decision and the top-k choice are piecewise constant, so
+ *     the routed counts f_e carry no gradient; aux reaches the router through
+ *     P_e only;
+ *   - gates are not renormalised after a drop, so a dropped assignment still
+ *     shapes the gates of the kept ones: its gate gradient is 0, but its logit
+ *     receives the softmax-over-k terms of the others;
+ *   - under the reroute policy an assignment keeps the gate of the expert the
+ *     router chose, so the gate gradient goes to that expert's logit while the
+ *     FFN evaluated (and differentiated) is the serving expert's.
+ * With a = x w1, b = x w3, s = silu(a), u = s * b, y = u w2 and
+ * silu'(a) = sig(a) (1 + a (1 - sig(a))):
+ *   dy = g G_t,  dg = <G_t, y>,  dw2 += u^T dy,  du = w2 dy,
+ *   da = du * b * silu'(a),  db = du * s,
+ *   dw1 += x^T da,  dw3 += x^T db,  dx += w1 da + w3 db;
+ *   softmax over the kept k:  dz[idx_j] += g_j (dg_j - sum_q g_q dg_q);
+ *   aux = E sum_e f_e P_e, P_e = mean_t p_te:
+ *     dz[t][e] += aux_coef (E / T) p_te (f_e - sum_i f_i p_ti);
+ *   router z = x Wr + b:  dWr += x^T dz,  db_router += dz,  dx += Wr dz.
+ * Shared experts take dy = G_t (gate 1) and have no gate gradient. */
+
+/* One expert's FFN forward and backward for one token.  Adds into dw1, dw3
+ * ([d][h] at w_off13), dw2 ([h][d] at w_off2) and dx ([d]); returns
+ * <G_t, y>.  dw1 == NULL skips the weight gradients.  a, b, u, du are scratch
+ * of length h; y of length d. */
+static double ffn_backward(int d, int h, int dtype, const void* x, int64_t x_off,
+                           const void* G, double g, const void* w1, const void* w3,
+                           const void* w2, int64_t w_off13, int64_t w_off2, double* dw1,
+                           double* dw3, double* dw2, double* dx, double* a, double* b,
+                           double* u, double* du, double* y) {
+    for (int i = 0; i < h; ++i) { a[i] = 0.0; b[i] = 0.0; }
+    for (int c = 0; c < d; ++c) {
+        const double xc = elem(x, dtype, x_off + c);
+        const int64_t row = w_off13 + (int64_t)c * h;
+        for (int i = 0; i < h; ++i) {
+            a[i] += xc * elem(w1, dtype, row + i);
+            b[i] += xc * elem(w3, dtype, row + i);
+        }
+    }
+    for (int i = 0; i < h; ++i) u[i] = a[i] / (1.0 + exp(-a[i])) * b[i];
+    for (int o = 0; o < d; ++o) y[o] = 0.0;
+    for (int i = 0; i < h; ++i) {
+        const int64_t row = w_off2 + (int64_t)i * d;
+        for (int o = 0; o < d; ++o) y[o] += u[i] * elem(w2, dtype, row + o);
+    }
+    double dg = 0.0;
+    for (int o = 0; o < d; ++o) dg += elem(G, dtype, x_off + o) * y[o];
+    /* dy = g G_t, used through its entries below */
+    for (int i = 0; i < h; ++i) {
+        const int64_t row = w_off2 + (int64_t)i * d;
+        double s = 0.0;
+        for (int o = 0; o < d; ++o) {
+            const double dyo = g * elem(G, dtype, x_off + o);
+            if (dw1) dw2[row + o] += u[i] * dyo;
+            s += elem(w2, dtype, row + o) * dyo;
+        }
+        du[i] = s;
+    }
+    for (int i = 0; i < h; ++i) {
+        const double sig = 1.0 / (1.0 + exp(-a[i]));
+        const double silu = a[i] * sig;
+        const double da = du[i] * b[i] * sig * (1.0 + a[i] * (1.0 - sig));
+        const double db = du[i] * silu;
+        a[i] = da;  /* reuse the scratch: a <- da, b <- db */
+        b[i] = db;
+    }
+    for (int c = 0; c < d; ++c) {
+        const double xc = elem(x, dtype, x_off + c);
+        const int64_t row = w_off13 + (int64_t)c * h;
+        double s = 0.0;
+        for (int i = 0; i < h; ++i) {
+            if (dw1) {
+                dw1[row + i] += xc * a[i];
+                dw3[row + i] += xc * b[i];
+            }
+            s += elem(w1, dtype, row + i) * a[i] + elem(w3, dtype, row + i) * b[i];
+        }
+        dx[c] += s;
+    }
+    return dg;
+}
+
+/* Gradient of the router logits of token t (gate path and aux path).
+ *   dgt[j]  <G_t, y_j> for kept assignments, 0 for dropped ones
+ *   f[e]    routed[e] / (T k);  dzt[E] out */
+static void router_logit_grad(const oracle_cfg* c, const double* zt, const int32_t* it,
+                              const double* gt, const double* dgt, const double* f,
+                              double aux_coef, double* dzt) {
+    const int E = c->E, k = c->k;
+    for (int e = 0; e < E; ++e) dzt[e] = 0.0;
+    double m = 0.0;
+    for (int j = 0; j < k; ++j) m += gt[j] * dgt[j];
+    for (int j = 0; j < k; ++j) dzt[it[j]] += gt[j] * (dgt[j] - m);
+    double zmax = zt[0];
+    for (int e = 1; e < E; ++e) if (zt[e] > zmax) zmax = zt[e];
+    double den = 0.0;
+    for (int e = 0; e < E; ++e) den += exp(zt[e] - zmax);
+    double q = 0.0;
+    for (int e = 0; e < E; ++e) q += f[e] * exp(zt[e] - zmax) / den;
+    const double scale = aux_coef * (double)E / (double)c->T;
+    for (int e = 0; e < E; ++e) {
+        const double p = exp(zt[e] - zmax) / den;
+        dzt[e] += scale * p * (f[e] - q);
+    }
+}
+
+/* The whole backward pass.  Inputs: the forward's logits z [T][E] (bias
+ * included), router choice idx, serving expert, gates, keep flags and routed
+ * counts; G [T][d] in the layer dtype.  Outputs (all overwritten, fp64):
+ *   dx [T][d], dWr [d][E], db [E], dz [T][E],
+ *   dw1, dw3 [E][d][h], dw2 [E][h][d], and (n_shared > 0) dw1s, dw3s
+ *   [S][d][hs], dw2s [S][hs][d].
+ * Tokens are visited in increasing order and every sum runs in one fixed
+ * order; single-threaded (small cases only). */
+void oracle_backward(const oracle_cfg* c, const void* x, const float* Wr, const double* z,
+                     const int32_t* idx, const int32_t* expert, const double* gate,
+                     const int8_t* keep, const int32_t* routed, const void* w1,
+                     const void* w3, const void* w2, const void* w1s, const void* w3s,
+                     const void* w2s, const void* G, double aux_coef, double* dx, double* dWr,
+                     double* db, double* dz, double* dw1, double* dw3, double* dw2,
+                     double* dw1s, double* dw3s, double* dw2s) {
+    const int64_t T = c->T;
+    const int d = c->d, h = c->h, E = c->E, k = c->k, S = c->n_shared, hs = c->h_shared;
+    const int hmax = h > hs ? h : hs;
+    memset(dx, 0, sizeof(double) * (size_t)(T * d));
+    memset(dWr, 0, sizeof(double) * (size_t)d * E);
+    memset(db, 0, sizeof(double) * (size_t)E);
+    memset(dz, 0, sizeof(double) * (size_t)(T * E));
+    memset(dw1, 0, sizeof(double) * (size_t)E * d * h);
+    memset(dw3, 0, sizeof(double) * (size_t)E * d * h);
+    memset(dw2, 0, sizeof(double) * (size_t)E * h * d);
+    if (S > 0) {
+        memset(dw1s, 0, sizeof(double) * (size_t)S * d * hs);
+        memset(dw3s, 0, sizeof(double) * (size_t)S * d * hs);
+        memset(dw2s, 0, sizeof(double) * (size_t)S * hs * d);
+    }
+    if (T == 0) return;
+    double* a = (double*)malloc(sizeof(double) * (size_t)hmax);
+    double* b = (double*)malloc(sizeof(double) * (size_t)hmax);
+    double* u = (double*)malloc(sizeof(double) * (size_t)hmax);
+    double* du = (double*)malloc(sizeof(double) * (size_t)hmax);
+    double* y = (double*)malloc(sizeof(double) * (size_t)d);
+    double* f = (double*)malloc(sizeof(double) * (size_t)E);
+    double* dg = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int e = 0; e < E; ++e) f[e] = (double)routed[e] / ((double)T * k);
+    for (int64_t t = 0; t < T; ++t) {
+        double* dxt = dx + t * d;
+        for (int j = 0; j < k; ++j) {
+            dg[j] = 0.0;
+            if (!keep[t * k + j]) continue;
+            const int64_t e = expert[t * k + j];
+            dg[j] = ffn_backward(d, h, c->dtype, x, t * d, G, gate[t * k + j], w1, w3, w2,
+                                 e * d * h, e * h * d, dw1, dw3, dw2, dxt, a, b, u, du, y);
+        }
+        for (int s = 0; s < S; ++s)
+            (void)ffn_backward(d, hs, c->dtype, x, t * d, G, 1.0, w1s, w3s, w2s,
+                               (int64_t)s * d * hs, (int64_t)s * hs * d, dw1s, dw3s, dw2s, dxt,
+                               a, b, u, du, y);
+        double* dzt = dz + t * E;
+        router_logit_grad(c, z + t * E, idx + t * k, gate + t * k, dg, f, aux_coef, dzt);
+        for (int cc = 0; cc < d; ++cc) {
+            const double xc = elem(x, c->dtype, t * d + cc);
+            double s = 0.0;
+            for (int e = 0; e < E; ++e) {
+                dWr[(int64_t)cc * E + e] += xc * dzt[e];
+                s += (double)Wr[(int64_t)cc * E + e] * dzt[e];
+            }
+            dxt[cc] += s;
+        }
+        for (int e = 0; e < E; ++e) db[e] += dzt[e];
+    }
+    free(a); free(b); free(u); free(du); free(y); free(f); free(dg);
+}
+
+/* dx and dz rows of selected tokens (no weight gradients), for checks of
+ * large batches: each row needs only its own token, the routed counts and
+ * the token's experts.  rows[n_rows] lists the tokens; dx_rows [n_rows][d],
+ * dz_rows [n_rows][E]. */
+void oracle_backward_rows(const oracle_cfg* c, const void* x, const float* Wr, const double* z,
+                          const int32_t* idx, const int32_t* expert, const double* gate,
+                          const int8_t* keep, const int32_t* routed, const void* w1,
+                          const void* w3, const void* w2, const void* w1s, const void* w3s,
+                          const void* w2s, const void* G, double aux_coef, const int64_t* rows,
+                          int64_t n_rows, double* dx_rows, double* dz_rows) {
+    const int64_t T = c->T;
+    const int d = c->d, h = c->h, E = c->E, k = c->k, S = c->n_shared, hs = c->h_shared;
+    const int hmax = h > hs ? h : hs;
+    double* f = (double*)malloc(sizeof(double) * (size_t)E);
+    for (int e = 0; e < E; ++e) f[e] = T > 0 ? (double)routed[e] / ((double)T * k) : 0.0;
+#pragma omp parallel
+    {
+        double* a = (double*)malloc(sizeof(double) * (size_t)hmax);
+        double* b = (double*)malloc(sizeof(double) * (size_t)hmax);
+        double* u = (double*)malloc(sizeof(double) * (size_t)hmax);
+        double* du = (double*)malloc(sizeof(double) * (size_t)hmax);
+        double* y = (double*)malloc(sizeof(double) * (size_t)d);
+        double* dg = (double*)malloc(sizeof(double) * (size_t)k);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            const int64_t t = rows[r];
+            double* dxt = dx_rows + r * d;
+            for (int cc = 0; cc < d; ++cc) dxt[cc] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                dg[j] = 0.0;
+                if (!keep[t * k + j]) continue;
+                const int64_t e = expert[t * k + j];
+                dg[j] = ffn_backward(d, h, c->dtype, x, t * d, G, gate[t * k + j], w1, w3, w2,
+                                     e * d * h, e * h * d, NULL, NULL, NULL, dxt, a, b, u, du, y);
+            }
+            for (int s = 0; s < S; ++s)
+                (void)ffn_backward(d, hs, c->dtype, x, t * d, G, 1.0, w1s, w3s, w2s,
+                                   (int64_t)s * d * hs, (int64_t)s * hs * d, NULL, NULL, NULL,
+                                   dxt, a, b, u, du, y);
+            double* dzt = dz_rows + r * E;
+            router_logit_grad(c, z + t * E, idx + t * k, gate + t * k, dg, f, aux_coef, dzt);
+            for (int cc = 0; cc < d; ++cc) {
+                double s = 0.0;
+                for (int e = 0; e < E; ++e) s += (double)Wr[(int64_t)cc * E + e] * dzt[e];
+                dxt[cc] += s;
+            }
+        }
+        free(a); free(b); free(u); free(du); free(y); free(dg);
+    }
+    free(f);
+}
+
+/* A block of one expert's weight gradients, for checks of large batches.
+ * Expert `e` of the routed set (shared == 0; tokens whose kept assignment is
+ * served by e, with their gates) or shared expert `e` (shared == 1; every
+ * token, gate 1).  For hidden indices hi[ni] and model indices ci[nc]:
+ *   out1[a][b] = dw1[ci[b]][hi[a]],  out3[a][b] = dw3[ci[b]][hi[a]],
+ *   out2[a][b] = dw2[hi[a]][ci[b]]    (each [ni][nc]).
+ * Tokens are visited in increasing order. */
+void oracle_wgrad_block(const oracle_cfg* c, const void* x, const int32_t* expert,
+                        const double* gate, const int8_t* keep, const void* w1, const void* w3,
+                        const void* w2, const void* G, int shared, int e, const int32_t* hi,
+                        int ni, const int32_t* ci, int nc, double* out1, double* out3,
+                        double* out2) {
+    const int64_t T = c->T;
+    const int d = c->d, k = c->k;
+    const int h = shared ? c->h_shared : c->h;
+    const int64_t off13 = (int64_t)e * d * h, off2 = (int64_t)e * h * d;
+    for (int i = 0; i < ni * nc; ++i) { out1[i] = 0.0; out3[i] = 0.0; out2[i] = 0.0; }
+#pragma omp parallel for schedule(static)
+    for (int q = 0; q < ni; ++q) {
+        const int i = hi[q];
+        for (int64_t t = 0; t < T; ++t) {
+            for (int j = 0; j < (shared ? 1 : k); ++j) {
+                double g = 1.0;
+                if (!shared) {
+                    if (!keep[t * k + j] || expert[t * k + j] != e) continue;
+                    g = gate[t * k + j];
+                }
+                double a = 0.0, b = 0.0, du = 0.0;
+                for (int cc = 0; cc < d; ++cc) {
+                    const double xc = elem(x, c->dtype, t * d + cc);
+                    a += xc * elem(w1, c->dtype, off13 + (int64_t)cc * h + i);
+                    b += xc * elem(w3, c->dtype, off13 + (int64_t)cc * h + i);
+                }
+                for (int o = 0; o < d; ++o)
+                    du += elem(w2, c->dtype, off2 + (int64_t)i * d + o) * g *
+                          elem(G, c->dtype, t * d + o);
+                const double sig = 1.0 / (1.0 + exp(-a));
+                const double u = a * sig * b;
+                const double da = du * b * sig * (1.0 + a * (1.0 - sig));
+                const double dbv = du * a * sig;
+                for (int r = 0; r < nc; ++r) {
+                    const double xc = elem(x, c->dtype, t * d + ci[r]);
+                    out1[q * nc + r] += xc * da;
+                    out3[q * nc + r] += xc * dbv;
+                    out2[q * nc + r] += u * g * elem(G, c->dtype, t * d + ci[r]);
+                }
+            }
+        }
+    }
+}

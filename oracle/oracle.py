@@ -54,6 +54,12 @@ def _bind(path: str):
     L.oracle_ffn.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
     L.oracle_layer_rows.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int64, P]
     L.oracle_threads.restype = ctypes.c_int
+    L.oracle_backward.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                  ctypes.c_double, P, P, P, P, P, P, P, P, P, P]
+    L.oracle_backward_rows.argtypes = [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                       ctypes.c_double, P, ctypes.c_int64, P, P]
+    L.oracle_wgrad_block.argtypes = [C, P, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                     P, ctypes.c_int, P, ctypes.c_int, P, P, P]
     return L
 
 
@@ -212,3 +218,73 @@ def forward(cfg: OracleCfg, inp: Dict, rows=None) -> Dict:
                           inp["w3"], inp["w2"], inp.get("w1s"), inp.get("w3s"),
                           inp.get("w2s"), rows)
     return r
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def backward(cfg: OracleCfg, inp: Dict, r: Dict, G, aux_coef: float = 0.0) -> Dict:
+    """Gradients of L = <G, out> + aux_coef * aux (see oracle_backward).
+
+    `r` is the routing of the same inputs (route()); G [T, d] in the layer
+    dtype.  Returns fp64 arrays dx, dWr, db, dz, dw1, dw3, dw2 (and dw1s,
+    dw3s, dw2s with shared experts) in the layer's own layouts."""
+    T, d, h, E, k = cfg.T, cfg.d, cfg.h, cfg.E, cfg.k
+    S, hs = cfg.n_shared, cfg.h_shared
+    out = {"dx": np.empty((T, d)), "dWr": np.empty((d, E)), "db": np.empty(E),
+           "dz": np.empty((T, E)), "dw1": np.empty((E, d, h)), "dw3": np.empty((E, d, h)),
+           "dw2": np.empty((E, h, d))}
+    if S:
+        out.update({"dw1s": np.empty((S, d, hs)), "dw3s": np.empty((S, d, hs)),
+                    "dw2s": np.empty((S, hs, d))})
+    z = _c(r["z"], np.float64)
+    idx = _c(r["idx"], np.int32)
+    expert = _c(r["expert"], np.int32)
+    gate = _c(r["gate"], np.float64)
+    keep = _c(r["keep"], np.int8)
+    routed = _c(r["routed"], np.int32)
+    lib().oracle_backward(
+        ctypes.byref(cfg), _ptr(inp["x"]), _ptr(inp["Wr"]), _ptr(z), _ptr(idx), _ptr(expert),
+        _ptr(gate), _ptr(keep), _ptr(routed), _ptr(inp["w1"]), _ptr(inp["w3"]), _ptr(inp["w2"]),
+        _ptr(inp.get("w1s")), _ptr(inp.get("w3s")), _ptr(inp.get("w2s")), _ptr(G),
+        float(aux_coef), _ptr(out["dx"]), _ptr(out["dWr"]), _ptr(out["db"]), _ptr(out["dz"]),
+        _ptr(out["dw1"]), _ptr(out["dw3"]), _ptr(out["dw2"]), _ptr(out.get("dw1s")),
+        _ptr(out.get("dw3s")), _ptr(out.get("dw2s")))
+    return out
+
+
+def backward_rows(cfg: OracleCfg, inp: Dict, r: Dict, G, aux_coef: float, rows) -> Dict:
+    """dx and dz rows of the listed tokens only (see oracle_backward_rows)."""
+    rows_arr = _c(rows, np.int64)
+    n = rows_arr.shape[0]
+    dx = np.empty((n, cfg.d))
+    dz = np.empty((n, cfg.E))
+    lib().oracle_backward_rows(
+        ctypes.byref(cfg), _ptr(inp["x"]), _ptr(inp["Wr"]), _ptr(_c(r["z"], np.float64)),
+        _ptr(_c(r["idx"], np.int32)), _ptr(_c(r["expert"], np.int32)),
+        _ptr(_c(r["gate"], np.float64)), _ptr(_c(r["keep"], np.int8)),
+        _ptr(_c(r["routed"], np.int32)), _ptr(inp["w1"]), _ptr(inp["w3"]), _ptr(inp["w2"]),
+        _ptr(inp.get("w1s")), _ptr(inp.get("w3s")), _ptr(inp.get("w2s")), _ptr(G),
+        float(aux_coef), _ptr(rows_arr), n, _ptr(dx), _ptr(dz))
+    return {"dx": dx, "dz": dz}
+
+
+def wgrad_block(cfg: OracleCfg, inp: Dict, r: Dict, G, e: int, hi, ci,
+                shared: bool = False) -> Dict:
+    """dw1[ci, hi], dw3[ci, hi] and dw2[hi, ci] of one routed (or shared) expert,
+    each returned as [len(hi), len(ci)] (see oracle_wgrad_block)."""
+    hi_a = _c(hi, np.int32)
+    ci_a = _c(ci, np.int32)
+    ni, nc = hi_a.shape[0], ci_a.shape[0]
+    o1, o3, o2 = np.empty((ni, nc)), np.empty((ni, nc)), np.empty((ni, nc))
+    if shared:
+        w1, w3, w2 = inp["w1s"], inp["w3s"], inp["w2s"]
+    else:
+        w1, w3, w2 = inp["w1"], inp["w3"], inp["w2"]
+    lib().oracle_wgrad_block(
+        ctypes.byref(cfg), _ptr(inp["x"]), _ptr(_c(r["expert"], np.int32)),
+        _ptr(_c(r["gate"], np.float64)), _ptr(_c(r["keep"], np.int8)), _ptr(w1), _ptr(w3),
+        _ptr(w2), _ptr(G), 1 if shared else 0, int(e), _ptr(hi_a), ni, _ptr(ci_a), nc,
+        _ptr(o1), _ptr(o3), _ptr(o2))
+    return {"dw1": o1, "dw3": o3, "dw2": o2}

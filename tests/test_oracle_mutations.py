@@ -8,6 +8,7 @@ import subprocess
 import pytest
 
 import oracle as O
+import test_oracle_backward_pins as bpins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(O.__file__), "moe_oracle.c")
@@ -57,6 +58,38 @@ MUTATIONS = [
      [pins.test_reroute_matches_simulation_and_invariants]),
     ("reroute may reuse an expert", "if (used) continue;", "",
      [pins.test_reroute_matches_simulation_and_invariants]),
+    # backward pass
+    ("silu derivative drops a term", "sig * (1.0 + a[i] * (1.0 - sig))", "sig * (1.0 + a[i] * sig)",
+     [bpins.test_backward_matches_finite_differences]),
+    ("gate gradient sign", "dzt[it[j]] += gt[j] * (dgt[j] - m);",
+     "dzt[it[j]] += gt[j] * (m - dgt[j]);", [bpins.test_backward_matches_finite_differences]),
+    ("aux gradient misses the mean term", "dzt[e] += scale * p * (f[e] - q);",
+     "dzt[e] += scale * p * f[e];", [bpins.test_backward_matches_finite_differences]),
+    ("aux gradient not scaled by E", "const double scale = aux_coef * (double)E / (double)c->T;",
+     "const double scale = aux_coef / (double)c->T;", [bpins.test_backward_matches_finite_differences]),
+    ("output gradient not scaled by the gate", "const double dyo = g * elem(G, dtype, x_off + o);",
+     "const double dyo = elem(G, dtype, x_off + o);", [bpins.test_backward_matches_finite_differences]),
+    ("up gradient uses the gate pre-activation", "const double db = du[i] * silu;",
+     "const double db = du[i] * a[i];", [bpins.test_backward_matches_finite_differences]),
+    ("router term missing from dx",
+     "            dxt[cc] += s;\n        }\n        for (int e = 0; e < E; ++e) db[e] += dzt[e];",
+     "            (void)s;\n        }\n        for (int e = 0; e < E; ++e) db[e] += dzt[e];", [bpins.test_backward_matches_finite_differences]),
+    ("dropped assignment differentiated",
+     "            if (!keep[t * k + j]) continue;\n            const int64_t e = expert[t * k + j];\n"
+     "            dg[j] = ffn_backward(d, h, c->dtype, x, t * d, G, gate[t * k + j], w1, w3, w2,\n"
+     "                                 e * d * h, e * h * d, dw1,",
+     "            const int64_t e = expert[t * k + j];\n"
+     "            dg[j] = ffn_backward(d, h, c->dtype, x, t * d, G, gate[t * k + j], w1, w3, w2,\n"
+     "                                 e * d * h, e * h * d, dw1,", [bpins.test_backward_matches_finite_differences]),
+    ("gate gradient sent to the serving expert",
+     "router_logit_grad(c, z + t * E, idx + t * k, gate + t * k, dg, f, aux_coef, dzt);\n"
+     "        for (int cc = 0; cc < d; ++cc) {\n            const double xc",
+     "router_logit_grad(c, z + t * E, expert + t * k, gate + t * k, dg, f, aux_coef, dzt);\n"
+     "        for (int cc = 0; cc < d; ++cc) {\n            const double xc", [bpins.test_backward_matches_finite_differences]),
+    ("router weight gradient transposed", "dWr[(int64_t)cc * E + e] += xc * dzt[e];",
+     "dWr[(int64_t)e * d + cc] += xc * dzt[e];", [bpins.test_backward_matches_finite_differences]),
+    ("down-projection gradient uses the gated input", "if (dw1) dw2[row + o] += u[i] * dyo;",
+     "if (dw1) dw2[row + o] += a[i] * dyo;", [bpins.test_backward_matches_finite_differences]),
 ]
 
 
