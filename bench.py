@@ -10,7 +10,9 @@ runs its own batch (weak scaling; weights replicated) and the per-rank
 routing statistics are summed across ranks with one NCCL all-reduce.
 
 Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
-instead, on a bounded sample of the same workload.
+instead, on a bounded sample of the same workload.  `--backward` (1 GPU) times
+a training step instead: moe_forward with the pre-activations kept, then
+moe_backward (gradients of <G, out> + 0.01 aux for every input and weight).
 """
 
 import argparse
@@ -63,7 +65,12 @@ def parse():
                    help="override the expert hidden width (small profiling cases only)")
     p.add_argument("--graph", action="store_true",
                    help="capture one step in a CUDA graph and replay it (1 GPU)")
+    p.add_argument("--backward", action="store_true",
+                   help="time forward + backward (a training step) instead of the forward (1 GPU)")
     return p.parse_args()
+
+
+AUX_COEF = 0.01
 
 
 # ---------------------------------------------------------------- helpers
@@ -95,12 +102,42 @@ def algorithmic(wl, kept):
     return flops, byt, N, active
 
 
+def backward_algorithmic(wl, kept):
+    """Algorithmic FLOPs and bytes of one backward pass: the backward GEMMs
+    (12 N d h, shared 12 T d S hs), the router's two products (4 T d E); the
+    bytes read (the backward-layout weights of active experts, G, x) and
+    written (fp32 gradients of every weight, dx)."""
+    d, h, E, T = wl.d, wl.h, wl.E, wl.T
+    N = int(sum(kept))
+    active = sum(1 for n in kept if n > 0)
+    hs = wl.n_shared * wl.h_shared
+    flops = 12.0 * N * d * h + 12.0 * T * d * hs + 4.0 * T * d * E
+    byt = (active * 3 * d * h * 2 + 3 * d * hs * 2 + 2 * T * d * 2
+           + E * 3 * d * h * 4 + 3 * d * hs * 4 + d * E * 4 + T * d * 4)
+    return flops, byt
+
+
 def kernel_work(name, wl, kept, splits):
     """Algorithmic work of one launch of a GEMM kernel: (bound, amount, unit)."""
     d, h = wl.d, wl.h
     ab = 2 if wl.dtype == "bf16" else 4
     N = int(sum(kept))
     active = sum(1 for n in kept if n > 0)
+    E = wl.E
+    # backward GEMMs (token-major tiles): the binding one of FLOPs and bytes
+    kt = N + 63 * active
+    bwd = {
+        "gemm_dgate": (2.0 * N * d * h, active * h * d * 2 + N * d * 2 + 4 * N * 2 * h),
+        "gemm_dx": (4.0 * N * d * h, active * 2 * h * d * 2 + N * 2 * h * 2 + N * d * 4),
+        "gemm_dw2": (2.0 * N * d * h, E * d * h * 4 + (d + h) * kt * 2),
+        "gemm_dw13": (4.0 * N * d * h, E * 2 * h * d * 4 + (2 * h + d) * kt * 2),
+    }
+    if name in bwd:
+        fl, by = bwd[name]
+        pk, _ = peaks()
+        if fl / (pk["bf16_tflops"] * 1e12) >= by / (pk["hbm_gbs"] * 1e9):
+            return "tensor", fl, "flops"
+        return "hbm", by, "bytes"
     C = min(B.moe_capacity(B.config_of(wl)), wl.T)
     swapped = C <= 256
     if name == "gemm_gateup":
@@ -193,18 +230,22 @@ def cpu_threads():
 
 # ---------------------------------------------------------------- inputs
 
-def build_inputs(wl, rank, world, dev, keep_host):
-    """Per-rank tokens; expert weights drawn on rank 0 and broadcast."""
+def build_inputs(wl, rank, world, dev, keep_host, train=False):
+    """Per-rank tokens; expert weights drawn on rank 0 and broadcast.  With
+    train, also the backward-layout weights (one GPU)."""
     Wr = I.router_weights(wl)
     bias = I.router_bias(wl)
     x, _ = I.tokens(wl, Wr=Wr, b=bias, stream=dp.token_stream(rank))
-    cfg = B.config_of(wl)
+    cfg = B.config_of(wl, train=train)
+    Wb = (None, None, None, None)
     host = {"x": x, "Wr": Wr, "bias": bias}
     dt = I.torch_dtype(wl.dtype)
     if rank == 0:
         w = I.expert_weights(wl)
         w1, w3, w2 = (w[k].to(dev) for k in ("w1", "w3", "w2"))
         W13, W2p = B.pack_weights(cfg, w1, w3, w2)
+        if train:
+            Wb = B.pack_weights_backward(cfg, w1, w3, w2) + (None, None)
         del w1, w3, w2
         if keep_host:
             host.update(w)
@@ -213,6 +254,8 @@ def build_inputs(wl, rank, world, dev, keep_host):
             s = I.expert_weights(wl, shared=True)
             s1, s3, s2 = (s[k].to(dev) for k in ("w1", "w3", "w2"))
             W13s, W2s = B.pack_weights(cfg, s1, s3, s2, shared=True)
+            if train:
+                Wb = Wb[:2] + B.pack_weights_backward(cfg, s1, s3, s2, shared=True)
             del s1, s3, s2
             if keep_host:
                 host.update({"w1s": s["w1"], "w3s": s["w3"], "w2s": s["w2"]})
@@ -228,7 +271,9 @@ def build_inputs(wl, rank, world, dev, keep_host):
         dp.broadcast_weights([W13, W2p, W13s, W2s], src=0)
     torch.cuda.synchronize()
     dev_in = {"x": x.to(dev), "Wr": Wr.to(dev), "bias": bias.to(dev) if bias is not None else None}
-    return cfg, host, dev_in, (W13, W2p, W13s, W2s)
+    if train:
+        dev_in["G"] = I.grad_out(wl).to(dev)
+    return cfg, host, dev_in, (W13, W2p, W13s, W2s), Wb
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -343,10 +388,15 @@ def main():
         wl = wl.scaled(h=args.hidden, name=f"{wl.name}_h{args.hidden}")
     if args.overflow:
         wl = wl.scaled(overflow=args.overflow)
-    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
-    cfg, host, g, W = build_inputs(wl, rank, world, dev, keep_host=want_cpu)
+    if args.backward and world > 1:
+        raise SystemExit("--backward runs on one GPU")
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward
+    cfg, host, g, W, Wb = build_inputs(wl, rank, world, dev, keep_host=want_cpu,
+                                       train=args.backward)
     W13, W2p, W13s, W2s = W
+    W13t, W2t, W13st, W2st = Wb
     bufs = B.alloc_layer(cfg, dev)
+    grads = B.alloc_grads(cfg, dev) if args.backward else None
     sums = torch.zeros(dp.sums_len(wl.E), dtype=torch.float64, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -355,6 +405,9 @@ def main():
             B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
                           bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
                           bufs["slot_of"], bufs["stats"], bufs["ws"])
+            if args.backward:
+                B.backward(cfg, g["G"], AUX_COEF, g["x"], g["Wr"], g["bias"], W13t, W2t, W13st,
+                           W2st, bufs, grads)
         else:
             B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
                           bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
@@ -364,6 +417,10 @@ def main():
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
+    c0 = B.moe_launch_count()
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = B.moe_launch_count() - c0
     status = B.moe_read_device_status(bufs["ws"])
     if status != 0:
         raise SystemExit(f"device status {status} after warm-up")
@@ -384,6 +441,7 @@ def main():
         torch.cuda.synchronize()
     run = graph.replay if graph is not None else step
     trace_on = not args.no_trace and graph is None
+    calls = 2 if args.backward else 1  # library calls per step that launch kernels
 
     # ------------------------------------------------ timed region (device resident)
     clocks = ClockSampler(local)
@@ -391,17 +449,21 @@ def main():
     time.sleep(0.3)
     if trace_on:
         # bracket only the dominant kernel (the one the roofline is quoted on)
-        B.moe_trace_begin(args.steps, None if args.trace_all else "gemm_gateup")
+        only = None if (args.trace_all or args.backward) else "gemm_gateup"
+        B.moe_trace_begin(args.steps * calls, only)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    n0 = B.moe_launch_count()
     ev0.record(stream)
     for _ in range(args.steps):
         run()
     ev1.record(stream)
     torch.cuda.synchronize()
+    # kernels launched in the timed region (a replayed graph launches its captured step)
+    launched = (B.moe_launch_count() - n0) if graph is None else launches_per_step * args.steps
     if dist:
         dist.barrier()
     clk = clocks.stop()
@@ -420,11 +482,18 @@ def main():
         out_h = torch.empty(bufs["out"].shape, dtype=bufs["out"].dtype).pin_memory()
         st_h = torch.empty(bufs["stats"].shape, dtype=bufs["stats"].dtype).pin_memory()
 
+        G_h = g["G"].cpu().pin_memory() if args.backward else None
+        dx_h = grads["dx"].cpu().pin_memory() if args.backward else None
+
         def e2e_step():
             g["x"].copy_(x_h, non_blocking=True)
+            if args.backward:
+                g["G"].copy_(G_h, non_blocking=True)
             step()
             out_h.copy_(bufs["out"], non_blocking=True)
             st_h.copy_(bufs["stats"], non_blocking=True)
+            if args.backward:
+                dx_h.copy_(grads["dx"], non_blocking=True)
 
         for _ in range(3):
             e2e_step()
@@ -441,22 +510,30 @@ def main():
         e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
         if dist:
             dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        h2d = x_h.numel() * x_h.element_size()
+        d2h = out_h.numel() * out_h.element_size() + st_h.numel() * st_h.element_size()
+        if args.backward:
+            h2d += G_h.numel() * G_h.element_size()
+            d2h += dx_h.numel() * dx_h.element_size()
         e2e = {"value": world * wl.T * args.steps / (float(e_ms.item()) / 1000.0), "unit": UNIT,
-               "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
-               "d2h_bytes_per_step": out_h.numel() * out_h.element_size()
-               + st_h.numel() * st_h.element_size()}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ------------------------------------------------ report
     kept = bufs["kept"].cpu().tolist()
     stats = B.stats_dict(bufs["stats"])
     pk, pk_kind = peaks()
     flops, byts, N, active = algorithmic(wl, kept)
+    if args.backward:
+        bf, bb = backward_algorithmic(wl, kept)
+        flops, byts = flops + bf, byts + bb
     t_step = ms_max / 1000.0 / args.steps
     roof_t = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
     kernels = {n: {"launches": c, "ms_per_launch": t / c} for n, c, t in trace}
-    top = max(trace, key=lambda r: r[2]) if trace else None
-    roofline = None
     splits = B.moe_ffn_splits(cfg)
+    # the dominant kernel among those with a stated algorithmic work (the GEMMs)
+    known = [r for r in trace if kernel_work(r[0], wl, kept, splits)]
+    top = max(known, key=lambda r: r[2]) if known else None
+    roofline = None
     if top is not None:
         name, launches, tot_ms = top
         per = tot_ms / launches / 1000.0
@@ -472,9 +549,8 @@ def main():
                         "unit": unit, "frac": ach / peak, "peak_source": pk_kind,
                         "algorithmic_per_launch": amount,
                         "traffic": traffic_from_profile(name, wl.name)}
-    launches_total = sum(c for _, c, _ in trace)
     line = {
-        "metric": METRIC,
+        "metric": METRIC if not args.backward else METRIC + ", training step (forward + backward)",
         "value": world * wl.T * args.steps / (ms_max / 1000.0),
         "unit": UNIT,
         "n_gpus": world,
@@ -497,7 +573,7 @@ def main():
                            "frac": roof_t / t_step, "kept_assignments": N,
                            "active_experts": active},
         "kernels": kernels,
-        "gpu_launches": launches_total,
+        "gpu_launches": launched,
         "clocks": clk,
         "e2e": e2e,
         "stats": stats,

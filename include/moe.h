@@ -85,7 +85,10 @@ typedef enum { MOE_OVERFLOW_DROP = 0, MOE_OVERFLOW_REROUTE = 1 } moe_overflow;
  *   cf_num / cf_den  capacity factor; cf_den == 0 means no capacity limit
  *   act_dtype MOE_BF16 (tensor-core path) or MOE_F32 (fp32 SIMT path; no TF32)
  *   has_bias  1 if the router has a bias vector b[E]
- *   overflow  moe_overflow (0 = drop)                                       */
+ *   overflow  moe_overflow (0 = drop)
+ *   train     1: moe_forward also keeps in ws what moe_backward reads (the
+ *             gate/up pre-activations, bf16); bf16 configs only.  The
+ *             workspace grows accordingly (moe_workspace_size).          */
 typedef struct {
     int64_t T;
     int32_t d, h, E, k, n_shared, h_shared;
@@ -93,6 +96,7 @@ typedef struct {
     int32_t act_dtype;
     int32_t has_bias;
     int32_t overflow;
+    int32_t train;
 } moe_config;
 
 /* Routing statistics [MoE routing fully explained, "Easy explanation" ¶4 and
@@ -144,7 +148,14 @@ MOE_API const char* moe_last_error(void);
  * which = 1 (shared): w1, w3 [S][d][hs], w2 [S][hs][d] are fused into one
  *   expert of width S*hs (hidden index s*hs + j) and packed the same way:
  *   W13 [2*S*hs][d], W2p [d][S*hs].
- * All in act dtype.  One-time transform; inputs are not modified. */
+ * which = 2 (routed, backward layout; bf16): the transposes the backward
+ *   GEMMs read, W13 <- W13t [E][d][2h] (row c holds w1[c][:] and w3[c][:] with
+ *   the same 128-wide block interleave along 2h) and W2p <- W2t [E][h][d]
+ *   (= w2, the model dim contiguous).
+ * which = 3 (shared, backward layout; bf16): the fused shared expert the same
+ *   way, W13t [d][2*S*hs] and W2t [S*hs][d].
+ * All in act dtype.  Inputs are not modified.  Training re-packs after each
+ * weight update (the packed tensors are the layer's parameters as stored). */
 MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const void* w3,
                      const void* w2, void* W13, void* W2p, void* stream);
 
@@ -227,6 +238,46 @@ MOE_API int moe_forward(const moe_config* cfg, const void* x, const float* Wr, c
                 int32_t* kept, int32_t* slot_of, moe_stats* stats, void* ws, size_t ws_bytes,
                 void* stream);
 
+/* ---- backward pass ------------------------------------------------------ */
+
+/* Bytes of the second workspace moe_backward needs for this config. */
+MOE_API int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes);
+
+/* Gradients of the layer [the softmax weighting and the load-balancing loss
+ * the pages describe are what training acts on: MoE routing fully explained,
+ * "Easy explanation" ¶2 and ¶4] for the loss
+ *   L = sum_t <grad_out_t, out_t> + aux_coef * aux_loss,
+ * after a moe_forward of the same batch with cfg->train = 1 (bf16 only).
+ * Readings: the top-k choice, the capacity decision and the routed counts f_e
+ * are piecewise constant and carry no gradient (aux reaches the router
+ * through P_e); gates are not renormalised after a drop, so a dropped
+ * assignment has gate gradient 0 but its logit still receives the
+ * softmax-over-k terms; under reroute the gate gradient goes to the router's
+ * chosen expert while the serving expert's FFN is differentiated.
+ * Inputs:
+ *   grad_out [T][d] act dtype; aux_coef the weight of the aux loss
+ *   x, Wr, bias        the forward's inputs (bias ignored unless has_bias)
+ *   W13t, W2t          routed weights in the backward layout (pack which = 2)
+ *   W13st, W2st        shared expert, backward layout (pack which = 3), or NULL
+ *   topk_idx, topk_gate, routed, kept, slot_of   the forward's outputs
+ *   ws, ws_bytes       the forward's workspace, unchanged since that call
+ * Outputs (device, fp32, overwritten):
+ *   dx [T][d]; dWr [d][E]; db [E] (NULL allowed; written only with has_bias);
+ *   dW13 [E][2h][d] and dW2p [E][d][h] in the forward packed layout (which = 0);
+ *   dW13s [2*S*hs][d], dW2s [d][S*hs] (shared; NULL when n_shared == 0);
+ *   dlogits [T][E] (optional, NULL = not written): dL/dz.
+ * bws, bws_bytes: the backward workspace (moe_backward_workspace_size),
+ * 256-byte aligned.  Asynchronous on `stream`; bounded waits record
+ * MOE_ERR_TIMEOUT in ws's status word like the forward. */
+MOE_API int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef,
+                         const void* x, const float* Wr, const float* bias, const void* W13t,
+                         const void* W2t, const void* W13st, const void* W2st,
+                         const int32_t* topk_idx, const float* topk_gate,
+                         const int32_t* routed, const int32_t* kept, const int32_t* slot_of,
+                         void* ws, size_t ws_bytes, float* dx, float* dWr, float* db,
+                         float* dW13, float* dW2p, float* dW13s, float* dW2s, float* dlogits,
+                         void* bws, size_t bws_bytes, void* stream);
+
 /* ---- routing without a workspace ----------------------------------------- */
 
 /* The pages have no counterpart to this call; it exists for callers that
@@ -256,6 +307,11 @@ MOE_API int moe_route_static(const moe_config* cfg, const void* x, const float* 
 /* Copies the device status word from ws to *status (MOE_OK or
  * MOE_ERR_TIMEOUT) and clears it.  This call synchronises `stream`. */
 MOE_API int moe_read_device_status(const void* ws, int32_t* status, void* stream);
+
+/* Kernels this library has launched since it was loaded, over all threads
+ * and devices (a running count; the difference of two reads counts the
+ * launches in between). */
+MOE_API int moe_launch_count(uint64_t* n);
 
 /* Upper bound, in nanoseconds, on every device-side wait of the tensor-core
  * kernels (default 2e9).  A wait that runs out records MOE_ERR_TIMEOUT in

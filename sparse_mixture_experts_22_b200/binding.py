@@ -27,7 +27,8 @@ EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_split
            "moe_last_error", "moe_pack_weights", "moe_route", "moe_dispatch", "moe_expert_ffn",
            "moe_combine", "moe_aux_stats", "moe_stats_sums", "moe_stats_finalize", "moe_forward",
            "moe_read_device_status", "moe_set_wait_limit_ns", "moe_set_test_stall",
-           "moe_trace_begin", "moe_trace_end"]
+           "moe_trace_begin", "moe_trace_end", "moe_backward_workspace_size", "moe_backward",
+           "moe_launch_count"]
 
 
 class MoEError(RuntimeError):
@@ -50,6 +51,7 @@ class MoEConfig(ctypes.Structure):
         ("act_dtype", ctypes.c_int32),
         ("has_bias", ctypes.c_int32),
         ("overflow", ctypes.c_int32),
+        ("train", ctypes.c_int32),
     ]
 
 
@@ -87,6 +89,10 @@ def load() -> ctypes.CDLL:
             "moe_set_test_stall": [I],
             "moe_trace_begin": [I, ctypes.c_char_p],
             "moe_trace_end": [P, P, P, I, P],
+            "moe_backward_workspace_size": [C, P],
+            "moe_launch_count": [P],
+            "moe_backward": [C, P, ctypes.c_float, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P,
+                             P, P, P, P, P, P, P, P, S, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -127,16 +133,16 @@ OVERFLOW = {"drop": 0, "reroute": 1}
 
 
 def make_config(T, d, h, E, k, n_shared=0, h_shared=0, cf=None, dtype="bf16",
-                has_bias=False, overflow="drop") -> MoEConfig:
+                has_bias=False, overflow="drop", train=False) -> MoEConfig:
     num, den = (0, 0) if cf is None else cf
     return MoEConfig(T, d, h, E, k, n_shared, h_shared, num, den,
                      MOE_BF16 if dtype == "bf16" else MOE_F32, 1 if has_bias else 0,
-                     OVERFLOW[overflow])
+                     OVERFLOW[overflow], 1 if train else 0)
 
 
-def config_of(wl: Workload, T: Optional[int] = None) -> MoEConfig:
+def config_of(wl: Workload, T: Optional[int] = None, train: bool = False) -> MoEConfig:
     return make_config(wl.T if T is None else T, wl.d, wl.h, wl.E, wl.k, wl.n_shared,
-                       wl.h_shared, wl.cf, wl.dtype, wl.has_bias, wl.overflow)
+                       wl.h_shared, wl.cf, wl.dtype, wl.has_bias, wl.overflow, train)
 
 
 def act_dtype(cfg: MoEConfig) -> torch.dtype:
@@ -223,9 +229,32 @@ def moe_forward(cfg, x, Wr, bias, W13, W2p, W13s, W2s, out, topk_idx, topk_gate,
                               ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def moe_backward_workspace_size(cfg: MoEConfig) -> int:
+    v = ctypes.c_size_t()
+    _check(load().moe_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(v)))
+    return v.value
+
+
+def moe_backward(cfg, grad_out, aux_coef, x, Wr, bias, W13t, W2t, W13st, W2st, topk_idx,
+                 topk_gate, routed, kept, slot_of, ws, dx, dWr, db, dW13, dW2p, dW13s, dW2s,
+                 dlogits, bws, stream=None):
+    _check(load().moe_backward(
+        ctypes.byref(cfg), _p(grad_out), float(aux_coef), _p(x), _p(Wr), _p(bias), _p(W13t),
+        _p(W2t), _p(W13st), _p(W2st), _p(topk_idx), _p(topk_gate), _p(routed), _p(kept),
+        _p(slot_of), _p(ws), ws.numel() * ws.element_size(), _p(dx), _p(dWr), _p(db), _p(dW13),
+        _p(dW2p), _p(dW13s), _p(dW2s), _p(dlogits), _p(bws), bws.numel() * bws.element_size(),
+        _stream(stream)))
+
+
 def moe_read_device_status(ws, stream=None) -> int:
     v = ctypes.c_int32()
     _check(load().moe_read_device_status(_p(ws), ctypes.byref(v), _stream(stream)))
+    return v.value
+
+
+def moe_launch_count() -> int:
+    v = ctypes.c_uint64()
+    _check(load().moe_launch_count(ctypes.byref(v)))
     return v.value
 
 
@@ -294,3 +323,50 @@ def forward(cfg: MoEConfig, x, Wr, bias, W13, W2p, W13s=None, W2s=None, bufs=Non
                 bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
                 bufs["slot_of"], bufs["stats"] if with_stats else None, bufs["ws"], stream)
     return bufs
+
+
+def pack_weights_backward(cfg: MoEConfig, w1, w3, w2, shared: bool = False, stream=None):
+    """Backward-layout copies (W13t, W2t) of [n, d, hid] / [n, hid, d] weights."""
+    n, d, hid = w1.shape
+    if shared:
+        W13t = torch.empty((d, 2 * n * hid), dtype=w1.dtype, device=w1.device)
+        W2t = torch.empty((n * hid, d), dtype=w1.dtype, device=w1.device)
+    else:
+        W13t = torch.empty((n, d, 2 * hid), dtype=w1.dtype, device=w1.device)
+        W2t = torch.empty((n, hid, d), dtype=w1.dtype, device=w1.device)
+    moe_pack_weights(cfg, 3 if shared else 2, w1, w3, w2, W13t, W2t, stream)
+    return W13t, W2t
+
+
+def alloc_grads(cfg: MoEConfig, device="cuda") -> Dict[str, torch.Tensor]:
+    """Gradient outputs and backward workspace of one moe_backward call."""
+    T, E, d, h = cfg.T, cfg.E, cfg.d, cfg.h
+    f32 = dict(dtype=torch.float32, device=device)
+    g = {
+        "dx": torch.empty((T, d), **f32),
+        "dWr": torch.empty((d, E), **f32),
+        "db": torch.empty(E, **f32),
+        "dW13": torch.empty((E, 2 * h, d), **f32),
+        "dW2p": torch.empty((E, d, h), **f32),
+        "dlogits": torch.empty((T, E), **f32),
+        "bws": torch.empty(max(moe_backward_workspace_size(cfg), 256), dtype=torch.uint8,
+                           device=device),
+    }
+    if cfg.n_shared:
+        hsum = cfg.n_shared * cfg.h_shared
+        g["dW13s"] = torch.empty((2 * hsum, d), **f32)
+        g["dW2s"] = torch.empty((d, hsum), **f32)
+    return g
+
+
+def backward(cfg: MoEConfig, grad_out, aux_coef, x, Wr, bias, W13t, W2t, W13st, W2st, bufs,
+             grads=None, stream=None) -> Dict[str, torch.Tensor]:
+    """One moe_backward call after forward(...) filled `bufs` (cfg.train = 1)."""
+    if grads is None:
+        grads = alloc_grads(cfg, x.device)
+    moe_backward(cfg, grad_out, aux_coef, x, Wr, bias if cfg.has_bias else None, W13t, W2t,
+                 W13st, W2st, bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
+                 bufs["slot_of"], bufs["ws"], grads["dx"], grads["dWr"], grads["db"],
+                 grads["dW13"], grads["dW2p"], grads.get("dW13s"), grads.get("dW2s"),
+                 grads["dlogits"], grads["bws"], stream)
+    return grads

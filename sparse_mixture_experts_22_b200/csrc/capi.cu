@@ -9,6 +9,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -52,10 +53,17 @@ int report_error(int code, const char* text) {
         if (_s != MOE_OK) return _s;    \
     } while (0)
 
+cudaError_t& last_launch_error() {
+    static thread_local cudaError_t e = cudaSuccess;
+    return e;
+}
+
 static int launched(int rc, const char* what) {
     if (rc == 0) return MOE_OK;
-    cudaError_t e = cudaGetLastError();
-    return fail(MOE_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    cudaError_t e = last_launch_error();
+    last_launch_error() = cudaSuccess;
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return fail(MOE_ERR_CUDA, "%s: launch failed: %s (%d)", what, cudaGetErrorString(e), (int)e);
 }
 
 // ---------------------------------------------------------------- plan
@@ -81,6 +89,11 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     if (c.overflow != MOE_OVERFLOW_DROP && c.overflow != MOE_OVERFLOW_REROUTE) {
         *why = "overflow must be MOE_OVERFLOW_DROP or MOE_OVERFLOW_REROUTE";
         return MOE_ERR_ARG;
+    }
+    if (c.train != 0 && c.train != 1) { *why = "train must be 0 or 1"; return MOE_ERR_ARG; }
+    if (c.train && c.act_dtype != MOE_BF16) {
+        *why = "train = 1 (backward pass) needs act_dtype MOE_BF16";
+        return MOE_ERR_UNSUPPORTED;
     }
 
     Plan& P = *p;
@@ -168,7 +181,37 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.off_Hs = take(P.S ? (size_t)c.T * P.hsum * P.act_bytes : 0);
     P.off_ys = take(P.S ? (size_t)c.T * c.d * 4 : 0);
     P.off_sums = take((size_t)(2 + 3 * c.E) * 8);
+    P.train = c.train != 0;
+    P.off_AB = take(P.train ? (size_t)P.perm_rows * 2 * c.h * 2 : 0);
+    P.off_ABs = take(P.train && P.S ? (size_t)c.T * 2 * P.hsum * 2 : 0);
     P.total = o;
+
+    // backward workspace
+    P.kt = c.T > 0 ? (kept_max + (int64_t)c.E * 63 + 63) / 64 * 64 : 0;
+    P.tp = (c.T + 63) / 64 * 64;
+    P.wr_chunks = P.train ? wr_grad_chunks(c.T, c.d, c.E) : 1;
+    o = 0;
+    const bool tr = P.train;
+    P.b_dY = take(tr ? (size_t)P.perm_rows * c.d * 2 : 0);
+    P.b_dg = take(tr ? (size_t)c.T * c.k * 4 : 0);
+    P.b_dz = take(tr ? (size_t)c.T * c.E * 4 : 0);
+    P.b_dAB = take(tr ? (size_t)P.perm_rows * 2 * c.h * 2 : 0);
+    P.b_dXp = take(tr ? (size_t)P.perm_rows * c.d * 4 : 0);
+    P.b_kofs = take(tr ? (size_t)(c.E + 1) * 4 : 0);
+    P.b_XT = take(tr ? (size_t)c.d * P.kt * 2 : 0);
+    P.b_dYT = take(tr ? (size_t)c.d * P.kt * 2 : 0);
+    P.b_HT = take(tr ? (size_t)c.h * P.kt * 2 : 0);
+    P.b_dABT = take(tr ? (size_t)2 * c.h * P.kt * 2 : 0);
+    const bool ts = tr && P.S > 0;
+    P.b_dABs = take(ts ? (size_t)c.T * 2 * P.hsum * 2 : 0);
+    P.b_dXs = take(ts ? (size_t)c.T * c.d * 4 : 0);
+    P.b_GT = take(ts ? (size_t)c.d * P.tp * 2 : 0);
+    P.b_xT = take(ts ? (size_t)c.d * P.tp * 2 : 0);
+    P.b_HsT = take(ts ? (size_t)P.hsum * P.tp * 2 : 0);
+    P.b_dABsT = take(ts ? (size_t)2 * P.hsum * P.tp * 2 : 0);
+    P.b_wrpart = take(tr ? (size_t)P.wr_chunks * (c.d + 1) * c.E * 4 : 0);
+    P.b_dXr = take(tr ? (size_t)c.T * c.d * 4 : 0);
+    P.b_total = o;
     return MOE_OK;
 }
 
@@ -246,6 +289,12 @@ static int tmap_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
                     (long long)rows, (long long)cols);
     return MOE_OK;
 }
+
+// ---------------------------------------------------------------- launch count
+
+static std::atomic<uint64_t> g_launches{0};
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 // ---------------------------------------------------------------- limits and tracing
 
@@ -511,8 +560,8 @@ static int step_route_dispatch(const Plan& P, const Device& dv, const void* x, c
 static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
                       const int32_t* rows, const int32_t* offs, int dense_rows, const void* act,
                       int64_t act_rows, const void* W13, const void* W2p, int hid, void* H,
-                      float* y, int splits, int nt_max, int32_t* status, cudaStream_t st,
-                      const char* tag1, const char* tag2) {
+                      void* AB, float* y, int splits, int nt_max, int32_t* status,
+                      cudaStream_t st, const char* tag1, const char* tag2) {
     const bool tok = path == PATH_TOKEN_MAJOR;
     CUtensorMap m_act, m_w;
     TcArgs a;
@@ -538,6 +587,8 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.out = H;
     a.out_ld = hid;
     a.split_stride = 0;
+    a.aux = AB;  // pre-activations for the backward pass (null: not kept)
+    a.aux_ld = 2 * (int64_t)hid;
     a.stages = tc_max_stages(mode1, 256, nt_max, groups, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag1);
@@ -556,6 +607,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.out = y;
     a.out_ld = P.d;
     a.split_stride = act_rows * (int64_t)P.d;
+    a.aux = nullptr;
     a.stages = tc_max_stages(mode2, bn, nt_max, groups, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag2);
@@ -584,8 +636,9 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
                          "f32_down"));
         trace_mark(st, "f32_down");
     } else {
+        void* AB = P.train ? at<void>(ws, P.off_AB) : nullptr;
         MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, 0, x_perm, P.perm_rows, W13, W2p,
-                           P.h, H, y_perm, P.splits, P.nt_max, status, st, "gemm_gateup",
+                           P.h, H, AB, y_perm, P.splits, P.nt_max, status, st, "gemm_gateup",
                            "gemm_down"));
     }
     if (P.S > 0) {
@@ -604,9 +657,10 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
             trace_mark(st, "f32_shared_down");
         } else {
             const int nt = (int)((P.T + 15) / 16 * 16);
+            void* ABs = P.train ? at<void>(ws, P.off_ABs) : nullptr;
             MOE_TRY(run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, (int)P.T, x, P.T, W13s,
-                               W2s, P.hsum, Hs, y_shared, 1, nt, status, st, "gemm_shared_gateup",
-                               "gemm_shared_down"));
+                               W2s, P.hsum, Hs, ABs, y_shared, 1, nt, status, st,
+                               "gemm_shared_gateup", "gemm_shared_down"));
         }
     }
     return MOE_OK;
@@ -647,6 +701,112 @@ static int step_stats(const Plan& P, const int32_t* routed, const int32_t* kept,
     MOE_TRY(launched(launch_stats(stats_params(P, routed, kept, ws, sums, stats), st), "stats"));
     trace_mark(st, "stats");
     return MOE_OK;
+}
+
+// ---------------------------------------------------------------- backward steps
+
+// Backward GEMMs of one set of groups: dAB = SiLU*mul backward of dY W2t^T
+// (bf16, interleaved like AB), then dX = dAB W13t^T (fp32).
+static int run_tc_backward(const Plan& P, const Device& dv, int groups, const int32_t* rows,
+                           const int32_t* offs, int dense_rows, int64_t act_rows, const void* dY,
+                           const void* W2t, const void* AB, void* dAB, const void* W13t,
+                           float* dX, int hid, int32_t* status, cudaStream_t st, const char* tag1,
+                           const char* tag2) {
+    CUtensorMap m_act, m_w;
+    TcArgs a;
+    memset(&a, 0, sizeof a);
+    a.num_groups = groups;
+    a.group_rows = rows;
+    a.group_off = offs;
+    a.dense_rows = dense_rows;
+    a.status = status;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.test_stall = g_test_stall;
+    a.nt_max = 16;
+    a.splits = 1;
+
+    const int bn1 = hid % 256 == 0 ? 256 : 128;
+    MOE_TRY(tmap_bf16(&m_act, dY, act_rows, P.d, 128));
+    MOE_TRY(tmap_bf16(&m_w, W2t, (int64_t)groups * hid, P.d, bn1));
+    a.K = P.d;
+    a.n_feat = hid;
+    a.w_rows_per_group = hid;
+    a.out = dAB;
+    a.out_ld = 2 * (int64_t)hid;
+    a.aux = const_cast<void*>(AB);
+    a.aux_ld = 2 * (int64_t)hid;
+    a.stages = tc_max_stages(TC_DGATE_TOK, bn1, 16, groups, dv.smem_optin);
+    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    trace_pre(st, tag1);
+    MOE_TRY(launched(launch_tc_gemm(TC_DGATE_TOK, bn1, m_act, m_w, a, dv.sms, st), tag1));
+    trace_mark(st, tag1);
+
+    const int bn2 = P.d % 256 == 0 ? 256 : 128;
+    MOE_TRY(tmap_bf16(&m_act, dAB, act_rows, 2 * hid, 128));
+    MOE_TRY(tmap_bf16(&m_w, W13t, (int64_t)groups * P.d, 2 * hid, bn2));
+    a.K = 2 * hid;
+    a.n_feat = P.d;
+    a.w_rows_per_group = P.d;
+    a.out = dX;
+    a.out_ld = P.d;
+    a.aux = nullptr;
+    a.stages = tc_max_stages(TC_DOWN_TOK, bn2, 16, groups, dv.smem_optin);
+    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    trace_pre(st, tag2);
+    MOE_TRY(launched(launch_tc_gemm(TC_DOWN_TOK, bn2, m_act, m_w, a, dv.sms, st), tag2));
+    trace_mark(st, tag2);
+    return MOE_OK;
+}
+
+// Weight gradient C[g] [m_rows][n_rows] = AT[:, K_g] BT[:, K_g]^T, K_g the
+// g-th group's 64-aligned token range (rows[g] tokens; dense: one group).
+static int run_tc_wgrad(const Plan& P, const Device& dv, int groups, const int32_t* rows,
+                        int dense_rows, const void* AT, int m_rows, const void* BT, int n_rows,
+                        int64_t kcols, float* out, int32_t* status, cudaStream_t st,
+                        const char* tag) {
+    (void)P;
+    CUtensorMap m_a, m_b;
+    TcArgs a;
+    memset(&a, 0, sizeof a);
+    const int bn = n_rows % 256 == 0 ? 256 : 128;
+    MOE_TRY(tmap_bf16(&m_a, AT, m_rows, kcols, 128));
+    MOE_TRY(tmap_bf16(&m_b, BT, n_rows, kcols, bn));
+    a.num_groups = groups;
+    a.group_rows = rows;
+    a.dense_rows = dense_rows;
+    a.status = status;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.test_stall = g_test_stall;
+    a.nt_max = 16;
+    a.splits = 1;
+    a.n_feat = n_rows;
+    a.m_rows = m_rows;
+    a.out = out;
+    a.out_ld = n_rows;
+    a.group_stride = (int64_t)m_rows * n_rows;
+    a.stages = tc_max_stages(TC_WGRAD, bn, 16, groups, dv.smem_optin);
+    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+    trace_pre(st, tag);
+    MOE_TRY(launched(launch_tc_gemm(TC_WGRAD, bn, m_a, m_b, a, dv.sms, st), tag));
+    trace_mark(st, tag);
+    return MOE_OK;
+}
+
+static TransposeJob tjob(const void* src, int64_t src_ld, void* dst, int64_t dst_ld, int features,
+                         int groups, const int32_t* rows, const int32_t* off,
+                         const int32_t* kofs, int dense_rows) {
+    TransposeJob j;
+    j.src = src;
+    j.src_ld = src_ld;
+    j.dst = dst;
+    j.dst_ld = dst_ld;
+    j.features = features;
+    j.groups = groups;
+    j.rows = rows;
+    j.off = off;
+    j.kofs = kofs;
+    j.dense_rows = dense_rows;
+    return j;
 }
 
 }  // namespace moe
@@ -701,8 +861,10 @@ int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const voi
                      const void* w2, void* W13, void* W2p, void* stream) {
     Plan P;
     MOE_TRY(plan_or_fail(cfg, &P));
-    if (which != 0 && which != 1) return fail(MOE_ERR_ARG, "which must be 0 (routed) or 1 (shared)");
-    if (which == 1 && P.S == 0) return fail(MOE_ERR_ARG, "config has no shared experts");
+    if (which < 0 || which > 3)
+        return fail(MOE_ERR_ARG, "which must be 0/1 (routed/shared) or 2/3 (backward layouts)");
+    if ((which == 1 || which == 3) && P.S == 0) return fail(MOE_ERR_ARG, "config has no shared experts");
+    if (which >= 2 && !P.bf16) return fail(MOE_ERR_DTYPE, "backward layouts are bf16 only");
     MOE_TRY(need(w1, "w1"));
     MOE_TRY(need(w3, "w3"));
     MOE_TRY(need(w2, "w2"));
@@ -712,10 +874,27 @@ int moe_pack_weights(const moe_config* cfg, int which, const void* w1, const voi
     MOE_TRY(device_facts(&dv));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int eb = P.act_bytes;
-    const int n = which == 0 ? P.E : P.S;
-    const int hid = which == 0 ? P.h : P.hs;
+    const bool routed_set = which == 0 || which == 2;
+    const int n = routed_set ? P.E : P.S;
+    const int hid = routed_set ? P.h : P.hs;
     const int64_t d = P.d;
     const int64_t m13 = d * hid;  // elements of one w1 / w3 / w2 matrix
+    if (which >= 2) {
+        // W13t [n][d][2 hid] (routed) or [d][2 S hs] (shared): rows of w1 / w3
+        // with the gate/up interleave along the hidden axis; W2t = w2 itself
+        const bool routed = which == 2;
+        const int64_t ld = routed ? 2 * (int64_t)hid : 2 * (int64_t)P.hsum;
+        const int64_t dstride = routed ? d * 2 * hid : 0;
+        const int step = routed ? 0 : hid;
+        MOE_TRY(launched(launch_pack_cols(w1, W13, (int)d, hid, ld, 0, 0, n, m13, dstride, step, st),
+                         "pack"));
+        MOE_TRY(launched(launch_pack_cols(w3, W13, (int)d, hid, ld, 0, 1, n, m13, dstride, step, st),
+                         "pack"));
+        if (cudaMemcpyAsync(W2p, w2, (size_t)n * m13 * eb, cudaMemcpyDeviceToDevice, st) !=
+            cudaSuccess)
+            return fail(MOE_ERR_CUDA, "pack: copy of w2 failed");
+        return ok();
+    }
     if (which == 0) {
         // expert e: W13[e] [2h][d] and W2p[e] [d][h]
         MOE_TRY(launched(launch_pack(w1, W13, eb, (int)d, hid, d, 0, 0, n, m13, 2 * m13, 0, st),
@@ -908,6 +1087,175 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
     return ok();
 }
 
+int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes) {
+    if (!bytes) return fail(MOE_ERR_ARG, "bytes is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (!P.train) return fail(MOE_ERR_ARG, "the backward pass needs cfg->train = 1");
+    *bytes = P.b_total;
+    return ok();
+}
+
+int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef, const void* x,
+                 const float* Wr, const float* bias, const void* W13t, const void* W2t,
+                 const void* W13st, const void* W2st, const int32_t* topk_idx,
+                 const float* topk_gate, const int32_t* routed, const int32_t* kept,
+                 const int32_t* slot_of, void* ws, size_t ws_bytes, float* dx, float* dWr,
+                 float* db, float* dW13, float* dW2p, float* dW13s, float* dW2s, float* dlogits,
+                 void* bws, size_t bws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (!P.train) return fail(MOE_ERR_ARG, "the backward pass needs cfg->train = 1");
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    if (!bws) return fail(MOE_ERR_ARG, "bws is NULL");
+    if (reinterpret_cast<uintptr_t>(bws) & 255)
+        return fail(MOE_ERR_ALIGN, "bws is not 256-byte aligned");
+    if (bws_bytes < P.b_total)
+        return fail(MOE_ERR_WORKSPACE, "backward workspace has %zu bytes; this config needs %zu",
+                    bws_bytes, P.b_total);
+    MOE_TRY(need(dWr, "dWr"));
+    MOE_TRY(need(dW13, "dW13"));
+    MOE_TRY(need(dW2p, "dW2p"));
+    MOE_TRY(maybe(db, "db"));
+    MOE_TRY(maybe(dlogits, "dlogits"));
+    if (P.S > 0) {
+        MOE_TRY(need(dW13s, "dW13s"));
+        MOE_TRY(need(dW2s, "dW2s"));
+    }
+    if (P.T > 0) {
+        MOE_TRY(need(grad_out, "grad_out"));
+        MOE_TRY(need(x, "x"));
+        MOE_TRY(need(Wr, "Wr"));
+        MOE_TRY(need(W13t, "W13t"));
+        MOE_TRY(need(W2t, "W2t"));
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(topk_gate, "topk_gate"));
+        MOE_TRY(need(routed, "routed"));
+        MOE_TRY(need(kept, "kept"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(need(dx, "dx"));
+        if (cfg->has_bias) MOE_TRY(need(bias, "bias"));
+        if (P.S > 0) {
+            MOE_TRY(need(W13st, "W13st"));
+            MOE_TRY(need(W2st, "W2st"));
+        }
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t T = P.T;
+    const int d = P.d, h = P.h, E = P.E, k = P.k;
+    if (T == 0) {
+        // nothing was routed: every gradient is zero
+        if (cudaMemsetAsync(dWr, 0, (size_t)d * E * 4, st) != cudaSuccess ||
+            (db && cfg->has_bias && cudaMemsetAsync(db, 0, (size_t)E * 4, st) != cudaSuccess) ||
+            cudaMemsetAsync(dW13, 0, (size_t)E * 2 * h * d * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(dW2p, 0, (size_t)E * d * h * 4, st) != cudaSuccess ||
+            (P.S && cudaMemsetAsync(dW13s, 0, (size_t)2 * P.hsum * d * 4, st) != cudaSuccess) ||
+            (P.S && cudaMemsetAsync(dW2s, 0, (size_t)d * P.hsum * 4, st) != cudaSuccess))
+            return fail(MOE_ERR_CUDA, "memset failed");
+        return ok();
+    }
+    trace_call_begin(st);
+    int32_t* status = at<int32_t>(ws, P.off_status);
+    const int32_t* offsets = at<int32_t>(ws, P.off_offsets);
+    const void* x_perm = at<void>(ws, P.off_xperm);
+    const void* H = at<void>(ws, P.off_H);
+    const float* y = at<float>(ws, P.off_y);
+    const void* AB = at<void>(ws, P.off_AB);
+    const float* z = at<float>(ws, P.off_logits);
+    void* dY = at<void>(bws, P.b_dY);
+    float* dg = at<float>(bws, P.b_dg);
+    float* dz = dlogits ? dlogits : at<float>(bws, P.b_dz);
+    void* dAB = at<void>(bws, P.b_dAB);
+    float* dXp = at<float>(bws, P.b_dXp);
+    int32_t* kofs = at<int32_t>(bws, P.b_kofs);
+    float* dXr = at<float>(bws, P.b_dXr);
+    const int splits = P.path == PATH_SWAP ? P.splits : 1;
+
+    // gate-scaled output gradients per kept slot, and the gate gradients
+    trace_pre(st, "bwd_gather");
+    MOE_TRY(launched(launch_bwd_gather(grad_out, y, splits, P.perm_rows * (int64_t)d, slot_of,
+                                       topk_gate, dY, dg, T, d, k, dv.sms, st),
+                     "bwd_gather"));
+    trace_mark(st, "bwd_gather");
+    // router logits: the forward left z with the bias added on these paths
+    const bool z_has_bias = P.router_kind == ROUTER_TC || P.reroute;
+    const float* b_add = (cfg->has_bias && !z_has_bias) ? bias : nullptr;
+    trace_pre(st, "router_bwd");
+    MOE_TRY(launched(launch_router_bwd(z, b_add, topk_idx, topk_gate, dg, routed, aux_coef, dz, T,
+                                       E, k, dv.sms, st),
+                     "router_bwd"));
+    trace_mark(st, "router_bwd");
+    trace_pre(st, "wr_grad");
+    MOE_TRY(launched(launch_wr_grad(x, dz, at<float>(bws, P.b_wrpart), dWr,
+                                    cfg->has_bias ? db : nullptr, T, d, E, st),
+                     "wr_grad"));
+    trace_mark(st, "wr_grad");
+    trace_pre(st, "dxr");
+    MOE_TRY(launched(launch_dxr(dz, Wr, dXr, T, d, E, st), "dxr"));
+    trace_mark(st, "dxr");
+
+    // routed experts: dAB, dX, then the weight gradients over each expert's tokens
+    MOE_TRY(run_tc_backward(P, dv, E, kept, offsets, 0, P.perm_rows, dY, W2t, AB, dAB, W13t, dXp, h,
+                            status, st, "gemm_dgate", "gemm_dx"));
+    trace_pre(st, "kofs");
+    MOE_TRY(launched(launch_kofs(kept, E, kofs, st), "kofs"));
+    trace_mark(st, "kofs");
+    void* XT = at<void>(bws, P.b_XT);
+    void* dYT = at<void>(bws, P.b_dYT);
+    void* HT = at<void>(bws, P.b_HT);
+    void* dABT = at<void>(bws, P.b_dABT);
+    TransposeJobs tj;
+    tj.n = 4;
+    tj.job[0] = tjob(x_perm, d, XT, P.kt, d, E, kept, offsets, kofs, 0);
+    tj.job[1] = tjob(dY, d, dYT, P.kt, d, E, kept, offsets, kofs, 0);
+    tj.job[2] = tjob(H, h, HT, P.kt, h, E, kept, offsets, kofs, 0);
+    tj.job[3] = tjob(dAB, 2 * h, dABT, P.kt, 2 * h, E, kept, offsets, kofs, 0);
+    trace_pre(st, "transpose");
+    MOE_TRY(launched(launch_transpose(tj, P.kt, st), "transpose"));
+    trace_mark(st, "transpose");
+    MOE_TRY(run_tc_wgrad(P, dv, E, kept, 0, dYT, d, HT, h, P.kt, dW2p, status, st, "gemm_dw2"));
+    MOE_TRY(run_tc_wgrad(P, dv, E, kept, 0, dABT, 2 * h, XT, d, P.kt, dW13, status, st,
+                         "gemm_dw13"));
+
+    // shared experts: gate 1, every token
+    float* dXs = nullptr;
+    if (P.S > 0) {
+        const void* Hs = at<void>(ws, P.off_Hs);
+        const void* ABs = at<void>(ws, P.off_ABs);
+        void* dABs = at<void>(bws, P.b_dABs);
+        dXs = at<float>(bws, P.b_dXs);
+        MOE_TRY(run_tc_backward(P, dv, 1, nullptr, nullptr, (int)T, T, grad_out, W2st, ABs, dABs,
+                                W13st, dXs, P.hsum, status, st, "gemm_shared_dgate",
+                                "gemm_shared_dx"));
+        void* GT = at<void>(bws, P.b_GT);
+        void* xT = at<void>(bws, P.b_xT);
+        void* HsT = at<void>(bws, P.b_HsT);
+        void* dABsT = at<void>(bws, P.b_dABsT);
+        TransposeJobs ts;
+        ts.n = 4;
+        ts.job[0] = tjob(grad_out, d, GT, P.tp, d, 1, nullptr, nullptr, nullptr, (int)T);
+        ts.job[1] = tjob(x, d, xT, P.tp, d, 1, nullptr, nullptr, nullptr, (int)T);
+        ts.job[2] = tjob(Hs, P.hsum, HsT, P.tp, P.hsum, 1, nullptr, nullptr, nullptr, (int)T);
+        ts.job[3] = tjob(dABs, 2 * P.hsum, dABsT, P.tp, 2 * P.hsum, 1, nullptr, nullptr, nullptr,
+                         (int)T);
+        trace_pre(st, "shared_transpose");
+        MOE_TRY(launched(launch_transpose(ts, P.tp, st), "shared_transpose"));
+        trace_mark(st, "shared_transpose");
+        MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, (int)T, GT, d, HsT, P.hsum, P.tp, dW2s, status, st,
+                             "gemm_shared_dw2"));
+        MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, (int)T, dABsT, 2 * P.hsum, xT, d, P.tp, dW13s,
+                             status, st, "gemm_shared_dw13"));
+    }
+
+    trace_pre(st, "combine_bwd");
+    MOE_TRY(launched(launch_combine_bwd(dXp, slot_of, dXs, dXr, dx, T, d, k, dv.sms, st),
+                     "combine_bwd"));
+    trace_mark(st, "combine_bwd");
+    return ok();
+}
+
 int moe_read_device_status(const void* ws, int32_t* status, void* stream) {
     MOE_TRY(need(ws, "ws"));
     if (!status) return fail(MOE_ERR_ARG, "status is NULL");
@@ -920,6 +1268,12 @@ int moe_read_device_status(const void* ws, int32_t* status, void* stream) {
     if (cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof v, st) != cudaSuccess)
         return fail(MOE_ERR_CUDA, "clearing the device status failed");
     *status = v;
+    return ok();
+}
+
+int moe_launch_count(uint64_t* n) {
+    if (!n) return fail(MOE_ERR_ARG, "n is NULL");
+    *n = g_launches.load(std::memory_order_relaxed);
     return ok();
 }
 

@@ -192,17 +192,20 @@ int launch_combine(const float* y, int splits, int64_t split_stride, const int32
     else
         combine_kernel<false><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
                                                       y_shared, out, T, d, k, s);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_stats(const StatsParams& a, cudaStream_t st) {
     stats_kernel<<<1, 256, 0, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStream_t st) {
     stats_finalize_kernel<<<1, 32, 0, st>>>(sums, E, k, reinterpret_cast<moe_stats*>(stats));
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64_t ld_dst,
@@ -217,7 +220,8 @@ int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64
         pack_kernel<float><<<grid, block, 0, st>>>(
             reinterpret_cast<const float*>(src), reinterpret_cast<float*>(dst), R, Cc, ld_dst,
             col_off, interleave, src_stride, dst_stride, col_step);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 }  // namespace moe

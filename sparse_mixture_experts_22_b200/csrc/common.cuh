@@ -213,6 +213,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 16 consecutive floats <-> 16 bf16 (round to nearest even); 16-byte aligned.
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float* v) {
+    uint4 o0, o1;
+    o0.x = pack_bf16x2(v[0], v[1]);
+    o0.y = pack_bf16x2(v[2], v[3]);
+    o0.z = pack_bf16x2(v[4], v[5]);
+    o0.w = pack_bf16x2(v[6], v[7]);
+    o1.x = pack_bf16x2(v[8], v[9]);
+    o1.y = pack_bf16x2(v[10], v[11]);
+    o1.z = pack_bf16x2(v[12], v[13]);
+    o1.w = pack_bf16x2(v[14], v[15]);
+    reinterpret_cast<uint4*>(dst)[0] = o0;
+    reinterpret_cast<uint4*>(dst)[1] = o1;
+}
+
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* src, float* v) {
+    const uint4 i0 = reinterpret_cast<const uint4*>(src)[0];
+    const uint4 i1 = reinterpret_cast<const uint4*>(src)[1];
+    const uint32_t w[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
 // Device status word codes (stored in the workspace).
 enum : int32_t { DEV_OK = 0, DEV_TIMEOUT = 7 };
 

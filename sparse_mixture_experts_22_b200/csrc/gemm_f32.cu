@@ -83,7 +83,8 @@ int launch_f32_gateup(const float* A, const float* W13, float* H, int num_groups
     dim3 grid((h + TILE - 1) / TILE, (unsigned)((rows_bound + TILE - 1) / TILE));
     f32_ffn_kernel<true><<<grid, dim3(TILE, TILE), 0, st>>>(
         A, W13, H, num_groups, group_rows, group_off, dense_rows, rows_bound, d, h, 2LL * h);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_f32_down(const float* H, const float* W2p, float* Y, int num_groups,
@@ -93,7 +94,8 @@ int launch_f32_down(const float* H, const float* W2p, float* Y, int num_groups,
     dim3 grid((d + TILE - 1) / TILE, (unsigned)((rows_bound + TILE - 1) / TILE));
     f32_ffn_kernel<false><<<grid, dim3(TILE, TILE), 0, st>>>(
         H, W2p, Y, num_groups, group_rows, group_off, dense_rows, rows_bound, h, d, (int64_t)d);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 }  // namespace moe

@@ -59,6 +59,8 @@ __host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, uint32
     switch (mode) {
         case TC_GATEUP_TOK:
         case TC_DOWN_TOK:
+        case TC_DGATE_TOK:
+        case TC_WGRAD:
             *a = BM * BK * 2;
             *b = bn * BK * 2;
             break;
@@ -126,10 +128,17 @@ __device__ __forceinline__ Unit decode_unit(const GroupTable& t, int u, const Tc
     x.kb0 = 0;
     x.kb1 = kblocks;
     x.ntok = 0;
-    if (MODE == TC_GATEUP_TOK) {
+    if (MODE == TC_GATEUP_TOK || MODE == TC_DGATE_TOK) {
         const int mtiles = (x.rows + BM - 1) / BM;
         x.mt = local % mtiles;
         x.nb = local / mtiles;
+    } else if (MODE == TC_WGRAD) {
+        // the group's reduction range: its tokens, at 64-aligned offset row0
+        const int mtiles = a.m_rows / BM;
+        x.mt = local % mtiles;
+        x.nb = local / mtiles;
+        x.kb0 = x.row0 / BK;
+        x.kb1 = x.kb0 + (x.rows + BK - 1) / BK;
     } else if (MODE == TC_DOWN_TOK) {
         // m tile fastest, then n tile, then K split
         const int mtiles = (x.rows + BM - 1) / BM;
@@ -159,7 +168,10 @@ __device__ __forceinline__ Unit decode_unit(const GroupTable& t, int u, const Tc
 
 template <int MODE, int BN>
 __device__ __forceinline__ int units_of_group(int rows, const TcArgs& a) {
+    // every weight-gradient tile is written, zeros for a group without tokens
+    if (MODE == TC_WGRAD) return (a.m_rows / BM) * (a.n_feat / BN);
     if (rows <= 0) return 0;
+    if (MODE == TC_DGATE_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / BN);
     if (MODE == TC_GATEUP_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / 128);
     if (MODE == TC_DOWN_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / BN) * a.splits;
     if (MODE == TC_GATEUP_SWAP) return a.n_feat / 128;
@@ -170,7 +182,8 @@ template <int MODE, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
-    constexpr bool TOK = (MODE == TC_GATEUP_TOK || MODE == TC_DOWN_TOK);
+    constexpr bool TOK = (MODE == TC_GATEUP_TOK || MODE == TC_DOWN_TOK ||
+                          MODE == TC_DGATE_TOK || MODE == TC_WGRAD);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (align_up(raw, 1024) - raw);
@@ -226,10 +239,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_relinquish();
     }
     if (warp == 2 && lane == 0) {
-        int acc = 0;
+        int acc = 0, koff = 0;
         for (int g = 0; g < groups; ++g) {
             int r = args.group_rows ? args.group_rows[g] : args.dense_rows;
             int o = args.group_off ? args.group_off[g] : 0;
+            if (MODE == TC_WGRAD) {
+                // groups follow one another along K, each padded to a multiple of BK
+                o = koff;
+                koff += (r + BK - 1) / BK * BK;
+            }
             g_rows[g] = r;
             g_off[g] = o;
             g_start[g] = acc;
@@ -270,10 +288,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const int kc = kb * BK;
                     if (TOK) {
                         mbar_arrive_expect_tx(&full[stage], (BM + BN) * BK * 2);
-                        tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
-                        tma_load_2d(sb, &tm_w, &full[stage], kc,
-                                    x.g * args.w_rows_per_group +
-                                        x.nb * (MODE == TC_GATEUP_TOK ? 256 : BN));
+                        if (MODE == TC_WGRAD) {
+                            // both operands hold every group along K
+                            tma_load_2d(sa, &tm_act, &full[stage], kc, x.mt * BM);
+                            tma_load_2d(sb, &tm_w, &full[stage], kc, x.nb * BN);
+                        } else {
+                            tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
+                            tma_load_2d(sb, &tm_w, &full[stage], kc,
+                                        x.g * args.w_rows_per_group +
+                                            x.nb * (MODE == TC_GATEUP_TOK ? 256 : BN));
+                        }
                     } else {
                         const int wa = (MODE == TC_GATEUP_SWAP) ? 2 * BM : BM;
                         mbar_arrive_expect_tx(&full[stage], (wa + x.ntok) * BK * 2);
@@ -377,12 +401,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const bool valid = r < x.rows;
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
                                      (int64_t)(x.row0 + r) * args.out_ld + x.nb * 128;
+                __nv_bfloat16* abrow =
+                    args.aux ? reinterpret_cast<__nv_bfloat16*>(args.aux) +
+                                   (int64_t)(x.row0 + r) * args.aux_ld + x.nb * 256
+                             : nullptr;
 #pragma unroll 1
                 for (int c = 0; c < 128; c += 16) {
                     float g[16], v[16];
                     tmem_ld16(t0 + c, g);
                     tmem_ld16(t0 + 128 + c, v);
                     tmem_ld_wait();
+                    if (valid && abrow) {
+                        // pre-activations kept for the backward pass
+                        store_bf16x16(abrow + c, g);
+                        store_bf16x16(abrow + 128 + c, v);
+                    }
                     if (valid) {
                         uint4 o0, o1;
                         o0.x = pack_bf16x2(silu_f(g[0]) * v[0], silu_f(g[1]) * v[1]);
@@ -417,6 +450,55 @@ __global__ void __launch_bounds__(THREADS, 1)
                                     make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
                     }
                 }
+            } else if (MODE == TC_DGATE_TOK) {
+                // dH[r][f] for BN hidden features f; with a = x w1, b = x w3 of
+                // the forward (AB, bf16): dA = dH b silu'(a), dB = dH silu(a),
+                // stored interleaved per 128-wide block like AB itself
+                const int r = x.mt * BM + row;
+                const bool valid = r < x.rows;
+                const int64_t rowoff = (int64_t)(x.row0 + r) * args.aux_ld;
+                const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(args.aux) + rowoff;
+                __nv_bfloat16* dab = reinterpret_cast<__nv_bfloat16*>(args.out) + rowoff;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float dh[16];
+                    tmem_ld16(t0 + c, dh);
+                    tmem_ld_wait();
+                    if (valid) {
+                        const int f = x.nb * BN + c;
+                        const int64_t col = (int64_t)(f >> 7) * 256 + (f & 127);
+                        float a[16], b[16], da[16], db[16];
+                        load_bf16x16(ab + col, a);
+                        load_bf16x16(ab + col + 128, b);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float sig = 1.0f / (1.0f + __expf(-a[i]));
+                            da[i] = dh[i] * b[i] * sig * (1.0f + a[i] * (1.0f - sig));
+                            db[i] = dh[i] * a[i] * sig;
+                        }
+                        store_bf16x16(dab + col, da);
+                        store_bf16x16(dab + col + 128, db);
+                    }
+                }
+            } else if (MODE == TC_WGRAD) {
+                float* dst = reinterpret_cast<float*>(args.out) + x.g * args.group_stride +
+                             (int64_t)(x.mt * BM + row) * args.out_ld + x.nb * BN;
+                const bool empty = x.kb1 == x.kb0;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    if (!empty) {
+                        tmem_ld16(t0 + c, v);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<float4*>(dst + c + i) =
+                            make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                }
             } else if (MODE == TC_GATEUP_SWAP) {
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
                                      (int64_t)x.row0 * args.out_ld + x.nb * 128 + row;
@@ -431,6 +513,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                         if (c + i < x.rows)
                             dst[(int64_t)(c + i) * args.out_ld] =
                                 __float2bfloat16_rn(silu_f(g[i]) * v[i]);
+                    if (args.aux) {
+                        __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(args.aux) +
+                                            (int64_t)x.row0 * args.aux_ld + x.nb * 256 + row;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c + i < x.rows) {
+                                ab[(int64_t)(c + i) * args.aux_ld] = __float2bfloat16_rn(g[i]);
+                                ab[(int64_t)(c + i) * args.aux_ld + 128] =
+                                    __float2bfloat16_rn(v[i]);
+                            }
+                    }
                 }
             } else {
                 float* dst = reinterpret_cast<float*>(args.out) + x.ks * args.split_stride +
@@ -473,7 +566,8 @@ int launch_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, i
         configured_bytes = L.total;
     }
     kern<<<grid, THREADS, L.total, st>>>(act, w, a);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 }  // namespace
@@ -496,6 +590,12 @@ int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& 
             return launch_mode<TC_GATEUP_SWAP, 128>(act, w, a, grid, st);
         case TC_DOWN_SWAP:
             return launch_mode<TC_DOWN_SWAP, 128>(act, w, a, grid, st);
+        case TC_DGATE_TOK:
+            return bn == 256 ? launch_mode<TC_DGATE_TOK, 256>(act, w, a, grid, st)
+                             : launch_mode<TC_DGATE_TOK, 128>(act, w, a, grid, st);
+        case TC_WGRAD:
+            return bn == 256 ? launch_mode<TC_WGRAD, 256>(act, w, a, grid, st)
+                             : launch_mode<TC_WGRAD, 128>(act, w, a, grid, st);
     }
     return -1;
 }

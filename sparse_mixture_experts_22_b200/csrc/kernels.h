@@ -8,6 +8,20 @@
 
 namespace moe {
 
+// Counts one kernel launch (every launch site calls it; moe_launch_count).
+void note_launch();
+
+// The calling thread's error of its last failed launch (cudaSuccess if none).
+cudaError_t& last_launch_error();
+
+// 0 if the launches so far succeeded; else records the error and returns -1.
+inline int launch_result() {
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return 0;
+    last_launch_error() = e;
+    return -1;
+}
+
 // ---------------------------------------------------------------- router
 // logits z[T][E] = x[T][d] Wr[d][E] on the CUDA cores (fp32 accumulate, no bias)
 int launch_router_logits(const void* x, bool x_bf16, const float* Wr, float* z, int64_t T, int d,
@@ -70,7 +84,14 @@ int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num
                           cudaStream_t st);
 
 // ---------------------------------------------------------------- tensor-core GEMMs
-enum TcMode : int { TC_GATEUP_TOK = 0, TC_DOWN_TOK = 1, TC_GATEUP_SWAP = 2, TC_DOWN_SWAP = 3 };
+enum TcMode : int {
+    TC_GATEUP_TOK = 0,   // H = silu(A w1) * (A w3), token-major tiles
+    TC_DOWN_TOK = 1,     // y = A W^T (fp32), token-major tiles, optional split-K
+    TC_GATEUP_SWAP = 2,  // gate/up with weight rows as M (few tokens per group)
+    TC_DOWN_SWAP = 3,    // down with weight rows as M, split-K
+    TC_DGATE_TOK = 4,    // backward: dH = dY W2^T, SiLU*mul backward in the epilogue
+    TC_WGRAD = 5,        // backward: C[g] = A[:, K_g] B[:, K_g]^T over each group's token range
+};
 
 struct TcArgs {
     int num_groups;
@@ -90,6 +111,11 @@ struct TcArgs {
     int32_t* status;            // device status word
     uint64_t wait_limit_ns;
     int test_stall;             // test hook: CTA 0 withholds its first accumulator-ready signal
+    void* aux;                  // gate/up: pre-activation output AB (bf16, may be null);
+                                // dgate: AB input
+    int64_t aux_ld;             // elements per AB row (2 x hidden width)
+    int m_rows;                 // wgrad: rows of A (output rows per group)
+    int64_t group_stride;       // wgrad: elements between the groups' outputs
 };
 
 int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);
@@ -133,5 +159,54 @@ int launch_stats_finalize(const double* sums, int E, int k, void* stats, cudaStr
 int launch_pack(const void* src, void* dst, int elem_bytes, int R, int Cc, int64_t ld_dst,
                 int col_off, int interleave, int n, int64_t src_stride, int64_t dst_stride,
                 int col_step, cudaStream_t st);
+
+// ---------------------------------------------------------------- backward pass
+// dY[slot] = gate * G[t] (bf16) for every kept slot; dg[t][j] = <G[t], y[slot]>
+// (y summed over its split-K partials), 0 for dropped assignments
+int launch_bwd_gather(const void* G, const float* y, int splits, int64_t split_stride,
+                      const int32_t* slot_of, const float* gate, void* dY, float* dg, int64_t T,
+                      int d, int k, int num_sms, cudaStream_t st);
+// dz[t][e] = softmax-over-k backward of dg + aux_coef (E/T) p (f - sum f p);
+// z are the forward logits, bias added here when given
+int launch_router_bwd(const float* z, const float* bias, const int32_t* idx, const float* gate,
+                      const float* dg, const int32_t* routed, float aux_coef, float* dz, int64_t T,
+                      int E, int k, int num_sms, cudaStream_t st);
+// token chunks of the router-weight gradient (partials [chunks][d + 1][E])
+int wr_grad_chunks(int64_t T, int d, int E);
+// dWr = x^T dz, db = column sums of dz (db may be null)
+int launch_wr_grad(const void* x, const float* dz, float* part, float* dWr, float* db, int64_t T,
+                   int d, int E, cudaStream_t st);
+// dxr[t][c] = sum_e dz[t][e] Wr[c][e]
+int launch_dxr(const float* dz, const float* Wr, float* dxr, int64_t T, int d, int E,
+               cudaStream_t st);
+// kofs[g] = sum of rows[g'] rounded up to 64 over g' < g; kofs[G] = total
+int launch_kofs(const int32_t* rows, int G, int32_t* kofs, cudaStream_t st);
+
+struct TransposeJob {
+    const void* src;        // bf16 [rows][features], row stride src_ld
+    int64_t src_ld;
+    void* dst;              // bf16 [features][K], row stride dst_ld
+    int64_t dst_ld;
+    int features;           // multiple of 64
+    int groups;
+    const int32_t* rows;    // device [groups] rows per group (null: one dense group)
+    const int32_t* off;     // device [groups] first source row
+    const int32_t* kofs;    // device [groups + 1] first destination column
+    int dense_rows;
+};
+struct TransposeJobs {
+    TransposeJob job[4];
+    int n;
+};
+// dst[f][kofs[g] + i] = src[off[g] + i][f], zero-filled to multiples of 64
+int launch_transpose(const TransposeJobs& jobs, int64_t k_bound, cudaStream_t st);
+// dx[t] = sum over kept slots of dXp[slot] + dXs[t] (may be null) + dXr[t]
+int launch_combine_bwd(const float* dXp, const int32_t* slot_of, const float* dXs,
+                       const float* dXr, float* dx, int64_t T, int d, int k, int num_sms,
+                       cudaStream_t st);
+// dst[r][col(c)] = src[r][c], bf16, no transpose (backward weight layout)
+int launch_pack_cols(const void* src, void* dst, int R, int Cc, int64_t ld_dst, int col_off,
+                     int interleave, int n, int64_t src_stride, int64_t dst_stride, int col_step,
+                     cudaStream_t st);
 
 }  // namespace moe

@@ -148,7 +148,8 @@ int launch_logits_t(const XT* x, const float* Wr, float* z, int64_t T, int d, in
         configured = smem;
     }
     kern<<<grid, RT_WARPS * 32, smem, st>>>(x, Wr, z, T, d, E, dch);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 template <typename XT>
@@ -338,7 +339,8 @@ int launch_router_rows(const void* x, bool x_bf16, const float* Wr, float* z, in
     else
         router_rows_kernel<float><<<grid, RR_THREADS, 0, st>>>(reinterpret_cast<const float*>(x),
                                                                Wr, z, d, E);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_router_reduce(const float* src, int nsplit, int64_t split_stride, int row_stride,
@@ -348,13 +350,15 @@ int launch_router_reduce(const float* src, int nsplit, int64_t split_stride, int
     const int64_t n = T * E;
     router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
         src, nsplit, split_stride, row_stride, nparts, bias, z, T, E);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_router_split(const float* Wr, void* Ws, int d, int E, cudaStream_t st) {
     dim3 grid((d + 31) / 32, (E + 31) / 32), block(32, 8);
     router_split_kernel<<<grid, block, 0, st>>>(Wr, reinterpret_cast<__nv_bfloat16*>(Ws), d, E);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 }  // namespace moe

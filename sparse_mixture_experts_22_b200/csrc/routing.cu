@@ -789,7 +789,8 @@ int launch_topk(const RouteParams& r, cudaStream_t st) {
     const size_t smem = topk_smem_bytes(r.E, nthreads);
     if (set_smem(topk_kernel, smem)) return -1;
     topk_kernel<<<blocks, nthreads, smem, st>>>(topk_args(r), r.cnt);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt, int32_t* tot,
@@ -799,12 +800,14 @@ int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* c
     const int64_t scan_threads = (int64_t)p.E * 32;
     dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nblk,
                                                                                 p.E);
-    if (cudaGetLastError() != cudaSuccess) return -1;
+    note_launch();
+    if (launch_result() != 0) return -1;
     const size_t smem = dispatch_smem_bytes(p.E, p.k);
     if (set_smem(dispatch_kernel, smem)) return -1;
     dim3 grid(nblk, copy_splits(nblk, p.T, p.k, num_sms));
     dispatch_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(dispatch_args(p), topk_idx, cnt, tot);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_reroute_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt,
@@ -816,20 +819,24 @@ int launch_reroute_dispatch(const DispatchParams& p, const int32_t* topk_idx, in
     const int64_t scan_threads = (int64_t)p.E * 32;
     dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nblk,
                                                                                 p.E);
-    if (cudaGetLastError() != cudaSuccess) return -1;
+    note_launch();
+    if (launch_result() != 0) return -1;
     const size_t smem = dispatch_smem_bytes(p.E, p.k);
     if (set_smem(rank_kernel, smem) || set_smem(place_kernel, smem)) return -1;
     rank_kernel<<<nblk, ROUTE_BLOCK, smem, st>>>(a, topk_idx, cnt, expert_of, rank_of);
-    if (cudaGetLastError() != cudaSuccess) return -1;
+    note_launch();
+    if (launch_result() != 0) return -1;
     const size_t rsmem = reroute_smem_bytes(p.E, p.k);
     if (set_smem(reroute_kernel, rsmem)) return -1;
     reroute_kernel<<<1, RR_THREADS, rsmem, st>>>(topk_idx, expert_of, rank_of, tot, z, nullptr,
                                                  p.T, p.E, p.k, p.C, p.pad, p.routed, p.kept,
                                                  p.offsets);
-    if (cudaGetLastError() != cudaSuccess) return -1;
+    note_launch();
+    if (launch_result() != 0) return -1;
     dim3 grid(nblk, copy_splits(nblk, p.T, p.k, num_sms));
     place_kernel<<<grid, ROUTE_BLOCK, smem, st>>>(a, expert_of, rank_of);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num_sms,
@@ -840,7 +847,8 @@ int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num
     if (set_smem(route_dispatch_kernel, smem)) return -1;
     route_dispatch_kernel<<<copy_splits(1, p.T, p.k, num_sms), ROUTE_BLOCK, smem, st>>>(
         topk_args(r), dispatch_args(p), r.cnt);
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    note_launch();
+    return launch_result();
 }
 
 }  // namespace moe

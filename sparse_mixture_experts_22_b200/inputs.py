@@ -17,6 +17,8 @@ seed and the tensor's name, so any tensor can be regenerated alone):
   w1, w3 ~ N(0, 1/d)          [E, d, h]   gate and up projections
   w2     ~ N(0, 1/h)          [E, h, d]   down projection
   shared experts: w1s, w3s [S, d, hs] ~ N(0, 1/d); w2s [S, hs, d] ~ N(0, 1/hs)
+  G      ~ N(0, 1)            [T, d]      gradient of the loss w.r.t. the layer
+                                          output (backward pass), workload dtype
 """
 
 import hashlib
@@ -147,3 +149,9 @@ def layer_inputs(wl: Workload, T: Optional[int] = None, weights: bool = True) ->
             s = expert_weights(wl, shared=True)
             out.update({"w1s": s["w1"], "w3s": s["w3"], "w2s": s["w2"]})
     return out
+
+
+def grad_out(wl: Workload, T: Optional[int] = None) -> torch.Tensor:
+    """G = dL/dout [T, d] for the backward pass, in the workload dtype."""
+    T = wl.T if T is None else T
+    return normal((T, wl.d), 1.0, generator(wl.seed, "grad_out"), torch_dtype(wl.dtype))

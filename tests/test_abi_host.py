@@ -91,3 +91,27 @@ def test_null_config_is_rejected():
     v = ctypes.c_int64()
     assert lib.moe_capacity(None, ctypes.byref(v)) == 1
     assert b"NULL" in lib.moe_last_error()
+
+
+def test_training_workspaces():
+    for name, wl in WORKLOADS.items():
+        if wl.dtype != "bf16":
+            continue
+        inf = M.moe_workspace_size(M.config_of(wl))
+        tr = M.config_of(wl, train=True)
+        # the forward keeps the gate/up pre-activations (bf16 [perm_rows][2h])
+        assert M.moe_workspace_size(tr) >= inf + M.moe_perm_rows(tr) * 2 * wl.h * 2
+        assert M.moe_backward_workspace_size(tr) > 0
+    # fp32 layers have no backward pass; train must be 0 or 1
+    with pytest.raises(B.MoEError) as e:
+        M.moe_workspace_size(M.make_config(8, 128, 128, 4, 2, dtype="f32", train=True))
+    assert e.value.code == 8
+    cfg = M.make_config(8, 128, 128, 4, 2)
+    cfg.train = 2
+    with pytest.raises(B.MoEError) as e:
+        M.moe_workspace_size(cfg)
+    assert e.value.code == 1
+    # the backward workspace exists only for a training config
+    with pytest.raises(B.MoEError) as e:
+        M.moe_backward_workspace_size(M.make_config(8, 128, 128, 4, 2))
+    assert e.value.code == 1
