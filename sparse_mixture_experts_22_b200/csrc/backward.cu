@@ -13,12 +13,10 @@
 //              aux_coef (E / T) p_te (f_e - sum_i f_i p_ti)
 //   wr_grad    dWr = x^T dz and db = column sums of dz, split over token
 //              chunks into partials reduced in a fixed order
-//   dxr        the router's share of dx: dz Wr^T
-//   kofs       each expert's 64-aligned offset along the token axis of the
-//              transposed activations the weight-gradient GEMMs contract
-//   transpose  [rows][features] -> [features][tokens] per expert segment,
-//              zero-filled up to the next multiple of 64 tokens
-//   combine    dx_t = sum over kept slots of dXp + shared dX + router dX
+//   zero_pad   zeros in the rows between an expert's last token and the next
+//              multiple of 64 (the weight-gradient GEMMs read whole 64-row
+//              blocks of the row-major activations as MN-major operands)
+//   combine    dx_t = sum over kept slots of dXp + shared dX + dz_t Wr^T
 // Every sum runs in a fixed order: the results are identical run to run.
 #include "common.cuh"
 #include "kernels.h"
@@ -140,45 +138,69 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------- router weights
 
 constexpr int WR_THREADS = 128;
-constexpr int WR_ET = 32;   // experts per block
 constexpr int WR_TT = 32;   // tokens staged per step
 
 // part[ch][c][e] = sum over the chunk's tokens of x[t][c] dz[t][e]; row c == d
-// holds the column sums of dz (the bias gradient).
-template <typename XT>
+// holds the column sums of dz (the bias gradient).  A thread owns CV
+// consecutive columns (one vector load of x per token) and ET experts.
+template <int CV, int ET>
 __global__ void __launch_bounds__(WR_THREADS)
-    wr_grad_kernel(const XT* __restrict__ x, const float* __restrict__ dz, float* __restrict__ part,
-                   int64_t T, int d, int E, int64_t chunk) {
-    __shared__ float dzs[WR_TT][WR_ET];
-    const int c = blockIdx.x * WR_THREADS + threadIdx.x;
-    const int e0 = blockIdx.z * WR_ET;
-    const int ne = min(WR_ET, E - e0);
+    wr_grad_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dz,
+                   float* __restrict__ part, int64_t T, int d, int E, int64_t chunk) {
+    __shared__ float dzs[WR_TT][ET];
+    const int c0 = (blockIdx.x * WR_THREADS + threadIdx.x) * CV;
+    const int e0 = blockIdx.z * ET;
+    const int ne = min(ET, E - e0);
     const int64_t t0 = (int64_t)blockIdx.y * chunk;
     const int64_t t1 = min(T, t0 + chunk);
-    float acc[WR_ET];
+    const bool ones = c0 == d;  // the bias row
+    float acc[CV][ET];
 #pragma unroll
-    for (int i = 0; i < WR_ET; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < CV; ++i)
+#pragma unroll
+        for (int j = 0; j < ET; ++j) acc[i][j] = 0.0f;
     for (int64_t tb = t0; tb < t1; tb += WR_TT) {
         __syncthreads();
-        for (int i = threadIdx.x; i < WR_TT * WR_ET; i += WR_THREADS) {
-            const int tt = i / WR_ET, ee = i % WR_ET;
+        for (int i = threadIdx.x; i < WR_TT * ET; i += WR_THREADS) {
+            const int tt = i / ET, ee = i % ET;
             dzs[tt][ee] = (tb + tt < t1 && ee < ne) ? dz[(tb + tt) * E + e0 + ee] : 0.0f;
         }
         __syncthreads();
-        if (c <= d) {
+        if (c0 <= d) {
             const int nt = (int)min((int64_t)WR_TT, t1 - tb);
             for (int tt = 0; tt < nt; ++tt) {
-                const float xv = c < d ? (float)x[(tb + tt) * d + c] : 1.0f;
+                float xv[CV];
+                if (!ones) {
+                    const __nv_bfloat16* px = x + (tb + tt) * d + c0;
+                    if (CV == 8) {
+                        load_bf16x8(px, xv);
+                    } else {
 #pragma unroll
-                for (int i = 0; i < WR_ET; ++i) acc[i] += xv * dzs[tt][i];
+                        for (int i = 0; i < CV; ++i) xv[i] = __bfloat162float(px[i]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < CV; ++i) xv[i] = i == 0 ? 1.0f : 0.0f;
+                }
+#pragma unroll
+                for (int j = 0; j < ET; ++j) {
+                    const float z = dzs[tt][j];
+#pragma unroll
+                    for (int i = 0; i < CV; ++i) acc[i][j] += xv[i] * z;
+                }
             }
         }
     }
-    if (c <= d) {
-        float* dst = part + ((int64_t)blockIdx.y * (d + 1) + c) * E + e0;
+    if (c0 <= d) {
+        const int nrow = ones ? 1 : CV;
 #pragma unroll
-        for (int i = 0; i < WR_ET; ++i)
-            if (i < ne) dst[i] = acc[i];
+        for (int i = 0; i < CV; ++i) {
+            if (i >= nrow) break;
+            float* dst = part + ((int64_t)blockIdx.y * (d + 1) + c0 + i) * E + e0;
+#pragma unroll
+            for (int j = 0; j < ET; ++j)
+                if (j < ne) dst[j] = acc[i][j];
+        }
     }
 }
 
@@ -196,13 +218,102 @@ __global__ void wr_reduce_kernel(const float* __restrict__ part, int nch, int64_
     }
 }
 
-// ---------------------------------------------------------------- router share of dx
+// ---------------------------------------------------------------- padding rows
+
+// Zeroes rows [off[g] + rows[g], off[g] + rows[g] rounded up to 64) of each
+// bf16 buffer: the weight-gradient GEMMs contract whole 64-row blocks of every
+// expert segment, so the rows past an expert's tokens must hold zeros.
+__global__ void __launch_bounds__(256) zero_pad_kernel(PadJobs p) {
+    const int g = blockIdx.x;
+    const PadJob& jb = p.job[blockIdx.y];
+    const int32_t n = p.rows[g];
+    const int64_t r0 = (int64_t)p.off[g] + n;
+    const int64_t r1 = (int64_t)p.off[g] + (n + 63) / 64 * 64;
+    const int w8 = jb.width / 8;
+    const int64_t total = (r1 - r0) * w8;
+    uint4* base = reinterpret_cast<uint4*>(jb.buf);
+    for (int64_t i = (int64_t)blockIdx.z * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.z * blockDim.x) {
+        const int64_t row = r0 + i / w8;
+        base[row * w8 + i % w8] = make_uint4(0, 0, 0, 0);
+    }
+}
+
+// ---------------------------------------------------------------- dx
+
+// The router's share of dx is dz_t Wr^T, a product with K = E.  Up to
+// E = 16 a thread keeps Wr's rows for its four columns in registers and the
+// share is formed inside the combine; for more experts it is a tiled product
+// of its own (dxr), which the combine then adds.
+
+constexpr int CB_TOK = 64;   // tokens per block of the combine
+
+// dx[t][c..c+3] = sum_j dXp[slot_of[t][j]][c..] (kept slots, j order)
+//               + dXs[t][c..] + (EREG ? sum_e dz[t][e] Wr[c..][e] : dxr[t][c..])
+template <int EREG>
+__global__ void __launch_bounds__(256)
+    combine_bwd_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ slot_of,
+                       const float* __restrict__ dXs, const float* __restrict__ dz,
+                       const float* __restrict__ Wr, const float* __restrict__ dxr,
+                       float* __restrict__ dx, int64_t T, int d, int k, int E) {
+    __shared__ float zs[CB_TOK][EREG > 0 ? EREG : 1];
+    __shared__ int32_t slots[CB_TOK][8];
+    const int64_t t0 = (int64_t)blockIdx.y * CB_TOK;
+    const int c = (blockIdx.x * 256 + threadIdx.x) * 4;
+    for (int i = threadIdx.x; i < CB_TOK * 8; i += 256) {
+        const int tt = i / 8, j = i % 8;
+        slots[tt][j] = (t0 + tt < T && j < k) ? slot_of[(t0 + tt) * k + j] : -1;
+    }
+    float w[4][EREG > 0 ? EREG : 1];
+    if (EREG > 0) {
+        for (int i = threadIdx.x; i < CB_TOK * EREG; i += 256) {
+            const int tt = i / EREG, e = i % EREG;
+            zs[tt][e] = (t0 + tt < T && e < E) ? dz[(t0 + tt) * E + e] : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int e = 0; e < (EREG > 0 ? EREG : 1); ++e)
+                w[i][e] = (c < d && e < E) ? Wr[(int64_t)(c + i) * E + e] : 0.0f;
+    }
+    __syncthreads();
+    if (c >= d) return;
+    const int nt = (int)min((int64_t)CB_TOK, T - t0);
+    for (int tt = 0; tt < nt; ++tt) {
+        const int64_t t = t0 + tt;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const int32_t r = slots[tt][j];
+            if (r < 0) continue;
+            const float4 v = *reinterpret_cast<const float4*>(dXp + (int64_t)r * d + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        if (dXs) {
+            const float4 v = *reinterpret_cast<const float4*>(dXs + t * d + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        if (EREG > 0) {
+            float r[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < (EREG > 0 ? EREG : 1); ++e) {
+                const float z = zs[tt][e];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) r[i] += z * w[i][e];
+            }
+            acc.x += r[0]; acc.y += r[1]; acc.z += r[2]; acc.w += r[3];
+        } else {
+            const float4 v = *reinterpret_cast<const float4*>(dxr + t * d + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        *reinterpret_cast<float4*>(dx + t * d + c) = acc;
+    }
+}
 
 constexpr int DXR_TT = 32;   // tokens per block
 constexpr int DXR_CT = 128;  // model columns per block (one per thread)
 constexpr int DXR_EK = 32;   // experts staged per step
 
-// dxr[t][c] = sum_e dz[t][e] Wr[c][e]
+// dxr[t][c] = sum_e dz[t][e] Wr[c][e], tiled over e through shared memory
 __global__ void __launch_bounds__(DXR_CT)
     dxr_kernel(const float* __restrict__ dz, const float* __restrict__ Wr, float* __restrict__ dxr,
                int64_t T, int d, int E) {
@@ -227,110 +338,14 @@ __global__ void __launch_bounds__(DXR_CT)
         __syncthreads();
 #pragma unroll 4
         for (int ee = 0; ee < DXR_EK; ++ee) {
-            const float w = ws[tid][ee];
+            const float wv = ws[tid][ee];
 #pragma unroll
-            for (int tt = 0; tt < DXR_TT; ++tt) acc[tt] += zs[tt][ee] * w;
+            for (int tt = 0; tt < DXR_TT; ++tt) acc[tt] += zs[tt][ee] * wv;
         }
     }
+#pragma unroll
     for (int tt = 0; tt < DXR_TT; ++tt)
         if (t0 + tt < T) dxr[(t0 + tt) * d + c0 + tid] = acc[tt];
-}
-
-// ---------------------------------------------------------------- token offsets
-
-// kofs[g] = sum over g' < g of rows[g'] rounded up to 64; kofs[G] = total
-__global__ void kofs_kernel(const int32_t* __restrict__ rows, int G, int32_t* __restrict__ kofs) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int32_t acc = 0;
-    for (int g = 0; g < G; ++g) {
-        kofs[g] = acc;
-        acc += (rows[g] + 63) / 64 * 64;
-    }
-    kofs[G] = acc;
-}
-
-// ---------------------------------------------------------------- transpose
-
-constexpr int TP = 64;  // tile: 64 tokens x 64 features
-
-// dst[f][kofs[g] + i] = src[off[g] + i][f] for i < rows[g]; zero for
-// rows[g] <= i < the next multiple of 64.  Dense jobs use one group of
-// `dense_rows` rows at offset 0 (rows == null).
-__global__ void __launch_bounds__(256)
-    transpose_kernel(TransposeJobs jobs) {
-    __shared__ uint16_t tile[TP][TP + 2];
-    const TransposeJob& jb = jobs.job[blockIdx.z];
-    const int f0 = blockIdx.y * TP;
-    if (f0 >= jb.features) return;
-    const int G = jb.groups;
-    const int32_t* kofs = jb.kofs;
-    const int kt = blockIdx.x * TP;
-    const int total = kofs ? kofs[G] : (jb.dense_rows + TP - 1) / TP * TP;
-    if (kt >= total) return;
-    int g = 0, local = kt, n = jb.dense_rows, r0 = 0;
-    if (kofs) {
-        int lo = 0, hi = G - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (kofs[mid] <= kt) lo = mid; else hi = mid - 1;
-        }
-        g = lo;
-        local = kt - kofs[g];
-        n = jb.rows[g];
-        r0 = jb.off[g];
-    }
-    const int valid = min(TP, n - local);
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(jb.src);
-    // load: 64 rows x 64 features, 8 features (16 bytes) per access
-    for (int i = threadIdx.x; i < TP * (TP / 8); i += blockDim.x) {
-        const int rr = i / (TP / 8), cc = (i % (TP / 8)) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (rr < valid)
-            v = *reinterpret_cast<const uint4*>(src + (int64_t)(r0 + local + rr) * jb.src_ld +
-                                                f0 + cc);
-        const uint16_t* pv = reinterpret_cast<const uint16_t*>(&v);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) tile[rr][cc + q] = pv[q];
-    }
-    __syncthreads();
-    uint16_t* dst = reinterpret_cast<uint16_t*>(jb.dst);
-    for (int i = threadIdx.x; i < TP * (TP / 8); i += blockDim.x) {
-        const int ff = i / (TP / 8), tt = (i % (TP / 8)) * 8;
-        uint16_t pv[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) pv[q] = tile[tt + q][ff];
-        *reinterpret_cast<uint4*>(dst + (int64_t)(f0 + ff) * jb.dst_ld + kt + tt) =
-            *reinterpret_cast<const uint4*>(pv);
-    }
-}
-
-// ---------------------------------------------------------------- dx
-
-// dx[t] = sum_j dXp[slot_of[t][j]] (kept slots, in j order) + dXs[t] + dXr[t]
-__global__ void combine_bwd_kernel(const float* __restrict__ dXp, const int32_t* __restrict__ slot_of,
-                                   const float* __restrict__ dXs, const float* __restrict__ dXr,
-                                   float* __restrict__ dx, int64_t T, int d, int k) {
-    const int q = d / 4;
-    const int64_t n = T * q;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = i / q;
-        const int c = (int)(i % q) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const int32_t r = slot_of[t * k + j];
-            if (r < 0) continue;
-            const float4 v = *reinterpret_cast<const float4*>(dXp + (int64_t)r * d + c);
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-        }
-        if (dXs) {
-            const float4 v = *reinterpret_cast<const float4*>(dXs + t * d + c);
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-        }
-        const float4 v = *reinterpret_cast<const float4*>(dXr + t * d + c);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-        *reinterpret_cast<float4*>(dx + t * d + c) = acc;
-    }
 }
 
 // ---------------------------------------------------------------- backward weight layout
@@ -400,9 +415,15 @@ int launch_wr_grad(const void* x, const float* dz, float* part, float* dWr, floa
                    int d, int E, cudaStream_t st) {
     const int nch = wr_grad_chunks(T, d, E);
     const int64_t chunk = ((T + nch - 1) / nch + WR_TT - 1) / WR_TT * WR_TT;
-    dim3 grid((d + 1 + WR_THREADS - 1) / WR_THREADS, nch, (E + WR_ET - 1) / WR_ET);
-    wr_grad_kernel<__nv_bfloat16><<<grid, WR_THREADS, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(x), dz, part, T, d, E, chunk);
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (E <= 8) {
+        // one extra thread (column d) computes the bias row
+        dim3 grid((d + 8 + WR_THREADS * 8 - 1) / (WR_THREADS * 8), nch, 1);
+        wr_grad_kernel<8, 8><<<grid, WR_THREADS, 0, st>>>(xb, dz, part, T, d, E, chunk);
+    } else {
+        dim3 grid((d + 4 + WR_THREADS * 4 - 1) / (WR_THREADS * 4), nch, (E + 15) / 16);
+        wr_grad_kernel<4, 16><<<grid, WR_THREADS, 0, st>>>(xb, dz, part, T, d, E, chunk);
+    }
     note_launch();
     if (launch_result() != 0) return -1;
     const int64_t n = (int64_t)(d + 1) * E;
@@ -411,35 +432,42 @@ int launch_wr_grad(const void* x, const float* dz, float* part, float* dWr, floa
     return launch_result();
 }
 
-int launch_dxr(const float* dz, const float* Wr, float* dxr, int64_t T, int d, int E,
-               cudaStream_t st) {
-    dim3 grid(d / DXR_CT, (unsigned)((T + DXR_TT - 1) / DXR_TT));
-    dxr_kernel<<<grid, DXR_CT, 0, st>>>(dz, Wr, dxr, T, d, E);
-    note_launch();
-    return launch_result();
-}
-
-int launch_kofs(const int32_t* rows, int G, int32_t* kofs, cudaStream_t st) {
-    kofs_kernel<<<1, 32, 0, st>>>(rows, G, kofs);
-    note_launch();
-    return launch_result();
-}
-
-int launch_transpose(const TransposeJobs& jobs, int64_t k_bound, cudaStream_t st) {
-    int fmax = 0;
-    for (int i = 0; i < jobs.n; ++i) fmax = jobs.job[i].features > fmax ? jobs.job[i].features : fmax;
-    if (jobs.n == 0 || k_bound <= 0) return 0;
-    dim3 grid((unsigned)((k_bound + TP - 1) / TP), (fmax + TP - 1) / TP, jobs.n);
-    transpose_kernel<<<grid, 256, 0, st>>>(jobs);
+int launch_zero_pad(const PadJobs& p, cudaStream_t st) {
+    if (p.n == 0 || p.groups == 0) return 0;
+    // blocks per (segment, buffer): enough for the widest buffer's 63 padding
+    // rows, but about 1200 blocks over the whole launch
+    int wmax = 0;
+    for (int i = 0; i < p.n; ++i) wmax = p.job[i].width > wmax ? p.job[i].width : wmax;
+    const int per = (int)(((int64_t)63 * (wmax / 8) + 255) / 256);
+    const int share = 1200 / (p.groups * p.n);
+    int z = per < share ? per : share;
+    z = z < 1 ? 1 : (z > 64 ? 64 : z);
+    zero_pad_kernel<<<dim3(p.groups, p.n, z), 256, 0, st>>>(p);
     note_launch();
     return launch_result();
 }
 
 int launch_combine_bwd(const float* dXp, const int32_t* slot_of, const float* dXs,
-                       const float* dXr, float* dx, int64_t T, int d, int k, int num_sms,
-                       cudaStream_t st) {
-    combine_bwd_kernel<<<grid_for(T * (d / 4), 256, num_sms * 16), 256, 0, st>>>(
-        dXp, slot_of, dXs, dXr, dx, T, d, k);
+                       const float* dz, const float* Wr, float* dxr, float* dx, int64_t T, int d,
+                       int k, int E, cudaStream_t st) {
+    dim3 grid((d / 4 + 255) / 256, (unsigned)((T + CB_TOK - 1) / CB_TOK));
+    if (E <= 8) {
+        combine_bwd_kernel<8><<<grid, 256, 0, st>>>(dXp, slot_of, dXs, dz, Wr, nullptr, dx, T, d,
+                                                    k, E);
+        note_launch();
+        return launch_result();
+    }
+    if (E <= 16) {
+        combine_bwd_kernel<16><<<grid, 256, 0, st>>>(dXp, slot_of, dXs, dz, Wr, nullptr, dx, T,
+                                                     d, k, E);
+        note_launch();
+        return launch_result();
+    }
+    dim3 gr(d / DXR_CT, (unsigned)((T + DXR_TT - 1) / DXR_TT));
+    dxr_kernel<<<gr, DXR_CT, 0, st>>>(dz, Wr, dxr, T, d, E);
+    note_launch();
+    if (launch_result() != 0) return -1;
+    combine_bwd_kernel<0><<<grid, 256, 0, st>>>(dXp, slot_of, dXs, dz, Wr, dxr, dx, T, d, k, E);
     note_launch();
     return launch_result();
 }

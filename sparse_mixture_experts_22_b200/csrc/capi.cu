@@ -119,7 +119,8 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     } else {
         P.path = nmax <= SWAP_MAX_TOKENS ? PATH_SWAP : PATH_TOKEN_MAJOR;
         P.shared_path = P.T <= SWAP_MAX_TOKENS ? PATH_SWAP : PATH_TOKEN_MAJOR;
-        P.pad = P.path == PATH_TOKEN_MAJOR ? 128 : 16;
+        // the backward pass contracts whole 64-row blocks of each segment
+        P.pad = P.path == PATH_TOKEN_MAJOR ? 128 : (c.train ? 64 : 16);
     }
     P.nt_max = (int)(((nmax > 0 ? nmax : 1) + 15) / 16 * 16);
     // split-K of the swapped down projection: enough units for ~6.5 waves of 148 SMs
@@ -187,8 +188,6 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.total = o;
 
     // backward workspace
-    P.kt = c.T > 0 ? (kept_max + (int64_t)c.E * 63 + 63) / 64 * 64 : 0;
-    P.tp = (c.T + 63) / 64 * 64;
     P.wr_chunks = P.train ? wr_grad_chunks(c.T, c.d, c.E) : 1;
     o = 0;
     const bool tr = P.train;
@@ -197,20 +196,11 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.b_dz = take(tr ? (size_t)c.T * c.E * 4 : 0);
     P.b_dAB = take(tr ? (size_t)P.perm_rows * 2 * c.h * 2 : 0);
     P.b_dXp = take(tr ? (size_t)P.perm_rows * c.d * 4 : 0);
-    P.b_kofs = take(tr ? (size_t)(c.E + 1) * 4 : 0);
-    P.b_XT = take(tr ? (size_t)c.d * P.kt * 2 : 0);
-    P.b_dYT = take(tr ? (size_t)c.d * P.kt * 2 : 0);
-    P.b_HT = take(tr ? (size_t)c.h * P.kt * 2 : 0);
-    P.b_dABT = take(tr ? (size_t)2 * c.h * P.kt * 2 : 0);
     const bool ts = tr && P.S > 0;
     P.b_dABs = take(ts ? (size_t)c.T * 2 * P.hsum * 2 : 0);
     P.b_dXs = take(ts ? (size_t)c.T * c.d * 4 : 0);
-    P.b_GT = take(ts ? (size_t)c.d * P.tp * 2 : 0);
-    P.b_xT = take(ts ? (size_t)c.d * P.tp * 2 : 0);
-    P.b_HsT = take(ts ? (size_t)P.hsum * P.tp * 2 : 0);
-    P.b_dABsT = take(ts ? (size_t)2 * P.hsum * P.tp * 2 : 0);
     P.b_wrpart = take(tr ? (size_t)P.wr_chunks * (c.d + 1) * c.E * 4 : 0);
-    P.b_dXr = take(tr ? (size_t)c.T * c.d * 4 : 0);
+    P.b_dxr = take(tr && c.E > 16 ? (size_t)c.T * c.d * 4 : 0);
     P.b_total = o;
     return MOE_OK;
 }
@@ -758,21 +748,25 @@ static int run_tc_backward(const Plan& P, const Device& dv, int groups, const in
     return MOE_OK;
 }
 
-// Weight gradient C[g] [m_rows][n_rows] = AT[:, K_g] BT[:, K_g]^T, K_g the
-// g-th group's 64-aligned token range (rows[g] tokens; dense: one group).
+// Weight gradient C[g] [m_rows][n_rows] = sum over the token rows r of group g
+// of A[r][:]^T B[r][:]: A [act_rows][m_rows] and B [act_rows][n_rows] are the
+// row-major activations, read as MN-major operands; group g covers the rows
+// offs[g] .. offs[g] + rows[g] rounded up to 64 (offs a multiple of 64, the
+// rows past rows[g] zero); dense: one group of dense_rows rows from row 0.
 static int run_tc_wgrad(const Plan& P, const Device& dv, int groups, const int32_t* rows,
-                        int dense_rows, const void* AT, int m_rows, const void* BT, int n_rows,
-                        int64_t kcols, float* out, int32_t* status, cudaStream_t st,
-                        const char* tag) {
+                        const int32_t* offs, int dense_rows, int64_t act_rows, const void* A,
+                        int m_rows, const void* Bm, int n_rows, float* out, int32_t* status,
+                        cudaStream_t st, const char* tag) {
     (void)P;
     CUtensorMap m_a, m_b;
     TcArgs a;
     memset(&a, 0, sizeof a);
     const int bn = n_rows % 256 == 0 ? 256 : 128;
-    MOE_TRY(tmap_bf16(&m_a, AT, m_rows, kcols, 128));
-    MOE_TRY(tmap_bf16(&m_b, BT, n_rows, kcols, bn));
+    MOE_TRY(tmap_bf16(&m_a, A, act_rows, m_rows, 64));
+    MOE_TRY(tmap_bf16(&m_b, Bm, act_rows, n_rows, 64));
     a.num_groups = groups;
     a.group_rows = rows;
+    a.group_off = offs;
     a.dense_rows = dense_rows;
     a.status = status;
     a.wait_limit_ns = g_wait_limit_ns;
@@ -784,29 +778,13 @@ static int run_tc_wgrad(const Plan& P, const Device& dv, int groups, const int32
     a.out = out;
     a.out_ld = n_rows;
     a.group_stride = (int64_t)m_rows * n_rows;
+    a.n_fastest = n_rows < m_rows ? 1 : 0;
     a.stages = tc_max_stages(TC_WGRAD, bn, 16, groups, dv.smem_optin);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag);
     MOE_TRY(launched(launch_tc_gemm(TC_WGRAD, bn, m_a, m_b, a, dv.sms, st), tag));
     trace_mark(st, tag);
     return MOE_OK;
-}
-
-static TransposeJob tjob(const void* src, int64_t src_ld, void* dst, int64_t dst_ld, int features,
-                         int groups, const int32_t* rows, const int32_t* off,
-                         const int32_t* kofs, int dense_rows) {
-    TransposeJob j;
-    j.src = src;
-    j.src_ld = src_ld;
-    j.dst = dst;
-    j.dst_ld = dst_ld;
-    j.features = features;
-    j.groups = groups;
-    j.rows = rows;
-    j.off = off;
-    j.kofs = kofs;
-    j.dense_rows = dense_rows;
-    return j;
 }
 
 }  // namespace moe
@@ -1169,8 +1147,6 @@ int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef, co
     float* dz = dlogits ? dlogits : at<float>(bws, P.b_dz);
     void* dAB = at<void>(bws, P.b_dAB);
     float* dXp = at<float>(bws, P.b_dXp);
-    int32_t* kofs = at<int32_t>(bws, P.b_kofs);
-    float* dXr = at<float>(bws, P.b_dXr);
     const int splits = P.path == PATH_SWAP ? P.splits : 1;
 
     // gate-scaled output gradients per kept slot, and the gate gradients
@@ -1192,32 +1168,28 @@ int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef, co
                                     cfg->has_bias ? db : nullptr, T, d, E, st),
                      "wr_grad"));
     trace_mark(st, "wr_grad");
-    trace_pre(st, "dxr");
-    MOE_TRY(launched(launch_dxr(dz, Wr, dXr, T, d, E, st), "dxr"));
-    trace_mark(st, "dxr");
 
     // routed experts: dAB, dX, then the weight gradients over each expert's tokens
     MOE_TRY(run_tc_backward(P, dv, E, kept, offsets, 0, P.perm_rows, dY, W2t, AB, dAB, W13t, dXp, h,
                             status, st, "gemm_dgate", "gemm_dx"));
-    trace_pre(st, "kofs");
-    MOE_TRY(launched(launch_kofs(kept, E, kofs, st), "kofs"));
-    trace_mark(st, "kofs");
-    void* XT = at<void>(bws, P.b_XT);
-    void* dYT = at<void>(bws, P.b_dYT);
-    void* HT = at<void>(bws, P.b_HT);
-    void* dABT = at<void>(bws, P.b_dABT);
-    TransposeJobs tj;
-    tj.n = 4;
-    tj.job[0] = tjob(x_perm, d, XT, P.kt, d, E, kept, offsets, kofs, 0);
-    tj.job[1] = tjob(dY, d, dYT, P.kt, d, E, kept, offsets, kofs, 0);
-    tj.job[2] = tjob(H, h, HT, P.kt, h, E, kept, offsets, kofs, 0);
-    tj.job[3] = tjob(dAB, 2 * h, dABT, P.kt, 2 * h, E, kept, offsets, kofs, 0);
-    trace_pre(st, "transpose");
-    MOE_TRY(launched(launch_transpose(tj, P.kt, st), "transpose"));
-    trace_mark(st, "transpose");
-    MOE_TRY(run_tc_wgrad(P, dv, E, kept, 0, dYT, d, HT, h, P.kt, dW2p, status, st, "gemm_dw2"));
-    MOE_TRY(run_tc_wgrad(P, dv, E, kept, 0, dABT, 2 * h, XT, d, P.kt, dW13, status, st,
-                         "gemm_dw13"));
+    // the rows between each expert's tokens and the next multiple of 64 are
+    // zeroed in the four activations the weight gradients contract
+    PadJobs pj;
+    pj.n = 4;
+    pj.job[0] = {const_cast<void*>(x_perm), d};
+    pj.job[1] = {const_cast<void*>(H), h};
+    pj.job[2] = {dY, d};
+    pj.job[3] = {dAB, 2 * h};
+    pj.off = offsets;
+    pj.rows = kept;
+    pj.groups = E;
+    trace_pre(st, "zero_pad");
+    MOE_TRY(launched(launch_zero_pad(pj, st), "zero_pad"));
+    trace_mark(st, "zero_pad");
+    MOE_TRY(run_tc_wgrad(P, dv, E, kept, offsets, 0, P.perm_rows, dY, d, H, h, dW2p, status, st,
+                         "gemm_dw2"));
+    MOE_TRY(run_tc_wgrad(P, dv, E, kept, offsets, 0, P.perm_rows, dAB, 2 * h, x_perm, d, dW13,
+                         status, st, "gemm_dw13"));
 
     // shared experts: gate 1, every token
     float* dXs = nullptr;
@@ -1229,28 +1201,15 @@ int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef, co
         MOE_TRY(run_tc_backward(P, dv, 1, nullptr, nullptr, (int)T, T, grad_out, W2st, ABs, dABs,
                                 W13st, dXs, P.hsum, status, st, "gemm_shared_dgate",
                                 "gemm_shared_dx"));
-        void* GT = at<void>(bws, P.b_GT);
-        void* xT = at<void>(bws, P.b_xT);
-        void* HsT = at<void>(bws, P.b_HsT);
-        void* dABsT = at<void>(bws, P.b_dABsT);
-        TransposeJobs ts;
-        ts.n = 4;
-        ts.job[0] = tjob(grad_out, d, GT, P.tp, d, 1, nullptr, nullptr, nullptr, (int)T);
-        ts.job[1] = tjob(x, d, xT, P.tp, d, 1, nullptr, nullptr, nullptr, (int)T);
-        ts.job[2] = tjob(Hs, P.hsum, HsT, P.tp, P.hsum, 1, nullptr, nullptr, nullptr, (int)T);
-        ts.job[3] = tjob(dABs, 2 * P.hsum, dABsT, P.tp, 2 * P.hsum, 1, nullptr, nullptr, nullptr,
-                         (int)T);
-        trace_pre(st, "shared_transpose");
-        MOE_TRY(launched(launch_transpose(ts, P.tp, st), "shared_transpose"));
-        trace_mark(st, "shared_transpose");
-        MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, (int)T, GT, d, HsT, P.hsum, P.tp, dW2s, status, st,
-                             "gemm_shared_dw2"));
-        MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, (int)T, dABsT, 2 * P.hsum, xT, d, P.tp, dW13s,
-                             status, st, "gemm_shared_dw13"));
+        MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, nullptr, (int)T, T, grad_out, d, Hs, P.hsum,
+                             dW2s, status, st, "gemm_shared_dw2"));
+        MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, nullptr, (int)T, T, dABs, 2 * P.hsum, x, d,
+                             dW13s, status, st, "gemm_shared_dw13"));
     }
 
     trace_pre(st, "combine_bwd");
-    MOE_TRY(launched(launch_combine_bwd(dXp, slot_of, dXs, dXr, dx, T, d, k, dv.sms, st),
+    MOE_TRY(launched(launch_combine_bwd(dXp, slot_of, dXs, dz, Wr, at<float>(bws, P.b_dxr), dx,
+                                        T, d, k, E, st),
                      "combine_bwd"));
     trace_mark(st, "combine_bwd");
     return ok();

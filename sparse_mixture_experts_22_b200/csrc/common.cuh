@@ -186,6 +186,27 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major tile stored with the
+// 128-byte swizzle, as TMA writes a box of 64 elements (128 B) of the M (or N)
+// dimension by rows of K: each K row is 128 B, 8-row swizzle atoms of 1 KB
+// follow one another along K (stride 1 KB), and the next 64 elements of M sit
+// `mn_stride` bytes further (the next TMA box).  K advances by whole rows.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t mn_stride) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address / 16
+    d |= (uint64_t)(mn_stride >> 4) << 16;     // leading byte offset: next 64 elements of M/N
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: next 8 rows of K
+    d |= (uint64_t)1 << 46;                    // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                    // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor as idesc_bf16_f32 with both operands MN-major
+// (the transpose bits of A and B).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N) {
+    return idesc_bf16_f32(M, N) | (1u << 15) | (1u << 16);
+}
+
 // 32 lanes x 32 bits, 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
     uint32_t r[16];
@@ -226,6 +247,16 @@ __device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float* v
     o1.w = pack_bf16x2(v[14], v[15]);
     reinterpret_cast<uint4*>(dst)[0] = o0;
     reinterpret_cast<uint4*>(dst)[1] = o1;
+}
+
+__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* src, float* v) {
+    const uint4 i0 = *reinterpret_cast<const uint4*>(src);
+    const uint32_t w[4] = {i0.x, i0.y, i0.z, i0.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
 }
 
 __device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* src, float* v) {

@@ -49,8 +49,18 @@ constexpr uint64_t TEARDOWN_NS = 200000000ull;  // 0.2 s bound on draining in-fl
 
 struct SharedLayout {
     uint32_t a_bytes, b_bytes, stage_bytes;
+    uint32_t stg_off;  // fp32 epilogue staging (token-major down, weight gradient)
     uint32_t bar_off, grp_off, total;
 };
+
+// fp32 epilogues stage each warp's 32 x 32 block in shared memory so that a
+// warp stores whole 128-byte row segments; rows padded to 36 floats.
+constexpr int STG_LD = 36;
+constexpr uint32_t STG_WARP_BYTES = 32 * STG_LD * 4;
+
+__host__ __device__ inline bool staged_epilogue(int mode) {
+    return mode == TC_DOWN_TOK || mode == TC_WGRAD;
+}
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
@@ -82,7 +92,8 @@ __host__ __device__ inline SharedLayout shared_layout(int mode, int bn, int nt_m
     L.a_bytes = align_up(L.a_bytes, 1024);
     L.b_bytes = align_up(L.b_bytes, 1024);
     L.stage_bytes = L.a_bytes + L.b_bytes;
-    L.bar_off = L.stage_bytes * stages;
+    L.stg_off = L.stage_bytes * stages;
+    L.bar_off = L.stg_off + (staged_epilogue(mode) ? 4 * STG_WARP_BYTES : 0);
     // full[S], empty[S], acc_full[2], acc_empty[2], drain, tmem slot
     L.grp_off = L.bar_off + align_up((2 * stages + 5) * 8 + 8, 16);
     L.total = L.grp_off + (3 * groups + 1) * 4 + 1024;  // + 1 KB for base alignment
@@ -133,10 +144,19 @@ __device__ __forceinline__ Unit decode_unit(const GroupTable& t, int u, const Tc
         x.mt = local % mtiles;
         x.nb = local / mtiles;
     } else if (MODE == TC_WGRAD) {
-        // the group's reduction range: its tokens, at 64-aligned offset row0
+        // the group's reduction range: its token rows, from the 64-aligned
+        // segment start row0 on, rounded up to 64 (the rows past the group's
+        // count are zero); the operand with fewer features is swept fastest
+        // so that it stays in L2 while the other streams once
         const int mtiles = a.m_rows / BM;
-        x.mt = local % mtiles;
-        x.nb = local / mtiles;
+        const int ntiles = a.n_feat / BN;
+        if (a.n_fastest) {
+            x.nb = local % ntiles;
+            x.mt = local / ntiles;
+        } else {
+            x.mt = local % mtiles;
+            x.nb = local / mtiles;
+        }
         x.kb0 = x.row0 / BK;
         x.kb1 = x.kb0 + (x.rows + BK - 1) / BK;
     } else if (MODE == TC_DOWN_TOK) {
@@ -176,6 +196,26 @@ __device__ __forceinline__ int units_of_group(int rows, const TcArgs& a) {
     if (MODE == TC_DOWN_TOK) return ((rows + BM - 1) / BM) * (a.n_feat / BN) * a.splits;
     if (MODE == TC_GATEUP_SWAP) return a.n_feat / 128;
     return (a.n_feat / 128) * a.splits;
+}
+
+// Stores 32 columns of fp32 for the warp's 32 rows: v holds row `lane`'s
+// values; row r of the block goes to dst_row0 + r * ld (columns 0..31), rows
+// at or past `valid` are skipped.  stg is the warp's staging buffer.
+__device__ __forceinline__ void store_rows_f32x32(float* stg, const float* v, int lane,
+                                                  float* dst_row0, int64_t ld, int valid) {
+    float4* srow = reinterpret_cast<float4*>(stg + lane * STG_LD);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) srow[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    __syncwarp();
+    const int sub = lane >> 3, col = (lane & 7) * 4;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + sub;
+        if (r < valid)
+            *reinterpret_cast<float4*>(dst_row0 + r * ld + col) =
+                *reinterpret_cast<const float4*>(stg + r * STG_LD + col);
+    }
+    __syncwarp();
 }
 
 template <int MODE, int BN>
@@ -239,15 +279,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_relinquish();
     }
     if (warp == 2 && lane == 0) {
-        int acc = 0, koff = 0;
+        int acc = 0;
         for (int g = 0; g < groups; ++g) {
             int r = args.group_rows ? args.group_rows[g] : args.dense_rows;
             int o = args.group_off ? args.group_off[g] : 0;
-            if (MODE == TC_WGRAD) {
-                // groups follow one another along K, each padded to a multiple of BK
-                o = koff;
-                koff += (r + BK - 1) / BK * BK;
-            }
             g_rows[g] = r;
             g_off[g] = o;
             g_start[g] = acc;
@@ -289,9 +324,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (TOK) {
                         mbar_arrive_expect_tx(&full[stage], (BM + BN) * BK * 2);
                         if (MODE == TC_WGRAD) {
-                            // both operands hold every group along K
-                            tma_load_2d(sa, &tm_act, &full[stage], kc, x.mt * BM);
-                            tma_load_2d(sb, &tm_w, &full[stage], kc, x.nb * BN);
+                            // MN-major operands straight from the row-major
+                            // activations: boxes of 64 features x 64 token rows
+#pragma unroll
+                            for (int i = 0; i < BM / 64; ++i)
+                                tma_load_2d(sa + i * 8192, &tm_act, &full[stage],
+                                            x.mt * BM + 64 * i, kc);
+#pragma unroll
+                            for (int i = 0; i < BN / 64; ++i)
+                                tma_load_2d(sb + i * 8192, &tm_w, &full[stage],
+                                            x.nb * BN + 64 * i, kc);
                         } else {
                             tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
                             tma_load_2d(sb, &tm_w, &full[stage], kc,
@@ -331,7 +373,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            const uint32_t idesc_tok = idesc_bf16_f32(BM, BN);
+            const uint32_t idesc_tok =
+                MODE == TC_WGRAD ? idesc_bf16_f32_mn(BM, BN) : idesc_bf16_f32(BM, BN);
             for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
                 const Unit x = decode_unit<MODE, BN>(tab, u, args);
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, limit)) {
@@ -353,6 +396,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
                         const uint32_t acc_flag = (kb > x.kb0 || kk > 0) ? 1u : 0u;
+                        if (MODE == TC_WGRAD) {
+                            // K steps of 16 rows of 128 B
+                            umma_bf16(d_tmem, sdesc_mnmajor_sw128(sa + kk * UK * 128, 8192),
+                                      sdesc_mnmajor_sw128(sb + kk * UK * 128, 8192), idesc,
+                                      acc_flag);
+                            continue;
+                        }
                         const uint64_t bdesc = sdesc_kmajor_sw128(sb + kk * UK * 2);
                         umma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * UK * 2), bdesc, idesc,
                                   acc_flag);
@@ -431,23 +481,37 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             } else if (MODE == TC_DOWN_TOK) {
-                const int r = x.mt * BM + row;
-                const bool valid = r < x.rows;
-                float* dst = reinterpret_cast<float*>(args.out) + x.ks * args.split_stride +
-                             (int64_t)(x.row0 + r) * args.out_ld + x.nb * BN;
-                // columns past out_cols (padding of the router GEMM) are not stored
-                const int ncol = args.out_cols > 0 ? min(BN, args.out_cols - x.nb * BN) : BN;
+                const int r0 = x.mt * BM + q * 32;  // first row of this warp's block
+                const int valid = min(32, x.rows - r0);
+                float* dst0 = reinterpret_cast<float*>(args.out) + x.ks * args.split_stride +
+                              (int64_t)(x.row0 + r0) * args.out_ld + x.nb * BN;
+                float* stg = reinterpret_cast<float*>(smem + L.stg_off) + q * (32 * STG_LD);
+                if (args.out_cols > 0) {
+                    // router GEMM: compact rows of out_cols columns (a multiple of
+                    // 4), stored thread by thread; padding columns are skipped
+                    const int ncol = min(BN, args.out_cols - x.nb * BN);
+                    float* dst = dst0 + (int64_t)lane * args.out_ld;
 #pragma unroll 1
-                for (int c = 0; c < ncol; c += 16) {
-                    float v[16];
-                    tmem_ld16(t0 + c, v);
-                    tmem_ld_wait();
-                    if (valid) {
+                    for (int c = 0; c < ncol; c += 16) {
+                        float v[16];
+                        tmem_ld16(t0 + c, v);
+                        tmem_ld_wait();
+                        if (lane < valid) {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4)
-                            if (c + i < ncol)
-                                *reinterpret_cast<float4*>(dst + c + i) =
-                                    make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                            for (int i = 0; i < 16; i += 4)
+                                if (c + i < ncol)
+                                    *reinterpret_cast<float4*>(dst + c + i) =
+                                        make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                        }
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 32) {
+                        float v[32];
+                        tmem_ld16(t0 + c, v);
+                        tmem_ld16(t0 + c + 16, v + 16);
+                        tmem_ld_wait();
+                        store_rows_f32x32(stg, v, lane, dst0 + c, args.out_ld, valid);
                     }
                 }
             } else if (MODE == TC_DGATE_TOK) {
@@ -459,17 +523,45 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int64_t rowoff = (int64_t)(x.row0 + r) * args.aux_ld;
                 const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(args.aux) + rowoff;
                 __nv_bfloat16* dab = reinterpret_cast<__nv_bfloat16*>(args.out) + rowoff;
+                // the pre-activations of the next 16 features are loaded while
+                // the current ones are used (the loads are the epilogue's latency)
+                auto ab_col = [&](int c) {
+                    const int f = x.nb * BN + c;
+                    return (int64_t)(f >> 7) * 256 + (f & 127);
+                };
+                uint4 na0 = make_uint4(0, 0, 0, 0), na1 = na0, nb0 = na0, nb1 = na0;
+                if (valid) {
+                    const uint4* pa = reinterpret_cast<const uint4*>(ab + ab_col(0));
+                    na0 = pa[0];
+                    na1 = pa[1];
+                    nb0 = pa[16];
+                    nb1 = pa[17];
+                }
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 16) {
                     float dh[16];
                     tmem_ld16(t0 + c, dh);
+                    const uint4 ca0 = na0, ca1 = na1, cb0 = nb0, cb1 = nb1;
+                    if (valid && c + 16 < BN) {
+                        const uint4* pa = reinterpret_cast<const uint4*>(ab + ab_col(c + 16));
+                        na0 = pa[0];
+                        na1 = pa[1];
+                        nb0 = pa[16];
+                        nb1 = pa[17];
+                    }
                     tmem_ld_wait();
                     if (valid) {
-                        const int f = x.nb * BN + c;
-                        const int64_t col = (int64_t)(f >> 7) * 256 + (f & 127);
+                        const int64_t col = ab_col(c);
                         float a[16], b[16], da[16], db[16];
-                        load_bf16x16(ab + col, a);
-                        load_bf16x16(ab + col + 128, b);
+                        const uint32_t wa[8] = {ca0.x, ca0.y, ca0.z, ca0.w, ca1.x, ca1.y, ca1.z, ca1.w};
+                        const uint32_t wb[8] = {cb0.x, cb0.y, cb0.z, cb0.w, cb1.x, cb1.y, cb1.z, cb1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            a[2 * i] = __uint_as_float(wa[i] << 16);
+                            a[2 * i + 1] = __uint_as_float(wa[i] & 0xFFFF0000u);
+                            b[2 * i] = __uint_as_float(wb[i] << 16);
+                            b[2 * i + 1] = __uint_as_float(wb[i] & 0xFFFF0000u);
+                        }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float sig = 1.0f / (1.0f + __expf(-a[i]));
@@ -481,23 +573,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             } else if (MODE == TC_WGRAD) {
-                float* dst = reinterpret_cast<float*>(args.out) + x.g * args.group_stride +
-                             (int64_t)(x.mt * BM + row) * args.out_ld + x.nb * BN;
+                float* dst0 = reinterpret_cast<float*>(args.out) + x.g * args.group_stride +
+                              (int64_t)(x.mt * BM + q * 32) * args.out_ld + x.nb * BN;
+                float* stg = reinterpret_cast<float*>(smem + L.stg_off) + q * (32 * STG_LD);
                 const bool empty = x.kb1 == x.kb0;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    float v[16];
+                for (int c = 0; c < BN; c += 32) {
+                    float v[32];
                     if (!empty) {
                         tmem_ld16(t0 + c, v);
+                        tmem_ld16(t0 + c + 16, v + 16);
                         tmem_ld_wait();
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
                     }
-#pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<float4*>(dst + c + i) =
-                            make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    store_rows_f32x32(stg, v, lane, dst0 + c, args.out_ld, 32);
                 }
             } else if (MODE == TC_GATEUP_SWAP) {
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +

@@ -116,6 +116,7 @@ struct TcArgs {
     int64_t aux_ld;             // elements per AB row (2 x hidden width)
     int m_rows;                 // wgrad: rows of A (output rows per group)
     int64_t group_stride;       // wgrad: elements between the groups' outputs
+    int n_fastest;              // wgrad: consecutive units step through N tiles first
 };
 
 int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);
@@ -176,34 +177,24 @@ int wr_grad_chunks(int64_t T, int d, int E);
 // dWr = x^T dz, db = column sums of dz (db may be null)
 int launch_wr_grad(const void* x, const float* dz, float* part, float* dWr, float* db, int64_t T,
                    int d, int E, cudaStream_t st);
-// dxr[t][c] = sum_e dz[t][e] Wr[c][e]
-int launch_dxr(const float* dz, const float* Wr, float* dxr, int64_t T, int d, int E,
-               cudaStream_t st);
-// kofs[g] = sum of rows[g'] rounded up to 64 over g' < g; kofs[G] = total
-int launch_kofs(const int32_t* rows, int G, int32_t* kofs, cudaStream_t st);
-
-struct TransposeJob {
-    const void* src;        // bf16 [rows][features], row stride src_ld
-    int64_t src_ld;
-    void* dst;              // bf16 [features][K], row stride dst_ld
-    int64_t dst_ld;
-    int features;           // multiple of 64
-    int groups;
-    const int32_t* rows;    // device [groups] rows per group (null: one dense group)
-    const int32_t* off;     // device [groups] first source row
-    const int32_t* kofs;    // device [groups + 1] first destination column
-    int dense_rows;
+struct PadJob {
+    void* buf;              // bf16 [rows][width], width a multiple of 8
+    int width;
 };
-struct TransposeJobs {
-    TransposeJob job[4];
+struct PadJobs {
+    PadJob job[4];
     int n;
+    const int32_t* off;     // device [groups] segment starts
+    const int32_t* rows;    // device [groups] rows in use
+    int groups;
 };
-// dst[f][kofs[g] + i] = src[off[g] + i][f], zero-filled to multiples of 64
-int launch_transpose(const TransposeJobs& jobs, int64_t k_bound, cudaStream_t st);
-// dx[t] = sum over kept slots of dXp[slot] + dXs[t] (may be null) + dXr[t]
+// zeroes rows [off[g] + rows[g], off[g] + rows[g] rounded up to 64) of each buffer
+int launch_zero_pad(const PadJobs& p, cudaStream_t st);
+// dx[t] = sum over kept slots of dXp[slot] + dXs[t] (may be null) + sum_e dz[t][e] Wr[:, e];
+// dxr [T][d] is scratch for the router's share when E > 16
 int launch_combine_bwd(const float* dXp, const int32_t* slot_of, const float* dXs,
-                       const float* dXr, float* dx, int64_t T, int d, int k, int num_sms,
-                       cudaStream_t st);
+                       const float* dz, const float* Wr, float* dxr, float* dx, int64_t T, int d,
+                       int k, int E, cudaStream_t st);
 // dst[r][col(c)] = src[r][c], bf16, no transpose (backward weight layout)
 int launch_pack_cols(const void* src, void* dst, int R, int Cc, int64_t ld_dst, int col_off,
                      int interleave, int n, int64_t src_stride, int64_t dst_stride, int col_step,

@@ -51,16 +51,13 @@ struct Plan {
     int router_ld;      // tensor cores: row length of the partial logits (3E rounded to 4)
     int router_splits;  // tensor cores: split-K
     bool train;         // forward keeps the gate/up pre-activations for the backward pass
-    int64_t kt;         // backward: columns of the transposed per-expert activations
-    int64_t tp;         // backward: T rounded up to 64 (transposed shared activations)
     int wr_chunks;      // backward: token chunks of the router-weight gradient
 
     // workspace byte offsets
     size_t off_status, off_logits, off_wsplit, off_z3, off_ppart, off_hpart, off_cnt, off_tot, off_expert, off_rank, off_offsets, off_perm,
         off_xperm, off_H, off_y, off_Hs, off_ys, off_sums, off_AB, off_ABs, total;
     // backward workspace byte offsets
-    size_t b_dY, b_dg, b_dz, b_dAB, b_dXp, b_kofs, b_XT, b_dYT, b_HT, b_dABT, b_dABs, b_dXs,
-        b_GT, b_xT, b_HsT, b_dABsT, b_wrpart, b_dXr, b_total;
+    size_t b_dY, b_dg, b_dz, b_dAB, b_dXp, b_dABs, b_dXs, b_wrpart, b_dxr, b_total;
 };
 
 // Fills *p; returns MOE_OK or an error code with the message in *why.
