@@ -539,10 +539,10 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
 // tokens beyond capacity, rerouting them to a spare expert].  Three steps:
 // rank_kernel records every assignment's rank in its expert's queue;
 // reroute_kernel visits the dropped ones in token order and moves each to the
-// token's best-scoring unused expert that still has room (it keeps its gate),
-// which is inherently sequential -- one warp walks the batch while the whole
-// CTA stages each chunk's logits in shared memory; place_kernel then writes
-// slots and copies rows as for the drop policy.
+// token's best-scoring unused expert that still has room (it keeps its gate);
+// the rule is sequential, and the kernel reproduces it in a few parallel
+// rounds (see reroute_kernel); place_kernel then writes slots and copies rows
+// as for the drop policy.
 
 __global__ void __launch_bounds__(ROUTE_BLOCK)
     rank_kernel(DispatchArgs a, const int32_t* __restrict__ topk_idx,
@@ -567,22 +567,27 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
             }
 }
 
-constexpr int RR_THREADS = 1024;
-constexpr int RR_MAX_ASSIGN = 2048;  // assignments staged per chunk
-
-__host__ __device__ inline int reroute_chunk_tokens(int E, int k) {
-    // logits (E floats) and choices (2k ints) per token within ~160 KB
-    int n = RR_MAX_ASSIGN / k;
-    const int by_smem = (160 * 1024) / (E * 4 + 2 * k * 4);
-    if (n > by_smem) n = by_smem;
-    return n < 1 ? 1 : n;
-}
+constexpr int RR_THREADS = 1024;  // one token per thread, chunks of 1024 tokens
 
 __host__ __device__ inline size_t reroute_smem_bytes(int E, int k) {
-    const int nt = reroute_chunk_tokens(E, k);
-    return sizeof(int32_t) * ((size_t)E + (size_t)nt * 2 * k) + sizeof(float) * (size_t)nt * E;
+    // fill [E] | warp sums [32] | control [4] | unresolved masks [1024] (int32)
+    // | picks and serving experts [1024][k] (int16) | ordered pick list [1024 k] (uint16)
+    return sizeof(int32_t) * ((size_t)E + 32 + 4 + RR_THREADS) +
+           3 * sizeof(int16_t) * (size_t)RR_THREADS * k;
 }
 
+// The reroute pass in rounds.  Each thread owns one token of a 1024-token
+// chunk.  In a round every thread picks, for each of its unresolved dropped
+// assignments in j order, the best-scoring expert (ties: lower index) that
+// still has room under the fill levels at the start of the round and that the
+// token does not use.  The picks are listed in (token, j) order and warp 0
+// commits them 32 at a time -- a pick's queue position is its expert's fill
+// plus the earlier picks of the same expert in the list (__match_any_sync) --
+// stopping at the first pick whose expert is full by then.  Up to that point
+// the picks equal those of the one-at-a-time rule (room only shrinks, so an
+// expert that was best with room stays best while it has room); the next
+// round re-picks from there.  Every stop leaves one more expert full, so a
+// chunk takes at most E + 1 rounds.
 __global__ void __launch_bounds__(RR_THREADS)
     reroute_kernel(const int32_t* __restrict__ topk_idx, int32_t* __restrict__ expert_of,
                    int32_t* __restrict__ rank_of, const int32_t* __restrict__ tot,
@@ -590,78 +595,135 @@ __global__ void __launch_bounds__(RR_THREADS)
                    int k, int64_t C, int pad, int32_t* __restrict__ routed,
                    int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
     extern __shared__ int32_t sm[];
-    const int nt = reroute_chunk_tokens(E, k);
-    int32_t* fill = sm;                     // [E]
-    int32_t* cidx = fill + E;               // [nt][k] router choices
-    int32_t* cexp = cidx + nt * k;          // [nt][k] serving experts
-    float* cz = reinterpret_cast<float*>(cexp + nt * k);  // [nt][E] logits + bias
+    int32_t* fill = sm;                                            // [E]
+    int32_t* wsum = fill + E;                                      // [32] per-warp pick counts
+    int32_t* ctl = wsum + 32;                                      // [0] done, [1] list length
+    uint32_t* um = reinterpret_cast<uint32_t*>(ctl + 4);           // [1024] unresolved j bits
+    int16_t* pick = reinterpret_cast<int16_t*>(um + RR_THREADS);   // [1024][k]
+    int16_t* srv = pick + RR_THREADS * k;                          // [1024][k] serving experts
+    uint16_t* plist = reinterpret_cast<uint16_t*>(srv + RR_THREADS * k);  // [1024 k] tl*8 + j
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int e = tid; e < E; e += RR_THREADS) {
         fill[e] = capped(tot[e], C);
         routed[e] = tot[e];
     }
-    __syncthreads();
-    for (int64_t t0 = 0; t0 < T; t0 += nt) {
-        const int n = (int)(T - t0 < nt ? T - t0 : nt);
-        const int64_t a0 = t0 * k;
-        // anything dropped in this chunk?
-        int any = 0;
-        for (int i = tid; i < n * k; i += RR_THREADS) any |= (int64_t)rank_of[a0 + i] >= C;
-        if (!__syncthreads_or(any)) continue;
-        for (int i = tid; i < n * k; i += RR_THREADS) {
-            cidx[i] = topk_idx[a0 + i];
-            cexp[i] = cidx[i];
+    for (int64_t t0 = 0; t0 < T; t0 += RR_THREADS) {
+        const int64_t t = t0 + tid;
+        const bool have = t < T;
+        int32_t ch[MAX_K];
+        uint32_t unres = 0;
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) {
+            ch[j] = (have && j < k) ? topk_idx[t * k + j] : -1;
+            if (have && j < k) {
+                srv[tid * k + j] = (int16_t)ch[j];
+                if ((int64_t)rank_of[t * k + j] >= C) unres |= 1u << j;
+            }
         }
-        for (int i = tid; i < n * E; i += RR_THREADS) {
-            const int e = i % E;
-            const float v = z[t0 * E + i];
-            cz[i] = bias ? v + bias[e] : v;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            for (int i0 = 0; i0 < n * k; i0 += 32) {
-                const int i = i0 + lane;
-                const bool dropped = i < n * k && (int64_t)rank_of[a0 + i] >= C;
-                unsigned m = __ballot_sync(0xffffffffu, dropped);
-                while (m) {
-                    const int b = __ffs(m) - 1;
-                    m &= m - 1;
-                    const int ii = i0 + b;
-                    const int tl = ii / k;
-                    // best-scoring expert with room that the token does not use
+        um[tid] = unres;
+        if (!__syncthreads_or(unres != 0)) continue;
+        for (int round = 0; round <= E + 1; ++round) {
+            // ------------------------------------------------ picks (all threads)
+            if (unres) {
+                const float* zt = z + t * E;
+                int32_t mine[MAX_K];  // experts this token picked earlier in the round
+#pragma unroll
+                for (int j = 0; j < MAX_K; ++j) mine[j] = -1;
+                for (int j = 0; j < k; ++j) {
+                    if (!((unres >> j) & 1u)) continue;
+                    int best = -1;
                     float bv = -INFINITY;
-                    int be = 0x7fffffff;
-                    for (int e = lane; e < E; e += 32) {
+                    for (int e = 0; e < E; ++e) {
                         if ((int64_t)fill[e] >= C) continue;
                         bool used = false;
                         for (int q = 0; q < k; ++q)
-                            used |= (cidx[tl * k + q] == e) || (cexp[tl * k + q] == e);
+                            used |= ch[q] == e || srv[tid * k + q] == e || mine[q] == e;
                         if (used) continue;
-                        const float v = cz[tl * E + e];
-                        const float vv = v != v ? -INFINITY : v;
-                        if (be == 0x7fffffff || vv > bv) {
-                            bv = vv;
-                            be = e;
+                        const float v = finite_or_minus_inf(zt[e] + (bias ? bias[e] : 0.0f));
+                        if (best < 0 || v > bv) {
+                            best = e;
+                            bv = v;
                         }
                     }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                        if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-                            bv = ov;
-                            be = oe;
-                        }
-                    }
-                    if (be != 0x7fffffff && lane == 0) {
-                        cexp[ii] = be;
-                        expert_of[a0 + ii] = be;
-                        rank_of[a0 + ii] = fill[be];
-                        fill[be] += 1;
-                    }
-                    __syncwarp();
+                    pick[tid * k + j] = (int16_t)best;
+                    mine[j] = best;
                 }
             }
+            // ------------------------------------------------ ordered pick list (block scan)
+            const int cnt = __popc(unres);
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (lane == 31) wsum[warp] = incl;
+            __syncthreads();
+            if (warp == 0) {
+                int w = wsum[lane];
+                int wi = w;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, wi, o);
+                    if (lane >= o) wi += v;
+                }
+                wsum[lane] = wi - w;  // exclusive prefix of the warp totals
+                if (lane == 31) ctl[1] = wi;
+            }
+            __syncthreads();
+            {
+                int pos = wsum[warp] + incl - cnt;
+                uint32_t u = unres;
+                while (u) {
+                    const int j = __ffs(u) - 1;
+                    u &= u - 1;
+                    plist[pos++] = (uint16_t)(tid * 8 + j);
+                }
+            }
+            __syncthreads();
+            // ------------------------------------------------ commit walk (warp 0)
+            if (warp == 0) {
+                const int n = ctl[1];
+                bool cut = false;
+                for (int base = 0; base < n && !cut; base += 32) {
+                    const int i = base + lane;
+                    const bool act = i < n;
+                    const int ent = act ? plist[i] : 0;
+                    const int tl = ent >> 3, j = ent & 7;
+                    const int p = act ? pick[tl * k + j] : -1;
+                    // inactive lanes and picks without room get keys no one else has
+                    const int key = (act && p >= 0) ? p : -1 - lane;
+                    const uint32_t grp = __match_any_sync(0xffffffffu, key);
+                    const int before = __popc(grp & ((1u << lane) - 1u));
+                    const int f = (act && p >= 0) ? fill[p] : 0;
+                    const bool full = act && p >= 0 && (int64_t)(f + before) >= C;
+                    const uint32_t fullm = __ballot_sync(0xffffffffu, full);
+                    const int lim = fullm ? __ffs(fullm) - 1 : 32;
+                    const bool commit = act && lane < lim;
+                    const uint32_t cm = __ballot_sync(0xffffffffu, commit);
+                    if (commit) {
+                        if (p >= 0) {
+                            const int64_t g = (t0 + tl) * k + j;
+                            srv[tl * k + j] = (int16_t)p;
+                            expert_of[g] = p;
+                            rank_of[g] = f + before;
+                        }
+                        // p < 0: no expert has room; the assignment stays dropped
+                        atomicAnd(&um[tl], ~(1u << j));
+                    }
+                    // the last committing pick of each expert advances its fill
+                    const uint32_t mine_c = grp & cm;
+                    if (commit && p >= 0 && (31 - __clz(mine_c)) == lane) fill[p] = f + before + 1;
+                    __syncwarp();
+                    cut = fullm != 0;
+                }
+                if (lane == 0) ctl[0] = cut ? 0 : 1;
+            }
+            __syncthreads();
+            unres = um[tid];
+            const bool done = ctl[0] != 0;
+            __syncthreads();
+            if (done) break;
         }
         __syncthreads();
     }
