@@ -278,6 +278,66 @@ MOE_API int moe_backward(const moe_config* cfg, const void* grad_out, float aux_
                          float* dW13, float* dW2p, float* dW13s, float* dW2s, float* dlogits,
                          void* bws, size_t bws_bytes, void* stream);
 
+/* ---- expert parallelism --------------------------------------------------- */
+
+/* Building blocks of the layer with its experts partitioned across G ranks
+ * [Mixtral explained, "Easy explanation" ¶4 and MoE routing fully explained,
+ * ¶3: experts spread over GPUs, tokens sent to the GPU that holds their
+ * expert].  The reading the library implements: G ranks with their own
+ * batches together compute exactly the single-GPU layer on the concatenated
+ * batch (rank 0's tokens first): capacity C = ceil(T_all k cf / E) and the
+ * arrival order run over the whole concatenation.  A rank calls moe_route on
+ * its batch (with a local config whose cf_den = 0), exchanges the per-expert
+ * counts (moe_route_counts), keeps for expert e at most
+ * cap[e] = C - (assignments to e on lower ranks) with moe_dispatch_capped,
+ * sends each expert's rows to its owner, which runs moe_expert_ffn_grouped on
+ * the (source rank, expert) groups it received, and gets the output rows back
+ * for moe_combine.  The host-side plan and the exchanges live in the Python
+ * package (ep.py). */
+
+/* Row padding of each expert segment in x_perm for this config (the
+ * receiver of a segment needs it to find the next one). */
+MOE_API int moe_segment_pad(const moe_config* cfg, int32_t* pad);
+
+/* counts[e] (device int32 [E]) = assignments of the batch to expert e,
+ * before any capacity limit.  Call after moe_route and before any dispatch
+ * on the same ws (dispatch consumes the router's histograms). */
+MOE_API int moe_route_counts(const moe_config* cfg, const void* ws, size_t ws_bytes,
+                             int32_t* counts, void* stream);
+
+/* moe_dispatch with a per-expert capacity: expert e keeps the first
+ * min(C, cap[e]) of the batch's assignments to it (token order); cap is
+ * device int32 [E] (negative counts as 0).  Drop policy only. */
+MOE_API int moe_dispatch_capped(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                                const int32_t* cap, int32_t* routed, int32_t* kept,
+                                int32_t* offsets, int32_t* perm_token, int32_t* slot_of,
+                                void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace of moe_expert_ffn_grouped for `rows` input rows. */
+MOE_API int moe_grouped_workspace_size(const moe_config* cfg, int64_t rows,
+                                       int32_t max_group_rows, size_t* bytes);
+
+/* The expert FFN (as moe_expert_ffn, bf16) over explicit groups of rows:
+ * group g is rows group_off[g] .. + group_rows[g] of x_rows [rows][d] and uses
+ * expert group_weight[g] of W13 / W2p (packed as moe_pack_weights which = 0,
+ * holding however many experts the caller owns; every index must be below
+ * that count).  All three arrays are device int32 [n_groups]; max_group_rows
+ * (host) bounds every group_rows[g] -- a larger one is clamped and
+ * MOE_ERR_SHAPE recorded in ws's status word.  y_rows [rows][d] fp32 receives
+ * the outputs of the group rows (other rows are not written). */
+MOE_API int moe_expert_ffn_grouped(const moe_config* cfg, const void* x_rows, int64_t rows,
+                                   int32_t n_groups, const int32_t* group_rows,
+                                   const int32_t* group_off, const int32_t* group_weight,
+                                   int32_t max_group_rows, const void* W13, const void* W2p,
+                                   float* y_rows, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_combine with the expert outputs in one fp32 buffer y_rows [rows][d]
+ * (no split-K partials), e.g. as returned by the expert owners: out[t] =
+ * sum over kept j of gate * y_rows[slot_of[t][j]] (+ y_shared[t]). */
+MOE_API int moe_combine_rows(const moe_config* cfg, const float* y_rows, const int32_t* slot_of,
+                             const float* topk_gate, const float* y_shared, void* out,
+                             void* stream);
+
 /* ---- routing without a workspace ----------------------------------------- */
 
 /* The pages have no counterpart to this call; it exists for callers that

@@ -28,7 +28,8 @@ EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_split
            "moe_combine", "moe_aux_stats", "moe_stats_sums", "moe_stats_finalize", "moe_forward",
            "moe_read_device_status", "moe_set_wait_limit_ns", "moe_set_test_stall",
            "moe_trace_begin", "moe_trace_end", "moe_backward_workspace_size", "moe_backward",
-           "moe_launch_count"]
+           "moe_launch_count", "moe_segment_pad", "moe_route_counts", "moe_dispatch_capped",
+           "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows"]
 
 
 class MoEError(RuntimeError):
@@ -91,6 +92,13 @@ def load() -> ctypes.CDLL:
             "moe_trace_end": [P, P, P, I, P],
             "moe_backward_workspace_size": [C, P],
             "moe_launch_count": [P],
+            "moe_segment_pad": [C, P],
+            "moe_route_counts": [C, P, S, P, P],
+            "moe_dispatch_capped": [C, P, P, P, P, P, P, P, P, P, P, S, P],
+            "moe_grouped_workspace_size": [C, ctypes.c_int64, ctypes.c_int32, P],
+            "moe_combine_rows": [C, P, P, P, P, P, P],
+            "moe_expert_ffn_grouped": [C, P, ctypes.c_int64, ctypes.c_int32, P, P, P,
+                                       ctypes.c_int32, P, P, P, P, S, P],
             "moe_backward": [C, P, ctypes.c_float, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P,
                              P, P, P, P, P, P, P, P, S, P],
         }
@@ -250,6 +258,45 @@ def moe_read_device_status(ws, stream=None) -> int:
     v = ctypes.c_int32()
     _check(load().moe_read_device_status(_p(ws), ctypes.byref(v), _stream(stream)))
     return v.value
+
+
+def moe_segment_pad(cfg: MoEConfig) -> int:
+    v = ctypes.c_int32()
+    _check(load().moe_segment_pad(ctypes.byref(cfg), ctypes.byref(v)))
+    return v.value
+
+
+def moe_route_counts(cfg, ws, counts, stream=None):
+    _check(load().moe_route_counts(ctypes.byref(cfg), _p(ws), ws.numel() * ws.element_size(),
+                                   _p(counts), _stream(stream)))
+
+
+def moe_dispatch_capped(cfg, topk_idx, x, cap, routed, kept, offsets, perm_token, slot_of,
+                        x_perm, ws, stream=None):
+    _check(load().moe_dispatch_capped(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(cap),
+                                      _p(routed), _p(kept), _p(offsets), _p(perm_token),
+                                      _p(slot_of), _p(x_perm), _p(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_grouped_workspace_size(cfg, rows: int, max_group_rows: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().moe_grouped_workspace_size(ctypes.byref(cfg), int(rows), int(max_group_rows),
+                                             ctypes.byref(v)))
+    return v.value
+
+
+def moe_expert_ffn_grouped(cfg, x_rows, rows, group_rows, group_off, group_weight,
+                           max_group_rows, W13, W2p, y_rows, ws, stream=None):
+    _check(load().moe_expert_ffn_grouped(
+        ctypes.byref(cfg), _p(x_rows), int(rows), int(group_rows.numel()), _p(group_rows),
+        _p(group_off), _p(group_weight), int(max_group_rows), _p(W13), _p(W2p), _p(y_rows),
+        _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_combine_rows(cfg, y_rows, slot_of, topk_gate, y_shared, out, stream=None):
+    _check(load().moe_combine_rows(ctypes.byref(cfg), _p(y_rows), _p(slot_of), _p(topk_gate),
+                                   _p(y_shared), _p(out), _stream(stream)))
 
 
 def moe_launch_count() -> int:

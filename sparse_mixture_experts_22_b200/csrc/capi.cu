@@ -471,6 +471,7 @@ static DispatchParams dispatch_params(const Plan& P, const void* x, int32_t* rou
     d.perm_token = perm_token;
     d.slot_of = slot_of;
     d.x_perm = x_perm;
+    d.cap = nullptr;
     return d;
 }
 
@@ -548,7 +549,8 @@ static int step_route_dispatch(const Plan& P, const Device& dv, const void* x, c
 
 // One grouped GEMM pair (gate/up then down) on the tensor cores.
 static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
-                      const int32_t* rows, const int32_t* offs, int dense_rows, const void* act,
+                      const int32_t* rows, const int32_t* offs, const int32_t* group_w,
+                      int dense_rows, const void* act,
                       int64_t act_rows, const void* W13, const void* W2p, int hid, void* H,
                       void* AB, float* y, int splits, int nt_max, int32_t* status,
                       cudaStream_t st, const char* tag1, const char* tag2) {
@@ -559,6 +561,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.num_groups = groups;
     a.group_rows = rows;
     a.group_off = offs;
+    a.group_w = group_w;
     a.dense_rows = dense_rows;
     a.status = status;
     a.wait_limit_ns = g_wait_limit_ns;
@@ -627,7 +630,8 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
         trace_mark(st, "f32_down");
     } else {
         void* AB = P.train ? at<void>(ws, P.off_AB) : nullptr;
-        MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, 0, x_perm, P.perm_rows, W13, W2p,
+        MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, nullptr, 0, x_perm, P.perm_rows,
+                           W13, W2p,
                            P.h, H, AB, y_perm, P.splits, P.nt_max, status, st, "gemm_gateup",
                            "gemm_down"));
     }
@@ -648,7 +652,8 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
         } else {
             const int nt = (int)((P.T + 15) / 16 * 16);
             void* ABs = P.train ? at<void>(ws, P.off_ABs) : nullptr;
-            MOE_TRY(run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, (int)P.T, x, P.T, W13s,
+            MOE_TRY(run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, nullptr, (int)P.T, x,
+                               P.T, W13s,
                                W2s, P.hsum, Hs, ABs, y_shared, 1, nt, status, st,
                                "gemm_shared_gateup", "gemm_shared_down"));
         }
@@ -1062,6 +1067,136 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
         MOE_TRY(step_combine(P, y, slot_of, topk_gate, ys, out, stats ? &sp : nullptr, st));
     else if (stats)
         MOE_TRY(step_stats(P, routed, kept, ws, at<double>(ws, P.off_sums), stats, st));
+    return ok();
+}
+
+// ---------------------------------------------------------------- expert parallelism
+
+int moe_segment_pad(const moe_config* cfg, int32_t* pad) {
+    if (!pad) return fail(MOE_ERR_ARG, "pad is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    *pad = P.pad;
+    return ok();
+}
+
+int moe_route_counts(const moe_config* cfg, const void* ws, size_t ws_bytes, int32_t* counts,
+                     void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(counts, "counts"));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (P.T == 0) {
+        if (cudaMemsetAsync(counts, 0, (size_t)P.E * 4, st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "memset failed");
+        return ok();
+    }
+    MOE_TRY(launched(launch_route_counts(at<int32_t>(ws, P.off_cnt), P.nblk, P.E, counts, st),
+                     "route_counts"));
+    return ok();
+}
+
+int moe_dispatch_capped(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                        const int32_t* cap, int32_t* routed, int32_t* kept, int32_t* offsets,
+                        int32_t* perm_token, int32_t* slot_of, void* x_perm, void* ws,
+                        size_t ws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (P.reroute) return fail(MOE_ERR_UNSUPPORTED, "moe_dispatch_capped: the drop policy only");
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(cap, "cap"));
+    MOE_TRY(need(routed, "routed"));
+    MOE_TRY(need(kept, "kept"));
+    MOE_TRY(need(offsets, "offsets"));
+    if (P.T > 0) {
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(x, "x"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(need(x_perm, "x_perm"));
+        MOE_TRY(maybe(perm_token, "perm_token"));
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st) == MOE_OK ? ok() : MOE_ERR_CUDA;
+    DispatchParams d = dispatch_params(P, x, routed, kept, offsets, perm_token, slot_of, x_perm);
+    d.cap = cap;
+    MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
+                                     at<int32_t>(ws, P.off_tot), dv.sms, st),
+                     "dispatch"));
+    return ok();
+}
+
+int moe_combine_rows(const moe_config* cfg, const float* y_rows, const int32_t* slot_of,
+                     const float* topk_gate, const float* y_shared, void* out, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (P.T > 0) {
+        MOE_TRY(need(y_rows, "y_rows"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(need(topk_gate, "topk_gate"));
+        MOE_TRY(need(out, "out"));
+        if (P.S > 0) MOE_TRY(need(y_shared, "y_shared"));
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    trace_pre(st, "combine");
+    MOE_TRY(launched(launch_combine(y_rows, 1, 0, slot_of, topk_gate,
+                                    P.S > 0 ? y_shared : nullptr, out, P.bf16, P.T, P.d, P.k,
+                                    nullptr, st),
+                     "combine"));
+    trace_mark(st, "combine");
+    return ok();
+}
+
+static size_t grouped_h_offset() { return 256; }
+
+int moe_grouped_workspace_size(const moe_config* cfg, int64_t rows, int32_t max_group_rows,
+                               size_t* bytes) {
+    if (!bytes) return fail(MOE_ERR_ARG, "bytes is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (rows < 0 || max_group_rows < 0) return fail(MOE_ERR_ARG, "rows and max_group_rows must be >= 0");
+    *bytes = grouped_h_offset() + align256((size_t)rows * P.h * P.act_bytes);
+    return ok();
+}
+
+int moe_expert_ffn_grouped(const moe_config* cfg, const void* x_rows, int64_t rows,
+                           int32_t n_groups, const int32_t* group_rows, const int32_t* group_off,
+                           const int32_t* group_weight, int32_t max_group_rows, const void* W13,
+                           const void* W2p, float* y_rows, void* ws, size_t ws_bytes,
+                           void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (!P.bf16) return fail(MOE_ERR_DTYPE, "moe_expert_ffn_grouped: bf16 only");
+    if (rows < 0 || n_groups < 0 || n_groups > 65536 || max_group_rows < 0)
+        return fail(MOE_ERR_ARG, "moe_expert_ffn_grouped: bad sizes");
+    if (!ws) return fail(MOE_ERR_ARG, "ws is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(MOE_ERR_ALIGN, "ws is not 256-byte aligned");
+    const size_t need_bytes = grouped_h_offset() + align256((size_t)rows * P.h * P.act_bytes);
+    if (ws_bytes < need_bytes)
+        return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes; this call needs %zu", ws_bytes,
+                    need_bytes);
+    if (rows == 0 || n_groups == 0) return ok();
+    MOE_TRY(need(x_rows, "x_rows"));
+    MOE_TRY(need(group_rows, "group_rows"));
+    MOE_TRY(need(group_off, "group_off"));
+    MOE_TRY(need(group_weight, "group_weight"));
+    MOE_TRY(need(W13, "W13"));
+    MOE_TRY(need(W2p, "W2p"));
+    MOE_TRY(need(y_rows, "y_rows"));
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int nmax = max_group_rows > 0 ? max_group_rows : 1;
+    const int path = nmax <= SWAP_MAX_TOKENS ? PATH_SWAP : PATH_TOKEN_MAJOR;
+    const int nt_max = (nmax + 15) / 16 * 16;
+    int32_t* status = at<int32_t>(ws, 0);
+    if (cudaMemsetAsync(status, 0, 4, st) != cudaSuccess) return fail(MOE_ERR_CUDA, "memset failed");
+    void* H = at<void>(ws, grouped_h_offset());
+    MOE_TRY(run_tc_ffn(P, dv, path, n_groups, group_rows, group_off, group_weight, 0, x_rows, rows,
+                       W13, W2p, P.h, H, nullptr, y_rows, 1, nt_max, status, st,
+                       "gemm_grouped_gateup", "gemm_grouped_down"));
     return ok();
 }
 

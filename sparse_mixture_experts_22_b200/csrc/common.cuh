@@ -271,7 +271,7 @@ __device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* src, float* v)
 }
 
 // Device status word codes (stored in the workspace).
-enum : int32_t { DEV_OK = 0, DEV_TIMEOUT = 7 };
+enum : int32_t { DEV_OK = 0, DEV_SHAPE = 2, DEV_TIMEOUT = 7 };
 
 __device__ __forceinline__ void report_timeout(int32_t* status) {
     if (status) atomicCAS(status, DEV_OK, DEV_TIMEOUT);

@@ -96,13 +96,14 @@ __host__ __device__ inline SharedLayout shared_layout(int mode, int bn, int nt_m
     L.bar_off = L.stg_off + (staged_epilogue(mode) ? 4 * STG_WARP_BYTES : 0);
     // full[S], empty[S], acc_full[2], acc_empty[2], drain, tmem slot
     L.grp_off = L.bar_off + align_up((2 * stages + 5) * 8 + 8, 16);
-    L.total = L.grp_off + (3 * groups + 1) * 4 + 1024;  // + 1 KB for base alignment
+    L.total = L.grp_off + (4 * groups + 1) * 4 + 1024;  // + 1 KB for base alignment
     return L;
 }
 
 // Where one unit of work sits.
 struct Unit {
     int g;        // group
+    int w;        // weight index of the group
     int rows;     // valid rows of the group
     int row0;     // first row of the group in the activation/output tensors
     int mt, nb;   // token-major: m tile, n tile;  swapped: feature block
@@ -115,6 +116,7 @@ struct GroupTable {
     const int* start;  // [groups + 1] unit prefix
     const int* rows;   // [groups]
     const int* off;    // [groups]
+    const int* wi;     // [groups] weight index
     int groups;
 };
 
@@ -131,6 +133,7 @@ template <int MODE, int BN>
 __device__ __forceinline__ Unit decode_unit(const GroupTable& t, int u, const TcArgs& a) {
     Unit x;
     x.g = find_group(t, u);
+    x.w = t.wi[x.g];
     x.rows = t.rows[x.g];
     x.row0 = t.off[x.g];
     const int local = u - t.start[x.g];
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int* g_start = reinterpret_cast<int*>(smem + L.grp_off);
     int* g_rows = g_start + groups + 1;
     int* g_off = g_rows + groups;
+    int* g_wi = g_off + groups;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -283,7 +287,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int g = 0; g < groups; ++g) {
             int r = args.group_rows ? args.group_rows[g] : args.dense_rows;
             int o = args.group_off ? args.group_off[g] : 0;
+            if (!TOK && r > args.nt_max) {
+                // a swapped tile holds at most nt_max token columns: clamp and
+                // flag the oversized group rather than overrun shared memory
+                if (args.status) atomicCAS(args.status, DEV_OK, DEV_SHAPE);
+                r = args.nt_max;
+            }
             g_rows[g] = r;
+            g_wi[g] = args.group_w ? args.group_w[g] : g;
             g_off[g] = o;
             g_start[g] = acc;
             acc += units_of_group<MODE, BN>(r, args);
@@ -294,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    GroupTable tab{g_start, g_rows, g_off, groups};
+    GroupTable tab{g_start, g_rows, g_off, g_wi, groups};
     const int total = g_start[groups];
     const uint64_t limit = args.wait_limit_ns;
 
@@ -337,13 +348,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                         } else {
                             tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
                             tma_load_2d(sb, &tm_w, &full[stage], kc,
-                                        x.g * args.w_rows_per_group +
+                                        x.w * args.w_rows_per_group +
                                             x.nb * (MODE == TC_GATEUP_TOK ? 256 : BN));
                         }
                     } else {
                         const int wa = (MODE == TC_GATEUP_SWAP) ? 2 * BM : BM;
                         mbar_arrive_expect_tx(&full[stage], (wa + x.ntok) * BK * 2);
-                        const int wrow = x.g * args.w_rows_per_group +
+                        const int wrow = x.w * args.w_rows_per_group +
                                          x.nb * (MODE == TC_GATEUP_SWAP ? 256 : BM);
                         tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
                         if (MODE == TC_GATEUP_SWAP)

@@ -66,9 +66,13 @@ struct DispatchParams {
     int32_t* perm_token;    // may be null
     int32_t* slot_of;
     void* x_perm;
+    const int32_t* cap;     // device [E] per-expert capacity (min with C), or null
 };
 
 int launch_topk(const RouteParams& r, cudaStream_t st);
+// counts[e] = routed assignments of the batch to expert e, from the top-k
+// histograms cnt [blocks][E] (before dispatch turns them into prefixes)
+int launch_route_counts(const int32_t* cnt, int nblk, int E, int32_t* counts, cudaStream_t st);
 // cnt [blocks][E] is turned in place into exclusive prefixes over blocks;
 // tot [E] receives the totals
 int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* cnt, int32_t* tot,
@@ -117,6 +121,7 @@ struct TcArgs {
     int m_rows;                 // wgrad: rows of A (output rows per group)
     int64_t group_stride;       // wgrad: elements between the groups' outputs
     int n_fastest;              // wgrad: consecutive units step through N tiles first
+    const int32_t* group_w;     // device [num_groups] weight index of each group, or null -> g
 };
 
 int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);

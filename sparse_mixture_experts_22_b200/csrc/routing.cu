@@ -312,7 +312,14 @@ struct DispatchArgs {
     int32_t* perm_token;   // [perm_rows] (may be null)
     int32_t* slot_of;      // [T][k]
     uint4* x_perm;         // [perm_rows][d]
+    const int32_t* cap;    // [E] per-expert capacity (min with C), or null
 };
+
+__device__ __forceinline__ int64_t expert_cap(const DispatchArgs& a, int e) {
+    if (!a.cap) return a.C;
+    const int64_t c = a.cap[e];
+    return c < a.C ? (c < 0 ? 0 : c) : a.C;
+}
 
 // Shared memory of the dispatch kernels: base [E], tot [E], rows [E],
 // off [E+1], wcnt [DWARPS][E], slots [ROUTE_BLOCK * k].
@@ -415,7 +422,8 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
         if (j >= k) break;
         int32_t slot = -1;
         if (valid) {
-            if (rank[j] >= 0 && (int64_t)rank[j] < a.C) slot = d.off[expert[j]] + rank[j];
+            if (rank[j] >= 0 && (int64_t)rank[j] < expert_cap(a, expert[j]))
+                slot = d.off[expert[j]] + rank[j];
             if (writer) {
                 a.slot_of[t * k + j] = slot;
                 if (slot >= 0 && a.perm_token) a.perm_token[slot] = (int32_t)t;
@@ -459,7 +467,7 @@ __device__ void dispatch_block(const DispatchArgs& a, int blk, int nblk, bool wr
                                int nsplit, const DispatchSmem& d, const int32_t* my) {
     const int E = a.E;
     const int tid = threadIdx.x;
-    for (int e = tid; e < E; e += ROUTE_BLOCK) d.rows[e] = capped(d.tot[e], a.C);
+    for (int e = tid; e < E; e += ROUTE_BLOCK) d.rows[e] = capped(d.tot[e], expert_cap(a, e));
     __syncthreads();
     segment_offsets(d.rows, E, a.pad, d.off);
     __syncthreads();
@@ -489,6 +497,20 @@ __global__ void __launch_bounds__(TK_WIDE_THREADS)
     __syncthreads();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x)
         cnt[(int64_t)blockIdx.x * a.E + e] = hist[e];
+}
+
+// counts[e] = sum over routing blocks of the histograms (the batch's routed
+// assignments per expert).  One warp per expert; integer sums.
+__global__ void route_counts_kernel(const int32_t* __restrict__ cnt, int nblk, int E,
+                                    int32_t* __restrict__ counts) {
+    const int e = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (e >= E) return;
+    int32_t s = 0;
+    for (int b = lane; b < nblk; b += 32) s += cnt[(int64_t)b * E + e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) counts[e] = s;
 }
 
 // Per expert e, the exclusive prefix over blocks of the histograms (in place:
@@ -830,6 +852,7 @@ DispatchArgs dispatch_args(const DispatchParams& p) {
     a.perm_token = p.perm_token;
     a.slot_of = p.slot_of;
     a.x_perm = reinterpret_cast<uint4*>(p.x_perm);
+    a.cap = p.cap;
     return a;
 }
 
@@ -843,6 +866,13 @@ int copy_splits(int nblk, int64_t T, int k, int num_sms) {
 }
 
 }  // namespace
+
+int launch_route_counts(const int32_t* cnt, int nblk, int E, int32_t* counts, cudaStream_t st) {
+    const int64_t threads = (int64_t)E * 32;
+    route_counts_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(cnt, nblk, E, counts);
+    note_launch();
+    return launch_result();
+}
 
 int launch_topk(const RouteParams& r, cudaStream_t st) {
     if (r.T == 0) return 0;

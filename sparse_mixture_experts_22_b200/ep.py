@@ -1,0 +1,269 @@
+"""Expert parallelism: the layer with its routed experts partitioned over G ranks.
+
+The pages' own multi-GPU story [Mixtral 8x7B and MoE explained, "Easy
+explanation" ¶4: the experts can be spread over GPUs; MoE routing fully
+explained, "Easy explanation" ¶3: tokens travel to the GPU that holds their
+expert, and the busiest expert sets the step time].  Rank r holds the experts
+r*E/G .. (r+1)*E/G - 1 and its own batch of tokens; the router weights are
+replicated.
+
+Reading taken: G ranks compute exactly the single-GPU layer on the
+concatenation of their batches (rank 0's tokens first).  The capacity is
+C = ceil(T_all k cf / E) over the whole concatenation, and an expert's queue
+fills in that arrival order: rank r may keep, for expert e, at most
+cap[r][e] = C - (assignments to e on lower ranks).  One step:
+
+  1. every rank routes its tokens (moe_route) and reads its per-expert counts
+     (moe_route_counts); the counts are all-gathered (G x E int32);
+  2. every rank computes the same plan from the counts (`make_plan`) and
+     dispatches under its caps (moe_dispatch_capped): its x_perm holds one
+     padded segment per expert, the segments of each destination contiguous;
+  3. all-to-all of the segment rows: rank r receives, from every source, the
+     rows of its own experts;
+  4. the owner runs the expert FFN on the (source, expert) groups it received
+     (moe_expert_ffn_grouped, fp32 rows out);
+  5. all-to-all back (the reverse splits): the output rows land where their
+     input rows were in the source's x_perm;
+  6. moe_combine_rows forms the outputs with the gates; the statistics are
+     summed across ranks as in data parallelism.
+
+The exchanges are torch.distributed collectives (NCCL between GPUs, gloo on
+the host in the tests) or, for one process standing in for G ranks on one
+GPU, plain copies (`forward_emulated`).  Only the routed experts are
+partitioned; the overflow policy is drop.
+"""
+
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+def capacity(T_all: int, k: int, E: int, cf) -> int:
+    """C = ceil(T_all k cf / E) in integers; no limit (cf None) -> T_all."""
+    if cf is None:
+        return T_all
+    num, den = cf
+    return ceil_div(T_all * k * num, E * den)
+
+
+@dataclass
+class Plan:
+    """The host-side plan of one step, identical on every rank."""
+    G: int
+    E: int
+    E_loc: int
+    C: int
+    pad: int
+    counts: np.ndarray            # [G][E] routed assignments, before the capacity
+    cap: np.ndarray = field(init=False)    # [G][E] per-rank capacity of each expert
+    kept: np.ndarray = field(init=False)   # [G][E] rows each rank keeps for each expert
+    seg: np.ndarray = field(init=False)    # [G][E] padded segment rows in the sender's x_perm
+    send: np.ndarray = field(init=False)   # [G][G] rows rank r sends to rank q
+
+    def __post_init__(self):
+        c = self.counts.astype(np.int64)
+        base = np.cumsum(c, axis=0) - c          # assignments to e on lower ranks
+        self.cap = np.clip(self.C - base, 0, None)
+        self.kept = np.minimum(c, self.cap)
+        self.seg = ceil_div_arr(self.kept, self.pad) * self.pad
+        self.send = self.seg.reshape(self.G, self.G, self.E_loc).sum(axis=2)
+
+    def owner(self, e: int) -> int:
+        return e // self.E_loc
+
+    def recv_rows(self, rank: int) -> np.ndarray:
+        """Rows rank `rank` receives from each source."""
+        return self.send[:, rank]
+
+    def groups(self, rank: int):
+        """(rows, first row, weight index) of every (source, local expert)
+        group in rank `rank`'s receive buffer, sources in order, then experts."""
+        rows, off, wi = [], [], []
+        at = 0
+        for src in range(self.G):
+            for el in range(self.E_loc):
+                e = rank * self.E_loc + el
+                rows.append(int(self.kept[src, e]))
+                off.append(at)
+                wi.append(el)
+                at += int(self.seg[src, e])
+        return np.array(rows, np.int32), np.array(off, np.int32), np.array(wi, np.int32)
+
+
+def ceil_div_arr(a: np.ndarray, b: int) -> np.ndarray:
+    return -(-a // b)
+
+
+def make_plan(counts: np.ndarray, T_all: int, k: int, E: int, cf, pad: int) -> Plan:
+    G = counts.shape[0]
+    if E % G:
+        raise ValueError("E must be a multiple of the number of ranks")
+    return Plan(G=G, E=E, E_loc=E // G, C=capacity(T_all, k, E, cf), pad=pad,
+                counts=np.asarray(counts, np.int64))
+
+
+# ---------------------------------------------------------------- exchanges
+
+def send_splits(plan: Plan, rank: int) -> List[int]:
+    return [int(v) for v in plan.send[rank]]
+
+
+def recv_splits(plan: Plan, rank: int) -> List[int]:
+    return [int(v) for v in plan.recv_rows(rank)]
+
+
+def exchange_rows(send: torch.Tensor, plan: Plan, rank: int, group=None) -> torch.Tensor:
+    """Step 3: rank `rank` sends its x_perm segments to their experts' owners
+    and receives its experts' rows from every source (source order)."""
+    import torch.distributed as dist
+    rs = recv_splits(plan, rank)
+    recv = torch.empty((sum(rs),) + tuple(send.shape[1:]), dtype=send.dtype, device=send.device)
+    dist.all_to_all_single(recv, send[:sum(send_splits(plan, rank))].contiguous(), rs,
+                           send_splits(plan, rank), group=group)
+    return recv
+
+
+def exchange_back(y: torch.Tensor, plan: Plan, rank: int, group=None) -> torch.Tensor:
+    """Step 5: the owner returns the output rows; they land where the input
+    rows were in each source's x_perm."""
+    import torch.distributed as dist
+    ss = send_splits(plan, rank)
+    back = torch.empty((sum(ss),) + tuple(y.shape[1:]), dtype=y.dtype, device=y.device)
+    dist.all_to_all_single(back, y.contiguous(), ss, recv_splits(plan, rank), group=group)
+    return back
+
+
+def all_gather_counts(counts: torch.Tensor, world: int, group=None) -> np.ndarray:
+    """Step 1's exchange: every rank's per-expert counts, [G][E]."""
+    import torch.distributed as dist
+    parts = [torch.empty_like(counts) for _ in range(world)]
+    dist.all_gather(parts, counts.contiguous(), group=group)
+    return torch.stack(parts).cpu().numpy().astype(np.int64)
+
+
+# ---------------------------------------------------------------- one rank
+
+class Rank:
+    """One rank's layer state: its batch, the replicated router, its experts'
+    packed weights, and the buffers of one step."""
+
+    def __init__(self, wl, rank: int, world: int, x, Wr, bias, W13_loc, W2p_loc):
+        if wl.E % world:
+            raise ValueError("E must be a multiple of the number of ranks")
+        if wl.n_shared or wl.overflow != "drop" or wl.dtype != "bf16":
+            raise ValueError("expert parallelism: bf16, routed experts, drop policy")
+        self.wl, self.rank, self.world = wl, rank, world
+        T = x.shape[0]
+        dev = x.device
+        # locally no capacity limit: the global one arrives as per-expert caps
+        self.cfg = B.make_config(T, wl.d, wl.h, wl.E, wl.k, dtype=wl.dtype,
+                                 has_bias=wl.has_bias)
+        self.x, self.Wr, self.bias = x, Wr, bias
+        self.W13, self.W2p = W13_loc, W2p_loc
+        self.pad = B.moe_segment_pad(self.cfg)
+        rows = max(B.moe_perm_rows(self.cfg), 1)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.b = {
+            "topk_idx": torch.empty((T, wl.k), **i32),
+            "topk_gate": torch.empty((T, wl.k), dtype=torch.float32, device=dev),
+            "counts": torch.empty(wl.E, **i32),
+            "routed": torch.empty(wl.E, **i32),
+            "kept": torch.empty(wl.E, **i32),
+            "offsets": torch.empty(wl.E + 1, **i32),
+            "perm_token": torch.empty(rows, **i32),
+            "slot_of": torch.empty((T, wl.k), **i32),
+            "x_perm": torch.empty((rows, wl.d), dtype=x.dtype, device=dev),
+            "out": torch.empty((T, wl.d), dtype=x.dtype, device=dev),
+            "sums": torch.zeros(2 + 3 * wl.E, dtype=torch.float64, device=dev),
+            "ws": torch.empty(max(B.moe_workspace_size(self.cfg), 256), dtype=torch.uint8,
+                              device=dev),
+        }
+
+    def route(self) -> torch.Tensor:
+        b = self.b
+        B.moe_route(self.cfg, self.x, self.Wr, self.bias if self.wl.has_bias else None,
+                    b["topk_idx"], b["topk_gate"], b["ws"])
+        B.moe_route_counts(self.cfg, b["ws"], b["counts"])
+        return b["counts"]
+
+    def dispatch(self, plan: Plan) -> torch.Tensor:
+        b = self.b
+        cap = torch.tensor(plan.cap[self.rank].clip(max=2 ** 31 - 1), dtype=torch.int32,
+                           device=self.x.device)
+        B.moe_dispatch_capped(self.cfg, b["topk_idx"], self.x, cap, b["routed"], b["kept"],
+                              b["offsets"], b["perm_token"], b["slot_of"], b["x_perm"], b["ws"])
+        return b["x_perm"][:int(plan.seg[self.rank].sum())]
+
+    def ffn(self, plan: Plan, recv: torch.Tensor) -> torch.Tensor:
+        rows, off, wi = plan.groups(self.rank)
+        dev = self.x.device
+        y = torch.empty((recv.shape[0], self.wl.d), dtype=torch.float32, device=dev)
+        if recv.shape[0] == 0:
+            return y
+        mx = int(rows.max()) if rows.size else 0
+        ws = torch.empty(B.moe_grouped_workspace_size(self.cfg, recv.shape[0], mx),
+                         dtype=torch.uint8, device=dev)
+        B.moe_expert_ffn_grouped(self.cfg, recv, recv.shape[0], torch.from_numpy(rows).to(dev),
+                                 torch.from_numpy(off).to(dev), torch.from_numpy(wi).to(dev), mx,
+                                 self.W13, self.W2p, y, ws)
+        self.ffn_ws = ws
+        return y
+
+    def combine(self, y_back: torch.Tensor) -> torch.Tensor:
+        b = self.b
+        B.moe_combine_rows(self.cfg, y_back, b["slot_of"], b["topk_gate"], None, b["out"])
+        return b["out"]
+
+    def stats_sums(self) -> torch.Tensor:
+        b = self.b
+        B.moe_stats_sums(self.cfg, b["routed"], b["kept"], b["ws"], b["sums"])
+        return b["sums"]
+
+
+# ---------------------------------------------------------------- drivers
+
+def forward_dist(r: Rank, T_all: int, group=None):
+    """One step on this rank, the exchanges as torch.distributed collectives.
+    Returns (out, stats tensor, plan)."""
+    counts = all_gather_counts(r.route(), r.world, group)
+    plan = make_plan(counts, T_all, r.wl.k, r.wl.E, r.wl.cf, r.pad)
+    recv = exchange_rows(r.dispatch(plan), plan, r.rank, group)
+    back = exchange_back(r.ffn(plan, recv), plan, r.rank, group)
+    out = r.combine(back)
+    import torch.distributed as dist
+    sums = r.stats_sums()
+    dist.all_reduce(sums, group=group)
+    stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
+    B.moe_stats_finalize(r.cfg, sums, stats)
+    return out, stats, plan
+
+
+def forward_emulated(ranks: List[Rank], T_all: int):
+    """G ranks in one process on one device: the same phases, rank by rank,
+    with the exchanges done as copies (no kernel waits on another).  Returns
+    ([out per rank], stats tensor, plan)."""
+    G = len(ranks)
+    counts = np.stack([r.route().cpu().numpy() for r in ranks]).astype(np.int64)
+    wl = ranks[0].wl
+    plan = make_plan(counts, T_all, wl.k, wl.E, wl.cf, ranks[0].pad)
+    sends = [r.dispatch(plan) for r in ranks]
+    starts = np.concatenate([np.zeros((G, 1), np.int64), np.cumsum(plan.send, axis=1)], axis=1)
+    recvs = [torch.cat([sends[s][starts[s, q]:starts[s, q + 1]] for s in range(G)])
+             for q in range(G)]
+    ys = [ranks[q].ffn(plan, recvs[q]) for q in range(G)]
+    rstarts = [np.concatenate([[0], np.cumsum(plan.recv_rows(q))]) for q in range(G)]
+    backs = [torch.cat([ys[q][rstarts[q][s]:rstarts[q][s + 1]] for q in range(G)])
+             for s in range(G)]
+    outs = [ranks[s].combine(backs[s]) for s in range(G)]
+    sums = sum(r.stats_sums().clone() for r in ranks)
+    stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
+    B.moe_stats_finalize(ranks[0].cfg, sums, stats)
+    return outs, stats, plan
