@@ -256,7 +256,8 @@ __global__ void __launch_bounds__(256)
                        const float* __restrict__ dXs, const float* __restrict__ dz,
                        const float* __restrict__ Wr, const float* __restrict__ dxr,
                        float* __restrict__ dx, int64_t T, int d, int k, int E) {
-    __shared__ float zs[CB_TOK][EREG > 0 ? EREG : 1];
+    constexpr int ER = EREG > 0 ? EREG : 1;
+    __shared__ float zs[CB_TOK][ER];
     __shared__ int32_t slots[CB_TOK][8];
     const int64_t t0 = (int64_t)blockIdx.y * CB_TOK;
     const int c = (blockIdx.x * 256 + threadIdx.x) * 4;
@@ -266,8 +267,8 @@ __global__ void __launch_bounds__(256)
     }
     float w[4][EREG > 0 ? EREG : 1];
     if (EREG > 0) {
-        for (int i = threadIdx.x; i < CB_TOK * EREG; i += 256) {
-            const int tt = i / EREG, e = i % EREG;
+        for (int i = threadIdx.x; i < CB_TOK * ER; i += 256) {
+            const int tt = i / ER, e = i % ER;
             zs[tt][e] = (t0 + tt < T && e < E) ? dz[(t0 + tt) * E + e] : 0.0f;
         }
 #pragma unroll
