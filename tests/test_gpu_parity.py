@@ -43,6 +43,9 @@ SMALL = {
                            cf=(1, 2), dtype="f32", zipf_s=1.0),
     # degenerate: one token; one expert; k = E; heavy skew
     "one_token": Workload("one_token", T=1, d=128, h=128, E=8, k=2),
+    # shared expert on 200 tokens: swapped gate/up tiles of 64 gate + 64 up rows
+    "shared_swap64": Workload("shared_swap64", T=200, d=256, h=256, E=8, k=2, n_shared=1,
+                              h_shared=256, cf=(1, 1)),
     "one_expert": Workload("one_expert", T=130, d=128, h=256, E=1, k=1),
     "k_equals_E": Workload("k_equals_E", T=64, d=128, h=128, E=4, k=4),
     "top1": Workload("top1", T=257, d=256, h=128, E=8, k=1, cf=(2, 1)),
