@@ -65,6 +65,8 @@ def parse():
                    help="override the expert hidden width (small profiling cases only)")
     p.add_argument("--graph", action="store_true",
                    help="capture one step in a CUDA graph and replay it (1 GPU)")
+    p.add_argument("--no-pdl", action="store_true",
+                   help="launch the forward chain without programmatic dependent launch")
     p.add_argument("--backward", action="store_true",
                    help="time forward + backward (a training step) instead of the forward (1 GPU)")
     return p.parse_args()
@@ -390,6 +392,7 @@ def main():
         wl = wl.scaled(overflow=args.overflow)
     if args.backward and world > 1:
         raise SystemExit("--backward runs on one GPU")
+    B.moe_set_pdl(not args.no_pdl)
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward
     cfg, host, g, W, Wb = build_inputs(wl, rank, world, dev, keep_host=want_cpu,
                                        train=args.backward)

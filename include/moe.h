@@ -373,6 +373,13 @@ MOE_API int moe_read_device_status(const void* ws, int32_t* status, void* stream
  * launches in between). */
 MOE_API int moe_launch_count(uint64_t* n);
 
+/* Programmatic dependent launch inside moe_forward (default on): the
+ * kernels of the layer's chain may start while their predecessor finishes,
+ * each waiting on the device before it reads what the predecessor writes, and
+ * the swapped gate/up GEMM prefetches its first weight tiles into L2 while the
+ * routing runs.  Results are identical either way.  Process-wide. */
+MOE_API int moe_set_pdl(int on);
+
 /* Upper bound, in nanoseconds, on every device-side wait of the tensor-core
  * kernels (default 2e9).  A wait that runs out records MOE_ERR_TIMEOUT in
  * the device status word and its kernel returns early.  Process-wide. */

@@ -29,7 +29,7 @@ EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_split
            "moe_read_device_status", "moe_set_wait_limit_ns", "moe_set_test_stall",
            "moe_trace_begin", "moe_trace_end", "moe_backward_workspace_size", "moe_backward",
            "moe_launch_count", "moe_segment_pad", "moe_route_counts", "moe_dispatch_capped",
-           "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows"]
+           "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows", "moe_set_pdl"]
 
 
 class MoEError(RuntimeError):
@@ -97,6 +97,7 @@ def load() -> ctypes.CDLL:
             "moe_dispatch_capped": [C, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_grouped_workspace_size": [C, ctypes.c_int64, ctypes.c_int32, P],
             "moe_combine_rows": [C, P, P, P, P, P, P],
+            "moe_set_pdl": [I],
             "moe_expert_ffn_grouped": [C, P, ctypes.c_int64, ctypes.c_int32, P, P, P,
                                        ctypes.c_int32, P, P, P, P, S, P],
             "moe_backward": [C, P, ctypes.c_float, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P,
@@ -303,6 +304,10 @@ def moe_launch_count() -> int:
     v = ctypes.c_uint64()
     _check(load().moe_launch_count(ctypes.byref(v)))
     return v.value
+
+
+def moe_set_pdl(on: bool):
+    _check(load().moe_set_pdl(1 if on else 0))
 
 
 def moe_set_wait_limit_ns(ns: int):

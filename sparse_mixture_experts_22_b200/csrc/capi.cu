@@ -280,6 +280,18 @@ static int tmap_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
     return MOE_OK;
 }
 
+// ---------------------------------------------------------------- dependent launch
+
+static int g_pdl_enabled = 1;
+static thread_local bool g_pdl_in_forward = false;
+
+bool pdl_active() { return g_pdl_enabled && g_pdl_in_forward; }
+
+struct PdlScope {
+    PdlScope() { g_pdl_in_forward = true; }
+    ~PdlScope() { g_pdl_in_forward = false; }
+};
+
 // ---------------------------------------------------------------- launch count
 
 static std::atomic<uint64_t> g_launches{0};
@@ -583,6 +595,9 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.aux = AB;  // pre-activations for the backward pass (null: not kept)
     a.aux_ld = 2 * (int64_t)hid;
     a.stages = tc_max_stages(mode1, 256, nt_max, groups, smem_limit);
+    // while the routing finishes, prefetch the start of each CTA's first weight
+    // tile (the unit it gets when every expert has tokens) into L2
+    a.prefetch_kb = (!tok && !group_w && pdl_active()) ? 16 : 0;
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag1);
     MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
@@ -601,6 +616,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.out_ld = P.d;
     a.split_stride = act_rows * (int64_t)P.d;
     a.aux = nullptr;
+    a.prefetch_kb = 0;
     a.stages = tc_max_stages(mode2, bn, nt_max, groups, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag2);
@@ -1053,6 +1069,7 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
     MOE_TRY(device_facts(&dv));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     trace_call_begin(st);
+    PdlScope pdl;  // the forward chain's kernels may overlap their predecessors' tails
     int32_t* offsets = at<int32_t>(ws, P.off_offsets);
     int32_t* perm = at<int32_t>(ws, P.off_perm);
     void* x_perm = at<void>(ws, P.off_xperm);
@@ -1368,6 +1385,11 @@ int moe_read_device_status(const void* ws, int32_t* status, void* stream) {
 int moe_launch_count(uint64_t* n) {
     if (!n) return fail(MOE_ERR_ARG, "n is NULL");
     *n = g_launches.load(std::memory_order_relaxed);
+    return ok();
+}
+
+int moe_set_pdl(int on) {
+    g_pdl_enabled = on ? 1 : 0;
     return ok();
 }
 

@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(256)
                    const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
                    const float* __restrict__ ys, void* __restrict__ out, int64_t T, int d, int k,
                    StatsParams sp) {
+    pdl_wait();
     if (sp.sums && blockIdx.x == gridDim.x - 1) {
         stats_block(sp);
         return;
@@ -104,9 +105,36 @@ __global__ void __launch_bounds__(256)
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    if (splits == 1) {
+        // every kept row's 32 bytes are requested before any is used, so the
+        // k loads of a thread are in flight together
+        float4 ra[MAX_K], rb[MAX_K];
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) {
+            ra[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            rb[j] = ra[j];
+            if (slot[j] >= 0) {
+                const float* p = y + (int64_t)slot[j] * d + c;
+                ra[j] = __ldg(reinterpret_cast<const float4*>(p));
+                rb[j] = __ldg(reinterpret_cast<const float4*>(p + 4));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) {
+            if (slot[j] < 0) continue;
+            acc[0] = fmaf(g[j], ra[j].x, acc[0]);
+            acc[1] = fmaf(g[j], ra[j].y, acc[1]);
+            acc[2] = fmaf(g[j], ra[j].z, acc[2]);
+            acc[3] = fmaf(g[j], ra[j].w, acc[3]);
+            acc[4] = fmaf(g[j], rb[j].x, acc[4]);
+            acc[5] = fmaf(g[j], rb[j].y, acc[5]);
+            acc[6] = fmaf(g[j], rb[j].z, acc[6]);
+            acc[7] = fmaf(g[j], rb[j].w, acc[7]);
+        }
+    }
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
-        if (slot[j] < 0) continue;
+        if (splits == 1 || slot[j] < 0) continue;
         float v[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) v[q] = 0.f;
@@ -187,11 +215,11 @@ int launch_combine(const float* y, int splits, int64_t split_stride, const int32
     const StatsParams& s = sp ? *sp : none;
     const unsigned blocks = (unsigned)((n + 255) / 256) + (sp ? 1 : 0);
     if (out_bf16)
-        combine_kernel<true><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
-                                                     y_shared, out, T, d, k, s);
+        launch_ex(pdl_active(), combine_kernel<true>, dim3(blocks), dim3(256), 0, st, y, splits,
+                  split_stride, slot_of, gate, y_shared, out, T, d, k, s);
     else
-        combine_kernel<false><<<blocks, 256, 0, st>>>(y, splits, split_stride, slot_of, gate,
-                                                      y_shared, out, T, d, k, s);
+        launch_ex(pdl_active(), combine_kernel<false>, dim3(blocks), dim3(256), 0, st, y, splits,
+                  split_stride, slot_of, gate, y_shared, out, T, d, k, s);
     note_launch();
     return launch_result();
 }

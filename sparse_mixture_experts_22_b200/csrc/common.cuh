@@ -114,6 +114,27 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// L2 prefetch of one box of a 2-D tensor map (no shared memory, no multicast).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+// ---------------------------------------------------------------- dependent launch
+
+// A kernel launched with programmatic stream serialization may start while
+// its predecessor in the stream still runs.  pdl_wait() blocks until the
+// predecessor has completed and its writes are visible (it returns at once
+// for a kernel launched without the attribute); pdl_trigger() lets the
+// successor begin launching.  Every kernel that can be launched this way
+// calls pdl_wait() before it touches memory another kernel writes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 // Allocate ncols (power of two >= 32) TMEM columns; the address lands in

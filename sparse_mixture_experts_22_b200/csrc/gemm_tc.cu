@@ -282,6 +282,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
     }
+    if (MODE == TC_GATEUP_SWAP && args.prefetch_kb > 0 && warp == 0 && lane == 0) {
+        // the predecessor (routing) may still run: prefetch into L2 the start of
+        // the weight tile this CTA's first unit has when every expert has tokens
+        // (a wrong guess only wastes the prefetch; weights are never written)
+        const int ub = args.n_feat / 128;
+        const int u = blockIdx.x;
+        if (u < args.num_groups * ub) {
+            const int wrow = (u / ub) * args.w_rows_per_group + (u % ub) * 256;
+            const int nk = min(args.prefetch_kb, args.K / BK);
+            for (int kb = 0; kb < nk; ++kb) {
+                tma_prefetch_2d(&tm_w, kb * BK, wrow);
+                tma_prefetch_2d(&tm_w, kb * BK, wrow + BM);
+            }
+        }
+    }
+    // everything below may read what the previous kernel in the stream wrote
+    pdl_wait();
+    pdl_trigger();
     if (warp == 2 && lane == 0) {
         int acc = 0;
         for (int g = 0; g < groups; ++g) {
@@ -667,7 +685,7 @@ int launch_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, i
             return -1;
         configured_bytes = L.total;
     }
-    kern<<<grid, THREADS, L.total, st>>>(act, w, a);
+    launch_ex(pdl_active(), kern, dim3(grid), dim3(THREADS), L.total, st, act, w, a);
     note_launch();
     return launch_result();
 }

@@ -14,6 +14,28 @@ void note_launch();
 // The calling thread's error of its last failed launch (cudaSuccess if none).
 cudaError_t& last_launch_error();
 
+// True while moe_forward launches its kernels on this thread: the kernels of
+// its chain are then launched with programmatic stream serialization (they
+// call pdl_wait() before touching memory their predecessor writes).
+bool pdl_active();
+
+// Launches `kern`, with programmatic stream serialization when `pdl` is set.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_ex(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                             size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = grid;
+    c.blockDim = block;
+    c.dynamicSmemBytes = smem;
+    c.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    c.attrs = pdl ? at : nullptr;
+    c.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&c, kern, args...);
+}
+
 // 0 if the launches so far succeeded; else records the error and returns -1.
 inline int launch_result() {
     const cudaError_t e = cudaGetLastError();
@@ -122,6 +144,8 @@ struct TcArgs {
     int64_t group_stride;       // wgrad: elements between the groups' outputs
     int n_fastest;              // wgrad: consecutive units step through N tiles first
     const int32_t* group_w;     // device [num_groups] weight index of each group, or null -> g
+    int prefetch_kb;            // swapped gate/up: k-blocks of the first weight tile to prefetch
+                                // into L2 before waiting on the predecessor (0: none)
 };
 
 int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);

@@ -203,6 +203,8 @@ __global__ void __launch_bounds__(RR_THREADS)
     router_rows_kernel(const XT* __restrict__ x, const float* __restrict__ Wr,
                        float* __restrict__ z, int d, int E) {
     __shared__ float red[RR_THREADS / 32][RT_EXP];
+    pdl_wait();
+    pdl_trigger();
     const int t = blockIdx.x;
     const int e0 = blockIdx.y * RT_EXP;
     const int ne = min(RT_EXP, E - e0);
@@ -334,11 +336,11 @@ int launch_router_rows(const void* x, bool x_bf16, const float* Wr, float* z, in
     if (T == 0) return 0;
     dim3 grid(T, (E + RT_EXP - 1) / RT_EXP);
     if (x_bf16)
-        router_rows_kernel<__nv_bfloat16><<<grid, RR_THREADS, 0, st>>>(
-            reinterpret_cast<const __nv_bfloat16*>(x), Wr, z, d, E);
+        launch_ex(pdl_active(), router_rows_kernel<__nv_bfloat16>, grid, dim3(RR_THREADS), 0, st,
+                  reinterpret_cast<const __nv_bfloat16*>(x), Wr, z, d, E);
     else
-        router_rows_kernel<float><<<grid, RR_THREADS, 0, st>>>(reinterpret_cast<const float*>(x),
-                                                               Wr, z, d, E);
+        launch_ex(pdl_active(), router_rows_kernel<float>, grid, dim3(RR_THREADS), 0, st,
+                  reinterpret_cast<const float*>(x), Wr, z, d, E);
     note_launch();
     return launch_result();
 }

@@ -787,6 +787,8 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
 __global__ void __launch_bounds__(ROUTE_BLOCK)
     route_dispatch_kernel(TopkArgs ta, DispatchArgs da, int32_t* __restrict__ cnt) {
     extern __shared__ int32_t dyn[];
+    pdl_wait();
+    pdl_trigger();
     const int E = ta.E;
     int32_t* hist = dyn;
     float* zs = reinterpret_cast<float*>(dyn + E);
@@ -937,8 +939,8 @@ int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num
     if (r.T > ROUTE_BLOCK) return -1;
     const size_t smem = topk_smem_bytes(r.E, ROUTE_BLOCK) + dispatch_smem_bytes(p.E, p.k);
     if (set_smem(route_dispatch_kernel, smem)) return -1;
-    route_dispatch_kernel<<<copy_splits(1, p.T, p.k, num_sms), ROUTE_BLOCK, smem, st>>>(
-        topk_args(r), dispatch_args(p), r.cnt);
+    launch_ex(pdl_active(), route_dispatch_kernel, dim3(copy_splits(1, p.T, p.k, num_sms)),
+              dim3(ROUTE_BLOCK), smem, st, topk_args(r), dispatch_args(p), r.cnt);
     note_launch();
     return launch_result();
 }

@@ -174,3 +174,22 @@ def test_full_size_workload(name):
     ref = oracle_rows(wl, inp, r, rows)
     e = check_output(b["out"][torch.as_tensor(rows, device="cuda")], ref, f"{name} sampled rows")
     print(f"{name}: {e} logit_err={zerr:.2e}")
+
+
+@pytest.mark.parametrize("name", ["swap", "tok_cap", "shared"])
+def test_dependent_launch_gives_identical_bits(name):
+    """The forward chain launched with and without programmatic dependent
+    launch (and the gate/up weight prefetch it enables) gives the same bits."""
+    wl = SMALL[name]
+    inp = host_inputs(wl)
+    cfg, g, W = device_layer(wl, inp)
+    B.moe_set_pdl(True)
+    a = run_forward(cfg, g, W)
+    out_on = a["out"].clone()
+    try:
+        B.moe_set_pdl(False)
+        b = run_forward(cfg, g, W)
+    finally:
+        B.moe_set_pdl(True)
+    assert torch.equal(out_on, b["out"])
+    assert B.moe_read_device_status(b["ws"]) == 0
