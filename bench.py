@@ -403,19 +403,26 @@ def main():
     sums = torch.zeros(dp.sums_len(wl.E), dtype=torch.float64, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def layer(x, out, stats, G=None, dx=None):
+        """One step of the public API on the given input and output buffers."""
         if world == 1:
-            B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
+            B.moe_forward(cfg, x, g["Wr"], g["bias"], W13, W2p, W13s, W2s, out,
                           bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
-                          bufs["slot_of"], bufs["stats"], bufs["ws"])
+                          bufs["slot_of"], stats, bufs["ws"])
             if args.backward:
-                B.backward(cfg, g["G"], AUX_COEF, g["x"], g["Wr"], g["bias"], W13t, W2t, W13st,
-                           W2st, bufs, grads)
+                gr = dict(grads)
+                gr["dx"] = dx
+                B.backward(cfg, G, AUX_COEF, x, g["Wr"], g["bias"], W13t, W2t, W13st, W2st, bufs,
+                           gr)
         else:
-            B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
+            B.moe_forward(cfg, x, g["Wr"], g["bias"], W13, W2p, W13s, W2s, out,
                           bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
                           bufs["slot_of"], None, bufs["ws"])
-            dp.global_stats(cfg, bufs["routed"], bufs["kept"], bufs["ws"], sums, bufs["stats"])
+            dp.global_stats(cfg, bufs["routed"], bufs["kept"], bufs["ws"], sums, stats)
+
+    def step():
+        layer(g["x"], bufs["out"], bufs["stats"], g.get("G"),
+              grads["dx"] if args.backward else None)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -479,47 +486,85 @@ def main():
     status = B.moe_read_device_status(bufs["ws"])
 
     # ------------------------------------------------ end to end (host buffers, copies timed)
+    # Every step copies its batch in from pinned host memory and its output and
+    # statistics (and, training, dx) back, all inside the timed region.  The
+    # copies run on their own streams with two sets of device buffers, so step
+    # i + 1's input travels while step i computes and step i's output travels
+    # while step i + 1 computes -- the pipelining a user of the API would do.
     e2e = None
     if not args.no_e2e:
+        NB = 2
+        xs = [g["x"], torch.empty_like(g["x"])]
+        outs = [bufs["out"], torch.empty_like(bufs["out"])]
+        sts = [bufs["stats"], torch.zeros_like(bufs["stats"])]
         x_h = g["x"].cpu().pin_memory()
-        out_h = torch.empty(bufs["out"].shape, dtype=bufs["out"].dtype).pin_memory()
-        st_h = torch.empty(bufs["stats"].shape, dtype=bufs["stats"].dtype).pin_memory()
+        out_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        st_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in sts]
+        Gs = dxs = G_h = dx_h = None
+        if args.backward:
+            Gs = [g["G"], torch.empty_like(g["G"])]
+            dxs = [grads["dx"], torch.empty_like(grads["dx"])]
+            G_h = g["G"].cpu().pin_memory()
+            dx_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dxs]
+        cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(NB)]    # input of the buffer copied in
+        ev_done = [torch.cuda.Event() for _ in range(NB)]  # compute done with the buffer
+        ev_out = [torch.cuda.Event() for _ in range(NB)]   # output of the buffer copied out
 
-        G_h = g["G"].cpu().pin_memory() if args.backward else None
-        dx_h = grads["dx"].cpu().pin_memory() if args.backward else None
+        def issue_input(i, start=None):
+            b = i % NB
+            with torch.cuda.stream(cin):
+                if start is not None:
+                    cin.wait_event(start)
+                cin.wait_event(ev_done[b])   # step i - 2 no longer reads this buffer
+                xs[b].copy_(x_h, non_blocking=True)
+                if args.backward:
+                    Gs[b].copy_(G_h, non_blocking=True)
+                ev_in[b].record(cin)
 
-        def e2e_step():
-            g["x"].copy_(x_h, non_blocking=True)
-            if args.backward:
-                g["G"].copy_(G_h, non_blocking=True)
-            step()
-            out_h.copy_(bufs["out"], non_blocking=True)
-            st_h.copy_(bufs["stats"], non_blocking=True)
-            if args.backward:
-                dx_h.copy_(grads["dx"], non_blocking=True)
+        def run(i):
+            b = i % NB
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])     # step i - 2's output has left this buffer
+            layer(xs[b], outs[b], sts[b], Gs[b] if Gs else None, dxs[b] if dxs else None)
+            ev_done[b].record(stream)
+            with torch.cuda.stream(cout):
+                cout.wait_event(ev_done[b])
+                out_h[b].copy_(outs[b], non_blocking=True)
+                st_h[b].copy_(sts[b], non_blocking=True)
+                if args.backward:
+                    dx_h[b].copy_(dxs[b], non_blocking=True)
+                ev_out[b].record(cout)
 
-        for _ in range(3):
-            e2e_step()
+        def e2e_steps(n, start=None):
+            issue_input(0, start)
+            for i in range(n):
+                if i + 1 < n:
+                    issue_input(i + 1)
+                run(i)
+            stream.wait_event(ev_out[(n - 1) % NB])
+
+        e2e_steps(3)
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_steps(args.steps, start=e0)
         e1.record(stream)
         torch.cuda.synchronize()
         e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
         if dist:
             dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
         h2d = x_h.numel() * x_h.element_size()
-        d2h = out_h.numel() * out_h.element_size() + st_h.numel() * st_h.element_size()
+        d2h = out_h[0].numel() * out_h[0].element_size() + st_h[0].numel() * st_h[0].element_size()
         if args.backward:
             h2d += G_h.numel() * G_h.element_size()
-            d2h += dx_h.numel() * dx_h.element_size()
+            d2h += dx_h[0].numel() * dx_h[0].element_size()
         e2e = {"value": world * wl.T * args.steps / (float(e_ms.item()) / 1000.0), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipelined": "input of step i+1 and output of step i copied while step i computes"}
 
     # ------------------------------------------------ report
     kept = bufs["kept"].cpu().tolist()
