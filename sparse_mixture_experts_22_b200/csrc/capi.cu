@@ -125,7 +125,9 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.nt_max = (int)(((nmax > 0 ? nmax : 1) + 15) / 16 * 16);
     // split-K of the swapped down projection: enough units for ~6.5 waves of 148 SMs
     P.splits = 1;
-    if (P.path == PATH_SWAP) {
+    // split-K partials only for the swapped down projection, which serves groups
+    // of at most 128 tokens (larger ones take the token-major down tiles)
+    if (P.path == PATH_SWAP && P.nt_max <= DOWN_SWAP_MAX_TOKENS) {
         const int64_t units = (int64_t)P.E * (P.d / 128);
         const int kblocks = P.h / 64;
         while (P.splits < 8 && units * P.splits < 960 && kblocks % (P.splits * 2) == 0)
@@ -604,14 +606,20 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     trace_mark(st, tag1);
 
     // down: H [act_rows][hid] x W2p [groups * d][hid] -> y [splits][act_rows][d]
-    const int mode2 = tok ? TC_DOWN_TOK : TC_DOWN_SWAP;
+    // The down projection streams its weights through the wide B operand of the
+    // token-major tiles whenever a group may hold more than 128 tokens: a 256-row
+    // weight tile per stage keeps twice the weight bytes in flight of a swapped
+    // tile next to a token tile that large, and the accumulator stays
+    // double-buffered; the second token tile of a group is partly idle.
+    const bool dtok = tok || nt_max > DOWN_SWAP_MAX_TOKENS;
+    const int mode2 = dtok ? TC_DOWN_TOK : TC_DOWN_SWAP;
     const int bn = (P.d % 256 == 0) ? 256 : 128;
-    MOE_TRY(tmap_bf16(&m_act, H, act_rows, hid, tok ? 128 : 16));
-    MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, tok ? bn : 128));
+    MOE_TRY(tmap_bf16(&m_act, H, act_rows, hid, dtok ? 128 : 16));
+    MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, dtok ? bn : 128));
     a.K = hid;
     a.n_feat = P.d;
     a.w_rows_per_group = P.d;
-    a.splits = tok ? 1 : splits;
+    a.splits = dtok ? 1 : splits;
     a.out = y;
     a.out_ld = P.d;
     a.split_stride = act_rows * (int64_t)P.d;

@@ -28,6 +28,7 @@ constexpr int ROUTE_BLOCK = 128;  // tokens per router / dispatch block
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 8;
 constexpr int SWAP_MAX_TOKENS = 256;  // largest per-expert token count the swap path covers
+constexpr int DOWN_SWAP_MAX_TOKENS = 128;  // above this the down projection takes token-major tiles
 
 struct Plan {
     int64_t T;
