@@ -162,6 +162,8 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     const int64_t kept_max = assign < cap_all ? assign : cap_all;
     P.perm_rows = c.T > 0 ? kept_max + (int64_t)c.E * (P.pad - 1) : 0;
     P.nblk = (int)((c.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    // wide routing over more than one block: TOPK_SUB CTAs per block
+    P.nsub = (c.E > TOPK_WARP_E && c.T > ROUTE_BLOCK) ? TOPK_SUB : 1;
 
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
@@ -170,9 +172,9 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.off_wsplit = take(P.router_kind == ROUTER_TC ? (size_t)3 * c.E * c.d * 2 : 0);
     P.off_z3 = take(P.router_kind == ROUTER_TC ? (size_t)P.router_splits * c.T * P.router_ld * 4
                                                : 0);
-    P.off_ppart = take((size_t)P.nblk * c.E * 4);
-    P.off_hpart = take((size_t)P.nblk * 4);
-    P.off_cnt = take((size_t)P.nblk * c.E * 4);
+    P.off_ppart = take((size_t)P.nblk * P.nsub * c.E * 4);
+    P.off_hpart = take((size_t)P.nblk * P.nsub * 4);
+    P.off_cnt = take((size_t)P.nblk * P.nsub * c.E * 4);
     P.off_tot = take((size_t)c.E * 4);
     P.off_expert = take(P.reroute ? (size_t)c.T * c.k * 4 : 0);
     P.off_rank = take(P.reroute ? (size_t)c.T * c.k * 4 : 0);
@@ -463,6 +465,7 @@ static RouteParams route_params(const Plan& P, void* ws, int32_t* topk_idx, floa
     r.ppart = at<float>(ws, P.off_ppart);
     r.hpart = at<float>(ws, P.off_hpart);
     r.cnt = at<int32_t>(ws, P.off_cnt);
+    r.nsub = P.nsub;
     r.status = at<int32_t>(ws, P.off_status);
     return r;
 }
@@ -486,6 +489,7 @@ static DispatchParams dispatch_params(const Plan& P, const void* x, int32_t* rou
     d.slot_of = slot_of;
     d.x_perm = x_perm;
     d.cap = nullptr;
+    d.nsub = P.nsub;
     return d;
 }
 
@@ -690,7 +694,7 @@ static StatsParams stats_params(const Plan& P, const int32_t* routed, const int3
     StatsParams a;
     a.ppart = at<float>(ws, P.off_ppart);
     a.hpart = at<float>(ws, P.off_hpart);
-    a.nblk = P.nblk;
+    a.nblk = P.nblk * P.nsub;
     a.routed = routed;
     a.kept = kept;
     a.T = P.T;
@@ -1117,7 +1121,7 @@ int moe_route_counts(const moe_config* cfg, const void* ws, size_t ws_bytes, int
             return fail(MOE_ERR_CUDA, "memset failed");
         return ok();
     }
-    MOE_TRY(launched(launch_route_counts(at<int32_t>(ws, P.off_cnt), P.nblk, P.E, counts, st),
+    MOE_TRY(launched(launch_route_counts(at<int32_t>(ws, P.off_cnt), P.nblk * P.nsub, P.E, counts, st),
                      "route_counts"));
     return ok();
 }

@@ -68,10 +68,11 @@ struct RouteParams {
     int E, k;
     int32_t* topk_idx;      // [T][k]
     float* topk_gate;       // [T][k]
-    float* ppart;           // [blocks][E] full-softmax partial sums
-    float* hpart;           // [blocks] entropy partial sums
-    int32_t* cnt;           // [blocks][E] histogram of kept-expert choices
+    float* ppart;           // [blocks * nsub][E] full-softmax partial sums
+    float* hpart;           // [blocks * nsub] entropy partial sums
+    int32_t* cnt;           // [blocks * nsub][E] histogram of kept-expert choices
     int32_t* status;        // device status word (+ combine ticket)
+    int nsub;               // top-k CTAs per block of ROUTE_BLOCK tokens (E > TOPK_WARP_E)
 };
 
 struct DispatchParams {
@@ -89,6 +90,7 @@ struct DispatchParams {
     int32_t* slot_of;
     void* x_perm;
     const int32_t* cap;     // device [E] per-expert capacity (min with C), or null
+    int nsub;               // histogram rows per block of ROUTE_BLOCK tokens (see RouteParams)
 };
 
 int launch_topk(const RouteParams& r, cudaStream_t st);

@@ -25,6 +25,9 @@ enum RouterKind : int {
 };
 
 constexpr int ROUTE_BLOCK = 128;  // tokens per router / dispatch block
+constexpr int TOPK_WARP_E = 32;   // above this many experts one warp routes one token
+constexpr int TOPK_SUB = 4;       // ... and (batches above one block) a block's tokens are
+                                  // routed by TOPK_SUB CTAs, each with its own partials
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 8;
 constexpr int SWAP_MAX_TOKENS = 256;  // largest per-expert token count the swap path covers
@@ -45,6 +48,8 @@ struct Plan {
     int splits;         // split-K partials of the down projection
     int64_t perm_rows;  // rows of x_perm / each y_perm split
     int nblk;           // router blocks of ROUTE_BLOCK tokens
+    int nsub;           // top-k CTAs per router block (1 or TOPK_SUB); the routing partials
+                        // (histograms, P and entropy sums) are per CTA: nblk * nsub of them
     int hsum;           // S * hs (fused shared width)
     int router_kind;    // RouterKind
     int router_npad;    // tensor cores: padded GEMM width of the 3 bf16 parts of W_r

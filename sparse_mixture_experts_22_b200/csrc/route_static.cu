@@ -17,6 +17,8 @@
 // stream capture.  All calls share the array and each call overwrites what
 // the previous one left there; calls that overlap on the GPU (two streams,
 // two threads) race on it and must be serialised by the caller.
+#include <string.h>
+
 #include <mutex>
 
 #include "../../include/moe.h"
@@ -82,9 +84,10 @@ extern "C" MOE_API int moe_route_static(const moe_config* cfg, const void* x, co
     // partials | histograms (sized by the limits above, well inside the array)
     const size_t o_z = 256;
     const size_t o_pp = o_z + up256((size_t)P.T * P.E * 4);
-    const size_t o_hp = o_pp + up256((size_t)P.nblk * P.E * 4);
-    const size_t o_cnt = o_hp + up256((size_t)P.nblk * 4);
-    const size_t total = o_cnt + up256((size_t)P.nblk * P.E * 4);
+    const size_t nrows = (size_t)P.nblk * P.nsub;  // partial rows (top-k CTAs)
+    const size_t o_hp = o_pp + up256(nrows * P.E * 4);
+    const size_t o_cnt = o_hp + up256(nrows * 4);
+    const size_t total = o_cnt + up256(nrows * P.E * 4);
     if (total > kScratchBytes)
         return report_error(MOE_ERR_SHAPE, "moe_route_static: scratch array too small");
     if (P.T == 0) return report_error(MOE_OK, "");
@@ -103,6 +106,7 @@ extern "C" MOE_API int moe_route_static(const moe_config* cfg, const void* x, co
     if (launch_router_rows(x, P.bf16, Wr, z, (int)P.T, P.d, P.E, st) != 0)
         return report_error(MOE_ERR_CUDA, "moe_route_static: router launch failed");
     RouteParams r;
+    memset(&r, 0, sizeof r);
     r.src = z;
     r.bias = cfg->has_bias ? bias : nullptr;
     r.zbuf = z;
@@ -116,6 +120,7 @@ extern "C" MOE_API int moe_route_static(const moe_config* cfg, const void* x, co
     r.hpart = reinterpret_cast<float*>(scratch + o_hp);
     r.cnt = reinterpret_cast<int32_t*>(scratch + o_cnt);
     r.status = reinterpret_cast<int32_t*>(scratch);  // cleared by the top-k kernel
+    r.nsub = P.nsub;
     if (launch_topk(r, st) != 0)
         return report_error(MOE_ERR_CUDA, "moe_route_static: top-k launch failed");
     return report_error(MOE_OK, "");

@@ -45,9 +45,10 @@ struct TopkArgs {
     float* ppart;          // [blocks][E]
     float* hpart;          // [blocks]
     int32_t* status;       // device status word (cleared here: a layer call starts)
+    int nsub;              // CTAs per block of ROUTE_BLOCK tokens (1, or TOPK_SUB for E > TK_WARP_E)
 };
 
-constexpr int TK_WARP_E = 32;      // above this many experts one warp routes one token
+constexpr int TK_WARP_E = TOPK_WARP_E;  // above this many experts one warp routes one token
 constexpr int TK_WIDE_THREADS = 512;  // threads of the standalone top-k kernel in that case
 
 // Shared memory of topk_block for `nthreads` threads: hist [E] int32, then
@@ -86,23 +87,29 @@ __device__ __forceinline__ void topk_insert(float* val, int* id, int k, float v,
     }
 }
 
-// Routes the ROUTE_BLOCK tokens of block `blk` with blockDim.x >= ROUTE_BLOCK
-// threads.  Leaves the per-expert histogram of the block in hist[] (shared)
-// and, for threads below ROUTE_BLOCK, the kept experts of token `tid` in my[]
-// (-1 past k or for padding).  Global outputs are written only when `write`
-// is set.  Up to TK_WARP_E experts one thread routes one token; above that one
-// warp routes one token: each lane keeps the top k of its experts, and k
-// rounds of a warp-wide arg-max over the lanes' heads merge them.
-__device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist, float* zs,
-                           int32_t* my) {
+// Routes part `sub` of `nsub` of the ROUTE_BLOCK tokens of block `blk` with
+// blockDim.x >= ROUTE_BLOCK threads (nsub > 1 only above TK_WARP_E experts:
+// the tokens of a block are then shared by nsub CTAs so that a batch of few
+// blocks still spreads over the SMs).  Leaves the per-expert histogram of its
+// tokens in hist[] (shared) and, with nsub == 1, for threads below
+// ROUTE_BLOCK, the kept experts of token `tid` in my[] (-1 past k or for
+// padding).  Global outputs are written only when `write` is set; the
+// partials go to row blk * nsub + sub.  Up to TK_WARP_E experts one thread
+// routes one token; above that one warp routes one token: each lane keeps the
+// top k of its experts, and k rounds of a warp-wide arg-max over the lanes'
+// heads merge them.
+__device__ void topk_block(const TopkArgs& a, int blk, int sub, int nsub, bool write,
+                           int32_t* hist, float* zs, int32_t* my) {
     __shared__ float ps[ROUTE_BLOCK][TK_CHUNK + 1];
     __shared__ float hs[ROUTE_BLOCK];
     __shared__ int32_t sel[ROUTE_BLOCK][MAX_K];
     const int E = a.E, k = a.k;
     const bool in_smem = E <= TK_SMEM_E;
     const int tid = threadIdx.x, NT = blockDim.x;
-    const int64_t tb = (int64_t)blk * ROUTE_BLOCK;
-    const int nvalid = (int)(a.T - tb < ROUTE_BLOCK ? a.T - tb : ROUTE_BLOCK);
+    const int span = ROUTE_BLOCK / nsub;  // tokens of this CTA
+    const int64_t pidx = (int64_t)blk * nsub + sub;  // its partials' row
+    const int64_t tb = (int64_t)blk * ROUTE_BLOCK + (int64_t)sub * span;
+    const int nvalid = (int)(a.T - tb < span ? (a.T - tb > 0 ? a.T - tb : 0) : span);
     const int64_t t = tb + tid;
     const bool valid = tid < nvalid;
     float* pw = reinterpret_cast<float*>(zs) + (in_smem ? ROUTE_BLOCK * (E + 1) : 0);
@@ -192,7 +199,7 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
             if (write && tid < n) {
                 float acc = 0.f;
                 for (int r = 0; r < ROUTE_BLOCK; ++r) acc += ps[r][tid];
-                a.ppart[(int64_t)blk * E + c0 + tid] = acc;
+                a.ppart[pidx * E + c0 + tid] = acc;
             }
             __syncthreads();
         }
@@ -283,7 +290,7 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
             for (int e = tid; e < E; e += NT) {
                 float acc = 0.f;
                 for (int w = 0; w < nw; ++w) acc += pw[w * E + e];
-                a.ppart[(int64_t)blk * E + e] = acc;
+                a.ppart[pidx * E + e] = acc;
             }
         if (tid < ROUTE_BLOCK) {
 #pragma unroll
@@ -294,7 +301,7 @@ __device__ void topk_block(const TopkArgs& a, int blk, bool write, int32_t* hist
     if (write && tid == 0) {
         float acc = 0.f;
         for (int r = 0; r < ROUTE_BLOCK; ++r) acc += hs[r];
-        a.hpart[blk] = acc;
+        a.hpart[pidx] = acc;
     }
 }
 
@@ -313,6 +320,7 @@ struct DispatchArgs {
     int32_t* slot_of;      // [T][k]
     uint4* x_perm;         // [perm_rows][d]
     const int32_t* cap;    // [E] per-expert capacity (min with C), or null
+    int nsub;              // histogram rows per block (the top-k CTAs of a block)
 };
 
 __device__ __forceinline__ int64_t expert_cap(const DispatchArgs& a, int e) {
@@ -493,7 +501,8 @@ __global__ void __launch_bounds__(TK_WIDE_THREADS)
         a.status[0] = DEV_OK;  // a new layer call starts here
         a.status[1] = 0;       // combine's completion ticket
     }
-    topk_block(a, blockIdx.x, true, hist, zs, my);
+    // CTA b routes part b % nsub of block b / nsub; its histogram is row b
+    topk_block(a, blockIdx.x / a.nsub, blockIdx.x % a.nsub, a.nsub, true, hist, zs, my);
     __syncthreads();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x)
         cnt[(int64_t)blockIdx.x * a.E + e] = hist[e];
@@ -544,7 +553,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     const DispatchSmem d = dispatch_smem(sm, a.E);
     const int blk = blockIdx.x, nblk = gridDim.x;
     for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) {
-        d.base[e] = base_in[(int64_t)blk * a.E + e];
+        d.base[e] = base_in[(int64_t)blk * a.nsub * a.E + e];
         d.tot[e] = tot_in[e];
     }
     const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
@@ -573,7 +582,8 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     extern __shared__ int32_t sm[];
     const DispatchSmem d = dispatch_smem(sm, a.E);
     const int blk = blockIdx.x;
-    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) d.base[e] = base_in[(int64_t)blk * a.E + e];
+    for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK)
+        d.base[e] = base_in[(int64_t)blk * a.nsub * a.E + e];
     const int64_t t = (int64_t)blk * ROUTE_BLOCK + threadIdx.x;
     int32_t my[MAX_K], rank[MAX_K];
 #pragma unroll
@@ -801,7 +811,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
         ta.status[1] = 0;
     }
     int32_t my[MAX_K];
-    topk_block(ta, 0, leader, hist, zs, my);
+    topk_block(ta, 0, 0, 1, leader, hist, zs, my);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += ROUTE_BLOCK) {
         d.base[e] = 0;
@@ -835,6 +845,7 @@ TopkArgs topk_args(const RouteParams& r) {
     a.ppart = r.ppart;
     a.hpart = r.hpart;
     a.status = r.status;
+    a.nsub = r.nsub > 0 ? r.nsub : 1;
     return a;
 }
 
@@ -855,6 +866,7 @@ DispatchArgs dispatch_args(const DispatchParams& p) {
     a.slot_of = p.slot_of;
     a.x_perm = reinterpret_cast<uint4*>(p.x_perm);
     a.cap = p.cap;
+    a.nsub = p.nsub > 0 ? p.nsub : 1;
     return a;
 }
 
@@ -878,7 +890,9 @@ int launch_route_counts(const int32_t* cnt, int nblk, int E, int32_t* counts, cu
 
 int launch_topk(const RouteParams& r, cudaStream_t st) {
     if (r.T == 0) return 0;
-    const unsigned blocks = (unsigned)((r.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    const int nsub = r.nsub > 0 ? r.nsub : 1;
+    if (nsub > 1 && (r.E <= TK_WARP_E || ROUTE_BLOCK % nsub != 0)) return -1;
+    const unsigned blocks = (unsigned)((r.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK) * nsub;
     const int nthreads = r.E > TK_WARP_E ? TK_WIDE_THREADS : ROUTE_BLOCK;
     const size_t smem = topk_smem_bytes(r.E, nthreads);
     if (set_smem(topk_kernel, smem)) return -1;
@@ -891,8 +905,9 @@ int launch_dispatch(const DispatchParams& p, const int32_t* topk_idx, int32_t* c
                     int num_sms, cudaStream_t st) {
     if (p.T == 0) return 0;
     const int nblk = (int)((p.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
+    const int nrows = nblk * (p.nsub > 0 ? p.nsub : 1);  // histogram rows
     const int64_t scan_threads = (int64_t)p.E * 32;
-    dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nblk,
+    dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nrows,
                                                                                 p.E);
     note_launch();
     if (launch_result() != 0) return -1;
@@ -910,8 +925,9 @@ int launch_reroute_dispatch(const DispatchParams& p, const int32_t* topk_idx, in
     if (p.T == 0) return 0;
     const int nblk = (int)((p.T + ROUTE_BLOCK - 1) / ROUTE_BLOCK);
     const DispatchArgs a = dispatch_args(p);
+    const int nrows = nblk * a.nsub;  // histogram rows
     const int64_t scan_threads = (int64_t)p.E * 32;
-    dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nblk,
+    dispatch_scan_kernel<<<(unsigned)((scan_threads + 255) / 256), 256, 0, st>>>(cnt, tot, nrows,
                                                                                 p.E);
     note_launch();
     if (launch_result() != 0) return -1;

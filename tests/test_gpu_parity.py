@@ -43,7 +43,7 @@ SMALL = {
                            cf=(1, 2), dtype="f32", zipf_s=1.0),
     # degenerate: one token; one expert; k = E; heavy skew
     "one_token": Workload("one_token", T=1, d=128, h=128, E=8, k=2),
-    # shared expert on 200 tokens: swapped gate/up tiles of 64 gate + 64 up rows
+    # shared expert on 200 tokens: one swapped gate/up tile of 208 token columns
     "shared_swap64": Workload("shared_swap64", T=200, d=256, h=256, E=8, k=2, n_shared=1,
                               h_shared=256, cf=(1, 1)),
     "one_expert": Workload("one_expert", T=130, d=128, h=256, E=1, k=1),
@@ -61,6 +61,15 @@ SMALL = {
                              zipf_s=0.5, overflow="reroute"),
     "reroute_f32": Workload("reroute_f32", T=90, d=128, h=128, E=4, k=2, cf=(1, 2), dtype="f32",
                             zipf_s=1.0, overflow="reroute"),
+    # one warp per token above 32 experts, four top-k CTAs per 128-token block:
+    # the last block holds 44 tokens (CTAs of 32, 12, 0 and 0 tokens)
+    "wide_sub": Workload("wide_sub", T=300, d=128, h=128, E=64, k=3, cf=(5, 4), zipf_s=0.5),
+    "wide_sub_reroute": Workload("wide_sub_reroute", T=300, d=128, h=128, E=64, k=3, cf=(1, 1),
+                                 zipf_s=1.5, overflow="reroute"),
+    # logits past 256 experts live in global scratch; k at its limit of 8
+    "wide_zbuf": Workload("wide_zbuf", T=400, d=128, h=128, E=512, k=8, cf=(1, 1)),
+    # the largest expert count, one routing block (fused top-k and dispatch)
+    "max_experts": Workload("max_experts", T=64, d=128, h=128, E=1024, k=8),
 }
 
 
