@@ -338,6 +338,38 @@ MOE_API int moe_combine_rows(const moe_config* cfg, const float* y_rows, const i
                              const float* topk_gate, const float* y_shared, void* out,
                              void* stream);
 
+/* Expert parallelism over peer memory: the same step with the two
+ * exchanges folded into the dispatch and the combine.  World ranks, rank q
+ * owning experts q * E_loc .. (q + 1) * E_loc - 1 (E_loc = E / world).
+ *
+ * moe_dispatch_peers is moe_dispatch_capped whose row copies go straight to
+ * the owners: the kept rows of expert e (owner q = e / E_loc) are written,
+ * segment by segment as moe_dispatch_capped lays them out in x_perm, starting
+ * at dst_rows[q] -- rank q's receive buffer at the row where this rank's rows
+ * begin (the rows that lower ranks send to q come first).  dst_rows is a host
+ * array of `world` device pointers (16-byte aligned, [rows][d] of the
+ * activation type), each this GPU's memory or a peer's mapped into this
+ * process (CUDA IPC, symmetric memory); the kernel stores through them over
+ * NVLink.  offsets, slot_of and perm_token keep their local (x_perm)
+ * meaning.  The caller orders the stores before the owners read them (a
+ * stream-ordered barrier across the ranks).
+ *
+ * moe_combine_peers is moe_combine_rows with each output row read from its
+ * owner: y_rows is a host array of `world` device pointers, y_rows[q] = rank
+ * q's fp32 output rows [rows][d] at the row where this rank's rows begin (the
+ * same row as dst_rows[q]); topk_idx and offsets are this rank's, from the
+ * dispatch.  1 <= world <= MOE_MAX_PEERS, E % world == 0; drop policy. */
+#define MOE_MAX_PEERS 64
+MOE_API int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                               const int32_t* cap, int32_t world, void* const* dst_rows,
+                               int32_t* routed, int32_t* kept, int32_t* offsets,
+                               int32_t* perm_token, int32_t* slot_of, void* ws, size_t ws_bytes,
+                               void* stream);
+MOE_API int moe_combine_peers(const moe_config* cfg, int32_t world, const float* const* y_rows,
+                              const int32_t* topk_idx, const int32_t* offsets,
+                              const int32_t* slot_of, const float* topk_gate,
+                              const float* y_shared, void* out, void* stream);
+
 /* ---- routing without a workspace ----------------------------------------- */
 
 /* The pages have no counterpart to this call; it exists for callers that

@@ -29,7 +29,10 @@ EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_split
            "moe_read_device_status", "moe_set_wait_limit_ns", "moe_set_test_stall",
            "moe_trace_begin", "moe_trace_end", "moe_backward_workspace_size", "moe_backward",
            "moe_launch_count", "moe_segment_pad", "moe_route_counts", "moe_dispatch_capped",
-           "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows", "moe_set_pdl"]
+           "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows", "moe_set_pdl",
+           "moe_dispatch_peers", "moe_combine_peers"]
+
+MOE_MAX_PEERS = 64
 
 
 class MoEError(RuntimeError):
@@ -97,6 +100,8 @@ def load() -> ctypes.CDLL:
             "moe_dispatch_capped": [C, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_grouped_workspace_size": [C, ctypes.c_int64, ctypes.c_int32, P],
             "moe_combine_rows": [C, P, P, P, P, P, P],
+            "moe_dispatch_peers": [C, P, P, P, ctypes.c_int32, P, P, P, P, P, P, P, S, P],
+            "moe_combine_peers": [C, ctypes.c_int32, P, P, P, P, P, P, P, P],
             "moe_set_pdl": [I],
             "moe_expert_ffn_grouped": [C, P, ctypes.c_int64, ctypes.c_int32, P, P, P,
                                        ctypes.c_int32, P, P, P, P, S, P],
@@ -298,6 +303,32 @@ def moe_expert_ffn_grouped(cfg, x_rows, rows, group_rows, group_off, group_weigh
 def moe_combine_rows(cfg, y_rows, slot_of, topk_gate, y_shared, out, stream=None):
     _check(load().moe_combine_rows(ctypes.byref(cfg), _p(y_rows), _p(slot_of), _p(topk_gate),
                                    _p(y_shared), _p(out), _stream(stream)))
+
+
+def _ptr_array(ptrs):
+    """A host array of device addresses (ints) for the peer entry points."""
+    return (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(int(p)) for p in ptrs])
+
+
+def moe_dispatch_peers(cfg, topk_idx, x, cap, dst_rows, routed, kept, offsets, perm_token,
+                       slot_of, ws, stream=None):
+    """dst_rows: one device address per rank (ints), each the row of that
+    rank's receive buffer where this rank's rows begin."""
+    arr = _ptr_array(dst_rows)
+    _check(load().moe_dispatch_peers(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(cap),
+                                     len(dst_rows), arr, _p(routed), _p(kept), _p(offsets),
+                                     _p(perm_token), _p(slot_of), _p(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_combine_peers(cfg, y_rows, topk_idx, offsets, slot_of, topk_gate, y_shared, out,
+                      stream=None):
+    """y_rows: one device address per rank (ints), each the row of that
+    rank's fp32 output rows where this rank's rows begin."""
+    arr = _ptr_array(y_rows)
+    _check(load().moe_combine_peers(ctypes.byref(cfg), len(y_rows), arr, _p(topk_idx),
+                                    _p(offsets), _p(slot_of), _p(topk_gate), _p(y_shared),
+                                    _p(out), _stream(stream)))
 
 
 def moe_launch_count() -> int:

@@ -490,6 +490,9 @@ static DispatchParams dispatch_params(const Plan& P, const void* x, int32_t* rou
     d.x_perm = x_perm;
     d.cap = nullptr;
     d.nsub = P.nsub;
+    d.peer_rows = nullptr;  // one destination: x_perm
+    d.npeer = 0;
+    d.e_loc = P.E;
     return d;
 }
 
@@ -1154,6 +1157,81 @@ int moe_dispatch_capped(const moe_config* cfg, const int32_t* topk_idx, const vo
     MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
                                      at<int32_t>(ws, P.off_tot), dv.sms, st),
                      "dispatch"));
+    return ok();
+}
+
+static_assert(MOE_MAX_PEERS == MAX_PEERS, "peer table sizes differ");
+
+static int check_peers(const Plan& P, int32_t world, const void* const* ptrs, const char* what) {
+    if (world < 1 || world > MAX_PEERS) return fail(MOE_ERR_ARG, "world must be 1..MOE_MAX_PEERS");
+    if (P.E % world) return fail(MOE_ERR_SHAPE, "E must be a multiple of world");
+    if (P.reroute) return fail(MOE_ERR_UNSUPPORTED, "expert parallelism: the drop policy only");
+    if (!ptrs) return fail(MOE_ERR_ARG, what);
+    for (int q = 0; q < world; ++q) {
+        if (!ptrs[q]) return fail(MOE_ERR_ARG, what);
+        if (reinterpret_cast<uintptr_t>(ptrs[q]) & 15)
+            return fail(MOE_ERR_ALIGN, "peer row pointers must be 16-byte aligned");
+    }
+    return MOE_OK;
+}
+
+int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                       const int32_t* cap, int32_t world, void* const* dst_rows, int32_t* routed,
+                       int32_t* kept, int32_t* offsets, int32_t* perm_token, int32_t* slot_of,
+                       void* ws, size_t ws_bytes, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (!P.bf16) return fail(MOE_ERR_DTYPE, "moe_dispatch_peers: bf16 only");
+    MOE_TRY(need_ws(ws, ws_bytes, P));
+    MOE_TRY(need(cap, "cap"));
+    MOE_TRY(need(routed, "routed"));
+    MOE_TRY(need(kept, "kept"));
+    MOE_TRY(need(offsets, "offsets"));
+    if (P.T > 0) {
+        MOE_TRY(check_peers(P, world, reinterpret_cast<const void* const*>(dst_rows),
+                            "dst_rows is NULL or holds a NULL pointer"));
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(x, "x"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(maybe(perm_token, "perm_token"));
+    }
+    Device dv;
+    MOE_TRY(device_facts(&dv));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (P.T == 0) return empty_batch(P, ws, routed, kept, offsets, st) == MOE_OK ? ok() : MOE_ERR_CUDA;
+    DispatchParams d = dispatch_params(P, x, routed, kept, offsets, perm_token, slot_of, nullptr);
+    d.cap = cap;
+    d.peer_rows = dst_rows;
+    d.npeer = world;
+    d.e_loc = P.E / world;
+    MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
+                                     at<int32_t>(ws, P.off_tot), dv.sms, st),
+                     "dispatch"));
+    return ok();
+}
+
+int moe_combine_peers(const moe_config* cfg, int32_t world, const float* const* y_rows,
+                      const int32_t* topk_idx, const int32_t* offsets, const int32_t* slot_of,
+                      const float* topk_gate, const float* y_shared, void* out, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (P.T > 0) {
+        MOE_TRY(check_peers(P, world, reinterpret_cast<const void* const*>(y_rows),
+                            "y_rows is NULL or holds a NULL pointer"));
+        MOE_TRY(need(topk_idx, "topk_idx"));
+        MOE_TRY(need(offsets, "offsets"));
+        MOE_TRY(need(slot_of, "slot_of"));
+        MOE_TRY(need(topk_gate, "topk_gate"));
+        MOE_TRY(need(out, "out"));
+        if (P.S > 0) MOE_TRY(need(y_shared, "y_shared"));
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    trace_pre(st, "combine");
+    MOE_TRY(launched(launch_combine_peers(y_rows, world, P.E / world, topk_idx, offsets, slot_of,
+                                          topk_gate, P.S > 0 ? y_shared : nullptr, out, P.bf16,
+                                          P.T, P.d, P.k, st),
+                     "combine"));
+    trace_mark(st, "combine");
     return ok();
 }
 

@@ -169,6 +169,92 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Destinations of the expert-parallel combine: y row bases of the owners.
+struct PeerY {
+    const float* base[MAX_PEERS];
+    int npeer, e_loc;
+};
+
+// The combine with the expert outputs at their owners (expert parallelism):
+// the row of (t, j) is read from the owner of expert topk_idx[t][j], in this
+// GPU's memory or a peer's (NVLink loads), at its position in the segments
+// this rank sent there.  Same arithmetic and order as combine_kernel.
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+    combine_peers_kernel(PeerY py, const int32_t* __restrict__ topk_idx,
+                         const int32_t* __restrict__ offsets,
+                         const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
+                         const float* __restrict__ ys, void* __restrict__ out, int64_t T, int d,
+                         int k) {
+    __shared__ const float* sbase[MAX_PEERS];
+    __shared__ int32_t sfirst[MAX_PEERS];  // first slot of each owner's segments
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < MAX_PEERS; ++i)
+            if (i < py.npeer) sbase[i] = py.base[i];
+    }
+    if (threadIdx.x < py.npeer) sfirst[threadIdx.x] = offsets[threadIdx.x * py.e_loc];
+    __syncthreads();
+    const int vecs = d / 8;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * vecs) return;
+    const int64_t t = i / vecs;
+    const int c = (int)(i % vecs) * 8;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    // every kept row is requested before any is used
+    float4 ra[MAX_K], rb[MAX_K];
+    float g[MAX_K];
+    bool kept[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        ra[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        rb[j] = ra[j];
+        g[j] = 0.f;
+        const int32_t slot = j < k ? slot_of[t * k + j] : -1;
+        kept[j] = slot >= 0;
+        if (kept[j]) {
+            const int o = topk_idx[t * k + j] / py.e_loc;
+            const float* p = sbase[o] + (int64_t)(slot - sfirst[o]) * d + c;
+            ra[j] = *reinterpret_cast<const float4*>(p);
+            rb[j] = *reinterpret_cast<const float4*>(p + 4);
+            g[j] = gate[t * k + j];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+        if (!kept[j]) continue;
+        acc[0] = fmaf(g[j], ra[j].x, acc[0]);
+        acc[1] = fmaf(g[j], ra[j].y, acc[1]);
+        acc[2] = fmaf(g[j], ra[j].z, acc[2]);
+        acc[3] = fmaf(g[j], ra[j].w, acc[3]);
+        acc[4] = fmaf(g[j], rb[j].x, acc[4]);
+        acc[5] = fmaf(g[j], rb[j].y, acc[5]);
+        acc[6] = fmaf(g[j], rb[j].z, acc[6]);
+        acc[7] = fmaf(g[j], rb[j].w, acc[7]);
+    }
+    if (ys) {
+        const float* p = ys + t * d + c;
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    if (OUT_BF16) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + t * d + c) = o;
+    } else {
+        float* p = reinterpret_cast<float*>(out) + t * d + c;
+        *reinterpret_cast<float4*>(p) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
 __global__ void stats_finalize_kernel(const double* __restrict__ sums, int E, int k,
                                       moe_stats* __restrict__ st) {
     if (threadIdx.x == 0) finalize_stats(sums, E, k, st);
@@ -220,6 +306,28 @@ int launch_combine(const float* y, int splits, int64_t split_stride, const int32
     else
         launch_ex(pdl_active(), combine_kernel<false>, dim3(blocks), dim3(256), 0, st, y, splits,
                   split_stride, slot_of, gate, y_shared, out, T, d, k, s);
+    note_launch();
+    return launch_result();
+}
+
+int launch_combine_peers(const float* const* y_rows, int npeer, int e_loc,
+                         const int32_t* topk_idx, const int32_t* offsets,
+                         const int32_t* slot_of, const float* gate, const float* y_shared,
+                         void* out, bool out_bf16, int64_t T, int d, int k, cudaStream_t st) {
+    if (T == 0) return 0;
+    if (npeer < 1 || npeer > MAX_PEERS || e_loc < 1) return -1;
+    PeerY py;
+    for (int i = 0; i < MAX_PEERS; ++i) py.base[i] = i < npeer ? y_rows[i] : nullptr;
+    py.npeer = npeer;
+    py.e_loc = e_loc;
+    const int64_t n = T * (d / 8);
+    const unsigned blocks = (unsigned)((n + 255) / 256);
+    if (out_bf16)
+        combine_peers_kernel<true><<<blocks, 256, 0, st>>>(py, topk_idx, offsets, slot_of, gate,
+                                                          y_shared, out, T, d, k);
+    else
+        combine_peers_kernel<false><<<blocks, 256, 0, st>>>(py, topk_idx, offsets, slot_of, gate,
+                                                           y_shared, out, T, d, k);
     note_launch();
     return launch_result();
 }

@@ -91,6 +91,11 @@ struct DispatchParams {
     void* x_perm;
     const int32_t* cap;     // device [E] per-expert capacity (min with C), or null
     int nsub;               // histogram rows per block of ROUTE_BLOCK tokens (see RouteParams)
+    // Destinations of the row copies.  npeer == 0: x_perm, row = slot.  Else
+    // expert e's rows go to rank o = e / e_loc: row (slot - offsets[o * e_loc])
+    // of peer_rows[o] (a host array of npeer device pointers, read at launch).
+    void* const* peer_rows;
+    int npeer, e_loc;
 };
 
 int launch_topk(const RouteParams& r, cudaStream_t st);
@@ -179,6 +184,14 @@ struct StatsParams {
 
 // out[t] = sum_j gate * sum_s y[s][slot] + y_shared[t]; with sp, one more block
 // computes the statistics in the same launch
+// out[t] = sum over kept j of gate * y row of (t, j) (+ y_shared[t]), the y
+// row found at the expert's owner: expert e = topk_idx[t][j] belongs to rank
+// o = e / e_loc, and its row is slot - offsets[o * e_loc] of y_rows[o] (a host
+// array of npeer device pointers, read at launch).
+int launch_combine_peers(const float* const* y_rows, int npeer, int e_loc,
+                         const int32_t* topk_idx, const int32_t* offsets,
+                         const int32_t* slot_of, const float* gate, const float* y_shared,
+                         void* out, bool out_bf16, int64_t T, int d, int k, cudaStream_t st);
 int launch_combine(const float* y, int splits, int64_t split_stride, const int32_t* slot_of,
                    const float* gate, const float* y_shared, void* out, bool out_bf16,
                    int64_t T, int d, int k, const StatsParams* sp, cudaStream_t st);

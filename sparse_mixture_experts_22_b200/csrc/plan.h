@@ -30,6 +30,7 @@ constexpr int TOPK_SUB = 4;       // ... and (batches above one block) a block's
                                   // routed by TOPK_SUB CTAs, each with its own partials
 constexpr int MAX_E = 1024;
 constexpr int MAX_K = 8;
+constexpr int MAX_PEERS = 64;     // expert-parallel ranks one dispatch or combine addresses
 constexpr int SWAP_MAX_TOKENS = 256;  // largest per-expert token count the swap path covers
 constexpr int DOWN_SWAP_MAX_TOKENS = 128;  // above this the down projection takes token-major tiles
 

@@ -198,7 +198,8 @@ __device__ void topk_block(const TopkArgs& a, int blk, int sub, int nsub, bool w
             __syncthreads();
             if (write && tid < n) {
                 float acc = 0.f;
-                for (int r = 0; r < ROUTE_BLOCK; ++r) acc += ps[r][tid];
+                // rows past the block's tokens hold +0, which adds nothing
+                for (int r = 0; r < nvalid; ++r) acc += ps[r][tid];
                 a.ppart[pidx * E + c0 + tid] = acc;
             }
             __syncthreads();
@@ -300,7 +301,7 @@ __device__ void topk_block(const TopkArgs& a, int blk, int sub, int nsub, bool w
     __syncthreads();
     if (write && tid == 0) {
         float acc = 0.f;
-        for (int r = 0; r < ROUTE_BLOCK; ++r) acc += hs[r];
+        for (int r = 0; r < nvalid; ++r) acc += hs[r];
         a.hpart[pidx] = acc;
     }
 }
@@ -321,6 +322,8 @@ struct DispatchArgs {
     uint4* x_perm;         // [perm_rows][d]
     const int32_t* cap;    // [E] per-expert capacity (min with C), or null
     int nsub;              // histogram rows per block (the top-k CTAs of a block)
+    int npeer, e_loc;      // row destinations: expert e -> peer[e / e_loc] (see place_rows)
+    uint4* peer[MAX_PEERS];
 };
 
 __device__ __forceinline__ int64_t expert_cap(const DispatchArgs& a, int e) {
@@ -330,9 +333,12 @@ __device__ __forceinline__ int64_t expert_cap(const DispatchArgs& a, int e) {
 }
 
 // Shared memory of the dispatch kernels: base [E], tot [E], rows [E],
-// off [E+1], wcnt [DWARPS][E], slots [ROUTE_BLOCK * k].
+// off [E+1], wcnt [DWARPS][E], slots [ROUTE_BLOCK * k], owner [ROUTE_BLOCK * k],
+// then (8-byte aligned) the destination table [MAX_PEERS].
 __host__ __device__ inline size_t dispatch_smem_bytes(int E, int k) {
-    return sizeof(int32_t) * ((size_t)4 * E + 1 + (size_t)DWARPS * E + (size_t)ROUTE_BLOCK * k);
+    return sizeof(int32_t) *
+               ((size_t)4 * E + 1 + (size_t)DWARPS * E + (size_t)2 * ROUTE_BLOCK * k) +
+           8 + sizeof(uint4*) * MAX_PEERS;
 }
 
 struct DispatchSmem {
@@ -341,10 +347,12 @@ struct DispatchSmem {
     int32_t* rows;   // rows e serves (kept)
     int32_t* off;    // padded segment starts [E+1]
     int32_t* wcnt;   // per-warp counts [DWARPS][E]
-    int32_t* slots;  // [ROUTE_BLOCK * k]
+    int32_t* slots;  // [ROUTE_BLOCK * k] destination row of each (token, j), -1: dropped
+    int32_t* owner;  // [ROUTE_BLOCK * k] destination of each (token, j)
+    uint4** peer;    // [MAX_PEERS] destination bases
 };
 
-__device__ __forceinline__ DispatchSmem dispatch_smem(int32_t* sm, int E) {
+__device__ __forceinline__ DispatchSmem dispatch_smem(int32_t* sm, int E, int k) {
     DispatchSmem d;
     d.base = sm;
     d.tot = d.base + E;
@@ -352,6 +360,9 @@ __device__ __forceinline__ DispatchSmem dispatch_smem(int32_t* sm, int E) {
     d.off = d.rows + E;
     d.wcnt = d.off + E + 1;
     d.slots = d.wcnt + DWARPS * E;
+    d.owner = d.slots + ROUTE_BLOCK * k;
+    const uintptr_t p = reinterpret_cast<uintptr_t>(d.owner + ROUTE_BLOCK * k);
+    d.peer = reinterpret_cast<uint4**>((p + 7) & ~static_cast<uintptr_t>(7));
     return d;
 }
 
@@ -409,7 +420,10 @@ __device__ void block_ranks(int E, const int32_t* base, int32_t* wcnt, const int
 // served by expert[j] at position rank[j] of its queue, kept if rank < C.
 // d.off and d.rows must be filled.  When `writer`, writes slot_of and
 // perm_token (with -1 in padding rows and the unused tail).  `split`/`nsplit`:
-// this CTA copies every nsplit-th row.
+// this CTA copies every nsplit-th row.  The row of slot s of expert e goes to
+// destination o = e / e_loc at row s - off[o * e_loc]: with one destination
+// (e_loc = E) that is x_perm at row s; with expert parallelism, the receive
+// buffer of e's owner, in this GPU's memory or a peer's (NVLink stores).
 __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer, int split,
                            int nsplit, const DispatchSmem& d, const int32_t* expert,
                            const int32_t* rank) {
@@ -423,12 +437,19 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
              r += (int64_t)nblk * ROUTE_BLOCK)
             a.perm_token[r] = -1;
     }
+    if (tid == 0) {
+        // the destination table, indexed statically so it stays in the
+        // parameter space
+#pragma unroll
+        for (int i = 0; i < MAX_PEERS; ++i)
+            if (i < a.npeer) d.peer[i] = a.peer[i];
+    }
     const int64_t t = (int64_t)blk * ROUTE_BLOCK + tid;
     const bool valid = t < a.T;
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
         if (j >= k) break;
-        int32_t slot = -1;
+        int32_t slot = -1, row = -1, own = 0;
         if (valid) {
             if (rank[j] >= 0 && (int64_t)rank[j] < expert_cap(a, expert[j]))
                 slot = d.off[expert[j]] + rank[j];
@@ -436,8 +457,13 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
                 a.slot_of[t * k + j] = slot;
                 if (slot >= 0 && a.perm_token) a.perm_token[slot] = (int32_t)t;
             }
+            if (slot >= 0) {
+                own = expert[j] / a.e_loc;
+                row = slot - d.off[own * a.e_loc];
+            }
         }
-        d.slots[tid * k + j] = slot;
+        d.slots[tid * k + j] = row;
+        d.owner[tid * k + j] = own;
     }
     __syncthreads();
 
@@ -452,10 +478,10 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
 #pragma unroll
         for (int q = 0; q < G; ++q) {
             const int r = r0 + q * nsplit;
-            const int32_t slot = r < nrow ? d.slots[r] : -1;
+            const int32_t row = r < nrow ? d.slots[r] : -1;
             const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
-            src[q] = slot >= 0 ? a.x + tok * nv : nullptr;
-            dst[q] = slot >= 0 ? a.x_perm + (int64_t)slot * nv : nullptr;
+            src[q] = row >= 0 ? a.x + tok * nv : nullptr;
+            dst[q] = row >= 0 ? d.peer[d.owner[r]] + (int64_t)row * nv : nullptr;
         }
         for (int c = tid; c < nv; c += ROUTE_BLOCK) {
             uint4 v[G];
@@ -550,7 +576,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     dispatch_kernel(DispatchArgs a, const int32_t* __restrict__ topk_idx,
                     const int32_t* __restrict__ base_in, const int32_t* __restrict__ tot_in) {
     extern __shared__ int32_t sm[];
-    const DispatchSmem d = dispatch_smem(sm, a.E);
+    const DispatchSmem d = dispatch_smem(sm, a.E, a.k);
     const int blk = blockIdx.x, nblk = gridDim.x;
     for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) {
         d.base[e] = base_in[(int64_t)blk * a.nsub * a.E + e];
@@ -580,7 +606,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
                 const int32_t* __restrict__ base_in, int32_t* __restrict__ expert_of,
                 int32_t* __restrict__ rank_of) {
     extern __shared__ int32_t sm[];
-    const DispatchSmem d = dispatch_smem(sm, a.E);
+    const DispatchSmem d = dispatch_smem(sm, a.E, a.k);
     const int blk = blockIdx.x;
     for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK)
         d.base[e] = base_in[(int64_t)blk * a.nsub * a.E + e];
@@ -775,7 +801,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     place_kernel(DispatchArgs a, const int32_t* __restrict__ expert_of,
                  const int32_t* __restrict__ rank_of) {
     extern __shared__ int32_t sm[];
-    const DispatchSmem d = dispatch_smem(sm, a.E);
+    const DispatchSmem d = dispatch_smem(sm, a.E, a.k);
     const int blk = blockIdx.x, nblk = gridDim.x;
     for (int e = threadIdx.x; e < a.E; e += ROUTE_BLOCK) d.rows[e] = a.kept[e];
     for (int e = threadIdx.x; e <= a.E; e += ROUTE_BLOCK) d.off[e] = a.offsets[e];
@@ -804,7 +830,7 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     float* zs = reinterpret_cast<float*>(dyn + E);
     int32_t* dsm =
         reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(dyn) + topk_smem_bytes(E, ROUTE_BLOCK));
-    const DispatchSmem d = dispatch_smem(dsm, E);
+    const DispatchSmem d = dispatch_smem(dsm, E, da.k);
     const bool leader = blockIdx.x == 0;
     if (leader && threadIdx.x == 0 && ta.status) {
         ta.status[0] = DEV_OK;
@@ -867,6 +893,16 @@ DispatchArgs dispatch_args(const DispatchParams& p) {
     a.x_perm = reinterpret_cast<uint4*>(p.x_perm);
     a.cap = p.cap;
     a.nsub = p.nsub > 0 ? p.nsub : 1;
+    for (int i = 0; i < MAX_PEERS; ++i) a.peer[i] = nullptr;
+    if (p.npeer > 0) {
+        a.npeer = p.npeer;
+        a.e_loc = p.e_loc;
+        for (int i = 0; i < p.npeer; ++i) a.peer[i] = reinterpret_cast<uint4*>(p.peer_rows[i]);
+    } else {
+        a.npeer = 1;
+        a.e_loc = p.E;
+        a.peer[0] = a.x_perm;
+    }
     return a;
 }
 

@@ -31,6 +31,18 @@ The exchanges are torch.distributed collectives (NCCL between GPUs, gloo on
 the host in the tests) or, for one process standing in for G ranks on one
 GPU, plain copies (`forward_emulated`).  Only the routed experts are
 partitioned; the overflow policy is drop.
+
+The peer-memory form folds steps 3 and 5 into the kernels next to them:
+moe_dispatch_peers stores every kept row straight into its owner's receive
+buffer (NVLink stores from the SMs that gather it), and moe_combine_peers
+loads every output row straight from its owner's buffer; no staging copy and
+no collective carries the rows.  Rank s's rows start at row
+`peer_row_starts(plan, s)[q]` of rank q's buffers, after the rows of the lower
+ranks -- the layout the all-to-all produces.  Between the phases the ranks
+pass a stream-ordered barrier (the owners read only after every source has
+stored; the buffers are reused only after every source has combined):
+`forward_dist_peers` takes the buffers from torch's symmetric memory, and
+`forward_emulated_peers` runs the ranks' kernels one after another on one GPU.
 """
 
 from dataclasses import dataclass, field
@@ -141,6 +153,12 @@ def exchange_back(y: torch.Tensor, plan: Plan, rank: int, group=None) -> torch.T
     return back
 
 
+def peer_row_starts(plan: Plan, rank: int) -> np.ndarray:
+    """[G] first row of rank `rank`'s rows in each rank's receive (and
+    output) buffer: the rows every lower rank sends there come first."""
+    return plan.send[:rank].sum(axis=0).astype(np.int64)
+
+
 def all_gather_counts(counts: torch.Tensor, world: int, group=None) -> np.ndarray:
     """Step 1's exchange: every rank's per-expert counts, [G][E]."""
     import torch.distributed as dist
@@ -202,10 +220,11 @@ class Rank:
                               b["offsets"], b["perm_token"], b["slot_of"], b["x_perm"], b["ws"])
         return b["x_perm"][:int(plan.seg[self.rank].sum())]
 
-    def ffn(self, plan: Plan, recv: torch.Tensor) -> torch.Tensor:
+    def ffn(self, plan: Plan, recv: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
         rows, off, wi = plan.groups(self.rank)
         dev = self.x.device
-        y = torch.empty((recv.shape[0], self.wl.d), dtype=torch.float32, device=dev)
+        if y is None:
+            y = torch.empty((recv.shape[0], self.wl.d), dtype=torch.float32, device=dev)
         if recv.shape[0] == 0:
             return y
         mx = int(rows.max()) if rows.size else 0
@@ -216,6 +235,28 @@ class Rank:
                                  self.W13, self.W2p, y, ws)
         self.ffn_ws = ws
         return y
+
+    def dispatch_peers(self, plan: Plan, recv_bases: List[int]) -> None:
+        """Step 2 with step 3 folded in: recv_bases[q] = device address of
+        rank q's receive buffer (bf16 [rows][d])."""
+        b = self.b
+        cap = torch.tensor(plan.cap[self.rank].clip(max=2 ** 31 - 1), dtype=torch.int32,
+                           device=self.x.device)
+        row_bytes = self.wl.d * self.x.element_size()
+        starts = peer_row_starts(plan, self.rank)
+        dst = [int(recv_bases[q]) + int(starts[q]) * row_bytes for q in range(self.world)]
+        B.moe_dispatch_peers(self.cfg, b["topk_idx"], self.x, cap, dst, b["routed"], b["kept"],
+                             b["offsets"], b["perm_token"], b["slot_of"], b["ws"])
+
+    def combine_peers(self, plan: Plan, y_bases: List[int]) -> torch.Tensor:
+        """Steps 5 and 6: y_bases[q] = device address of rank q's fp32 output
+        rows [rows][d]."""
+        b = self.b
+        starts = peer_row_starts(plan, self.rank)
+        src = [int(y_bases[q]) + int(starts[q]) * self.wl.d * 4 for q in range(self.world)]
+        B.moe_combine_peers(self.cfg, src, b["topk_idx"], b["offsets"], b["slot_of"],
+                            b["topk_gate"], None, b["out"])
+        return b["out"]
 
     def combine(self, y_back: torch.Tensor) -> torch.Tensor:
         b = self.b
@@ -267,3 +308,62 @@ def forward_emulated(ranks: List[Rank], T_all: int):
     stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
     B.moe_stats_finalize(ranks[0].cfg, sums, stats)
     return outs, stats, plan
+
+
+def forward_emulated_peers(ranks: List[Rank], T_all: int):
+    """The peer-memory form with G ranks in one process on one device: every
+    rank's receive and output buffers live on that device, and the ranks'
+    kernels run one after another in stream order (which stands in for the
+    barriers).  Returns ([out per rank], stats tensor, plan)."""
+    G = len(ranks)
+    counts = np.stack([r.route().cpu().numpy() for r in ranks]).astype(np.int64)
+    wl = ranks[0].wl
+    plan = make_plan(counts, T_all, wl.k, wl.E, wl.cf, ranks[0].pad)
+    dev = ranks[0].x.device
+    recv = [torch.empty((max(int(plan.recv_rows(q).sum()), 1), wl.d), dtype=ranks[0].x.dtype,
+                        device=dev) for q in range(G)]
+    for r in ranks:
+        r.dispatch_peers(plan, [t.data_ptr() for t in recv])
+    ys = [ranks[q].ffn(plan, recv[q][:int(plan.recv_rows(q).sum())]) for q in range(G)]
+    ys = [y if y.shape[0] else torch.empty((1, wl.d), dtype=torch.float32, device=dev)
+          for y in ys]
+    outs = [r.combine_peers(plan, [y.data_ptr() for y in ys]) for r in ranks]
+    sums = sum(r.stats_sums().clone() for r in ranks)
+    stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
+    B.moe_stats_finalize(ranks[0].cfg, sums, stats)
+    return outs, stats, plan
+
+
+def forward_dist_peers(r: Rank, T_all: int, group=None, max_rows: Optional[int] = None):
+    """One step on this rank (one process per GPU) in the peer-memory form.
+    The receive and output buffers are symmetric memory (every rank maps
+    every other rank's), sized for `max_rows` received rows (default: every
+    token of every rank routed here, T_all * k); the barriers are symmetric
+    memory's stream-ordered barrier.  Returns (out, stats tensor, plan)."""
+    import torch.distributed as dist
+    import torch.distributed._symmetric_memory as symm_mem
+    wl = r.wl
+    counts = all_gather_counts(r.route(), r.world, group)
+    plan = make_plan(counts, T_all, wl.k, wl.E, wl.cf, r.pad)
+    rows = max_rows if max_rows is not None else T_all * wl.k + wl.E * r.pad
+    if int(plan.recv_rows(r.rank).sum()) > rows:
+        raise ValueError("the receive buffers are smaller than this step's rows")
+    if not hasattr(r, "_symm"):
+        grp = group if group is not None else dist.group.WORLD
+        recv = symm_mem.empty(rows, wl.d, dtype=r.x.dtype, device=r.x.device)
+        yb = symm_mem.empty(rows, wl.d, dtype=torch.float32, device=r.x.device)
+        r._symm = (recv, yb, symm_mem.rendezvous(recv, grp), symm_mem.rendezvous(yb, grp))
+    recv, yb, h_recv, h_y = r._symm
+    r.dispatch_peers(plan, list(h_recv.buffer_ptrs))
+    h_recv.barrier(channel=0)            # every source has stored its rows here
+    n = int(plan.recv_rows(r.rank).sum())
+    if n:
+        r.ffn(plan, recv[:n], yb[:n])
+    h_y.barrier(channel=0)               # every owner's outputs are in place
+    out = r.combine_peers(plan, list(h_y.buffer_ptrs))
+    h_y.barrier(channel=1)               # every source has read: buffers free for the next step
+    sums = r.stats_sums()
+    dist.all_reduce(sums, group=group)
+    stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
+    B.moe_stats_finalize(r.cfg, sums, stats)
+    return out, stats, plan

@@ -115,3 +115,39 @@ def test_training_workspaces():
     with pytest.raises(B.MoEError) as e:
         M.moe_backward_workspace_size(M.make_config(8, 128, 128, 4, 2))
     assert e.value.code == 1
+
+
+def _peer_call_codes(cfg, world, ptrs):
+    """Return codes of the two peer entry points for fake (never dereferenced)
+    addresses; every case here fails in the host-side checks."""
+    lib = B.load()
+    fake = ctypes.c_void_p(0x100000)
+    ws_bytes = M.moe_workspace_size(cfg)
+    arr = (ctypes.c_void_p * max(len(ptrs), 1))(*[ctypes.c_void_p(p) if p else None
+                                                  for p in ptrs])
+    d = lib.moe_dispatch_peers(ctypes.byref(cfg), fake, fake, fake, world, arr, fake, fake, fake,
+                               None, fake, fake, ws_bytes, None)
+    c = lib.moe_combine_peers(ctypes.byref(cfg), world, arr, fake, fake, fake, fake, None, fake,
+                              None)
+    return d, c
+
+
+@pytest.mark.parametrize("kw,world,ptrs,code", [
+    (dict(), 0, [], 1),                                  # no ranks
+    (dict(), 65, [0x200000] * 65, 1),                    # above MOE_MAX_PEERS
+    (dict(), 3, [0x200000] * 3, 2),                      # 8 experts over 3 ranks
+    (dict(), 2, [0x200000, 0x200008], 4),                # a row pointer off 16 bytes
+    (dict(), 2, [0x200000, 0], 1),                       # a NULL row pointer
+    (dict(overflow="reroute", cf=(1, 1)), 2, [0x200000] * 2, 8),  # drop policy only
+])
+def test_peer_calls_check_their_arguments(kw, world, ptrs, code):
+    cfg = M.make_config(64, 128, 128, 8, 2, **kw)
+    d, c = _peer_call_codes(cfg, world, ptrs)
+    assert d == code, B.load().moe_last_error()
+    assert c == code, B.load().moe_last_error()
+
+
+def test_peer_dispatch_is_bf16_only():
+    cfg = M.make_config(64, 128, 128, 8, 2, dtype="f32")
+    d, _ = _peer_call_codes(cfg, 2, [0x200000] * 2)
+    assert d == 3

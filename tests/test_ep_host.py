@@ -61,6 +61,33 @@ def test_plan_layout():
     assert plan.recv_rows(1).sum() == 48
 
 
+def test_peer_rows_land_where_the_exchange_puts_them():
+    """Every source's segments, placed at peer_row_starts in each owner's
+    buffer, rebuild exactly what the all-to-all concatenation (sources in
+    order, each source's split for the owner) receives."""
+    counts = np.array([[5, 0, 9, 3, 1, 7], [4, 7, 0, 1, 2, 2], [0, 3, 3, 8, 6, 1]])
+    G, E = counts.shape
+    plan = ep.make_plan(counts, 30, 2, E, (1, 1), pad=16)
+    sends = [_send_buffer(plan, r).numpy() for r in range(G)]
+    for q in range(G):
+        # the all-to-all: source s's split for q, sources in order
+        own = np.concatenate([np.zeros((G, 1)), np.cumsum(plan.send, axis=1)], axis=1).astype(int)
+        a2a = np.concatenate([sends[s][own[s, q]:own[s, q + 1]] for s in range(G)])
+        # the peer stores: source s writes its segment of expert e (owner q)
+        # at peer_row_starts(s)[q] + (its x_perm slot - its first slot for q)
+        buf = np.full((int(plan.recv_rows(q).sum()), 4), -7.0, np.float32)
+        for s in range(G):
+            seg_start = np.concatenate([[0], np.cumsum(plan.seg[s])]).astype(int)
+            first = seg_start[q * plan.E_loc]
+            for e in range(q * plan.E_loc, (q + 1) * plan.E_loc):
+                rows = sends[s][seg_start[e]:seg_start[e] + plan.kept[s, e]]
+                at = ep.peer_row_starts(plan, s)[q] + seg_start[e] - first
+                buf[at:at + len(rows)] = rows
+        kept_rows = a2a[:, 3] == 1
+        assert len(buf) == len(a2a)
+        np.testing.assert_array_equal(buf[kept_rows], a2a[kept_rows])
+
+
 # ---------------------------------------------------------------- gloo exchange
 
 WORLD = 2
@@ -133,3 +160,7 @@ def test_exchanges_over_gloo_ranks():
                 g += 1
         # the returned rows land where the sent rows were
         np.testing.assert_array_equal(back, send * 2.0)
+        # the peer-memory dispatch writes source src's rows where the
+        # all-to-all put them: its first group starts at peer_row_starts
+        for src in range(WORLD):
+            assert ep.peer_row_starts(plan, src)[rank] == off[src * plan.E_loc]

@@ -4,7 +4,10 @@ ever waits on another), against the fp64 oracle on the concatenated batch.
 
 The G ranks must reproduce the single-GPU layer on the concatenation of their
 batches: the routing sets, the rows every expert keeps under the global
-capacity (bit-exact), the output (the layer's bars) and the statistics."""
+capacity (bit-exact), the output (the layer's bars) and the statistics.  The
+peer-memory form (rows stored into, and read from, the owners' buffers by the
+dispatch and combine kernels) must give the exchange form's output bit for
+bit."""
 
 import numpy as np
 import pytest
@@ -72,6 +75,38 @@ def test_emulated_ranks_match_the_layer_on_the_concatenated_batch(name):
         assert ref["kept"].sum() < wl.T * wl.k, "the case should drop some assignments"
     check_output(out, ref["out"], name)
     check_stats(ref, stats, wl.T)
+
+
+def run_emulated_peers(wl, G, inp):
+    dev = torch.device("cuda")
+    cfg = M.config_of(wl)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    W13, W2p = M.pack_weights(cfg, g["w1"], g["w3"], g["w2"])
+    T_loc, E_loc = wl.T // G, wl.E // G
+    ranks = [ep.Rank(wl, r, G, g["x"][r * T_loc:(r + 1) * T_loc].contiguous(), g["Wr"],
+                     g["bias"], W13[r * E_loc:(r + 1) * E_loc], W2p[r * E_loc:(r + 1) * E_loc])
+             for r in range(G)]
+    outs, stats, plan = ep.forward_emulated_peers(ranks, wl.T)
+    torch.cuda.synchronize()
+    return ranks, torch.cat([o.clone() for o in outs]), stats, plan
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_peer_stores_and_loads_give_the_exchange_path_bit_for_bit(name):
+    """The dispatch that stores rows into the owners' buffers and the combine
+    that loads them from there reproduce the all-to-all path exactly, and so
+    the oracle."""
+    wl, G = CASES[name]
+    inp = host_inputs(wl)
+    _, out_x, stats_x, plan_x = run_emulated(wl, G, inp)
+    ranks, out_p, stats_p, plan_p = run_emulated_peers(wl, G, inp)
+    for r in ranks:
+        assert M.moe_read_device_status(r.b["ws"]) == 0
+    np.testing.assert_array_equal(plan_p.kept, plan_x.kept)
+    assert torch.equal(out_p, out_x)
+    assert torch.equal(stats_p, stats_x)
+    ref = O.forward(O.cfg_of(wl), inp)
+    check_output(out_p, ref["out"], name)
 
 
 def test_grouped_ffn_flags_an_oversized_group():
