@@ -45,6 +45,15 @@ constexpr int BM = 128;      // MMA M (TMEM lanes)
 constexpr int BK = 64;       // K elements per stage: one 128-byte swizzle row of bf16
 constexpr int UK = 16;       // K per tcgen05.mma (bf16)
 constexpr int THREADS = 192;
+
+// Threads of a CTA: the producer warp, the MMA warp and four epilogue warps
+// (one per TMEM lane quarter); the swapped gate/up has eight, two per
+// quarter, splitting the token columns: its accumulator is single-buffered
+// for wide token tiles, so the epilogue's length is time the MMAs wait.
+template <int MODE>
+constexpr int threads_of() {
+    return MODE == TC_GATEUP_SWAP ? THREADS + 128 : THREADS;
+}
 constexpr uint64_t TEARDOWN_NS = 200000000ull;  // 0.2 s bound on draining in-flight work
 
 struct SharedLayout {
@@ -222,7 +231,7 @@ __device__ __forceinline__ void store_rows_f32x32(float* stg, const float* v, in
 }
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads_of<MODE>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
     constexpr bool TOK = (MODE == TC_GATEUP_TOK || MODE == TC_DOWN_TOK ||
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 128);
+            mbar_init(&acc_empty[i], threads_of<MODE>() - 64);  // the epilogue threads
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -463,6 +472,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;       // which of the quarter's warps (swapped gate/up)
+        constexpr int NHALF = (threads_of<MODE>() - 64) / 128;
         const int row = q * 32 + lane;          // accumulator row (TMEM lane)
         const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
         int acc = 0;
@@ -623,7 +634,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
                                      (int64_t)x.row0 * args.out_ld + x.nb * 128 + row;
 #pragma unroll 1
-                for (int c = 0; c < x.ntok; c += 16) {
+                for (int c = 16 * half; c < x.ntok; c += 16 * NHALF) {
                     float g[16], v[16];
                     tmem_ld16(t0 + c, g);
                     tmem_ld16(t0 + args.nt_max + c, v);
@@ -685,7 +696,7 @@ int launch_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, i
             return -1;
         configured_bytes = L.total;
     }
-    launch_ex(pdl_active(), kern, dim3(grid), dim3(THREADS), L.total, st, act, w, a);
+    launch_ex(pdl_active(), kern, dim3(grid), dim3(threads_of<MODE>()), L.total, st, act, w, a);
     note_launch();
     return launch_result();
 }
