@@ -329,29 +329,48 @@ def run_reference(args):
     import numpy as np
     import oracle as O
     cfg = O.cfg_of(wl)
-    # each step: the whole batch routed, and the outputs of a bounded row sample
+    # each step: the whole batch routed, and the outputs of a bounded row sample;
+    # the sample is sized so that the whole run (warm-up and timed steps) takes
+    # about REF_BUDGET_S: rows per step, or one row every `every` steps when even
+    # one row per step would overrun
+    REF_BUDGET_S = 120.0
     t0 = time.perf_counter()
-    O.layer_rows(cfg, x, *(lambda r: (r["expert"], r["gate"], r["keep"]))(
-        O.route(cfg, x, Wr, bias)), host["w1"], host["w3"], host["w2"], host.get("w1s"),
-        host.get("w3s"), host.get("w2s"), [0])
-    t_row = time.perf_counter() - t0
-    rows = max(1, min(wl.T, int(0.5 / max(t_row, 1e-4))))
+    r0 = O.route(cfg, x, Wr, bias)
+    t_route = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.layer_rows(cfg, x, r0["expert"], r0["gate"], r0["keep"], host["w1"], host["w3"], host["w2"],
+                 host.get("w1s"), host.get("w3s"), host.get("w2s"), [0])
+    t_row = max(time.perf_counter() - t0, 1e-4)
+    nsteps = max(1, args.steps + args.warmup)
+    per_step = max(REF_BUDGET_S / nsteps - t_route, 0.0)
+    rows, every = max(1, min(wl.T, int(min(0.5, per_step) / t_row))), 1
+    if per_step < t_row:
+        every = int(np.ceil(t_row / max(per_step, 1e-6)))
     sample_rows = np.arange(rows)
+    count = [0]
 
-    def step():
+    def step(i):
         r = O.route(cfg, x, Wr, bias)
-        O.layer_rows(cfg, x, r["expert"], r["gate"], r["keep"], host["w1"], host["w3"], host["w2"],
-                     host.get("w1s"), host.get("w3s"), host.get("w2s"), sample_rows)
+        if i % every == 0:
+            O.layer_rows(cfg, x, r["expert"], r["gate"], r["keep"], host["w1"], host["w3"],
+                         host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"),
+                         sample_rows)
+            count[0] += rows
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(args.warmup):
+        step(i)
+    count[0] = 0
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        step(i)
     el = time.perf_counter() - t0
-    value = rows * args.steps / el
-    sample = (f"each step: fp64 routing, dispatch and statistics of the whole T={wl.T} batch "
-              f"plus the layer output of {rows} token row(s)")
+    value = max(count[0], 1) / el
+    if every == 1:
+        sample = (f"each step: fp64 routing, dispatch and statistics of the whole T={wl.T} batch "
+                  f"plus the layer output of {rows} token row(s)")
+    else:
+        sample = (f"each step: fp64 routing, dispatch and statistics of the whole T={wl.T} batch; "
+                  f"one step in {every} also the layer output of {rows} token row(s)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
