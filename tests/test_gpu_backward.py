@@ -19,7 +19,7 @@ its error from dg = <G, y> (y carries the forward's ~1.5e-3) and is held to
 the same bar.  The bias gradient db_e = sum_t dz_te
 is a sum over tokens whose terms largely cancel (sum_e db_e = 0), so its
 error, which grows like the root-sum-square of the summands' errors, is
-judged against sqrt(sum_t dz_te^2) per expert instead of |db_e|.
+measured against sqrt(sum_t dz_te^2) per expert instead of |db_e|.
 """
 
 import numpy as np
