@@ -32,6 +32,11 @@ CASES = {
     "g2_nocap": (Workload("ep_nocap", T=300, d=128, h=128, E=4, k=2), 2),
     # one rank: the plain layer through the expert-parallel calls
     "g1": (Workload("ep_g1", T=256, d=128, h=256, E=8, k=2, cf=(5, 4)), 1),
+    # eight ranks of two experts each, a skewed router: some owners receive
+    # nothing from some sources
+    "g8": (Workload("ep_g8", T=512, d=128, h=128, E=16, k=2, cf=(5, 4), zipf_s=1.5), 8),
+    # top-8 of 16 over two ranks, no limit
+    "g2_k8": (Workload("ep_k8", T=192, d=128, h=128, E=16, k=8), 2),
 }
 
 
