@@ -346,7 +346,9 @@ def forward_dist_peers(r: Rank, T_all: int, group=None, max_rows: Optional[int] 
     counts = all_gather_counts(r.route(), r.world, group)
     plan = make_plan(counts, T_all, wl.k, wl.E, wl.cf, r.pad)
     rows = max_rows if max_rows is not None else T_all * wl.k + wl.E * r.pad
-    if int(plan.recv_rows(r.rank).sum()) > rows:
+    # the same test on every rank (the plan is the same), so that all of them
+    # stop together rather than leave the others at a barrier
+    if int(plan.send.sum(axis=0).max()) > rows:
         raise ValueError("the receive buffers are smaller than this step's rows")
     if not hasattr(r, "_symm"):
         grp = group if group is not None else dist.group.WORLD
