@@ -187,6 +187,7 @@ class Rank:
         self.x, self.Wr, self.bias = x, Wr, bias
         self.W13, self.W2p = W13_loc, W2p_loc
         self.pad = B.moe_segment_pad(self.cfg)
+        self.symm = None  # peer-memory form: (recv, y, their symmetric-memory handles)
         rows = max(B.moe_perm_rows(self.cfg), 1)
         i32 = dict(dtype=torch.int32, device=dev)
         self.b = {
@@ -350,12 +351,14 @@ def forward_dist_peers(r: Rank, T_all: int, group=None, max_rows: Optional[int] 
     # stop together rather than leave the others at a barrier
     if int(plan.send.sum(axis=0).max()) > rows:
         raise ValueError("the receive buffers are smaller than this step's rows")
-    if not hasattr(r, "_symm"):
+    if r.symm is None:
         grp = group if group is not None else dist.group.WORLD
         recv = symm_mem.empty(rows, wl.d, dtype=r.x.dtype, device=r.x.device)
         yb = symm_mem.empty(rows, wl.d, dtype=torch.float32, device=r.x.device)
-        r._symm = (recv, yb, symm_mem.rendezvous(recv, grp), symm_mem.rendezvous(yb, grp))
-    recv, yb, h_recv, h_y = r._symm
+        r.symm = (recv, yb, symm_mem.rendezvous(recv, grp), symm_mem.rendezvous(yb, grp))
+    recv, yb, h_recv, h_y = r.symm
+    if recv.shape[0] < rows:
+        raise ValueError("max_rows is larger than the buffers allocated at the first step")
     r.dispatch_peers(plan, list(h_recv.buffer_ptrs))
     h_recv.barrier(channel=0)            # every source has stored its rows here
     n = int(plan.recv_rows(r.rank).sum())
