@@ -151,3 +151,10 @@ def test_peer_dispatch_is_bf16_only():
     cfg = M.make_config(64, 128, 128, 8, 2, dtype="f32")
     d, _ = _peer_call_codes(cfg, 2, [0x200000] * 2)
     assert d == 3
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        B._p(torch.zeros(4))
+    assert B._p(None) is None

@@ -164,3 +164,22 @@ def test_exchanges_over_gloo_ranks():
         # all-to-all put them: its first group starts at peer_row_starts
         for src in range(WORLD):
             assert ep.peer_row_starts(plan, src)[rank] == off[src * plan.E_loc]
+
+
+def test_plan_rejects_experts_not_divisible_by_ranks():
+    with pytest.raises(ValueError):
+        ep.make_plan(np.zeros((3, 8), np.int64), 30, 2, 8, (1, 1), pad=16)
+
+
+def test_capacity_is_the_integer_ceiling():
+    # 2048 tokens, top-2, cf 1.25, 8 experts -> 640; no limit -> every token
+    assert ep.capacity(2048, 2, 8, (5, 4)) == 640
+    assert ep.capacity(4096, 6, 160, (3, 2)) == 231
+    assert ep.capacity(100, 2, 8, None) == 100
+    assert ep.capacity(7, 1, 3, (1, 1)) == 3
+
+
+def test_plan_with_no_tokens_sends_nothing():
+    plan = ep.make_plan(np.zeros((2, 4), np.int64), 0, 2, 4, (1, 1), pad=16)
+    assert plan.send.sum() == 0 and plan.kept.sum() == 0
+    np.testing.assert_array_equal(ep.peer_row_starts(plan, 1), [0, 0])
