@@ -117,6 +117,10 @@ int launch_route_dispatch(const RouteParams& r, const DispatchParams& p, int num
                           cudaStream_t st);
 
 // ---------------------------------------------------------------- tensor-core GEMMs
+// One persistent CTA per SM: a TMA producer warp, an MMA-issuing warp and the
+// epilogue warps (four; sixteen for the swapped gate/up, whose accumulator is
+// single-buffered for wide token tiles).  The down projection takes the
+// swapped tiles only while every group fits 128 tokens.
 enum TcMode : int {
     TC_GATEUP_TOK = 0,   // H = silu(A w1) * (A w3), token-major tiles
     TC_DOWN_TOK = 1,     // y = A W^T (fp32), token-major tiles, optional split-K
