@@ -358,7 +358,10 @@ MOE_API int moe_combine_rows(const moe_config* cfg, const float* y_rows, const i
  * owner: y_rows is a host array of `world` device pointers, y_rows[q] = rank
  * q's fp32 output rows [rows][d] at the row where this rank's rows begin (the
  * same row as dst_rows[q]); topk_idx and offsets are this rank's, from the
- * dispatch.  1 <= world <= MOE_MAX_PEERS, E % world == 0; drop policy. */
+ * dispatch.  1 <= world <= MOE_MAX_PEERS, E % world == 0; drop policy; the
+ * dispatch takes bf16 activations (MOE_ERR_DTYPE otherwise).  Errors: bad
+ * world, a NULL or misaligned pointer, or a reroute config are reported
+ * before any launch. */
 #define MOE_MAX_PEERS 64
 MOE_API int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const void* x,
                                const int32_t* cap, int32_t world, void* const* dst_rows,
