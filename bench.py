@@ -3,11 +3,13 @@
 
 One step = one pass of the whole layer (router, top-k, capacity dispatch,
 expert FFNs, combine, statistics) over one batch of synthetic tokens, through
-the library's public call (moe_forward).  Default workload: the Mixtral-shaped
-decode layer (T=32 tokens, d=4096, h=14336, 8 experts, top-2, bf16), which
-streams all 2.82 GB of expert weights per step.  Under torchrun every rank
-runs its own batch (weak scaling; weights replicated) and the per-rank
-routing statistics are summed across ranks with one NCCL all-reduce.
+the library's public call (moe_forward).  Default workload: the large
+Mixtral-shaped prefill layer (T=16384 tokens, d=4096, h=14336, 8 experts,
+top-2, cf 1.5, Zipf(1.2) router bias, bf16), tensor-core bound; on one GPU the
+same process then times the T=32 decode layer (weight streaming, HBM-bound) and
+reports it under the line's "decode" key.  Under torchrun every rank runs its
+own batch (weak scaling; weights replicated) and the per-rank routing
+statistics are summed across ranks with one NCCL all-reduce.
 
 Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 instead, on a bounded sample of the same workload.  `--backward` (1 GPU) times
@@ -49,7 +51,11 @@ def parse():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="decode", choices=list(WORKLOADS))
+    p.add_argument("--workload", default="large", choices=list(WORKLOADS))
+    p.add_argument("--hidden-mode", default="auto", choices=["auto", "split", "bf16"],
+                   help="how H reaches the down projection (moe_config.hidden_mode)")
+    p.add_argument("--no-decode", action="store_true",
+                   help="skip the decode layer timed after the main workload")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -67,6 +73,8 @@ def parse():
                    help="capture one step in a CUDA graph and replay it (1 GPU)")
     p.add_argument("--no-pdl", action="store_true",
                    help="launch the forward chain without programmatic dependent launch")
+    p.add_argument("--no-pair", action="store_true",
+                   help="one SM per expert GEMM tile (no CTA pairs)")
     p.add_argument("--backward", action="store_true",
                    help="time forward + backward (a training step) instead of the forward (1 GPU)")
     return p.parse_args()
@@ -153,6 +161,93 @@ def kernel_work(name, wl, kept, splits):
     return None
 
 
+def dominant_roofline(trace, wl, cfg, kept):
+    """Roofline of the dominant GEMM among the traced kernels: its algorithmic
+    work per launch over its mean CUDA-event duration, against the measured
+    HBM copy bandwidth (weight-streaming GEMMs) or the measured bf16 tensor
+    rate (sustained for a kernel inside a long step; the burst figure beside)."""
+    pk, pk_kind = peaks()
+    splits = B.moe_ffn_splits(cfg)
+    known = [r for r in trace if kernel_work(r[0], wl, kept, splits)]
+    if not known:
+        return None
+    name, launches, tot_ms = max(known, key=lambda r: r[2])
+    per = tot_ms / launches / 1000.0
+    bound, amount, _ = kernel_work(name, wl, kept, splits)
+    if bound == "hbm":
+        ach, peak, unit = amount / per / 1e9, pk["hbm_gbs"], "GB/s"
+        extra = {}
+    else:
+        ach, unit = amount / per / 1e12, "TFLOP/s"
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        extra = {"peak_kind": "bf16 sustained", "peak_burst": pk["bf16_tflops"],
+                 "frac_burst": ach / pk["bf16_tflops"]}
+    out = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+           "frac": ach / peak, "peak_source": pk_kind, "algorithmic_per_launch": amount,
+           "launch_us": per * 1e6, "traffic": traffic_from_profile(name, wl.name)}
+    out.update(extra)
+    return out
+
+
+def decode_line(args, dev, stream, wl_main, W_main):
+    """The T=32 decode layer timed in the same process after the main workload
+    (inputs resident in HBM; its 2.82 GB of expert weights stream from HBM each
+    step), with its own dominant-kernel and layer rooflines."""
+    wl = WORKLOADS["decode"]
+    cfg = B.config_of(wl, hidden=args.hidden_mode)
+    Wr = I.router_weights(wl)
+    bias = I.router_bias(wl)
+    x, _ = I.tokens(wl, Wr=Wr, b=bias)
+    same = (wl.d, wl.h, wl.E, wl.seed, wl.dtype) == (wl_main.d, wl_main.h, wl_main.E,
+                                                     wl_main.seed, wl_main.dtype)
+    if same:  # the expert weights depend on the shape and the seed only
+        W13, W2p = W_main[0], W_main[1]
+    else:
+        w = I.expert_weights(wl)
+        W13, W2p = B.pack_weights(cfg, *(w[k].to(dev) for k in ("w1", "w3", "w2")))
+    g = {"x": x.to(dev), "Wr": Wr.to(dev), "bias": bias.to(dev) if bias is not None else None}
+    bufs = B.alloc_layer(cfg, dev)
+
+    def step():
+        B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, None, None, bufs["out"],
+                      bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
+                      bufs["slot_of"], bufs["stats"], bufs["ws"])
+
+    steps = max(args.steps, 200)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    B.moe_trace_begin(steps, "gemm_gateup")
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    trace = B.moe_trace_end()
+    ms = ev0.elapsed_time(ev1)
+    status = B.moe_read_device_status(bufs["ws"])
+    kept = bufs["kept"].cpu().tolist()
+    pk, _ = peaks()
+    flops, byts, N, active = algorithmic(wl, kept)
+    t_step = ms / 1000.0 / steps
+    roof_t = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    return {"workload": workload_label(wl), "value": wl.T * steps / (ms / 1000.0),
+            "unit": UNIT, "steps": steps, "ms_per_step": ms / steps,
+            "hidden": "split" if B.moe_hidden_split(cfg) else "bf16",
+            "roofline": dominant_roofline(trace, wl, cfg, kept),
+            "layer_roofline": {"flops": flops, "bytes": byts, "time_us": roof_t * 1e6,
+                               "frac": roof_t / t_step, "kept_assignments": N,
+                               "active_experts": active},
+            "clocks": clk, "device_status": status}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -232,13 +327,13 @@ def cpu_threads():
 
 # ---------------------------------------------------------------- inputs
 
-def build_inputs(wl, rank, world, dev, keep_host, train=False):
+def build_inputs(wl, rank, world, dev, keep_host, train=False, hidden="auto"):
     """Per-rank tokens; expert weights drawn on rank 0 and broadcast.  With
     train, also the backward-layout weights (one GPU)."""
     Wr = I.router_weights(wl)
     bias = I.router_bias(wl)
     x, _ = I.tokens(wl, Wr=Wr, b=bias, stream=dp.token_stream(rank))
-    cfg = B.config_of(wl, train=train)
+    cfg = B.config_of(wl, train=train, hidden=hidden)
     Wb = (None, None, None, None)
     host = {"x": x, "Wr": Wr, "bias": bias}
     dt = I.torch_dtype(wl.dtype)
@@ -412,9 +507,10 @@ def main():
     if args.backward and world > 1:
         raise SystemExit("--backward runs on one GPU")
     B.moe_set_pdl(not args.no_pdl)
+    B.moe_set_pair_tiles(not args.no_pair)
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward
     cfg, host, g, W, Wb = build_inputs(wl, rank, world, dev, keep_host=want_cpu,
-                                       train=args.backward)
+                                       train=args.backward, hidden=args.hidden_mode)
     W13, W2p, W13s, W2s = W
     W13t, W2t, W13st, W2st = Wb
     bufs = B.alloc_layer(cfg, dev)
@@ -596,26 +692,7 @@ def main():
     t_step = ms_max / 1000.0 / args.steps
     roof_t = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
     kernels = {n: {"launches": c, "ms_per_launch": t / c} for n, c, t in trace}
-    splits = B.moe_ffn_splits(cfg)
-    # the dominant kernel among those with a stated algorithmic work (the GEMMs)
-    known = [r for r in trace if kernel_work(r[0], wl, kept, splits)]
-    top = max(known, key=lambda r: r[2]) if known else None
-    roofline = None
-    if top is not None:
-        name, launches, tot_ms = top
-        per = tot_ms / launches / 1000.0
-        work = kernel_work(name, wl, kept, splits)
-        if work:
-            bound, amount, _ = work
-            if bound == "hbm":
-                ach, peak, unit = amount / per / 1e9, pk["hbm_gbs"], "GB/s"
-            else:
-                ach, peak, unit = amount / per / 1e12, pk.get("bf16_tflops_sustained",
-                                                            pk["bf16_tflops"]), "TFLOP/s"
-            roofline = {"kernel": name, "bound": bound, "achieved": ach, "peak": peak,
-                        "unit": unit, "frac": ach / peak, "peak_source": pk_kind,
-                        "algorithmic_per_launch": amount,
-                        "traffic": traffic_from_profile(name, wl.name)}
+    roofline = dominant_roofline(trace, wl, cfg, kept)
     line = {
         "metric": METRIC if not args.backward else METRIC + ", training step (forward + backward)",
         "value": world * wl.T * args.steps / (ms_max / 1000.0),
@@ -632,13 +709,14 @@ def main():
         "config": {"workload": workload_label(wl), "global_batch": world * wl.T,
                    "tokens_per_rank": wl.T,
                    "parallelism": f"dp{world}" if world > 1 else "single",
+                   "hidden": "split" if B.moe_hidden_split(cfg) else "bf16",
                    "l2": ("inputs larger than L2: the active expert weights "
                           f"({active * 3 * wl.d * wl.h * 2 / 1e9:.2f} GB) stream from HBM "
                           "every step")},
         "roofline": roofline,
         "layer_roofline": {"flops": flops, "bytes": byts, "time_us": roof_t * 1e6,
                            "frac": roof_t / t_step, "kept_assignments": N,
-                           "active_experts": active},
+                           "active_experts": active, "peaks": "bf16 burst, HBM copy"},
         "kernels": kernels,
         "gpu_launches": launched,
         "clocks": clk,
@@ -648,6 +726,9 @@ def main():
     }
     if want_cpu:
         line["cpu_baseline"] = time_oracle(wl, host, args.cpu_seconds)
+    if (world == 1 and not args.backward and not args.no_decode and wl.name != "decode"
+            and not args.graph and not args.hidden):
+        line["decode"] = decode_line(args, dev, stream, wl, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -72,6 +72,26 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * The third choice, processing everything, is cf_den = 0 (no limit). */
 typedef enum { MOE_OVERFLOW_DROP = 0, MOE_OVERFLOW_REROUTE = 1 } moe_overflow;
 
+/* How the expert hidden activations H = silu(x w1) * (x w3) reach the down
+ * projection in bf16 configs [the FFN's expand-then-contract, Mixtral 8x7B and
+ * MoE explained, "Easy explanation" ¶2].  H is computed in fp32; rounding it
+ * to bf16 alone costs about 2^-9 relative per element, which after the
+ * h-long sum leaves the layer output about 0.8e-3 (relative L1) further from
+ * the exact result than the bf16 store of the output does on its own.
+ *   MOE_HIDDEN_AUTO   split (below) when no expert can keep more than 128
+ *                     rows (min(C, T) <= 128): the down projection then
+ *                     streams its weights through tiles of 128 weight rows x
+ *                     the expert's tokens, and the extra MMAs run on tensor
+ *                     cores that wait for HBM anyway; bf16 otherwise
+ *   MOE_HIDDEN_SPLIT  H = H_hi + H_lo with H_hi = bf16(H), H_lo = bf16(H - H_hi)
+ *                     (16 significant bits); the down projection issues two
+ *                     MMAs per K step into one fp32 accumulator.  Costs 2 N d h
+ *                     more tensor FLOPs (a third more per layer), N h 2 bytes
+ *                     of workspace and their write and read.
+ *   MOE_HIDDEN_BF16   H rounded to bf16: one MMA per K step, the fastest.
+ * fp32 configs keep H in fp32 and ignore the field. */
+typedef enum { MOE_HIDDEN_AUTO = 0, MOE_HIDDEN_SPLIT = 1, MOE_HIDDEN_BF16 = 2 } moe_hidden_mode;
+
 /* Layer configuration.
  *   T         tokens in the batch (0 allowed: every call is a no-op that
  *             writes zero statistics)
@@ -88,7 +108,8 @@ typedef enum { MOE_OVERFLOW_DROP = 0, MOE_OVERFLOW_REROUTE = 1 } moe_overflow;
  *   overflow  moe_overflow (0 = drop)
  *   train     1: moe_forward also keeps in ws what moe_backward reads (the
  *             gate/up pre-activations, bf16); bf16 configs only.  The
- *             workspace grows accordingly (moe_workspace_size).          */
+ *             workspace grows accordingly (moe_workspace_size).
+ *   hidden_mode  moe_hidden_mode (0 = auto)                               */
 typedef struct {
     int64_t T;
     int32_t d, h, E, k, n_shared, h_shared;
@@ -97,6 +118,7 @@ typedef struct {
     int32_t has_bias;
     int32_t overflow;
     int32_t train;
+    int32_t hidden_mode;
 } moe_config;
 
 /* Routing statistics [MoE routing fully explained, "Easy explanation" ¶4 and
@@ -134,6 +156,11 @@ MOE_API int moe_perm_rows(const moe_config* cfg, int64_t* rows);
 /* Number of split-K partial buffers moe_expert_ffn writes into y_perm
  * (y_perm is [splits][moe_perm_rows][d] fp32). */
 MOE_API int moe_ffn_splits(const moe_config* cfg, int32_t* splits);
+
+/* *split = 1 if this config feeds the hidden activations to the down
+ * projection as two bf16 parts (moe_hidden_mode: MOE_HIDDEN_SPLIT, or
+ * MOE_HIDDEN_AUTO with min(C, T) <= 128; bf16 configs), else 0. */
+MOE_API int moe_hidden_split(const moe_config* cfg, int32_t* split);
 
 /* Text of the last failing call on this thread ("" if none). */
 MOE_API const char* moe_last_error(void);
@@ -292,8 +319,9 @@ MOE_API int moe_backward(const moe_config* cfg, const void* grad_out, float aux_
  * cap[e] = C - (assignments to e on lower ranks) with moe_dispatch_capped,
  * sends each expert's rows to its owner, which runs moe_expert_ffn_grouped on
  * the (source rank, expert) groups it received, and gets the output rows back
- * for moe_combine.  The host-side plan and the exchanges live in the Python
- * package (ep.py). */
+ * for moe_combine.  The exchanges live in the Python package (ep.py); the
+ * plan (caps, where each rank's rows land, the groups an owner receives) is
+ * either computed there on the host or on the device by moe_ep_plan. */
 
 /* Row padding of each expert segment in x_perm for this config (the
  * receiver of a segment needs it to find the next one). */
@@ -312,6 +340,30 @@ MOE_API int moe_dispatch_capped(const moe_config* cfg, const int32_t* topk_idx, 
                                 const int32_t* cap, int32_t* routed, int32_t* kept,
                                 int32_t* offsets, int32_t* perm_token, int32_t* slot_of,
                                 void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* The expert-parallel plan of rank `rank` of `world`, on the device, from
+ * counts (device int32 [world][E]: every rank's moe_route_counts, gathered in
+ * rank order) and the capacity C of the whole concatenated batch [MoE routing
+ * fully explained, "Easy explanation" ¶5]; cfg is the rank's local config
+ * (its segment padding is used).  With base[s][e] = sum of counts[s'][e] over
+ * s' < s, rank s keeps kept[s][e] = min(counts[s][e], max(C - base[s][e], 0))
+ * rows of expert e in a segment of seg[s][e] = kept rounded up to the padding:
+ *   cap [E]            max(C - base[rank][e], 0): moe_dispatch_capped's cap
+ *   row_start [world]  for owner q, the rows lower ranks send to q (the
+ *                      segments of q's experts): where this rank's rows begin
+ *                      in q's receive and output buffers
+ *   group_rows / group_off / group_weight [world * E/world]  the (source,
+ *                      local expert) groups this rank receives, sources in
+ *                      order, then experts: kept rows, first row, expert
+ *   recv_rows [1]      the rows this rank receives (padded)
+ * all device int32.  Nothing is read back to the host, so a step of the
+ * peer-memory form needs no host synchronisation.  Errors: world out of
+ * range or not dividing E, rank out of range, C < 0, a NULL or misaligned
+ * pointer; reported before any launch. */
+MOE_API int moe_ep_plan(const moe_config* cfg, int32_t world, int32_t rank,
+                        const int32_t* counts, int64_t C, int32_t* cap, int32_t* row_start,
+                        int32_t* group_rows, int32_t* group_off, int32_t* group_weight,
+                        int32_t* recv_rows, void* stream);
 
 /* Workspace of moe_expert_ffn_grouped for `rows` input rows. */
 MOE_API int moe_grouped_workspace_size(const moe_config* cfg, int64_t rows,
@@ -345,33 +397,36 @@ MOE_API int moe_combine_rows(const moe_config* cfg, const float* y_rows, const i
  * moe_dispatch_peers is moe_dispatch_capped whose row copies go straight to
  * the owners: the kept rows of expert e (owner q = e / E_loc) are written,
  * segment by segment as moe_dispatch_capped lays them out in x_perm, starting
- * at dst_rows[q] -- rank q's receive buffer at the row where this rank's rows
- * begin (the rows that lower ranks send to q come first).  dst_rows is a host
- * array of `world` device pointers (16-byte aligned, [rows][d] of the
- * activation type), each this GPU's memory or a peer's mapped into this
- * process (CUDA IPC, symmetric memory); the kernel stores through them over
- * NVLink.  offsets, slot_of and perm_token keep their local (x_perm)
- * meaning.  The caller orders the stores before the owners read them (a
- * stream-ordered barrier across the ranks).
+ * at row dst_row_start[q] of dst_rows[q] -- rank q's receive buffer, where
+ * this rank's rows begin after the rows that lower ranks send to q.
+ * dst_rows is a host array of `world` device pointers (16-byte aligned,
+ * [rows][d] of the activation type), each this GPU's memory or a peer's
+ * mapped into this process (CUDA IPC, symmetric memory); the kernel stores
+ * through them over NVLink.  dst_row_start is device int32 [world] (e.g.
+ * moe_ep_plan's row_start), or NULL when dst_rows[q] already point at this
+ * rank's first row.  offsets, slot_of and perm_token keep their local
+ * (x_perm) meaning.  The caller orders the stores before the owners read
+ * them (a stream-ordered barrier across the ranks).
  *
  * moe_combine_peers is moe_combine_rows with each output row read from its
  * owner: y_rows is a host array of `world` device pointers, y_rows[q] = rank
- * q's fp32 output rows [rows][d] at the row where this rank's rows begin (the
- * same row as dst_rows[q]); topk_idx and offsets are this rank's, from the
- * dispatch.  1 <= world <= MOE_MAX_PEERS, E % world == 0; drop policy; the
- * dispatch takes bf16 activations (MOE_ERR_DTYPE otherwise).  Errors: bad
- * world, a NULL or misaligned pointer, or a reroute config are reported
- * before any launch. */
+ * q's fp32 output rows [rows][d], this rank's rows from row y_row_start[q]
+ * on (device int32 [world], or NULL = 0); topk_idx and offsets are this
+ * rank's, from the dispatch.  1 <= world <= MOE_MAX_PEERS, E % world == 0;
+ * drop policy; the dispatch takes bf16 activations (MOE_ERR_DTYPE
+ * otherwise).  Errors: bad world, a NULL or misaligned pointer, or a reroute
+ * config are reported before any launch. */
 #define MOE_MAX_PEERS 64
 MOE_API int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const void* x,
                                const int32_t* cap, int32_t world, void* const* dst_rows,
-                               int32_t* routed, int32_t* kept, int32_t* offsets,
-                               int32_t* perm_token, int32_t* slot_of, void* ws, size_t ws_bytes,
-                               void* stream);
+                               const int32_t* dst_row_start, int32_t* routed, int32_t* kept,
+                               int32_t* offsets, int32_t* perm_token, int32_t* slot_of, void* ws,
+                               size_t ws_bytes, void* stream);
 MOE_API int moe_combine_peers(const moe_config* cfg, int32_t world, const float* const* y_rows,
-                              const int32_t* topk_idx, const int32_t* offsets,
-                              const int32_t* slot_of, const float* topk_gate,
-                              const float* y_shared, void* out, void* stream);
+                              const int32_t* y_row_start, const int32_t* topk_idx,
+                              const int32_t* offsets, const int32_t* slot_of,
+                              const float* topk_gate, const float* y_shared, void* out,
+                              void* stream);
 
 /* ---- routing without a workspace ----------------------------------------- */
 
@@ -383,13 +438,18 @@ MOE_API int moe_combine_peers(const moe_config* cfg, int32_t world, const float*
  * kernels, same results: topk_idx [T][k] int32 and topk_gate [T][k] fp32) but
  * takes no workspace and allocates nothing.  Its scratch (the logits and the
  * statistics partials) is a file-scope device array of
- * MOE_ROUTE_STATIC_SCRATCH bytes inside the library, held by every GPU that
- * loads the library until the process exits.  Limits: T <= MOE_ROUTE_STATIC_MAX_T
+ * MOE_ROUTE_STATIC_SCRATCH bytes inside the library, held by a GPU from the
+ * first call on it until the process exits.  Limits: T <= MOE_ROUTE_STATIC_MAX_T
  * and T * E <= MOE_ROUTE_STATIC_MAX_TE, else MOE_ERR_SHAPE.  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) and should
- * come before any stream capture.  All calls share the array and each call
- * overwrites what the last one left; calls that overlap on the GPU race, so
- * the caller must serialise them (one stream, or events between streams). */
+ * device looks up the array's device address (cudaGetSymbolAddress); under
+ * CUDA's lazy module loading (the default) that is also when the array is
+ * placed on the device, so a caller whose device footprint must not grow later
+ * makes one warm-up call per device at start-up, and that first call should
+ * come before any stream capture.  The address is looked up again when the
+ * device's context changes (after cudaDeviceReset).  All calls share the
+ * array and each call overwrites what the last one left; calls that overlap on
+ * the GPU race, so the caller must serialise them (one stream, or events
+ * between streams). */
 #define MOE_ROUTE_STATIC_SCRATCH (512u * 1024u)
 #define MOE_ROUTE_STATIC_MAX_T 256
 #define MOE_ROUTE_STATIC_MAX_TE 65536
@@ -414,6 +474,14 @@ MOE_API int moe_launch_count(uint64_t* n);
  * the swapped gate/up GEMM prefetches its first weight tiles into L2 while the
  * routing runs.  Results are identical either way.  Process-wide. */
 MOE_API int moe_set_pdl(int on);
+
+/* Expert GEMMs whose experts each keep more than 128 and at most 256 tokens
+ * (default on): each tile runs as one tcgen05 MMA over a pair of SMs (a
+ * cluster of two CTAs), M = 256 weight rows, each SM staging half of the
+ * expert's token rows, which leaves room for a deeper load pipeline and a
+ * double-buffered accumulator.  Off: one SM per tile.  Results agree within
+ * the layer's tolerance (the fp32 sums run in the same order).  Process-wide. */
+MOE_API int moe_set_pair_tiles(int on);
 
 /* Upper bound, in nanoseconds, on every device-side wait of the tensor-core
  * kernels (default 2e9).  A wait that runs out records MOE_ERR_TIMEOUT in

@@ -30,7 +30,8 @@ EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_split
            "moe_trace_begin", "moe_trace_end", "moe_backward_workspace_size", "moe_backward",
            "moe_launch_count", "moe_segment_pad", "moe_route_counts", "moe_dispatch_capped",
            "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows", "moe_set_pdl",
-           "moe_dispatch_peers", "moe_combine_peers"]
+           "moe_dispatch_peers", "moe_combine_peers", "moe_hidden_split", "moe_set_pair_tiles",
+           "moe_ep_plan"]
 
 MOE_MAX_PEERS = 64
 
@@ -56,6 +57,7 @@ class MoEConfig(ctypes.Structure):
         ("has_bias", ctypes.c_int32),
         ("overflow", ctypes.c_int32),
         ("train", ctypes.c_int32),
+        ("hidden_mode", ctypes.c_int32),
     ]
 
 
@@ -79,6 +81,7 @@ def load() -> ctypes.CDLL:
             "moe_workspace_size": [C, P],
             "moe_perm_rows": [C, P],
             "moe_ffn_splits": [C, P],
+            "moe_hidden_split": [C, P],
             "moe_pack_weights": [C, I, P, P, P, P, P, P],
             "moe_route": [C, P, P, P, P, P, P, P, S, P],
             "moe_dispatch": [C, P, P, P, P, P, P, P, P, P, S, P],
@@ -100,9 +103,12 @@ def load() -> ctypes.CDLL:
             "moe_dispatch_capped": [C, P, P, P, P, P, P, P, P, P, P, S, P],
             "moe_grouped_workspace_size": [C, ctypes.c_int64, ctypes.c_int32, P],
             "moe_combine_rows": [C, P, P, P, P, P, P],
-            "moe_dispatch_peers": [C, P, P, P, ctypes.c_int32, P, P, P, P, P, P, P, S, P],
-            "moe_combine_peers": [C, ctypes.c_int32, P, P, P, P, P, P, P, P],
+            "moe_dispatch_peers": [C, P, P, P, ctypes.c_int32, P, P, P, P, P, P, P, P, S, P],
+            "moe_combine_peers": [C, ctypes.c_int32, P, P, P, P, P, P, P, P, P],
+            "moe_ep_plan": [C, ctypes.c_int32, ctypes.c_int32, P, ctypes.c_int64, P, P, P, P, P,
+                            P, P],
             "moe_set_pdl": [I],
+            "moe_set_pair_tiles": [I],
             "moe_expert_ffn_grouped": [C, P, ctypes.c_int64, ctypes.c_int32, P, P, P,
                                        ctypes.c_int32, P, P, P, P, S, P],
             "moe_backward": [C, P, ctypes.c_float, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P,
@@ -144,19 +150,28 @@ def _stream(stream) -> ctypes.c_void_p:
 # ---------------------------------------------------------------- config
 
 OVERFLOW = {"drop": 0, "reroute": 1}
+HIDDEN = {"auto": 0, "split": 1, "bf16": 2}
 
 
 def make_config(T, d, h, E, k, n_shared=0, h_shared=0, cf=None, dtype="bf16",
-                has_bias=False, overflow="drop", train=False) -> MoEConfig:
+                has_bias=False, overflow="drop", train=False, hidden="auto") -> MoEConfig:
     num, den = (0, 0) if cf is None else cf
     return MoEConfig(T, d, h, E, k, n_shared, h_shared, num, den,
                      MOE_BF16 if dtype == "bf16" else MOE_F32, 1 if has_bias else 0,
-                     OVERFLOW[overflow], 1 if train else 0)
+                     OVERFLOW[overflow], 1 if train else 0, HIDDEN[hidden])
 
 
-def config_of(wl: Workload, T: Optional[int] = None, train: bool = False) -> MoEConfig:
+def config_of(wl: Workload, T: Optional[int] = None, train: bool = False,
+              hidden: str = "auto") -> MoEConfig:
     return make_config(wl.T if T is None else T, wl.d, wl.h, wl.E, wl.k, wl.n_shared,
-                       wl.h_shared, wl.cf, wl.dtype, wl.has_bias, wl.overflow, train)
+                       wl.h_shared, wl.cf, wl.dtype, wl.has_bias, wl.overflow, train, hidden)
+
+
+def moe_hidden_split(cfg: MoEConfig) -> bool:
+    """Whether this config feeds H to the down projection as two bf16 parts."""
+    v = ctypes.c_int32()
+    _check(load().moe_hidden_split(ctypes.byref(cfg), ctypes.byref(v)))
+    return bool(v.value)
 
 
 def act_dtype(cfg: MoEConfig) -> torch.dtype:
@@ -311,24 +326,34 @@ def _ptr_array(ptrs):
 
 
 def moe_dispatch_peers(cfg, topk_idx, x, cap, dst_rows, routed, kept, offsets, perm_token,
-                       slot_of, ws, stream=None):
-    """dst_rows: one device address per rank (ints), each the row of that
-    rank's receive buffer where this rank's rows begin."""
+                       slot_of, ws, dst_row_start=None, stream=None):
+    """dst_rows: one device address per rank (ints), each rank's receive
+    buffer; this rank's rows begin at row dst_row_start[q] there (device
+    int32 [world]) or, when it is None, at dst_rows[q] itself."""
     arr = _ptr_array(dst_rows)
     _check(load().moe_dispatch_peers(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(cap),
-                                     len(dst_rows), arr, _p(routed), _p(kept), _p(offsets),
-                                     _p(perm_token), _p(slot_of), _p(ws),
+                                     len(dst_rows), arr, _p(dst_row_start), _p(routed),
+                                     _p(kept), _p(offsets), _p(perm_token), _p(slot_of), _p(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_combine_peers(cfg, y_rows, topk_idx, offsets, slot_of, topk_gate, y_shared, out,
-                      stream=None):
-    """y_rows: one device address per rank (ints), each the row of that
-    rank's fp32 output rows where this rank's rows begin."""
+                      y_row_start=None, stream=None):
+    """y_rows: one device address per rank (ints), each rank's fp32 output
+    rows; this rank's rows begin at row y_row_start[q] (device int32
+    [world]) or, when it is None, at y_rows[q] itself."""
     arr = _ptr_array(y_rows)
-    _check(load().moe_combine_peers(ctypes.byref(cfg), len(y_rows), arr, _p(topk_idx),
-                                    _p(offsets), _p(slot_of), _p(topk_gate), _p(y_shared),
-                                    _p(out), _stream(stream)))
+    _check(load().moe_combine_peers(ctypes.byref(cfg), len(y_rows), arr, _p(y_row_start),
+                                    _p(topk_idx), _p(offsets), _p(slot_of), _p(topk_gate),
+                                    _p(y_shared), _p(out), _stream(stream)))
+
+
+def moe_ep_plan(cfg, world: int, rank: int, counts, C: int, cap, row_start, group_rows,
+                group_off, group_weight, recv_rows, stream=None):
+    """The expert-parallel plan of `rank` on the device (see include/moe.h)."""
+    _check(load().moe_ep_plan(ctypes.byref(cfg), int(world), int(rank), _p(counts), int(C),
+                              _p(cap), _p(row_start), _p(group_rows), _p(group_off),
+                              _p(group_weight), _p(recv_rows), _stream(stream)))
 
 
 def moe_launch_count() -> int:
@@ -339,6 +364,10 @@ def moe_launch_count() -> int:
 
 def moe_set_pdl(on: bool):
     _check(load().moe_set_pdl(1 if on else 0))
+
+
+def moe_set_pair_tiles(on: bool):
+    _check(load().moe_set_pair_tiles(1 if on else 0))
 
 
 def moe_set_wait_limit_ns(ns: int):

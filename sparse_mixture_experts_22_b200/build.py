@@ -37,8 +37,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *extra, "-shared", "-o", tmp, *sources(), "-lcuda" if False else ""]
-    cmd = [c for c in cmd if c]
+    cmd = [nvcc, *NVCC_FLAGS, *extra, "-shared", "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

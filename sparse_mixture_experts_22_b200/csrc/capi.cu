@@ -95,6 +95,11 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
         *why = "train = 1 (backward pass) needs act_dtype MOE_BF16";
         return MOE_ERR_UNSUPPORTED;
     }
+    if (c.hidden_mode != MOE_HIDDEN_AUTO && c.hidden_mode != MOE_HIDDEN_SPLIT &&
+        c.hidden_mode != MOE_HIDDEN_BF16) {
+        *why = "hidden_mode must be MOE_HIDDEN_AUTO, MOE_HIDDEN_SPLIT or MOE_HIDDEN_BF16";
+        return MOE_ERR_ARG;
+    }
 
     Plan& P = *p;
     P.T = c.T; P.d = c.d; P.h = c.h; P.E = c.E; P.k = c.k; P.S = c.n_shared;
@@ -112,6 +117,12 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     const int64_t nmax = P.C < P.T ? P.C : P.T;  // most rows one expert can keep
     P.bf16 = c.act_dtype == MOE_BF16;
     P.act_bytes = P.bf16 ? 2 : 4;
+    // H as two bf16 parts: asked for, or (auto) when no expert can keep more
+    // than DOWN_SWAP_MAX_TOKENS rows -- the down projection then streams its
+    // weights through swapped tiles, and the second MMA per K step runs on
+    // tensor cores that wait for HBM anyway
+    P.split = P.bf16 && (c.hidden_mode == MOE_HIDDEN_SPLIT ||
+                         (c.hidden_mode == MOE_HIDDEN_AUTO && nmax <= DOWN_SWAP_MAX_TOKENS));
     if (!P.bf16) {
         P.path = PATH_F32;
         P.shared_path = PATH_F32;
@@ -181,9 +192,10 @@ int make_plan(const moe_config* cfg, Plan* p, const char** why) {
     P.off_offsets = take((size_t)(c.E + 1) * 4);
     P.off_perm = take((size_t)P.perm_rows * 4);
     P.off_xperm = take((size_t)P.perm_rows * c.d * P.act_bytes);
-    P.off_H = take((size_t)P.perm_rows * c.h * P.act_bytes);
+    // H [perm_rows][h]; split: the low parts in the next perm_rows rows
+    P.off_H = take((size_t)(P.split ? 2 : 1) * P.perm_rows * c.h * P.act_bytes);
     P.off_y = take((size_t)P.splits * P.perm_rows * c.d * 4);
-    P.off_Hs = take(P.S ? (size_t)c.T * P.hsum * P.act_bytes : 0);
+    P.off_Hs = take(P.S ? (size_t)(P.split ? 2 : 1) * c.T * P.hsum * P.act_bytes : 0);
     P.off_ys = take(P.S ? (size_t)c.T * c.d * 4 : 0);
     P.off_sums = take((size_t)(2 + 3 * c.E) * 8);
     P.train = c.train != 0;
@@ -288,6 +300,7 @@ static int tmap_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
 
 static int g_pdl_enabled = 1;
 static thread_local bool g_pdl_in_forward = false;
+static int g_pair_enabled = 1;  // swapped tiles of more than 128 tokens on CTA pairs
 
 bool pdl_active() { return g_pdl_enabled && g_pdl_in_forward; }
 
@@ -409,7 +422,7 @@ static int run_tc_router(const Plan& P, const Device& dv, const void* x, const v
     // rows past 3E of the split weights lie outside the tensor map: TMA reads zeros there
     MOE_TRY(tmap_bf16(&m_act, x, P.T, P.d, 128));
     MOE_TRY(tmap_bf16(&m_w, Ws, 3LL * P.E, P.d, P.router_bn));
-    a.stages = tc_max_stages(TC_DOWN_TOK, P.router_bn, 16, 1, dv.smem_optin);
+    a.stages = tc_max_stages(TC_DOWN_TOK, P.router_bn, 16, 1, false, dv.smem_optin);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, "router_gemm");
     MOE_TRY(launched(launch_tc_gemm(TC_DOWN_TOK, P.router_bn, m_act, m_w, a, dv.sms, st),
@@ -492,6 +505,7 @@ static DispatchParams dispatch_params(const Plan& P, const void* x, int32_t* rou
     d.nsub = P.nsub;
     d.peer_rows = nullptr;  // one destination: x_perm
     d.npeer = 0;
+    d.peer_start = nullptr;
     d.e_loc = P.E;
     return d;
 }
@@ -590,6 +604,9 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.nt_max = nt_max;
     const int smem_limit = dv.smem_optin;
 
+    // split H: its low bf16 parts follow the high ones, act_rows rows further
+    a.lo_rows = P.split ? act_rows : 0;
+
     // gate/up: act [act_rows][d] x W13 [groups * 2hid][d] -> H [act_rows][hid]
     const int mode1 = tok ? TC_GATEUP_TOK : TC_GATEUP_SWAP;
     MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, tok ? 128 : 16));
@@ -603,14 +620,27 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.split_stride = 0;
     a.aux = AB;  // pre-activations for the backward pass (null: not kept)
     a.aux_ld = 2 * (int64_t)hid;
-    a.stages = tc_max_stages(mode1, 256, nt_max, groups, smem_limit);
-    // while the routing finishes, prefetch the start of each CTA's first weight
-    // tile (the unit it gets when every expert has tokens) into L2
-    a.prefetch_kb = (!tok && !group_w && pdl_active()) ? 16 : 0;
-    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
-    trace_pre(st, tag1);
-    MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
-    trace_mark(st, tag1);
+    // groups of more than 128 (and at most 256) tokens: swapped tiles on CTA
+    // pairs, each SM staging half of the token rows
+    const bool pair = !tok && g_pair_enabled && nt_max > DOWN_SWAP_MAX_TOKENS;
+    if (pair) {
+        MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 8));
+        MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 64));
+        a.stages = tc_pair_max_stages(TC_PAIR_GATEUP, nt_max, groups, false, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP, m_act, m_w, a, st), tag1));
+        trace_mark(st, tag1);
+    } else {
+        a.stages = tc_max_stages(mode1, 256, nt_max, groups, false, smem_limit);
+        // while the routing finishes, prefetch the start of each CTA's first weight
+        // tile (the unit it gets when every expert has tokens) into L2
+        a.prefetch_kb = (!tok && !group_w && pdl_active()) ? 16 : 0;
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
+        trace_mark(st, tag1);
+    }
 
     // down: H [act_rows][hid] x W2p [groups * d][hid] -> y [splits][act_rows][d]
     // The down projection streams its weights through the wide B operand of the
@@ -618,10 +648,30 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     // weight tile per stage keeps twice the weight bytes in flight of a swapped
     // tile next to a token tile that large, and the accumulator stays
     // double-buffered; the second token tile of a group is partly idle.
+    const bool pair_down = pair && P.d % 256 == 0;
+    if (pair_down) {
+        MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 8));
+        MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
+        a.K = hid;
+        a.n_feat = P.d;
+        a.w_rows_per_group = P.d;
+        a.splits = 1;
+        a.out = y;
+        a.out_ld = P.d;
+        a.split_stride = act_rows * (int64_t)P.d;
+        a.aux = nullptr;
+        a.prefetch_kb = 0;
+        a.stages = tc_pair_max_stages(TC_PAIR_DOWN, nt_max, groups, P.split, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag2);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN, m_act, m_w, a, st), tag2));
+        trace_mark(st, tag2);
+        return MOE_OK;
+    }
     const bool dtok = tok || nt_max > DOWN_SWAP_MAX_TOKENS;
     const int mode2 = dtok ? TC_DOWN_TOK : TC_DOWN_SWAP;
     const int bn = (P.d % 256 == 0) ? 256 : 128;
-    MOE_TRY(tmap_bf16(&m_act, H, act_rows, hid, dtok ? 128 : 16));
+    MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, dtok ? 128 : 16));
     MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, dtok ? bn : 128));
     a.K = hid;
     a.n_feat = P.d;
@@ -632,7 +682,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.split_stride = act_rows * (int64_t)P.d;
     a.aux = nullptr;
     a.prefetch_kb = 0;
-    a.stages = tc_max_stages(mode2, bn, nt_max, groups, smem_limit);
+    a.stages = tc_max_stages(mode2, bn, nt_max, groups, P.split, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag2);
     MOE_TRY(launched(launch_tc_gemm(mode2, bn, m_act, m_w, a, dv.sms, st), tag2));
@@ -761,7 +811,7 @@ static int run_tc_backward(const Plan& P, const Device& dv, int groups, const in
     a.out_ld = 2 * (int64_t)hid;
     a.aux = const_cast<void*>(AB);
     a.aux_ld = 2 * (int64_t)hid;
-    a.stages = tc_max_stages(TC_DGATE_TOK, bn1, 16, groups, dv.smem_optin);
+    a.stages = tc_max_stages(TC_DGATE_TOK, bn1, 16, groups, false, dv.smem_optin);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag1);
     MOE_TRY(launched(launch_tc_gemm(TC_DGATE_TOK, bn1, m_act, m_w, a, dv.sms, st), tag1));
@@ -776,7 +826,7 @@ static int run_tc_backward(const Plan& P, const Device& dv, int groups, const in
     a.out = dX;
     a.out_ld = P.d;
     a.aux = nullptr;
-    a.stages = tc_max_stages(TC_DOWN_TOK, bn2, 16, groups, dv.smem_optin);
+    a.stages = tc_max_stages(TC_DOWN_TOK, bn2, 16, groups, false, dv.smem_optin);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag2);
     MOE_TRY(launched(launch_tc_gemm(TC_DOWN_TOK, bn2, m_act, m_w, a, dv.sms, st), tag2));
@@ -815,7 +865,7 @@ static int run_tc_wgrad(const Plan& P, const Device& dv, int groups, const int32
     a.out_ld = n_rows;
     a.group_stride = (int64_t)m_rows * n_rows;
     a.n_fastest = n_rows < m_rows ? 1 : 0;
-    a.stages = tc_max_stages(TC_WGRAD, bn, 16, groups, dv.smem_optin);
+    a.stages = tc_max_stages(TC_WGRAD, bn, 16, groups, false, dv.smem_optin);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag);
     MOE_TRY(launched(launch_tc_gemm(TC_WGRAD, bn, m_a, m_b, a, dv.sms, st), tag));
@@ -868,6 +918,14 @@ int moe_ffn_splits(const moe_config* cfg, int32_t* splits) {
     Plan P;
     MOE_TRY(plan_or_fail(cfg, &P));
     *splits = P.path == PATH_SWAP ? P.splits : 1;
+    return ok();
+}
+
+int moe_hidden_split(const moe_config* cfg, int32_t* split) {
+    if (!split) return fail(MOE_ERR_ARG, "split is NULL");
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    *split = P.split ? 1 : 0;
     return ok();
 }
 
@@ -1129,6 +1187,29 @@ int moe_route_counts(const moe_config* cfg, const void* ws, size_t ws_bytes, int
     return ok();
 }
 
+int moe_ep_plan(const moe_config* cfg, int32_t world, int32_t rank, const int32_t* counts,
+                int64_t C, int32_t* cap, int32_t* row_start, int32_t* group_rows,
+                int32_t* group_off, int32_t* group_weight, int32_t* recv_rows, void* stream) {
+    Plan P;
+    MOE_TRY(plan_or_fail(cfg, &P));
+    if (world < 1 || world > MAX_PEERS) return fail(MOE_ERR_ARG, "world must be 1..MOE_MAX_PEERS");
+    if (P.E % world) return fail(MOE_ERR_SHAPE, "E must be a multiple of world");
+    if (rank < 0 || rank >= world) return fail(MOE_ERR_ARG, "rank must be in [0, world)");
+    if (C < 0) return fail(MOE_ERR_ARG, "C must be >= 0");
+    MOE_TRY(need(counts, "counts"));
+    MOE_TRY(need(cap, "cap"));
+    MOE_TRY(need(row_start, "row_start"));
+    MOE_TRY(need(group_rows, "group_rows"));
+    MOE_TRY(need(group_off, "group_off"));
+    MOE_TRY(need(group_weight, "group_weight"));
+    MOE_TRY(need(recv_rows, "recv_rows"));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    MOE_TRY(launched(launch_ep_plan(counts, world, P.E, rank, C, P.pad, cap, row_start,
+                                    group_rows, group_off, group_weight, recv_rows, st),
+                     "ep_plan"));
+    return ok();
+}
+
 int moe_dispatch_capped(const moe_config* cfg, const int32_t* topk_idx, const void* x,
                         const int32_t* cap, int32_t* routed, int32_t* kept, int32_t* offsets,
                         int32_t* perm_token, int32_t* slot_of, void* x_perm, void* ws,
@@ -1176,9 +1257,10 @@ static int check_peers(const Plan& P, int32_t world, const void* const* ptrs, co
 }
 
 int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const void* x,
-                       const int32_t* cap, int32_t world, void* const* dst_rows, int32_t* routed,
-                       int32_t* kept, int32_t* offsets, int32_t* perm_token, int32_t* slot_of,
-                       void* ws, size_t ws_bytes, void* stream) {
+                       const int32_t* cap, int32_t world, void* const* dst_rows,
+                       const int32_t* dst_row_start, int32_t* routed, int32_t* kept,
+                       int32_t* offsets, int32_t* perm_token, int32_t* slot_of, void* ws,
+                       size_t ws_bytes, void* stream) {
     Plan P;
     MOE_TRY(plan_or_fail(cfg, &P));
     if (!P.bf16) return fail(MOE_ERR_DTYPE, "moe_dispatch_peers: bf16 only");
@@ -1203,6 +1285,7 @@ int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const voi
     d.cap = cap;
     d.peer_rows = dst_rows;
     d.npeer = world;
+    d.peer_start = dst_row_start;
     d.e_loc = P.E / world;
     MOE_TRY(launched(launch_dispatch(d, topk_idx, at<int32_t>(ws, P.off_cnt),
                                      at<int32_t>(ws, P.off_tot), dv.sms, st),
@@ -1211,8 +1294,9 @@ int moe_dispatch_peers(const moe_config* cfg, const int32_t* topk_idx, const voi
 }
 
 int moe_combine_peers(const moe_config* cfg, int32_t world, const float* const* y_rows,
-                      const int32_t* topk_idx, const int32_t* offsets, const int32_t* slot_of,
-                      const float* topk_gate, const float* y_shared, void* out, void* stream) {
+                      const int32_t* y_row_start, const int32_t* topk_idx,
+                      const int32_t* offsets, const int32_t* slot_of, const float* topk_gate,
+                      const float* y_shared, void* out, void* stream) {
     Plan P;
     MOE_TRY(plan_or_fail(cfg, &P));
     if (P.T > 0) {
@@ -1227,9 +1311,11 @@ int moe_combine_peers(const moe_config* cfg, int32_t world, const float* const* 
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     trace_pre(st, "combine");
-    MOE_TRY(launched(launch_combine_peers(y_rows, world, P.E / world, topk_idx, offsets, slot_of,
-                                          topk_gate, P.S > 0 ? y_shared : nullptr, out, P.bf16,
-                                          P.T, P.d, P.k, st),
+    MOE_TRY(maybe(y_row_start, "y_row_start"));
+    MOE_TRY(launched(launch_combine_peers(y_rows, y_row_start, world, P.E / world, topk_idx,
+                                          offsets, slot_of, topk_gate,
+                                          P.S > 0 ? y_shared : nullptr, out, P.bf16, P.T, P.d,
+                                          P.k, st),
                      "combine"));
     trace_mark(st, "combine");
     return ok();
@@ -1264,7 +1350,7 @@ int moe_grouped_workspace_size(const moe_config* cfg, int64_t rows, int32_t max_
     Plan P;
     MOE_TRY(plan_or_fail(cfg, &P));
     if (rows < 0 || max_group_rows < 0) return fail(MOE_ERR_ARG, "rows and max_group_rows must be >= 0");
-    *bytes = grouped_h_offset() + align256((size_t)rows * P.h * P.act_bytes);
+    *bytes = grouped_h_offset() + align256((size_t)(P.split ? 2 : 1) * rows * P.h * P.act_bytes);
     return ok();
 }
 
@@ -1280,7 +1366,8 @@ int moe_expert_ffn_grouped(const moe_config* cfg, const void* x_rows, int64_t ro
         return fail(MOE_ERR_ARG, "moe_expert_ffn_grouped: bad sizes");
     if (!ws) return fail(MOE_ERR_ARG, "ws is NULL");
     if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(MOE_ERR_ALIGN, "ws is not 256-byte aligned");
-    const size_t need_bytes = grouped_h_offset() + align256((size_t)rows * P.h * P.act_bytes);
+    const size_t need_bytes =
+        grouped_h_offset() + align256((size_t)(P.split ? 2 : 1) * rows * P.h * P.act_bytes);
     if (ws_bytes < need_bytes)
         return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes; this call needs %zu", ws_bytes,
                     need_bytes);
@@ -1480,6 +1567,11 @@ int moe_launch_count(uint64_t* n) {
 
 int moe_set_pdl(int on) {
     g_pdl_enabled = on ? 1 : 0;
+    return ok();
+}
+
+int moe_set_pair_tiles(int on) {
+    g_pair_enabled = on ? 1 : 0;
     return ok();
 }
 

@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(256)
 // Destinations of the expert-parallel combine: y row bases of the owners.
 struct PeerY {
     const float* base[MAX_PEERS];
+    const int32_t* start;  // device [npeer] rows to skip at each owner, or null
     int npeer, e_loc;
 };
 
@@ -193,7 +194,10 @@ __global__ void __launch_bounds__(256)
         for (int i = 0; i < MAX_PEERS; ++i)
             if (i < py.npeer) sbase[i] = py.base[i];
     }
-    if (threadIdx.x < py.npeer) sfirst[threadIdx.x] = offsets[threadIdx.x * py.e_loc];
+    // row of slot s at owner o: s - offsets[o * e_loc] + start[o]
+    if (threadIdx.x < py.npeer)
+        sfirst[threadIdx.x] = offsets[threadIdx.x * py.e_loc] -
+                              (py.start ? py.start[threadIdx.x] : 0);
     __syncthreads();
     const int vecs = d / 8;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -310,8 +314,8 @@ int launch_combine(const float* y, int splits, int64_t split_stride, const int32
     return launch_result();
 }
 
-int launch_combine_peers(const float* const* y_rows, int npeer, int e_loc,
-                         const int32_t* topk_idx, const int32_t* offsets,
+int launch_combine_peers(const float* const* y_rows, const int32_t* y_start, int npeer,
+                         int e_loc, const int32_t* topk_idx, const int32_t* offsets,
                          const int32_t* slot_of, const float* gate, const float* y_shared,
                          void* out, bool out_bf16, int64_t T, int d, int k, cudaStream_t st) {
     if (T == 0) return 0;
@@ -320,6 +324,7 @@ int launch_combine_peers(const float* const* y_rows, int npeer, int e_loc,
     for (int i = 0; i < MAX_PEERS; ++i) py.base[i] = i < npeer ? y_rows[i] : nullptr;
     py.npeer = npeer;
     py.e_loc = e_loc;
+    py.start = y_start;
     const int64_t n = T * (d / 8);
     const unsigned blocks = (unsigned)((n + 255) / 256);
     if (out_bf16)

@@ -1,0 +1,524 @@
+// gemm_pair.cu -- expert GEMMs with few tokens per expert, on CTA pairs.
+//
+// The expert FFN [Mixtral 8x7B and MoE explained, "Easy explanation" ¶2: each
+// expert widens the embedding and narrows it back; ¶4: unselected experts are
+// not computed] for layers whose experts each keep up to 256 tokens, such as
+// the DeepSeek-V2-style layer [MoE routing fully explained, "Easy
+// explanation" ¶4: many small routed experts].  The weights then dominate
+// the bytes, so the tiles put weight rows on M and an expert's tokens on N
+// ("swapped" tiles), and the kernel's job is to stream weights at HBM speed.
+//
+// Here each tile is one tcgen05 MMA over a pair of SMs (a cluster of two
+// CTAs, cta_group::2): M = 256 weight rows, 128 in each CTA's shared memory,
+// and the expert's N token rows split N/2 + N/2 between them.  Against a
+// one-SM tile of the same weight rows each SM stages half the token rows, so
+// about twice the pipeline stages fit and the accumulator of up to 256
+// token columns fits twice in TMEM (the epilogue of one tile overlaps the
+// MMAs of the next).
+//
+//   gate/up : unit = 128 hidden features of one expert; CTA v holds the gate
+//             rows of features 64v..64v+63 (accumulator lanes 0-63) and
+//             their up rows (lanes 64-127); the epilogue pairs each gate
+//             warp with the up warp of the same features and exchanges
+//             half of the columns through shared memory, so that each
+//             computes H = silu(gate) * up for half of the tokens.
+//   down    : unit = 256 output features; CTA v holds W2 rows 128v..128v+127
+//             and receives y for them; with H in two bf16 parts a second
+//             MMA per K step adds H_lo.
+//
+// Roles (each CTA, 10 warps): warp 0 loads this CTA's halves with TMA into
+// its own stages (own barriers; no multicast); in the even CTA warp 1 issues
+// the pair MMAs once both CTAs' stages are full, in the odd CTA warp 1
+// relays "my stage is full" to the even CTA; warps 2-9 are the epilogue.
+// The MMA's completion is signalled to both CTAs' barriers at once
+// (tcgen05.commit multicast); the epilogues of both CTAs release an
+// accumulator on the even CTA's barrier.  Every wait is bounded; on a
+// time-out the kernel records MOE_ERR_TIMEOUT, lets the copies it issued
+// land and the MMAs drain, and both CTAs meet at a cluster barrier before
+// TMEM is released.
+#include <stdio.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int PBM = 128;   // weight rows per CTA (accumulator lanes)
+constexpr int PBK = 64;    // K per stage: one 128-byte swizzle row of bf16
+constexpr int PUK = 16;    // K per MMA
+constexpr int PEPI = 8;    // epilogue warps
+constexpr int PTHREADS = 64 + 32 * PEPI;
+constexpr uint64_t P_TEARDOWN_NS = 200000000ull;
+
+__host__ __device__ inline uint32_t p_align(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+struct PairLayout {
+    uint32_t a_bytes, b_bytes, b_lo, stage_bytes, xch_off, flag_off, bar_off, grp_off, total;
+};
+
+// Shared memory of one CTA.  B holds nt_max / 2 token rows (the high parts of
+// H, then as many low parts when split).  The gate/up exchange buffers: per
+// pair of epilogue warps two directions x two chunks x 32 lanes x 8 floats.
+__host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stages, int groups,
+                                                  bool split) {
+    PairLayout L;
+    L.a_bytes = PBM * PBK * 2;
+    L.b_lo = (uint32_t)(nt_max / 2) * PBK * 2;
+    L.b_bytes = p_align(L.b_lo * (split ? 2u : 1u), 1024);
+    L.stage_bytes = L.a_bytes + L.b_bytes;
+    L.xch_off = L.stage_bytes * stages;
+    const uint32_t xch = mode == TC_PAIR_GATEUP ? (PEPI / 2) * 2 * 2 * 32 * 8 * 4 : 0;
+    L.flag_off = L.xch_off + xch;
+    L.bar_off = p_align(L.flag_off + PEPI * 2 * 4, 16);
+    // full[S], relay[S], empty[S], acc_full[2], acc_empty[2], drain, tmem slot
+    L.grp_off = L.bar_off + p_align((3 * stages + 5) * 8 + 8, 16);
+    L.total = L.grp_off + (4 * groups + 1) * 4 + 1024;
+    return L;
+}
+
+struct PUnit {
+    int g, w, rows, row0, nb, ntok;
+};
+
+struct PGroups {
+    const int* start;
+    const int* rows;
+    const int* off;
+    const int* wi;
+    int groups;
+};
+
+__device__ __forceinline__ PUnit p_decode(const PGroups& t, int u) {
+    int lo = 0, hi = t.groups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (t.start[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    PUnit x;
+    x.g = lo;
+    x.w = t.wi[lo];
+    x.rows = t.rows[lo];
+    x.row0 = t.off[lo];
+    x.nb = u - t.start[lo];
+    x.ntok = (x.rows + 15) & ~15;
+    return x;
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
+    tc_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
+                   const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
+    constexpr bool GU = MODE == TC_PAIR_GATEUP;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (p_align(raw, 1024) - raw);
+
+    const int groups = args.num_groups;
+    const bool split = !GU && args.lo_rows != 0;
+    const int S = args.stages;
+    const PairLayout L = pair_layout(MODE, args.nt_max, S, groups, split);
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+    uint64_t* relay = full + S;
+    uint64_t* empty = relay + S;
+    uint64_t* acc_full = empty + S;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    int* g_start = reinterpret_cast<int*>(smem + L.grp_off);
+    int* g_rows = g_start + groups + 1;
+    int* g_off = g_rows + groups;
+    int* g_wi = g_off + groups;
+    int* flags = reinterpret_cast<int*>(smem + L.flag_off);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t v = cluster_ctarank();       // 0: issues the MMAs; 1: relays
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    // accumulator: 128 lanes x nt_max columns, twice when it fits
+    const int acc_stride = args.nt_max;
+    const int n_acc = 2 * acc_stride <= 512 ? 2 : 1;
+    uint32_t tmem_cols = 32;
+    while (tmem_cols < (uint32_t)(acc_stride * n_acc)) tmem_cols <<= 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&relay[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 2 * PEPI);  // one arrive per epilogue warp of each CTA
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_act);
+        prefetch_tmap(&tm_w);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, tmem_cols);
+        tmem_relinquish_pair();
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (warp == 2 && lane == 0) {
+        int acc = 0;
+        for (int g = 0; g < groups; ++g) {
+            int r = args.group_rows ? args.group_rows[g] : args.dense_rows;
+            if (r > args.nt_max) {
+                // a tile holds at most nt_max token columns: clamp and flag
+                if (args.status) atomicCAS(args.status, DEV_OK, DEV_SHAPE);
+                r = args.nt_max;
+            }
+            g_rows[g] = r;
+            g_off[g] = args.group_off ? args.group_off[g] : 0;
+            g_wi[g] = args.group_w ? args.group_w[g] : g;
+            g_start[g] = acc;
+            acc += r > 0 ? args.n_feat / (GU ? 128 : 256) : 0;
+        }
+        g_start[groups] = acc;
+    }
+    tc_fence_before();
+    __syncthreads();
+    // barrier initialisation and TMEM allocation visible to the peer CTA
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const PGroups tab{g_start, g_rows, g_off, g_wi, groups};
+    const int total = g_start[groups];
+    const uint64_t limit = args.wait_limit_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_a = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_par = 0;
+            bool ok = true;
+            const int kblocks = args.K / PBK;
+            for (int u = pair; u < total && ok; u += npairs) {
+                const PUnit x = p_decode(tab, u);
+                const int half = x.ntok / 2;          // token rows this CTA stages
+                const int trow = x.row0 + (int)v * half;
+                const uint32_t bytes =
+                    (uint32_t)PBM * PBK * 2 + (uint32_t)half * PBK * 2 * (split ? 2u : 1u);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, limit)) {
+                        report_timeout(args.status);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * L.stage_bytes;
+                    uint8_t* sb = sa + L.a_bytes;
+                    const int kc = kb * PBK;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    if (GU) {
+                        // gate rows of features 64v.., then their up rows
+                        const int wrow = x.w * args.w_rows_per_group + x.nb * 256 + (int)v * 64;
+                        tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
+                        tma_load_2d_hint(sa + 64 * PBK * 2, &tm_w, &full[stage], kc, wrow + 128,
+                                         pol_w);
+                    } else {
+                        const int wrow = x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM;
+                        tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
+                    }
+                    for (int r = 0; r < half; r += 8)
+                        tma_load_2d_hint(sb + r * PBK * 2, &tm_act, &full[stage], kc, trow + r,
+                                         pol_a);
+                    if (split)  // the low parts of H behind the high ones
+                        for (int r = 0; r < half; r += 8)
+                            tma_load_2d_hint(sb + L.b_lo + r * PBK * 2, &tm_act, &full[stage], kc,
+                                             trow + r + (int)args.lo_rows, pol_a);
+                    issued |= 1u << stage;
+                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // every copy this CTA issued lands before the CTA may leave
+            for (int s = 0; s < S; ++s)
+                if (issued & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1, P_TEARDOWN_NS);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && v == 1) {
+            // ------------------------------------------------------------ relay (odd CTA)
+            const uint32_t peer_relay0 = map_shared_rank(smem_addr(&relay[0]), 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            const int kblocks = args.K / PBK;
+            for (int u = pair; u < total && ok; u += npairs) {
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, limit)) {
+                        report_timeout(args.status);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(peer_relay0 + stage * 8);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        } else if (lane == 0) {
+            // ------------------------------------------------------------ MMA issuer (even CTA)
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            const int kblocks = args.K / PBK;
+            for (int u = pair; u < total && ok; u += npairs) {
+                const PUnit x = p_decode(tab, u);
+                if (!mbar_wait_cl(&acc_empty[acc], acc_phase ^ 1, limit)) {
+                    report_timeout(args.status);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * acc_stride;
+                const uint32_t idesc = idesc_bf16_f32(256, x.ntok);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, limit) ||
+                        !mbar_wait_cl(&relay[stage], phase, limit)) {
+                        report_timeout(args.status);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + stage * L.stage_bytes);
+                    const uint32_t sb = sa + L.a_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < PBK / PUK; ++kk) {
+                        const uint64_t adesc = sdesc_kmajor_sw128(sa + kk * PUK * 2);
+                        umma_bf16_pair(d_tmem, adesc, sdesc_kmajor_sw128(sb + kk * PUK * 2), idesc,
+                                       (kb > 0 || kk > 0) ? 1u : 0u);
+                        if (split)  // + W . H_lo
+                            umma_bf16_pair(d_tmem, adesc,
+                                           sdesc_kmajor_sw128(sb + L.b_lo + kk * PUK * 2), idesc,
+                                           1u);
+                    }
+                    umma_commit_pair_both(&empty[stage]);
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                // test hook: the first unit of pair 0 never signals its epilogues
+                const bool withhold = args.test_stall && pair == 0 && u == pair;
+                if (!withhold) umma_commit_pair_both(&acc_full[acc]);
+                if (++acc == n_acc) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // every pair MMA completes before either CTA releases memory
+            umma_commit_pair(drain);
+            mbar_wait(drain, 0, P_TEARDOWN_NS);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 2;                 // 0..7
+        const int q = warp & 3;                  // TMEM lane quarter this warp may access
+        const int part = ew >> 2;                // which half of the columns
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+        const uint32_t leader_acc_empty = map_shared_rank(smem_addr(&acc_empty[0]), 0);
+        // gate/up: quarters 0,1 hold gate, 2,3 the up rows of the same features;
+        // the warp pair (q, q + 2) of the same part exchanges through `xb`
+        const int pidx = part * 2 + (q & 1);     // pair of warps 0..3
+        float4* xb = reinterpret_cast<float4*>(smem + L.xch_off) + pidx * (2 * 2 * 2 * 32);
+        const bool is_gate = q < 2;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int it = 0;
+        for (int u = pair; u < total; u += npairs, ++it) {
+            const PUnit x = p_decode(tab, u);
+            bool ok = mbar_wait(&acc_full[acc], acc_phase, limit);
+            if (GU) {
+                // both warps of a pair go on only if both saw the accumulator
+                if (lane == 0) flags[ew * 2 + (it & 1)] = ok ? 1 : 0;
+                named_sync(1 + pidx, 64);
+                const int partner = is_gate ? ew - 2 : ew + 2;
+                ok = flags[ew * 2 + (it & 1)] && flags[partner * 2 + (it & 1)];
+            }
+            if (!ok) {
+                report_timeout(args.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = lane_addr + acc * acc_stride;
+            if (GU) {
+                // feature of this lane and its H column
+                const int f = x.nb * 128 + (int)v * 64 + (q & 1) * 32 + lane;
+                __nv_bfloat16* hdst =
+                    reinterpret_cast<__nv_bfloat16*>(args.out) + (int64_t)x.row0 * args.out_ld + f;
+                __nv_bfloat16* abdst =
+                    args.aux ? reinterpret_cast<__nv_bfloat16*>(args.aux) +
+                                   (int64_t)x.row0 * args.aux_ld + (f >> 7) * 256 +
+                                   (is_gate ? 0 : 128) + (f & 127)
+                             : nullptr;
+                int ci = 0;
+#pragma unroll 1
+                for (int c = 16 * part; c < x.ntok; c += 32, ++ci) {
+                    float mine[16];
+                    tmem_ld16(t0 + c, mine);
+                    tmem_ld_wait();
+                    if (abdst) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c + i < x.rows)
+                                abdst[(int64_t)(c + i) * args.aux_ld] = __float2bfloat16_rn(mine[i]);
+                    }
+                    // gate warps compute columns c..c+7, up warps c+8..c+15: each
+                    // sends the other half of its values to its partner
+                    float4* out_buf = xb + ((is_gate ? 0 : 1) * 2 + (ci & 1)) * 64;
+                    float4* in_buf = xb + ((is_gate ? 1 : 0) * 2 + (ci & 1)) * 64;
+                    float give[8], keepv[8];  // values sent / kept (static indices only)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        give[i] = is_gate ? mine[8 + i] : mine[i];
+                        keepv[i] = is_gate ? mine[i] : mine[8 + i];
+                    }
+                    out_buf[lane] = make_float4(give[0], give[1], give[2], give[3]);
+                    out_buf[32 + lane] = make_float4(give[4], give[5], give[6], give[7]);
+                    named_sync(1 + pidx, 64);
+                    const float4 o0 = in_buf[lane], o1 = in_buf[32 + lane];
+                    const float other[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+                    const int keep = is_gate ? 0 : 8;  // this warp's columns within the chunk
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int col = c + keep + i;
+                        if (col < x.rows) {
+                            const float g = is_gate ? keepv[i] : other[i];
+                            const float up = is_gate ? other[i] : keepv[i];
+                            const float hv = silu_f(g) * up;
+                            hdst[(int64_t)col * args.out_ld] = __float2bfloat16_rn(hv);
+                            if (args.lo_rows)
+                                hdst[(int64_t)(col + args.lo_rows) * args.out_ld] =
+                                    __float2bfloat16_rn(hv - bf16_round(hv));
+                        }
+                    }
+                }
+            } else {
+                const int f = x.nb * 256 + (int)v * PBM + q * 32 + lane;
+                float* dst = reinterpret_cast<float*>(args.out) + (int64_t)x.row0 * args.out_ld + f;
+#pragma unroll 1
+                for (int c = 16 * part; c < x.ntok; c += 32) {
+                    float val[16];
+                    tmem_ld16(t0 + c, val);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c + i < x.rows) dst[(int64_t)(c + i) * args.out_ld] = val[i];
+                }
+            }
+            // this warp is done with the accumulator: release it on the even CTA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acc_empty + acc * 8);
+            if (++acc == n_acc) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // neither CTA leaves (or frees TMEM) while the other may still touch its
+    // shared memory or TMEM
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, tmem_cols);
+}
+
+// Pairs that fit the device at once (cached per device and mode).
+int pair_grid(const void* kern, uint32_t smem, int mode) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static int cached[kMaxDevices][2] = {};
+    static uint32_t cached_smem[kMaxDevices][2] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    const int m = mode == TC_PAIR_GATEUP ? 0 : 1;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[dev][m] == 0 || cached_smem[dev][m] != smem) {
+        // the cluster shape comes from the kernel's __cluster_dims__
+        cudaLaunchConfig_t c = {};
+        c.gridDim = dim3(2);
+        c.blockDim = dim3(PTHREADS);
+        c.dynamicSmemBytes = smem;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &c) != cudaSuccess || n < 1) return 0;
+        cached[dev][m] = n;
+        cached_smem[dev][m] = smem;
+    }
+    return cached[dev][m];
+}
+
+template <int MODE>
+int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
+                     cudaStream_t st) {
+    const PairLayout L = pair_layout(MODE, a.nt_max, a.stages, a.num_groups,
+                                     MODE == TC_PAIR_DOWN && a.lo_rows != 0);
+    auto kern = tc_pair_kernel<MODE>;
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static int configured_bytes[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if ((int)L.total > configured_bytes[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     L.total) != cudaSuccess)
+                return -1;
+            configured_bytes[dev] = L.total;
+        }
+    }
+    const int pairs = pair_grid(reinterpret_cast<const void*>(kern), L.total, MODE);
+    if (pairs < 1) {
+        last_launch_error() = cudaErrorInvalidConfiguration;
+        return -1;
+    }
+    // the cluster shape is part of the kernel (__cluster_dims__)
+    launch_ex(pdl_active(), kern, dim3(2 * pairs), dim3(PTHREADS), L.total, st, act, w, a);
+    note_launch();
+    return launch_result();
+}
+
+}  // namespace
+
+int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_limit) {
+    for (int s = 8; s >= 2; --s)
+        if ((int)pair_layout(mode, nt_max, s, groups, mode == TC_PAIR_DOWN && split).total <=
+            smem_limit)
+            return s;
+    return 0;
+}
+
+int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
+                   cudaStream_t st) {
+    if (a.nt_max < 16 || a.nt_max > 256 || a.nt_max % 16) return -1;
+    switch (mode) {
+        case TC_PAIR_GATEUP:
+            return launch_pair_mode<TC_PAIR_GATEUP>(act, w, a, st);
+        case TC_PAIR_DOWN:
+            return launch_pair_mode<TC_PAIR_DOWN>(act, w, a, st);
+    }
+    return -1;
+}
+
+}  // namespace moe

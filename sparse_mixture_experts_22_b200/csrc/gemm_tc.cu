@@ -34,6 +34,8 @@
 // letting its in-flight copies and MMAs finish before TMEM is released.
 #include <stdio.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -74,14 +76,24 @@ __host__ __device__ inline bool staged_epilogue(int mode) {
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Bytes of operand per stage for each mode.
-__host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, uint32_t* a, uint32_t* b) {
+// Whether a launch's down projection reads H as two bf16 parts (high, low):
+// its activation tiles are then staged twice per K step.
+__host__ __device__ inline bool down_split(int mode, int64_t lo_rows) {
+    return (mode == TC_DOWN_TOK || mode == TC_DOWN_SWAP) && lo_rows != 0;
+}
+
+// Bytes of operand per stage for each mode.  With a split H the token-major
+// down stages the high and the low 128-row tile one after the other (A), the
+// swapped down the high and the low token tile (B, nt_max rows each).
+__host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, bool split, uint32_t* a,
+                                            uint32_t* b) {
+    const uint32_t parts = split ? 2 : 1;
     switch (mode) {
         case TC_GATEUP_TOK:
         case TC_DOWN_TOK:
         case TC_DGATE_TOK:
         case TC_WGRAD:
-            *a = BM * BK * 2;
+            *a = (mode == TC_DOWN_TOK ? parts : 1) * BM * BK * 2;
             *b = bn * BK * 2;
             break;
         case TC_GATEUP_SWAP:
@@ -90,15 +102,15 @@ __host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, uint32
             break;
         default:
             *a = BM * BK * 2;
-            *b = nt_max * BK * 2;
+            *b = parts * nt_max * BK * 2;
             break;
     }
 }
 
 __host__ __device__ inline SharedLayout shared_layout(int mode, int bn, int nt_max, int stages,
-                                                      int groups) {
+                                                      int groups, bool split) {
     SharedLayout L;
-    stage_bytes(mode, bn, nt_max, &L.a_bytes, &L.b_bytes);
+    stage_bytes(mode, bn, nt_max, split, &L.a_bytes, &L.b_bytes);
     L.a_bytes = align_up(L.a_bytes, 1024);
     L.b_bytes = align_up(L.b_bytes, 1024);
     L.stage_bytes = L.a_bytes + L.b_bytes;
@@ -242,7 +254,8 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
     uint8_t* smem = smem_raw + (align_up(raw, 1024) - raw);
 
     const int groups = args.num_groups;
-    const SharedLayout L = shared_layout(MODE, BN, args.nt_max, args.stages, groups);
+    const bool dsplit = down_split(MODE, args.lo_rows);
+    const SharedLayout L = shared_layout(MODE, BN, args.nt_max, args.stages, groups, dsplit);
     const int S = args.stages;
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
@@ -361,7 +374,8 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                     uint8_t* sb = sa + L.a_bytes;
                     const int kc = kb * BK;
                     if (TOK) {
-                        mbar_arrive_expect_tx(&full[stage], (BM + BN) * BK * 2);
+                        mbar_arrive_expect_tx(&full[stage],
+                                              (BM * (dsplit ? 2 : 1) + BN) * BK * 2);
                         if (MODE == TC_WGRAD) {
                             // MN-major operands straight from the row-major
                             // activations: boxes of 64 features x 64 token rows
@@ -375,13 +389,17 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                                             x.nb * BN + 64 * i, kc);
                         } else {
                             tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
+                            if (dsplit)  // the same rows' low parts of H
+                                tma_load_2d(sa + BM * BK * 2, &tm_act, &full[stage], kc,
+                                            x.row0 + x.mt * BM + (int)args.lo_rows);
                             tma_load_2d(sb, &tm_w, &full[stage], kc,
                                         x.w * args.w_rows_per_group +
                                             x.nb * (MODE == TC_GATEUP_TOK ? 256 : BN));
                         }
                     } else {
                         const int wa = (MODE == TC_GATEUP_SWAP) ? 2 * BM : BM;
-                        mbar_arrive_expect_tx(&full[stage], (wa + x.ntok) * BK * 2);
+                        mbar_arrive_expect_tx(&full[stage],
+                                              (wa + x.ntok * (dsplit ? 2 : 1)) * BK * 2);
                         const int wrow = x.w * args.w_rows_per_group +
                                          x.nb * (MODE == TC_GATEUP_SWAP ? 256 : BM);
                         tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
@@ -391,6 +409,11 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                         for (int r = 0; r < x.ntok; r += 16)
                             tma_load_2d_hint(sb + r * BK * 2, &tm_act, &full[stage], kc,
                                              x.row0 + r, pol_a);
+                        if (dsplit)  // the low parts of H behind the high ones
+                            for (int r = 0; r < x.ntok; r += 16)
+                                tma_load_2d_hint(sb + (args.nt_max + r) * BK * 2, &tm_act,
+                                                 &full[stage], kc,
+                                                 x.row0 + r + (int)args.lo_rows, pol_a);
                     }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -443,8 +466,15 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                             continue;
                         }
                         const uint64_t bdesc = sdesc_kmajor_sw128(sb + kk * UK * 2);
-                        umma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * UK * 2), bdesc, idesc,
-                                  acc_flag);
+                        const uint64_t adesc = sdesc_kmajor_sw128(sa + kk * UK * 2);
+                        umma_bf16(d_tmem, adesc, bdesc, idesc, acc_flag);
+                        if (MODE == TC_DOWN_TOK && dsplit)  // + H_lo . W
+                            umma_bf16(d_tmem, sdesc_kmajor_sw128(sa + BM * BK * 2 + kk * UK * 2),
+                                      bdesc, idesc, 1u);
+                        if (MODE == TC_DOWN_SWAP && dsplit)  // + W . H_lo
+                            umma_bf16(d_tmem, adesc,
+                                      sdesc_kmajor_sw128(sb + args.nt_max * BK * 2 + kk * UK * 2),
+                                      idesc, 1u);
                         if (MODE == TC_GATEUP_SWAP)
                             umma_bf16(d_tmem + args.nt_max,
                                       sdesc_kmajor_sw128(sa + BM * BK * 2 + kk * UK * 2), bdesc,
@@ -508,17 +538,17 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                         store_bf16x16(abrow + 128 + c, v);
                     }
                     if (valid) {
-                        uint4 o0, o1;
-                        o0.x = pack_bf16x2(silu_f(g[0]) * v[0], silu_f(g[1]) * v[1]);
-                        o0.y = pack_bf16x2(silu_f(g[2]) * v[2], silu_f(g[3]) * v[3]);
-                        o0.z = pack_bf16x2(silu_f(g[4]) * v[4], silu_f(g[5]) * v[5]);
-                        o0.w = pack_bf16x2(silu_f(g[6]) * v[6], silu_f(g[7]) * v[7]);
-                        o1.x = pack_bf16x2(silu_f(g[8]) * v[8], silu_f(g[9]) * v[9]);
-                        o1.y = pack_bf16x2(silu_f(g[10]) * v[10], silu_f(g[11]) * v[11]);
-                        o1.z = pack_bf16x2(silu_f(g[12]) * v[12], silu_f(g[13]) * v[13]);
-                        o1.w = pack_bf16x2(silu_f(g[14]) * v[14], silu_f(g[15]) * v[15]);
-                        *reinterpret_cast<uint4*>(dst + c) = o0;
-                        *reinterpret_cast<uint4*>(dst + c + 8) = o1;
+                        float hv[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) hv[i] = silu_f(g[i]) * v[i];
+                        if (args.lo_rows) {
+                            // low parts: H - bf16(H) is exact in fp32, then rounded
+                            float lo[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) lo[i] = hv[i] - bf16_round(hv[i]);
+                            store_bf16x16(dst + args.lo_rows * args.out_ld + c, lo);
+                        }
+                        store_bf16x16(dst + c, hv);
                     }
                 }
             } else if (MODE == TC_DOWN_TOK) {
@@ -642,9 +672,13 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        if (c + i < x.rows)
-                            dst[(int64_t)(c + i) * args.out_ld] =
-                                __float2bfloat16_rn(silu_f(g[i]) * v[i]);
+                        if (c + i < x.rows) {
+                            const float hv = silu_f(g[i]) * v[i];
+                            dst[(int64_t)(c + i) * args.out_ld] = __float2bfloat16_rn(hv);
+                            if (args.lo_rows)  // low part, lo_rows rows further
+                                dst[(int64_t)(c + i + args.lo_rows) * args.out_ld] =
+                                    __float2bfloat16_rn(hv - bf16_round(hv));
+                        }
                     if (args.aux) {
                         __nv_bfloat16* ab = reinterpret_cast<__nv_bfloat16*>(args.aux) +
                                             (int64_t)x.row0 * args.aux_ld + x.nb * 256 + row;
@@ -688,14 +722,24 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
 template <int MODE, int BN>
 int launch_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, int grid,
                 cudaStream_t st) {
-    const SharedLayout L = shared_layout(MODE, BN, a.nt_max, a.stages, a.num_groups);
+    const SharedLayout L =
+        shared_layout(MODE, BN, a.nt_max, a.stages, a.num_groups, down_split(MODE, a.lo_rows));
     auto kern = tc_gemm_kernel<MODE, BN>;
-    static int configured_bytes = 0;
-    if ((int)L.total > configured_bytes) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total) !=
-            cudaSuccess)
-            return -1;
-        configured_bytes = L.total;
+    // the shared-memory opt-in is a property of the kernel on each device: kept
+    // per device (and per instantiation), under a lock for callers on several threads
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static int configured_bytes[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if ((int)L.total > configured_bytes[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     L.total) != cudaSuccess)
+                return -1;
+            configured_bytes[dev] = L.total;
+        }
     }
     launch_ex(pdl_active(), kern, dim3(grid), dim3(threads_of<MODE>()), L.total, st, act, w, a);
     note_launch();
@@ -704,9 +748,10 @@ int launch_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, i
 
 }  // namespace
 
-int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit) {
+int tc_max_stages(int mode, int bn, int nt_max, int groups, bool split, int smem_limit) {
+    const bool ds = down_split(mode, split ? 1 : 0);
     for (int s = 8; s >= 2; --s)
-        if ((int)shared_layout(mode, bn, nt_max, s, groups).total <= smem_limit) return s;
+        if ((int)shared_layout(mode, bn, nt_max, s, groups, ds).total <= smem_limit) return s;
     return 0;
 }
 

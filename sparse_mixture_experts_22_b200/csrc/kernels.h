@@ -96,6 +96,7 @@ struct DispatchParams {
     // of peer_rows[o] (a host array of npeer device pointers, read at launch).
     void* const* peer_rows;
     int npeer, e_loc;
+    const int32_t* peer_start;  // device [npeer]: rows to skip at each destination, or null
 };
 
 int launch_topk(const RouteParams& r, cudaStream_t st);
@@ -128,6 +129,8 @@ enum TcMode : int {
     TC_DOWN_SWAP = 3,    // down with weight rows as M, split-K
     TC_DGATE_TOK = 4,    // backward: dH = dY W2^T, SiLU*mul backward in the epilogue
     TC_WGRAD = 5,        // backward: C[g] = A[:, K_g] B[:, K_g]^T over each group's token range
+    TC_PAIR_GATEUP = 6,  // gate/up on CTA pairs: 2 x (64 gate + 64 up weight rows) x the tokens
+    TC_PAIR_DOWN = 7,    // down on CTA pairs: 2 x 128 weight rows x the tokens (fp32 out)
 };
 
 struct TcArgs {
@@ -157,11 +160,26 @@ struct TcArgs {
     const int32_t* group_w;     // device [num_groups] weight index of each group, or null -> g
     int prefetch_kb;            // swapped gate/up: k-blocks of the first weight tile to prefetch
                                 // into L2 before waiting on the predecessor (0: none)
+    int64_t lo_rows;            // H as bf16 high + low parts (0: bf16 H alone): gate/up writes
+                                // row r's low parts to row r + lo_rows of `out`; down reads
+                                // them there from the activation tensor and issues a second
+                                // MMA per K step into the same accumulator
 };
 
-int tc_max_stages(int mode, int bn, int nt_max, int groups, int smem_limit);
+// Deepest pipeline (2..8 stages) whose shared memory fits smem_limit; `split`
+// sizes the down projection's stages for H's two parts.
+int tc_max_stages(int mode, int bn, int nt_max, int groups, bool split, int smem_limit);
 int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& w,
                    const TcArgs& a, int grid, cudaStream_t st);
+
+// Swapped tiles on CTA pairs (clusters of two; gemm_pair.cu), for groups of up to
+// 256 tokens: TC_PAIR_GATEUP (act = x rows, 8-row boxes; w = W13, 64-row boxes;
+// n_feat = hidden width) and TC_PAIR_DOWN (act = H rows, 8-row boxes; w = W2p,
+// 128-row boxes; n_feat = model width, a multiple of 256).  nt_max is a multiple
+// of 16 in [16, 256]; the grid is as many pairs as the device holds at once.
+int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_limit);
+int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
+                   cudaStream_t st);
 
 // ---------------------------------------------------------------- fp32 SIMT FFN
 // gate/up: H[r][f] = silu(A_r . W13[g][gate f]) * (A_r . W13[g][up f]);
@@ -192,10 +210,19 @@ struct StatsParams {
 // row found at the expert's owner: expert e = topk_idx[t][j] belongs to rank
 // o = e / e_loc, and its row is slot - offsets[o * e_loc] of y_rows[o] (a host
 // array of npeer device pointers, read at launch).
-int launch_combine_peers(const float* const* y_rows, int npeer, int e_loc,
-                         const int32_t* topk_idx, const int32_t* offsets,
+// y_start (device [npeer], or null) skips that many rows at each owner first.
+int launch_combine_peers(const float* const* y_rows, const int32_t* y_start, int npeer,
+                         int e_loc, const int32_t* topk_idx, const int32_t* offsets,
                          const int32_t* slot_of, const float* gate, const float* y_shared,
                          void* out, bool out_bf16, int64_t T, int d, int k, cudaStream_t st);
+
+// Expert-parallel plan of rank `rank` of G from the gathered counts [G][E]
+// (device), all on the device: cap [E], row_start [G] (rows of lower ranks
+// at each owner), and the (source, local expert) groups this rank receives:
+// g_rows, g_off, g_w [G * E/G], recv [1] their padded total.
+int launch_ep_plan(const int32_t* counts, int G, int E, int rank, int64_t C, int pad,
+                   int32_t* cap, int32_t* row_start, int32_t* g_rows, int32_t* g_off,
+                   int32_t* g_w, int32_t* recv, cudaStream_t st);
 int launch_combine(const float* y, int splits, int64_t split_stride, const int32_t* slot_of,
                    const float* gate, const float* y_shared, void* out, bool out_bf16,
                    int64_t T, int d, int k, const StatsParams* sp, cudaStream_t st);

@@ -58,6 +58,7 @@ struct Plan {
     int router_ld;      // tensor cores: row length of the partial logits (3E rounded to 4)
     int router_splits;  // tensor cores: split-K
     bool train;         // forward keeps the gate/up pre-activations for the backward pass
+    bool split;         // H reaches the down projection as bf16 high + low parts
     int wr_chunks;      // backward: token chunks of the router-weight gradient
 
     // workspace byte offsets

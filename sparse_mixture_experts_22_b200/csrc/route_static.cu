@@ -7,16 +7,21 @@
 // kernels as moe_route (one CTA per token for the logits, then top-k and the
 // gates), but its scratch -- the logits and the per-block statistics
 // partials -- lives in one fixed array of device memory owned by this
-// library.  Every GPU that loads the library holds that array (its size is
-// MOE_ROUTE_STATIC_SCRATCH bytes) until the process exits.
+// library (MOE_ROUTE_STATIC_SCRATCH bytes), held by a GPU from the first call
+// on it until the process exits.
 //
 // Host code cannot use the array's name as a device address (on the host it
 // names a stand-in object), so the device address is looked up once per
 // device with cudaGetSymbolAddress, with that device current, on the first
-// call that runs on the device.  That first call should come before any
-// stream capture.  All calls share the array and each call overwrites what
-// the previous one left there; calls that overlap on the GPU (two streams,
-// two threads) race on it and must be serialised by the caller.
+// call that runs on the device.  Under CUDA's lazy module loading (the
+// default) that lookup is also when the array comes into being on the
+// device, so a caller that must keep its device footprint fixed makes one
+// warm-up call per device at start-up; that first call should also come
+// before any stream capture.  The address is cached with the id of the
+// context it belongs to and looked up again if the device's context changes
+// (after a cudaDeviceReset, say).  All calls share the array and each call
+// overwrites what the previous one left there; calls that overlap on the GPU
+// (two streams, two threads) race on it and must be serialised by the caller.
 #include <string.h>
 
 #include <mutex>
@@ -39,20 +44,53 @@ __device__ __align__(256) uint8_t g_route_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};
 
-// Device address of the scratch array for the current device.
+// Unique id of the current thread's CUDA context (cuCtxGetId through the
+// runtime's driver entry point; 0 when it cannot be had).
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrent)(CUcontext*);
+    typedef CUresult (*GetId)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+        get_id(ctx, &id) == CUDA_SUCCESS)
+        return id;
+    return 0;
+}
+
+// Device address of the scratch array for the current device, looked up on
+// the first call on the device (and again when its context has changed).
 int scratch_for_current_device(uint8_t** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return report_error(MOE_ERR_CUDA, "moe_route_static: cudaGetDevice failed");
+    // 0 when no context is current yet: the lookup below then makes the
+    // device's primary context current
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
         if (e != cudaSuccess || !p)
             return report_error(MOE_ERR_CUDA,
                                 "moe_route_static: cudaGetSymbolAddress of the scratch failed");
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = ctx != 0 ? ctx : current_context_id();
     }
     *out = static_cast<uint8_t*>(g_scratch_ptr[dev]);
     return MOE_OK;

@@ -140,13 +140,11 @@ int launch_logits_t(const XT* x, const float* Wr, float* z, int64_t T, int d, in
     const int dch = d < RT_DCH ? d : RT_DCH;
     const size_t smem = (size_t)RT_EXP * (dch + 4) * sizeof(float);
     auto kern = router_logits_kernel<XT, TPW>;
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    // the opt-in is per device: set it on every launch that needs it
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
-            return -1;
-        configured = smem;
-    }
+        return -1;
     kern<<<grid, RT_WARPS * 32, smem, st>>>(x, Wr, z, T, d, E, dch);
     note_launch();
     return launch_result();

@@ -324,6 +324,7 @@ struct DispatchArgs {
     int nsub;              // histogram rows per block (the top-k CTAs of a block)
     int npeer, e_loc;      // row destinations: expert e -> peer[e / e_loc] (see place_rows)
     uint4* peer[MAX_PEERS];
+    const int32_t* peer_start;  // device [npeer] first row at each destination, or null (0)
 };
 
 __device__ __forceinline__ int64_t expert_cap(const DispatchArgs& a, int e) {
@@ -334,11 +335,12 @@ __device__ __forceinline__ int64_t expert_cap(const DispatchArgs& a, int e) {
 
 // Shared memory of the dispatch kernels: base [E], tot [E], rows [E],
 // off [E+1], wcnt [DWARPS][E], slots [ROUTE_BLOCK * k], owner [ROUTE_BLOCK * k],
-// then (8-byte aligned) the destination table [MAX_PEERS].
+// then (8-byte aligned) the destination table [MAX_PEERS] and its first rows
+// [MAX_PEERS].
 __host__ __device__ inline size_t dispatch_smem_bytes(int E, int k) {
     return sizeof(int32_t) *
                ((size_t)4 * E + 1 + (size_t)DWARPS * E + (size_t)2 * ROUTE_BLOCK * k) +
-           8 + sizeof(uint4*) * MAX_PEERS;
+           8 + sizeof(uint4*) * MAX_PEERS + sizeof(int32_t) * MAX_PEERS;
 }
 
 struct DispatchSmem {
@@ -350,6 +352,7 @@ struct DispatchSmem {
     int32_t* slots;  // [ROUTE_BLOCK * k] destination row of each (token, j), -1: dropped
     int32_t* owner;  // [ROUTE_BLOCK * k] destination of each (token, j)
     uint4** peer;    // [MAX_PEERS] destination bases
+    int32_t* start;  // [MAX_PEERS] first row of this rank's rows at each destination
 };
 
 __device__ __forceinline__ DispatchSmem dispatch_smem(int32_t* sm, int E, int k) {
@@ -363,6 +366,7 @@ __device__ __forceinline__ DispatchSmem dispatch_smem(int32_t* sm, int E, int k)
     d.owner = d.slots + ROUTE_BLOCK * k;
     const uintptr_t p = reinterpret_cast<uintptr_t>(d.owner + ROUTE_BLOCK * k);
     d.peer = reinterpret_cast<uint4**>((p + 7) & ~static_cast<uintptr_t>(7));
+    d.start = reinterpret_cast<int32_t*>(d.peer + MAX_PEERS);
     return d;
 }
 
@@ -444,6 +448,7 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
         for (int i = 0; i < MAX_PEERS; ++i)
             if (i < a.npeer) d.peer[i] = a.peer[i];
     }
+    if (tid < a.npeer) d.start[tid] = a.peer_start ? a.peer_start[tid] : 0;
     const int64_t t = (int64_t)blk * ROUTE_BLOCK + tid;
     const bool valid = t < a.T;
 #pragma unroll
@@ -481,7 +486,8 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
             const int32_t row = r < nrow ? d.slots[r] : -1;
             const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
             src[q] = row >= 0 ? a.x + tok * nv : nullptr;
-            dst[q] = row >= 0 ? d.peer[d.owner[r]] + (int64_t)row * nv : nullptr;
+            dst[q] = row >= 0 ? d.peer[d.owner[r]] + (int64_t)(row + d.start[d.owner[r]]) * nv
+                              : nullptr;
         }
         for (int c = tid; c < nv; c += ROUTE_BLOCK) {
             uint4 v[G];
@@ -893,6 +899,7 @@ DispatchArgs dispatch_args(const DispatchParams& p) {
     a.x_perm = reinterpret_cast<uint4*>(p.x_perm);
     a.cap = p.cap;
     a.nsub = p.nsub > 0 ? p.nsub : 1;
+    a.peer_start = p.peer_start;
     for (int i = 0; i < MAX_PEERS; ++i) a.peer[i] = nullptr;
     if (p.npeer > 0) {
         a.npeer = p.npeer;

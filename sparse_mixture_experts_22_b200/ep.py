@@ -43,6 +43,18 @@ pass a stream-ordered barrier (the owners read only after every source has
 stored; the buffers are reused only after every source has combined):
 `forward_dist_peers` takes the buffers from torch's symmetric memory, and
 `forward_emulated_peers` runs the ranks' kernels one after another on one GPU.
+
+In the peer-memory form the plan can stay on the device (`device_plan=True`,
+the default of `forward_dist_peers`): the counts are gathered into a device
+tensor, moe_ep_plan derives every rank's caps, row offsets and received
+groups from them on the GPU, and the kernels take those offsets from device
+memory, so a step never waits for the host.  The collective form keeps the
+host plan: NCCL's all-to-all takes its split sizes on the host.
+
+`StepTimer` measures the share of a step spent in the inter-GPU dispatch
+[MoE routing fully explained, "Main insights" ¶3: the dispatch time share is
+one of the routing metrics to watch]: CUDA events around the exchange phases
+(with their barriers), against the whole step.
 """
 
 from dataclasses import dataclass, field
@@ -159,6 +171,48 @@ def peer_row_starts(plan: Plan, rank: int) -> np.ndarray:
     return plan.send[:rank].sum(axis=0).astype(np.int64)
 
 
+def device_plan(r: "Rank", counts_all: torch.Tensor, C: int) -> dict:
+    """The plan of rank r on the device (moe_ep_plan) from the gathered
+    counts [G * E] (device int32); nothing is read back to the host."""
+    G, E = r.world, r.wl.E
+    dev = counts_all.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    p = {"cap": torch.empty(E, **i32), "row_start": torch.empty(G, **i32),
+         "group_rows": torch.empty(E, **i32), "group_off": torch.empty(E, **i32),
+         "group_weight": torch.empty(E, **i32), "recv_rows": torch.empty(1, **i32)}
+    B.moe_ep_plan(r.cfg, G, r.rank, counts_all, C, p["cap"], p["row_start"], p["group_rows"],
+                  p["group_off"], p["group_weight"], p["recv_rows"])
+    return p
+
+
+class StepTimer:
+    """CUDA events around the phases of one expert-parallel step; `share()`
+    is the fraction of the step spent dispatching rows to their experts'
+    owners and bringing the outputs back (the exchanges and their barriers)."""
+
+    def __init__(self):
+        self.ev = {}
+
+    def mark(self, name: str):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.ev[name] = e
+
+    def ms(self, a: str, b: str) -> float:
+        return self.ev[a].elapsed_time(self.ev[b])
+
+    def share(self) -> dict:
+        torch.cuda.synchronize()
+        step = self.ms("start", "end")
+        xch = self.ms("dispatch0", "dispatch1") + self.ms("combine0", "combine1")
+        return {"step_ms": step, "exchange_ms": xch, "dispatch_share": xch / step if step else 0.0}
+
+
+def _mark(timer: Optional["StepTimer"], name: str):
+    if timer is not None:
+        timer.mark(name)
+
+
 def all_gather_counts(counts: torch.Tensor, world: int, group=None) -> np.ndarray:
     """Step 1's exchange: every rank's per-expert counts, [G][E]."""
     import torch.distributed as dist
@@ -237,6 +291,36 @@ class Rank:
         self.ffn_ws = ws
         return y
 
+    def dispatch_peers_dev(self, dplan: dict, recv_bases: List[int]) -> None:
+        """Step 2 with step 3 folded in, the plan on the device: this rank's
+        rows start at row dplan["row_start"][q] of rank q's receive buffer."""
+        b = self.b
+        B.moe_dispatch_peers(self.cfg, b["topk_idx"], self.x, dplan["cap"],
+                             [int(p) for p in recv_bases], b["routed"], b["kept"], b["offsets"],
+                             b["perm_token"], b["slot_of"], b["ws"],
+                             dst_row_start=dplan["row_start"])
+
+    def ffn_dev(self, dplan: dict, recv: torch.Tensor, y: torch.Tensor, bound: int) -> None:
+        """Step 4 with the received groups described on the device; `bound`
+        (host) bounds every group's rows."""
+        if recv.shape[0] == 0:
+            return
+        ws = getattr(self, "ffn_ws_dev", None)
+        need = B.moe_grouped_workspace_size(self.cfg, recv.shape[0], bound)
+        if ws is None or ws.numel() < need:
+            ws = torch.empty(need, dtype=torch.uint8, device=recv.device)
+            self.ffn_ws_dev = ws
+        B.moe_expert_ffn_grouped(self.cfg, recv, recv.shape[0], dplan["group_rows"],
+                                 dplan["group_off"], dplan["group_weight"], bound, self.W13,
+                                 self.W2p, y, ws)
+
+    def combine_peers_dev(self, dplan: dict, y_bases: List[int]) -> torch.Tensor:
+        b = self.b
+        B.moe_combine_peers(self.cfg, [int(p) for p in y_bases], b["topk_idx"], b["offsets"],
+                            b["slot_of"], b["topk_gate"], None, b["out"],
+                            y_row_start=dplan["row_start"])
+        return b["out"]
+
     def dispatch_peers(self, plan: Plan, recv_bases: List[int]) -> None:
         """Step 2 with step 3 folded in: recv_bases[q] = device address of
         rank q's receive buffer (bf16 [rows][d])."""
@@ -272,19 +356,27 @@ class Rank:
 
 # ---------------------------------------------------------------- drivers
 
-def forward_dist(r: Rank, T_all: int, group=None):
+def forward_dist(r: Rank, T_all: int, group=None, timer: Optional[StepTimer] = None):
     """One step on this rank, the exchanges as torch.distributed collectives.
     Returns (out, stats tensor, plan)."""
+    _mark(timer, "start")
     counts = all_gather_counts(r.route(), r.world, group)
     plan = make_plan(counts, T_all, r.wl.k, r.wl.E, r.wl.cf, r.pad)
-    recv = exchange_rows(r.dispatch(plan), plan, r.rank, group)
-    back = exchange_back(r.ffn(plan, recv), plan, r.rank, group)
+    send = r.dispatch(plan)
+    _mark(timer, "dispatch0")
+    recv = exchange_rows(send, plan, r.rank, group)
+    _mark(timer, "dispatch1")
+    y = r.ffn(plan, recv)
+    _mark(timer, "combine0")
+    back = exchange_back(y, plan, r.rank, group)
+    _mark(timer, "combine1")
     out = r.combine(back)
     import torch.distributed as dist
     sums = r.stats_sums()
     dist.all_reduce(sums, group=group)
     stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
     B.moe_stats_finalize(r.cfg, sums, stats)
+    _mark(timer, "end")
     return out, stats, plan
 
 
@@ -335,22 +427,68 @@ def forward_emulated_peers(ranks: List[Rank], T_all: int):
     return outs, stats, plan
 
 
-def forward_dist_peers(r: Rank, T_all: int, group=None, max_rows: Optional[int] = None):
+def forward_emulated_peers_device(ranks: List[Rank], T_all: int, max_rows: int,
+                                  timer: Optional[StepTimer] = None):
+    """The peer-memory form with the plan on the device, G ranks emulated in
+    one process on one GPU (stream order stands in for the barriers).  No
+    count or plan value is read back to the host.  Returns ([out per rank],
+    stats tensor)."""
+    G = len(ranks)
+    wl = ranks[0].wl
+    dev = ranks[0].x.device
+    _mark(timer, "start")
+    counts_all = torch.cat([r.route() for r in ranks])          # [G * E] on the device
+    C = capacity(T_all, wl.k, wl.E, wl.cf)
+    plans = [device_plan(r, counts_all, C) for r in ranks]
+    recv = [torch.empty((max_rows, wl.d), dtype=ranks[0].x.dtype, device=dev) for _ in range(G)]
+    ys = [torch.empty((max_rows, wl.d), dtype=torch.float32, device=dev) for _ in range(G)]
+    _mark(timer, "dispatch0")
+    for r, p in zip(ranks, plans):
+        r.dispatch_peers_dev(p, [t.data_ptr() for t in recv])
+    _mark(timer, "dispatch1")
+    bound = min(C, T_all)
+    for q in range(G):
+        ranks[q].ffn_dev(plans[q], recv[q], ys[q], bound)
+    _mark(timer, "combine0")
+    outs = [r.combine_peers_dev(p, [y.data_ptr() for y in ys]) for r, p in zip(ranks, plans)]
+    _mark(timer, "combine1")
+    sums = sum(r.stats_sums().clone() for r in ranks)
+    stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
+    B.moe_stats_finalize(ranks[0].cfg, sums, stats)
+    _mark(timer, "end")
+    return outs, stats, plans
+
+
+def forward_dist_peers(r: Rank, T_all: int, group=None, max_rows: Optional[int] = None,
+                       device_plan_on: bool = True, timer: Optional[StepTimer] = None):
     """One step on this rank (one process per GPU) in the peer-memory form.
     The receive and output buffers are symmetric memory (every rank maps
     every other rank's), sized for `max_rows` received rows (default: every
     token of every rank routed here, T_all * k); the barriers are symmetric
-    memory's stream-ordered barrier.  Returns (out, stats tensor, plan)."""
+    memory's stream-ordered barrier.  With device_plan_on the plan is computed
+    on the GPU (moe_ep_plan) and the step reads nothing back to the host; the
+    buffers must then hold the largest possible receive (the default size).
+    Returns (out, stats tensor, plan: the host Plan, or the device plan's
+    tensors)."""
     import torch.distributed as dist
     import torch.distributed._symmetric_memory as symm_mem
     wl = r.wl
-    counts = all_gather_counts(r.route(), r.world, group)
-    plan = make_plan(counts, T_all, wl.k, wl.E, wl.cf, r.pad)
+    _mark(timer, "start")
     rows = max_rows if max_rows is not None else T_all * wl.k + wl.E * r.pad
-    # the same test on every rank (the plan is the same), so that all of them
-    # stop together rather than leave the others at a barrier
-    if int(plan.send.sum(axis=0).max()) > rows:
-        raise ValueError("the receive buffers are smaller than this step's rows")
+    if device_plan_on:
+        if rows < T_all * wl.k + wl.E * r.pad:
+            raise ValueError("with the plan on the device the buffers hold the largest receive")
+        counts_all = torch.empty(r.world * wl.E, dtype=torch.int32, device=r.x.device)
+        dist.all_gather_into_tensor(counts_all, r.route().contiguous(), group=group)
+        C = capacity(T_all, wl.k, wl.E, wl.cf)
+        plan = device_plan(r, counts_all, C)
+    else:
+        counts = all_gather_counts(r.route(), r.world, group)
+        plan = make_plan(counts, T_all, wl.k, wl.E, wl.cf, r.pad)
+        # the same test on every rank (the plan is the same), so that all of them
+        # stop together rather than leave the others at a barrier
+        if int(plan.send.sum(axis=0).max()) > rows:
+            raise ValueError("the receive buffers are smaller than this step's rows")
     if r.symm is None:
         grp = group if group is not None else dist.group.WORLD
         recv = symm_mem.empty(rows, wl.d, dtype=r.x.dtype, device=r.x.device)
@@ -359,16 +497,30 @@ def forward_dist_peers(r: Rank, T_all: int, group=None, max_rows: Optional[int] 
     recv, yb, h_recv, h_y = r.symm
     if recv.shape[0] < rows:
         raise ValueError("max_rows is larger than the buffers allocated at the first step")
-    r.dispatch_peers(plan, list(h_recv.buffer_ptrs))
+    _mark(timer, "dispatch0")
+    if device_plan_on:
+        r.dispatch_peers_dev(plan, list(h_recv.buffer_ptrs))
+    else:
+        r.dispatch_peers(plan, list(h_recv.buffer_ptrs))
     h_recv.barrier(channel=0)            # every source has stored its rows here
-    n = int(plan.recv_rows(r.rank).sum())
-    if n:
-        r.ffn(plan, recv[:n], yb[:n])
+    _mark(timer, "dispatch1")
+    if device_plan_on:
+        r.ffn_dev(plan, recv[:rows], yb[:rows], min(C, T_all))
+    else:
+        n = int(plan.recv_rows(r.rank).sum())
+        if n:
+            r.ffn(plan, recv[:n], yb[:n])
     h_y.barrier(channel=0)               # every owner's outputs are in place
-    out = r.combine_peers(plan, list(h_y.buffer_ptrs))
+    _mark(timer, "combine0")
+    if device_plan_on:
+        out = r.combine_peers_dev(plan, list(h_y.buffer_ptrs))
+    else:
+        out = r.combine_peers(plan, list(h_y.buffer_ptrs))
     h_y.barrier(channel=1)               # every source has read: buffers free for the next step
+    _mark(timer, "combine1")
     sums = r.stats_sums()
     dist.all_reduce(sums, group=group)
     stats = torch.zeros(5, dtype=torch.float64, device=sums.device)
     B.moe_stats_finalize(r.cfg, sums, stats)
+    _mark(timer, "end")
     return out, stats, plan

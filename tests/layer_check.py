@@ -4,12 +4,16 @@ compare every output with the fp64 oracle on the same seeded inputs.
 Bars (the layer's stated tolerances):
   routing sets, counts, ranks, permutation, dropped set   bit-exact
   logits, gates                                          |err| <= 2.5e-5
-  output    max|err| <= 1e-2 * max|ref|  and  sum|err| / sum|ref| <= 2e-3, the
-            latter against the reference rounded to the output dtype
+  output    max|err| <= 1e-2 * max|ref|  and  sum|err| / sum|ref| <= 2e-3
+            against the fp64 reference itself when H reaches the down
+            projection as two bf16 parts (and for fp32 layers); with bf16 H
+            alone the relative L1 bar holds against the reference rounded to
+            the output dtype, and the unrounded figure is reported beside it
   aux loss  relative error <= 1e-5; overflow rate exact; entropy rel <= 1e-5
-The output bound follows from bf16 storage of H and of the output (unit
-roundoff 2^-8): each rounding adds a relative error of at most ~1.3e-3 in the
-L1 sense, and the gate/up and down sums accumulate in fp32.
+Why: storing the output in bf16 (unit roundoff 2^-8) alone leaves ~1.41e-3
+relative L1 against the unrounded value; rounding H to bf16 adds ~0.8e-3 more
+(2.2-2.3e-3 in all), while the two-part H (16 significant bits) adds ~1e-6.
+The gate/up and down sums accumulate in fp32.
 """
 
 import math
@@ -51,8 +55,8 @@ def host_inputs(wl: Workload) -> Dict:
     return inp
 
 
-def device_layer(wl: Workload, inp: Dict, dev="cuda"):
-    cfg = M.config_of(wl)
+def device_layer(wl: Workload, inp: Dict, dev="cuda", hidden: str = "auto"):
+    cfg = M.config_of(wl, hidden=hidden)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     W13, W2p = M.pack_weights(cfg, g["w1"], g["w3"], g["w2"])
     W13s = W2s = None
@@ -189,11 +193,19 @@ def check_offsets(wl: Workload, r: Dict, offsets: np.ndarray, pad: int):
     assert offsets[wl.E] == o
 
 
-def check_output(out_gpu: torch.Tensor, ref: np.ndarray, what: str = "out"):
-    """max|err| against the fp64 reference; mean relative error against the
-    correctly rounded result (the fp64 reference stored in the output dtype,
-    round-to-nearest-even), since the layer's output is defined as stored in
-    that dtype.  The error against the unrounded reference is returned too."""
+def strict_output(cfg) -> bool:
+    """Whether the output bar holds against the unrounded fp64 reference:
+    fp32 layers, and bf16 layers whose H reaches the down projection in two
+    parts."""
+    return cfg.act_dtype == M.MOE_F32 or M.moe_hidden_split(cfg)
+
+
+def check_output(out_gpu: torch.Tensor, ref: np.ndarray, what: str = "out",
+                 strict: bool = True):
+    """max|err| against the fp64 reference.  Mean relative error (relative L1)
+    against the unrounded fp64 reference when `strict`; always also against
+    the correctly rounded result (the fp64 reference stored in the output
+    dtype, round-to-nearest-even), which is the bar for bf16 H."""
     g = out_gpu.double().cpu().numpy()
     ref_q = torch.from_numpy(ref).to(out_gpu.dtype).double().numpy()
     err = np.abs(g - ref)
@@ -203,11 +215,14 @@ def check_output(out_gpu: torch.Tensor, ref: np.ndarray, what: str = "out"):
     floor = np.abs(ref_q - ref).sum() / max(np.abs(ref).sum(), 1e-300)
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     assert err.max() <= MAX_ERR_FRAC * scale, f"{what}: max|err| {err.max()} > 1e-2 * {scale}"
-    assert rel_l1 <= REL_L1, (f"{what}: relative L1 {rel_l1} (vs unrounded {rel_l1_raw}, "
-                              f"storage floor {floor})")
+    if strict:
+        assert rel_l1_raw <= REL_L1, (f"{what}: relative L1 {rel_l1_raw} against the unrounded "
+                                      f"reference (storage floor {floor})")
+    assert rel_l1 <= REL_L1, (f"{what}: relative L1 {rel_l1} against the rounded reference "
+                              f"(vs unrounded {rel_l1_raw}, storage floor {floor})")
     return {"max_err_frac": float(err.max() / scale) if scale > 0 else 0.0,
             "rel_l1": float(rel_l1), "rel_l1_unrounded": float(rel_l1_raw),
-            "storage_floor": float(floor)}
+            "storage_floor": float(floor), "strict": bool(strict)}
 
 
 def check_stats(r: Dict, stats: torch.Tensor, T: int):
@@ -231,3 +246,25 @@ def sample_rows(T: int, n: int, seed: int = 0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     rest = rng.choice(np.arange(1, T - 1), size=n - 2, replace=False)
     return np.sort(np.concatenate([[0, T - 1], rest]))
+
+
+def tile_rows(r: Dict, n_extra: int, T: int, seed: int = 0, tile: int = 128) -> np.ndarray:
+    """Token rows that reach every tile of every expert: for each expert with
+    kept rows, a token in each `tile`-row block of its queue (the blocks the
+    GEMMs cut it into), the tokens at the head and at the tail of its queue
+    (the ragged last tile), plus n_extra rows spread over the batch.  Built
+    from the oracle's dispatch (serving expert and queue position of every
+    kept assignment), which the GPU matches bit for bit."""
+    keep, expert, rank = r["keep"], r["expert"], r["rank"]
+    first: Dict = {}
+    last: Dict = {}
+    for t, j in zip(*np.nonzero(keep)):
+        e, q = int(expert[t, j]), int(rank[t, j])
+        key = (e, q // tile)
+        if key not in first or q < first[key][0]:
+            first[key] = (q, int(t))
+        if e not in last or q > last[e][0]:
+            last[e] = (q, int(t))
+    rows = {t for _, t in first.values()} | {t for _, t in last.values()}
+    rows |= set(sample_rows(T, n_extra, seed).tolist())
+    return np.array(sorted(rows), dtype=np.int64)

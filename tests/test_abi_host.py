@@ -125,10 +125,10 @@ def _peer_call_codes(cfg, world, ptrs):
     ws_bytes = M.moe_workspace_size(cfg)
     arr = (ctypes.c_void_p * max(len(ptrs), 1))(*[ctypes.c_void_p(p) if p else None
                                                   for p in ptrs])
-    d = lib.moe_dispatch_peers(ctypes.byref(cfg), fake, fake, fake, world, arr, fake, fake, fake,
-                               None, fake, fake, ws_bytes, None)
-    c = lib.moe_combine_peers(ctypes.byref(cfg), world, arr, fake, fake, fake, fake, None, fake,
-                              None)
+    d = lib.moe_dispatch_peers(ctypes.byref(cfg), fake, fake, fake, world, arr, None, fake, fake,
+                               fake, None, fake, fake, ws_bytes, None)
+    c = lib.moe_combine_peers(ctypes.byref(cfg), world, arr, None, fake, fake, fake, fake, None,
+                              fake, None)
     return d, c
 
 
@@ -145,6 +145,22 @@ def test_peer_calls_check_their_arguments(kw, world, ptrs, code):
     d, c = _peer_call_codes(cfg, world, ptrs)
     assert d == code, B.load().moe_last_error()
     assert c == code, B.load().moe_last_error()
+
+
+@pytest.mark.parametrize("world,rank,C,code", [
+    (0, 0, 10, 1),     # no ranks
+    (65, 0, 10, 1),    # above MOE_MAX_PEERS
+    (3, 0, 10, 2),     # 8 experts over 3 ranks
+    (2, 2, 10, 1),     # rank out of range
+    (2, -1, 10, 1),
+    (2, 0, -1, 1),     # negative capacity
+])
+def test_ep_plan_checks_its_arguments(world, rank, C, code):
+    cfg = M.make_config(64, 128, 128, 8, 2)
+    fake = ctypes.c_void_p(0x100000)
+    rc = B.load().moe_ep_plan(ctypes.byref(cfg), world, rank, fake, C, fake, fake, fake, fake,
+                              fake, fake, None)
+    assert rc == code, B.load().moe_last_error()
 
 
 def test_peer_dispatch_is_bf16_only():

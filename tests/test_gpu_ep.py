@@ -15,7 +15,7 @@ import torch
 
 import oracle as O
 import sparse_mixture_experts_22_b200 as M
-from layer_check import check_output, check_stats, host_inputs
+from layer_check import check_output, check_stats, host_inputs, strict_output
 from sparse_mixture_experts_22_b200 import ep
 from sparse_mixture_experts_22_b200.workloads import Workload
 
@@ -78,7 +78,7 @@ def test_emulated_ranks_match_the_layer_on_the_concatenated_batch(name):
     np.testing.assert_array_equal(plan.kept.sum(0), ref["kept"])
     if wl.cf is not None and name != "g1":
         assert ref["kept"].sum() < wl.T * wl.k, "the case should drop some assignments"
-    check_output(out, ref["out"], name)
+    check_output(out, ref["out"], name, strict=strict_output(ranks[0].cfg))
     check_stats(ref, stats, wl.T)
 
 
@@ -111,7 +111,70 @@ def test_peer_stores_and_loads_give_the_exchange_path_bit_for_bit(name):
     assert torch.equal(out_p, out_x)
     assert torch.equal(stats_p, stats_x)
     ref = O.forward(O.cfg_of(wl), inp)
-    check_output(out_p, ref["out"], name)
+    check_output(out_p, ref["out"], name, strict=strict_output(ranks[0].cfg))
+
+
+def _ranks(wl, G, inp):
+    dev = torch.device("cuda")
+    cfg = M.config_of(wl)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    W13, W2p = M.pack_weights(cfg, g["w1"], g["w3"], g["w2"])
+    T_loc, E_loc = wl.T // G, wl.E // G
+    return [ep.Rank(wl, r, G, g["x"][r * T_loc:(r + 1) * T_loc].contiguous(), g["Wr"],
+                    g["bias"], W13[r * E_loc:(r + 1) * E_loc], W2p[r * E_loc:(r + 1) * E_loc])
+            for r in range(G)]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_device_plan_equals_the_host_plan(name):
+    """moe_ep_plan on the gathered counts gives every rank exactly the host
+    plan: its caps, where its rows start at each owner, and the groups it
+    receives (rows, first row, expert) with their total."""
+    wl, G = CASES[name]
+    inp = host_inputs(wl)
+    ranks = _ranks(wl, G, inp)
+    counts = [r.route().clone() for r in ranks]
+    host = ep.make_plan(np.stack([c.cpu().numpy() for c in counts]).astype(np.int64), wl.T, wl.k,
+                        wl.E, wl.cf, ranks[0].pad)
+    counts_all = torch.cat(counts)
+    C = ep.capacity(wl.T, wl.k, wl.E, wl.cf)
+    for r in ranks:
+        d = ep.device_plan(r, counts_all, C)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(d["cap"].cpu().numpy(),
+                                      host.cap[r.rank].clip(max=2 ** 31 - 1))
+        np.testing.assert_array_equal(d["row_start"].cpu().numpy(),
+                                      ep.peer_row_starts(host, r.rank))
+        rows, off, wi = host.groups(r.rank)
+        np.testing.assert_array_equal(d["group_rows"].cpu().numpy(), rows)
+        np.testing.assert_array_equal(d["group_off"].cpu().numpy(), off)
+        np.testing.assert_array_equal(d["group_weight"].cpu().numpy(), wi)
+        assert int(d["recv_rows"].item()) == int(host.recv_rows(r.rank).sum())
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_device_plan_step_matches_the_host_plan_step(name):
+    """The peer-memory step with the plan on the device (nothing read back to
+    the host) gives the host-planned step's output and statistics bit for
+    bit."""
+    wl, G = CASES[name]
+    inp = host_inputs(wl)
+    _, out_h, stats_h, _ = run_emulated_peers(wl, G, inp)
+    ranks = _ranks(wl, G, inp)
+    pad = ranks[0].pad
+    timer = ep.StepTimer()
+    outs, stats_d, _ = ep.forward_emulated_peers_device(ranks, wl.T, wl.T * wl.k + wl.E * pad,
+                                                        timer=timer)
+    torch.cuda.synchronize()
+    m4 = timer.share()
+    assert 0.0 < m4["dispatch_share"] < 1.0, m4
+    print(f"{name}: dispatch-time share {m4}")
+    for r in ranks:
+        assert M.moe_read_device_status(r.b["ws"]) == 0
+        assert M.moe_read_device_status(r.ffn_ws_dev) == 0
+    out_d = torch.cat([o.clone() for o in outs])
+    assert torch.equal(out_d, out_h)
+    assert torch.equal(stats_d, stats_h)
 
 
 def test_grouped_ffn_flags_an_oversized_group():

@@ -1,8 +1,10 @@
 """moe_route_static: routing for callers that cannot allocate device memory
 (a workspace-free variant of moe_route whose scratch is a fixed device array
 inside the library).  Called through the C ABI, it must give what moe_route
-gives on the same batch, on two calls in a row with different batches (so a
-stale result left in the shared array would be caught).
+gives on the same batch, and what the fp64 oracle's routing gives (the same
+expert sets, gates within the parity tests' bound), on two calls in a row with
+different batches (so a stale result left in the shared array would be
+caught).
 
 This file is collected last on purpose; it runs alone as well.
 """
@@ -12,6 +14,8 @@ import ctypes
 import numpy as np
 import pytest
 import torch
+
+import oracle as O
 
 from sparse_mixture_experts_22_b200 import binding as B
 from sparse_mixture_experts_22_b200 import inputs as I
@@ -67,6 +71,7 @@ def test_static_route_matches_workspace_route_twice(wl):
     for call in range(2):
         x, _ = I.tokens(wl, Wr=Wr.cpu(), b=bias.cpu() if bias is not None else None,
                         stream=f"x.static{call}")
+        x_host = x.clone()
         x = x.cuda()
         idx_s, gate_s = _route_static(fn, cfg, x, Wr, bias)
         idx_w, gate_w = _route_with_workspace(cfg, x, Wr, bias)
@@ -74,6 +79,15 @@ def test_static_route_matches_workspace_route_twice(wl):
         assert torch.equal(idx_s, idx_w), f"call {call}: top-k differs"
         err = (gate_s - gate_w).abs().max().item()
         assert err <= GATE_ABS, f"call {call}: gates differ by {err}"
+        # against the fp64 oracle: expert sets bit-exact, gates per (token, expert)
+        r = O.route(O.cfg_of(wl), x_host, Wr.cpu(), bias.cpu() if bias is not None else None)
+        idx = idx_s.cpu().numpy()
+        gate = gate_s.cpu().numpy()
+        assert np.array_equal(np.sort(idx, 1), np.sort(r["idx"], 1)), f"call {call}: sets"
+        g_gpu = np.take_along_axis(gate, np.argsort(idx, 1), 1)
+        g_ref = np.take_along_axis(r["gate"], np.argsort(r["idx"], 1), 1)
+        oerr = np.abs(g_gpu - g_ref).max()
+        assert oerr <= GATE_ABS, f"call {call}: gates off the oracle by {oerr}"
 
 
 def test_static_route_rejects_oversized_batches():
