@@ -161,6 +161,21 @@ def kernel_work(name, wl, kept, splits):
     return None
 
 
+def tile_stats(wl, kept, sms):
+    """Token-major tile bookkeeping from the run's kept counts: the rows the
+    128- and 256-row m tiles cover over the kept rows (padding), and the
+    gate/up work units (m tiles x 128-wide hidden blocks) in waves of the SMs
+    (one tile per SM, or per SM pair for 256-row tiles)."""
+    N = max(int(sum(kept)), 1)
+    out = {}
+    for m, per in ((128, 1), (256, 2)):
+        tiles = sum(-(-int(n) // m) for n in kept if n > 0)
+        units = tiles * (wl.h // 128)
+        out[f"m{m}"] = {"m_tiles": tiles, "padded_rows_frac": tiles * m / N,
+                        "gateup_units": units, "waves": units / (sms // per)}
+    return out
+
+
 def dominant_roofline(trace, wl, cfg, kept):
     """Roofline of the dominant GEMM among the traced kernels: its algorithmic
     work per launch over its mean CUDA-event duration, against the measured
@@ -717,6 +732,7 @@ def main():
         "layer_roofline": {"flops": flops, "bytes": byts, "time_us": roof_t * 1e6,
                            "frac": roof_t / t_step, "kept_assignments": N,
                            "active_experts": active, "peaks": "bf16 burst, HBM copy"},
+        "tiles": tile_stats(wl, kept, torch.cuda.get_device_properties(dev).multi_processor_count),
         "kernels": kernels,
         "gpu_launches": launched,
         "clocks": clk,

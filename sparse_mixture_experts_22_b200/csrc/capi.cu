@@ -623,6 +623,37 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     // groups of more than 128 (and at most 256) tokens: swapped tiles on CTA
     // pairs, each SM staging half of the token rows
     const bool pair = !tok && g_pair_enabled && nt_max > DOWN_SWAP_MAX_TOKENS;
+    // groups that may hold thousands of tokens: token-major tiles of 256 tokens on
+    // CTA pairs (a third less shared-memory fill per flop; the 256-row tiles pad
+    // an expert's rows more than 128-row tiles, which pays off for large groups)
+    const bool pair_tok = tok && g_pair_enabled && nt_max >= PAIR_TOK_MIN_TOKENS &&
+                          hid % 128 == 0 && P.d % 256 == 0;
+    if (pair_tok) {
+        MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 128));
+        MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 128));
+        a.stages = tc_pair_max_stages(TC_PAIR_GATEUP_TOK, nt_max, groups, false, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP_TOK, m_act, m_w, a, st), tag1));
+        trace_mark(st, tag1);
+        MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 128));
+        MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
+        a.K = hid;
+        a.n_feat = P.d;
+        a.w_rows_per_group = P.d;
+        a.splits = 1;
+        a.out = y;
+        a.out_ld = P.d;
+        a.split_stride = act_rows * (int64_t)P.d;
+        a.aux = nullptr;
+        a.prefetch_kb = 0;
+        a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, nt_max, groups, P.split, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag2);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, st), tag2));
+        trace_mark(st, tag2);
+        return MOE_OK;
+    }
     if (pair) {
         MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 8));
         MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 64));

@@ -26,6 +26,15 @@
 //             and receives y for them; with H in two bf16 parts a second
 //             MMA per K step adds H_lo.
 //
+// The same pairing serves experts with thousands of tokens (token-major
+// tiles, the large prefill layer): M = 256 tokens, 128 rows in each CTA, and
+// N = 256 weight rows, 128 in each CTA -- for gate/up CTA 0 stages the 128
+// gate rows of a hidden block and CTA 1 their up rows, so that each CTA's
+// accumulator holds [gate | up] for its own 128 tokens, as the one-SM tile
+// does.  Each SM then stages 32 KB per K step for a 256 x 256 x 64 MMA
+// instead of 48 KB for 128 x 256 x 64: a third less shared-memory fill (L2
+// traffic) per flop.
+//
 // Roles (each CTA, 10 warps): warp 0 loads this CTA's halves with TMA into
 // its own stages (own barriers; no multicast); in the even CTA warp 1 issues
 // the pair MMAs once both CTAs' stages are full, in the odd CTA warp 1
@@ -50,9 +59,16 @@ namespace {
 constexpr int PBM = 128;   // weight rows per CTA (accumulator lanes)
 constexpr int PBK = 64;    // K per stage: one 128-byte swizzle row of bf16
 constexpr int PUK = 16;    // K per MMA
-constexpr int PEPI = 8;    // epilogue warps
-constexpr int PTHREADS = 64 + 32 * PEPI;
 constexpr uint64_t P_TEARDOWN_NS = 200000000ull;
+constexpr int P_STG_LD = 36;  // fp32 staging row (32 values + 4 of padding)
+
+__host__ __device__ constexpr bool p_tok(int mode) {
+    return mode == TC_PAIR_GATEUP_TOK || mode == TC_PAIR_DOWN_TOK;
+}
+// epilogue warps: two per TMEM lane quarter on swapped tiles (splitting the
+// token columns), one per quarter on token-major tiles
+__host__ __device__ constexpr int p_epi(int mode) { return p_tok(mode) ? 4 : 8; }
+__host__ __device__ constexpr int p_threads(int mode) { return 64 + 32 * p_epi(mode); }
 
 __host__ __device__ inline uint32_t p_align(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
@@ -60,20 +76,32 @@ struct PairLayout {
     uint32_t a_bytes, b_bytes, b_lo, stage_bytes, xch_off, flag_off, bar_off, grp_off, total;
 };
 
-// Shared memory of one CTA.  B holds nt_max / 2 token rows (the high parts of
-// H, then as many low parts when split).  The gate/up exchange buffers: per
-// pair of epilogue warps two directions x two chunks x 32 lanes x 8 floats.
+// Shared memory of one CTA.  Swapped: A = 128 weight rows, B = nt_max / 2
+// token rows (the high parts of H, then as many low parts when split).
+// Token-major: A = 128 token rows (then their low parts when split), B = 128
+// weight rows.  Then the gate/up exchange buffers of the swapped epilogue (per
+// pair of warps two directions x two chunks x 32 lanes x 8 floats) or the
+// fp32 staging of the token-major down epilogue (32 x 36 floats per warp).
 __host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stages, int groups,
                                                   bool split) {
     PairLayout L;
-    L.a_bytes = PBM * PBK * 2;
-    L.b_lo = (uint32_t)(nt_max / 2) * PBK * 2;
-    L.b_bytes = p_align(L.b_lo * (split ? 2u : 1u), 1024);
+    const uint32_t parts = split ? 2u : 1u;
+    if (p_tok(mode)) {
+        L.a_bytes = PBM * PBK * 2 * (mode == TC_PAIR_DOWN_TOK ? parts : 1u);
+        L.b_lo = 0;
+        L.b_bytes = PBM * PBK * 2;
+    } else {
+        L.a_bytes = PBM * PBK * 2;
+        L.b_lo = (uint32_t)(nt_max / 2) * PBK * 2;
+        L.b_bytes = p_align(L.b_lo * parts, 1024);
+    }
     L.stage_bytes = L.a_bytes + L.b_bytes;
     L.xch_off = L.stage_bytes * stages;
-    const uint32_t xch = mode == TC_PAIR_GATEUP ? (PEPI / 2) * 2 * 2 * 32 * 8 * 4 : 0;
+    uint32_t xch = 0;
+    if (mode == TC_PAIR_GATEUP) xch = (p_epi(mode) / 2) * 2 * 2 * 32 * 8 * 4;
+    if (mode == TC_PAIR_DOWN_TOK) xch = p_epi(mode) * 32 * P_STG_LD * 4;
     L.flag_off = L.xch_off + xch;
-    L.bar_off = p_align(L.flag_off + PEPI * 2 * 4, 16);
+    L.bar_off = p_align(L.flag_off + p_epi(mode) * 2 * 4, 16);
     // full[S], relay[S], empty[S], acc_full[2], acc_empty[2], drain, tmem slot
     L.grp_off = L.bar_off + p_align((3 * stages + 5) * 8 + 8, 16);
     L.total = L.grp_off + (4 * groups + 1) * 4 + 1024;
@@ -81,7 +109,7 @@ __host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stag
 }
 
 struct PUnit {
-    int g, w, rows, row0, nb, ntok;
+    int g, w, rows, row0, nb, mt, ntok;
 };
 
 struct PGroups {
@@ -92,6 +120,7 @@ struct PGroups {
     int groups;
 };
 
+template <int MODE>
 __device__ __forceinline__ PUnit p_decode(const PGroups& t, int u) {
     int lo = 0, hi = t.groups - 1;
     while (lo < hi) {
@@ -103,22 +132,56 @@ __device__ __forceinline__ PUnit p_decode(const PGroups& t, int u) {
     x.w = t.wi[lo];
     x.rows = t.rows[lo];
     x.row0 = t.off[lo];
-    x.nb = u - t.start[lo];
-    x.ntok = (x.rows + 15) & ~15;
+    const int local = u - t.start[lo];
+    if (p_tok(MODE)) {
+        // m tile fastest: the units after one another share the weight tile
+        const int mtiles = (x.rows + 255) / 256;
+        x.mt = local % mtiles;
+        x.nb = local / mtiles;
+        x.ntok = 256;
+    } else {
+        x.mt = 0;
+        x.nb = local;
+        x.ntok = (x.rows + 15) & ~15;
+    }
     return x;
 }
 
+// Stores 32 fp32 columns of the warp's 32 rows through the warp's staging
+// buffer so that every store is a whole 128-byte row segment; rows at or
+// past `valid` are skipped.
+__device__ __forceinline__ void p_store_rows_f32x32(float* stg, const float* v, int lane,
+                                                    float* dst_row0, int64_t ld, int valid) {
+    float4* srow = reinterpret_cast<float4*>(stg + lane * P_STG_LD);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        srow[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    __syncwarp();
+    const int sub = lane >> 3, col = (lane & 7) * 4;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + sub;
+        if (r < valid)
+            *reinterpret_cast<float4*>(dst_row0 + r * ld + col) =
+                *reinterpret_cast<const float4*>(stg + r * P_STG_LD + col);
+    }
+    __syncwarp();
+}
+
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     tc_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
     constexpr bool GU = MODE == TC_PAIR_GATEUP;
+    constexpr bool TOK = p_tok(MODE);
+    constexpr int NEPI = p_epi(MODE);
+    constexpr bool DOWN = MODE == TC_PAIR_DOWN || MODE == TC_PAIR_DOWN_TOK;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (p_align(raw, 1024) - raw);
 
     const int groups = args.num_groups;
-    const bool split = !GU && args.lo_rows != 0;
+    const bool split = DOWN && args.lo_rows != 0;
     const int S = args.stages;
     const PairLayout L = pair_layout(MODE, args.nt_max, S, groups, split);
 
@@ -141,8 +204,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
 
-    // accumulator: 128 lanes x nt_max columns, twice when it fits
-    const int acc_stride = args.nt_max;
+    // accumulator: 128 lanes x nt_max (token-major: 256) columns, twice when it fits
+    const int acc_stride = TOK ? 256 : args.nt_max;
     const int n_acc = 2 * acc_stride <= 512 ? 2 : 1;
     uint32_t tmem_cols = 32;
     while (tmem_cols < (uint32_t)(acc_stride * n_acc)) tmem_cols <<= 1;
@@ -155,7 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 2 * PEPI);  // one arrive per epilogue warp of each CTA
+            mbar_init(&acc_empty[i], 2 * NEPI);  // one arrive per epilogue warp of each CTA
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -172,7 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         int acc = 0;
         for (int g = 0; g < groups; ++g) {
             int r = args.group_rows ? args.group_rows[g] : args.dense_rows;
-            if (r > args.nt_max) {
+            if (!TOK && r > args.nt_max) {
                 // a tile holds at most nt_max token columns: clamp and flag
                 if (args.status) atomicCAS(args.status, DEV_OK, DEV_SHAPE);
                 r = args.nt_max;
@@ -181,7 +244,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
             g_off[g] = args.group_off ? args.group_off[g] : 0;
             g_wi[g] = args.group_w ? args.group_w[g] : g;
             g_start[g] = acc;
-            acc += r > 0 ? args.n_feat / (GU ? 128 : 256) : 0;
+            const int per = args.n_feat / (GU || MODE == TC_PAIR_GATEUP_TOK ? 128 : 256);
+            acc += r > 0 ? per * (TOK ? (r + 255) / 256 : 1) : 0;
         }
         g_start[groups] = acc;
     }
@@ -200,15 +264,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         if (lane == 0) {
             const uint64_t pol_w = l2_policy_evict_first();
             const uint64_t pol_a = l2_policy_evict_last();
+            (void)pol_a;
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_par = 0;
             bool ok = true;
             const int kblocks = args.K / PBK;
             for (int u = pair; u < total && ok; u += npairs) {
-                const PUnit x = p_decode(tab, u);
+                const PUnit x = p_decode<MODE>(tab, u);
                 const int half = x.ntok / 2;          // token rows this CTA stages
-                const int trow = x.row0 + (int)v * half;
+                const int trow = TOK ? x.row0 + x.mt * 256 + (int)v * PBM : x.row0 + (int)v * half;
                 const uint32_t bytes =
                     (uint32_t)PBM * PBK * 2 + (uint32_t)half * PBK * 2 * (split ? 2u : 1u);
                 for (int kb = 0; kb < kblocks; ++kb) {
@@ -221,7 +286,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
                     uint8_t* sb = sa + L.a_bytes;
                     const int kc = kb * PBK;
                     mbar_arrive_expect_tx(&full[stage], bytes);
-                    if (GU) {
+                    if (TOK) {
+                        // A: this CTA's 128 token rows (then their low parts); B: the
+                        // weight rows of this CTA's half of N (gate/up: CTA 0 the gate
+                        // rows of the hidden block, CTA 1 its up rows)
+                        tma_load_2d(sa, &tm_act, &full[stage], kc, trow);
+                        if (split)
+                            tma_load_2d(sa + PBM * PBK * 2, &tm_act, &full[stage], kc,
+                                        trow + (int)args.lo_rows);
+                        tma_load_2d(sb, &tm_w, &full[stage], kc,
+                                    x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM);
+                    } else if (GU) {
                         // gate rows of features 64v.., then their up rows
                         const int wrow = x.w * args.w_rows_per_group + x.nb * 256 + (int)v * 64;
                         tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
@@ -231,13 +306,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
                         const int wrow = x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM;
                         tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
                     }
-                    for (int r = 0; r < half; r += 8)
-                        tma_load_2d_hint(sb + r * PBK * 2, &tm_act, &full[stage], kc, trow + r,
-                                         pol_a);
-                    if (split)  // the low parts of H behind the high ones
+                    if (!TOK) {
                         for (int r = 0; r < half; r += 8)
-                            tma_load_2d_hint(sb + L.b_lo + r * PBK * 2, &tm_act, &full[stage], kc,
-                                             trow + r + (int)args.lo_rows, pol_a);
+                            tma_load_2d_hint(sb + r * PBK * 2, &tm_act, &full[stage], kc,
+                                             trow + r, pol_a);
+                        if (split)  // the low parts of H behind the high ones
+                            for (int r = 0; r < half; r += 8)
+                                tma_load_2d_hint(sb + L.b_lo + r * PBK * 2, &tm_act, &full[stage],
+                                                 kc, trow + r + (int)args.lo_rows, pol_a);
+                    }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == S) {
@@ -281,7 +358,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
             bool ok = true;
             const int kblocks = args.K / PBK;
             for (int u = pair; u < total && ok; u += npairs) {
-                const PUnit x = p_decode(tab, u);
+                const PUnit x = p_decode<MODE>(tab, u);
                 if (!mbar_wait_cl(&acc_empty[acc], acc_phase ^ 1, limit)) {
                     report_timeout(args.status);
                     break;
@@ -302,9 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < PBK / PUK; ++kk) {
                         const uint64_t adesc = sdesc_kmajor_sw128(sa + kk * PUK * 2);
-                        umma_bf16_pair(d_tmem, adesc, sdesc_kmajor_sw128(sb + kk * PUK * 2), idesc,
-                                       (kb > 0 || kk > 0) ? 1u : 0u);
-                        if (split)  // + W . H_lo
+                        const uint64_t bdesc = sdesc_kmajor_sw128(sb + kk * PUK * 2);
+                        umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        if (split && TOK)  // + H_lo . W
+                            umma_bf16_pair(d_tmem,
+                                           sdesc_kmajor_sw128(sa + PBM * PBK * 2 + kk * PUK * 2),
+                                           bdesc, idesc, 1u);
+                        if (split && !TOK)  // + W . H_lo
                             umma_bf16_pair(d_tmem, adesc,
                                            sdesc_kmajor_sw128(sb + L.b_lo + kk * PUK * 2), idesc,
                                            1u);
@@ -330,7 +411,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        const int ew = warp - 2;                 // 0..7
+        const int ew = warp - 2;                 // 0..NEPI-1
         const int q = warp & 3;                  // TMEM lane quarter this warp may access
         const int part = ew >> 2;                // which half of the columns
         const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -344,7 +425,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         uint32_t acc_phase = 0;
         int it = 0;
         for (int u = pair; u < total; u += npairs, ++it) {
-            const PUnit x = p_decode(tab, u);
+            const PUnit x = p_decode<MODE>(tab, u);
             bool ok = mbar_wait(&acc_full[acc], acc_phase, limit);
             if (GU) {
                 // both warps of a pair go on only if both saw the accumulator
@@ -359,7 +440,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
             }
             tc_fence_after();
             const uint32_t t0 = lane_addr + acc * acc_stride;
-            if (GU) {
+            if (MODE == TC_PAIR_GATEUP_TOK) {
+                // [gate | up] of this CTA's 128 tokens: H = silu(gate) * up
+                const int r = x.mt * 256 + (int)v * PBM + q * 32 + lane;
+                const bool valid = r < x.rows;
+                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
+                                     (int64_t)(x.row0 + r) * args.out_ld + x.nb * 128;
+                __nv_bfloat16* abrow =
+                    args.aux ? reinterpret_cast<__nv_bfloat16*>(args.aux) +
+                                   (int64_t)(x.row0 + r) * args.aux_ld + x.nb * 256
+                             : nullptr;
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 16) {
+                    float g[16], up[16];
+                    tmem_ld16(t0 + c, g);
+                    tmem_ld16(t0 + 128 + c, up);
+                    tmem_ld_wait();
+                    if (valid && abrow) {
+                        store_bf16x16(abrow + c, g);
+                        store_bf16x16(abrow + 128 + c, up);
+                    }
+                    if (valid) {
+                        float hv[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) hv[i] = silu_f(g[i]) * up[i];
+                        if (args.lo_rows) {
+                            float lo[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) lo[i] = hv[i] - bf16_round(hv[i]);
+                            store_bf16x16(dst + args.lo_rows * args.out_ld + c, lo);
+                        }
+                        store_bf16x16(dst + c, hv);
+                    }
+                }
+            } else if (MODE == TC_PAIR_DOWN_TOK) {
+                const int r0 = x.mt * 256 + (int)v * PBM + q * 32;  // this warp's first row
+                const int valid = min(32, x.rows - r0);
+                float* dst0 = reinterpret_cast<float*>(args.out) +
+                              (int64_t)(x.row0 + r0) * args.out_ld + x.nb * 256;
+                float* stg = reinterpret_cast<float*>(smem + L.xch_off) + ew * (32 * P_STG_LD);
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 32) {
+                    float val[32];
+                    tmem_ld16(t0 + c, val);
+                    tmem_ld16(t0 + c + 16, val + 16);
+                    tmem_ld_wait();
+                    if (valid > 0)
+                        p_store_rows_f32x32(stg, val, lane, dst0 + c, args.out_ld, valid);
+                }
+            } else if (GU) {
                 // feature of this lane and its H column
                 const int f = x.nb * 128 + (int)v * 64 + (q & 1) * 32 + lane;
                 __nv_bfloat16* hdst =
@@ -448,17 +577,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
 int pair_grid(const void* kern, uint32_t smem, int mode) {
     constexpr int kMaxDevices = 64;
     static std::mutex mu;
-    static int cached[kMaxDevices][2] = {};
-    static uint32_t cached_smem[kMaxDevices][2] = {};
+    static int cached[kMaxDevices][4] = {};
+    static uint32_t cached_smem[kMaxDevices][4] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-    const int m = mode == TC_PAIR_GATEUP ? 0 : 1;
+    const int m = mode - TC_PAIR_GATEUP;
     std::lock_guard<std::mutex> lk(mu);
     if (cached[dev][m] == 0 || cached_smem[dev][m] != smem) {
         // the cluster shape comes from the kernel's __cluster_dims__
         cudaLaunchConfig_t c = {};
         c.gridDim = dim3(2);
-        c.blockDim = dim3(PTHREADS);
+        c.blockDim = dim3(p_threads(mode));
         c.dynamicSmemBytes = smem;
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, kern, &c) != cudaSuccess || n < 1) return 0;
@@ -471,8 +600,9 @@ int pair_grid(const void* kern, uint32_t smem, int mode) {
 template <int MODE>
 int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
                      cudaStream_t st) {
-    const PairLayout L = pair_layout(MODE, a.nt_max, a.stages, a.num_groups,
-                                     MODE == TC_PAIR_DOWN && a.lo_rows != 0);
+    const PairLayout L =
+        pair_layout(MODE, a.nt_max, a.stages, a.num_groups,
+                    (MODE == TC_PAIR_DOWN || MODE == TC_PAIR_DOWN_TOK) && a.lo_rows != 0);
     auto kern = tc_pair_kernel<MODE>;
     constexpr int kMaxDevices = 64;
     static std::mutex mu;
@@ -494,7 +624,7 @@ int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs&
         return -1;
     }
     // the cluster shape is part of the kernel (__cluster_dims__)
-    launch_ex(pdl_active(), kern, dim3(2 * pairs), dim3(PTHREADS), L.total, st, act, w, a);
+    launch_ex(pdl_active(), kern, dim3(2 * pairs), dim3(p_threads(MODE)), L.total, st, act, w, a);
     note_launch();
     return launch_result();
 }
@@ -502,21 +632,24 @@ int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs&
 }  // namespace
 
 int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_limit) {
+    const bool ds = (mode == TC_PAIR_DOWN || mode == TC_PAIR_DOWN_TOK) && split;
     for (int s = 8; s >= 2; --s)
-        if ((int)pair_layout(mode, nt_max, s, groups, mode == TC_PAIR_DOWN && split).total <=
-            smem_limit)
-            return s;
+        if ((int)pair_layout(mode, nt_max, s, groups, ds).total <= smem_limit) return s;
     return 0;
 }
 
 int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
                    cudaStream_t st) {
-    if (a.nt_max < 16 || a.nt_max > 256 || a.nt_max % 16) return -1;
+    if (!p_tok(mode) && (a.nt_max < 16 || a.nt_max > 256 || a.nt_max % 16)) return -1;
     switch (mode) {
         case TC_PAIR_GATEUP:
             return launch_pair_mode<TC_PAIR_GATEUP>(act, w, a, st);
         case TC_PAIR_DOWN:
             return launch_pair_mode<TC_PAIR_DOWN>(act, w, a, st);
+        case TC_PAIR_GATEUP_TOK:
+            return launch_pair_mode<TC_PAIR_GATEUP_TOK>(act, w, a, st);
+        case TC_PAIR_DOWN_TOK:
+            return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, a, st);
     }
     return -1;
 }

@@ -131,6 +131,8 @@ enum TcMode : int {
     TC_WGRAD = 5,        // backward: C[g] = A[:, K_g] B[:, K_g]^T over each group's token range
     TC_PAIR_GATEUP = 6,  // gate/up on CTA pairs: 2 x (64 gate + 64 up weight rows) x the tokens
     TC_PAIR_DOWN = 7,    // down on CTA pairs: 2 x 128 weight rows x the tokens (fp32 out)
+    TC_PAIR_GATEUP_TOK = 8,  // gate/up on CTA pairs, token-major: 2 x 128 tokens x 256
+    TC_PAIR_DOWN_TOK = 9,    // down on CTA pairs, token-major: 2 x 128 tokens x 256 (fp32 out)
 };
 
 struct TcArgs {
@@ -172,11 +174,13 @@ int tc_max_stages(int mode, int bn, int nt_max, int groups, bool split, int smem
 int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& w,
                    const TcArgs& a, int grid, cudaStream_t st);
 
-// Swapped tiles on CTA pairs (clusters of two; gemm_pair.cu), for groups of up to
-// 256 tokens: TC_PAIR_GATEUP (act = x rows, 8-row boxes; w = W13, 64-row boxes;
-// n_feat = hidden width) and TC_PAIR_DOWN (act = H rows, 8-row boxes; w = W2p,
-// 128-row boxes; n_feat = model width, a multiple of 256).  nt_max is a multiple
-// of 16 in [16, 256]; the grid is as many pairs as the device holds at once.
+// Tiles on CTA pairs (clusters of two; gemm_pair.cu).  Swapped, for groups of up
+// to 256 tokens: TC_PAIR_GATEUP (act = x rows, 8-row boxes; w = W13, 64-row
+// boxes; n_feat = hidden width) and TC_PAIR_DOWN (act = H rows, 8-row boxes;
+// w = W2p, 128-row boxes; n_feat = model width, a multiple of 256); nt_max is a
+// multiple of 16 in [16, 256].  Token-major, for groups of any size:
+// TC_PAIR_GATEUP_TOK and TC_PAIR_DOWN_TOK (act and w both 128-row boxes).  The
+// grid is as many pairs as the device holds at once.
 int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_limit);
 int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
                    cudaStream_t st);

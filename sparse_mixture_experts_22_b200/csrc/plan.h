@@ -33,6 +33,7 @@ constexpr int MAX_K = 8;
 constexpr int MAX_PEERS = 64;     // expert-parallel ranks one dispatch or combine addresses
 constexpr int SWAP_MAX_TOKENS = 256;  // largest per-expert token count the swap path covers
 constexpr int DOWN_SWAP_MAX_TOKENS = 128;  // above this the down projection takes token-major tiles
+constexpr int PAIR_TOK_MIN_TOKENS = 1024;  // token-major tiles on CTA pairs from this group bound on
 
 struct Plan {
     int64_t T;

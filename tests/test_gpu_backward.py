@@ -28,7 +28,7 @@ import torch
 
 import oracle as O
 import sparse_mixture_experts_22_b200 as M
-from layer_check import host_inputs, oracle_route
+from layer_check import host_inputs, oracle_route, tile_rows
 from sparse_mixture_experts_22_b200 import inputs as I
 from sparse_mixture_experts_22_b200.workloads import WORKLOADS, Workload
 
@@ -185,6 +185,9 @@ FULL_ROWS = 6
 
 @pytest.mark.parametrize("name", ["decode", "prefill", "deepseek", "large"])
 def test_backward_full_size_sampled(name):
+    """dx and dz on rows that reach every 128-row tile of every expert's queue
+    (plus a few random ones), and a block of dw1, dw3, dw2 of every expert
+    that kept tokens (and of the shared expert), against the oracle."""
     wl = WORKLOADS[name]
     inp = host_inputs(wl)
     G = I.grad_out(wl)
@@ -192,18 +195,18 @@ def test_backward_full_size_sampled(name):
     r = oracle_route(wl, inp)
     ocfg = O.cfg_of(wl)
     rng = np.random.default_rng(5)
-    rows = np.sort(rng.choice(wl.T, size=min(FULL_ROWS, wl.T), replace=False))
+    rows = tile_rows(r, FULL_ROWS, wl.T, seed=5)
     ref = O.backward_rows(ocfg, inp, r, G, AUX_COEF, rows)
     report = {}
     check("dx rows", grads["dx"][torch.from_numpy(rows).cuda()].double().cpu().numpy(),
           ref["dx"], report)
     check("dz rows", grads["dlogits"][torch.from_numpy(rows).cuda()].double().cpu().numpy(),
           ref["dz"], report)
-    # weight-gradient blocks of the busiest and the least busy expert
+    # a weight-gradient block of every expert that kept tokens
     kept = r["kept"]
     hi = sorted(rng.choice(wl.h, size=8, replace=False).tolist())
     ci = sorted(rng.choice(wl.d, size=16, replace=False).tolist())
-    for e in {int(np.argmax(kept)), int(np.argmin(kept))}:
+    for e in [int(e) for e in np.nonzero(kept)[0]]:
         b = O.wgrad_block(ocfg, inp, r, G, e, hi, ci)
         W13 = grads["dW13"][e]
         rows1 = [256 * (i // 128) + i % 128 for i in hi]

@@ -78,6 +78,9 @@ SMALL = {
     # pair tiles with shared experts (a dense group of 200 tokens) and drops
     "pair_shared": Workload("pair_shared", T=200, d=256, h=256, E=4, k=2, n_shared=2,
                             h_shared=128, cf=(1, 1), zipf_s=0.5),
+    # experts of over 1024 tokens: token-major tiles of 256 tokens on CTA pairs,
+    # ragged last tiles (an expert's second CTA half partly or wholly past its rows)
+    "pair_tok": Workload("pair_tok", T=1300, d=256, h=384, E=3, k=2, zipf_s=0.3),
 }
 
 
@@ -234,7 +237,7 @@ def test_full_size_workload(name, hidden):
     print(f"{name} ({hidden} H, {len(rows)} rows): {e} logit_err={zerr:.2e}")
 
 
-@pytest.mark.parametrize("name", ["pair_tiles", "pair_shared", "swap_cap"])
+@pytest.mark.parametrize("name", ["pair_tiles", "pair_shared", "swap_cap", "pair_tok"])
 def test_pair_tiles_match_single_sm_tiles(name):
     """Experts of more than 128 tokens run their GEMMs on CTA pairs; the same
     layer with one SM per tile gives the same output within the bar, and the
