@@ -472,31 +472,48 @@ __device__ void place_rows(const DispatchArgs& a, int blk, int nblk, bool writer
     }
     __syncthreads();
 
-    // gather: this CTA copies every nsplit-th (t, j) row of its block, eight
-    // rows at a time so that each thread keeps eight loads in flight
-    const int nrow = ROUTE_BLOCK * k;
-    const int nv = a.row_vecs;
+    // gather: every token's row is read once and stored to each slot it keeps.
+    // Warp w of this CTA takes the block's tokens split + nsplit * (w + W i);
+    // when the CTAs of a block outnumber its tokens' warps' work, the columns
+    // of a row are split between the warps that share the token.
+    constexpr int W = ROUTE_BLOCK / 32;
     constexpr int G = 8;
-    for (int r0 = split; r0 < nrow; r0 += G * nsplit) {
-        const uint4* src[G];
-        uint4* dst[G];
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nv = a.row_vecs;
+    const int64_t tok0 = (int64_t)blk * ROUTE_BLOCK;
+    const int ntok = (int)((a.T - tok0) < ROUTE_BLOCK ? (a.T - tok0) : ROUTE_BLOCK);
+    const int workers = nsplit * W;                       // warps over this block
+    const int wid = split + nsplit * warp;                // this warp among them
+    const int cparts = workers > ntok ? workers / ntok : 1;  // column parts per token
+    const int cp = wid % cparts;                          // this warp's column part
+    for (int tl = wid / cparts; tl < ntok; tl += workers / cparts) {
+        uint4* dst[MAX_K];
+        bool any = false;
 #pragma unroll
-        for (int q = 0; q < G; ++q) {
-            const int r = r0 + q * nsplit;
-            const int32_t row = r < nrow ? d.slots[r] : -1;
-            const int64_t tok = (int64_t)blk * ROUTE_BLOCK + r / k;
-            src[q] = row >= 0 ? a.x + tok * nv : nullptr;
-            dst[q] = row >= 0 ? d.peer[d.owner[r]] + (int64_t)(row + d.start[d.owner[r]]) * nv
+        for (int j = 0; j < MAX_K; ++j) {
+            const int32_t row = j < k ? d.slots[tl * k + j] : -1;
+            dst[j] = row >= 0 ? d.peer[d.owner[tl * k + j]] +
+                                    (int64_t)(row + d.start[d.owner[tl * k + j]]) * nv
                               : nullptr;
+            any |= row >= 0;
         }
-        for (int c = tid; c < nv; c += ROUTE_BLOCK) {
+        if (!any) continue;
+        const uint4* src = a.x + (tok0 + tl) * nv;
+        // this warp's share of the row's 16-byte columns
+        const int c_lo = (int)((int64_t)nv * cp / cparts);
+        const int c_hi = (int)((int64_t)nv * (cp + 1) / cparts);
+        for (int c0 = c_lo + lane; c0 < c_hi; c0 += 32 * G) {
             uint4 v[G];
 #pragma unroll
             for (int q = 0; q < G; ++q)
-                if (src[q]) v[q] = __ldg(src[q] + c);
+                if (c0 + 32 * q < c_hi) v[q] = __ldg(src + c0 + 32 * q);
 #pragma unroll
-            for (int q = 0; q < G; ++q)
-                if (dst[q]) dst[q][c] = v[q];
+            for (int j = 0; j < MAX_K; ++j) {
+                if (!dst[j]) continue;
+#pragma unroll
+                for (int q = 0; q < G; ++q)
+                    if (c0 + 32 * q < c_hi) dst[j][c0 + 32 * q] = v[q];
+            }
         }
     }
 }
