@@ -75,6 +75,8 @@ def parse():
                    help="launch the forward chain without programmatic dependent launch")
     p.add_argument("--no-pair", action="store_true",
                    help="one SM per expert GEMM tile (no CTA pairs)")
+    p.add_argument("--no-overlap", action="store_true",
+                   help="shared experts after the routed ones on one stream")
     p.add_argument("--backward", action="store_true",
                    help="time forward + backward (a training step) instead of the forward (1 GPU)")
     return p.parse_args()
@@ -523,6 +525,7 @@ def main():
         raise SystemExit("--backward runs on one GPU")
     B.moe_set_pdl(not args.no_pdl)
     B.moe_set_pair_tiles(not args.no_pair)
+    B.moe_set_shared_overlap(not args.no_overlap)
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward
     cfg, host, g, W, Wb = build_inputs(wl, rank, world, dev, keep_host=want_cpu,
                                        train=args.backward, hidden=args.hidden_mode)

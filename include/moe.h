@@ -483,6 +483,15 @@ MOE_API int moe_set_pdl(int on);
  * the layer's tolerance (the fp32 sums run in the same order).  Process-wide. */
 MOE_API int moe_set_pair_tiles(int on);
 
+/* Shared experts beside the routed ones in moe_forward (default on): they
+ * need only x, so they run on a second stream (one per device, created by the
+ * library on first use) from the start of the call, beside the routing and
+ * the routed experts, and the combine waits for them; the call still returns
+ * with all its work ordered on `stream`.  Calls from several threads on one
+ * device share that second stream.  Off: one stream, shared experts after the
+ * routed ones.  Results are identical either way.  Process-wide. */
+MOE_API int moe_set_shared_overlap(int on);
+
 /* Upper bound, in nanoseconds, on every device-side wait of the tensor-core
  * kernels (default 2e9).  A wait that runs out records MOE_ERR_TIMEOUT in
  * the device status word and its kernel returns early.  Process-wide. */

@@ -721,10 +721,40 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     return MOE_OK;
 }
 
+// The shared experts' FFN over every token (fused into one expert of width
+// S * hs): gate 1, no capacity, reads x directly.
+static int step_shared_ffn(const Plan& P, const Device& dv, const void* x, const void* W13s,
+                           const void* W2s, float* y_shared, void* ws, cudaStream_t st) {
+    if (P.T == 0 || P.S == 0) return MOE_OK;
+    int32_t* status = at<int32_t>(ws, P.off_status);
+    void* Hs = at<void>(ws, P.off_Hs);
+    if (P.shared_path == PATH_F32) {
+        MOE_TRY(launched(launch_f32_gateup(reinterpret_cast<const float*>(x),
+                                           reinterpret_cast<const float*>(W13s),
+                                           reinterpret_cast<float*>(Hs), 1, nullptr, nullptr,
+                                           (int)P.T, P.T, P.d, P.hsum, st),
+                         "f32_shared_gateup"));
+        trace_mark(st, "f32_shared_gateup");
+        MOE_TRY(launched(launch_f32_down(reinterpret_cast<const float*>(Hs),
+                                         reinterpret_cast<const float*>(W2s), y_shared, 1,
+                                         nullptr, nullptr, (int)P.T, P.T, P.d, P.hsum, st),
+                         "f32_shared_down"));
+        trace_mark(st, "f32_shared_down");
+        return MOE_OK;
+    }
+    const int nt = (int)((P.T + 15) / 16 * 16);
+    void* ABs = P.train ? at<void>(ws, P.off_ABs) : nullptr;
+    return run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, nullptr, (int)P.T, x, P.T, W13s,
+                      W2s, P.hsum, Hs, ABs, y_shared, 1, nt, status, st, "gemm_shared_gateup",
+                      "gemm_shared_down");
+}
+
+// The routed experts' FFN over the dispatched rows; with `shared`, then the
+// shared experts' on the same stream.
 static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const int32_t* offsets,
                     const int32_t* kept, const void* W13, const void* W2p, const void* x,
                     const void* W13s, const void* W2s, float* y_perm, float* y_shared, void* ws,
-                    cudaStream_t st) {
+                    cudaStream_t st, bool shared = true) {
     if (P.T == 0) return MOE_OK;
     void* H = at<void>(ws, P.off_H);
     int32_t* status = at<int32_t>(ws, P.off_status);
@@ -747,31 +777,41 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
                            P.h, H, AB, y_perm, P.splits, P.nt_max, status, st, "gemm_gateup",
                            "gemm_down"));
     }
-    if (P.S > 0) {
-        void* Hs = at<void>(ws, P.off_Hs);
-        if (P.shared_path == PATH_F32) {
-            MOE_TRY(launched(launch_f32_gateup(reinterpret_cast<const float*>(x),
-                                               reinterpret_cast<const float*>(W13s),
-                                               reinterpret_cast<float*>(Hs), 1, nullptr, nullptr,
-                                               (int)P.T, P.T, P.d, P.hsum, st),
-                             "f32_shared_gateup"));
-            trace_mark(st, "f32_shared_gateup");
-            MOE_TRY(launched(launch_f32_down(reinterpret_cast<const float*>(Hs),
-                                             reinterpret_cast<const float*>(W2s), y_shared, 1,
-                                             nullptr, nullptr, (int)P.T, P.T, P.d, P.hsum, st),
-                             "f32_shared_down"));
-            trace_mark(st, "f32_shared_down");
-        } else {
-            const int nt = (int)((P.T + 15) / 16 * 16);
-            void* ABs = P.train ? at<void>(ws, P.off_ABs) : nullptr;
-            MOE_TRY(run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, nullptr, (int)P.T, x,
-                               P.T, W13s,
-                               W2s, P.hsum, Hs, ABs, y_shared, 1, nt, status, st,
-                               "gemm_shared_gateup", "gemm_shared_down"));
-        }
-    }
+    if (shared) MOE_TRY(step_shared_ffn(P, dv, x, W13s, W2s, y_shared, ws, st));
     return MOE_OK;
 }
+
+// ---------------------------------------------------------------- shared experts beside the routed
+
+// A second stream per device for the shared experts of moe_forward, and the
+// events that fork it from and join it back into the caller's stream.
+struct SideStream {
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+static int side_stream(SideStream* out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static SideStream cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return fail(MOE_ERR_CUDA, "cudaGetDevice failed");
+    std::lock_guard<std::mutex> lk(mu);
+    SideStream& c = cache[dev];
+    if (!c.st) {
+        if (cudaStreamCreateWithFlags(&c.st, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) != cudaSuccess) {
+            c = SideStream();
+            return fail(MOE_ERR_CUDA, "could not create the shared-expert stream");
+        }
+    }
+    *out = c;
+    return MOE_OK;
+}
+
+static int g_shared_overlap = 1;
 
 static StatsParams stats_params(const Plan& P, const int32_t* routed, const int32_t* kept,
                                 const void* ws, double* sums, moe_stats* stats) {
@@ -1179,9 +1219,30 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
     void* x_perm = at<void>(ws, P.off_xperm);
     float* y = at<float>(ws, P.off_y);
     float* ys = P.S ? at<float>(ws, P.off_ys) : nullptr;
+    // The shared experts need only x: with the overlap on they run on a second
+    // stream from the start of the call, beside the routing and the routed
+    // experts, and the combine waits for them.  (Off while every kernel is
+    // being timed, whose events assume one stream.)
+    const bool side = P.T > 0 && P.S > 0 && P.bf16 && g_shared_overlap &&
+                      !(g_trace.on && g_trace.only.empty());
+    SideStream ss;
+    if (side) {
+        MOE_TRY(side_stream(&ss));
+        if (cudaEventRecord(ss.fork, st) != cudaSuccess ||
+            cudaStreamWaitEvent(ss.st, ss.fork, 0) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "could not fork the shared-expert stream");
+        g_pdl_in_forward = false;  // the first launch on the side stream follows an event
+        const int rc = step_shared_ffn(P, dv, x, W13s, W2s, ys, ws, ss.st);
+        g_pdl_in_forward = true;
+        MOE_TRY(rc);
+        if (cudaEventRecord(ss.join, ss.st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "could not join the shared-expert stream");
+    }
     MOE_TRY(step_route_dispatch(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate,
                                 routed, kept, offsets, perm, slot_of, x_perm, ws, st));
-    MOE_TRY(step_ffn(P, dv, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st));
+    MOE_TRY(step_ffn(P, dv, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st, !side));
+    if (side && cudaStreamWaitEvent(st, ss.join, 0) != cudaSuccess)
+        return fail(MOE_ERR_CUDA, "could not join the shared-expert stream");
     // combine, with the statistics computed by one extra block of the same launch
     StatsParams sp = stats_params(P, routed, kept, ws, at<double>(ws, P.off_sums), stats);
     if (P.T > 0)
@@ -1603,6 +1664,11 @@ int moe_set_pdl(int on) {
 
 int moe_set_pair_tiles(int on) {
     g_pair_enabled = on ? 1 : 0;
+    return ok();
+}
+
+int moe_set_shared_overlap(int on) {
+    g_shared_overlap = on ? 1 : 0;
     return ok();
 }
 

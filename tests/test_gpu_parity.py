@@ -263,6 +263,27 @@ def test_pair_tiles_match_single_sm_tiles(name):
     print(f"{name}: pair {e1} single {e2} max|pair - single| {d:.3e}")
 
 
+@pytest.mark.parametrize("name", ["shared", "shared_small", "pair_shared", "shared_swap64"])
+def test_shared_overlap_gives_identical_bits(name):
+    """Shared experts on a second stream beside the routed ones, or after them
+    on one stream: the same bits; and the overlapped run matches the oracle."""
+    wl = SMALL[name]
+    inp = host_inputs(wl)
+    cfg, g, W = device_layer(wl, inp)
+    B.moe_set_shared_overlap(True)
+    a = run_forward(cfg, g, W)
+    out_on = a["out"].clone()
+    try:
+        B.moe_set_shared_overlap(False)
+        b = run_forward(cfg, g, W)
+    finally:
+        B.moe_set_shared_overlap(True)
+    assert torch.equal(out_on, b["out"])
+    assert B.moe_read_device_status(b["ws"]) == 0
+    r = oracle_route(wl, inp)
+    check_output(out_on, oracle_rows(wl, inp, r), strict=strict_output(cfg))
+
+
 @pytest.mark.parametrize("name", ["swap", "tok_cap", "shared"])
 def test_dependent_launch_gives_identical_bits(name):
     """The forward chain launched with and without programmatic dependent
