@@ -588,7 +588,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
                       int dense_rows, const void* act,
                       int64_t act_rows, const void* W13, const void* W2p, int hid, void* H,
                       void* AB, float* y, int splits, int nt_max, int32_t* status,
-                      cudaStream_t st, const char* tag1, const char* tag2) {
+                      cudaStream_t st, const char* tag1, const char* tag2, int ctr_slot = 0) {
     const bool tok = path == PATH_TOKEN_MAJOR;
     CUtensorMap m_act, m_w;
     TcArgs a;
@@ -606,6 +606,14 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
 
     // split H: its low bf16 parts follow the high ones, act_rows rows further
     a.lo_rows = P.split ? act_rows : 0;
+    // the CTA-pair kernels take their units from a counter in the status area
+    // (one per stream that may run them at once), zeroed before each launch
+    a.unit_ctr = status + UNIT_CTR_WORD + ctr_slot;
+    auto zero_ctr = [&]() -> int {
+        if (cudaMemsetAsync(a.unit_ctr, 0, sizeof(int32_t), st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "memset failed");
+        return MOE_OK;
+    };
 
     // gate/up: act [act_rows][d] x W13 [groups * 2hid][d] -> H [act_rows][hid]
     const int mode1 = tok ? TC_GATEUP_TOK : TC_GATEUP_SWAP;
@@ -633,6 +641,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 128));
         a.stages = tc_pair_max_stages(TC_PAIR_GATEUP_TOK, nt_max, groups, false, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
         trace_pre(st, tag1);
         MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP_TOK, m_act, m_w, a, st), tag1));
         trace_mark(st, tag1);
@@ -649,6 +658,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         a.prefetch_kb = 0;
         a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, nt_max, groups, P.split, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
         trace_pre(st, tag2);
         MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, st), tag2));
         trace_mark(st, tag2);
@@ -659,6 +669,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 64));
         a.stages = tc_pair_max_stages(TC_PAIR_GATEUP, nt_max, groups, false, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
         trace_pre(st, tag1);
         MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP, m_act, m_w, a, st), tag1));
         trace_mark(st, tag1);
@@ -694,6 +705,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         a.prefetch_kb = 0;
         a.stages = tc_pair_max_stages(TC_PAIR_DOWN, nt_max, groups, P.split, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
         trace_pre(st, tag2);
         MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN, m_act, m_w, a, st), tag2));
         trace_mark(st, tag2);
@@ -746,7 +758,7 @@ static int step_shared_ffn(const Plan& P, const Device& dv, const void* x, const
     void* ABs = P.train ? at<void>(ws, P.off_ABs) : nullptr;
     return run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, nullptr, (int)P.T, x, P.T, W13s,
                       W2s, P.hsum, Hs, ABs, y_shared, 1, nt, status, st, "gemm_shared_gateup",
-                      "gemm_shared_down");
+                      "gemm_shared_down", 1);
 }
 
 // The routed experts' FFN over the dispatched rows; with `shared`, then the

@@ -41,7 +41,11 @@
 // relays "my stage is full" to the even CTA; warps 2-9 are the epilogue.
 // The MMA's completion is signalled to both CTAs' barriers at once
 // (tcgen05.commit multicast); the epilogues of both CTAs release an
-// accumulator on the even CTA's barrier.  Every wait is bounded; on a
+// accumulator on the even CTA's barrier.  The pairs take their work units
+// from a device counter (the even CTA's producer fetches the next unit and
+// publishes it to every role of both CTAs through a small queue in shared
+// memory), so the work spreads over however many pairs are resident at once.
+// Every wait is bounded; on a
 // time-out the kernel records MOE_ERR_TIMEOUT, lets the copies it issued
 // land and the MMAs drain, and both CTAs meet at a cluster barrier before
 // TMEM is released.
@@ -61,6 +65,7 @@ constexpr int PBK = 64;    // K per stage: one 128-byte swizzle row of bf16
 constexpr int PUK = 16;    // K per MMA
 constexpr uint64_t P_TEARDOWN_NS = 200000000ull;
 constexpr int P_STG_LD = 36;  // fp32 staging row (32 values + 4 of padding)
+constexpr int P_QN = 4;       // slots of the unit queue
 
 __host__ __device__ constexpr bool p_tok(int mode) {
     return mode == TC_PAIR_GATEUP_TOK || mode == TC_PAIR_DOWN_TOK;
@@ -102,8 +107,9 @@ __host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stag
     if (mode == TC_PAIR_DOWN_TOK) xch = p_epi(mode) * 32 * P_STG_LD * 4;
     L.flag_off = L.xch_off + xch;
     L.bar_off = p_align(L.flag_off + p_epi(mode) * 2 * 4, 16);
-    // full[S], relay[S], empty[S], acc_full[2], acc_empty[2], drain, tmem slot
-    L.grp_off = L.bar_off + p_align((3 * stages + 5) * 8 + 8, 16);
+    // full[S], relay[S], empty[S], acc_full[2], acc_empty[2], drain, q_full[QN],
+    // q_empty[QN], tmem slot, q_unit[QN]
+    L.grp_off = L.bar_off + p_align((3 * stages + 5 + 2 * P_QN) * 8 + 8 + 4 * P_QN, 16);
     L.total = L.grp_off + (4 * groups + 1) * 4 + 1024;
     return L;
 }
@@ -191,7 +197,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     uint64_t* acc_full = empty + S;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* q_full = drain + 1;        // unit published (both CTAs)
+    uint64_t* q_empty = q_full + P_QN;   // unit read by every consumer (even CTA)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + P_QN);
+    int* q_unit = reinterpret_cast<int*>(tmem_slot + 1);
     int* g_start = reinterpret_cast<int*>(smem + L.grp_off);
     int* g_rows = g_start + groups + 1;
     int* g_off = g_rows + groups;
@@ -202,7 +211,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     const int lane = threadIdx.x & 31;
     const uint32_t v = cluster_ctarank();       // 0: issues the MMAs; 1: relays
     const int pair = blockIdx.x >> 1;
-    const int npairs = gridDim.x >> 1;
 
     // accumulator: 128 lanes x nt_max (token-major: 256) columns, twice when it fits
     const int acc_stride = TOK ? 256 : args.nt_max;
@@ -221,6 +229,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             mbar_init(&acc_empty[i], 2 * NEPI);  // one arrive per epilogue warp of each CTA
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < P_QN; ++i) {
+            mbar_init(&q_full[i], 1);
+            // consumers: the MMA thread and epilogue warps of the even CTA, the
+            // producer, relay and epilogue warps of the odd one
+            mbar_init(&q_empty[i], 3 + 2 * NEPI);
+        }
         fence_mbar_init();
         prefetch_tmap(&tm_act);
         prefetch_tmap(&tm_w);
@@ -258,6 +272,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     const PGroups tab{g_start, g_rows, g_off, g_wi, groups};
     const int total = g_start[groups];
     const uint64_t limit = args.wait_limit_ns;
+    // the unit queue: slot j holds the j-th unit (mod P_QN) of this pair, or
+    // `total` when there is no more work
+    const uint32_t lead_q_empty0 = map_shared_rank(smem_addr(&q_empty[0]), 0);
+    auto take_unit = [&](int& slot, uint32_t& qph, bool arrive, int* u) -> bool {
+        if (!mbar_wait_cl(&q_full[slot], qph, limit)) return false;
+        *u = *reinterpret_cast<volatile int*>(&q_unit[slot]);
+        if (arrive) mbar_arrive_cluster(lead_q_empty0 + slot * 8);
+        if (++slot == P_QN) {
+            slot = 0;
+            qph ^= 1;
+        }
+        return true;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -270,7 +297,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             uint32_t issued = 0, issued_par = 0;
             bool ok = true;
             const int kblocks = args.K / PBK;
-            for (int u = pair; u < total && ok; u += npairs) {
+            int qs = 0;
+            uint32_t qph = 0;
+            const uint32_t peer_unit0 = map_shared_rank(smem_addr(&q_unit[0]), 1);
+            const uint32_t peer_full0 = map_shared_rank(smem_addr(&q_full[0]), 1);
+            while (ok) {
+                int u = total;
+                if (v == 0) {
+                    // the scheduler: next unit of this pair, published to both CTAs
+                    if (!mbar_wait_cl(&q_empty[qs], qph ^ 1, limit)) {
+                        report_timeout(args.status);
+                        break;
+                    }
+                    u = atomicAdd(args.unit_ctr, 1);
+                    if (u > total) u = total;
+                    q_unit[qs] = u;
+                    st_cluster_u32(peer_unit0 + qs * 4, (uint32_t)u);
+                    mbar_arrive(&q_full[qs]);
+                    mbar_arrive_cluster(peer_full0 + qs * 8);
+                    if (++qs == P_QN) {
+                        qs = 0;
+                        qph ^= 1;
+                    }
+                } else if (!take_unit(qs, qph, true, &u)) {
+                    report_timeout(args.status);
+                    break;
+                }
+                if (u >= total) break;
                 const PUnit x = p_decode<MODE>(tab, u);
                 const int half = x.ntok / 2;          // token rows this CTA stages
                 const int trow = TOK ? x.row0 + x.mt * 256 + (int)v * PBM : x.row0 + (int)v * half;
@@ -335,7 +388,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             uint32_t phase = 0;
             bool ok = true;
             const int kblocks = args.K / PBK;
-            for (int u = pair; u < total && ok; u += npairs) {
+            int qs = 0;
+            uint32_t qph = 0;
+            while (ok) {
+                int u = total;
+                if (!take_unit(qs, qph, true, &u)) {
+                    report_timeout(args.status);
+                    break;
+                }
+                if (u >= total) break;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&full[stage], phase, limit)) {
                         report_timeout(args.status);
@@ -357,7 +418,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             const int kblocks = args.K / PBK;
-            for (int u = pair; u < total && ok; u += npairs) {
+            int qs = 0;
+            uint32_t qph = 0;
+            bool first = true;
+            while (ok) {
+                int u = total;
+                if (!take_unit(qs, qph, true, &u)) {
+                    report_timeout(args.status);
+                    break;
+                }
+                if (u >= total) break;
                 const PUnit x = p_decode<MODE>(tab, u);
                 if (!mbar_wait_cl(&acc_empty[acc], acc_phase ^ 1, limit)) {
                     report_timeout(args.status);
@@ -398,7 +468,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                 }
                 if (!ok) break;
                 // test hook: the first unit of pair 0 never signals its epilogues
-                const bool withhold = args.test_stall && pair == 0 && u == pair;
+                const bool withhold = args.test_stall && pair == 0 && first;
+                first = false;
                 if (!withhold) umma_commit_pair_both(&acc_full[acc]);
                 if (++acc == n_acc) {
                     acc = 0;
@@ -423,21 +494,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
         const bool is_gate = q < 2;
         int acc = 0;
         uint32_t acc_phase = 0;
-        int it = 0;
-        for (int u = pair; u < total; u += npairs, ++it) {
-            const PUnit x = p_decode<MODE>(tab, u);
-            bool ok = mbar_wait(&acc_full[acc], acc_phase, limit);
+        int qs = 0;
+        uint32_t qph = 0;
+        for (int it = 0;; ++it) {
+            int u = total;
+            bool ok = take_unit(qs, qph, false, &u);
+            __syncwarp();
+            if (ok && lane == 0) mbar_arrive_cluster(lead_q_empty0 + ((qs + P_QN - 1) % P_QN) * 8);
+            const bool done = ok && u >= total;
+            if (ok && !done) ok = mbar_wait(&acc_full[acc], acc_phase, limit);
             if (GU) {
-                // both warps of a pair go on only if both saw the accumulator
-                if (lane == 0) flags[ew * 2 + (it & 1)] = ok ? 1 : 0;
+                // both warps of a pair go on, or stop, together: 0 a wait ran
+                // out, 1 the accumulator is ready, 2 no more work
+                if (lane == 0) flags[ew * 2 + (it & 1)] = !ok ? 0 : (done ? 2 : 1);
                 named_sync(1 + pidx, 64);
                 const int partner = is_gate ? ew - 2 : ew + 2;
-                ok = flags[ew * 2 + (it & 1)] && flags[partner * 2 + (it & 1)];
+                const int f0 = flags[ew * 2 + (it & 1)], f1 = flags[partner * 2 + (it & 1)];
+                if (f0 == 0 || f1 == 0) {
+                    report_timeout(args.status);
+                    break;
+                }
+                if (f0 == 2 || f1 == 2) break;
+            } else {
+                if (!ok) {
+                    report_timeout(args.status);
+                    break;
+                }
+                if (done) break;
             }
-            if (!ok) {
-                report_timeout(args.status);
-                break;
-            }
+            const PUnit x = p_decode<MODE>(tab, u);
             tc_fence_after();
             const uint32_t t0 = lane_addr + acc * acc_stride;
             if (MODE == TC_PAIR_GATEUP_TOK) {
@@ -573,28 +658,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     if (warp == 1) tmem_dealloc_pair(tmem_base, tmem_cols);
 }
 
-// Pairs that fit the device at once (cached per device and mode).
-int pair_grid(const void* kern, uint32_t smem, int mode) {
-    constexpr int kMaxDevices = 64;
-    static std::mutex mu;
-    static int cached[kMaxDevices][4] = {};
-    static uint32_t cached_smem[kMaxDevices][4] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-    const int m = mode - TC_PAIR_GATEUP;
-    std::lock_guard<std::mutex> lk(mu);
-    if (cached[dev][m] == 0 || cached_smem[dev][m] != smem) {
-        // the cluster shape comes from the kernel's __cluster_dims__
-        cudaLaunchConfig_t c = {};
-        c.gridDim = dim3(2);
-        c.blockDim = dim3(p_threads(mode));
-        c.dynamicSmemBytes = smem;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &c) != cudaSuccess || n < 1) return 0;
-        cached[dev][m] = n;
-        cached_smem[dev][m] = smem;
-    }
-    return cached[dev][m];
+// One pair per two SMs: the pairs take their units from a counter, so any that
+// are not resident at once only start later and find less work.
+int pair_grid() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms / 2;
 }
 
 template <int MODE>
@@ -618,8 +689,8 @@ int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs&
             configured_bytes[dev] = L.total;
         }
     }
-    const int pairs = pair_grid(reinterpret_cast<const void*>(kern), L.total, MODE);
-    if (pairs < 1) {
+    const int pairs = pair_grid();
+    if (pairs < 1 || !a.unit_ctr) {
         last_launch_error() = cudaErrorInvalidConfiguration;
         return -1;
     }

@@ -162,6 +162,8 @@ struct TcArgs {
     const int32_t* group_w;     // device [num_groups] weight index of each group, or null -> g
     int prefetch_kb;            // swapped gate/up: k-blocks of the first weight tile to prefetch
                                 // into L2 before waiting on the predecessor (0: none)
+    int32_t* unit_ctr;          // CTA-pair kernels: device counter the pairs take their units
+                                // from (zero at launch)
     int64_t lo_rows;            // H as bf16 high + low parts (0: bf16 H alone): gate/up writes
                                 // row r's low parts to row r + lo_rows of `out`; down reads
                                 // them there from the activation tensor and issues a second

@@ -34,6 +34,10 @@ constexpr int MAX_PEERS = 64;     // expert-parallel ranks one dispatch or combi
 constexpr int SWAP_MAX_TOKENS = 256;  // largest per-expert token count the swap path covers
 constexpr int DOWN_SWAP_MAX_TOKENS = 128;  // above this the down projection takes token-major tiles
 constexpr int PAIR_TOK_MIN_TOKENS = 1024;  // token-major tiles on CTA pairs from this group bound on
+// int32 words of the workspace's 256-byte status area: [0] the status word,
+// [1] the combine's ticket, [8..9] the CTA-pair kernels' unit counters (one per
+// stream of a moe_forward: the routed experts', the shared experts')
+constexpr int UNIT_CTR_WORD = 8;
 
 struct Plan {
     int64_t T;

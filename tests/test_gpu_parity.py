@@ -138,8 +138,8 @@ def test_small_layer_other_hidden_mode(name):
     auto_split = B.moe_hidden_split(B.config_of(wl))
     cfg, g, W = device_layer(wl, inp, hidden="bf16" if auto_split else "split")
     assert B.moe_hidden_split(cfg) != auto_split
-    b = run_forward(cfg, g, W)
-    assert B.moe_read_device_status(b["ws"]) == 0
+    b = run_steps(cfg, g, W)
+    assert b["status"] == 0
     check_routing(wl, r, b)
     offsets = b["offsets"].cpu().numpy()
     check_offsets(wl, r, offsets, _pad(cfg))
