@@ -83,8 +83,9 @@ __host__ __device__ inline bool down_split(int mode, int64_t lo_rows) {
 }
 
 // Bytes of operand per stage for each mode.  With a split H the token-major
-// down stages the high and the low 128-row tile one after the other (A), the
-// swapped down the high and the low token tile (B, nt_max rows each).
+// down stages the high and the low 128-row tile one after the other (A); the
+// swapped down stages a unit's ntok high-part rows and right after them its
+// ntok low-part rows (B, room for 2 nt_max rows), read by one MMA of N = 2 ntok.
 __host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, bool split, uint32_t* a,
                                             uint32_t* b) {
     const uint32_t parts = split ? 2 : 1;
@@ -281,7 +282,9 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
         acc_stride = 2 * args.nt_max;
         n_acc = (2 * acc_stride <= 512) ? 2 : 1;
     } else {
-        acc_stride = args.nt_max;
+        // swapped down: with split H the low parts' columns follow the high
+        // parts' in the same accumulator (one MMA of N = 2 ntok per K step)
+        acc_stride = args.nt_max * (dsplit ? 2 : 1);
         n_acc = 2;
     }
     uint32_t tmem_cols = 32;
@@ -409,9 +412,9 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                         for (int r = 0; r < x.ntok; r += 16)
                             tma_load_2d_hint(sb + r * BK * 2, &tm_act, &full[stage], kc,
                                              x.row0 + r, pol_a);
-                        if (dsplit)  // the low parts of H behind the high ones
+                        if (dsplit)  // the low parts of H right behind the high ones
                             for (int r = 0; r < x.ntok; r += 16)
-                                tma_load_2d_hint(sb + (args.nt_max + r) * BK * 2, &tm_act,
+                                tma_load_2d_hint(sb + (x.ntok + r) * BK * 2, &tm_act,
                                                  &full[stage], kc,
                                                  x.row0 + r + (int)args.lo_rows, pol_a);
                     }
@@ -445,7 +448,11 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * acc_stride;
-                const uint32_t idesc = TOK ? idesc_tok : idesc_bf16_f32(BM, x.ntok);
+                // swapped down with split H: B = [H_hi; H_lo] rows, N = 2 ntok, so
+                // that the weight tile is read once for both parts
+                const uint32_t idesc =
+                    TOK ? idesc_tok
+                        : idesc_bf16_f32(BM, x.ntok * (MODE == TC_DOWN_SWAP && dsplit ? 2 : 1));
                 for (int kb = x.kb0; kb < x.kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, limit)) {
                         report_timeout(args.status);
@@ -471,10 +478,6 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                         if (MODE == TC_DOWN_TOK && dsplit)  // + H_lo . W
                             umma_bf16(d_tmem, sdesc_kmajor_sw128(sa + BM * BK * 2 + kk * UK * 2),
                                       bdesc, idesc, 1u);
-                        if (MODE == TC_DOWN_SWAP && dsplit)  // + W . H_lo
-                            umma_bf16(d_tmem, adesc,
-                                      sdesc_kmajor_sw128(sb + args.nt_max * BK * 2 + kk * UK * 2),
-                                      idesc, 1u);
                         if (MODE == TC_GATEUP_SWAP)
                             umma_bf16(d_tmem + args.nt_max,
                                       sdesc_kmajor_sw128(sa + BM * BK * 2 + kk * UK * 2), bdesc,
@@ -698,6 +701,14 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                 for (int c = 0; c < x.ntok; c += 16) {
                     float v[16];
                     tmem_ld16(t0 + c, v);
+                    if (dsplit) {
+                        // + the low parts' columns: y = W.H_hi + W.H_lo
+                        float w[16];
+                        tmem_ld16(t0 + x.ntok + c, w);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] += w[i];
+                    }
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
