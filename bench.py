@@ -19,6 +19,7 @@ moe_backward (gradients of <G, out> + 0.01 aux for every input and weight).
 
 import argparse
 import datetime
+import glob
 import hashlib
 import json
 import math
@@ -42,7 +43,8 @@ METRIC = "MoE-layer tokens/s (1xB200) and % of roofline (BF16 TC / HBM)"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILES = os.path.join(ROOT, "profiles")
-GEMM_SRC = os.path.join(ROOT, "sparse_mixture_experts_22_b200", "csrc", "gemm_tc.cu")
+GEMM_SRCS = [os.path.join(ROOT, "sparse_mixture_experts_22_b200", "csrc", n)
+             for n in ("gemm_tc.cu", "gemm_pair.cu", "common.cuh")]
 
 
 def parse():
@@ -316,23 +318,37 @@ class ClockSampler:
 
 def traffic_from_profile(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current GEMM source; None otherwise."""
-    path = os.path.join(PROFILES, f"{kernel}_{workload}.ncu.txt")
-    if not os.path.exists(path):
-        return None
-    vals = {}
-    with open(path) as f:
-        for line in f:
-            if "=" in line and not line.startswith("#"):
-                k, v = line.split("=", 1)
-                vals[k.strip()] = v.strip()
-    sha = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
-    if vals.get("gemm_source_sha256") != sha:
-        return None
-    try:
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    on the current GEMM sources; None otherwise.  A summary of a smaller case
+    of the workload (`<kernel>_<workload>_h<width>.ncu.txt`, the hidden width
+    cut) records `scale_to_full`, the factor by which the launch's work units
+    (and so its traffic) grow at full size."""
+    cands = [os.path.join(PROFILES, f"{kernel}_{workload}.ncu.txt")]
+    cands += sorted(glob.glob(os.path.join(PROFILES, f"{kernel}_{workload}_h*.ncu.txt")))
+    for path in cands:
+        if not os.path.exists(path):
+            continue
+        vals = {}
+        with open(path) as f:
+            for line in f:
+                if "=" in line and not line.startswith("#"):
+                    k, v = line.split("=", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("gemm_source_sha256") != gemm_sources_sha():
+            continue
+        try:
+            return float(vals["dram_bytes_per_launch"]) * float(vals.get("scale_to_full", 1))
+        except (KeyError, ValueError):
+            continue
+    return None
+
+
+def gemm_sources_sha():
+    """SHA-256 over the tensor-core GEMM sources (one-SM and CTA-pair kernels)."""
+    h = hashlib.sha256()
+    for path in GEMM_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def cpu_threads():

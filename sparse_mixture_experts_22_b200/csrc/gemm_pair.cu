@@ -35,13 +35,16 @@
 // instead of 48 KB for 128 x 256 x 64: a third less shared-memory fill (L2
 // traffic) per flop.
 //
-// Roles (each CTA, 10 warps): warp 0 loads this CTA's halves with TMA into
-// its own stages (own barriers; no multicast); in the even CTA warp 1 issues
-// the pair MMAs once both CTAs' stages are full, in the odd CTA warp 1
-// relays "my stage is full" to the even CTA; warps 2-9 are the epilogue.
-// The MMA's completion is signalled to both CTAs' barriers at once
-// (tcgen05.commit multicast); the epilogues of both CTAs release an
-// accumulator on the even CTA's barrier.  The pairs take their work units
+// Roles (each CTA): warp 0 loads this CTA's halves with TMA into its own
+// stages, every copy signalling the even CTA's "stage full" barrier (the
+// cta_group::2 form of the copy; no multicast), which the even CTA's producer
+// arms with both CTAs' bytes; in the even CTA warp 1 issues the pair MMAs
+// once a stage is full; the other warps are the epilogue.  The MMA's
+// completion is signalled to both CTAs' barriers at once (tcgen05.commit
+// multicast); the epilogues of both CTAs release an accumulator on the even
+// CTA's barrier.  (A first version had the odd CTA's copies complete on its
+// own barrier and a thread forward each stage to the even CTA with a
+// cluster-scope release: that per-stage hop kept the tensor pipe 33% busy.)  The pairs take their work units
 // from a device counter (the even CTA's producer fetches the next unit and
 // publishes it to every role of both CTAs through a small queue in shared
 // memory), so the work spreads over however many pairs are resident at once.
@@ -107,9 +110,9 @@ __host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stag
     if (mode == TC_PAIR_DOWN_TOK) xch = p_epi(mode) * 32 * P_STG_LD * 4;
     L.flag_off = L.xch_off + xch;
     L.bar_off = p_align(L.flag_off + p_epi(mode) * 2 * 4, 16);
-    // full[S], relay[S], empty[S], acc_full[2], acc_empty[2], drain, q_full[QN],
-    // q_empty[QN], tmem slot, q_unit[QN]
-    L.grp_off = L.bar_off + p_align((3 * stages + 5 + 2 * P_QN) * 8 + 8 + 4 * P_QN, 16);
+    // full[S], empty[S], acc_full[2], acc_empty[2], drain, q_full[QN], q_empty[QN],
+    // tmem slot, q_unit[QN]
+    L.grp_off = L.bar_off + p_align((2 * stages + 5 + 2 * P_QN) * 8 + 8 + 4 * P_QN, 16);
     L.total = L.grp_off + (4 * groups + 1) * 4 + 1024;
     return L;
 }
@@ -192,8 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     const PairLayout L = pair_layout(MODE, args.nt_max, S, groups, split);
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-    uint64_t* relay = full + S;
-    uint64_t* empty = relay + S;
+    uint64_t* empty = full + S;
     uint64_t* acc_full = empty + S;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
@@ -209,7 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint32_t v = cluster_ctarank();       // 0: issues the MMAs; 1: relays
+    const uint32_t v = cluster_ctarank();       // 0: issues the MMAs
     const int pair = blockIdx.x >> 1;
 
     // accumulator: 128 lanes x nt_max (token-major: 256) columns, twice when it fits
@@ -220,8 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&relay[s], 1);
+            mbar_init(&full[s], 1);  // the even CTA's: armed once with both CTAs' bytes
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -232,8 +233,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
         for (int i = 0; i < P_QN; ++i) {
             mbar_init(&q_full[i], 1);
             // consumers: the MMA thread and epilogue warps of the even CTA, the
-            // producer, relay and epilogue warps of the odd one
-            mbar_init(&q_empty[i], 3 + 2 * NEPI);
+            // producer and epilogue warps of the odd one
+            mbar_init(&q_empty[i], 2 + 2 * NEPI);
         }
         fence_mbar_init();
         prefetch_tmap(&tm_act);
@@ -289,9 +290,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
+            // swapped: weights stream once (evict first), an expert's token rows
+            // are read again for each of its units (evict last); token-major: the
+            // default policy for both
             const uint64_t pol_w = l2_policy_evict_first();
-            const uint64_t pol_a = l2_policy_evict_last();
-            (void)pol_a;
+            const uint64_t pol_a = TOK ? l2_policy_evict_normal() : l2_policy_evict_last();
+            const uint64_t pol_n = l2_policy_evict_normal();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_par = 0;
@@ -301,6 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             uint32_t qph = 0;
             const uint32_t peer_unit0 = map_shared_rank(smem_addr(&q_unit[0]), 1);
             const uint32_t peer_full0 = map_shared_rank(smem_addr(&q_full[0]), 1);
+            const uint32_t lead_full0 = map_shared_rank(smem_addr(&full[0]), 0);
             while (ok) {
                 int u = total;
                 if (v == 0) {
@@ -338,35 +343,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                     uint8_t* sa = smem + stage * L.stage_bytes;
                     uint8_t* sb = sa + L.a_bytes;
                     const int kc = kb * PBK;
-                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    // the even CTA arms its barrier with both CTAs' bytes (the same
+                    // for both); every copy below completes on that barrier
+                    if (v == 0) mbar_arrive_expect_tx(&full[stage], 2 * bytes);
+                    const uint32_t fb = lead_full0 + stage * 8;
                     if (TOK) {
                         // A: this CTA's 128 token rows (then their low parts); B: the
                         // weight rows of this CTA's half of N (gate/up: CTA 0 the gate
                         // rows of the hidden block, CTA 1 its up rows)
-                        tma_load_2d(sa, &tm_act, &full[stage], kc, trow);
+                        tma_load_2d_pair(sa, &tm_act, fb, kc, trow, pol_a);
                         if (split)
-                            tma_load_2d(sa + PBM * PBK * 2, &tm_act, &full[stage], kc,
-                                        trow + (int)args.lo_rows);
-                        tma_load_2d(sb, &tm_w, &full[stage], kc,
-                                    x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM);
+                            tma_load_2d_pair(sa + PBM * PBK * 2, &tm_act, fb, kc,
+                                             trow + (int)args.lo_rows, pol_a);
+                        tma_load_2d_pair(sb, &tm_w, fb, kc,
+                                         x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM,
+                                         pol_n);
                     } else if (GU) {
                         // gate rows of features 64v.., then their up rows
                         const int wrow = x.w * args.w_rows_per_group + x.nb * 256 + (int)v * 64;
-                        tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
-                        tma_load_2d_hint(sa + 64 * PBK * 2, &tm_w, &full[stage], kc, wrow + 128,
-                                         pol_w);
+                        tma_load_2d_pair(sa, &tm_w, fb, kc, wrow, pol_w);
+                        tma_load_2d_pair(sa + 64 * PBK * 2, &tm_w, fb, kc, wrow + 128, pol_w);
                     } else {
                         const int wrow = x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM;
-                        tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
+                        tma_load_2d_pair(sa, &tm_w, fb, kc, wrow, pol_w);
                     }
                     if (!TOK) {
                         for (int r = 0; r < half; r += 8)
-                            tma_load_2d_hint(sb + r * PBK * 2, &tm_act, &full[stage], kc,
-                                             trow + r, pol_a);
+                            tma_load_2d_pair(sb + r * PBK * 2, &tm_act, fb, kc, trow + r, pol_a);
                         if (split)  // the low parts of H behind the high ones
                             for (int r = 0; r < half; r += 8)
-                                tma_load_2d_hint(sb + L.b_lo + r * PBK * 2, &tm_act, &full[stage],
-                                                 kc, trow + r + (int)args.lo_rows, pol_a);
+                                tma_load_2d_pair(sb + L.b_lo + r * PBK * 2, &tm_act, fb, kc,
+                                                 trow + r + (int)args.lo_rows, pol_a);
                     }
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -376,41 +383,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                     }
                 }
             }
-            // every copy this CTA issued lands before the CTA may leave
-            for (int s = 0; s < S; ++s)
-                if (issued & (1u << s)) mbar_wait(&full[s], (issued_par >> s) & 1, P_TEARDOWN_NS);
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && v == 1) {
-            // ------------------------------------------------------------ relay (odd CTA)
-            const uint32_t peer_relay0 = map_shared_rank(smem_addr(&relay[0]), 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            const int kblocks = args.K / PBK;
-            int qs = 0;
-            uint32_t qph = 0;
-            while (ok) {
-                int u = total;
-                if (!take_unit(qs, qph, true, &u)) {
-                    report_timeout(args.status);
-                    break;
-                }
-                if (u >= total) break;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, limit)) {
-                        report_timeout(args.status);
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_cluster(peer_relay0 + stage * 8);
-                    if (++stage == S) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
+            // every copy issued lands before either CTA may leave: the even CTA's
+            // barrier counts both CTAs' bytes of every stage it armed; the odd CTA,
+            // which cannot watch that barrier, gives copies it issued after a
+            // time-out a moment to land (the two producers time out on the same
+            // barriers, so the even CTA has armed all the others)
+            if (v == 0) {
+                for (int s = 0; s < S; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait(&full[s], (issued_par >> s) & 1, P_TEARDOWN_NS);
+            } else if (!ok && issued) {
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 100000ull) {
                 }
             }
-        } else if (lane == 0) {
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && v == 0) {
             // ------------------------------------------------------------ MMA issuer (even CTA)
             int stage = 0;
             uint32_t phase = 0;
@@ -437,8 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                 const uint32_t d_tmem = tmem_base + acc * acc_stride;
                 const uint32_t idesc = idesc_bf16_f32(256, x.ntok);
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, limit) ||
-                        !mbar_wait_cl(&relay[stage], phase, limit)) {
+                    if (!mbar_wait_cl(&full[stage], phase, limit)) {
                         report_timeout(args.status);
                         ok = false;
                         break;

@@ -361,6 +361,14 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                 pol_w = l2_policy_evict_first();
                 pol_a = l2_policy_evict_last();
             }
+            // weight gradient: the operand swept fastest (fewer features) is
+            // re-read for every tile of the other, which streams once: keep the
+            // first in L2 ahead of the second
+            uint64_t pol_wg_a = 0, pol_wg_b = 0;
+            if (MODE == TC_WGRAD) {
+                pol_wg_a = args.n_fastest ? l2_policy_evict_first() : l2_policy_evict_last();
+                pol_wg_b = args.n_fastest ? l2_policy_evict_last() : l2_policy_evict_first();
+            }
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_par = 0;  // per-stage bits: loads issued / their parity
@@ -384,12 +392,12 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                             // activations: boxes of 64 features x 64 token rows
 #pragma unroll
                             for (int i = 0; i < BM / 64; ++i)
-                                tma_load_2d(sa + i * 8192, &tm_act, &full[stage],
-                                            x.mt * BM + 64 * i, kc);
+                                tma_load_2d_hint(sa + i * 8192, &tm_act, &full[stage],
+                                                 x.mt * BM + 64 * i, kc, pol_wg_a);
 #pragma unroll
                             for (int i = 0; i < BN / 64; ++i)
-                                tma_load_2d(sb + i * 8192, &tm_w, &full[stage],
-                                            x.nb * BN + 64 * i, kc);
+                                tma_load_2d_hint(sb + i * 8192, &tm_w, &full[stage],
+                                                 x.nb * BN + 64 * i, kc, pol_wg_b);
                         } else {
                             tma_load_2d(sa, &tm_act, &full[stage], kc, x.row0 + x.mt * BM);
                             if (dsplit)  // the same rows' low parts of H
