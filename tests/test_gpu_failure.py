@@ -21,6 +21,10 @@ SHORT_LIMIT_NS = 5_000_000
 @pytest.mark.parametrize("wl", [
     Workload("swap_timeout", T=100, d=256, h=512, E=6, k=2),            # swapped GEMMs
     Workload("tok_timeout", T=600, d=256, h=384, E=4, k=2, cf=(5, 4)),  # token-major GEMMs
+    # CTA-pair GEMMs: swapped tiles (experts of up to 219 tokens) and token-major
+    # tiles of 256 tokens (experts of over 1024 tokens)
+    Workload("pair_swap_timeout", T=700, d=512, h=384, E=8, k=2, cf=(5, 4), zipf_s=0.8),
+    Workload("pair_tok_timeout", T=1300, d=256, h=384, E=3, k=2, zipf_s=0.3),
 ])
 def test_wait_bound_reports_timeout_and_context_survives(wl):
     inp = host_inputs(wl)
