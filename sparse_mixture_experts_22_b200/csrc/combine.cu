@@ -105,6 +105,13 @@ __global__ void __launch_bounds__(256)
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    // the shared experts' row is requested together with the routed rows
+    float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+    if (ys) {
+        const float* p = ys + t * d + c;
+        sa = __ldg(reinterpret_cast<const float4*>(p));
+        sb = __ldg(reinterpret_cast<const float4*>(p + 4));
+    }
     if (splits == 1) {
         // every kept row's 32 bytes are requested before any is used, so the
         // k loads of a thread are in flight together
@@ -149,11 +156,8 @@ __global__ void __launch_bounds__(256)
         for (int q = 0; q < 8; ++q) acc[q] = fmaf(g[j], v[q], acc[q]);
     }
     if (ys) {
-        const float* p = ys + t * d + c;
-        const float4 a = *reinterpret_cast<const float4*>(p);
-        const float4 b = *reinterpret_cast<const float4*>(p + 4);
-        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+        acc[0] += sa.x; acc[1] += sa.y; acc[2] += sa.z; acc[3] += sa.w;
+        acc[4] += sb.x; acc[5] += sb.y; acc[6] += sb.z; acc[7] += sb.w;
     }
     if (OUT_BF16) {
         uint4 o;
