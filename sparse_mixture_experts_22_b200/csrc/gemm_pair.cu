@@ -212,7 +212,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t v = cluster_ctarank();       // 0: issues the MMAs
-    const int pair = blockIdx.x >> 1;
 
     // accumulator: 128 lanes x nt_max (token-major: 256) columns, twice when it fits
     const int acc_stride = TOK ? 256 : args.nt_max;
@@ -409,7 +408,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             const int kblocks = args.K / PBK;
             int qs = 0;
             uint32_t qph = 0;
-            bool first = true;
             while (ok) {
                 int u = total;
                 if (!take_unit(qs, qph, true, &u)) {
@@ -455,9 +453,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                     }
                 }
                 if (!ok) break;
-                // test hook: the first unit of pair 0 never signals its epilogues
-                const bool withhold = args.test_stall && pair == 0 && first;
-                first = false;
+                // test hook: the pair that takes unit 0 never signals its epilogues
+                // for it (any pair may take it: the units come from a counter)
+                const bool withhold = args.test_stall && u == 0;
                 if (!withhold) umma_commit_pair_both(&acc_full[acc]);
                 if (++acc == n_acc) {
                     acc = 0;
