@@ -75,8 +75,8 @@ def parse():
                    help="capture one step in a CUDA graph and replay it (1 GPU)")
     p.add_argument("--no-pdl", action="store_true",
                    help="launch the forward chain without programmatic dependent launch")
-    p.add_argument("--no-pair", action="store_true",
-                   help="one SM per expert GEMM tile (no CTA pairs)")
+    p.add_argument("--pair", type=int, default=1, choices=[0, 1, 2],
+                   help="CTA-pair GEMM tiles: 0 none, 1 token-major (default), 2 also swapped")
     p.add_argument("--no-overlap", action="store_true",
                    help="shared experts after the routed ones on one stream")
     p.add_argument("--backward", action="store_true",
@@ -540,7 +540,7 @@ def main():
     if args.backward and world > 1:
         raise SystemExit("--backward runs on one GPU")
     B.moe_set_pdl(not args.no_pdl)
-    B.moe_set_pair_tiles(not args.no_pair)
+    B.moe_set_pair_tiles(args.pair)
     B.moe_set_shared_overlap(not args.no_overlap)
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward
     cfg, host, g, W, Wb = build_inputs(wl, rank, world, dev, keep_host=want_cpu,

@@ -475,13 +475,20 @@ MOE_API int moe_launch_count(uint64_t* n);
  * routing runs.  Results are identical either way.  Process-wide. */
 MOE_API int moe_set_pdl(int on);
 
-/* Expert GEMMs whose experts each keep more than 128 and at most 256 tokens
- * (default on): each tile runs as one tcgen05 MMA over a pair of SMs (a
- * cluster of two CTAs), M = 256 weight rows, each SM staging half of the
- * expert's token rows, which leaves room for a deeper load pipeline and a
- * double-buffered accumulator.  Off: one SM per tile.  Results agree within
- * the layer's tolerance (the fp32 sums run in the same order).  Process-wide. */
-MOE_API int moe_set_pair_tiles(int on);
+/* Expert GEMM tiles on pairs of SMs (a cluster of two CTAs running one
+ * tcgen05 MMA, M = 256, each SM staging half of A and half of B), process-wide:
+ *   0  one SM per tile everywhere
+ *   1  (default) token-major tiles of 256 tokens x 256 features on SM pairs
+ *      for expert groups that may hold >= 1024 rows (the large prefill layer,
+ *      a shared expert over a long batch): a third less shared-memory fill per
+ *      flop than the one-SM 128 x 256 tile
+ *   2  also the swapped tiles (weight rows x tokens) of experts that keep
+ *      129..256 tokens on SM pairs -- measured slower than one SM per tile on
+ *      the DeepSeek-V2-style layer (the HBM stream is latency-bound there), so
+ *      off by default
+ * Results are identical in every mode (the fp32 sums run in the same order).
+ * MOE_ERR_ARG for another value. */
+MOE_API int moe_set_pair_tiles(int mode);
 
 /* Shared experts beside the routed ones in moe_forward (default on): they
  * need only x, so they run on a second stream (one per device, created by the

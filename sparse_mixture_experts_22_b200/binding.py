@@ -367,8 +367,14 @@ def moe_set_pdl(on: bool):
     _check(load().moe_set_pdl(1 if on else 0))
 
 
-def moe_set_pair_tiles(on: bool):
-    _check(load().moe_set_pair_tiles(1 if on else 0))
+def moe_set_pair_tiles(mode):
+    """0 none, 1 token-major pair tiles (default), 2 also swapped pair tiles;
+    True means 2 (every pair tile), False 0."""
+    if mode is True:
+        mode = 2
+    elif mode is False:
+        mode = 0
+    _check(load().moe_set_pair_tiles(int(mode)))
 
 
 def moe_set_shared_overlap(on: bool):

@@ -300,7 +300,9 @@ static int tmap_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
 
 static int g_pdl_enabled = 1;
 static thread_local bool g_pdl_in_forward = false;
-static int g_pair_enabled = 1;  // swapped tiles of more than 128 tokens on CTA pairs
+// CTA-pair GEMM tiles: 0 none, 1 token-major tiles of groups that may hold
+// >= PAIR_TOK_MIN_TOKENS rows, 2 also swapped tiles of groups of 129..256 rows
+static int g_pair_enabled = 1;
 
 bool pdl_active() { return g_pdl_enabled && g_pdl_in_forward; }
 
@@ -630,11 +632,11 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.aux_ld = 2 * (int64_t)hid;
     // groups of more than 128 (and at most 256) tokens: swapped tiles on CTA
     // pairs, each SM staging half of the token rows
-    const bool pair = !tok && g_pair_enabled && nt_max > DOWN_SWAP_MAX_TOKENS;
+    const bool pair = !tok && g_pair_enabled >= 2 && nt_max > DOWN_SWAP_MAX_TOKENS;
     // groups that may hold thousands of tokens: token-major tiles of 256 tokens on
     // CTA pairs (a third less shared-memory fill per flop; the 256-row tiles pad
     // an expert's rows more than 128-row tiles, which pays off for large groups)
-    const bool pair_tok = tok && g_pair_enabled && nt_max >= PAIR_TOK_MIN_TOKENS &&
+    const bool pair_tok = tok && g_pair_enabled >= 1 && nt_max >= PAIR_TOK_MIN_TOKENS &&
                           hid % 128 == 0 && P.d % 256 == 0;
     if (pair_tok) {
         MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 128));
@@ -1674,8 +1676,9 @@ int moe_set_pdl(int on) {
     return ok();
 }
 
-int moe_set_pair_tiles(int on) {
-    g_pair_enabled = on ? 1 : 0;
+int moe_set_pair_tiles(int mode) {
+    if (mode < 0 || mode > 2) return fail(MOE_ERR_ARG, "mode must be 0, 1 or 2");
+    g_pair_enabled = mode;
     return ok();
 }
 

@@ -35,12 +35,14 @@ def test_wait_bound_reports_timeout_and_context_survives(wl):
 
     B.moe_set_wait_limit_ns(SHORT_LIMIT_NS)
     B.moe_set_test_stall(True)
+    B.moe_set_pair_tiles(2)  # the swapped pair tiles too
     try:
         bad = run_forward(cfg, g, W)
         status = B.moe_read_device_status(bad["ws"])
     finally:
         B.moe_set_test_stall(False)
         B.moe_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+        B.moe_set_pair_tiles(1)
     assert status == 7  # MOE_ERR_TIMEOUT
 
     # the context still works and the layer gives the same bits again

@@ -247,14 +247,14 @@ def test_pair_tiles_match_single_sm_tiles(name):
     r = oracle_route(wl, inp)
     ref = oracle_rows(wl, inp, r)
     cfg, g, W = device_layer(wl, inp)
-    B.moe_set_pair_tiles(True)
-    a = run_forward(cfg, g, W)
-    out_pair = a["out"].clone()
     try:
-        B.moe_set_pair_tiles(False)
+        B.moe_set_pair_tiles(2)  # every pair tile, the swapped ones included
+        a = run_forward(cfg, g, W)
+        out_pair = a["out"].clone()
+        B.moe_set_pair_tiles(0)
         b = run_forward(cfg, g, W)
     finally:
-        B.moe_set_pair_tiles(True)
+        B.moe_set_pair_tiles(1)
     assert B.moe_read_device_status(b["ws"]) == 0
     assert torch.equal(a["slot_of"], b["slot_of"])
     e1 = check_output(out_pair, ref, strict=strict_output(cfg))
