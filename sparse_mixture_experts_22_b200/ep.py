@@ -275,14 +275,17 @@ class Rank:
                               b["offsets"], b["perm_token"], b["slot_of"], b["x_perm"], b["ws"])
         return b["x_perm"][:int(plan.seg[self.rank].sum())]
 
-    def ffn(self, plan: Plan, recv: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    def ffn(self, plan: Plan, recv: torch.Tensor, y: Optional[torch.Tensor] = None,
+            bound: Optional[int] = None) -> torch.Tensor:
+        """Step 4 on the host plan's groups; `bound` (default: the largest group)
+        is the bound on a group's rows that picks the GEMM layout."""
         rows, off, wi = plan.groups(self.rank)
         dev = self.x.device
         if y is None:
             y = torch.empty((recv.shape[0], self.wl.d), dtype=torch.float32, device=dev)
         if recv.shape[0] == 0:
             return y
-        mx = int(rows.max()) if rows.size else 0
+        mx = bound if bound is not None else (int(rows.max()) if rows.size else 0)
         ws = torch.empty(B.moe_grouped_workspace_size(self.cfg, recv.shape[0], mx),
                          dtype=torch.uint8, device=dev)
         B.moe_expert_ffn_grouped(self.cfg, recv, recv.shape[0], torch.from_numpy(rows).to(dev),
@@ -403,11 +406,12 @@ def forward_emulated(ranks: List[Rank], T_all: int):
     return outs, stats, plan
 
 
-def forward_emulated_peers(ranks: List[Rank], T_all: int):
+def forward_emulated_peers(ranks: List[Rank], T_all: int, bound: Optional[int] = None):
     """The peer-memory form with G ranks in one process on one device: every
     rank's receive and output buffers live on that device, and the ranks'
     kernels run one after another in stream order (which stands in for the
-    barriers).  Returns ([out per rank], stats tensor, plan)."""
+    barriers).  `bound`: as Rank.ffn.  Returns ([out per rank], stats tensor,
+    plan)."""
     G = len(ranks)
     counts = np.stack([r.route().cpu().numpy() for r in ranks]).astype(np.int64)
     wl = ranks[0].wl
@@ -417,7 +421,8 @@ def forward_emulated_peers(ranks: List[Rank], T_all: int):
                         device=dev) for q in range(G)]
     for r in ranks:
         r.dispatch_peers(plan, [t.data_ptr() for t in recv])
-    ys = [ranks[q].ffn(plan, recv[q][:int(plan.recv_rows(q).sum())]) for q in range(G)]
+    ys = [ranks[q].ffn(plan, recv[q][:int(plan.recv_rows(q).sum())], bound=bound)
+          for q in range(G)]
     ys = [y if y.shape[0] else torch.empty((1, wl.d), dtype=torch.float32, device=dev)
           for y in ys]
     outs = [r.combine_peers(plan, [y.data_ptr() for y in ys]) for r in ranks]
