@@ -58,6 +58,8 @@ def parse():
                    help="how H reaches the down projection (moe_config.hidden_mode)")
     p.add_argument("--no-decode", action="store_true",
                    help="skip the decode layer timed after the main workload")
+    p.add_argument("--no-split-line", action="store_true",
+                   help="skip the same workload timed with H split (when the run's H is bf16)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -264,6 +266,48 @@ def decode_line(args, dev, stream, wl_main, W_main):
             "layer_roofline": {"flops": flops, "bytes": byts, "time_us": roof_t * 1e6,
                                "frac": roof_t / t_step, "kept_assignments": N,
                                "active_experts": active},
+            "clocks": clk, "device_status": status}
+
+
+def split_line(args, dev, stream, wl, g, W):
+    """The same workload timed with H fed to the down projection as two bf16
+    parts (the mode whose output meets the relative-L1 bar against the
+    unrounded fp64 reference), same inputs and weights, device-resident."""
+    cfg = B.config_of(wl, hidden="split")
+    W13, W2p, W13s, W2s = W
+    bufs = B.alloc_layer(cfg, dev)
+
+    def step():
+        B.moe_forward(cfg, g["x"], g["Wr"], g["bias"], W13, W2p, W13s, W2s, bufs["out"],
+                      bufs["topk_idx"], bufs["topk_gate"], bufs["routed"], bufs["kept"],
+                      bufs["slot_of"], bufs["stats"], bufs["ws"])
+
+    steps = max(5, min(args.steps, 20))
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    kept = bufs["kept"].cpu().tolist()
+    pk, _ = peaks()
+    flops, byts, N, active = algorithmic(wl, kept)
+    t_step = ms / 1000.0 / steps
+    roof_t = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    status = B.moe_read_device_status(bufs["ws"])
+    del bufs
+    return {"hidden": "split", "value": wl.T * steps / (ms / 1000.0), "unit": UNIT,
+            "steps": steps, "ms_per_step": ms / steps,
+            "layer_roofline": {"frac": roof_t / t_step, "time_us": roof_t * 1e6},
             "clocks": clk, "device_status": status}
 
 
@@ -764,6 +808,9 @@ def main():
     if (world == 1 and not args.backward and not args.no_decode and wl.name != "decode"
             and not args.graph and not args.hidden):
         line["decode"] = decode_line(args, dev, stream, wl, W)
+    if (world == 1 and not args.backward and not args.no_split_line and not args.graph
+            and not B.moe_hidden_split(cfg) and wl.dtype == "bf16"):
+        line["split_hidden"] = split_line(args, dev, stream, wl, g, W)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
