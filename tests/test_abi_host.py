@@ -174,3 +174,30 @@ def test_binding_refuses_host_and_strided_tensors():
     with pytest.raises(ValueError):
         B._p(torch.zeros(4))
     assert B._p(None) is None
+
+
+def test_pair_tile_mode_is_checked():
+    lib = B.load()
+    assert lib.moe_set_pair_tiles(3) == 1
+    assert lib.moe_set_pair_tiles(-1) == 1
+    assert lib.moe_set_pair_tiles(1) == 0  # the default, restored
+
+
+def test_hidden_mode_is_checked_and_reported():
+    cfg = M.make_config(64, 128, 128, 8, 2)
+    assert M.moe_hidden_split(cfg)          # auto: every expert keeps <= 128 rows
+    cfg_big = M.make_config(4096, 128, 128, 8, 2)
+    assert not M.moe_hidden_split(cfg_big)  # auto: experts of up to 4096 rows
+    assert M.moe_hidden_split(M.make_config(4096, 128, 128, 8, 2, hidden="split"))
+    assert not M.moe_hidden_split(M.make_config(64, 128, 128, 8, 2, hidden="bf16"))
+    assert not M.moe_hidden_split(M.make_config(64, 128, 128, 8, 2, dtype="f32",
+                                                hidden="split"))
+    cfg.hidden_mode = 3
+    with pytest.raises(B.MoEError) as e:
+        M.moe_workspace_size(cfg)
+    assert e.value.code == 1
+    # the split doubles the hidden activations' share of the workspace
+    a = M.moe_workspace_size(M.make_config(4096, 128, 256, 8, 2, hidden="bf16"))
+    b = M.moe_workspace_size(M.make_config(4096, 128, 256, 8, 2, hidden="split"))
+    rows = M.moe_perm_rows(M.make_config(4096, 128, 256, 8, 2))
+    assert b - a >= rows * 256 * 2
