@@ -714,6 +714,30 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         return MOE_OK;
     }
     const bool dtok = tok || nt_max > DOWN_SWAP_MAX_TOKENS;
+    // groups of 129..256 tokens (swapped gate/up): the down projection on the
+    // token-major CTA-pair tile, one pair unit per expert and 256 output features,
+    // each SM streaming its own 128 weight rows (6 stages of 16 KB) rather than
+    // two one-SM m tiles sharing a 256-row weight tile through L2
+    if (!tok && dtok && g_pair_enabled >= 1 && P.d % 256 == 0 && hid % 128 == 0) {
+        MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 128));
+        MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
+        a.K = hid;
+        a.n_feat = P.d;
+        a.w_rows_per_group = P.d;
+        a.splits = 1;
+        a.out = y;
+        a.out_ld = P.d;
+        a.split_stride = act_rows * (int64_t)P.d;
+        a.aux = nullptr;
+        a.prefetch_kb = 0;
+        a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, nt_max, groups, P.split, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
+        trace_pre(st, tag2);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, st), tag2));
+        trace_mark(st, tag2);
+        return MOE_OK;
+    }
     const int mode2 = dtok ? TC_DOWN_TOK : TC_DOWN_SWAP;
     const int bn = (P.d % 256 == 0) ? 256 : 128;
     MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, dtok ? 128 : 16));
