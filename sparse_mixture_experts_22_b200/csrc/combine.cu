@@ -46,7 +46,7 @@ __device__ void finalize_stats(const double* sums, int E, int k, moe_stats* st) 
 // sums = [T, entropy sum, P sums (E), routed (E), kept (E)], each a fixed-order
 // fp64 reduction of the router's per-block partials; then the statistics.
 // Run by one block of any size.
-__device__ void stats_block(const StatsParams& a) {
+__device__ __noinline__ void stats_block(const StatsParams& a) {
     const float* ppart = a.ppart;
     const float* hpart = a.hpart;
     const int nblk = a.nblk, E = a.E, k = a.k;
@@ -78,7 +78,9 @@ __global__ void stats_kernel(StatsParams a) { stats_block(a); }
 
 // The last block of the grid computes the statistics instead when
 // sp.sums is set (they need only the router partials and the counts).
-template <bool OUT_BF16>
+// KMAX >= k bounds the per-thread arrays: sized for the config's k, the
+// kernel keeps few registers and many threads (so many row loads) in flight.
+template <bool OUT_BF16, int KMAX>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ y, int splits, int64_t split_stride,
                    const int32_t* __restrict__ slot_of, const float* __restrict__ gate,
@@ -95,10 +97,10 @@ __global__ void __launch_bounds__(256)
     const int64_t t = i / vecs;
     const int c = (int)(i % vecs) * 8;
     // all slots and gates first, so that every row load below is independent
-    int32_t slot[MAX_K];
-    float g[MAX_K];
+    int32_t slot[KMAX];
+    float g[KMAX];
 #pragma unroll
-    for (int j = 0; j < MAX_K; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         slot[j] = j < k ? slot_of[t * k + j] : -1;
         g[j] = j < k ? gate[t * k + j] : 0.f;
     }
@@ -115,9 +117,9 @@ __global__ void __launch_bounds__(256)
     if (splits == 1) {
         // every kept row's 32 bytes are requested before any is used, so the
         // k loads of a thread are in flight together
-        float4 ra[MAX_K], rb[MAX_K];
+        float4 ra[KMAX], rb[KMAX];
 #pragma unroll
-        for (int j = 0; j < MAX_K; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
             ra[j] = make_float4(0.f, 0.f, 0.f, 0.f);
             rb[j] = ra[j];
             if (slot[j] >= 0) {
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(256)
             }
         }
 #pragma unroll
-        for (int j = 0; j < MAX_K; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
             if (slot[j] < 0) continue;
             acc[0] = fmaf(g[j], ra[j].x, acc[0]);
             acc[1] = fmaf(g[j], ra[j].y, acc[1]);
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(256)
         }
     }
 #pragma unroll
-    for (int j = 0; j < MAX_K; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         if (splits == 1 || slot[j] < 0) continue;
         float v[8];
 #pragma unroll
@@ -308,12 +310,16 @@ int launch_combine(const float* y, int splits, int64_t split_stride, const int32
     memset(&none, 0, sizeof none);
     const StatsParams& s = sp ? *sp : none;
     const unsigned blocks = (unsigned)((n + 255) / 256) + (sp ? 1 : 0);
-    if (out_bf16)
-        launch_ex(pdl_active(), combine_kernel<true>, dim3(blocks), dim3(256), 0, st, y, splits,
-                  split_stride, slot_of, gate, y_shared, out, T, d, k, s);
+    auto go = [&](auto kern) {
+        launch_ex(pdl_active(), kern, dim3(blocks), dim3(256), 0, st, y, splits, split_stride,
+                  slot_of, gate, y_shared, out, T, d, k, s);
+    };
+    if (k <= 2)
+        out_bf16 ? go(combine_kernel<true, 2>) : go(combine_kernel<false, 2>);
+    else if (k <= 4)
+        out_bf16 ? go(combine_kernel<true, 4>) : go(combine_kernel<false, 4>);
     else
-        launch_ex(pdl_active(), combine_kernel<false>, dim3(blocks), dim3(256), 0, st, y, splits,
-                  split_stride, slot_of, gate, y_shared, out, T, d, k, s);
+        out_bf16 ? go(combine_kernel<true, MAX_K>) : go(combine_kernel<false, MAX_K>);
     note_launch();
     return launch_result();
 }
