@@ -81,6 +81,9 @@ def parse():
                    help="CTA-pair GEMM tiles: 0 none, 1 token-major (default), 2 also swapped")
     p.add_argument("--no-overlap", action="store_true",
                    help="shared experts after the routed ones on one stream")
+    p.add_argument("--shared-sms", type=int, default=-1,
+                   help="SMs set aside for the shared experts beside the routed ones "
+                        "(-1: the library's default)")
     p.add_argument("--backward", action="store_true",
                    help="time forward + backward (a training step) instead of the forward (1 GPU)")
     return p.parse_args()
@@ -586,6 +589,8 @@ def main():
     B.moe_set_pdl(not args.no_pdl)
     B.moe_set_pair_tiles(args.pair)
     B.moe_set_shared_overlap(not args.no_overlap)
+    if args.shared_sms >= 0:
+        B.moe_set_shared_sms(args.shared_sms)
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward
     cfg, host, g, W, Wb = build_inputs(wl, rank, world, dev, keep_host=want_cpu,
                                        train=args.backward, hidden=args.hidden_mode)
@@ -788,6 +793,8 @@ def main():
                    "tokens_per_rank": wl.T,
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "hidden": "split" if B.moe_hidden_split(cfg) else "bf16",
+                   **({"shared_sms": args.shared_sms}
+                      if wl.n_shared and args.shared_sms >= 0 else {}),
                    "l2": ("inputs larger than L2: the active expert weights "
                           f"({active * 3 * wl.d * wl.h * 2 / 1e9:.2f} GB) stream from HBM "
                           "every step")},

@@ -499,6 +499,18 @@ MOE_API int moe_set_pair_tiles(int mode);
  * routed ones.  Results are identical either way.  Process-wide. */
 MOE_API int moe_set_shared_overlap(int on);
 
+/* SMs set aside for the shared experts while they overlap the routed ones
+ * (default 0: none).  With sms > 0, moe_forward launches the shared experts'
+ * GEMMs with grids of `sms` SMs and the routed experts' GEMMs with grids of
+ * the rest, so that the HBM-bound routed GEMMs and the compute-bound shared
+ * ones run side by side instead of the second starting in the tail of the
+ * first.  Applies only when the overlap is on, the layer has shared experts
+ * and at least 32 SMs remain for the routed ones; the block scheduler decides
+ * where the CTAs land, so this shapes the grids, it does not pin SMs.  Results
+ * are identical for every value.  MOE_ERR_ARG unless sms is even and in
+ * [0, 1024].  Process-wide. */
+MOE_API int moe_set_shared_sms(int sms);
+
 /* Upper bound, in nanoseconds, on every device-side wait of the tensor-core
  * kernels (default 2e9).  A wait that runs out records MOE_ERR_TIMEOUT in
  * the device status word and its kernel returns early.  Process-wide. */

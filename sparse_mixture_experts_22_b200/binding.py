@@ -31,7 +31,7 @@ EXPORTS = ["moe_capacity", "moe_workspace_size", "moe_perm_rows", "moe_ffn_split
            "moe_launch_count", "moe_segment_pad", "moe_route_counts", "moe_dispatch_capped",
            "moe_grouped_workspace_size", "moe_expert_ffn_grouped", "moe_combine_rows", "moe_set_pdl",
            "moe_dispatch_peers", "moe_combine_peers", "moe_hidden_split", "moe_set_pair_tiles",
-           "moe_ep_plan", "moe_set_shared_overlap"]
+           "moe_ep_plan", "moe_set_shared_overlap", "moe_set_shared_sms"]
 
 MOE_MAX_PEERS = 64
 
@@ -110,6 +110,7 @@ def load() -> ctypes.CDLL:
             "moe_set_pdl": [I],
             "moe_set_pair_tiles": [I],
             "moe_set_shared_overlap": [I],
+            "moe_set_shared_sms": [I],
             "moe_expert_ffn_grouped": [C, P, ctypes.c_int64, ctypes.c_int32, P, P, P,
                                        ctypes.c_int32, P, P, P, P, S, P],
             "moe_backward": [C, P, ctypes.c_float, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P,
@@ -379,6 +380,11 @@ def moe_set_pair_tiles(mode):
 
 def moe_set_shared_overlap(on: bool):
     _check(load().moe_set_shared_overlap(1 if on else 0))
+
+
+def moe_set_shared_sms(sms: int):
+    """SMs set aside for the shared experts beside the routed ones (0: none)."""
+    _check(load().moe_set_shared_sms(int(sms)))
 
 
 def moe_set_wait_limit_ns(ns: int):

@@ -645,7 +645,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
         trace_pre(st, tag1);
-        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP_TOK, m_act, m_w, a, st), tag1));
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP_TOK, m_act, m_w, a, dv.sms / 2, st), tag1));
         trace_mark(st, tag1);
         MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 128));
         MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
@@ -662,7 +662,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
         trace_pre(st, tag2);
-        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, st), tag2));
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, dv.sms / 2, st), tag2));
         trace_mark(st, tag2);
         return MOE_OK;
     }
@@ -673,7 +673,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
         trace_pre(st, tag1);
-        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP, m_act, m_w, a, st), tag1));
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP, m_act, m_w, a, dv.sms / 2, st), tag1));
         trace_mark(st, tag1);
     } else {
         a.stages = tc_max_stages(mode1, 256, nt_max, groups, false, smem_limit);
@@ -709,7 +709,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
         trace_pre(st, tag2);
-        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN, m_act, m_w, a, st), tag2));
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN, m_act, m_w, a, dv.sms / 2, st), tag2));
         trace_mark(st, tag2);
         return MOE_OK;
     }
@@ -734,7 +734,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
         trace_pre(st, tag2);
-        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, st), tag2));
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, dv.sms / 2, st), tag2));
         trace_mark(st, tag2);
         return MOE_OK;
     }
@@ -850,6 +850,7 @@ static int side_stream(SideStream* out) {
 }
 
 static int g_shared_overlap = 1;
+static int g_shared_sms = 0;  // SMs set aside for the shared experts (0: none)
 
 static StatsParams stats_params(const Plan& P, const int32_t* routed, const int32_t* kept,
                                 const void* ws, double* sums, moe_stats* stats) {
@@ -1263,6 +1264,15 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
     // being timed, whose events assume one stream.)
     const bool side = P.T > 0 && P.S > 0 && P.bf16 && g_shared_overlap &&
                       !(g_trace.on && g_trace.only.empty());
+    // With SMs set aside for them, the shared experts' GEMMs take that many SMs
+    // and the routed experts' the rest, so that the two run side by side (the
+    // routed GEMMs stream weights from HBM; the shared ones are compute-bound)
+    // rather than one in the tail of the other.
+    Device dv_routed = dv, dv_shared = dv;
+    if (side && g_shared_sms > 0 && g_shared_sms <= dv.sms - 32) {
+        dv_shared.sms = g_shared_sms;
+        dv_routed.sms = dv.sms - g_shared_sms;
+    }
     SideStream ss;
     if (side) {
         MOE_TRY(side_stream(&ss));
@@ -1270,7 +1280,7 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
             cudaStreamWaitEvent(ss.st, ss.fork, 0) != cudaSuccess)
             return fail(MOE_ERR_CUDA, "could not fork the shared-expert stream");
         g_pdl_in_forward = false;  // the first launch on the side stream follows an event
-        const int rc = step_shared_ffn(P, dv, x, W13s, W2s, ys, ws, ss.st);
+        const int rc = step_shared_ffn(P, dv_shared, x, W13s, W2s, ys, ws, ss.st);
         g_pdl_in_forward = true;
         MOE_TRY(rc);
         if (cudaEventRecord(ss.join, ss.st) != cudaSuccess)
@@ -1278,7 +1288,8 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
     }
     MOE_TRY(step_route_dispatch(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate,
                                 routed, kept, offsets, perm, slot_of, x_perm, ws, st));
-    MOE_TRY(step_ffn(P, dv, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st, !side));
+    MOE_TRY(step_ffn(P, dv_routed, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st,
+                     !side));
     if (side && cudaStreamWaitEvent(st, ss.join, 0) != cudaSuccess)
         return fail(MOE_ERR_CUDA, "could not join the shared-expert stream");
     // combine, with the statistics computed by one extra block of the same launch
@@ -1708,6 +1719,13 @@ int moe_set_pair_tiles(int mode) {
 
 int moe_set_shared_overlap(int on) {
     g_shared_overlap = on ? 1 : 0;
+    return ok();
+}
+
+int moe_set_shared_sms(int sms) {
+    if (sms < 0 || sms > 1024 || sms % 2)
+        return fail(MOE_ERR_ARG, "sms must be an even count in [0, 1024]");
+    g_shared_sms = sms;
     return ok();
 }
 

@@ -644,18 +644,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     if (warp == 1) tmem_dealloc_pair(tmem_base, tmem_cols);
 }
 
-// One pair per two SMs: the pairs take their units from a counter, so any that
-// are not resident at once only start later and find less work.
-int pair_grid() {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 0;
-    return sms / 2;
-}
-
 template <int MODE>
-int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
+int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, int pairs,
                      cudaStream_t st) {
     const PairLayout L =
         pair_layout(MODE, a.nt_max, a.stages, a.num_groups,
@@ -675,7 +665,6 @@ int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs&
             configured_bytes[dev] = L.total;
         }
     }
-    const int pairs = pair_grid();
     if (pairs < 1 || !a.unit_ctr) {
         last_launch_error() = cudaErrorInvalidConfiguration;
         return -1;
@@ -696,17 +685,17 @@ int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_li
 }
 
 int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
-                   cudaStream_t st) {
+                   int pairs, cudaStream_t st) {
     if (!p_tok(mode) && (a.nt_max < 16 || a.nt_max > 256 || a.nt_max % 16)) return -1;
     switch (mode) {
         case TC_PAIR_GATEUP:
-            return launch_pair_mode<TC_PAIR_GATEUP>(act, w, a, st);
+            return launch_pair_mode<TC_PAIR_GATEUP>(act, w, a, pairs, st);
         case TC_PAIR_DOWN:
-            return launch_pair_mode<TC_PAIR_DOWN>(act, w, a, st);
+            return launch_pair_mode<TC_PAIR_DOWN>(act, w, a, pairs, st);
         case TC_PAIR_GATEUP_TOK:
-            return launch_pair_mode<TC_PAIR_GATEUP_TOK>(act, w, a, st);
+            return launch_pair_mode<TC_PAIR_GATEUP_TOK>(act, w, a, pairs, st);
         case TC_PAIR_DOWN_TOK:
-            return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, a, st);
+            return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, a, pairs, st);
     }
     return -1;
 }

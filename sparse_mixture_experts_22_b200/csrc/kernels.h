@@ -182,10 +182,12 @@ int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& 
 // w = W2p, 128-row boxes; n_feat = model width, a multiple of 256); nt_max is a
 // multiple of 16 in [16, 256].  Token-major, for groups of any size:
 // TC_PAIR_GATEUP_TOK and TC_PAIR_DOWN_TOK (act and w both 128-row boxes).  The
-// grid is as many pairs as the device holds at once.
+// grid is `pairs` clusters of two CTAs (one per two SMs); the pairs take their
+// units from a counter, so pairs that are not resident at once only start
+// later and find less work.
 int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_limit);
 int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
-                   cudaStream_t st);
+                   int pairs, cudaStream_t st);
 
 // ---------------------------------------------------------------- fp32 SIMT FFN
 // gate/up: H[r][f] = silu(A_r . W13[g][gate f]) * (A_r . W13[g][up f]);

@@ -183,6 +183,15 @@ def test_pair_tile_mode_is_checked():
     assert lib.moe_set_pair_tiles(1) == 0  # the default, restored
 
 
+def test_shared_sm_budget_is_checked():
+    lib = B.load()
+    assert lib.moe_set_shared_sms(3) == 1      # odd: SMs go in pairs
+    assert lib.moe_set_shared_sms(-2) == 1
+    assert lib.moe_set_shared_sms(2048) == 1
+    assert lib.moe_set_shared_sms(24) == 0
+    assert lib.moe_set_shared_sms(0) == 0      # the default, restored
+
+
 def test_hidden_mode_is_checked_and_reported():
     cfg = M.make_config(64, 128, 128, 8, 2)
     assert M.moe_hidden_split(cfg)          # auto: every expert keeps <= 128 rows

@@ -280,6 +280,14 @@ def test_shared_overlap_gives_identical_bits(name):
         B.moe_set_shared_overlap(True)
     assert torch.equal(out_on, b["out"])
     assert B.moe_read_device_status(b["ws"]) == 0
+    # SMs set aside for the shared experts: the grids change, the bits do not
+    try:
+        B.moe_set_shared_sms(24)
+        c = run_forward(cfg, g, W)
+    finally:
+        B.moe_set_shared_sms(0)
+    assert torch.equal(out_on, c["out"])
+    assert B.moe_read_device_status(c["ws"]) == 0
     r = oracle_route(wl, inp)
     check_output(out_on, oracle_rows(wl, inp, r), strict=strict_output(cfg))
 
