@@ -481,13 +481,17 @@ MOE_API int moe_set_pdl(int on);
  *   1  (default) token-major tiles of 256 tokens x 256 features on SM pairs
  *      for expert groups that may hold >= 1024 rows (the large prefill layer,
  *      a shared expert over a long batch): a third less shared-memory fill per
- *      flop than the one-SM 128 x 256 tile
- *   2  also the swapped tiles (weight rows x tokens) of experts that keep
- *      129..256 tokens on SM pairs -- measured slower than one SM per tile on
- *      the DeepSeek-V2-style layer (the HBM stream is latency-bound there), so
- *      off by default
- * Results are identical in every mode (the fp32 sums run in the same order).
- * MOE_ERR_ARG for another value. */
+ *      flop than the one-SM 128 x 256 tile; and the down projection of groups
+ *      of 129..256 tokens (one pair tile per 256 output features, each weight
+ *      row read once)
+ *   2  also the swapped gate/up and down tiles (weight rows x tokens) of
+ *      experts that keep 129..256 tokens on SM pairs -- measured slower than
+ *      one SM per tile on the DeepSeek-V2-style layer (the HBM stream is
+ *      latency-bound there), so off by default
+ *   3  as 1, and the gate/up of groups of 129..256 tokens on token-major pair
+ *      tiles too (in place of the one-SM swapped tile)
+ * Every mode gives the same routing bits and an output within the same
+ * tolerance of the exact layer.  MOE_ERR_ARG for another value. */
 MOE_API int moe_set_pair_tiles(int mode);
 
 /* Shared experts beside the routed ones in moe_forward (default on): they

@@ -237,18 +237,20 @@ def test_full_size_workload(name, hidden):
     print(f"{name} ({hidden} H, {len(rows)} rows): {e} logit_err={zerr:.2e}")
 
 
+@pytest.mark.parametrize("mode", [2, 3])
 @pytest.mark.parametrize("name", ["pair_tiles", "pair_shared", "swap_cap", "pair_tok"])
-def test_pair_tiles_match_single_sm_tiles(name):
-    """Experts of more than 128 tokens run their GEMMs on CTA pairs; the same
-    layer with one SM per tile gives the same output within the bar, and the
-    same routing bit for bit."""
+def test_pair_tiles_match_single_sm_tiles(name, mode):
+    """Experts of more than 128 tokens run their GEMMs on CTA pairs (mode 2:
+    swapped pair tiles for groups of 129..256 tokens; mode 3: token-major pair
+    tiles for them); the same layer with one SM per tile gives the same output
+    within the bar, and the same routing bit for bit."""
     wl = SMALL[name]
     inp = host_inputs(wl)
     r = oracle_route(wl, inp)
     ref = oracle_rows(wl, inp, r)
     cfg, g, W = device_layer(wl, inp)
     try:
-        B.moe_set_pair_tiles(2)  # every pair tile, the swapped ones included
+        B.moe_set_pair_tiles(mode)
         a = run_forward(cfg, g, W)
         out_pair = a["out"].clone()
         B.moe_set_pair_tiles(0)
@@ -260,7 +262,7 @@ def test_pair_tiles_match_single_sm_tiles(name):
     e1 = check_output(out_pair, ref, strict=strict_output(cfg))
     e2 = check_output(b["out"], ref, strict=strict_output(cfg))
     d = (out_pair.float() - b["out"].float()).abs().max().item()
-    print(f"{name}: pair {e1} single {e2} max|pair - single| {d:.3e}")
+    print(f"{name} mode {mode}: pair {e1} single {e2} max|pair - single| {d:.3e}")
 
 
 @pytest.mark.parametrize("name", ["shared", "shared_small", "pair_shared", "shared_swap64"])
