@@ -77,9 +77,8 @@ def parse():
                    help="capture one step in a CUDA graph and replay it (1 GPU)")
     p.add_argument("--no-pdl", action="store_true",
                    help="launch the forward chain without programmatic dependent launch")
-    p.add_argument("--pair", type=int, default=1, choices=[0, 1, 2, 3],
-                   help="CTA-pair GEMM tiles: 0 none, 1 token-major (default), 2 also swapped, "
-                        "3 token-major also for experts of 129..256 tokens")
+    p.add_argument("--pair", type=int, default=1, choices=[0, 1, 2],
+                   help="CTA-pair GEMM tiles: 0 none, 1 token-major (default), 2 also swapped")
     p.add_argument("--no-overlap", action="store_true",
                    help="shared experts after the routed ones on one stream")
     p.add_argument("--shared-sms", type=int, default=-1,

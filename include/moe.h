@@ -488,10 +488,8 @@ MOE_API int moe_set_pdl(int on);
  *      experts that keep 129..256 tokens on SM pairs -- measured slower than
  *      one SM per tile on the DeepSeek-V2-style layer (the HBM stream is
  *      latency-bound there), so off by default
- *   3  as 1, and the gate/up of groups of 129..256 tokens on token-major pair
- *      tiles too (in place of the one-SM swapped tile)
- * Every mode gives the same routing bits and an output within the same
- * tolerance of the exact layer.  MOE_ERR_ARG for another value. */
+ * Results are identical in every mode (the fp32 sums run in the same order).
+ * MOE_ERR_ARG for another value. */
 MOE_API int moe_set_pair_tiles(int mode);
 
 /* Shared experts beside the routed ones in moe_forward (default on): they

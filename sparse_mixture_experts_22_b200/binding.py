@@ -369,9 +369,8 @@ def moe_set_pdl(on: bool):
 
 
 def moe_set_pair_tiles(mode):
-    """0 none, 1 token-major pair tiles (default), 2 also swapped pair tiles,
-    3 token-major pair tiles also for the gate/up of groups of 129..256 tokens;
-    True means 2, False 0."""
+    """0 none, 1 token-major pair tiles (default), 2 also swapped pair tiles;
+    True means 2 (every pair tile), False 0."""
     if mode is True:
         mode = 2
     elif mode is False:

@@ -632,16 +632,12 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     a.aux_ld = 2 * (int64_t)hid;
     // groups of more than 128 (and at most 256) tokens: swapped tiles on CTA
     // pairs, each SM staging half of the token rows
-    const bool pair = !tok && g_pair_enabled == 2 && nt_max > DOWN_SWAP_MAX_TOKENS;
+    const bool pair = !tok && g_pair_enabled >= 2 && nt_max > DOWN_SWAP_MAX_TOKENS;
     // groups that may hold thousands of tokens: token-major tiles of 256 tokens on
     // CTA pairs (a third less shared-memory fill per flop; the 256-row tiles pad
-    // an expert's rows more than 128-row tiles, which pays off for large groups);
-    // in mode 3 also groups of 129..256 tokens (one m tile each) in place of the
-    // swapped tiles
-    const bool mid_tok = !tok && g_pair_enabled == 3 && nt_max > DOWN_SWAP_MAX_TOKENS;
-    const bool pair_tok =
-        ((tok && g_pair_enabled >= 1 && nt_max >= PAIR_TOK_MIN_TOKENS) || mid_tok) &&
-        hid % 128 == 0 && P.d % 256 == 0;
+    // an expert's rows more than 128-row tiles, which pays off for large groups)
+    const bool pair_tok = tok && g_pair_enabled >= 1 && nt_max >= PAIR_TOK_MIN_TOKENS &&
+                          hid % 128 == 0 && P.d % 256 == 0;
     if (pair_tok) {
         MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 128));
         MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 128));
@@ -1716,7 +1712,7 @@ int moe_set_pdl(int on) {
 }
 
 int moe_set_pair_tiles(int mode) {
-    if (mode < 0 || mode > 3) return fail(MOE_ERR_ARG, "mode must be 0, 1, 2 or 3");
+    if (mode < 0 || mode > 2) return fail(MOE_ERR_ARG, "mode must be 0, 1 or 2");
     g_pair_enabled = mode;
     return ok();
 }

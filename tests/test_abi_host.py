@@ -178,9 +178,8 @@ def test_binding_refuses_host_and_strided_tensors():
 
 def test_pair_tile_mode_is_checked():
     lib = B.load()
-    assert lib.moe_set_pair_tiles(4) == 1
+    assert lib.moe_set_pair_tiles(3) == 1
     assert lib.moe_set_pair_tiles(-1) == 1
-    assert lib.moe_set_pair_tiles(3) == 0
     assert lib.moe_set_pair_tiles(1) == 0  # the default, restored
 
 
