@@ -892,12 +892,14 @@ static int step_stats(const Plan& P, const int32_t* routed, const int32_t* kept,
 // ---------------------------------------------------------------- backward steps
 
 // Backward GEMMs of one set of groups: dAB = SiLU*mul backward of dY W2t^T
-// (bf16, interleaved like AB), then dX = dAB W13t^T (fp32).
+// (bf16, interleaved like AB), then dX = dAB W13t^T (fp32).  nt_max bounds a
+// group's rows: groups that may hold 1024+ rows take dX on CTA-pair tiles, as
+// the forward's down projection does.
 static int run_tc_backward(const Plan& P, const Device& dv, int groups, const int32_t* rows,
                            const int32_t* offs, int dense_rows, int64_t act_rows, const void* dY,
                            const void* W2t, const void* AB, void* dAB, const void* W13t,
-                           float* dX, int hid, int32_t* status, cudaStream_t st, const char* tag1,
-                           const char* tag2) {
+                           float* dX, int hid, int64_t nt_max, int32_t* status, cudaStream_t st,
+                           const char* tag1, const char* tag2, int ctr_slot) {
     CUtensorMap m_act, m_w;
     TcArgs a;
     memset(&a, 0, sizeof a);
@@ -928,14 +930,27 @@ static int run_tc_backward(const Plan& P, const Device& dv, int groups, const in
     trace_mark(st, tag1);
 
     const int bn2 = P.d % 256 == 0 ? 256 : 128;
-    MOE_TRY(tmap_bf16(&m_act, dAB, act_rows, 2 * hid, 128));
-    MOE_TRY(tmap_bf16(&m_w, W13t, (int64_t)groups * P.d, 2 * hid, bn2));
     a.K = 2 * hid;
     a.n_feat = P.d;
     a.w_rows_per_group = P.d;
     a.out = dX;
     a.out_ld = P.d;
     a.aux = nullptr;
+    if (g_pair_enabled >= 1 && nt_max >= PAIR_TOK_MIN_TOKENS && P.d % 256 == 0) {
+        MOE_TRY(tmap_bf16(&m_act, dAB, act_rows, 2 * hid, 128));
+        MOE_TRY(tmap_bf16(&m_w, W13t, (int64_t)groups * P.d, 2 * hid, 128));
+        a.unit_ctr = status + UNIT_CTR_WORD + ctr_slot;
+        a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, 256, groups, false, dv.smem_optin);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        if (cudaMemsetAsync(a.unit_ctr, 0, sizeof(int32_t), st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "memset failed");
+        trace_pre(st, tag2);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, dv.sms / 2, st), tag2));
+        trace_mark(st, tag2);
+        return MOE_OK;
+    }
+    MOE_TRY(tmap_bf16(&m_act, dAB, act_rows, 2 * hid, 128));
+    MOE_TRY(tmap_bf16(&m_w, W13t, (int64_t)groups * P.d, 2 * hid, bn2));
     a.stages = tc_max_stages(TC_DOWN_TOK, bn2, 16, groups, false, dv.smem_optin);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag2);
@@ -1641,7 +1656,7 @@ int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef, co
 
     // routed experts: dAB, dX, then the weight gradients over each expert's tokens
     MOE_TRY(run_tc_backward(P, dv, E, kept, offsets, 0, P.perm_rows, dY, W2t, AB, dAB, W13t, dXp, h,
-                            status, st, "gemm_dgate", "gemm_dx"));
+                            P.nt_max, status, st, "gemm_dgate", "gemm_dx", 0));
     // the rows between each expert's tokens and the next multiple of 64 are
     // zeroed in the four activations the weight gradients contract
     PadJobs pj;
@@ -1669,8 +1684,8 @@ int moe_backward(const moe_config* cfg, const void* grad_out, float aux_coef, co
         void* dABs = at<void>(bws, P.b_dABs);
         dXs = at<float>(bws, P.b_dXs);
         MOE_TRY(run_tc_backward(P, dv, 1, nullptr, nullptr, (int)T, T, grad_out, W2st, ABs, dABs,
-                                W13st, dXs, P.hsum, status, st, "gemm_shared_dgate",
-                                "gemm_shared_dx"));
+                                W13st, dXs, P.hsum, T, status, st, "gemm_shared_dgate",
+                                "gemm_shared_dx", 1));
         MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, nullptr, (int)T, T, grad_out, d, Hs, P.hsum,
                              dW2s, status, st, "gemm_shared_dw2"));
         MOE_TRY(run_tc_wgrad(P, dv, 1, nullptr, nullptr, (int)T, T, dABs, 2 * P.hsum, x, d,

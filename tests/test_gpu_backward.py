@@ -55,6 +55,12 @@ SMALL = {
     "collapse": Workload("collapse", T=512, d=128, h=128, E=8, k=2, cf=(5, 4), zipf_s=12.0),
     # a single token
     "one_token": Workload("one_token", T=1, d=128, h=256, E=4, k=2),
+    # experts that may keep 1024+ rows: the forward's GEMMs and the backward's dX
+    # on CTA-pair tiles (a ragged last 256-row tile per expert)
+    "pair_tok": Workload("pair_tok", T=1300, d=256, h=384, E=3, k=2, zipf_s=0.3),
+    # a shared expert over 1100 tokens (its dX on CTA-pair tiles too)
+    "pair_shared": Workload("pair_shared", T=1100, d=256, h=128, E=8, k=2, n_shared=1,
+                            h_shared=256, cf=(3, 2)),
 }
 
 
