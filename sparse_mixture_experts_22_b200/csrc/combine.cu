@@ -175,6 +175,94 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// k <= 2, one partial per row, d % 16 == 0: 16 columns per thread, so that each
+// thread keeps twice the row bytes in flight (same arithmetic order as
+// combine_kernel; the large layer's combine: 168 -> 144 us).
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+    combine16_kernel(const float* __restrict__ y, const int32_t* __restrict__ slot_of,
+                     const float* __restrict__ gate, const float* __restrict__ ys,
+                     void* __restrict__ out, int64_t T, int d, int k, StatsParams sp) {
+    pdl_wait();
+    if (sp.sums && blockIdx.x == gridDim.x - 1) {
+        stats_block(sp);
+        return;
+    }
+    const int vecs = d / 16;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * vecs) return;
+    const int64_t t = i / vecs;
+    const int c = (int)(i % vecs) * 16;
+    int32_t slot[2];
+    float g[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        slot[j] = j < k ? slot_of[t * k + j] : -1;
+        g[j] = j < k ? gate[t * k + j] : 0.f;
+    }
+    float4 sv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ys) {
+        const float4* p = reinterpret_cast<const float4*>(ys + t * d + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sv[q] = __ldg(p + q);
+    }
+    float4 r[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) r[j][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (slot[j] >= 0) {
+            const float4* p = reinterpret_cast<const float4*>(y + (int64_t)slot[j] * d + c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) r[j][q] = __ldg(p + q);
+        }
+    }
+    float acc[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        if (slot[j] < 0) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc[4 * q + 0] = fmaf(g[j], r[j][q].x, acc[4 * q + 0]);
+            acc[4 * q + 1] = fmaf(g[j], r[j][q].y, acc[4 * q + 1]);
+            acc[4 * q + 2] = fmaf(g[j], r[j][q].z, acc[4 * q + 2]);
+            acc[4 * q + 3] = fmaf(g[j], r[j][q].w, acc[4 * q + 3]);
+        }
+    }
+    if (ys) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc[4 * q + 0] += sv[q].x;
+            acc[4 * q + 1] += sv[q].y;
+            acc[4 * q + 2] += sv[q].z;
+            acc[4 * q + 3] += sv[q].w;
+        }
+    }
+    if (OUT_BF16) {
+        uint4 o0, o1;
+        o0.x = pack_bf16x2(acc[0], acc[1]);
+        o0.y = pack_bf16x2(acc[2], acc[3]);
+        o0.z = pack_bf16x2(acc[4], acc[5]);
+        o0.w = pack_bf16x2(acc[6], acc[7]);
+        o1.x = pack_bf16x2(acc[8], acc[9]);
+        o1.y = pack_bf16x2(acc[10], acc[11]);
+        o1.z = pack_bf16x2(acc[12], acc[13]);
+        o1.w = pack_bf16x2(acc[14], acc[15]);
+        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + t * d + c);
+        o[0] = o0;
+        o[1] = o1;
+    } else {
+        float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + t * d + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            o[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+    }
+}
+
 // Destinations of the expert-parallel combine: y row bases of the owners.
 struct PeerY {
     const float* base[MAX_PEERS];
@@ -314,8 +402,15 @@ int launch_combine(const float* y, int splits, int64_t split_stride, const int32
         launch_ex(pdl_active(), kern, dim3(blocks), dim3(256), 0, st, y, splits, split_stride,
                   slot_of, gate, y_shared, out, T, d, k, s);
     };
-    if (k <= 2)
+    if (k <= 2 && splits == 1 && d % 16 == 0) {
+        const int64_t n16 = T * (d / 16);
+        const unsigned b16 = (unsigned)((n16 + 255) / 256) + (sp ? 1 : 0);
+        auto kern = out_bf16 ? combine16_kernel<true> : combine16_kernel<false>;
+        launch_ex(pdl_active(), kern, dim3(b16), dim3(256), 0, st, y, slot_of, gate, y_shared,
+                  out, T, d, k, s);
+    } else if (k <= 2) {
         out_bf16 ? go(combine_kernel<true, 2>) : go(combine_kernel<false, 2>);
+    }
     else if (k <= 4)
         out_bf16 ? go(combine_kernel<true, 4>) : go(combine_kernel<false, 4>);
     else

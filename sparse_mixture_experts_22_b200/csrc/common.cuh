@@ -401,6 +401,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // 16 consecutive floats <-> 16 bf16 (round to nearest even); 16-byte aligned.
+// 16-byte store with an L2 cache policy (e.g. evict-first for outputs that no
+// kernel reads soon).
+__device__ __forceinline__ void st_global_f32x4_hint(float* p, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float* v) {
     uint4 o0, o1;
     o0.x = pack_bf16x2(v[0], v[1]);

@@ -226,20 +226,28 @@ __device__ __forceinline__ int units_of_group(int rows, const TcArgs& a) {
 
 // Stores 32 columns of fp32 for the warp's 32 rows: v holds row `lane`'s
 // values; row r of the block goes to dst_row0 + r * ld (columns 0..31), rows
-// at or past `valid` are skipped.  stg is the warp's staging buffer.
+// at or past `valid` are skipped.  stg is the warp's staging buffer.  With
+// `stream` the stores carry an L2 evict-first policy (outputs no kernel of the
+// layer reads again, so that they do not push the operands out of L2).
 __device__ __forceinline__ void store_rows_f32x32(float* stg, const float* v, int lane,
-                                                  float* dst_row0, int64_t ld, int valid) {
+                                                  float* dst_row0, int64_t ld, int valid,
+                                                  bool stream = false) {
     float4* srow = reinterpret_cast<float4*>(stg + lane * STG_LD);
 #pragma unroll
     for (int j = 0; j < 8; ++j) srow[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     __syncwarp();
     const int sub = lane >> 3, col = (lane & 7) * 4;
+    const uint64_t pol = stream ? l2_policy_evict_first() : 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int r = 4 * i + sub;
-        if (r < valid)
-            *reinterpret_cast<float4*>(dst_row0 + r * ld + col) =
-                *reinterpret_cast<const float4*>(stg + r * STG_LD + col);
+        if (r < valid) {
+            const float4 w = *reinterpret_cast<const float4*>(stg + r * STG_LD + col);
+            if (stream)
+                st_global_f32x4_hint(dst_row0 + r * ld + col, w, pol);
+            else
+                *reinterpret_cast<float4*>(dst_row0 + r * ld + col) = w;
+        }
     }
     __syncwarp();
 }
@@ -670,7 +678,8 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = 0.0f;
                     }
-                    store_rows_f32x32(stg, v, lane, dst0 + c, args.out_ld, 32);
+                    // the weight gradients: read by no later kernel of the step
+                    store_rows_f32x32(stg, v, lane, dst0 + c, args.out_ld, 32, true);
                 }
             } else if (MODE == TC_GATEUP_SWAP) {
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.out) +
