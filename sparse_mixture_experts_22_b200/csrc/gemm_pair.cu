@@ -44,14 +44,13 @@
 // multicast); the epilogues of both CTAs release an accumulator on the even
 // CTA's barrier.  (A first version had the odd CTA's copies complete on its
 // own barrier and a thread forward each stage to the even CTA with a
-// cluster-scope release: that per-stage hop kept the tensor pipe 33% busy.)  The pairs take their work units
-// from a device counter (the even CTA's producer fetches the next unit and
-// publishes it to every role of both CTAs through a small queue in shared
-// memory), so the work spreads over however many pairs are resident at once.
-// Every wait is bounded; on a
-// time-out the kernel records MOE_ERR_TIMEOUT, lets the copies it issued
-// land and the MMAs drain, and both CTAs meet at a cluster barrier before
-// TMEM is released.
+// cluster-scope release: that per-stage hop kept the tensor pipe 33% busy.)
+// The pairs take their work units from a device counter (the even CTA's
+// producer fetches the next unit and publishes it to every role of both CTAs
+// through a small queue in shared memory), so the work spreads over however
+// many pairs are resident at once.  Every wait is bounded; on a time-out the
+// kernel records MOE_ERR_TIMEOUT, lets the copies it issued land and the MMAs
+// drain, and both CTAs meet at a cluster barrier before TMEM is released.
 #include <stdio.h>
 
 #include <mutex>
