@@ -256,9 +256,14 @@ MOE_API int moe_stats_finalize(const moe_config* cfg, const double* sums, moe_st
                        void* stream);
 
 /* The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine and
- * moe_aux_stats in sequence on one stream, with the intermediates in ws.
- * W13s/W2s may be NULL when n_shared == 0; bias may be NULL when !has_bias;
- * stats may be NULL to skip the statistics. */
+ * moe_aux_stats in sequence on `stream`, with the intermediates in ws (the
+ * shared experts may run on a second stream forked from and joined back into
+ * `stream`, see moe_set_shared_overlap).  W13s/W2s may be NULL when
+ * n_shared == 0; bias may be NULL when !has_bias; stats may be NULL to skip
+ * the statistics.  The call reads nothing back to the host, so it can be
+ * captured in a CUDA graph once one uncaptured call on the device has set the
+ * kernels' attributes and created the second stream; every replay gives the
+ * bits of an uncaptured call on the same inputs. */
 MOE_API int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const float* bias,
                 const void* W13, const void* W2p, const void* W13s, const void* W2s,
                 void* out, int32_t* topk_idx, float* topk_gate, int32_t* routed,
