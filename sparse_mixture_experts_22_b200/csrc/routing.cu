@@ -21,6 +21,10 @@
 // row copies into x_perm, so a decode batch spreads its gather over many SMs.
 #include <math.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -871,13 +875,35 @@ __global__ void __launch_bounds__(ROUTE_BLOCK)
     dispatch_block(da, 0, 1, leader, blockIdx.x, gridDim.x, d, my);
 }
 
+// Opts the kernel in to `bytes` of dynamic shared memory when its static plus
+// dynamic shared memory exceeds the 48 KB a launch gets without opting in
+// (the top-k kernels hold ~21.5 KB of static arrays beside their dynamic
+// buffer).  Per device and kernel the limit only ever grows, so callers with
+// smaller needs on other threads are not cut short.
 template <typename K>
 int set_smem(K kern, size_t bytes) {
-    if (bytes <= 48 * 1024) return 0;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
-                   cudaSuccess
-               ? 0
-               : -1;
+    struct Entry {
+        size_t static_bytes;
+        size_t optin;
+    };
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, Entry> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lk(mu);
+    const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kern));
+    auto it = cache.find(key);
+    if (it == cache.end()) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return -1;
+        it = cache.emplace(key, Entry{fa.sharedSizeBytes, 0}).first;
+    }
+    if (it->second.static_bytes + bytes <= 48 * 1024 || bytes <= it->second.optin) return 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return -1;
+    it->second.optin = bytes;
+    return 0;
 }
 
 TopkArgs topk_args(const RouteParams& r) {

@@ -9,6 +9,8 @@ workloads compare everything exactly except the expert outputs, which the
 oracle computes for a sample of rows.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -241,9 +243,11 @@ def test_full_size_workload(name, hidden):
 @pytest.mark.parametrize("name", ["pair_tiles", "pair_shared", "swap_cap", "pair_tok"])
 def test_pair_tiles_match_single_sm_tiles(name, mode):
     """Experts of more than 128 tokens run their GEMMs on CTA pairs (mode 1:
-    token-major pair tiles; mode 2: the swapped pair tiles too); the same layer
-    with one SM per tile gives the same output within the bar, and the same
-    routing bit for bit."""
+    token-major pair tiles, with the shared experts' down projection in the
+    routed experts' pair launch; mode 2: the swapped pair tiles too); the same
+    layer with one SM per tile and separate launches gives the same routing and
+    the same output bit for bit (the fp32 sums run in the same order), within
+    the bar of the oracle."""
     wl = SMALL[name]
     inp = host_inputs(wl)
     r = oracle_route(wl, inp)
@@ -263,6 +267,7 @@ def test_pair_tiles_match_single_sm_tiles(name, mode):
     e2 = check_output(b["out"], ref, strict=strict_output(cfg))
     d = (out_pair.float() - b["out"].float()).abs().max().item()
     print(f"{name} mode {mode}: pair {e1} single {e2} max|pair - single| {d:.3e}")
+    assert torch.equal(out_pair, b["out"])
 
 
 @pytest.mark.parametrize("name", ["shared", "shared_small", "pair_shared", "shared_swap64"])
@@ -311,3 +316,27 @@ def test_dependent_launch_gives_identical_bits(name):
         B.moe_set_pdl(True)
     assert torch.equal(out_on, b["out"])
     assert B.moe_read_device_status(b["ws"]) == 0
+
+
+@pytest.mark.parametrize("name", ["wide_sub", "wide_zbuf", "max_experts"])
+def test_first_call_in_a_fresh_process(name):
+    """A layer whose routing kernels need a shared-memory opt-in (their static
+    arrays plus the dynamic buffer exceed 48 KB) works as the first call of a
+    process, whatever ran before it elsewhere."""
+    import subprocess
+    import sys
+    HERE = os.path.dirname(os.path.abspath(__file__))
+    code = (
+        "import sys; sys.path[:0] = [%r, %r]\n"
+        "import torch\n"
+        "from test_gpu_parity import SMALL\n"
+        "from layer_check import device_layer, host_inputs, run_forward\n"
+        "import sparse_mixture_experts_22_b200 as M\n"
+        "wl = SMALL[%r]\n"
+        "cfg, g, W = device_layer(wl, host_inputs(wl))\n"
+        "b = run_forward(cfg, g, W)\n"
+        "assert M.moe_read_device_status(b['ws']) == 0\n"
+        "assert torch.isfinite(b['out'].float()).all()\n"
+    ) % (HERE, os.path.dirname(HERE), name)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
