@@ -584,31 +584,13 @@ static int step_route_dispatch(const Plan& P, const Device& dv, const void* x, c
     return MOE_OK;
 }
 
-// Which GEMMs of an expert FFN a run_tc_ffn call launches.
-enum FfnPhase { FFN_BOTH = 0, FFN_GATEUP = 1, FFN_DOWN = 2 };
-
-// A dense group that rides along in the token-major CTA-pair down projection
-// of other groups (the shared experts beside the routed ones): its H rows
-// (rows x hid, low parts `rows` rows further when H is split), its W2
-// ([d][hid]) and its fp32 output ([rows][d]).
-struct ExtraDown {
-    const void* H;
-    int rows;
-    int hid;
-    const void* W2;
-    float* y;
-};
-
-// One grouped GEMM pair (gate/up then down) on the tensor cores, or one of the
-// two (`phase`); `extra` adds a dense group to a token-major pair down.
+// One grouped GEMM pair (gate/up then down) on the tensor cores.
 static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
                       const int32_t* rows, const int32_t* offs, const int32_t* group_w,
                       int dense_rows, const void* act,
                       int64_t act_rows, const void* W13, const void* W2p, int hid, void* H,
                       void* AB, float* y, int splits, int nt_max, int32_t* status,
-                      cudaStream_t st, const char* tag1, const char* tag2, int ctr_slot = 0,
-                      int phase = FFN_BOTH, const ExtraDown* extra = nullptr) {
-    const bool do_gu = phase != FFN_DOWN, do_down = phase != FFN_GATEUP;
+                      cudaStream_t st, const char* tag1, const char* tag2, int ctr_slot = 0) {
     const bool tok = path == PATH_TOKEN_MAJOR;
     CUtensorMap m_act, m_w;
     TcArgs a;
@@ -656,50 +638,53 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     // an expert's rows more than 128-row tiles, which pays off for large groups)
     const bool pair_tok = tok && g_pair_enabled >= 1 && nt_max >= PAIR_TOK_MIN_TOKENS &&
                           hid % 128 == 0 && P.d % 256 == 0;
-    const bool dtok = tok || nt_max > DOWN_SWAP_MAX_TOKENS;
-    const bool pair_down = pair && P.d % 256 == 0;
-    // groups of 129..256 tokens (swapped gate/up): the down projection on the
-    // token-major CTA-pair tile, one pair unit per expert and 256 output features,
-    // each SM streaming its own 128 weight rows (6 stages of 16 KB) rather than
-    // two one-SM m tiles sharing a 256-row weight tile through L2
-    const bool mid_down = !tok && dtok && !pair_down && g_pair_enabled >= 1 &&
-                          P.d % 256 == 0 && hid % 128 == 0;
-    // the down projection on token-major pair tiles; only there can an extra
-    // group (the shared experts) ride along
-    const bool down_pair_tok = pair_tok || mid_down;
-    if (extra && !down_pair_tok) return fail(MOE_ERR_UNSUPPORTED, "no pair tile for the extra group");
-
-    if (do_gu) {
-        if (pair_tok) {
-            MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 128));
-            MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 128));
-            a.stages = tc_pair_max_stages(TC_PAIR_GATEUP_TOK, nt_max, groups, false, smem_limit);
-            if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
-            MOE_TRY(zero_ctr());
-            trace_pre(st, tag1);
-            MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP_TOK, m_act, m_w, a, dv.sms / 2, st), tag1));
-            trace_mark(st, tag1);
-        } else if (pair) {
-            MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 8));
-            MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 64));
-            a.stages = tc_pair_max_stages(TC_PAIR_GATEUP, nt_max, groups, false, smem_limit);
-            if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
-            MOE_TRY(zero_ctr());
-            trace_pre(st, tag1);
-            MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP, m_act, m_w, a, dv.sms / 2, st), tag1));
-            trace_mark(st, tag1);
-        } else {
-            a.stages = tc_max_stages(mode1, 256, nt_max, groups, false, smem_limit);
-            // while the routing finishes, prefetch the start of each CTA's first weight
-            // tile (the unit it gets when every expert has tokens) into L2
-            a.prefetch_kb = (!tok && !group_w && pdl_active()) ? 16 : 0;
-            if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
-            trace_pre(st, tag1);
-            MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
-            trace_mark(st, tag1);
-        }
+    if (pair_tok) {
+        MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 128));
+        MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 128));
+        a.stages = tc_pair_max_stages(TC_PAIR_GATEUP_TOK, nt_max, groups, false, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP_TOK, m_act, m_w, a, dv.sms / 2, st), tag1));
+        trace_mark(st, tag1);
+        MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 128));
+        MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
+        a.K = hid;
+        a.n_feat = P.d;
+        a.w_rows_per_group = P.d;
+        a.splits = 1;
+        a.out = y;
+        a.out_ld = P.d;
+        a.split_stride = act_rows * (int64_t)P.d;
+        a.aux = nullptr;
+        a.prefetch_kb = 0;
+        a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, nt_max, groups, P.split, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
+        trace_pre(st, tag2);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DOWN_TOK, m_act, m_w, a, dv.sms / 2, st), tag2));
+        trace_mark(st, tag2);
+        return MOE_OK;
     }
-    if (!do_down) return MOE_OK;
+    if (pair) {
+        MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 8));
+        MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 64));
+        a.stages = tc_pair_max_stages(TC_PAIR_GATEUP, nt_max, groups, false, smem_limit);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        MOE_TRY(zero_ctr());
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_GATEUP, m_act, m_w, a, dv.sms / 2, st), tag1));
+        trace_mark(st, tag1);
+    } else {
+        a.stages = tc_max_stages(mode1, 256, nt_max, groups, false, smem_limit);
+        // while the routing finishes, prefetch the start of each CTA's first weight
+        // tile (the unit it gets when every expert has tokens) into L2
+        a.prefetch_kb = (!tok && !group_w && pdl_active()) ? 16 : 0;
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_gemm(mode1, 256, m_act, m_w, a, dv.sms, st), tag1));
+        trace_mark(st, tag1);
+    }
 
     // down: H [act_rows][hid] x W2p [groups * d][hid] -> y [splits][act_rows][d]
     // The down projection streams its weights through the wide B operand of the
@@ -707,18 +692,19 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     // weight tile per stage keeps twice the weight bytes in flight of a swapped
     // tile next to a token tile that large, and the accumulator stays
     // double-buffered; the second token tile of a group is partly idle.
-    a.K = hid;
-    a.n_feat = P.d;
-    a.w_rows_per_group = P.d;
-    a.splits = 1;
-    a.out = y;
-    a.out_ld = P.d;
-    a.split_stride = act_rows * (int64_t)P.d;
-    a.aux = nullptr;
-    a.prefetch_kb = 0;
+    const bool pair_down = pair && P.d % 256 == 0;
     if (pair_down) {
         MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 8));
         MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
+        a.K = hid;
+        a.n_feat = P.d;
+        a.w_rows_per_group = P.d;
+        a.splits = 1;
+        a.out = y;
+        a.out_ld = P.d;
+        a.split_stride = act_rows * (int64_t)P.d;
+        a.aux = nullptr;
+        a.prefetch_kb = 0;
         a.stages = tc_pair_max_stages(TC_PAIR_DOWN, nt_max, groups, P.split, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
@@ -727,30 +713,23 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         trace_mark(st, tag2);
         return MOE_OK;
     }
-    if (down_pair_tok) {
+    const bool dtok = tok || nt_max > DOWN_SWAP_MAX_TOKENS;
+    // groups of 129..256 tokens (swapped gate/up): the down projection on the
+    // token-major CTA-pair tile, one pair unit per expert and 256 output features,
+    // each SM streaming its own 128 weight rows (6 stages of 16 KB) rather than
+    // two one-SM m tiles sharing a 256-row weight tile through L2
+    if (!tok && dtok && g_pair_enabled >= 1 && P.d % 256 == 0 && hid % 128 == 0) {
         MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 128));
         MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
-        if (extra) {
-            // the extra group: its own H rows, weights and output
-            CUtensorMap m_act2, m_w2;
-            MOE_TRY(tmap_bf16(&m_act2, extra->H, (P.split ? 2 : 1) * (int64_t)extra->rows,
-                              extra->hid, 128));
-            MOE_TRY(tmap_bf16(&m_w2, extra->W2, P.d, extra->hid, 128));
-            a.extra_rows = extra->rows;
-            a.extra_K = extra->hid;
-            a.extra_out = extra->y;
-            a.extra_lo_rows = P.split ? extra->rows : 0;
-            a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, nt_max, groups + 1, P.split,
-                                          smem_limit);
-            if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
-            MOE_TRY(zero_ctr());
-            trace_pre(st, tag2);
-            MOE_TRY(launched(launch_tc_pair_down_extra(m_act, m_w, m_act2, m_w2, a, dv.sms / 2,
-                                                       st),
-                             tag2));
-            trace_mark(st, tag2);
-            return MOE_OK;
-        }
+        a.K = hid;
+        a.n_feat = P.d;
+        a.w_rows_per_group = P.d;
+        a.splits = 1;
+        a.out = y;
+        a.out_ld = P.d;
+        a.split_stride = act_rows * (int64_t)P.d;
+        a.aux = nullptr;
+        a.prefetch_kb = 0;
         a.stages = tc_pair_max_stages(TC_PAIR_DOWN_TOK, nt_max, groups, P.split, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
         MOE_TRY(zero_ctr());
@@ -763,7 +742,15 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     const int bn = (P.d % 256 == 0) ? 256 : 128;
     MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, dtok ? 128 : 16));
     MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, dtok ? bn : 128));
+    a.K = hid;
+    a.n_feat = P.d;
+    a.w_rows_per_group = P.d;
     a.splits = dtok ? 1 : splits;
+    a.out = y;
+    a.out_ld = P.d;
+    a.split_stride = act_rows * (int64_t)P.d;
+    a.aux = nullptr;
+    a.prefetch_kb = 0;
     a.stages = tc_max_stages(mode2, bn, nt_max, groups, P.split, smem_limit);
     if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
     trace_pre(st, tag2);
@@ -775,8 +762,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
 // The shared experts' FFN over every token (fused into one expert of width
 // S * hs): gate 1, no capacity, reads x directly.
 static int step_shared_ffn(const Plan& P, const Device& dv, const void* x, const void* W13s,
-                           const void* W2s, float* y_shared, void* ws, cudaStream_t st,
-                           int phase = FFN_BOTH) {
+                           const void* W2s, float* y_shared, void* ws, cudaStream_t st) {
     if (P.T == 0 || P.S == 0) return MOE_OK;
     int32_t* status = at<int32_t>(ws, P.off_status);
     void* Hs = at<void>(ws, P.off_Hs);
@@ -798,33 +784,15 @@ static int step_shared_ffn(const Plan& P, const Device& dv, const void* x, const
     void* ABs = P.train ? at<void>(ws, P.off_ABs) : nullptr;
     return run_tc_ffn(P, dv, P.shared_path, 1, nullptr, nullptr, nullptr, (int)P.T, x, P.T, W13s,
                       W2s, P.hsum, Hs, ABs, y_shared, 1, nt, status, st, "gemm_shared_gateup",
-                      "gemm_shared_down", 1, phase);
-}
-
-// Whether the routed experts' down projection runs on token-major CTA-pair
-// tiles (the same rule as run_tc_ffn's), so that the shared experts' down
-// projection can ride in its launch as one more group: the HBM-bound routed
-// units and the compute-bound shared units then share the SMs.
-static bool fuse_shared_down(const Plan& P) {
-    if (P.S == 0 || !P.bf16 || P.path == PATH_F32 || P.shared_path == PATH_F32) return false;
-    if (g_pair_enabled < 1 || P.d % 256 != 0 || P.h % 128 != 0 || P.hsum % 128 != 0)
-        return false;
-    const bool tok = P.path == PATH_TOKEN_MAJOR;
-    if (tok) return P.nt_max >= PAIR_TOK_MIN_TOKENS;
-    // swapped gate/up: the down on pair tiles for groups of 129..256 tokens,
-    // unless the swapped pair tiles take it (mode 2)
-    return P.nt_max > DOWN_SWAP_MAX_TOKENS && g_pair_enabled < 2;
+                      "gemm_shared_down", 1);
 }
 
 // The routed experts' FFN over the dispatched rows; with `shared`, then the
-// shared experts' on the same stream.  With `extra`, the down projection also
-// computes that dense group (the shared experts' down projection, whose H the
-// caller has computed, or will have once `before_down` has fired).
+// shared experts' on the same stream.
 static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const int32_t* offsets,
                     const int32_t* kept, const void* W13, const void* W2p, const void* x,
                     const void* W13s, const void* W2s, float* y_perm, float* y_shared, void* ws,
-                    cudaStream_t st, bool shared = true, const ExtraDown* extra = nullptr,
-                    cudaEvent_t before_down = nullptr) {
+                    cudaStream_t st, bool shared = true) {
     if (P.T == 0) return MOE_OK;
     void* H = at<void>(ws, P.off_H);
     int32_t* status = at<int32_t>(ws, P.off_status);
@@ -842,26 +810,10 @@ static int step_ffn(const Plan& P, const Device& dv, const void* x_perm, const i
         trace_mark(st, "f32_down");
     } else {
         void* AB = P.train ? at<void>(ws, P.off_AB) : nullptr;
-        if (extra) {
-            MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, nullptr, 0, x_perm,
-                               P.perm_rows, W13, W2p, P.h, H, AB, y_perm, P.splits, P.nt_max,
-                               status, st, "gemm_gateup", "gemm_down", 0, FFN_GATEUP));
-            if (before_down && cudaStreamWaitEvent(st, before_down, 0) != cudaSuccess)
-                return fail(MOE_ERR_CUDA, "could not join the shared-expert stream");
-            // a launch right after an event wait goes without the programmatic edge
-            const bool pdl_was = g_pdl_in_forward;
-            if (before_down) g_pdl_in_forward = false;
-            const int rc = run_tc_ffn(P, dv, P.path, P.E, kept, offsets, nullptr, 0, x_perm,
-                                      P.perm_rows, W13, W2p, P.h, H, AB, y_perm, P.splits,
-                                      P.nt_max, status, st, "gemm_gateup", "gemm_down", 0,
-                                      FFN_DOWN, extra);
-            g_pdl_in_forward = pdl_was;
-            MOE_TRY(rc);
-        } else {
-            MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, nullptr, 0, x_perm,
-                               P.perm_rows, W13, W2p, P.h, H, AB, y_perm, P.splits, P.nt_max,
-                               status, st, "gemm_gateup", "gemm_down"));
-        }
+        MOE_TRY(run_tc_ffn(P, dv, P.path, P.E, kept, offsets, nullptr, 0, x_perm, P.perm_rows,
+                           W13, W2p,
+                           P.h, H, AB, y_perm, P.splits, P.nt_max, status, st, "gemm_gateup",
+                           "gemm_down"));
     }
     if (shared) MOE_TRY(step_shared_ffn(P, dv, x, W13s, W2s, y_shared, ws, st));
     return MOE_OK;
@@ -1336,12 +1288,6 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
         dv_shared.sms = g_shared_sms;
         dv_routed.sms = dv.sms - g_shared_sms;
     }
-    // Where the routed down projection runs on token-major CTA-pair tiles, the
-    // shared experts' down projection rides in the same launch (one more group),
-    // and only their gate/up runs beside the routing and the routed gate/up.
-    const bool fuse = P.T > 0 && fuse_shared_down(P);
-    const ExtraDown ex{P.S ? at<void>(ws, P.off_Hs) : nullptr, (int)P.T, P.hsum, W2s, ys};
-    const int shared_phase = fuse ? FFN_GATEUP : FFN_BOTH;
     SideStream ss;
     if (side) {
         MOE_TRY(side_stream(&ss));
@@ -1349,19 +1295,17 @@ int moe_forward(const moe_config* cfg, const void* x, const float* Wr, const flo
             cudaStreamWaitEvent(ss.st, ss.fork, 0) != cudaSuccess)
             return fail(MOE_ERR_CUDA, "could not fork the shared-expert stream");
         g_pdl_in_forward = false;  // the first launch on the side stream follows an event
-        const int rc = step_shared_ffn(P, dv_shared, x, W13s, W2s, ys, ws, ss.st, shared_phase);
+        const int rc = step_shared_ffn(P, dv_shared, x, W13s, W2s, ys, ws, ss.st);
         g_pdl_in_forward = true;
         MOE_TRY(rc);
         if (cudaEventRecord(ss.join, ss.st) != cudaSuccess)
             return fail(MOE_ERR_CUDA, "could not join the shared-expert stream");
-    } else if (fuse) {
-        MOE_TRY(step_shared_ffn(P, dv, x, W13s, W2s, ys, ws, st, FFN_GATEUP));
     }
     MOE_TRY(step_route_dispatch(P, dv, x, Wr, cfg->has_bias ? bias : nullptr, topk_idx, topk_gate,
                                 routed, kept, offsets, perm, slot_of, x_perm, ws, st));
     MOE_TRY(step_ffn(P, dv_routed, x_perm, offsets, kept, W13, W2p, x, W13s, W2s, y, ys, ws, st,
-                     !side && !fuse, fuse ? &ex : nullptr, (side && fuse) ? ss.join : nullptr));
-    if (side && !fuse && cudaStreamWaitEvent(st, ss.join, 0) != cudaSuccess)
+                     !side));
+    if (side && cudaStreamWaitEvent(st, ss.join, 0) != cudaSuccess)
         return fail(MOE_ERR_CUDA, "could not join the shared-expert stream");
     // combine, with the statistics computed by one extra block of the same launch
     StatsParams sp = stats_params(P, routed, kept, ws, at<double>(ws, P.off_sums), stats);

@@ -118,7 +118,6 @@ __host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stag
 
 struct PUnit {
     int g, w, rows, row0, nb, mt, ntok;
-    bool ex;  // the extra group (second pair of tensor maps)
 };
 
 struct PGroups {
@@ -126,8 +125,7 @@ struct PGroups {
     const int* rows;
     const int* off;
     const int* wi;
-    int groups;  // groups in the table, the extra one included
-    int base;    // groups before the extra one
+    int groups;
 };
 
 template <int MODE>
@@ -142,7 +140,6 @@ __device__ __forceinline__ PUnit p_decode(const PGroups& t, int u) {
     x.w = t.wi[lo];
     x.rows = t.rows[lo];
     x.row0 = t.off[lo];
-    x.ex = lo >= t.base;
     const int local = u - t.start[lo];
     if (p_tok(MODE)) {
         // m tile fastest: the units after one another share the weight tile
@@ -182,9 +179,7 @@ __device__ __forceinline__ void p_store_rows_f32x32(float* stg, const float* v, 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     tc_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
-                   const __grid_constant__ CUtensorMap tm_w,
-                   const __grid_constant__ CUtensorMap tm_act2,
-                   const __grid_constant__ CUtensorMap tm_w2, const TcArgs args) {
+                   const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
     constexpr bool GU = MODE == TC_PAIR_GATEUP;
     constexpr bool TOK = p_tok(MODE);
     constexpr int NEPI = p_epi(MODE);
@@ -194,12 +189,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     uint8_t* smem = smem_raw + (p_align(raw, 1024) - raw);
 
     const int groups = args.num_groups;
-    // token-major down: an extra dense group read through tm_act2 / tm_w2
-    const bool has_extra = MODE == TC_PAIR_DOWN_TOK && args.extra_rows > 0;
-    const int gt = groups + (has_extra ? 1 : 0);
     const bool split = DOWN && args.lo_rows != 0;
     const int S = args.stages;
-    const PairLayout L = pair_layout(MODE, args.nt_max, S, gt, split);
+    const PairLayout L = pair_layout(MODE, args.nt_max, S, groups, split);
 
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
     uint64_t* empty = full + S;
@@ -211,9 +203,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + P_QN);
     int* q_unit = reinterpret_cast<int*>(tmem_slot + 1);
     int* g_start = reinterpret_cast<int*>(smem + L.grp_off);
-    int* g_rows = g_start + gt + 1;
-    int* g_off = g_rows + gt;
-    int* g_wi = g_off + gt;
+    int* g_rows = g_start + groups + 1;
+    int* g_off = g_rows + groups;
+    int* g_wi = g_off + groups;
     int* flags = reinterpret_cast<int*>(smem + L.flag_off);
 
     const int warp = threadIdx.x >> 5;
@@ -245,10 +237,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
         fence_mbar_init();
         prefetch_tmap(&tm_act);
         prefetch_tmap(&tm_w);
-        if (has_extra) {
-            prefetch_tmap(&tm_act2);
-            prefetch_tmap(&tm_w2);
-        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, tmem_cols);
@@ -272,14 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             const int per = args.n_feat / (GU || MODE == TC_PAIR_GATEUP_TOK ? 128 : 256);
             acc += r > 0 ? per * (TOK ? (r + 255) / 256 : 1) : 0;
         }
-        if (has_extra) {
-            g_rows[groups] = args.extra_rows;
-            g_off[groups] = 0;
-            g_wi[groups] = 0;
-            g_start[groups] = acc;
-            acc += (args.n_feat / 256) * ((args.extra_rows + 255) / 256);
-        }
-        g_start[gt] = acc;
+        g_start[groups] = acc;
     }
     tc_fence_before();
     __syncthreads();
@@ -287,8 +268,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const PGroups tab{g_start, g_rows, g_off, g_wi, gt, groups};
-    const int total = g_start[gt];
+    const PGroups tab{g_start, g_rows, g_off, g_wi, groups};
+    const int total = g_start[groups];
     const uint64_t limit = args.wait_limit_ns;
     // the unit queue: slot j holds the j-th unit (mod P_QN) of this pair, or
     // `total` when there is no more work
@@ -317,6 +298,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             uint32_t phase = 0;
             uint32_t issued = 0, issued_par = 0;
             bool ok = true;
+            const int kblocks = args.K / PBK;
             int qs = 0;
             uint32_t qph = 0;
             const uint32_t peer_unit0 = map_shared_rank(smem_addr(&q_unit[0]), 1);
@@ -350,11 +332,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                 const int trow = TOK ? x.row0 + x.mt * 256 + (int)v * PBM : x.row0 + (int)v * half;
                 const uint32_t bytes =
                     (uint32_t)PBM * PBK * 2 + (uint32_t)half * PBK * 2 * (split ? 2u : 1u);
-                // the extra group's units read their own activations and weights
-                const CUtensorMap* m_act = x.ex ? &tm_act2 : &tm_act;
-                const CUtensorMap* m_w = x.ex ? &tm_w2 : &tm_w;
-                const int lo_rows = (int)(x.ex ? args.extra_lo_rows : args.lo_rows);
-                const int kblocks = (x.ex ? args.extra_K : args.K) / PBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, limit)) {
                         report_timeout(args.status);
@@ -372,11 +349,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                         // A: this CTA's 128 token rows (then their low parts); B: the
                         // weight rows of this CTA's half of N (gate/up: CTA 0 the gate
                         // rows of the hidden block, CTA 1 its up rows)
-                        tma_load_2d_pair(sa, m_act, fb, kc, trow, pol_a);
+                        tma_load_2d_pair(sa, &tm_act, fb, kc, trow, pol_a);
                         if (split)
-                            tma_load_2d_pair(sa + PBM * PBK * 2, m_act, fb, kc, trow + lo_rows,
-                                             pol_a);
-                        tma_load_2d_pair(sb, m_w, fb, kc,
+                            tma_load_2d_pair(sa + PBM * PBK * 2, &tm_act, fb, kc,
+                                             trow + (int)args.lo_rows, pol_a);
+                        tma_load_2d_pair(sb, &tm_w, fb, kc,
                                          x.w * args.w_rows_per_group + x.nb * 256 + (int)v * PBM,
                                          pol_n);
                     } else if (GU) {
@@ -427,6 +404,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
+            const int kblocks = args.K / PBK;
             int qs = 0;
             uint32_t qph = 0;
             while (ok) {
@@ -444,7 +422,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * acc_stride;
                 const uint32_t idesc = idesc_bf16_f32(256, x.ntok);
-                const int kblocks = (x.ex ? args.extra_K : args.K) / PBK;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_cl(&full[stage], phase, limit)) {
                         report_timeout(args.status);
@@ -569,7 +546,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
             } else if (MODE == TC_PAIR_DOWN_TOK) {
                 const int r0 = x.mt * 256 + (int)v * PBM + q * 32;  // this warp's first row
                 const int valid = min(32, x.rows - r0);
-                float* dst0 = reinterpret_cast<float*>(x.ex ? args.extra_out : args.out) +
+                float* dst0 = reinterpret_cast<float*>(args.out) +
                               (int64_t)(x.row0 + r0) * args.out_ld + x.nb * 256;
                 float* stg = reinterpret_cast<float*>(smem + L.xch_off) + ew * (32 * P_STG_LD);
 #pragma unroll 1
@@ -667,11 +644,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
 }
 
 template <int MODE>
-int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const CUtensorMap& act2,
-                     const CUtensorMap& w2, const TcArgs& a, int pairs, cudaStream_t st) {
-    const bool extra = MODE == TC_PAIR_DOWN_TOK && a.extra_rows > 0;
+int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a, int pairs,
+                     cudaStream_t st) {
     const PairLayout L =
-        pair_layout(MODE, a.nt_max, a.stages, a.num_groups + (extra ? 1 : 0),
+        pair_layout(MODE, a.nt_max, a.stages, a.num_groups,
                     (MODE == TC_PAIR_DOWN || MODE == TC_PAIR_DOWN_TOK) && a.lo_rows != 0);
     auto kern = tc_pair_kernel<MODE>;
     constexpr int kMaxDevices = 64;
@@ -693,8 +669,7 @@ int launch_pair_mode(const CUtensorMap& act, const CUtensorMap& w, const CUtenso
         return -1;
     }
     // the cluster shape is part of the kernel (__cluster_dims__)
-    launch_ex(pdl_active(), kern, dim3(2 * pairs), dim3(p_threads(MODE)), L.total, st, act, w,
-              act2, w2, a);
+    launch_ex(pdl_active(), kern, dim3(2 * pairs), dim3(p_threads(MODE)), L.total, st, act, w, a);
     note_launch();
     return launch_result();
 }
@@ -711,27 +686,17 @@ int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_li
 int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
                    int pairs, cudaStream_t st) {
     if (!p_tok(mode) && (a.nt_max < 16 || a.nt_max > 256 || a.nt_max % 16)) return -1;
-    if (a.extra_rows) return -1;  // the extra group: launch_tc_pair_down_extra
     switch (mode) {
         case TC_PAIR_GATEUP:
-            return launch_pair_mode<TC_PAIR_GATEUP>(act, w, act, w, a, pairs, st);
+            return launch_pair_mode<TC_PAIR_GATEUP>(act, w, a, pairs, st);
         case TC_PAIR_DOWN:
-            return launch_pair_mode<TC_PAIR_DOWN>(act, w, act, w, a, pairs, st);
+            return launch_pair_mode<TC_PAIR_DOWN>(act, w, a, pairs, st);
         case TC_PAIR_GATEUP_TOK:
-            return launch_pair_mode<TC_PAIR_GATEUP_TOK>(act, w, act, w, a, pairs, st);
+            return launch_pair_mode<TC_PAIR_GATEUP_TOK>(act, w, a, pairs, st);
         case TC_PAIR_DOWN_TOK:
-            return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, act, w, a, pairs, st);
+            return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, a, pairs, st);
     }
     return -1;
-}
-
-int launch_tc_pair_down_extra(const CUtensorMap& act, const CUtensorMap& w,
-                              const CUtensorMap& act2, const CUtensorMap& w2, const TcArgs& a,
-                              int pairs, cudaStream_t st) {
-    if (a.extra_rows < 1 || !a.extra_out || a.extra_K < PBK || a.extra_K % PBK ||
-        (a.lo_rows != 0) != (a.extra_lo_rows != 0))
-        return -1;
-    return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, act2, w2, a, pairs, st);
 }
 
 }  // namespace moe

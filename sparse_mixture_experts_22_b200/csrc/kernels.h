@@ -168,16 +168,6 @@ struct TcArgs {
                                 // row r's low parts to row r + lo_rows of `out`; down reads
                                 // them there from the activation tensor and issues a second
                                 // MMA per K step into the same accumulator
-    // CTA-pair token-major down only: one more (dense) group after the
-    // num_groups groups, read through the second pair of tensor maps -- its own
-    // activations (extra_K columns, low parts extra_lo_rows rows further when
-    // H is split) and weights (weight index 0) -- and written to extra_out
-    // (fp32, out_ld per row).  The shared experts' down projection rides in the
-    // routed experts' launch this way.  0 rows: none.
-    int extra_rows;
-    int extra_K;
-    void* extra_out;
-    int64_t extra_lo_rows;
 };
 
 // Deepest pipeline (2..8 stages) whose shared memory fits smem_limit; `split`
@@ -198,10 +188,6 @@ int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& 
 int tc_pair_max_stages(int mode, int nt_max, int groups, bool split, int smem_limit);
 int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const TcArgs& a,
                    int pairs, cudaStream_t st);
-// The token-major down with the extra group of TcArgs (act2/w2: its tensor maps).
-int launch_tc_pair_down_extra(const CUtensorMap& act, const CUtensorMap& w,
-                              const CUtensorMap& act2, const CUtensorMap& w2, const TcArgs& a,
-                              int pairs, cudaStream_t st);
 
 // ---------------------------------------------------------------- fp32 SIMT FFN
 // gate/up: H[r][f] = silu(A_r . W13[g][gate f]) * (A_r . W13[g][up f]);

@@ -243,11 +243,9 @@ def test_full_size_workload(name, hidden):
 @pytest.mark.parametrize("name", ["pair_tiles", "pair_shared", "swap_cap", "pair_tok"])
 def test_pair_tiles_match_single_sm_tiles(name, mode):
     """Experts of more than 128 tokens run their GEMMs on CTA pairs (mode 1:
-    token-major pair tiles, with the shared experts' down projection in the
-    routed experts' pair launch; mode 2: the swapped pair tiles too); the same
-    layer with one SM per tile and separate launches gives the same routing and
-    the same output bit for bit (the fp32 sums run in the same order), within
-    the bar of the oracle."""
+    token-major pair tiles; mode 2: the swapped pair tiles too); the same layer
+    with one SM per tile gives the same routing and the same output bit for bit
+    (the fp32 sums run in the same order), within the bar of the oracle."""
     wl = SMALL[name]
     inp = host_inputs(wl)
     r = oracle_route(wl, inp)
