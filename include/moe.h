@@ -524,8 +524,8 @@ MOE_API int moe_set_shared_sms(int sms);
 MOE_API int moe_set_wait_limit_ns(uint64_t ns);
 
 /* Test hook for the time-out path (off by default).  When on, in every expert
- * FFN GEMM launch the first work unit of CTA 0 withholds its
- * "accumulator ready" signal, so that CTA's epilogue wait can only run out:
+ * FFN GEMM launch work unit 0 (whichever CTA or CTA pair takes it) withholds
+ * its "accumulator ready" signal, so that its epilogue wait can only run out:
  * after the wait limit (set a short one with moe_set_wait_limit_ns) the
  * kernel records MOE_ERR_TIMEOUT, drains its in-flight copies and MMAs,
  * releases tensor memory and returns.  Results of such a call are garbage;

@@ -1,6 +1,6 @@
 """Failure detection without a GPU fault: every wait of the tensor-core kernels
-is bounded.  The test hook makes one CTA's epilogue wait on a signal that is
-never sent; with a 5 ms bound the wait runs out, and the kernels must record
+is bounded.  The test hook makes the epilogue that takes work unit 0 wait on a
+signal that is never sent; with a 5 ms bound the wait runs out, and the kernels must record
 MOE_ERR_TIMEOUT in the device status word, let their in-flight copies and MMAs
 finish, release tensor memory and return, leaving the context usable -- the
 next call with the hook off gives the normal result bit for bit."""
