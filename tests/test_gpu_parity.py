@@ -83,6 +83,10 @@ SMALL = {
     # experts of over 1024 tokens: token-major tiles of 256 tokens on CTA pairs,
     # ragged last tiles (an expert's second CTA half partly or wholly past its rows)
     "pair_tok": Workload("pair_tok", T=1300, d=256, h=384, E=3, k=2, zipf_s=0.3),
+    # a model width that is not a multiple of 256: the down projection on
+    # 128-wide output tiles (three of them), swapped and token-major
+    "d384_swap": Workload("d384_swap", T=300, d=384, h=256, E=6, k=2, cf=(5, 4), zipf_s=0.5),
+    "d384_tok": Workload("d384_tok", T=1000, d=384, h=256, E=4, k=2, cf=(1, 1), zipf_s=0.5),
 }
 
 
