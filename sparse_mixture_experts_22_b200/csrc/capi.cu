@@ -893,8 +893,8 @@ static int step_stats(const Plan& P, const int32_t* routed, const int32_t* kept,
 
 // Backward GEMMs of one set of groups: dAB = SiLU*mul backward of dY W2t^T
 // (bf16, interleaved like AB), then dX = dAB W13t^T (fp32).  nt_max bounds a
-// group's rows: groups that may hold 1024+ rows take dX on CTA-pair tiles, as
-// the forward's down projection does.
+// group's rows: groups that may hold 1024+ rows take both on CTA-pair tiles, as
+// the forward's GEMMs do.
 static int run_tc_backward(const Plan& P, const Device& dv, int groups, const int32_t* rows,
                            const int32_t* offs, int dense_rows, int64_t act_rows, const void* dY,
                            const void* W2t, const void* AB, void* dAB, const void* W13t,
@@ -914,8 +914,6 @@ static int run_tc_backward(const Plan& P, const Device& dv, int groups, const in
     a.splits = 1;
 
     const int bn1 = hid % 256 == 0 ? 256 : 128;
-    MOE_TRY(tmap_bf16(&m_act, dY, act_rows, P.d, 128));
-    MOE_TRY(tmap_bf16(&m_w, W2t, (int64_t)groups * hid, P.d, bn1));
     a.K = P.d;
     a.n_feat = hid;
     a.w_rows_per_group = hid;
@@ -923,11 +921,29 @@ static int run_tc_backward(const Plan& P, const Device& dv, int groups, const in
     a.out_ld = 2 * (int64_t)hid;
     a.aux = const_cast<void*>(AB);
     a.aux_ld = 2 * (int64_t)hid;
-    a.stages = tc_max_stages(TC_DGATE_TOK, bn1, 16, groups, false, dv.smem_optin);
-    if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
-    trace_pre(st, tag1);
-    MOE_TRY(launched(launch_tc_gemm(TC_DGATE_TOK, bn1, m_act, m_w, a, dv.sms, st), tag1));
-    trace_mark(st, tag1);
+    // groups that may hold 1024+ rows: dgate on CTA-pair tiles too
+    const bool pair = g_pair_enabled >= 1 && nt_max >= PAIR_TOK_MIN_TOKENS && hid % 256 == 0;
+    if (pair) {
+        MOE_TRY(tmap_bf16(&m_act, dY, act_rows, P.d, 128));
+        MOE_TRY(tmap_bf16(&m_w, W2t, (int64_t)groups * hid, P.d, 128));
+        a.unit_ctr = status + UNIT_CTR_WORD + ctr_slot;
+        a.stages = tc_pair_max_stages(TC_PAIR_DGATE_TOK, 256, groups, false, dv.smem_optin);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        if (cudaMemsetAsync(a.unit_ctr, 0, sizeof(int32_t), st) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "memset failed");
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_pair(TC_PAIR_DGATE_TOK, m_act, m_w, a, dv.sms / 2, st), tag1));
+        trace_mark(st, tag1);
+        a.unit_ctr = nullptr;
+    } else {
+        MOE_TRY(tmap_bf16(&m_act, dY, act_rows, P.d, 128));
+        MOE_TRY(tmap_bf16(&m_w, W2t, (int64_t)groups * hid, P.d, bn1));
+        a.stages = tc_max_stages(TC_DGATE_TOK, bn1, 16, groups, false, dv.smem_optin);
+        if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
+        trace_pre(st, tag1);
+        MOE_TRY(launched(launch_tc_gemm(TC_DGATE_TOK, bn1, m_act, m_w, a, dv.sms, st), tag1));
+        trace_mark(st, tag1);
+    }
 
     const int bn2 = P.d % 256 == 0 ? 256 : 128;
     a.K = 2 * hid;

@@ -70,7 +70,7 @@ constexpr int P_STG_LD = 36;  // fp32 staging row (32 values + 4 of padding)
 constexpr int P_QN = 4;       // slots of the unit queue
 
 __host__ __device__ constexpr bool p_tok(int mode) {
-    return mode == TC_PAIR_GATEUP_TOK || mode == TC_PAIR_DOWN_TOK;
+    return mode == TC_PAIR_GATEUP_TOK || mode == TC_PAIR_DOWN_TOK || mode == TC_PAIR_DGATE_TOK;
 }
 // epilogue warps: two per TMEM lane quarter on swapped tiles (splitting the
 // token columns), one per quarter on token-major tiles
@@ -543,6 +543,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                         store_bf16x16(dst + c, hv);
                     }
                 }
+            } else if (MODE == TC_PAIR_DGATE_TOK) {
+                // dH of this CTA's 128 tokens for 256 hidden features; with the
+                // forward's pre-activations a, b (AB, bf16): dA = dH b silu'(a),
+                // dB = dH silu(a), stored interleaved per 128-wide block like AB
+                const int r = x.mt * 256 + (int)v * PBM + q * 32 + lane;
+                const bool valid = r < x.rows;
+                const int64_t rowoff = (int64_t)(x.row0 + r) * args.aux_ld;
+                const __nv_bfloat16* ab =
+                    reinterpret_cast<const __nv_bfloat16*>(args.aux) + rowoff;
+                __nv_bfloat16* dab = reinterpret_cast<__nv_bfloat16*>(args.out) + rowoff;
+                auto ab_col = [&](int c) {
+                    const int f = x.nb * 256 + c;
+                    return (int64_t)(f >> 7) * 256 + (f & 127);
+                };
+                // the pre-activations of the next 16 features load while the
+                // current ones are used
+                uint4 na0 = make_uint4(0, 0, 0, 0), na1 = na0, nb0 = na0, nb1 = na0;
+                if (valid) {
+                    const uint4* pa = reinterpret_cast<const uint4*>(ab + ab_col(0));
+                    na0 = pa[0];
+                    na1 = pa[1];
+                    nb0 = pa[16];
+                    nb1 = pa[17];
+                }
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 16) {
+                    float dh[16];
+                    tmem_ld16(t0 + c, dh);
+                    const uint4 ca0 = na0, ca1 = na1, cb0 = nb0, cb1 = nb1;
+                    if (valid && c + 16 < 256) {
+                        const uint4* pa = reinterpret_cast<const uint4*>(ab + ab_col(c + 16));
+                        na0 = pa[0];
+                        na1 = pa[1];
+                        nb0 = pa[16];
+                        nb1 = pa[17];
+                    }
+                    tmem_ld_wait();
+                    if (valid) {
+                        const int64_t col = ab_col(c);
+                        float a[16], b[16], da[16], db[16];
+                        const uint32_t wa[8] = {ca0.x, ca0.y, ca0.z, ca0.w,
+                                                ca1.x, ca1.y, ca1.z, ca1.w};
+                        const uint32_t wb[8] = {cb0.x, cb0.y, cb0.z, cb0.w,
+                                                cb1.x, cb1.y, cb1.z, cb1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            a[2 * i] = __uint_as_float(wa[i] << 16);
+                            a[2 * i + 1] = __uint_as_float(wa[i] & 0xFFFF0000u);
+                            b[2 * i] = __uint_as_float(wb[i] << 16);
+                            b[2 * i + 1] = __uint_as_float(wb[i] & 0xFFFF0000u);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float sig = 1.0f / (1.0f + __expf(-a[i]));
+                            da[i] = dh[i] * b[i] * sig * (1.0f + a[i] * (1.0f - sig));
+                            db[i] = dh[i] * a[i] * sig;
+                        }
+                        store_bf16x16(dab + col, da);
+                        store_bf16x16(dab + col + 128, db);
+                    }
+                }
             } else if (MODE == TC_PAIR_DOWN_TOK) {
                 const int r0 = x.mt * 256 + (int)v * PBM + q * 32;  // this warp's first row
                 const int valid = min(32, x.rows - r0);
@@ -695,6 +756,9 @@ int launch_tc_pair(int mode, const CUtensorMap& act, const CUtensorMap& w, const
             return launch_pair_mode<TC_PAIR_GATEUP_TOK>(act, w, a, pairs, st);
         case TC_PAIR_DOWN_TOK:
             return launch_pair_mode<TC_PAIR_DOWN_TOK>(act, w, a, pairs, st);
+        case TC_PAIR_DGATE_TOK:
+            if (a.n_feat % 256 || !a.aux) return -1;
+            return launch_pair_mode<TC_PAIR_DGATE_TOK>(act, w, a, pairs, st);
     }
     return -1;
 }

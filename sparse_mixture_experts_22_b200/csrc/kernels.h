@@ -133,6 +133,7 @@ enum TcMode : int {
     TC_PAIR_DOWN = 7,    // down on CTA pairs: 2 x 128 weight rows x the tokens (fp32 out)
     TC_PAIR_GATEUP_TOK = 8,  // gate/up on CTA pairs, token-major: 2 x 128 tokens x 256
     TC_PAIR_DOWN_TOK = 9,    // down on CTA pairs, token-major: 2 x 128 tokens x 256 (fp32 out)
+    TC_PAIR_DGATE_TOK = 10,  // backward dgate on CTA pairs, token-major: 2 x 128 tokens x 256
 };
 
 struct TcArgs {
@@ -181,7 +182,9 @@ int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& 
 // boxes; n_feat = hidden width) and TC_PAIR_DOWN (act = H rows, 8-row boxes;
 // w = W2p, 128-row boxes; n_feat = model width, a multiple of 256); nt_max is a
 // multiple of 16 in [16, 256].  Token-major, for groups of any size:
-// TC_PAIR_GATEUP_TOK and TC_PAIR_DOWN_TOK (act and w both 128-row boxes).  The
+// TC_PAIR_GATEUP_TOK, TC_PAIR_DOWN_TOK and the backward TC_PAIR_DGATE_TOK (act =
+// dY rows, w = W2t, aux = AB, out = dAB; n_feat a multiple of 256) with act and
+// w both in 128-row boxes.  The
 // grid is `pairs` clusters of two CTAs (one per two SMs); the pairs take their
 // units from a counter, so pairs that are not resident at once only start
 // later and find less work.

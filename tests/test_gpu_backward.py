@@ -58,7 +58,10 @@ SMALL = {
     # experts that may keep 1024+ rows: the forward's GEMMs and the backward's dX
     # on CTA-pair tiles (a ragged last 256-row tile per expert)
     "pair_tok": Workload("pair_tok", T=1300, d=256, h=384, E=3, k=2, zipf_s=0.3),
-    # a shared expert over 1100 tokens (its dX on CTA-pair tiles too)
+    # the same with a hidden width that is a multiple of 256: dgate on CTA-pair
+    # tiles as well
+    "pair_tok_h512": Workload("pair_tok_h512", T=1300, d=256, h=512, E=3, k=2, zipf_s=0.3),
+    # a shared expert over 1100 tokens (its dgate and dX on CTA-pair tiles too)
     "pair_shared": Workload("pair_shared", T=1100, d=256, h=128, E=8, k=2, n_shared=1,
                             h_shared=256, cf=(3, 2)),
 }
