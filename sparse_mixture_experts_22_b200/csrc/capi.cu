@@ -619,7 +619,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
 
     // gate/up: act [act_rows][d] x W13 [groups * 2hid][d] -> H [act_rows][hid]
     const int mode1 = tok ? TC_GATEUP_TOK : TC_GATEUP_SWAP;
-    MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, tok ? 128 : 16));
+    MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, tok ? 128 : swap_gateup_tok_box(nt_max)));
     MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, tok ? 256 : 128));
     a.K = P.d;
     a.n_feat = hid;

@@ -97,10 +97,12 @@ __host__ __device__ inline void stage_bytes(int mode, int bn, int nt_max, bool s
             *a = (mode == TC_DOWN_TOK ? parts : 1) * BM * BK * 2;
             *b = bn * BK * 2;
             break;
-        case TC_GATEUP_SWAP:
+        case TC_GATEUP_SWAP: {
+            const int tb = swap_gateup_tok_box(nt_max);
             *a = 2 * BM * BK * 2;
-            *b = nt_max * BK * 2;
+            *b = (nt_max + tb - 1) / tb * tb * BK * 2;
             break;
+        }
         default:
             *a = BM * BK * 2;
             *b = parts * nt_max * BK * 2;
@@ -417,15 +419,19 @@ __global__ void __launch_bounds__(threads_of<MODE>(), 1)
                         }
                     } else {
                         const int wa = (MODE == TC_GATEUP_SWAP) ? 2 * BM : BM;
+                        // token rows in boxes of tb: whole boxes land in shared memory
+                        const int tb =
+                            MODE == TC_GATEUP_SWAP ? swap_gateup_tok_box(args.nt_max) : 16;
+                        const int trows = (x.ntok + tb - 1) / tb * tb;
                         mbar_arrive_expect_tx(&full[stage],
-                                              (wa + x.ntok * (dsplit ? 2 : 1)) * BK * 2);
+                                              (wa + trows * (dsplit ? 2 : 1)) * BK * 2);
                         const int wrow = x.w * args.w_rows_per_group +
                                          x.nb * (MODE == TC_GATEUP_SWAP ? 256 : BM);
                         tma_load_2d_hint(sa, &tm_w, &full[stage], kc, wrow, pol_w);
                         if (MODE == TC_GATEUP_SWAP)
                             tma_load_2d_hint(sa + BM * BK * 2, &tm_w, &full[stage], kc, wrow + BM,
                                              pol_w);
-                        for (int r = 0; r < x.ntok; r += 16)
+                        for (int r = 0; r < x.ntok; r += tb)
                             tma_load_2d_hint(sb + r * BK * 2, &tm_act, &full[stage], kc,
                                              x.row0 + r, pol_a);
                         if (dsplit)  // the low parts of H right behind the high ones

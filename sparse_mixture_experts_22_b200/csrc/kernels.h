@@ -171,6 +171,15 @@ struct TcArgs {
                                 // MMA per K step into the same accumulator
 };
 
+// Token rows per TMA box of the swapped gate/up (TC_GATEUP_SWAP): nt_max up to
+// 64, else 64, so that a stage of up to 256 token rows takes at most four copies
+// (a copy's fixed cost, not its bytes, bounds a stage of many 16-row boxes).
+// The tensor map of the token rows must use this box height; a stage's token
+// region holds nt_max rows rounded up to a whole box.  Rows of a group's last
+// box past its tokens are the next group's (or the zero fill past the tensor)
+// and lie outside the MMA's N columns.
+__host__ __device__ inline int swap_gateup_tok_box(int nt_max) { return nt_max < 64 ? nt_max : 64; }
+
 // Deepest pipeline (2..8 stages) whose shared memory fits smem_limit; `split`
 // sizes the down projection's stages for H's two parts.
 int tc_max_stages(int mode, int bn, int nt_max, int groups, bool split, int smem_limit);

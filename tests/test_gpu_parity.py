@@ -87,6 +87,11 @@ SMALL = {
     # 128-wide output tiles (three of them), swapped and token-major
     "d384_swap": Workload("d384_swap", T=300, d=384, h=256, E=6, k=2, cf=(5, 4), zipf_s=0.5),
     "d384_tok": Workload("d384_tok", T=1000, d=384, h=256, E=4, k=2, cf=(1, 1), zipf_s=0.5),
+    # swapped gate/up tiles of up to 256 token columns (C = 250) with a model
+    # width of 384: the token rows arrive in boxes of 64, and a group's last box
+    # runs into the next group's rows (or past the tensor's end)
+    "d384_swap_wide": Workload("d384_swap_wide", T=600, d=384, h=256, E=6, k=2, cf=(5, 4),
+                               zipf_s=0.5),
 }
 
 
