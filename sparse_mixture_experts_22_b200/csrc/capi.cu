@@ -667,7 +667,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
         return MOE_OK;
     }
     if (pair) {
-        MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, 8));
+        MOE_TRY(tmap_bf16(&m_act, act, act_rows, P.d, pair_swap_tok_box(nt_max)));
         MOE_TRY(tmap_bf16(&m_w, W13, (int64_t)groups * 2 * hid, P.d, 64));
         a.stages = tc_pair_max_stages(TC_PAIR_GATEUP, nt_max, groups, false, smem_limit);
         if (a.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "shared memory too small for the GEMM tiles");
@@ -694,7 +694,7 @@ static int run_tc_ffn(const Plan& P, const Device& dv, int path, int groups,
     // double-buffered; the second token tile of a group is partly idle.
     const bool pair_down = pair && P.d % 256 == 0;
     if (pair_down) {
-        MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, 8));
+        MOE_TRY(tmap_bf16(&m_act, H, (P.split ? 2 : 1) * act_rows, hid, pair_swap_tok_box(nt_max)));
         MOE_TRY(tmap_bf16(&m_w, W2p, (int64_t)groups * P.d, hid, 128));
         a.K = hid;
         a.n_feat = P.d;

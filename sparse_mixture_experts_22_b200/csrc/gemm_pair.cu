@@ -98,8 +98,10 @@ __host__ __device__ inline PairLayout pair_layout(int mode, int nt_max, int stag
         L.b_lo = 0;
         L.b_bytes = PBM * PBK * 2;
     } else {
+        // nt_max / 2 token rows rounded up to whole TMA boxes
+        const int tb = pair_swap_tok_box(nt_max);
         L.a_bytes = PBM * PBK * 2;
-        L.b_lo = (uint32_t)(nt_max / 2) * PBK * 2;
+        L.b_lo = (uint32_t)((nt_max / 2 + tb - 1) / tb * tb) * PBK * 2;
         L.b_bytes = p_align(L.b_lo * parts, 1024);
     }
     L.stage_bytes = L.a_bytes + L.b_bytes;
@@ -330,8 +332,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                 const PUnit x = p_decode<MODE>(tab, u);
                 const int half = x.ntok / 2;          // token rows this CTA stages
                 const int trow = TOK ? x.row0 + x.mt * 256 + (int)v * PBM : x.row0 + (int)v * half;
+                // token rows per CTA and stage: token-major, half = 128 (the A
+                // tile); swapped, half rounded up to whole boxes of tb rows (the
+                // last box may run into the other CTA's or the next group's rows)
+                const int tb = TOK ? 128 : pair_swap_tok_box(args.nt_max);
+                const int hrows = (half + tb - 1) / tb * tb;
                 const uint32_t bytes =
-                    (uint32_t)PBM * PBK * 2 + (uint32_t)half * PBK * 2 * (split ? 2u : 1u);
+                    (uint32_t)PBM * PBK * 2 + (uint32_t)hrows * PBK * 2 * (split ? 2u : 1u);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, limit)) {
                         report_timeout(args.status);
@@ -366,10 +373,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(p_threads(MODE), 1)
                         tma_load_2d_pair(sa, &tm_w, fb, kc, wrow, pol_w);
                     }
                     if (!TOK) {
-                        for (int r = 0; r < half; r += 8)
+                        for (int r = 0; r < half; r += tb)
                             tma_load_2d_pair(sb + r * PBK * 2, &tm_act, fb, kc, trow + r, pol_a);
                         if (split)  // the low parts of H behind the high ones
-                            for (int r = 0; r < half; r += 8)
+                            for (int r = 0; r < half; r += tb)
                                 tma_load_2d_pair(sb + L.b_lo + r * PBK * 2, &tm_act, fb, kc,
                                                  trow + r + (int)args.lo_rows, pol_a);
                     }

@@ -180,6 +180,12 @@ struct TcArgs {
 // and lie outside the MMA's N columns.
 __host__ __device__ inline int swap_gateup_tok_box(int nt_max) { return nt_max < 64 ? nt_max : 64; }
 
+// The same for the swapped CTA-pair tiles (TC_PAIR_GATEUP, TC_PAIR_DOWN), where
+// each CTA stages half of a unit's token rows: nt_max / 2 up to 64, else 64.
+__host__ __device__ inline int pair_swap_tok_box(int nt_max) {
+    return nt_max / 2 < 64 ? nt_max / 2 : 64;
+}
+
 // Deepest pipeline (2..8 stages) whose shared memory fits smem_limit; `split`
 // sizes the down projection's stages for H's two parts.
 int tc_max_stages(int mode, int bn, int nt_max, int groups, bool split, int smem_limit);
@@ -187,8 +193,8 @@ int launch_tc_gemm(int mode, int bn, const CUtensorMap& act, const CUtensorMap& 
                    const TcArgs& a, int grid, cudaStream_t st);
 
 // Tiles on CTA pairs (clusters of two; gemm_pair.cu).  Swapped, for groups of up
-// to 256 tokens: TC_PAIR_GATEUP (act = x rows, 8-row boxes; w = W13, 64-row
-// boxes; n_feat = hidden width) and TC_PAIR_DOWN (act = H rows, 8-row boxes;
+// to 256 tokens: TC_PAIR_GATEUP (act = x rows, pair_swap_tok_box rows; w = W13, 64-row
+// boxes; n_feat = hidden width) and TC_PAIR_DOWN (act = H rows, pair_swap_tok_box rows;
 // w = W2p, 128-row boxes; n_feat = model width, a multiple of 256); nt_max is a
 // multiple of 16 in [16, 256].  Token-major, for groups of any size:
 // TC_PAIR_GATEUP_TOK, TC_PAIR_DOWN_TOK and the backward TC_PAIR_DGATE_TOK (act =
