@@ -490,9 +490,9 @@ MOE_API int moe_set_pdl(int on);
  *      of 129..256 tokens (one pair tile per 256 output features, each weight
  *      row read once)
  *   2  also the swapped gate/up and down tiles (weight rows x tokens) of
- *      experts that keep 129..256 tokens on SM pairs -- measured slower than
- *      one SM per tile on the DeepSeek-V2-style layer (the HBM stream is
- *      latency-bound there), so off by default
+ *      experts that keep 129..256 tokens on SM pairs -- measured level with
+ *      one SM per tile on the DeepSeek-V2-style layer (its gate/up within 2 %,
+ *      the layer slightly slower), so off by default
  * Results are identical in every mode (the fp32 sums run in the same order).
  * MOE_ERR_ARG for another value. */
 MOE_API int moe_set_pair_tiles(int mode);
