@@ -455,6 +455,19 @@ def build_inputs(wl, rank, world, dev, keep_host, train=False, hidden="auto"):
 
 # ---------------------------------------------------------------- CPU oracle timing
 
+def oracle_row_seconds(O, cfg, x, r, host, T):
+    """Seconds of oracle work per layer-output row: one untimed call first (its
+    first-call costs: thread start-up, first touch of the weights), then a
+    timed probe of a few rows per host thread."""
+    import numpy as np
+    w = (host["w1"], host["w3"], host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"))
+    O.layer_rows(cfg, x, r["expert"], r["gate"], r["keep"], *w, [0])
+    probe = max(1, min(T, 2 * O.threads()))
+    t0 = time.perf_counter()
+    O.layer_rows(cfg, x, r["expert"], r["gate"], r["keep"], *w, np.arange(probe))
+    return max((time.perf_counter() - t0) / probe, 1e-6)
+
+
 def time_oracle(wl, host, budget_s):
     """Oracle on the host cores: routing of the whole batch plus the expert
     FFN rows of as many tokens as fit in about budget_s seconds."""
@@ -464,12 +477,8 @@ def time_oracle(wl, host, budget_s):
     t0 = time.perf_counter()
     r = O.route(cfg, host["x"], host["Wr"], host["bias"])
     t_route = time.perf_counter() - t0
-    # probe one row, then size the sample
-    t0 = time.perf_counter()
-    O.layer_rows(cfg, host["x"], r["expert"], r["gate"], r["keep"], host["w1"], host["w3"],
-                 host["w2"], host.get("w1s"), host.get("w3s"), host.get("w2s"), [0])
-    t_row = max(time.perf_counter() - t0, 1e-4)
-    rows_per_pass = max(1, min(wl.T, int(budget_s / (t_row + t_route / max(wl.T, 1)))))
+    t_row = oracle_row_seconds(O, cfg, host["x"], r, host, wl.T)
+    rows_per_pass = max(1, min(wl.T, int(max(budget_s - t_route, 0.0) / t_row)))
     done, elapsed, passes = 0, 0.0, 0
     while elapsed < budget_s or passes == 0:
         t0 = time.perf_counter()
@@ -512,10 +521,7 @@ def run_reference(args):
     t0 = time.perf_counter()
     r0 = O.route(cfg, x, Wr, bias)
     t_route = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    O.layer_rows(cfg, x, r0["expert"], r0["gate"], r0["keep"], host["w1"], host["w3"], host["w2"],
-                 host.get("w1s"), host.get("w3s"), host.get("w2s"), [0])
-    t_row = max(time.perf_counter() - t0, 1e-4)
+    t_row = oracle_row_seconds(O, cfg, x, r0, host, wl.T)
     nsteps = max(1, args.steps + args.warmup)
     per_step = max(REF_BUDGET_S / nsteps - t_route, 0.0)
     rows, every = max(1, min(wl.T, int(min(0.5, per_step) / t_row))), 1
